@@ -1,0 +1,192 @@
+/*
+ * echo.h - C ABI of libecho.so: Echo's error-compensated 4-bit all-reduce on
+ * one B200 (sm_100a).
+ *
+ * The method [rit.work "Echo 4-bit GPU communication", section "How Echo
+ * returns the error to later calls"; heraldofai.com "Come Echo permette ai
+ * modelli AI...", section "Come Echo evita che gli errori si accumulino"]:
+ * tensor-parallel ranks hold partial sums of one tensor; each rank sends its
+ * segments as 4-bit integers to the segment's owner; the owner restores them,
+ * adds them in high precision, requantises the total to 4 bits and sends it
+ * back to every rank, so each element is rounded at most twice whatever the
+ * number of ranks. The owner measures the error of its rounding from the
+ * high-precision sum and folds it into two smoothed estimates (fast, slow),
+ * kept separately for the forward and the backward pass, that correct later
+ * calls.
+ *
+ * On one GPU the P ranks are P device buffers in the same HBM and the "wire"
+ * is the packed 4-bit buffers the ranks write and read; the bytes that would
+ * cross a link are counted (echo_stats), not sent.
+ *
+ * Fixed readings of what the pages leave open (every entry point follows
+ * them): group of G = 32 consecutive elements; scale 2^e stored as the byte
+ * e+127, e the smallest integer >= -127 with max|v| <= 7*2^e; codes
+ * round(v/2^e) with halves to even, in [-7, 7], two per byte (element 2j in
+ * the low nibble); rank s owns the contiguous segment [s*n/P, (s+1)*n/P) and
+ * only it adds the correction c = lambda*f + (1-lambda)*s_est to its partial
+ * before rounding #1; the owner sums in binary32, rank 0 first; the captured
+ * error is err = S - Y; f <- beta_f*f + (1-beta_f)*err and
+ * s_est <- beta_s*s_est + (1-beta_s)*err; every product and sum rounded to
+ * binary32 on its own, subnormals kept. Defaults: lambda = 1/2, beta_f = 1/2,
+ * beta_s = 7/8, compensation on. Inputs must be finite with |x| < 2^120.
+ *
+ * Conventions for every entry point:
+ *   - "stream" is a cudaStream_t passed as void* (NULL: the legacy default
+ *     stream). Work is enqueued on it; calls on one handle must be ordered on
+ *     streams by the caller (they share the handle's state and wire).
+ *   - Device pointers are CUDA device addresses on the current device; host
+ *     pointers are ordinary (preferably page-locked) host memory.
+ *   - Return: ECHO_OK (0) or a negative ECHO_ERR_* code; on error nothing is
+ *     enqueued and no state changes, and echo_last_error() describes it.
+ *     No entry point aborts or traps.
+ */
+#ifndef ECHO_H
+#define ECHO_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct echo_handle echo_handle; /* opaque, owned by the library */
+
+typedef enum { ECHO_BF16 = 0, ECHO_FP32 = 1 } echo_dtype;
+typedef enum { ECHO_FWD = 0, ECHO_BWD = 1 } echo_phase;
+
+enum {
+    ECHO_OK = 0,
+    ECHO_ERR_INVALID = -1,     /* bad argument: nothing enqueued */
+    ECHO_ERR_UNSUPPORTED = -2, /* valid but not built (group != 32, n too large) */
+    ECHO_ERR_CUDA = -3,        /* a CUDA runtime call failed; message has its string */
+    ECHO_ERR_OOM = -4          /* device allocation failed */
+};
+
+#define ECHO_MAX_RANKS 16
+#define ECHO_GROUP 32
+
+/*
+ * echo_create - a handle for all-reduces of P ranks x n elements of dtype.
+ *   P      number of simulated tensor-parallel ranks, 2..16.
+ *   n      elements per rank; n % (P*group) == 0 and n <= 2^36.
+ *   group  elements per scale; only 32 is built (else ECHO_ERR_UNSUPPORTED).
+ *   dtype  ECHO_BF16 or ECHO_FP32: the element type of the rank buffers.
+ * Allocates on the current device: stage-1 wire (P x n/2 code bytes and
+ * P x n/32 scale bytes), the requantised wire (n/2 + n/32 bytes) and the
+ * compensator state (2 phases x 2 estimates x n binary32, zeroed).
+ * Returns NULL on any error (see echo_last_error). The handle is bound to the
+ * device that was current at creation.
+ */
+echo_handle *echo_create(int P, size_t n, int group, int dtype);
+
+/*
+ * echo_allreduce - in-place Echo all-reduce of P rank buffers.
+ *   rank_ptrs  P device pointers, each n elements of the handle's dtype,
+ *              16-byte aligned, pairwise non-overlapping. Caller-owned.
+ *   phase      ECHO_FWD or ECHO_BWD: which compensator state is read and
+ *              updated (the two never mix).
+ * Enqueues three kernels (compensate+quantise+pack, owner reduce+requantise,
+ * gather+dequantise) and returns. When the stream reaches the end, every
+ * rank_ptrs[r] holds the same value Y = Q*2^E, exactly representable in the
+ * dtype, and the phase's state holds the updated estimates.
+ */
+int echo_allreduce(echo_handle *h, void *const rank_ptrs[], int phase, void *stream);
+
+/*
+ * echo_allreduce_out - the same all-reduce out of place: reads send_ptrs[r],
+ * writes recv_ptrs[r]. Each send buffer may equal its own recv buffer; no
+ * other overlap is allowed. Same alignment and size rules.
+ */
+int echo_allreduce_out(echo_handle *h, const void *const send_ptrs[],
+                       void *const recv_ptrs[], int phase, void *stream);
+
+/*
+ * echo_allreduce_host - end to end from host memory: copies the P host
+ * partials host_send[r] (n elements each) to library-owned device buffers,
+ * runs the all-reduce, and copies the result (identical on every rank, n
+ * elements) back to host_recv. Copies and kernels are enqueued on stream in
+ * chunks so transfers overlap compute; the call returns after the result is
+ * in host_recv (it synchronises the stream). The device staging buffers
+ * (P x n elements) are allocated on first use and kept until echo_destroy.
+ */
+int echo_allreduce_host(echo_handle *h, const void *const host_send[], void *host_recv,
+                        int phase, void *stream);
+
+/* echo_reset - zero the compensator state of the phases in phase_mask
+ * (bit 0 forward, bit 1 backward), enqueued on the legacy default stream and
+ * completed before return. */
+int echo_reset(echo_handle *h, int phase_mask);
+
+/* echo_destroy - free everything the handle owns (synchronises the device
+ * first). NULL is a no-op. The handle must not be used afterwards. */
+int echo_destroy(echo_handle *h);
+
+/* echo_last_error - message of the last failed call on this thread
+ * ("" if none). The string stays valid until the thread's next failing call. */
+const char *echo_last_error(void);
+
+/*
+ * echo_set_params - compensator settings for later calls: beta_fast and
+ * beta_slow in [0, 1), lambda in [0, 1], enable 0 (no correction, state
+ * neither read nor written) or 1. Out-of-range values: ECHO_ERR_INVALID.
+ */
+int echo_set_params(echo_handle *h, float beta_fast, float beta_slow, float lambda,
+                    int enable);
+
+/* echo_get_state / echo_set_state - synchronous copies of a phase's two
+ * estimates (n binary32 each) to / from host memory. A checkpoint is the pair
+ * for both phases. */
+int echo_get_state(echo_handle *h, int phase, float *f_host, float *s_host);
+int echo_set_state(echo_handle *h, int phase, const float *f_host, const float *s_host);
+
+/* Range variants: elements [offset, offset+count). */
+int echo_get_state_range(echo_handle *h, int phase, size_t offset, size_t count,
+                         float *f_host, float *s_host);
+
+/*
+ * echo_get_wire - synchronous copy of the wire left by the last call.
+ *   stage 1: rank's packed codes (n/2 bytes) and scale bytes (n/32);
+ *   stage 2: the requantised total (rank ignored).
+ * Either output pointer may be NULL to skip it.
+ */
+int echo_get_wire(echo_handle *h, int stage, int rank, uint8_t *codes_host,
+                  uint8_t *scales_host);
+
+/* Range variant over groups [group_offset, group_offset+ngroups):
+ * 16*ngroups code bytes and ngroups scale bytes. */
+int echo_get_wire_range(echo_handle *h, int stage, int rank, size_t group_offset,
+                        size_t ngroups, uint8_t *codes_host, uint8_t *scales_host);
+
+/*
+ * echo_stats - counters since creation: bytes that would cross links
+ * (reduce-scatter + all-gather, 2(P-1) * n * 17/32 per call), modelled HBM
+ * bytes (sum of the three kernels' algorithmic bytes), and calls made. Any
+ * output pointer may be NULL.
+ */
+int echo_stats(echo_handle *h, uint64_t *link_bytes, uint64_t *model_hbm_bytes,
+               uint64_t *calls);
+
+/*
+ * echo_model_bytes - algorithmic bytes of one call, host-only arithmetic:
+ *   out[0..2]  HBM bytes read + written by kernels 1, 2, 3
+ *              (P*b + 8 + P*w, P*w + 16 + w, P*w + P*b per element, w = 17/32,
+ *               b = element bytes; the 8/16 state terms vanish with
+ *               compensation off),
+ *   out[3]     link bytes of one call, 2(P-1) * n * w.
+ * Same argument rules as echo_create.
+ */
+int echo_model_bytes(int P, size_t n, int dtype, int enable, uint64_t out[4]);
+
+/*
+ * echo_set_timing / echo_last_kernel_ms - when timing is on, each call records
+ * CUDA events around each of its three kernels on its stream; ms[0..2] then
+ * returns their durations for the last call (waiting for it to finish).
+ */
+int echo_set_timing(echo_handle *h, int enable);
+int echo_last_kernel_ms(echo_handle *h, float ms[3]);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* ECHO_H */

@@ -1,0 +1,102 @@
+/*
+ * echo_oracle.h - CPU oracle for Echo's error-compensated 4-bit all-reduce.
+ *
+ * TEST INFRASTRUCTURE. This library exists to check the CUDA library against
+ * a plain restatement of the method. Only the test suite, the package's
+ * smoke check and the benchmark's CPU-baseline leg load it. It shares no
+ * code, header, table or helper with the CUDA library, and neither side
+ * includes or links the other.
+ *
+ * Sources restated (both pages are digests of the preprint "Echo:
+ * Error-Compensated 4-Bit Tensor-Parallel Communication for LLM Training and
+ * Inference"):
+ *   [rit.work "Echo 4-bit GPU communication", section "How Echo returns the
+ *    error to later calls"]: segments travel as 4-bit integers; the segment
+ *    owner restores and adds them in high precision; the compressed total goes
+ *    back to every rank; each element is rounded at most twice whatever the
+ *    group size; the error of the last rounding is measured from the
+ *    high-precision sum, stored, and added back in later calls; two smoothed
+ *    estimates (fast, slow) are kept; forward and backward keep separate state.
+ *   [heraldofai.com "Come Echo permette ai modelli AI...", section "Come Echo
+ *    evita che gli errori si accumulino"]: the same mechanism.
+ *
+ * The pages give no group size, scale format, rounding mode, EMA coefficients
+ * or combining rule. The readings fixed here (all are also the CUDA
+ * library's contract):
+ *   - group G of consecutive elements (32 in the product; any even G >= 2 here);
+ *   - power-of-two scale 2^e stored as the byte e+127, e the smallest integer
+ *     >= -127 with max|v| <= 7 * 2^e (no code ever saturates);
+ *   - codes q = round-half-to-even(v / 2^e) in [-7, 7], two per byte, element
+ *     2j in the low nibble, element 2j+1 in the high nibble, two's complement;
+ *   - the owner of element i is the rank whose contiguous segment holds it;
+ *   - only the owner adds the correction c to its own partial, before its
+ *     rounding #1;
+ *   - the owner sums the P dequantised values in binary32, rank 0 first;
+ *   - the captured error is err = S - Y with Y the requantised total;
+ *   - f <- beta_f*f + (1-beta_f)*err, s <- beta_s*s + (1-beta_s)*err and
+ *     c = lambda*f + (1-lambda)*s, every product and sum rounded to binary32
+ *     on its own (no fused multiply-add), subnormals kept.
+ *
+ * Status codes: 0 on success, -1 on an invalid argument or a non-finite
+ * value, -2 when a value leaves the domain (output not exactly
+ * representable in bf16, scale search past e = 126).
+ */
+#ifndef ECHO_ORACLE_H
+#define ECHO_ORACLE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define ECHO_ORACLE_BF16 0
+#define ECHO_ORACLE_FP32 1
+
+/* Scale choice and rounding of one group (rounding #1 at a sender, #2 at the
+ * owner). v: G binary32 values. Writes G codes to q. Returns the scale byte
+ * e+127 (0..253), or -1 for a non-finite value, -2 past the domain. */
+int echo_oracle_quantize_group(const float *v, int G, int8_t *q);
+
+/* Value of code q under scale byte b: q * 2^(b-127), exact in binary32. */
+float echo_oracle_dequant(int q, int b);
+
+/* Pack count codes (count even) two per byte; unpack the reverse. */
+void echo_oracle_pack(const int8_t *q, size_t count, uint8_t *out);
+void echo_oracle_unpack(const uint8_t *in, size_t count, int8_t *q);
+
+/*
+ * One all-reduce call over ngroups groups of G elements.
+ *
+ * x        P rank partials, rank-major: x[r*m + i], m = ngroups*G elements
+ *          each; uint16 bf16 bit patterns (dtype 0) or binary32 (dtype 1).
+ * owner    owner rank of each group (0..P-1).
+ * f, s     the phase's compensator state, m binary32 each, read and updated
+ *          in place (untouched when enable == 0).
+ * out      m elements of dtype: the value every rank receives.
+ * codes1   optional [P][m/2] stage-1 packed codes, scales1 [P][ngroups].
+ * qcodes   optional [m/2] requantised codes, qscales [ngroups].
+ * c_out    optional [m] correction the owner added (0 when off).
+ * err_out  optional [m] captured error S - Y.
+ */
+int echo_oracle_allreduce_groups(int P, int G, size_t ngroups,
+                                 const int32_t *owner, int dtype,
+                                 const void *x, void *out, float *f, float *s,
+                                 float lambda, float beta_f, float beta_s,
+                                 int enable, uint8_t *codes1, uint8_t *scales1,
+                                 uint8_t *qcodes, uint8_t *qscales,
+                                 float *c_out, float *err_out);
+
+/* Same call over n elements per rank with contiguous segments: rank r owns
+ * elements [r*n/P, (r+1)*n/P). Requires n % (P*G) == 0. */
+int echo_oracle_allreduce(int P, size_t n, int G, int dtype, const void *x,
+                          void *out, float *f, float *s, float lambda,
+                          float beta_f, float beta_s, int enable,
+                          uint8_t *codes1, uint8_t *scales1, uint8_t *qcodes,
+                          uint8_t *qscales, float *c_out, float *err_out);
+
+#ifdef __cplusplus
+}
+#endif
+#endif

@@ -1,0 +1,467 @@
+"""Pins: checks that tie the CPU oracle to what the pages and the mathematics
+fix, without trusting the oracle's own code.
+
+Each pin takes an ``Oracle`` and raises ``AssertionError`` (or any error) when
+the oracle disagrees. ``test_oracle_pins.py`` runs them on the oracle;
+``test_oracle_mutants.py`` runs them on deliberately altered copies of it and
+requires every alteration to be caught by at least one pin.
+
+What the pages fix (Echo digests: [rit.work "Echo 4-bit GPU communication",
+section "How Echo returns the error to later calls"], [heraldofai.com "Come
+Echo permette ai modelli AI...", section "Come Echo evita che gli errori si
+accumulino"]):
+  * segments travel as 4-bit integers; the owner restores and sums them in high
+    precision, then sends back a 4-bit total: at most two roundings per element
+    whatever the group size;
+  * the error of the owner's rounding is measured from the high-precision sum
+    and added back in later calls, through a fast and a slow smoothed estimate;
+  * with the correction, the running sum of injected error stays bounded;
+    without it, it keeps growing.
+Everything else (group, scale rule, rounding, op order, coefficients) is a
+fixed reading, pinned here by hand-worked values and closed forms.
+"""
+from __future__ import annotations
+
+import json
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+
+from bit_error_compensated_rank_b200.workloads import bf16_bits, bf16_to_f32, gaussian, rng
+from bruteforce import bf_quantize, value_of
+from oracle.oracle import Params
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+F32 = np.float32
+
+
+def _load(name):
+    with open(os.path.join(GOLDEN, name)) as fh:
+        return json.load(fh)
+
+
+def _parse_value(expr: str) -> np.float32:
+    """Parse the small expressions of the boundary fixture: a decimal or a
+    fraction, ``2^k``, ``a*2^k``, ``next_up(expr)``, ``FLT_MAX``."""
+    expr = expr.strip()
+    if expr == "FLT_MAX":
+        return np.finfo(F32).max
+    if expr.startswith("next_up(") and expr.endswith(")"):
+        return np.nextafter(_parse_value(expr[len("next_up("):-1]), F32(np.inf))
+    if "2^" in expr:
+        coef, _, power = expr.partition("2^")
+        coef = coef.rstrip("*") or "1"
+        return F32(math.ldexp(float(Fraction(coef)), int(power)))
+    return F32(float(Fraction(expr)))
+
+
+def _frac_list(items):
+    return [Fraction(t) for t in items]
+
+
+def _values(x_bits_or_f32):
+    a = np.asarray(x_bits_or_f32)
+    return bf16_to_f32(a) if a.dtype == np.uint16 else a.astype(F32)
+
+
+def _unpack_ref(packed) -> list[int]:
+    """Layout reading: element 2j in the low nibble, 2j+1 in the high nibble,
+    two's complement."""
+    out = []
+    for byte in np.asarray(packed, dtype=np.uint8).tolist():
+        for nib in (byte & 0xF, byte >> 4):
+            out.append(nib - 16 if nib >= 8 else nib)
+    return out
+
+
+# ---------------------------------------------------------------------------
+# codec
+# ---------------------------------------------------------------------------
+def pin_scale_boundaries(orc):
+    """Hand-worked scale bytes at every boundary of the scale rule, and halves
+    rounded to even (fixture ``scale_boundaries.json``)."""
+    fx = _load("scale_boundaries.json")
+    for case in fx["scale_cases"]:
+        A = _parse_value(case["A"])
+        for sign in (1, -1):
+            v = np.zeros(32, F32)
+            v[5] = F32(sign) * A
+            v[9] = A * F32(0.25)
+            b, _ = orc.quantize_group(v)
+            assert b == case["byte"], (case, b)
+    t = fx["tie_cases_at_e0"]
+    v = np.zeros(32, F32)
+    vals = [F32(float(Fraction(s))) for s in t["values"]]
+    v[:len(vals)] = vals
+    b, q = orc.quantize_group(v)
+    assert b == 127
+    assert q[:len(vals)].tolist() == t["codes"], q[:len(vals)].tolist()
+
+
+def _random_groups(count, G, seed):
+    g = rng(seed, 99)
+    groups = []
+    for t in range(count):
+        kind = t % 6
+        if kind == 0:      # wide range of magnitudes
+            v = g.standard_normal(G) * 2.0 ** g.integers(-140, 100)
+        elif kind == 1:    # halves on a known grid: many ties
+            e = int(g.integers(-120, 100))
+            k = g.integers(-7, 7, G) + 0.5
+            k[0] = 7 * (1 if g.random() < 0.5 else -1)
+            v = k * 2.0 ** e
+        elif kind == 2:    # subnormal binary32 values
+            v = g.integers(-2 ** 20, 2 ** 20, G) * 2.0 ** -149
+        elif kind == 3:    # a single non-zero value
+            v = np.zeros(G)
+            v[g.integers(0, G)] = g.standard_normal() * 2.0 ** g.integers(-30, 30)
+        elif kind == 4:    # values near the 7*2^e boundary
+            e = int(g.integers(-100, 100))
+            v = g.uniform(-1, 1, G) * 7 * 2.0 ** e
+            v[g.integers(0, G)] = np.nextafter(F32(7 * 2.0 ** e), F32(np.inf * (1 if g.random() < .5 else -1)))
+        else:              # bf16-representable values
+            v = bf16_to_f32(bf16_bits(g.standard_normal(G).astype(F32) * 3))
+        groups.append(np.asarray(v, dtype=np.float64).astype(F32))
+    return groups
+
+
+def pin_quantizer_bruteforce(orc):
+    """Scale byte and every code equal an exhaustive search over exponents and
+    codes (ties to even), over ties, subnormals, boundaries and wide ranges."""
+    for G in (32, 8, 2):
+        for v in _random_groups(60 if G == 32 else 24, G, seed=G):
+            b, q = orc.quantize_group(v)
+            bb, bq = bf_quantize(v.tolist())
+            assert b == bb, (v, b, bb)
+            assert q.tolist() == bq, (v, q.tolist(), bq)
+
+
+def pin_roundtrip_bound(orc):
+    """One rounding moves a value by at most half a step: |v - q*2^e| <= 2^(e-1)
+    and |q| <= 7."""
+    for v in _random_groups(120, 32, seed=7):
+        b, q = orc.quantize_group(v)
+        half = Fraction(2) ** (b - 127 - 1)
+        for vi, qi in zip(v.tolist(), q.tolist()):
+            assert -7 <= qi <= 7
+            assert abs(Fraction(vi) - value_of(qi, b)) <= half
+
+
+def pin_pack_layout(orc):
+    """Two codes per byte, element 2j low, 2j+1 high, two's complement nibbles;
+    unpack inverts pack for every pair of nibble values."""
+    q = np.array([1, -1, -7, 7, 0, -2, 6, 3], np.int8)
+    assert orc.pack(q).tolist() == [0xF1, 0x79, 0xE0, 0x36]
+    pairs = [(a, b) for a in range(-8, 8) for b in range(-8, 8)]
+    flat = np.array([c for p in pairs for c in p], np.int8)
+    packed = orc.pack(flat)
+    assert _unpack_ref(packed) == flat.tolist()
+    assert orc.unpack(packed).tolist() == flat.tolist()
+    for b in list(range(0, 253, 11)) + [253]:
+        for qv in ((-3, -1, 0, 1, 3) if b == 253 else (-7, -1, 0, 3, 7)):
+            assert Fraction(orc.dequant(qv, b)) == value_of(qv, b)
+
+
+# ---------------------------------------------------------------------------
+# whole calls
+# ---------------------------------------------------------------------------
+def pin_hand_example(orc):
+    """Four calls of the hand-worked example (fixture
+    ``hand_example_p2_g32.json``): every wire byte, output, correction, error
+    and state value, for bf16 and binary32 inputs."""
+    fx = _load("hand_example_p2_g32.json")
+    n = fx["n"]
+    prm = Params(lam=float(Fraction(fx["params"]["lambda"])),
+                 beta_fast=float(Fraction(fx["params"]["beta_fast"])),
+                 beta_slow=float(Fraction(fx["params"]["beta_slow"])), enable=True)
+    x32 = np.zeros((2, n), F32)
+    x32[0, :4] = [float(v) for v in _frac_list(fx["x"]["rank0"])]
+    x32[1, :4] = [float(v) for v in _frac_list(fx["x"]["rank1"])]
+    for x in (bf16_bits(x32), x32):
+        f = np.zeros(n, F32)
+        s = np.zeros(n, F32)
+        for call in fx["calls"]:
+            res = orc.allreduce(x, f, s, prm, want_diag=True)
+            for key in ("c", "err", "f", "s", "out"):
+                want = [Fraction(t) for t in call[key]] + [Fraction(0)] * (n - 4)
+                have = {"c": res["c"], "err": res["err"], "f": f, "s": s,
+                        "out": _values(res["out"])}[key]
+                assert [Fraction(float(h)) for h in have] == want, (key, have[:4])
+            assert res["codes1"][0, :2].tolist() == call["codes1_rank0"]
+            assert res["codes1"][1, :2].tolist() == call["codes1_rank1"]
+            assert not res["codes1"][:, 2:].any()
+            assert res["scales1"].tolist() == call["scales1"]
+            assert res["qcodes"][:2].tolist() == call["qcodes"]
+            assert not res["qcodes"][2:].any()
+            assert res["qscales"].tolist() == call["qscales"]
+
+
+def _grid_partials(P, ngroups, G, seed):
+    """Partials that rounding #1 reproduces exactly: each group is k*2^e_rg,
+    |k| <= 7, with one |k| in 4..7 so that e_rg is the group's scale. Exponents
+    stay within a span of 8 so binary32 sums are exact."""
+    g = rng(seed, 31, P)
+    e0 = int(g.integers(-40, 30))
+    k = g.integers(-7, 8, (P, ngroups, G))
+    lead = g.integers(0, G, (P, ngroups))
+    sign = np.where(g.random((P, ngroups)) < 0.5, -1, 1)
+    for r in range(P):
+        for j in range(ngroups):
+            k[r, j, lead[r, j]] = sign[r, j] * g.integers(4, 8)
+    e = e0 + g.integers(0, 9, (P, ngroups))
+    x = (k * np.exp2(e)[:, :, None].astype(np.float64)).astype(F32)
+    return x.reshape(P, ngroups * G), k, e
+
+
+def pin_exact_sums_on_grid(orc):
+    """With partials already on their 4-bit grid, rounding #1 is exact, the sum
+    is exact, and the result equals the exhaustive quantiser applied to the
+    exact sum; err = exact sum - result. Covers P from 2 to 16, both dtypes,
+    compensation off and a first call with it on (zero state)."""
+    G = 32
+    for P in (2, 3, 4, 8, 16):
+        ngroups = 2 * P
+        m = ngroups * G
+        x32, k, e = _grid_partials(P, ngroups, G, seed=P)
+        exact = [sum(Fraction(float(x32[r, i])) for r in range(P)) for i in range(m)]
+        want_Y, want_bytes = [], []
+        for j in range(ngroups):
+            b, q = bf_quantize([float(t) for t in exact[j * G:(j + 1) * G]])
+            want_bytes.append(b)
+            want_Y += [value_of(c, b) for c in q]
+        for x in (x32, bf16_bits(x32)):
+            for enable in (False, True):
+                f = np.zeros(m, F32)
+                s = np.zeros(m, F32)
+                res = orc.allreduce(x, f, s, Params(enable=enable), want_diag=True)
+                assert res["scales1"].tolist() == (e + 127).tolist()
+                for r in range(P):
+                    assert _unpack_ref(res["codes1"][r]) == k[r].reshape(-1).tolist()
+                assert res["qscales"].tolist() == want_bytes
+                out = [Fraction(float(t)) for t in _values(res["out"])]
+                assert out == want_Y
+                err = [Fraction(float(t)) for t in res["err"]]
+                assert err == [a - b for a, b in zip(exact, want_Y)]
+
+
+def pin_p2_enumeration(orc):
+    """P = 2, every pair of codes (a, b) in [-7, 7]^2 at one position, with rank
+    0 at scale 2^0 and rank 1 at 2^-1 (fixed by a 7 elsewhere in each group):
+    the total a + b/2 is exact and the result is the exhaustive quantiser of the
+    exact total (every tie of rounding #2 appears)."""
+    G = 32
+    pairs = [(a, b) for a in range(-7, 8) for b in range(-7, 8)]
+    ngroups = 2 * len(pairs)      # pairs in segment 0, copies in segment 1
+    m = ngroups * G
+    x = np.zeros((2, m), F32)
+    for j, (a, b) in enumerate(pairs * 2):
+        x[0, j * G] = a
+        x[0, j * G + 1] = 7
+        x[1, j * G] = b * 0.5
+        x[1, j * G + 1] = 3.5
+    res = orc.allreduce(bf16_bits(x), params=Params(enable=False))
+    out = _values(res["out"])
+    for j, (a, b) in enumerate(pairs * 2):
+        grp = [Fraction(a) + Fraction(b, 2), Fraction(21, 2)] + [Fraction(0)] * (G - 2)
+        byte, q = bf_quantize([float(t) for t in grp])
+        assert res["qscales"][j] == byte
+        assert Fraction(float(out[j * G])) == value_of(q[0], byte), (a, b)
+        assert Fraction(float(out[j * G + 1])) == value_of(q[1], byte)
+
+
+def pin_rank_order(orc):
+    """The owner adds in binary32, rank 0 first. Ranks 0, 1, 2 send 2^24, 1 and
+    -2^24 (each exact after rounding #1): in that order binary32 gives
+    (2^24 + 1) -> 2^24 (half to even), then 0; any other order, or a wider
+    accumulator, gives 1."""
+    G = 32
+    P = 3
+    m = P * G
+    x = np.zeros((P, m), F32)
+    x[0, 0] = 2.0 ** 24
+    x[1, 0] = 1.0
+    x[2, 0] = -(2.0 ** 24)
+    for xx in (x, bf16_bits(x)):
+        res = orc.allreduce(xx, params=Params(enable=False), want_diag=True)
+        assert float(_values(res["out"])[0]) == 0.0
+        assert float(res["err"][0]) == 0.0
+        assert res["qscales"][0] == 0
+
+
+def pin_owner_injection(orc):
+    """Only the owner adds the correction, once, on its own contiguous segment.
+    Zero partials and f = s = 3/4 everywhere: c = 3/4, so each rank's codes are
+    6 at scale 2^-3 on its own segment and 0 elsewhere, every rank receives
+    exactly 3/4, err = 0, then f = 3/8 and s = 21/32."""
+    G = 32
+    P = 4
+    m = P * G * 2
+    x = np.zeros((P, m), np.uint16)
+    f = np.full(m, 0.75, F32)
+    s = np.full(m, 0.75, F32)
+    res = orc.allreduce(x, f, s, Params(), want_diag=True)
+    seg = m // P
+    for r in range(P):
+        codes = _unpack_ref(res["codes1"][r])
+        for i in range(m):
+            assert codes[i] == (6 if i // seg == r else 0), (r, i)
+        for j in range(m // G):
+            assert res["scales1"][r, j] == (124 if (j * G) // seg == r else 0)
+    assert (bf16_to_f32(res["out"]) == F32(0.75)).all()
+    assert (res["err"] == 0).all()
+    assert (f == F32(0.375)).all() and (s == F32(0.65625)).all()
+
+
+def pin_degenerate(orc):
+    """All-zero partials give scale byte 0, codes 0, output 0; opposite partials
+    on two ranks cancel exactly (rounding is symmetric)."""
+    G = 32
+    P = 2
+    m = P * G * 3
+    zero = np.zeros((P, m), np.uint16)
+    f = np.zeros(m, F32)
+    s = np.zeros(m, F32)
+    res = orc.allreduce(zero, f, s, Params(), want_diag=True)
+    assert not res["codes1"].any() and not res["scales1"].any()
+    assert not res["qcodes"].any() and not res["qscales"].any()
+    assert not res["out"].any() and not f.any() and not s.any()
+    x = gaussian(1, m, seed=3, call=0, dtype="fp32")[0]
+    opp = np.stack([x, -x])
+    res = orc.allreduce(opp, params=Params(enable=False), want_diag=True)
+    c0 = _unpack_ref(res["codes1"][0])
+    c1 = _unpack_ref(res["codes1"][1])
+    assert c1 == [-c for c in c0]
+    assert (res["out"] == 0).all() and (res["err"] == 0).all()
+
+
+def pin_error_feedback_special_case(orc):
+    """lambda = 1, beta_fast = 0 turns the compensator into textbook error
+    feedback: the correction of call k is exactly the error captured in call
+    k-1, so the running sum D_K = sum_{k<K} (c_k - err_k) telescopes to
+    exactly -err_{K-1}."""
+    P, G = 4, 32
+    m = P * G * 4
+    f = np.zeros(m, F32)
+    s = np.zeros(m, F32)
+    prm = Params(lam=1.0, beta_fast=0.0, beta_slow=0.875)
+    cs, errs = [], []
+    for k in range(12):
+        res = orc.allreduce(gaussian(P, m, seed=5, call=k), f, s, prm, want_diag=True)
+        cs.append(res["c"].astype(np.float64))
+        errs.append(res["err"].astype(np.float64))
+    assert not cs[0].any()
+    for k in range(1, len(cs)):
+        assert (cs[k] == errs[k - 1]).all()
+    for K in range(1, len(cs) + 1):
+        for i in range(0, m, 7):
+            D = math.fsum([cs[k][i] - errs[k][i] for k in range(K)])
+            assert D == -errs[K - 1][i]
+
+
+def pin_bounded_partial_sum(orc):
+    """Defaults (lambda = 1/2, beta_fast = 1/2, beta_slow = 7/8). The correction
+    of call k is sum_j h_{k-1-j} err_j with sum_m h_m = 1, so
+    D_K = -sum_j err_j * tail_{K-1-j}, tail_t = (beta_f^t + beta_s^t)/2, and
+    |D_K| <= max|err| * (1/2/(1-1/2) + 1/2/(1-7/8)) = 5 max|err| for every K.
+    Without compensation D_K = -sum err_k grows like sqrt(K)."""
+    P, G, K = 4, 32, 96
+    m = P * G * 8
+    f = np.zeros(m, F32)
+    s = np.zeros(m, F32)
+    D_on = np.zeros(m)
+    emax = np.zeros(m)
+    D_off = np.zeros(m)
+    for k in range(K):
+        x = gaussian(P, m, seed=9, call=k)
+        res = orc.allreduce(x, f, s, Params(), want_diag=True)
+        D_on += res["c"].astype(np.float64) - res["err"].astype(np.float64)
+        emax = np.maximum(emax, np.abs(res["err"].astype(np.float64)))
+        assert (np.abs(D_on) <= 5.0 * emax * (1 + 1e-4) + 1e-30).all(), k
+        off = orc.allreduce(x, params=Params(enable=False), want_diag=True)
+        assert not off["c"].any()
+        D_off -= off["err"].astype(np.float64)
+    rms_on = math.sqrt(float(np.mean(D_on ** 2)))
+    rms_off = math.sqrt(float(np.mean(D_off ** 2)))
+    assert rms_on < 0.35 * rms_off, (rms_on, rms_off)
+
+
+def pin_two_roundings_bound(orc):
+    """Each element passes through at most two roundings whatever P:
+    |Y - sum_r v_r| <= sum_r 2^(e_r - 1) + 2^(E - 1) + (P-1) * 2^-24 * sum_r |q_r 2^e_r|
+    (the last term bounds the binary32 additions), with v_r the value rank r
+    rounds (its partial, plus c at the owner)."""
+    G = 32
+    for P in (2, 8, 16):
+        m = P * G * 2
+        f = np.zeros(m, F32)
+        s = np.zeros(m, F32)
+        owner = np.arange(m) // (m // P)
+        for k in range(4):
+            x = gaussian(P, m, seed=P, call=k, dtype="fp32")
+            x[:, ::97] *= 50
+            res = orc.allreduce(x, f, s, Params(), want_diag=True)
+            Y = res["out"].astype(np.float64)
+            for i in range(0, m, 5):
+                j = i // G
+                total = Fraction(0)
+                bound = Fraction(2) ** (int(res["qscales"][j]) - 128)
+                mag = Fraction(0)
+                for r in range(P):
+                    v = x[r, i]
+                    if owner[i] == r:
+                        v = F32(v + res["c"][i])
+                    total += Fraction(float(v))
+                    b = int(res["scales1"][r, j])
+                    q = _unpack_ref(res["codes1"][r][i // 2:i // 2 + 1])[i % 2]
+                    bound += Fraction(2) ** (b - 128)
+                    mag += abs(value_of(q, b))
+                bound += (P - 1) * Fraction(1, 2 ** 24) * mag
+                assert abs(Fraction(float(Y[i])) - total) <= bound, (P, k, i)
+
+
+def pin_power_of_two_equivariance(orc):
+    """Scaling every partial and the state by 2^t scales every output, error
+    and state value by exactly 2^t and shifts every non-zero scale byte by t;
+    the codes do not change."""
+    P, G = 4, 32
+    m = P * G * 4
+    for dtype in ("bf16", "fp32"):
+        for t in (-9, 13):
+            f0, s0 = np.zeros(m, F32), np.zeros(m, F32)
+            f1, s1 = np.zeros(m, F32), np.zeros(m, F32)
+            for k in range(4):
+                x = gaussian(P, m, seed=11, call=k, dtype="fp32")
+                xs = (x * np.float32(2.0 ** t)).astype(F32)
+                if dtype == "bf16":
+                    x, xs = bf16_bits(x), bf16_bits(xs)
+                a = orc.allreduce(x, f0, s0, Params(), want_diag=True)
+                b = orc.allreduce(xs, f1, s1, Params(), want_diag=True)
+                scale = F32(2.0 ** t)
+                assert (_values(b["out"]) == _values(a["out"]) * scale).all()
+                assert (b["err"] == a["err"] * scale).all()
+                assert (f1 == f0 * scale).all() and (s1 == s0 * scale).all()
+                assert (a["codes1"] == b["codes1"]).all() and (a["qcodes"] == b["qcodes"]).all()
+                nz = a["scales1"] != 0
+                assert (b["scales1"][nz].astype(int) == a["scales1"][nz].astype(int) + t).all()
+                nzq = a["qscales"] != 0
+                assert (b["qscales"][nzq].astype(int) == a["qscales"][nzq].astype(int) + t).all()
+
+
+ALL_PINS = [
+    pin_scale_boundaries,
+    pin_quantizer_bruteforce,
+    pin_roundtrip_bound,
+    pin_pack_layout,
+    pin_hand_example,
+    pin_exact_sums_on_grid,
+    pin_p2_enumeration,
+    pin_rank_order,
+    pin_owner_injection,
+    pin_degenerate,
+    pin_error_feedback_special_case,
+    pin_bounded_partial_sum,
+    pin_two_roundings_bound,
+    pin_power_of_two_equivariance,
+]

@@ -1,0 +1,106 @@
+"""Plant plausible mistakes in copies of the oracle and require the pins to
+catch every one.
+
+Each mutant is the oracle's C source with one textual change, compiled to a
+temporary library on the CPU. A mutant passes this test only if at least one
+pin in ``pins.ALL_PINS`` fails on it; a mutant no pin notices would mean the
+pins do not actually tie that part of the oracle down.
+"""
+import os
+import shutil
+import subprocess
+
+import pytest
+
+from oracle.oracle import Oracle
+from pins import ALL_PINS
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+ORACLE_DIR = os.path.join(ROOT, "oracle")
+
+MUTANTS = [
+    ("ties_away_from_zero",
+     "double t = nearbyint(ldexp((double)v[k], -e));",
+     "double t = round(ldexp((double)v[k], -e));"),
+    ("scale_strict_boundary",
+     "while (!(A <= ldexp(7.0, e))) {",
+     "while (!(A < ldexp(7.0, e))) {"),
+    ("scale_range_8",
+     "while (!(A <= ldexp(7.0, e))) {",
+     "while (!(A <= ldexp(8.0, e))) {"),
+    ("absmax_wrong_compare",
+     "if (a > A)\n            A = a;",
+     "if (a < A)\n            A = a;"),
+    ("nibbles_swapped",
+     "out[j] = (uint8_t)(lo | (hi << 4));",
+     "out[j] = (uint8_t)(hi | (lo << 4));"),
+    ("dequant_off_by_one",
+     "return (float)ldexp((double)q, b - 127);",
+     "return (float)ldexp((double)q, b - 126);"),
+    ("sum_skips_rank0",
+     "for (int r = 0; r < P; r++) {\n                float d",
+     "for (int r = 1; r < P; r++) {\n                float d"),
+    ("sum_reversed_order",
+     "float d = echo_oracle_dequant(q1[(size_t)r * m + i], b1[(size_t)r * ngroups + g]);",
+     "float d = echo_oracle_dequant(q1[(size_t)(P - 1 - r) * m + i], b1[(size_t)(P - 1 - r) * ngroups + g]);"),
+    ("sum_in_binary64",
+     "float sum = 0.0f;",
+     "double sum = 0.0;"),
+    ("error_sign_flipped",
+     "float err = S[k] - Y;",
+     "float err = Y - S[k];"),
+    ("combine_minus",
+     "c[i] = from_fast + from_slow;",
+     "c[i] = from_fast - from_slow;"),
+    ("lambda_on_slow",
+     "float from_fast = lambda * f[i];",
+     "float from_fast = lambda * s[i];"),
+    ("every_rank_injects",
+     "if (enable && owner[g] == r)",
+     "if (enable)"),
+    ("wrong_owner",
+     "owner[g] = (int32_t)((g * (size_t)G) / seg);",
+     "owner[g] = (int32_t)(((g * (size_t)G) / seg + 1) % (size_t)P);"),
+    ("fast_uses_slow_beta",
+     "float f_keep = beta_f * f[i];",
+     "float f_keep = beta_s * f[i];"),
+    ("slow_weights_swapped",
+     "float s_new = one_minus_beta_s * err;",
+     "float s_new = beta_s * err;"),
+    ("state_not_updated",
+     "f[i] = f_keep + f_new;",
+     "f[i] = f[i];"),
+    ("captures_stage1_error_instead",
+     "float Y = echo_oracle_dequant(Q[i], bq);",
+     "float Y = S[k];"),
+    ("correction_not_added",
+     "v[k] = xi + c[i];",
+     "v[k] = xi;"),
+]
+
+
+@pytest.fixture(scope="module")
+def mutant_dir(tmp_path_factory):
+    return tmp_path_factory.mktemp("oracle_mutants")
+
+
+@pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_pins_catch_mutant(mutant_dir, name, old, new):
+    src = open(os.path.join(ORACLE_DIR, "echo_oracle.c")).read()
+    assert src.count(old) == 1, f"mutation site for {name} not unique/present"
+    work = os.path.join(str(mutant_dir), name)
+    os.makedirs(work, exist_ok=True)
+    shutil.copy(os.path.join(ORACLE_DIR, "echo_oracle.h"), work)
+    with open(os.path.join(work, "echo_oracle.c"), "w") as fh:
+        fh.write(src.replace(old, new))
+    lib = os.path.join(work, "libmutant.so")
+    subprocess.run(["gcc", "-std=c99", "-O2", "-ffp-contract=off", "-fPIC", "-shared",
+                    "-o", lib, os.path.join(work, "echo_oracle.c"), "-lm"], check=True)
+    orc = Oracle(lib)
+    caught = []
+    for pin in ALL_PINS:
+        try:
+            pin(orc)
+        except Exception:  # any failure, assertion or error, counts as caught
+            caught.append(pin.__name__)
+    assert caught, f"no pin catches mutant {name}"
