@@ -1,0 +1,419 @@
+"""Benchmark of the Echo error-compensated 4-bit all-reduce on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl echo|reference]
+
+Workload (one step = one all-reduce call, the whole hot path: compensate +
+quantise + pack, owner reduce + requantise, gather + dequantise): P = 8
+simulated tensor-parallel ranks, a 1 GiB bf16 message per rank (2^29
+elements), partials N(0, 1) with 0.1 % of values at 50x, group 32,
+compensation on, forward state. The ranks are 8 buffers in one GPU's HBM.
+
+Metric: bf16-equivalent all-reduce bandwidth, algbw = 2 n / t_call (the
+nccl-tests definition), and the call's fraction of the HBM roofline, where
+the roofline time is the three kernels' algorithmic bytes divided by the
+measured HBM copy bandwidth.
+
+With N > 1 (one process per GPU under torchrun) every GPU runs its own
+independent 8-rank problem (weak scaling, no collective on the data path);
+the value is the sum of all GPUs' work divided by the slowest GPU's time.
+
+``--impl reference`` times the plain CPU oracle instead (the slow reference
+program this library is checked against), on a bounded sample of the same
+workload per step; under torchrun only rank 0 runs it.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "bf16-equiv all-reduce GB/s and % of HBM roofline at P=8, 1 GiB msg"
+UNIT = "GB/s"
+P = 8
+N_ELEMS = 1 << 29          # 1 GiB of bf16 per rank
+SEED = 0
+WORKLOAD = "echo int4 all-reduce, P=8 ranks x 1 GiB bf16 per rank (2^29 elements), group 32, " \
+           "compensation on, fwd state, partials N(0,1) with 0.1% at 50x"
+HBM_FALLBACK_GBS = 6650.0  # used only when MEASURED_PEAKS.json is absent
+# CPU baseline / reference arm samples (elements per rank, same distribution)
+CPU_SAMPLE_N = 1 << 20
+REF_SAMPLE_N = 1 << 18
+
+
+# ---------------------------------------------------------------------------
+# process group plumbing
+# ---------------------------------------------------------------------------
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def init_dist(world: int, backend: str):
+    import datetime
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def barrier(world: int, device=None):
+    if world > 1:
+        import torch.distributed as dist
+        if device is not None:
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device if device is not None else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(value: float, world: int, device=None) -> float:
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device if device is not None else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# measured peaks and clocks
+# ---------------------------------------------------------------------------
+def hbm_peak() -> tuple[float, str]:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as fh:
+            return float(json.load(fh)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return HBM_FALLBACK_GBS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while running."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str, period_ms: int = 50):
+        self.gpu_id = gpu_id
+        self.period_ms = period_ms
+        self.rows: list[list[str]] = []
+        self.proc = None
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", str(self.period_ms)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+        time.sleep(0.3)
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append([c.strip() for c in line.split(",")])
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.1)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=5)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for row in self.rows:
+            if len(row) < 8:
+                continue
+            try:
+                sm.append(float(row[0]))
+                smax.append(float(row[1]))
+            except ValueError:
+                continue
+            for name, val in zip(names, row[4:8]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def gpu_selector(local_rank: int) -> str:
+    import torch
+    try:
+        uuid = str(torch.cuda.get_device_properties(local_rank).uuid)
+        return uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+    except Exception:
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+        if vis:
+            return vis.split(",")[local_rank]
+        return str(local_rank)
+
+
+# ---------------------------------------------------------------------------
+# the CPU oracle (baseline leg and reference arm)
+# ---------------------------------------------------------------------------
+def oracle_sample_rate(n_sample: int, budget_s: float, min_calls: int, max_calls: int, seed: int):
+    """Time the oracle on P x n_sample bf16 partials of the workload's
+    distribution, call after call (state carried), until budget_s is spent."""
+    import numpy as np
+    from bit_error_compensated_rank_b200 import workloads as wl
+    from oracle.oracle import Oracle, Params
+    orc = Oracle()
+    f = np.zeros(n_sample, np.float32)
+    s = np.zeros(n_sample, np.float32)
+    times = []
+    t_all = time.perf_counter()
+    k = 0
+    while k < min_calls or (time.perf_counter() - t_all < budget_s and k < max_calls):
+        x = wl.outlier_gaussian(P, n_sample, seed=seed, call=k)
+        t0 = time.perf_counter()
+        orc.allreduce(x, f, s, Params(), want_wire=False)
+        times.append(time.perf_counter() - t0)
+        k += 1
+    return times
+
+
+def cpu_baseline_leg() -> dict:
+    times = oracle_sample_rate(CPU_SAMPLE_N, budget_s=10.0, min_calls=3, max_calls=60, seed=1)
+    t = sum(times) / len(times)
+    return {
+        "value": round(2 * CPU_SAMPLE_N / t / 1e9, 6), "unit": UNIT, "cores": 1, "kind": "oracle",
+        "sample": f"P=8 x 2^20 bf16 elements per rank (2 MiB), same distribution, compensation on, "
+                  f"{len(times)} sequential calls, {sum(times):.1f} s single-threaded; "
+                  f"value = 2*n/t per call (bf16-equivalent)",
+    }
+
+
+def run_reference(args, rank: int, world: int) -> dict | None:
+    if rank != 0:
+        return None
+    times = oracle_sample_rate(REF_SAMPLE_N, budget_s=0.0, min_calls=args.warmup + args.steps,
+                               max_calls=args.warmup + args.steps, seed=2)
+    timed = times[args.warmup:]
+    t = sum(timed) / len(timed)
+    value = 2 * REF_SAMPLE_N / t / 1e9
+    sample = (f"P=8 x 2^18 bf16 elements per rank per step (512 KiB), same distribution as the "
+              f"1 GiB workload, compensation on; oracle single-threaded on the host")
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(t * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "P": P, "n_per_rank": N_ELEMS, "sample_n_per_rank": REF_SAMPLE_N,
+                   "parallelism": f"{world} independent replica(s)"},
+        "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+# ---------------------------------------------------------------------------
+# the CUDA path
+# ---------------------------------------------------------------------------
+# DRAM traffic per element of n for each kernel from one ncu capture
+# (dram__bytes_read.sum + dram__bytes_write.sum / n); reported only while the
+# kernel source still has the hash it had when captured.
+NCU_TRAFFIC = {}
+
+
+def _source_hash(path: str) -> str:
+    import hashlib
+    with open(path, "rb") as fh:
+        return hashlib.sha256(fh.read()).hexdigest()[:16]
+
+
+def run_echo(args, rank: int, world: int, local: int) -> dict | None:
+    import torch
+    from bit_error_compensated_rank_b200 import echo
+    from bit_error_compensated_rank_b200 import workloads as wl
+
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    dist = init_dist(world, "nccl")
+    n = args.n
+    stream = torch.cuda.current_stream(device)
+
+    # inputs resident in HBM before timing; outputs to separate buffers so
+    # every step sees the same fresh partials (out-of-place call, same bytes)
+    send = [torch.empty(n, dtype=torch.bfloat16, device=device) for _ in range(P)]
+    recv = [torch.empty(n, dtype=torch.bfloat16, device=device) for _ in range(P)]
+    for r in range(P):
+        wl.torch_outlier_gaussian_(send[r], seed=SEED + 1000 * rank, call=0, rank=r)
+    h = echo.Echo(P, n, echo.ECHO_BF16)
+    mb = echo.echo_model_bytes(P, n, echo.ECHO_BF16, True)
+    torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        h.allreduce_out(send, recv, echo.ECHO_FWD, stream)
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(gpu_selector(local))
+    clocks.start()
+    h.set_timing(True)
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    barrier(world, device)
+    torch.cuda.synchronize()
+    start.record(stream)
+    for _ in range(args.steps):
+        h.allreduce_out(send, recv, echo.ECHO_FWD, stream)
+    end.record(stream)
+    torch.cuda.synchronize()
+    barrier(world, device)
+    clk = clocks.stop()
+    h.set_timing(False)
+    kern_ms, timed_calls = h.kernel_ms_total()
+    elapsed_ms = start.elapsed_time(end)
+    ms_step = max_over_ranks(elapsed_ms / args.steps, world, device)
+    assert timed_calls == args.steps
+
+    # whole-job throughput: every GPU moved 2n bf16-equivalent bytes per step
+    total_bytes = sum_over_ranks(2.0 * n * args.steps, world, device)
+    value = total_bytes / (ms_step * args.steps * 1e-3) / 1e9
+    peak, peak_kind = hbm_peak()
+    call_bytes = mb["total"]
+    call_frac = call_bytes / (ms_step * 1e-3) / (peak * 1e9)
+
+    k_avg = [t / timed_calls for t in kern_ms]
+    names = ["k1_compensate_quantize_pack", "k2_owner_reduce_requant", "k3_gather_dequant"]
+    k_bytes = [mb["k1"], mb["k2"], mb["k3"]]
+    dom = max(range(3), key=lambda i: k_bytes[i])
+    achieved = k_bytes[dom] / (k_avg[dom] * 1e-3) / 1e9
+    src = os.path.join(ROOT, "bit_error_compensated_rank_b200", "csrc", names[dom] + ".cu")
+    traffic = None
+    rec = NCU_TRAFFIC.get(names[dom])
+    if rec and rec["source_sha"] == _source_hash(src):
+        traffic = round(rec["bytes_per_elem"] * n)
+
+    # end to end: pinned host partials in, host result out, through the C ABI
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(h, send, n, args, device, world)
+
+    result = {
+        "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, "P": P, "n_per_rank": n, "group": 32,
+                   "parallelism": f"{world} independent replica(s), ranks simulated in HBM",
+                   "l2": "inputs larger than L2 (8 GiB of partials per GPU vs 126 MB L2)"},
+        "hbm_roofline_frac": round(call_frac, 4),
+        "hbm_roofline": {"model_bytes_per_call": call_bytes,
+                         "bytes_per_elem": round(call_bytes / n, 5),
+                         "peak_gbs": peak, "peak_kind": peak_kind,
+                         "ideal_ms": round(call_bytes / (peak * 1e9) * 1e3, 4)},
+        "busbw": round(value * 2 * (P - 1) / P, 3),
+        "kernel_ms": {names[i]: round(k_avg[i], 4) for i in range(3)},
+        "kernel_frac": {names[i]: round(k_bytes[i] / (k_avg[i] * 1e-3) / 1e9 / peak, 4) for i in range(3)},
+        "link_bytes_per_call": mb["link"],
+        "roofline": {"kernel": names[dom], "bound": "hbm", "achieved": round(achieved, 1),
+                     "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
+                     "traffic": traffic, "peak_kind": peak_kind},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clk,
+    }
+    if e2e is not None:
+        result["e2e"] = e2e
+    h.close()
+    return result if rank == 0 else None
+
+
+def run_e2e(h, send, n, args, device, world) -> dict:
+    """Pinned host partials -> device -> all-reduce -> host result, per step."""
+    import torch
+    steps = max(1, min(args.steps, args.e2e_steps))
+    try:
+        host_in = [torch.empty(n, dtype=torch.bfloat16, pin_memory=True) for _ in range(P)]
+        host_out = torch.empty(n, dtype=torch.bfloat16, pin_memory=True)
+    except RuntimeError as exc:
+        return {"value": None, "unit": UNIT, "error": f"pinned host allocation failed: {exc}"}
+    for r in range(P):
+        host_in[r].copy_(send[r])
+    stream = torch.cuda.current_stream(device)
+    h.allreduce_host(host_in, host_out, 0, stream)  # warm-up (allocates staging)
+    torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    barrier(world, device)
+    start.record(stream)
+    for _ in range(steps):
+        h.allreduce_host(host_in, host_out, 0, stream)
+    end.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(start.elapsed_time(end) / steps, world, device)
+    total = sum_over_ranks(2.0 * n, world, device)
+    return {"value": round(total / (ms * 1e-3) / 1e9, 3), "unit": UNIT,
+            "h2d_bytes_per_step": P * n * 2, "d2h_bytes_per_step": n * 2,
+            "ms_per_step": round(ms, 3), "steps": steps}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["echo", "reference"], default="echo")
+    ap.add_argument("--n", type=int, default=N_ELEMS, help="elements per rank (default 2^29)")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    rank, world, local = dist_env()
+    if world != args.gpus:
+        ap.error(f"--gpus {args.gpus} but WORLD_SIZE is {world}")
+
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return 0
+
+    res = run_echo(args, rank, world, local)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    if res is not None:
+        if world == 1 and not args.no_cpu_baseline:
+            res["cpu_baseline"] = cpu_baseline_leg()
+        print(json.dumps(res), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,296 @@
+"""ctypes binding of ``libecho.so`` (the C ABI in ``include/echo.h``).
+
+Functions keep the C names and only marshal arguments: every step of the
+all-reduce runs in the library's CUDA kernels. There is no fallback: importing
+this module raises ``ImportError`` when the library has not been built, and
+every failing call raises :class:`EchoError` with the library's message.
+
+Device buffers are passed as integer addresses; the helpers that take torch
+tensors read ``data_ptr()`` and the current stream's handle, nothing more.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib", "libecho.so")
+
+ECHO_BF16 = 0
+ECHO_FP32 = 1
+ECHO_FWD = 0
+ECHO_BWD = 1
+ECHO_OK = 0
+ECHO_ERR_INVALID = -1
+ECHO_ERR_UNSUPPORTED = -2
+ECHO_ERR_CUDA = -3
+ECHO_ERR_OOM = -4
+ECHO_MAX_RANKS = 16
+ECHO_GROUP = 32
+
+EXPORTED = (
+    "echo_create", "echo_allreduce", "echo_allreduce_out", "echo_allreduce_host",
+    "echo_reset", "echo_destroy", "echo_last_error", "echo_last_status", "echo_set_params",
+    "echo_get_state", "echo_set_state", "echo_get_state_range", "echo_get_wire",
+    "echo_get_wire_range", "echo_stats", "echo_model_bytes", "echo_set_timing",
+    "echo_last_kernel_ms", "echo_kernel_ms_total",
+)
+
+_vp = ctypes.c_void_p
+_sz = ctypes.c_size_t
+_int = ctypes.c_int
+_f32p = ctypes.POINTER(ctypes.c_float)
+_u8p = ctypes.POINTER(ctypes.c_uint8)
+_u64p = ctypes.POINTER(ctypes.c_uint64)
+_vpp = ctypes.POINTER(ctypes.c_void_p)
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with `python -m bit_error_compensated_rank_b200.build`"
+            " (the CUDA library is the only implementation; there is no fallback)")
+    lib = ctypes.CDLL(LIB_PATH)
+    sig = {
+        "echo_create": (_vp, [_int, _sz, _int, _int]),
+        "echo_allreduce": (_int, [_vp, _vpp, _int, _vp]),
+        "echo_allreduce_out": (_int, [_vp, _vpp, _vpp, _int, _vp]),
+        "echo_allreduce_host": (_int, [_vp, _vpp, _vp, _int, _vp]),
+        "echo_reset": (_int, [_vp, _int]),
+        "echo_destroy": (_int, [_vp]),
+        "echo_last_error": (ctypes.c_char_p, []),
+        "echo_last_status": (_int, []),
+        "echo_set_params": (_int, [_vp, ctypes.c_float, ctypes.c_float, ctypes.c_float, _int]),
+        "echo_get_state": (_int, [_vp, _int, _f32p, _f32p]),
+        "echo_set_state": (_int, [_vp, _int, _f32p, _f32p]),
+        "echo_get_state_range": (_int, [_vp, _int, _sz, _sz, _f32p, _f32p]),
+        "echo_get_wire": (_int, [_vp, _int, _int, _u8p, _u8p]),
+        "echo_get_wire_range": (_int, [_vp, _int, _int, _sz, _sz, _u8p, _u8p]),
+        "echo_stats": (_int, [_vp, _u64p, _u64p, _u64p]),
+        "echo_model_bytes": (_int, [_int, _sz, _int, _int, _u64p]),
+        "echo_set_timing": (_int, [_vp, _int]),
+        "echo_last_kernel_ms": (_int, [_vp, _f32p]),
+        "echo_kernel_ms_total": (_int, [_vp, ctypes.POINTER(ctypes.c_double), _u64p]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+_lib = _load()
+
+
+class EchoError(RuntimeError):
+    def __init__(self, code: int, message: str):
+        super().__init__(f"echo error {code}: {message}")
+        self.code = code
+
+
+def echo_last_error() -> str:
+    return (_lib.echo_last_error() or b"").decode()
+
+
+def echo_last_status() -> int:
+    return _lib.echo_last_status()
+
+
+def _check(rc: int) -> None:
+    if rc != ECHO_OK:
+        raise EchoError(rc, echo_last_error())
+
+
+def _ptr_array(ptrs) -> ctypes.Array:
+    return (ctypes.c_void_p * len(ptrs))(*[int(p) for p in ptrs])
+
+
+def _np(a, ctype):
+    return None if a is None else a.ctypes.data_as(ctype)
+
+
+# ---- the C entry points, one to one --------------------------------------
+def echo_create(P: int, n: int, group: int = ECHO_GROUP, dtype: int = ECHO_BF16) -> int:
+    h = _lib.echo_create(P, n, group, dtype)
+    if not h:
+        raise EchoError(_lib.echo_last_status(), echo_last_error())
+    return h
+
+
+def echo_allreduce(h: int, rank_ptrs, phase: int = ECHO_FWD, stream: int = 0) -> None:
+    _check(_lib.echo_allreduce(h, _ptr_array(rank_ptrs), phase, stream))
+
+
+def echo_allreduce_out(h: int, send_ptrs, recv_ptrs, phase: int = ECHO_FWD, stream: int = 0) -> None:
+    _check(_lib.echo_allreduce_out(h, _ptr_array(send_ptrs), _ptr_array(recv_ptrs), phase, stream))
+
+
+def echo_allreduce_host(h: int, host_send_ptrs, host_recv_ptr: int, phase: int = ECHO_FWD,
+                        stream: int = 0) -> None:
+    _check(_lib.echo_allreduce_host(h, _ptr_array(host_send_ptrs), host_recv_ptr, phase, stream))
+
+
+def echo_reset(h: int, phase_mask: int = 3) -> None:
+    _check(_lib.echo_reset(h, phase_mask))
+
+
+def echo_destroy(h: int) -> None:
+    _check(_lib.echo_destroy(h))
+
+
+def echo_set_params(h: int, beta_fast: float = 0.5, beta_slow: float = 0.875, lam: float = 0.5,
+                    enable: bool = True) -> None:
+    _check(_lib.echo_set_params(h, beta_fast, beta_slow, lam, int(bool(enable))))
+
+
+def echo_get_state(h: int, phase: int, n: int) -> tuple[np.ndarray, np.ndarray]:
+    f = np.empty(n, np.float32)
+    s = np.empty(n, np.float32)
+    _check(_lib.echo_get_state(h, phase, _np(f, _f32p), _np(s, _f32p)))
+    return f, s
+
+
+def echo_set_state(h: int, phase: int, f: np.ndarray, s: np.ndarray) -> None:
+    f = np.ascontiguousarray(f, np.float32)
+    s = np.ascontiguousarray(s, np.float32)
+    _check(_lib.echo_set_state(h, phase, _np(f, _f32p), _np(s, _f32p)))
+
+
+def echo_get_state_range(h: int, phase: int, offset: int, count: int):
+    f = np.empty(count, np.float32)
+    s = np.empty(count, np.float32)
+    _check(_lib.echo_get_state_range(h, phase, offset, count, _np(f, _f32p), _np(s, _f32p)))
+    return f, s
+
+
+def echo_get_wire(h: int, stage: int, rank: int, n: int):
+    codes = np.empty(n // 2, np.uint8)
+    scales = np.empty(n // ECHO_GROUP, np.uint8)
+    _check(_lib.echo_get_wire(h, stage, rank, _np(codes, _u8p), _np(scales, _u8p)))
+    return codes, scales
+
+
+def echo_get_wire_range(h: int, stage: int, rank: int, group_offset: int, ngroups: int):
+    codes = np.empty(ngroups * ECHO_GROUP // 2, np.uint8)
+    scales = np.empty(ngroups, np.uint8)
+    _check(_lib.echo_get_wire_range(h, stage, rank, group_offset, ngroups,
+                                    _np(codes, _u8p), _np(scales, _u8p)))
+    return codes, scales
+
+
+def echo_stats(h: int) -> dict:
+    vals = (ctypes.c_uint64 * 3)()
+    _check(_lib.echo_stats(h, ctypes.byref(vals, 0), ctypes.byref(vals, 8), ctypes.byref(vals, 16)))
+    return {"link_bytes": vals[0], "model_hbm_bytes": vals[1], "calls": vals[2]}
+
+
+def echo_model_bytes(P: int, n: int, dtype: int = ECHO_BF16, enable: bool = True) -> dict:
+    out = (ctypes.c_uint64 * 4)()
+    _check(_lib.echo_model_bytes(P, n, dtype, int(bool(enable)), out))
+    return {"k1": out[0], "k2": out[1], "k3": out[2], "link": out[3],
+            "total": out[0] + out[1] + out[2]}
+
+
+def echo_set_timing(h: int, enable: bool = True) -> None:
+    _check(_lib.echo_set_timing(h, int(bool(enable))))
+
+
+def echo_last_kernel_ms(h: int) -> list[float]:
+    ms = (ctypes.c_float * 3)()
+    _check(_lib.echo_last_kernel_ms(h, ms))
+    return [ms[0], ms[1], ms[2]]
+
+
+def echo_kernel_ms_total(h: int) -> tuple[list[float], int]:
+    ms = (ctypes.c_double * 3)()
+    calls = ctypes.c_uint64()
+    _check(_lib.echo_kernel_ms_total(h, ms, ctypes.byref(calls)))
+    return [ms[0], ms[1], ms[2]], calls.value
+
+
+# ---- torch conveniences (plumbing only) -----------------------------------
+def _dtype_code(t) -> int:
+    import torch
+    if t.dtype == torch.bfloat16:
+        return ECHO_BF16
+    if t.dtype == torch.float32:
+        return ECHO_FP32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _stream(stream) -> int:
+    import torch
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+class Echo:
+    """Owning wrapper of one handle: ``Echo(P, n, dtype)``; call
+    :meth:`allreduce` with P device tensors (torch) of n elements each."""
+
+    def __init__(self, P: int, n: int, dtype: int = ECHO_BF16, group: int = ECHO_GROUP):
+        self.P, self.n, self.dtype = P, n, dtype
+        self.h = echo_create(P, n, group, dtype)
+
+    def allreduce(self, tensors, phase: int = ECHO_FWD, stream=None) -> None:
+        echo_allreduce(self.h, [t.data_ptr() for t in tensors], phase, _stream(stream))
+
+    def allreduce_out(self, send, recv, phase: int = ECHO_FWD, stream=None) -> None:
+        echo_allreduce_out(self.h, [t.data_ptr() for t in send], [t.data_ptr() for t in recv],
+                           phase, _stream(stream))
+
+    def allreduce_host(self, host_send, host_recv, phase: int = ECHO_FWD, stream=None) -> None:
+        echo_allreduce_host(self.h, [t.data_ptr() for t in host_send], host_recv.data_ptr(),
+                            phase, _stream(stream))
+
+    def set_params(self, beta_fast=0.5, beta_slow=0.875, lam=0.5, enable=True) -> None:
+        echo_set_params(self.h, beta_fast, beta_slow, lam, enable)
+
+    def reset(self, phase_mask: int = 3) -> None:
+        echo_reset(self.h, phase_mask)
+
+    def get_state(self, phase: int = ECHO_FWD):
+        return echo_get_state(self.h, phase, self.n)
+
+    def set_state(self, phase: int, f, s) -> None:
+        echo_set_state(self.h, phase, f, s)
+
+    def get_state_range(self, phase: int, offset: int, count: int):
+        return echo_get_state_range(self.h, phase, offset, count)
+
+    def get_wire(self, stage: int, rank: int = 0):
+        return echo_get_wire(self.h, stage, rank, self.n)
+
+    def get_wire_range(self, stage: int, rank: int, group_offset: int, ngroups: int):
+        return echo_get_wire_range(self.h, stage, rank, group_offset, ngroups)
+
+    def stats(self) -> dict:
+        return echo_stats(self.h)
+
+    def set_timing(self, enable: bool = True) -> None:
+        echo_set_timing(self.h, enable)
+
+    def last_kernel_ms(self) -> list[float]:
+        return echo_last_kernel_ms(self.h)
+
+    def kernel_ms_total(self) -> tuple[list[float], int]:
+        return echo_kernel_ms_total(self.h)
+
+    def close(self) -> None:
+        if self.h:
+            echo_destroy(self.h)
+            self.h = None
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.close()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -50,6 +50,10 @@
 extern "C" {
 #endif
 
+#ifndef ECHO_API
+#define ECHO_API __attribute__((visibility("default")))
+#endif
+
 typedef struct echo_handle echo_handle; /* opaque, owned by the library */
 
 typedef enum { ECHO_BF16 = 0, ECHO_FP32 = 1 } echo_dtype;
@@ -69,7 +73,7 @@ enum {
 /*
  * echo_create - a handle for all-reduces of P ranks x n elements of dtype.
  *   P      number of simulated tensor-parallel ranks, 2..16.
- *   n      elements per rank; n % (P*group) == 0 and n <= 2^36.
+ *   n      elements per rank; n % (P*group) == 0 and n <= 2^34.
  *   group  elements per scale; only 32 is built (else ECHO_ERR_UNSUPPORTED).
  *   dtype  ECHO_BF16 or ECHO_FP32: the element type of the rank buffers.
  * Allocates on the current device: stage-1 wire (P x n/2 code bytes and
@@ -78,7 +82,7 @@ enum {
  * Returns NULL on any error (see echo_last_error). The handle is bound to the
  * device that was current at creation.
  */
-echo_handle *echo_create(int P, size_t n, int group, int dtype);
+ECHO_API echo_handle *echo_create(int P, size_t n, int group, int dtype);
 
 /*
  * echo_allreduce - in-place Echo all-reduce of P rank buffers.
@@ -91,14 +95,14 @@ echo_handle *echo_create(int P, size_t n, int group, int dtype);
  * rank_ptrs[r] holds the same value Y = Q*2^E, exactly representable in the
  * dtype, and the phase's state holds the updated estimates.
  */
-int echo_allreduce(echo_handle *h, void *const rank_ptrs[], int phase, void *stream);
+ECHO_API int echo_allreduce(echo_handle *h, void *const rank_ptrs[], int phase, void *stream);
 
 /*
  * echo_allreduce_out - the same all-reduce out of place: reads send_ptrs[r],
  * writes recv_ptrs[r]. Each send buffer may equal its own recv buffer; no
  * other overlap is allowed. Same alignment and size rules.
  */
-int echo_allreduce_out(echo_handle *h, const void *const send_ptrs[],
+ECHO_API int echo_allreduce_out(echo_handle *h, const void *const send_ptrs[],
                        void *const recv_ptrs[], int phase, void *stream);
 
 /*
@@ -110,38 +114,41 @@ int echo_allreduce_out(echo_handle *h, const void *const send_ptrs[],
  * in host_recv (it synchronises the stream). The device staging buffers
  * (P x n elements) are allocated on first use and kept until echo_destroy.
  */
-int echo_allreduce_host(echo_handle *h, const void *const host_send[], void *host_recv,
+ECHO_API int echo_allreduce_host(echo_handle *h, const void *const host_send[], void *host_recv,
                         int phase, void *stream);
 
 /* echo_reset - zero the compensator state of the phases in phase_mask
  * (bit 0 forward, bit 1 backward), enqueued on the legacy default stream and
  * completed before return. */
-int echo_reset(echo_handle *h, int phase_mask);
+ECHO_API int echo_reset(echo_handle *h, int phase_mask);
 
 /* echo_destroy - free everything the handle owns (synchronises the device
  * first). NULL is a no-op. The handle must not be used afterwards. */
-int echo_destroy(echo_handle *h);
+ECHO_API int echo_destroy(echo_handle *h);
 
 /* echo_last_error - message of the last failed call on this thread
- * ("" if none). The string stays valid until the thread's next failing call. */
-const char *echo_last_error(void);
+ * ("" if none). The string stays valid until the thread's next failing call.
+ * echo_last_status - that call's ECHO_ERR_* code (ECHO_OK if none); the way
+ * to tell why echo_create returned NULL. */
+ECHO_API const char *echo_last_error(void);
+ECHO_API int echo_last_status(void);
 
 /*
  * echo_set_params - compensator settings for later calls: beta_fast and
  * beta_slow in [0, 1), lambda in [0, 1], enable 0 (no correction, state
  * neither read nor written) or 1. Out-of-range values: ECHO_ERR_INVALID.
  */
-int echo_set_params(echo_handle *h, float beta_fast, float beta_slow, float lambda,
+ECHO_API int echo_set_params(echo_handle *h, float beta_fast, float beta_slow, float lambda,
                     int enable);
 
 /* echo_get_state / echo_set_state - synchronous copies of a phase's two
  * estimates (n binary32 each) to / from host memory. A checkpoint is the pair
  * for both phases. */
-int echo_get_state(echo_handle *h, int phase, float *f_host, float *s_host);
-int echo_set_state(echo_handle *h, int phase, const float *f_host, const float *s_host);
+ECHO_API int echo_get_state(echo_handle *h, int phase, float *f_host, float *s_host);
+ECHO_API int echo_set_state(echo_handle *h, int phase, const float *f_host, const float *s_host);
 
 /* Range variants: elements [offset, offset+count). */
-int echo_get_state_range(echo_handle *h, int phase, size_t offset, size_t count,
+ECHO_API int echo_get_state_range(echo_handle *h, int phase, size_t offset, size_t count,
                          float *f_host, float *s_host);
 
 /*
@@ -150,12 +157,12 @@ int echo_get_state_range(echo_handle *h, int phase, size_t offset, size_t count,
  *   stage 2: the requantised total (rank ignored).
  * Either output pointer may be NULL to skip it.
  */
-int echo_get_wire(echo_handle *h, int stage, int rank, uint8_t *codes_host,
+ECHO_API int echo_get_wire(echo_handle *h, int stage, int rank, uint8_t *codes_host,
                   uint8_t *scales_host);
 
 /* Range variant over groups [group_offset, group_offset+ngroups):
  * 16*ngroups code bytes and ngroups scale bytes. */
-int echo_get_wire_range(echo_handle *h, int stage, int rank, size_t group_offset,
+ECHO_API int echo_get_wire_range(echo_handle *h, int stage, int rank, size_t group_offset,
                         size_t ngroups, uint8_t *codes_host, uint8_t *scales_host);
 
 /*
@@ -164,7 +171,7 @@ int echo_get_wire_range(echo_handle *h, int stage, int rank, size_t group_offset
  * bytes (sum of the three kernels' algorithmic bytes), and calls made. Any
  * output pointer may be NULL.
  */
-int echo_stats(echo_handle *h, uint64_t *link_bytes, uint64_t *model_hbm_bytes,
+ECHO_API int echo_stats(echo_handle *h, uint64_t *link_bytes, uint64_t *model_hbm_bytes,
                uint64_t *calls);
 
 /*
@@ -176,15 +183,20 @@ int echo_stats(echo_handle *h, uint64_t *link_bytes, uint64_t *model_hbm_bytes,
  *   out[3]     link bytes of one call, 2(P-1) * n * w.
  * Same argument rules as echo_create.
  */
-int echo_model_bytes(int P, size_t n, int dtype, int enable, uint64_t out[4]);
+ECHO_API int echo_model_bytes(int P, size_t n, int dtype, int enable, uint64_t out[4]);
 
 /*
- * echo_set_timing / echo_last_kernel_ms - when timing is on, each call records
- * CUDA events around each of its three kernels on its stream; ms[0..2] then
- * returns their durations for the last call (waiting for it to finish).
+ * Kernel timing. echo_set_timing(h, 1) starts a measurement: every later
+ * echo_allreduce / echo_allreduce_out call records CUDA events around each of
+ * its three kernels on its own stream (no host wait inside the calls).
+ * echo_last_kernel_ms returns the three durations of the last call (waiting
+ * for it); echo_kernel_ms_total returns their sums over every timed call since
+ * the measurement started, and how many calls that was (waiting for the last).
+ * echo_set_timing(h, 0) stops recording; the totals stay readable.
  */
-int echo_set_timing(echo_handle *h, int enable);
-int echo_last_kernel_ms(echo_handle *h, float ms[3]);
+ECHO_API int echo_set_timing(echo_handle *h, int enable);
+ECHO_API int echo_last_kernel_ms(echo_handle *h, float ms[3]);
+ECHO_API int echo_kernel_ms_total(echo_handle *h, double ms[3], uint64_t *timed_calls);
 
 #ifdef __cplusplus
 }

@@ -1,0 +1,119 @@
+"""The C ABI without a GPU: the library loads, exports every entry point the
+header declares, and rejects bad arguments before touching CUDA."""
+import os
+import re
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "echo.h")
+
+
+@pytest.fixture(scope="module")
+def echo():
+    from bit_error_compensated_rank_b200 import build
+    build.build()
+    from bit_error_compensated_rank_b200 import echo as mod
+    return mod
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"ECHO_API\s+[\w\s\*]*?\b(echo_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_symbols()
+    for required in ("echo_create", "echo_allreduce", "echo_reset", "echo_destroy",
+                     "echo_last_error", "echo_set_params", "echo_get_state", "echo_set_state",
+                     "echo_get_wire", "echo_stats"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(echo):
+    out = subprocess.run(["nm", "-D", "--defined-only", echo.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (echo_\w+)", out))
+    declared = set(declared_symbols())
+    assert declared <= exported, declared - exported
+    assert exported <= declared, exported - declared  # nothing undeclared leaks
+    assert set(echo.EXPORTED) == declared
+
+
+def test_model_bytes_per_element(echo):
+    # P*b + 8 + P*w | P*w + 16 + w | P*w + P*b per element, w = 17/32
+    P, n = 8, 1 << 29
+    mb = echo.echo_model_bytes(P, n, echo.ECHO_BF16, True)
+    w = 17 / 32
+    assert mb["k1"] == round((P * 2 + 8 + P * w) * n)
+    assert mb["k2"] == round((P * w + 16 + w) * n)
+    assert mb["k3"] == round((P * w + P * 2) * n)
+    assert mb["link"] == round(2 * (P - 1) * w * n)
+    assert abs(mb["total"] / n - 69.28125) < 1e-12
+    off = echo.echo_model_bytes(P, n, echo.ECHO_BF16, False)
+    assert mb["total"] - off["total"] == 24 * n
+    f32 = echo.echo_model_bytes(8, 65536, echo.ECHO_FP32, True)
+    assert abs(f32["total"] / 65536 - (2 * 8 * 4 + 25 * w + 24)) < 1e-12
+
+
+@pytest.mark.parametrize("P,n,group,dtype,status", [
+    (1, 64, 32, 0, -1), (17, 17 * 32, 32, 0, -1), (2, 0, 32, 0, -1), (2, 96, 32, 0, -1),
+    (4, 4 * 32 * 3 + 32, 32, 0, -1), (2, 64, 32, 7, -1), (2, 128, 64, 0, -2),
+    (2, 1 << 35, 32, 0, -2), (2, 64, 0, 0, -1),
+])
+def test_create_rejects_bad_shapes(echo, P, n, group, dtype, status):
+    with pytest.raises(echo.EchoError) as ei:
+        echo.echo_create(P, n, group, dtype)
+    assert ei.value.code == status
+    assert echo.echo_last_status() == status
+    assert echo.echo_last_error()
+
+
+def test_null_and_unknown_handles(echo):
+    for fn, args in [(echo._lib.echo_allreduce, (None, None, 0, None)),
+                     (echo._lib.echo_reset, (None, 1)),
+                     (echo._lib.echo_set_params, (None, 0.5, 0.875, 0.5, 1)),
+                     (echo._lib.echo_stats, (None, None, None, None)),
+                     (echo._lib.echo_set_timing, (None, 1))]:
+        assert fn(*args) == echo.ECHO_ERR_INVALID
+        assert "NULL" in echo.echo_last_error()
+    bogus = 0x1000
+    assert echo._lib.echo_reset(bogus, 1) == echo.ECHO_ERR_INVALID
+    assert "unknown or destroyed" in echo.echo_last_error()
+    assert echo._lib.echo_destroy(None) == echo.ECHO_OK
+
+
+def test_injected_allocation_failure():
+    code = (
+        "import os; os.environ['ECHO_FAULT'] = 'alloc'\n"
+        "from bit_error_compensated_rank_b200 import echo as e\n"
+        "try:\n"
+        "    e.echo_create(2, 64)\n"
+        "    raise SystemExit('no error')\n"
+        "except e.EchoError as err:\n"
+        "    assert err.code == e.ECHO_ERR_OOM, err\n"
+        "    assert 'injected' in str(err)\n"
+    )
+    res = subprocess.run([sys.executable, "-c", code], cwd=ROOT, capture_output=True, text=True)
+    assert res.returncode == 0, res.stderr + res.stdout
+
+
+def test_binding_fails_loudly_without_library(tmp_path):
+    """The binding has no fallback: with the library missing, import fails."""
+    code = (
+        "import sys, os, importlib.util\n"
+        "spec = importlib.util.spec_from_file_location('echo_copy', sys.argv[1])\n"
+        "mod = importlib.util.module_from_spec(spec)\n"
+        "try:\n"
+        "    spec.loader.exec_module(mod)\n"
+        "except ImportError as e:\n"
+        "    assert 'no fallback' in str(e)\n"
+        "    sys.exit(0)\n"
+        "sys.exit(1)\n"
+    )
+    copy = tmp_path / "echo.py"
+    copy.write_text(open(os.path.join(ROOT, "bit_error_compensated_rank_b200", "echo.py")).read())
+    res = subprocess.run([sys.executable, "-c", code, str(copy)], capture_output=True, text=True)
+    assert res.returncode == 0, res.stderr

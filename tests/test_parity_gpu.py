@@ -1,0 +1,240 @@
+"""CUDA path against the CPU oracle, bit for bit, on problems small enough to
+compare in full (several warp steps, CTAs and grid-stride rounds, ragged
+tails), through the C ABI."""
+import os
+import subprocess
+import sys
+
+import numpy as np
+import pytest
+
+from bit_error_compensated_rank_b200.workloads import bf16_bits, gaussian, outlier_gaussian, rng
+from gpu_harness import FullCompare, assert_same_bits, from_device, to_device
+from oracle.oracle import Params
+
+pytestmark = pytest.mark.gpu
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+# n = P * 32 * k with k chosen so the chunk count (n/8) is not a multiple of a
+# warp step (32 chunks) or of a CTA step (256 chunks): ragged tails everywhere.
+SHAPES = [(2, 2 * 32 * 37), (3, 3 * 32 * 41), (4, 4 * 32 * 64), (5, 5 * 32 * 29),
+          (8, 8 * 32 * 3001), (16, 16 * 32 * 101), (7, 7 * 32)]
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+@pytest.mark.parametrize("P,n", SHAPES)
+def test_sequence_both_phases(oracle, P, n, dtype):
+    fc = FullCompare(oracle, P, n, dtype)
+    try:
+        phases = [0, 0, 0, 1, 1, 0]
+        for k, ph in enumerate(phases):
+            x = outlier_gaussian(P, n, seed=P, call=k, dtype=dtype) if k % 2 else \
+                gaussian(P, n, seed=P, call=k, dtype=dtype)
+            fc.call(x, phase=ph)
+    finally:
+        fc.close()
+
+
+@pytest.mark.parametrize("params", [
+    Params(lam=0.25, beta_fast=0.3, beta_slow=0.95),
+    Params(lam=1.0, beta_fast=0.0, beta_slow=0.875),
+    Params(lam=0.5, beta_fast=0.5, beta_slow=0.875, enable=False),
+], ids=["asymmetric", "error_feedback", "off"])
+def test_parameters(oracle, params):
+    P, n = 4, 4 * 32 * 257
+    fc = FullCompare(oracle, P, n, "bf16", params)
+    try:
+        for k in range(5):
+            fc.call(gaussian(P, n, seed=21, call=k), phase=0)
+    finally:
+        fc.close()
+
+
+def test_out_of_place(oracle):
+    P, n = 8, 8 * 32 * 77
+    for dtype in ("bf16", "fp32"):
+        fc = FullCompare(oracle, P, n, dtype)
+        try:
+            for k in range(3):
+                fc.call(gaussian(P, n, seed=3, call=k, dtype=dtype), out_of_place=True)
+        finally:
+            fc.close()
+
+
+def _edge_inputs(P, n, kind):
+    g = rng(17, P, len(kind))
+    if kind == "zeros":
+        return np.zeros((P, n), np.float32)
+    if kind == "subnormal":
+        return (g.integers(-2 ** 20, 2 ** 20, (P, n)) * 2.0 ** -149).astype(np.float32)
+    if kind == "huge":
+        return (g.standard_normal((P, n)) * 2.0 ** 100).astype(np.float32)
+    if kind == "tiny_normal":
+        return (g.standard_normal((P, n)) * 2.0 ** -120).astype(np.float32)
+    if kind == "identical":
+        return np.repeat(g.standard_normal((1, n)).astype(np.float32), P, axis=0)
+    if kind == "cancel":
+        x = g.standard_normal((P, n)).astype(np.float32)
+        x[1::2] = -x[0::2][: x[1::2].shape[0]]
+        return x
+    if kind == "ties":
+        k = g.integers(-7, 7, (P, n)) + 0.5
+        k[:, ::32] = 7
+        return (k * 2.0 ** g.integers(-20, 20, (P, 1))).astype(np.float32)
+    if kind == "one_outlier":
+        x = g.standard_normal((P, n)).astype(np.float32)
+        x[:, 5::32] *= 1000
+        return x
+    raise ValueError(kind)
+
+
+@pytest.mark.parametrize("kind", ["zeros", "subnormal", "huge", "tiny_normal", "identical",
+                                  "cancel", "ties", "one_outlier"])
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+def test_edge_values(oracle, kind, dtype):
+    P, n = 4, 4 * 32 * 45
+    fc = FullCompare(oracle, P, n, dtype)
+    try:
+        for k in range(3):
+            x = _edge_inputs(P, n, kind)
+            if k:
+                x = x * np.float32(1 + k / 8)
+            fc.call(bf16_bits(x) if dtype == "bf16" else x)
+    finally:
+        fc.close()
+
+
+@pytest.mark.parametrize("P", list(range(2, 17)))
+def test_smallest_tensor(oracle, P):
+    n = P * 32  # one group per owner
+    fc = FullCompare(oracle, P, n, "bf16")
+    try:
+        for k in range(3):
+            fc.call(gaussian(P, n, seed=P, call=k))
+    finally:
+        fc.close()
+
+
+def test_state_set_get_reset(oracle):
+    from bit_error_compensated_rank_b200 import echo
+    P, n = 4, 4 * 32 * 33
+    fc = FullCompare(oracle, P, n, "bf16")
+    try:
+        g = rng(5, 5)
+        for ph in (0, 1):
+            f = (g.standard_normal(n) * 0.05).astype(np.float32)
+            s = (g.standard_normal(n) * 0.05).astype(np.float32)
+            fc.h.set_state(ph, f, s)
+            gf, gs = fc.h.get_state(ph)
+            assert_same_bits(gf, f, "set/get f")
+            assert_same_bits(gs, s, "set/get s")
+            fc.state[ph] = (f.copy(), s.copy())
+        for k in range(3):
+            fc.call(gaussian(P, n, seed=6, call=k), phase=k % 2)
+        fc.h.reset(1)
+        gf, gs = fc.h.get_state(0)
+        assert not gf.any() and not gs.any()
+        gf1, _ = fc.h.get_state(1)
+        assert_same_bits(gf1, fc.state[1][0], "bwd state kept by a fwd reset")
+        fc.state[0] = (np.zeros(n, np.float32), np.zeros(n, np.float32))
+        fc.call(gaussian(P, n, seed=6, call=9), phase=0)
+        st = fc.h.stats()
+        mb = echo.echo_model_bytes(P, n, echo.ECHO_BF16, True)
+        assert st["calls"] == 4
+        assert st["link_bytes"] == 4 * mb["link"]
+        assert st["model_hbm_bytes"] == 4 * mb["total"]
+    finally:
+        fc.close()
+
+
+def test_timing_events():
+    import torch
+    from bit_error_compensated_rank_b200 import echo
+    P, n = 8, 8 * 32 * 4096
+    h = echo.Echo(P, n)
+    try:
+        x = [torch.randn(n, device="cuda").to(torch.bfloat16) for _ in range(P)]
+        h.set_timing(True)
+        h.allreduce(x)
+        ms = h.last_kernel_ms()
+        assert len(ms) == 3 and all(m > 0 for m in ms)
+        h.set_timing(False)
+        h.allreduce(x)
+        with pytest.raises(echo.EchoError):
+            h.last_kernel_ms()
+    finally:
+        h.close()
+
+
+def test_rejects_bad_buffers_without_launching():
+    import torch
+    from bit_error_compensated_rank_b200 import echo
+    P, n = 4, 4 * 32 * 16
+    h = echo.Echo(P, n)
+    try:
+        x = [torch.zeros(n, device="cuda", dtype=torch.bfloat16) for _ in range(P)]
+        h.allreduce(x)
+        big = torch.zeros(P * n + 8, device="cuda", dtype=torch.bfloat16)
+        cases = {
+            "misaligned": [x[0].data_ptr() + 2] + [t.data_ptr() for t in x[1:]],
+            "overlap": [big.data_ptr() + r * (n - 8) * 2 for r in range(P)],
+            "duplicate": [x[0].data_ptr()] * P,
+            "host": [np.zeros(n, np.uint16).ctypes.data // 16 * 16 + 16] + [t.data_ptr() for t in x[1:]],
+            "null": [0] + [t.data_ptr() for t in x[1:]],
+        }
+        for name, ptrs in cases.items():
+            with pytest.raises(echo.EchoError) as ei:
+                echo.echo_allreduce(h.h, ptrs, 0, 0)
+            assert ei.value.code == echo.ECHO_ERR_INVALID, name
+        with pytest.raises(echo.EchoError):
+            echo.echo_allreduce(h.h, [t.data_ptr() for t in x], 2, 0)
+        with pytest.raises(echo.EchoError):
+            h.set_params(1.0, 0.5, 0.5, True)
+        assert h.stats()["calls"] == 1
+        torch.cuda.synchronize()
+    finally:
+        h.close()
+
+
+def test_injected_launch_failure():
+    code = (
+        "import os; os.environ['ECHO_FAULT'] = 'launch'\n"
+        "import torch\n"
+        "from bit_error_compensated_rank_b200 import echo as e\n"
+        "h = e.Echo(2, 64)\n"
+        "x = [torch.zeros(64, device='cuda', dtype=torch.bfloat16) for _ in range(2)]\n"
+        "try:\n"
+        "    h.allreduce(x)\n"
+        "    raise SystemExit('no error')\n"
+        "except e.EchoError as err:\n"
+        "    assert err.code == e.ECHO_ERR_CUDA and 'injected' in str(err), err\n"
+        "assert h.stats()['calls'] == 0\n"
+        "h.close()\n"
+    )
+    res = subprocess.run([sys.executable, "-c", code], cwd=ROOT, capture_output=True, text=True)
+    assert res.returncode == 0, res.stderr + res.stdout
+
+
+def test_host_end_to_end(oracle):
+    """Host buffers in, host result out (pipelined pieces of 2^22 elements)."""
+    import torch
+    from bit_error_compensated_rank_b200 import echo
+    P, n = 4, 4 * 32 * 80000  # 10.24 M elements per rank: three pieces
+    h = echo.Echo(P, n)
+    try:
+        f = np.zeros(n, np.float32)
+        s = np.zeros(n, np.float32)
+        for k in range(2):
+            x = gaussian(P, n, seed=8, call=k)
+            host_in = [torch.from_numpy(x[r].view(np.int16)).view(torch.bfloat16).pin_memory()
+                       for r in range(P)]
+            host_out = torch.empty(n, dtype=torch.bfloat16).pin_memory()
+            h.allreduce_host(host_in, host_out)
+            ref = oracle.allreduce(x, f, s, Params())
+            assert_same_bits(host_out.view(torch.int16).numpy().view(np.uint16), ref["out"], "host result")
+            gf, gs = h.get_state(0)
+            assert_same_bits(gf, f, "fast estimate")
+            assert_same_bits(gs, s, "slow estimate")
+    finally:
+        h.close()
