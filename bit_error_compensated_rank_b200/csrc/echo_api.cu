@@ -44,10 +44,12 @@ int cuda_error(cudaError_t e, const char *what)
     return set_error(ECHO_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorString(e), cudaGetErrorName(e));
 }
 
-// Host-side fault injection for tests: ECHO_FAULT=alloc makes echo_create
-// fail as if the device were out of memory; ECHO_FAULT=launch makes the
-// all-reduce entry points fail as if the launch had failed. Nothing reaches
-// the GPU in either case.
+// Fault injection for tests: ECHO_FAULT=alloc makes echo_create fail as if
+// the device were out of memory and ECHO_FAULT=launch makes the all-reduce
+// entry points fail as if the launch had failed (nothing reaches the GPU);
+// ECHO_FAULT=stall launches the kernels with no loads issued and a short
+// wait bound, so every CTA's first wait runs out and the kernels record a
+// timeout in the device status word and return.
 bool fault_injected(const char *what)
 {
     const char *e = std::getenv("ECHO_FAULT");
@@ -58,6 +60,10 @@ std::mutex g_mu;
 std::set<const echo_handle *> g_live; // handles created and not destroyed
 
 constexpr size_t kMaxN = size_t(1) << 34;  // chunk indices stay 32-bit
+// Bound of every kernel wait: about a second at B200 clocks (a tile normally
+// lands in microseconds); the injected stall uses about half a millisecond.
+constexpr long long kWaitCycles = 1LL << 31;
+constexpr long long kStallWaitCycles = 1LL << 20;
 constexpr size_t kHostPiece = size_t(1) << 22; // elements per pipelined host transfer
 constexpr int kTimingRing = 32;                 // event sets of timed calls in flight
 
@@ -100,9 +106,11 @@ struct echo_handle {
     int dtype = ECHO_BF16;
     int device = 0;
     uint8_t *codes1 = nullptr;  // [P][n/2]
-    uint8_t *scales1 = nullptr; // [P][n/32]
+    uint8_t *scales1 = nullptr; // [P][scale_stride]
     uint8_t *qcodes = nullptr;  // [n/2]
-    uint8_t *qscales = nullptr; // [n/32]
+    uint8_t *qscales = nullptr; // [scale_stride]
+    size_t scale_stride = 0;    // n/32 rounded up to 16 bytes (bulk-copy alignment)
+    int *dstatus = nullptr;     // device status word written by timed-out waits
     float *state = nullptr;     // [phase][f|s][n]
     float beta_f = 0.5f, beta_s = 0.875f, lambda = 0.5f;
     bool enable = true;
@@ -232,6 +240,10 @@ int fold_timings(echo_handle *h, uint64_t upto)
 int enqueue_call(echo_handle *h, const void *const send[], void *const recv[], int phase, cudaStream_t st,
                  uint32_t cb, uint32_t ce, bool record_events)
 {
+    // Tiles start at multiples of 512 elements from the range start, so every
+    // bulk copy (partials, codes, 16-byte scale rows, state) is 16-byte aligned.
+    if (cb % 64 != 0 || ce < cb)
+        return set_error(ECHO_ERR_INVALID, "internal: element range must start at a multiple of 512");
     cudaEvent_t *ev = nullptr;
     if (record_events) {
         if (h->ring_calls >= static_cast<uint64_t>(kTimingRing)) {
@@ -292,21 +304,36 @@ int enqueue_call(echo_handle *h, const void *const send[], void *const recv[], i
     a3.P = h->P;
     a3.bf16 = h->dtype == ECHO_BF16;
 
-    cudaError_t e;
-    if (ev && (e = cudaEventRecord(ev[0], st)) != cudaSuccess)
-        return cuda_error(e, "cudaEventRecord");
-    if ((e = echo::launch_k1_compensate_quantize_pack(a1, st, 0)) != cudaSuccess)
-        return cuda_error(e, "launch k1_compensate_quantize_pack");
-    if (ev && (e = cudaEventRecord(ev[1], st)) != cudaSuccess)
-        return cuda_error(e, "cudaEventRecord");
-    if ((e = echo::launch_k2_owner_reduce_requant(a2, st, 0)) != cudaSuccess)
-        return cuda_error(e, "launch k2_owner_reduce_requant");
-    if (ev && (e = cudaEventRecord(ev[2], st)) != cudaSuccess)
-        return cuda_error(e, "cudaEventRecord");
-    if ((e = echo::launch_k3_gather_dequant(a3, st, 0)) != cudaSuccess)
-        return cuda_error(e, "launch k3_gather_dequant");
-    if (ev && (e = cudaEventRecord(ev[3], st)) != cudaSuccess)
-        return cuda_error(e, "cudaEventRecord");
+    // Every wait in the kernels is bounded; ECHO_FAULT=stall (tests) issues no
+    // loads at all and shortens the bound, so each wait runs out quickly.
+    const bool stall = fault_injected("stall");
+    const echo::PipeCtl ctl{h->dstatus, stall ? kStallWaitCycles : kWaitCycles, stall};
+    a1.ctl = a2.ctl = a3.ctl = ctl;
+    a1.scale_stride = a2.scale_stride = h->scale_stride;
+
+    cudaError_t e = cudaSuccess;
+    const char *what = "cudaEventRecord";
+    if (ev)
+        e = cudaEventRecord(ev[0], st);
+    if (e == cudaSuccess && (e = echo::launch_k1_compensate_quantize_pack(a1, st)) != cudaSuccess)
+        what = "launch k1_compensate_quantize_pack";
+    if (e == cudaSuccess && ev)
+        e = cudaEventRecord(ev[1], st);
+    if (e == cudaSuccess && (e = echo::launch_k2_owner_reduce_requant(a2, st)) != cudaSuccess)
+        what = "launch k2_owner_reduce_requant";
+    if (e == cudaSuccess && ev)
+        e = cudaEventRecord(ev[2], st);
+    if (e == cudaSuccess && (e = echo::launch_k3_gather_dequant(a3, st)) != cudaSuccess)
+        what = "launch k3_gather_dequant";
+    if (e == cudaSuccess && ev)
+        e = cudaEventRecord(ev[3], st);
+    if (e != cudaSuccess) {
+        if (ev) { // the slot was not fully recorded: give it back
+            h->ring_calls -= 1;
+            h->last_slot = -1;
+        }
+        return cuda_error(e, what);
+    }
     return ECHO_OK;
 }
 
@@ -342,6 +369,7 @@ void free_handle(echo_handle *h)
     cudaFree(h->qcodes);
     cudaFree(h->qscales);
     cudaFree(h->state);
+    cudaFree(h->dstatus);
     cudaFree(h->staging);
     for (auto &slot : h->ring)
         for (cudaEvent_t e : slot)
@@ -360,7 +388,7 @@ void free_handle(echo_handle *h)
 
 namespace echo {
 
-int grid_for(uint32_t warp_tiles, int resident_per_sm, int max_ctas)
+int persistent_grid(uint32_t tiles, int resident_per_sm)
 {
     static int sms = 0;
     if (sms == 0) {
@@ -371,12 +399,22 @@ int grid_for(uint32_t warp_tiles, int resident_per_sm, int max_ctas)
         else
             sms = 148;
     }
-    const long full = static_cast<long>(sms) * resident_per_sm;
-    const long need = (static_cast<long>(warp_tiles) + 7) / 8; // 8 warps per CTA
-    long g = need < full ? need : full;
-    if (max_ctas > 0 && g > max_ctas)
-        g = max_ctas;
+    const long full = static_cast<long>(sms) * (resident_per_sm > 0 ? resident_per_sm : 1);
+    const long g = static_cast<long>(tiles) < full ? static_cast<long>(tiles) : full;
     return g < 1 ? 1 : static_cast<int>(g);
+}
+
+cudaError_t prepare_kernel(const void *kernel, int threads, int smem_bytes, int *resident)
+{
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
+    if (e != cudaSuccess)
+        return e;
+    int r = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&r, kernel, threads, smem_bytes);
+    if (e != cudaSuccess)
+        return e;
+    *resident = r > 0 ? r : 1;
+    return cudaSuccess;
 }
 
 } // namespace echo
@@ -414,6 +452,7 @@ echo_handle *echo_create(int P, size_t n, int group, int dtype)
     h->P = P;
     h->n = n;
     h->dtype = dtype;
+    h->scale_stride = (n / ECHO_GROUP + 15) / 16 * 16;
     cudaError_t e = cudaGetDevice(&h->device);
     if (e != cudaSuccess) {
         cuda_error(e, "cudaGetDevice");
@@ -425,10 +464,11 @@ echo_handle *echo_create(int P, size_t n, int group, int dtype)
         size_t bytes;
     } allocs[] = {
         {reinterpret_cast<void **>(&h->codes1), static_cast<size_t>(P) * (n / 2)},
-        {reinterpret_cast<void **>(&h->scales1), static_cast<size_t>(P) * (n / ECHO_GROUP)},
+        {reinterpret_cast<void **>(&h->scales1), static_cast<size_t>(P) * h->scale_stride},
         {reinterpret_cast<void **>(&h->qcodes), n / 2},
-        {reinterpret_cast<void **>(&h->qscales), n / ECHO_GROUP},
+        {reinterpret_cast<void **>(&h->qscales), h->scale_stride},
         {reinterpret_cast<void **>(&h->state), 4 * n * sizeof(float)},
+        {reinterpret_cast<void **>(&h->dstatus), sizeof(int)},
     };
     for (auto &a : allocs) {
         e = cudaMalloc(a.p, a.bytes);
@@ -443,6 +483,8 @@ echo_handle *echo_create(int P, size_t n, int group, int dtype)
         }
     }
     e = cudaMemset(h->state, 0, 4 * n * sizeof(float));
+    if (e == cudaSuccess)
+        e = cudaMemset(h->dstatus, 0, sizeof(int));
     if (e == cudaSuccess)
         e = cudaDeviceSynchronize();
     if (e != cudaSuccess) {
@@ -646,7 +688,7 @@ int echo_get_wire_range(echo_handle *h, int stage, int rank, size_t group_offset
     if (group_offset > groups || ngroups > groups - group_offset)
         return set_error(ECHO_ERR_INVALID, "group range exceeds %zu groups", groups);
     const uint8_t *codes = stage == 1 ? h->codes1 + static_cast<size_t>(rank) * (h->n / 2) : h->qcodes;
-    const uint8_t *scales = stage == 1 ? h->scales1 + static_cast<size_t>(rank) * groups : h->qscales;
+    const uint8_t *scales = stage == 1 ? h->scales1 + static_cast<size_t>(rank) * h->scale_stride : h->qscales;
     cudaError_t e = cudaDeviceSynchronize();
     if (e == cudaSuccess && codes_host)
         e = cudaMemcpy(codes_host, codes + group_offset * (ECHO_GROUP / 2), ngroups * (ECHO_GROUP / 2),
@@ -718,6 +760,23 @@ int echo_last_kernel_ms(echo_handle *h, float ms[3])
     for (int k = 0; k < 3 && e == cudaSuccess; k++)
         e = cudaEventElapsedTime(&ms[k], ev[k], ev[k + 1]);
     return e == cudaSuccess ? ECHO_OK : cuda_error(e, "echo_last_kernel_ms");
+}
+
+int echo_device_status(echo_handle *h, int *status, int clear)
+{
+    int rc;
+    if ((rc = check_handle(h)) != ECHO_OK || (rc = check_device(h)) != ECHO_OK)
+        return rc;
+    if (!status)
+        return set_error(ECHO_ERR_INVALID, "status is NULL");
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e == cudaSuccess)
+        e = cudaMemcpy(status, h->dstatus, sizeof(int), cudaMemcpyDeviceToHost);
+    if (e == cudaSuccess && clear)
+        e = cudaMemset(h->dstatus, 0, sizeof(int));
+    if (e == cudaSuccess && clear)
+        e = cudaDeviceSynchronize();
+    return e == cudaSuccess ? ECHO_OK : cuda_error(e, "echo_device_status");
 }
 
 int echo_kernel_ms_total(echo_handle *h, double ms[3], uint64_t *timed_calls)

@@ -1,0 +1,129 @@
+// echo_bulk.cuh - bulk-copy (TMA engine) pipeline helpers for sm_100a.
+//
+// The three kernels stream tiles between HBM and shared memory with the
+// untiled bulk copy (cp.async.bulk): one elected thread issues whole-tile
+// copies, completion is tracked by an mbarrier's transaction count, and the
+// rest of the CTA computes from shared memory. No copy uses cluster
+// multicast, and every copy reads or writes only this GPU's memory.
+//
+// Every wait is bounded in time: a CTA that does not see its tile arrive
+// within the limit records the failure in the device status word and leaves
+// its loop (see wait_tile), so a fault in the pipeline can never hang the GPU.
+#pragma once
+
+#include <cstdint>
+
+namespace echo {
+
+// Device status word bits (the host reads them with echo_device_status).
+constexpr int kStatusTimeoutK1 = 1;
+constexpr int kStatusTimeoutK2 = 2;
+constexpr int kStatusTimeoutK3 = 4;
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p)
+{
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+// Make barrier initialisation visible to the async proxy before first use.
+__device__ __forceinline__ void mbar_init_fence()
+{
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
+{
+    uint32_t done;
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(done)
+                 : "r"(smem_u32(bar)), "r"(parity)
+                 : "memory");
+    return done != 0;
+}
+
+// Poll the barrier's phase with parity `parity` for at most `limit` SM
+// clock cycles (a real-time bound, whatever try_wait's own suspend window is).
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity, long long limit)
+{
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity))
+        if (clock64() - t0 > limit)
+            return false;
+    return true;
+}
+
+// Global -> shared bulk copy of `bytes` (multiple of 16, both addresses
+// 16-byte aligned), completing `bytes` transactions on `bar`.
+__device__ __forceinline__ void bulk_load(void *smem_dst, const void *gmem_src, uint32_t bytes, uint64_t *bar)
+{
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_u32(smem_dst)),
+                 "l"(gmem_src), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
+
+// Shared -> global bulk copy, tracked by the issuing thread's bulk groups.
+__device__ __forceinline__ void bulk_store(void *gmem_dst, const void *smem_src, uint32_t bytes)
+{
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gmem_dst),
+                 "r"(smem_u32(smem_src)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+
+// Wait until at most N committed store groups still read shared memory.
+template <int N>
+__device__ __forceinline__ void bulk_wait_read()
+{
+    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+
+// Wait until every committed store group has completed.
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// Order this thread's generic-proxy writes to shared memory before later
+// async-proxy (bulk copy) reads of it.
+__device__ __forceinline__ void fence_proxy_async_smem()
+{
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Every thread waits (bounded) for the tile in `bar`'s current phase; the
+// outcome is made CTA-uniform with a barrier, so either all threads go on or
+// all leave together. On a timeout, thread 0 records `status_bit`.
+__device__ __forceinline__ bool wait_tile(uint64_t *bar, uint32_t parity, long long limit, int *status,
+                                          int status_bit)
+{
+    const bool ok = mbar_wait_bounded(bar, parity, limit);
+    const bool all = __syncthreads_and(ok) != 0;
+    if (!all && threadIdx.x == 0)
+        atomicOr(status, status_bit);
+    return all;
+}
+
+// After a timeout: give the loads still in flight (local tiles [from, to) of
+// an S-stage ring) a bounded chance to land before the CTA's shared memory is
+// released.
+__device__ __forceinline__ void drain_loads(uint64_t *full, int S, uint32_t from, uint32_t to, long long limit)
+{
+    if (threadIdx.x == 0)
+        for (uint32_t t = from; t < to; t++)
+            mbar_wait_bounded(&full[t % S], (t / S) & 1u, limit);
+    __syncthreads();
+}
+
+} // namespace echo

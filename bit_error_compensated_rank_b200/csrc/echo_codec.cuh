@@ -53,29 +53,63 @@ __device__ __forceinline__ float inv_step_of(uint32_t byte)
     return __uint_as_float((254u - byte) << 23);
 }
 
-// Nearest code of v at scale 1/inv (v*inv is exact whenever it is normal; a
-// subnormal product is below 1/2 and rounds to 0 either way).
-__device__ __forceinline__ int code_of(float v, float inv)
+// ---- rounding to a code ---------------------------------------------------
+// kRound = 1.5 * 2^23. For |t| <= 7, RN(t + kRound) lands in [2^23, 2^24),
+// where the spacing of binary32 is exactly 1, so the addition rounds t to the
+// nearest integer k, halves to the even one (kRound is even, so the last
+// significand bit is the parity of k), and the bit pattern of the result is
+// 0x4B400000 + k: its low byte is k as a two's-complement int8.
+// fma(v, inv, kRound) computes RN(v*inv + kRound) from the exact product
+// v*inv (inv is a power of two and |v*inv| <= 7 by the scale rule), so it is
+// round-half-even(v / 2^e) with no intermediate rounding, subnormals included.
+constexpr float kRound = 12582912.0f;      // 1.5 * 2^23, bits 0x4B400000
+constexpr uint32_t kRoundBits = 0x4B400000u;
+constexpr float kRoundPlus8 = 12582920.0f; // kRound + 8
+
+// Bit pattern kRoundBits + q of the nearest code q of v at step 1/inv.
+__device__ __forceinline__ uint32_t code_bits(float v, float inv)
 {
-    int q = __float2int_rn(__fmul_rn(v, inv));
-    q = q > 7 ? 7 : q;
-    return q < -7 ? -7 : q;
+    return __float_as_uint(__fmaf_rn(v, inv, kRound));
 }
 
-// Pack 8 codes (element k in nibble k) into one word.
-__device__ __forceinline__ uint32_t pack8(const int (&q)[kChunk])
+// Code q (as a float) from its rounded bit pattern (exact subtraction).
+__device__ __forceinline__ float code_value(uint32_t bits)
 {
-    uint32_t w = 0;
-#pragma unroll
-    for (int k = 0; k < kChunk; k++)
-        w |= (static_cast<uint32_t>(q[k]) & 0xFu) << (4 * k);
-    return w;
+    return __fsub_rn(__uint_as_float(bits), kRound);
 }
 
-// Signed code in nibble k of w.
-__device__ __forceinline__ int nibble(uint32_t w, int k)
+// Pack the codes of 8 rounded bit patterns (element k = low byte of b[k])
+// into one word, element 2j in the low nibble of byte j and 2j+1 in its high
+// nibble. prmt gathers the low bytes of the even and the odd elements; one
+// shift and one masked merge interleave them.
+__device__ __forceinline__ uint32_t pack8_bits(const uint32_t (&b)[kChunk])
 {
-    return static_cast<int>(w << (28 - 4 * k)) >> 28;
+    const uint32_t even = __byte_perm(__byte_perm(b[0], b[2], 0x0040), __byte_perm(b[4], b[6], 0x0040), 0x5410);
+    const uint32_t odd = __byte_perm(__byte_perm(b[1], b[3], 0x0040), __byte_perm(b[5], b[7], 0x0040), 0x5410);
+    return (even & 0x0F0F0F0Fu) | ((odd << 4) & 0xF0F0F0F0u);
+}
+
+// ---- restoring codes --------------------------------------------------------
+// A packed word holds 8 two's-complement nibbles. Flipping bit 3 of each
+// nibble turns q in [-8, 7] into q + 8 in [0, 15]; placing that byte in the
+// low byte of kRoundBits gives the binary32 kRound + q + 8, so subtracting
+// kRound + 8 yields q exactly.
+struct Unpacked {
+    uint32_t even; // bytes j: q_{2j} + 8
+    uint32_t odd;  // bytes j: q_{2j+1} + 8
+};
+
+__device__ __forceinline__ Unpacked unpack8(uint32_t w)
+{
+    return Unpacked{(w & 0x0F0F0F0Fu) ^ 0x08080808u, ((w >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u};
+}
+
+// Code of element k (0..7) as a float; k is a constant after unrolling.
+__device__ __forceinline__ float code_at(const Unpacked &u, int k)
+{
+    const uint32_t src = (k & 1) ? u.odd : u.even;
+    const uint32_t bits = __byte_perm(src, kRoundBits, 0x7650 + (k >> 1));
+    return __fsub_rn(__uint_as_float(bits), kRoundPlus8);
 }
 
 // Absolute maximum over the 4 lanes (32 elements) of a group. The lanes of a
@@ -98,13 +132,14 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4 &raw, float (&v)[kChun
     }
 }
 
-// Values q*2^e with |q| <= 7 have zero low halves, so truncation is exact.
+// Values q*2^e with |q| <= 7 have zero low halves, so keeping the upper
+// halves (one prmt per pair) is exact.
 __device__ __forceinline__ uint4 f32x8_to_bf16_exact(const float (&y)[kChunk])
 {
     uint32_t w[4];
 #pragma unroll
     for (int j = 0; j < 4; j++)
-        w[j] = (__float_as_uint(y[2 * j]) >> 16) | (__float_as_uint(y[2 * j + 1]) & 0xFFFF0000u);
+        w[j] = __byte_perm(__float_as_uint(y[2 * j]), __float_as_uint(y[2 * j + 1]), 0x7632);
     return make_uint4(w[0], w[1], w[2], w[3]);
 }
 

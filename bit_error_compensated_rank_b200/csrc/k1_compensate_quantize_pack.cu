@@ -8,14 +8,19 @@
 //
 // Layout: the rank partials are P separate buffers of n elements; the output
 // is the stage-1 wire, codes [P][n/2] (two per byte) and scale bytes
-// [P][n/32]. A lane owns 8 consecutive elements (one 128-bit bf16 load, one
-// 32-bit code word); 4 lanes form a group and find its maximum with two
-// shuffles. One warp step covers 256 elements of every rank, so per step a
-// warp issues P x 512 B of coalesced partial loads, 1 KB of state loads
-// (compensation on) and P x 128 B of code stores.
+// [P][scale_stride].
+//
+// Pipeline: a persistent CTA takes tiles of kTile consecutive elements. For
+// each tile, thread 0 bulk-copies the P partial tiles and the f, s tiles into
+// one stage of a kStages ring in shared memory (one mbarrier per stage counts
+// the bytes); the CTA computes from shared memory while the next stages are
+// in flight. A lane owns 8 consecutive elements of one rank; 4 lanes form a
+// group and find its maximum with two shuffles; codes leave as one coalesced
+// 32-bit store per lane.
 //
 // Algorithmic HBM bytes per element of n: P*b (partials) + 8 (f, s; each
 // element is corrected by exactly one rank) read, P*17/32 written.
+#include "echo_bulk.cuh"
 #include "echo_kernels.h"
 
 #include <cuda_runtime.h>
@@ -25,180 +30,182 @@ namespace {
 
 constexpr int kThreads = 256;
 
-template <bool BF16>
-struct Raw;
-template <>
-struct Raw<true> {
-    uint4 a;
-};
-template <>
-struct Raw<false> {
-    uint4 a, b;
+template <int P, bool BF16, bool COMP>
+struct K1Shape {
+    static constexpr int kEB = BF16 ? 2 : 4;
+    // Tile length keeps one stage near 12-24 KB whatever P and the dtype.
+    static constexpr int kTile = (P * kEB <= 16) ? 1024 : (P * kEB <= 32 ? 512 : 256);
+    static constexpr int kStages = 3;
+    static constexpr int kXBytes = kTile * kEB; // one rank's partial tile
+    static constexpr int kStageBytes = P * kXBytes + (COMP ? 2 * kTile * 4 : 0);
+    static constexpr int kSmem = kStages * kStageBytes + kStages * 8;
+    static constexpr int kChunksPerTile = kTile / kChunk; // a multiple of 32
 };
 
-// Partials are read once: stream them past L1 with an evict-first hint.
 template <bool BF16>
-__device__ __forceinline__ Raw<BF16> load_raw(const void *base, uint32_t chunk);
-template <>
-__device__ __forceinline__ Raw<true> load_raw<true>(const void *base, uint32_t chunk)
+__device__ __forceinline__ void load_chunk(const uint8_t *p, float (&v)[kChunk])
 {
-    return Raw<true>{__ldcs(reinterpret_cast<const uint4 *>(base) + chunk)};
-}
-template <>
-__device__ __forceinline__ Raw<false> load_raw<false>(const void *base, uint32_t chunk)
-{
-    const uint4 *p = reinterpret_cast<const uint4 *>(base) + 2 * static_cast<size_t>(chunk);
-    return Raw<false>{__ldcs(p), __ldcs(p + 1)};
-}
-
-__device__ __forceinline__ void to_f32(const Raw<true> &r, float (&v)[kChunk])
-{
-    bf16x8_to_f32(r.a, v);
-}
-__device__ __forceinline__ void to_f32(const Raw<false> &r, float (&v)[kChunk])
-{
-    v[0] = __uint_as_float(r.a.x);
-    v[1] = __uint_as_float(r.a.y);
-    v[2] = __uint_as_float(r.a.z);
-    v[3] = __uint_as_float(r.a.w);
-    v[4] = __uint_as_float(r.b.x);
-    v[5] = __uint_as_float(r.b.y);
-    v[6] = __uint_as_float(r.b.z);
-    v[7] = __uint_as_float(r.b.w);
+    if (BF16) {
+        bf16x8_to_f32(*reinterpret_cast<const uint4 *>(p), v);
+    } else {
+        const float4 a = reinterpret_cast<const float4 *>(p)[0];
+        const float4 b = reinterpret_cast<const float4 *>(p)[1];
+        v[0] = a.x, v[1] = a.y, v[2] = a.z, v[3] = a.w;
+        v[4] = b.x, v[5] = b.y, v[6] = b.z, v[7] = b.w;
+    }
 }
 
 template <int P, bool BF16, bool COMP>
 __global__ void __launch_bounds__(kThreads)
     k1_compensate_quantize_pack(const K1Args a)
 {
-    // Ranks whose partials are loaded together before any is processed: all
-    // of them for bf16 (4 registers each), eight at a time for binary32.
-    constexpr int kBatch = BF16 ? P : (P < 8 ? P : 8);
-    const uint32_t lane = threadIdx.x & 31u;
-    const uint32_t warp = (blockIdx.x * kThreads + threadIdx.x) >> 5;
-    const uint32_t nwarps = (gridDim.x * kThreads) >> 5;
-    const uint32_t ntiles = (a.chunk_end - a.chunk_begin + 31u) >> 5;
-    const size_t code_words = a.n / kChunk;   // 32-bit code words per rank
-    const size_t scale_bytes = a.n / kGroup;  // scale bytes per rank
+    using Sh = K1Shape<P, BF16, COMP>;
+    constexpr int S = Sh::kStages;
+    extern __shared__ __align__(128) uint8_t smem[];
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + S * Sh::kStageBytes);
 
-    for (uint32_t t = warp; t < ntiles; t += nwarps) {
-        const uint32_t chunk = a.chunk_begin + t * 32u + lane;
-        const bool active = chunk < a.chunk_end;
-        const uint32_t g = chunk / kLanesPerGroup;
+    const uint32_t tid = threadIdx.x;
+    const uint32_t lane = tid & 31u;
+    const size_t e0 = static_cast<size_t>(a.chunk_begin) * kChunk;
+    const size_t e1 = static_cast<size_t>(a.chunk_end) * kChunk;
+    const uint32_t ntiles = static_cast<uint32_t>((e1 - e0 + Sh::kTile - 1) / Sh::kTile);
+    const uint32_t mine = blockIdx.x < ntiles ? (ntiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+    const size_t code_words = a.n / kChunk; // 32-bit code words per rank
 
-        float c[kChunk];
-        uint32_t owner = 0xFFFFFFFFu;
-        if (COMP) {
-            owner = g / a.groups_per_seg;
-            float4 f0 = make_float4(0.f, 0.f, 0.f, 0.f), f1 = f0, s0 = f0, s1 = f0;
-            if (active) {
-                const float4 *fp = reinterpret_cast<const float4 *>(a.f) + 2 * static_cast<size_t>(chunk);
-                const float4 *sp = reinterpret_cast<const float4 *>(a.s) + 2 * static_cast<size_t>(chunk);
-                f0 = fp[0];
-                f1 = fp[1];
-                s0 = sp[0];
-                s1 = sp[1];
-            }
-            const float fv[kChunk] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
-            const float sv[kChunk] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+    if (tid == 0) {
+        for (int s = 0; s < S; s++)
+            mbar_init(&full[s], 1);
+        mbar_init_fence();
+    }
+    __syncthreads();
+
+    // Thread 0: bulk loads of local tile i into stage i % S.
+    auto issue = [&](uint32_t i) {
+        const size_t el0 = e0 + static_cast<size_t>(blockIdx.x + i * gridDim.x) * Sh::kTile;
+        const uint32_t cnt = static_cast<uint32_t>(e1 - el0 < size_t(Sh::kTile) ? e1 - el0 : Sh::kTile);
+        uint8_t *stage = smem + (i % S) * Sh::kStageBytes;
+        uint64_t *bar = &full[i % S];
+        mbar_arrive_expect_tx(bar, P * cnt * Sh::kEB + (COMP ? 2 * cnt * 4 : 0));
 #pragma unroll
-            for (int k = 0; k < kChunk; k++)
-                c[k] = __fadd_rn(__fmul_rn(a.lambda, fv[k]), __fmul_rn(a.one_minus_lambda, sv[k]));
+        for (int r = 0; r < P; r++)
+            bulk_load(stage + r * Sh::kXBytes, static_cast<const uint8_t *>(a.x.p[r]) + el0 * Sh::kEB,
+                      cnt * Sh::kEB, bar);
+        if (COMP) {
+            bulk_load(stage + P * Sh::kXBytes, a.f + el0, cnt * 4, bar);
+            bulk_load(stage + P * Sh::kXBytes + Sh::kTile * 4, a.s + el0, cnt * 4, bar);
+        }
+    };
+
+    uint32_t issued = 0; // meaningful on thread 0 only
+    if (tid == 0 && !a.ctl.stall)
+        for (; issued < mine && issued < static_cast<uint32_t>(S); issued++)
+            issue(issued);
+
+    for (uint32_t i = 0; i < mine; i++) {
+        if (!wait_tile(&full[i % S], (i / S) & 1u, a.ctl.wait_cycles, a.ctl.status, kStatusTimeoutK1)) {
+            drain_loads(full, S, i, issued, a.ctl.wait_cycles);
+            return;
+        }
+        // Every thread is past tile i-1, so its stage can take tile i-1+S.
+        if (tid == 0 && i >= 1 && i - 1 + S < mine) {
+            issue(i - 1 + S);
+            issued++;
         }
 
+        const size_t el0 = e0 + static_cast<size_t>(blockIdx.x + i * gridDim.x) * Sh::kTile;
+        const uint32_t cnt = static_cast<uint32_t>(e1 - el0 < size_t(Sh::kTile) ? e1 - el0 : Sh::kTile);
+        const uint8_t *stage = smem + (i % S) * Sh::kStageBytes;
+        const float *fs = reinterpret_cast<const float *>(stage + P * Sh::kXBytes);
+
+#pragma unroll 2
+        for (uint32_t it = tid; it < static_cast<uint32_t>(P * Sh::kChunksPerTile); it += kThreads) {
+            const uint32_t r = it / Sh::kChunksPerTile; // warp-uniform
+            const uint32_t c = it % Sh::kChunksPerTile;
+            const bool active = c * kChunk < cnt;
+            const size_t chunk = el0 / kChunk + c;
+            const uint32_t g = static_cast<uint32_t>(chunk / kLanesPerGroup);
+
+            float v[kChunk];
+            load_chunk<BF16>(stage + r * Sh::kXBytes + c * (kChunk * Sh::kEB), v);
+            if (COMP && g / a.groups_per_seg == r) {
+                const float4 f0 = reinterpret_cast<const float4 *>(fs)[2 * c];
+                const float4 f1 = reinterpret_cast<const float4 *>(fs)[2 * c + 1];
+                const float4 s0 = reinterpret_cast<const float4 *>(fs + Sh::kTile)[2 * c];
+                const float4 s1 = reinterpret_cast<const float4 *>(fs + Sh::kTile)[2 * c + 1];
+                const float fv[kChunk] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
+                const float sv[kChunk] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
 #pragma unroll
-        for (int r0 = 0; r0 < P; r0 += kBatch) {
-            Raw<BF16> raw[kBatch];
-#pragma unroll
-            for (int j = 0; j < kBatch; j++) {
-                if (r0 + j < P) {
-                    if (active)
-                        raw[j] = load_raw<BF16>(a.x.p[r0 + j], chunk);
-                    else
-                        raw[j] = Raw<BF16>{};
-                }
+                for (int k = 0; k < kChunk; k++)
+                    v[k] = __fadd_rn(v[k], __fadd_rn(__fmul_rn(a.lambda, fv[k]),
+                                                     __fmul_rn(a.one_minus_lambda, sv[k])));
             }
+            // max |v| as a tree (fmax is exact, so the order is free)
+            float m01 = fmaxf(fabsf(v[0]), fabsf(v[1])), m23 = fmaxf(fabsf(v[2]), fabsf(v[3]));
+            float m45 = fmaxf(fabsf(v[4]), fabsf(v[5])), m67 = fmaxf(fabsf(v[6]), fabsf(v[7]));
+            const float amax = group_absmax(fmaxf(fmaxf(m01, m23), fmaxf(m45, m67)));
+            const uint32_t byte = scale_byte(amax);
+            const float inv = inv_step_of(byte);
+            uint32_t qb[kChunk];
 #pragma unroll
-            for (int j = 0; j < kBatch; j++) {
-                const int r = r0 + j;
-                if (r >= P)
-                    continue;
-                float v[kChunk];
-                to_f32(raw[j], v);
-                if (COMP && owner == static_cast<uint32_t>(r)) {
-#pragma unroll
-                    for (int k = 0; k < kChunk; k++)
-                        v[k] = __fadd_rn(v[k], c[k]);
-                }
-                float amax = 0.f;
-#pragma unroll
-                for (int k = 0; k < kChunk; k++)
-                    amax = fmaxf(amax, fabsf(v[k]));
-                amax = group_absmax(amax);
-                const uint32_t byte = scale_byte(amax);
-                const float inv = inv_step_of(byte);
-                int q[kChunk];
-#pragma unroll
-                for (int k = 0; k < kChunk; k++)
-                    q[k] = code_of(v[k], inv);
-                if (active) {
-                    reinterpret_cast<uint32_t *>(a.codes)[static_cast<size_t>(r) * code_words + chunk] = pack8(q);
-                    if ((lane & 3u) == 0)
-                        a.scales[static_cast<size_t>(r) * scale_bytes + g] = static_cast<uint8_t>(byte);
-                }
+            for (int k = 0; k < kChunk; k++)
+                qb[k] = code_bits(v[k], inv);
+            const uint32_t word = pack8_bits(qb);
+            if (active) {
+                reinterpret_cast<uint32_t *>(a.codes)[static_cast<size_t>(r) * code_words + chunk] = word;
+                if ((lane & 3u) == 0)
+                    a.scales[static_cast<size_t>(r) * a.scale_stride + g] = static_cast<uint8_t>(byte);
             }
         }
     }
 }
 
 template <int P, bool BF16, bool COMP>
-cudaError_t launch_p(const K1Args &a, cudaStream_t st, int max_ctas)
+cudaError_t launch_p(const K1Args &a, cudaStream_t st)
 {
+    using Sh = K1Shape<P, BF16, COMP>;
     static int resident = 0;
     auto kern = k1_compensate_quantize_pack<P, BF16, COMP>;
     if (resident == 0) {
-        int r = 0;
-        cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&r, kern, kThreads, 0);
+        cudaError_t e = prepare_kernel(reinterpret_cast<const void *>(kern), kThreads, Sh::kSmem, &resident);
         if (e != cudaSuccess)
             return e;
-        resident = r > 0 ? r : 1;
     }
-    const uint32_t tiles = (a.chunk_end - a.chunk_begin + 31u) >> 5;
-    const int grid = grid_for(tiles, resident, max_ctas);
-    kern<<<grid, kThreads, 0, st>>>(a);
+    const size_t elems = static_cast<size_t>(a.chunk_end - a.chunk_begin) * kChunk;
+    const uint32_t tiles = static_cast<uint32_t>((elems + Sh::kTile - 1) / Sh::kTile);
+    kern<<<persistent_grid(tiles, resident), kThreads, Sh::kSmem, st>>>(a);
     return cudaGetLastError();
 }
 
 template <int P>
-cudaError_t dispatch_flags(const K1Args &a, cudaStream_t st, int max_ctas)
+cudaError_t dispatch_flags(const K1Args &a, cudaStream_t st)
 {
     if (a.bf16)
-        return a.enable ? launch_p<P, true, true>(a, st, max_ctas) : launch_p<P, true, false>(a, st, max_ctas);
-    return a.enable ? launch_p<P, false, true>(a, st, max_ctas) : launch_p<P, false, false>(a, st, max_ctas);
+        return a.enable ? launch_p<P, true, true>(a, st) : launch_p<P, true, false>(a, st);
+    return a.enable ? launch_p<P, false, true>(a, st) : launch_p<P, false, false>(a, st);
 }
 
 } // namespace
 
-cudaError_t launch_k1_compensate_quantize_pack(const K1Args &a, cudaStream_t st, int max_ctas)
+cudaError_t launch_k1_compensate_quantize_pack(const K1Args &a, cudaStream_t st)
 {
     if (a.chunk_end <= a.chunk_begin)
         return cudaSuccess;
     switch (a.P) {
-    case 2: return dispatch_flags<2>(a, st, max_ctas);
-    case 3: return dispatch_flags<3>(a, st, max_ctas);
-    case 4: return dispatch_flags<4>(a, st, max_ctas);
-    case 5: return dispatch_flags<5>(a, st, max_ctas);
-    case 6: return dispatch_flags<6>(a, st, max_ctas);
-    case 7: return dispatch_flags<7>(a, st, max_ctas);
-    case 8: return dispatch_flags<8>(a, st, max_ctas);
-    case 9: return dispatch_flags<9>(a, st, max_ctas);
-    case 10: return dispatch_flags<10>(a, st, max_ctas);
-    case 11: return dispatch_flags<11>(a, st, max_ctas);
-    case 12: return dispatch_flags<12>(a, st, max_ctas);
-    case 13: return dispatch_flags<13>(a, st, max_ctas);
-    case 14: return dispatch_flags<14>(a, st, max_ctas);
-    case 15: return dispatch_flags<15>(a, st, max_ctas);
-    case 16: return dispatch_flags<16>(a, st, max_ctas);
+    case 2: return dispatch_flags<2>(a, st);
+    case 3: return dispatch_flags<3>(a, st);
+    case 4: return dispatch_flags<4>(a, st);
+    case 5: return dispatch_flags<5>(a, st);
+    case 6: return dispatch_flags<6>(a, st);
+    case 7: return dispatch_flags<7>(a, st);
+    case 8: return dispatch_flags<8>(a, st);
+    case 9: return dispatch_flags<9>(a, st);
+    case 10: return dispatch_flags<10>(a, st);
+    case 11: return dispatch_flags<11>(a, st);
+    case 12: return dispatch_flags<12>(a, st);
+    case 13: return dispatch_flags<13>(a, st);
+    case 14: return dispatch_flags<14>(a, st);
+    case 15: return dispatch_flags<15>(a, st);
+    case 16: return dispatch_flags<16>(a, st);
     default: return cudaErrorInvalidValue;
     }
 }

@@ -15,10 +15,14 @@
 // err is exact: S and Y = Q*2^E differ by at most 2^(E-1) and both are
 // multiples of ulp(S).
 //
-// On one GPU the P owners' segments are contiguous slices of one index
-// space, so a launch simply covers the whole of it: lane = 8 elements, warp
-// step = 256 elements. Per element of n it reads P*17/32 bytes of wire and
-// 8 bytes of state, and writes 17/32 bytes of wire and 8 bytes of state.
+// Pipeline: a persistent CTA takes tiles of kTile elements; thread 0
+// bulk-copies the P code tiles, the P scale tiles and the f, s tiles of a
+// tile into one stage of a kStages ring; one thread then restores one chunk
+// of 8 elements across all P ranks. On one GPU the P owners' segments are
+// contiguous slices of one index space, so a launch covers all of them.
+// Per element of n: P*17/32 bytes of wire and 8 bytes of state read, 17/32
+// bytes of wire and 8 bytes of state written.
+#include "echo_bulk.cuh"
 #include "echo_kernels.h"
 
 #include <cuda_runtime.h>
@@ -29,136 +33,192 @@ namespace {
 constexpr int kThreads = 256;
 
 template <int P, bool COMP>
+struct K2Shape {
+    static constexpr int kTile = kThreads * kChunk;     // 2048: one chunk per thread
+    static constexpr int kStages = 3;
+    static constexpr int kCodeBytes = kTile / 2;         // one rank's code tile
+    static constexpr int kScaleBytes = kTile / kGroup;   // one rank's scale tile (64)
+    static constexpr int kStateOff = P * (kCodeBytes + kScaleBytes);
+    static constexpr int kStageBytes = kStateOff + (COMP ? 2 * kTile * 4 : 0);
+    static constexpr int kSmem = kStages * kStageBytes + kStages * 8;
+};
+
+__device__ __forceinline__ uint32_t round16(uint32_t x) { return (x + 15u) & ~15u; }
+
+template <int P, bool COMP>
 __global__ void __launch_bounds__(kThreads)
     k2_owner_reduce_requant(const K2Args a)
 {
-    const uint32_t lane = threadIdx.x & 31u;
-    const uint32_t warp = (blockIdx.x * kThreads + threadIdx.x) >> 5;
-    const uint32_t nwarps = (gridDim.x * kThreads) >> 5;
-    const uint32_t ntiles = (a.chunk_end - a.chunk_begin + 31u) >> 5;
-    const size_t code_words = a.n / kChunk;
-    const size_t scale_bytes = a.n / kGroup;
-    const uint32_t *codes = reinterpret_cast<const uint32_t *>(a.codes);
+    using Sh = K2Shape<P, COMP>;
+    constexpr int S = Sh::kStages;
+    extern __shared__ __align__(128) uint8_t smem[];
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + S * Sh::kStageBytes);
 
-    for (uint32_t t = warp; t < ntiles; t += nwarps) {
-        const uint32_t chunk = a.chunk_begin + t * 32u + lane;
-        const bool active = chunk < a.chunk_end;
-        const uint32_t g = chunk / kLanesPerGroup;
+    const uint32_t tid = threadIdx.x;
+    const uint32_t lane = tid & 31u;
+    const size_t e0 = static_cast<size_t>(a.chunk_begin) * kChunk;
+    const size_t e1 = static_cast<size_t>(a.chunk_end) * kChunk;
+    const uint32_t ntiles = static_cast<uint32_t>((e1 - e0 + Sh::kTile - 1) / Sh::kTile);
+    const uint32_t mine = blockIdx.x < ntiles ? (ntiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+    const size_t code_bytes = a.n / 2; // per rank
 
-        uint32_t w[P];
-        uint32_t b[P];
+    if (tid == 0) {
+        for (int s = 0; s < S; s++)
+            mbar_init(&full[s], 1);
+        mbar_init_fence();
+    }
+    __syncthreads();
+
+    // Thread 0: bulk loads of local tile i into stage i % S. The scale tile of
+    // a ragged last tile is rounded up to 16 bytes; scale rows are padded to
+    // 16 bytes, so the extra bytes stay inside the row and are never used.
+    auto issue = [&](uint32_t i) {
+        const size_t el0 = e0 + static_cast<size_t>(blockIdx.x + i * gridDim.x) * Sh::kTile;
+        const uint32_t cnt = static_cast<uint32_t>(e1 - el0 < size_t(Sh::kTile) ? e1 - el0 : Sh::kTile);
+        const uint32_t sc_bytes = round16(cnt / kGroup);
+        uint8_t *stage = smem + (i % S) * Sh::kStageBytes;
+        uint64_t *bar = &full[i % S];
+        mbar_arrive_expect_tx(bar, P * (cnt / 2 + sc_bytes) + (COMP ? 2 * cnt * 4 : 0));
 #pragma unroll
         for (int r = 0; r < P; r++) {
-            w[r] = active ? __ldcs(codes + static_cast<size_t>(r) * code_words + chunk) : 0u;
-            b[r] = active ? static_cast<uint32_t>(__ldcs(a.scales + static_cast<size_t>(r) * scale_bytes + g)) : 0u;
+            bulk_load(stage + r * Sh::kCodeBytes, a.codes + r * code_bytes + el0 / 2, cnt / 2, bar);
+            bulk_load(stage + P * Sh::kCodeBytes + r * Sh::kScaleBytes, a.scales + r * a.scale_stride + el0 / kGroup,
+                      sc_bytes, bar);
         }
-        float4 f0 = make_float4(0.f, 0.f, 0.f, 0.f), f1 = f0, s0 = f0, s1 = f0;
-        float4 *fp = reinterpret_cast<float4 *>(a.f) + 2 * static_cast<size_t>(chunk);
-        float4 *sp = reinterpret_cast<float4 *>(a.s) + 2 * static_cast<size_t>(chunk);
-        if (COMP && active) {
-            f0 = fp[0];
-            f1 = fp[1];
-            s0 = sp[0];
-            s1 = sp[1];
+        if (COMP) {
+            bulk_load(stage + Sh::kStateOff, a.f + el0, cnt * 4, bar);
+            bulk_load(stage + Sh::kStateOff + Sh::kTile * 4, a.s + el0, cnt * 4, bar);
+        }
+    };
+
+    uint32_t issued = 0; // meaningful on thread 0 only
+    if (tid == 0 && !a.ctl.stall)
+        for (; issued < mine && issued < static_cast<uint32_t>(S); issued++)
+            issue(issued);
+
+    for (uint32_t i = 0; i < mine; i++) {
+        if (!wait_tile(&full[i % S], (i / S) & 1u, a.ctl.wait_cycles, a.ctl.status, kStatusTimeoutK2)) {
+            drain_loads(full, S, i, issued, a.ctl.wait_cycles);
+            return;
+        }
+        if (tid == 0 && i >= 1 && i - 1 + S < mine) {
+            issue(i - 1 + S);
+            issued++;
         }
 
-        // Restore and add, rank 0 first.
-        float S[kChunk];
+        const size_t el0 = e0 + static_cast<size_t>(blockIdx.x + i * gridDim.x) * Sh::kTile;
+        const uint32_t cnt = static_cast<uint32_t>(e1 - el0 < size_t(Sh::kTile) ? e1 - el0 : Sh::kTile);
+        const uint8_t *stage = smem + (i % S) * Sh::kStageBytes;
+        const uint32_t c = tid; // chunk within the tile
+        const bool active = c * kChunk < cnt;
+        const size_t chunk = el0 / kChunk + c;
+        const size_t g = chunk / kLanesPerGroup;
+
+        // Restore and add, rank 0 first. The product q*2^e is exact, so
+        // fma(q, 2^e, S) = RN(S + q*2^e): one rounding per addition.
+        float S_[kChunk];
 #pragma unroll
         for (int k = 0; k < kChunk; k++)
-            S[k] = 0.f;
+            S_[k] = 0.f;
 #pragma unroll
         for (int r = 0; r < P; r++) {
-            const float st = step_of(b[r]);
+            const uint32_t w = reinterpret_cast<const uint32_t *>(stage + r * Sh::kCodeBytes)[c];
+            const uint32_t b = stage[P * Sh::kCodeBytes + r * Sh::kScaleBytes + c / kLanesPerGroup];
+            const float st = step_of(b);
+            const Unpacked u = unpack8(w);
 #pragma unroll
             for (int k = 0; k < kChunk; k++)
-                S[k] = __fadd_rn(S[k], __fmul_rn(static_cast<float>(nibble(w[r], k)), st));
+                S_[k] = __fmaf_rn(code_at(u, k), st, S_[k]);
         }
 
-        // Rounding #2.
-        float amax = 0.f;
-#pragma unroll
-        for (int k = 0; k < kChunk; k++)
-            amax = fmaxf(amax, fabsf(S[k]));
-        amax = group_absmax(amax);
+        // Rounding #2 and the error it injects.
+        float m01 = fmaxf(fabsf(S_[0]), fabsf(S_[1])), m23 = fmaxf(fabsf(S_[2]), fabsf(S_[3]));
+        float m45 = fmaxf(fabsf(S_[4]), fabsf(S_[5])), m67 = fmaxf(fabsf(S_[6]), fabsf(S_[7]));
+        const float amax = group_absmax(fmaxf(fmaxf(m01, m23), fmaxf(m45, m67)));
         const uint32_t byte = scale_byte(amax);
         const float inv = inv_step_of(byte);
         const float st = step_of(byte);
-        int q[kChunk];
+        uint32_t qb[kChunk];
         float err[kChunk];
 #pragma unroll
         for (int k = 0; k < kChunk; k++) {
-            q[k] = code_of(S[k], inv);
-            err[k] = __fsub_rn(S[k], __fmul_rn(static_cast<float>(q[k]), st));
+            qb[k] = code_bits(S_[k], inv);
+            err[k] = __fmaf_rn(-code_value(qb[k]), st, S_[k]); // S - Q*2^E, exact
         }
 
-        if (!active)
-            continue;
-        reinterpret_cast<uint32_t *>(a.qcodes)[chunk] = pack8(q);
-        if ((lane & 3u) == 0)
-            a.qscales[g] = static_cast<uint8_t>(byte);
-
-        if (COMP) {
-            float fv[kChunk] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
-            float sv[kChunk] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+        if (active) {
+            reinterpret_cast<uint32_t *>(a.qcodes)[chunk] = pack8_bits(qb);
+            if ((lane & 3u) == 0)
+                a.qscales[g] = static_cast<uint8_t>(byte);
+            if (COMP) {
+                const float *fs = reinterpret_cast<const float *>(stage + Sh::kStateOff);
+                const float4 f0 = reinterpret_cast<const float4 *>(fs)[2 * c];
+                const float4 f1 = reinterpret_cast<const float4 *>(fs)[2 * c + 1];
+                const float4 s0 = reinterpret_cast<const float4 *>(fs + Sh::kTile)[2 * c];
+                const float4 s1 = reinterpret_cast<const float4 *>(fs + Sh::kTile)[2 * c + 1];
+                float fv[kChunk] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
+                float sv[kChunk] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
 #pragma unroll
-            for (int k = 0; k < kChunk; k++) {
-                fv[k] = __fadd_rn(__fmul_rn(a.beta_f, fv[k]), __fmul_rn(a.one_minus_beta_f, err[k]));
-                sv[k] = __fadd_rn(__fmul_rn(a.beta_s, sv[k]), __fmul_rn(a.one_minus_beta_s, err[k]));
+                for (int k = 0; k < kChunk; k++) {
+                    fv[k] = __fadd_rn(__fmul_rn(a.beta_f, fv[k]), __fmul_rn(a.one_minus_beta_f, err[k]));
+                    sv[k] = __fadd_rn(__fmul_rn(a.beta_s, sv[k]), __fmul_rn(a.one_minus_beta_s, err[k]));
+                }
+                float4 *fo = reinterpret_cast<float4 *>(a.f) + 2 * chunk;
+                float4 *so = reinterpret_cast<float4 *>(a.s) + 2 * chunk;
+                fo[0] = make_float4(fv[0], fv[1], fv[2], fv[3]);
+                fo[1] = make_float4(fv[4], fv[5], fv[6], fv[7]);
+                so[0] = make_float4(sv[0], sv[1], sv[2], sv[3]);
+                so[1] = make_float4(sv[4], sv[5], sv[6], sv[7]);
             }
-            fp[0] = make_float4(fv[0], fv[1], fv[2], fv[3]);
-            fp[1] = make_float4(fv[4], fv[5], fv[6], fv[7]);
-            sp[0] = make_float4(sv[0], sv[1], sv[2], sv[3]);
-            sp[1] = make_float4(sv[4], sv[5], sv[6], sv[7]);
         }
     }
 }
 
 template <int P, bool COMP>
-cudaError_t launch_p(const K2Args &a, cudaStream_t st, int max_ctas)
+cudaError_t launch_p(const K2Args &a, cudaStream_t st)
 {
+    using Sh = K2Shape<P, COMP>;
     static int resident = 0;
     auto kern = k2_owner_reduce_requant<P, COMP>;
     if (resident == 0) {
-        int r = 0;
-        cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&r, kern, kThreads, 0);
+        cudaError_t e = prepare_kernel(reinterpret_cast<const void *>(kern), kThreads, Sh::kSmem, &resident);
         if (e != cudaSuccess)
             return e;
-        resident = r > 0 ? r : 1;
     }
-    const uint32_t tiles = (a.chunk_end - a.chunk_begin + 31u) >> 5;
-    kern<<<grid_for(tiles, resident, max_ctas), kThreads, 0, st>>>(a);
+    const size_t elems = static_cast<size_t>(a.chunk_end - a.chunk_begin) * kChunk;
+    const uint32_t tiles = static_cast<uint32_t>((elems + Sh::kTile - 1) / Sh::kTile);
+    kern<<<persistent_grid(tiles, resident), kThreads, Sh::kSmem, st>>>(a);
     return cudaGetLastError();
 }
 
 template <int P>
-cudaError_t dispatch_flags(const K2Args &a, cudaStream_t st, int max_ctas)
+cudaError_t dispatch_flags(const K2Args &a, cudaStream_t st)
 {
-    return a.enable ? launch_p<P, true>(a, st, max_ctas) : launch_p<P, false>(a, st, max_ctas);
+    return a.enable ? launch_p<P, true>(a, st) : launch_p<P, false>(a, st);
 }
 
 } // namespace
 
-cudaError_t launch_k2_owner_reduce_requant(const K2Args &a, cudaStream_t st, int max_ctas)
+cudaError_t launch_k2_owner_reduce_requant(const K2Args &a, cudaStream_t st)
 {
     if (a.chunk_end <= a.chunk_begin)
         return cudaSuccess;
     switch (a.P) {
-    case 2: return dispatch_flags<2>(a, st, max_ctas);
-    case 3: return dispatch_flags<3>(a, st, max_ctas);
-    case 4: return dispatch_flags<4>(a, st, max_ctas);
-    case 5: return dispatch_flags<5>(a, st, max_ctas);
-    case 6: return dispatch_flags<6>(a, st, max_ctas);
-    case 7: return dispatch_flags<7>(a, st, max_ctas);
-    case 8: return dispatch_flags<8>(a, st, max_ctas);
-    case 9: return dispatch_flags<9>(a, st, max_ctas);
-    case 10: return dispatch_flags<10>(a, st, max_ctas);
-    case 11: return dispatch_flags<11>(a, st, max_ctas);
-    case 12: return dispatch_flags<12>(a, st, max_ctas);
-    case 13: return dispatch_flags<13>(a, st, max_ctas);
-    case 14: return dispatch_flags<14>(a, st, max_ctas);
-    case 15: return dispatch_flags<15>(a, st, max_ctas);
-    case 16: return dispatch_flags<16>(a, st, max_ctas);
+    case 2: return dispatch_flags<2>(a, st);
+    case 3: return dispatch_flags<3>(a, st);
+    case 4: return dispatch_flags<4>(a, st);
+    case 5: return dispatch_flags<5>(a, st);
+    case 6: return dispatch_flags<6>(a, st);
+    case 7: return dispatch_flags<7>(a, st);
+    case 8: return dispatch_flags<8>(a, st);
+    case 9: return dispatch_flags<9>(a, st);
+    case 10: return dispatch_flags<10>(a, st);
+    case 11: return dispatch_flags<11>(a, st);
+    case 12: return dispatch_flags<12>(a, st);
+    case 13: return dispatch_flags<13>(a, st);
+    case 14: return dispatch_flags<14>(a, st);
+    case 15: return dispatch_flags<15>(a, st);
+    case 16: return dispatch_flags<16>(a, st);
     default: return cudaErrorInvalidValue;
     }
 }

@@ -34,7 +34,7 @@ EXPORTED = (
     "echo_reset", "echo_destroy", "echo_last_error", "echo_last_status", "echo_set_params",
     "echo_get_state", "echo_set_state", "echo_get_state_range", "echo_get_wire",
     "echo_get_wire_range", "echo_stats", "echo_model_bytes", "echo_set_timing",
-    "echo_last_kernel_ms", "echo_kernel_ms_total",
+    "echo_last_kernel_ms", "echo_kernel_ms_total", "echo_device_status",
 )
 
 _vp = ctypes.c_void_p
@@ -72,6 +72,7 @@ def _load():
         "echo_set_timing": (_int, [_vp, _int]),
         "echo_last_kernel_ms": (_int, [_vp, _f32p]),
         "echo_kernel_ms_total": (_int, [_vp, ctypes.POINTER(ctypes.c_double), _u64p]),
+        "echo_device_status": (_int, [_vp, ctypes.POINTER(ctypes.c_int), _int]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -180,9 +181,9 @@ def echo_get_wire_range(h: int, stage: int, rank: int, group_offset: int, ngroup
 
 
 def echo_stats(h: int) -> dict:
-    vals = (ctypes.c_uint64 * 3)()
-    _check(_lib.echo_stats(h, ctypes.byref(vals, 0), ctypes.byref(vals, 8), ctypes.byref(vals, 16)))
-    return {"link_bytes": vals[0], "model_hbm_bytes": vals[1], "calls": vals[2]}
+    link, hbm, calls = ctypes.c_uint64(), ctypes.c_uint64(), ctypes.c_uint64()
+    _check(_lib.echo_stats(h, ctypes.byref(link), ctypes.byref(hbm), ctypes.byref(calls)))
+    return {"link_bytes": link.value, "model_hbm_bytes": hbm.value, "calls": calls.value}
 
 
 def echo_model_bytes(P: int, n: int, dtype: int = ECHO_BF16, enable: bool = True) -> dict:
@@ -200,6 +201,12 @@ def echo_last_kernel_ms(h: int) -> list[float]:
     ms = (ctypes.c_float * 3)()
     _check(_lib.echo_last_kernel_ms(h, ms))
     return [ms[0], ms[1], ms[2]]
+
+
+def echo_device_status(h: int, clear: bool = False) -> int:
+    st = ctypes.c_int()
+    _check(_lib.echo_device_status(h, ctypes.byref(st), int(bool(clear))))
+    return st.value
 
 
 def echo_kernel_ms_total(h: int) -> tuple[list[float], int]:
@@ -277,6 +284,9 @@ class Echo:
 
     def kernel_ms_total(self) -> tuple[list[float], int]:
         return echo_kernel_ms_total(self.h)
+
+    def device_status(self, clear: bool = False) -> int:
+        return echo_device_status(self.h, clear)
 
     def close(self) -> None:
         if self.h:

@@ -194,6 +194,15 @@ ECHO_API int echo_model_bytes(int P, size_t n, int dtype, int enable, uint64_t o
  * the measurement started, and how many calls that was (waiting for the last).
  * echo_set_timing(h, 0) stops recording; the totals stay readable.
  */
+/*
+ * echo_device_status - the handle's device status word (synchronous): 0, or
+ * bits 1/2/4 when a wait inside kernel 1/2/3 ran out of its time bound (about
+ * a second). The kernels never spin without bound; a CTA whose tile did not
+ * arrive in time records the bit and returns, leaving that call's outputs
+ * incomplete. clear != 0 resets the word after reading it.
+ */
+ECHO_API int echo_device_status(echo_handle *h, int *status, int clear);
+
 ECHO_API int echo_set_timing(echo_handle *h, int enable);
 ECHO_API int echo_last_kernel_ms(echo_handle *h, float ms[3]);
 ECHO_API int echo_kernel_ms_total(echo_handle *h, double ms[3], uint64_t *timed_calls);

@@ -216,6 +216,41 @@ def test_injected_launch_failure():
     assert res.returncode == 0, res.stderr + res.stdout
 
 
+def test_bounded_waits_report_timeouts():
+    """With ECHO_FAULT=stall the kernels issue no loads, so the first wait of
+    every CTA runs out after its (short) bound: each kernel records its bit in
+    the device status word and returns, and the context stays usable."""
+    code = (
+        "import os; os.environ['ECHO_FAULT'] = 'stall'\n"
+        "import torch\n"
+        "from bit_error_compensated_rank_b200 import echo as e\n"
+        "h = e.Echo(4, 4 * 32 * 1000)\n"
+        "x = [torch.zeros(4 * 32 * 1000, device='cuda', dtype=torch.bfloat16) for _ in range(4)]\n"
+        "h.allreduce(x)\n"
+        "torch.cuda.synchronize()\n"
+        "assert h.device_status() == 7, h.device_status()\n"
+        "assert h.device_status(clear=True) == 7\n"
+        "assert h.device_status() == 0\n"
+        "y = torch.ones(1024, device='cuda') * 2\n"
+        "assert float(y.sum()) == 2048.0\n"
+        "h.close()\n"
+    )
+    res = subprocess.run([sys.executable, "-c", code], cwd=ROOT, capture_output=True, text=True,
+                         timeout=120)
+    assert res.returncode == 0, res.stderr + res.stdout
+
+
+def test_no_timeouts_in_normal_calls(oracle):
+    P, n = 8, 8 * 32 * 5000
+    fc = FullCompare(oracle, P, n, "bf16")
+    try:
+        for k in range(2):
+            fc.call(gaussian(P, n, seed=31, call=k))
+        assert fc.h.device_status() == 0
+    finally:
+        fc.close()
+
+
 def test_host_end_to_end(oracle):
     """Host buffers in, host result out (pipelined pieces of 2^22 elements)."""
     import torch
