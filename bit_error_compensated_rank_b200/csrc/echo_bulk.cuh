@@ -1,14 +1,16 @@
 // echo_bulk.cuh - bulk-copy (TMA engine) pipeline helpers for sm_100a.
 //
 // The three kernels stream tiles between HBM and shared memory with the
-// untiled bulk copy (cp.async.bulk): one elected thread issues whole-tile
-// copies, completion is tracked by an mbarrier's transaction count, and the
-// rest of the CTA computes from shared memory. No copy uses cluster
+// untiled bulk copy (cp.async.bulk): one elected thread of a producer warp
+// issues whole-tile copies, completion is tracked by an mbarrier's
+// transaction count ("full"), consumer warps compute from shared memory and
+// hand each stage back on a second mbarrier ("empty"). No copy uses cluster
 // multicast, and every copy reads or writes only this GPU's memory.
 //
-// Every wait is bounded in time: a CTA that does not see its tile arrive
-// within the limit records the failure in the device status word and leaves
-// its loop (see wait_tile), so a fault in the pipeline can never hang the GPU.
+// Every wait is bounded in time: a warp that does not see its barrier phase
+// complete within the limit records the failure in the device status word
+// and leaves its loop (warp_wait, produce_tiles), so a fault in the pipeline
+// can never hang the GPU.
 #pragma once
 
 #include <cstdint>
@@ -102,28 +104,46 @@ __device__ __forceinline__ void fence_proxy_async_smem()
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-// Every thread waits (bounded) for the tile in `bar`'s current phase; the
-// outcome is made CTA-uniform with a barrier, so either all threads go on or
-// all leave together. On a timeout, thread 0 records `status_bit`.
-__device__ __forceinline__ bool wait_tile(uint64_t *bar, uint32_t parity, long long limit, int *status,
-                                          int status_bit)
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar)
 {
-    const bool ok = mbar_wait_bounded(bar, parity, limit);
-    const bool all = __syncthreads_and(ok) != 0;
-    if (!all && threadIdx.x == 0)
-        atomicOr(status, status_bit);
-    return all;
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
-// After a timeout: give the loads still in flight (local tiles [from, to) of
-// an S-stage ring) a bounded chance to land before the CTA's shared memory is
-// released.
-__device__ __forceinline__ void drain_loads(uint64_t *full, int S, uint32_t from, uint32_t to, long long limit)
+// Every lane of the calling warp waits (bounded) for the phase with parity
+// `parity`; the outcome is made warp-uniform, so the warp goes on or leaves
+// as a whole. On a timeout lane 0 records `status_bit`.
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, long long limit, int *status,
+                                          int status_bit)
 {
-    if (threadIdx.x == 0)
-        for (uint32_t t = from; t < to; t++)
-            mbar_wait_bounded(&full[t % S], (t / S) & 1u, limit);
-    __syncthreads();
+    const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait_bounded(bar, parity, limit));
+    if (!ok && (threadIdx.x & 31u) == 0)
+        atomicOr(status, status_bit);
+    return ok;
+}
+
+// Producer side of an S-stage ring of tiles (one elected thread). issue(i)
+// must arm full[i % S] with the byte count and start the copies of local tile
+// i. Stage s is reused only after every consumer warp has released it on
+// empty[s]. Before returning, the producer waits (bounded) until the loads of
+// the last S tiles it issued have landed, so no copy is in flight when the CTA
+// leaves, also after a timeout.
+template <int S, typename Issue>
+__device__ __forceinline__ void produce_tiles(uint64_t *full, uint64_t *empty, uint32_t tiles, bool stall,
+                                              long long limit, int *status, int status_bit, Issue issue)
+{
+    uint32_t i = 0;
+    if (!stall) {
+        for (; i < tiles; i++) {
+            const uint32_t s = i % S;
+            if (i >= static_cast<uint32_t>(S) && !mbar_wait_bounded(&empty[s], ((i / S) - 1) & 1u, limit)) {
+                atomicOr(status, status_bit);
+                break;
+            }
+            issue(i);
+        }
+    }
+    for (uint32_t t = i > static_cast<uint32_t>(S) ? i - S : 0; t < i; t++)
+        mbar_wait_bounded(&full[t % S], (t / S) & 1u, limit);
 }
 
 } // namespace echo

@@ -10,13 +10,14 @@
 // is the stage-1 wire, codes [P][n/2] (two per byte) and scale bytes
 // [P][scale_stride].
 //
-// Pipeline: a persistent CTA takes tiles of kTile consecutive elements. For
-// each tile, thread 0 bulk-copies the P partial tiles and the f, s tiles into
-// one stage of a kStages ring in shared memory (one mbarrier per stage counts
-// the bytes); the CTA computes from shared memory while the next stages are
-// in flight. A lane owns 8 consecutive elements of one rank; 4 lanes form a
-// group and find its maximum with two shuffles; codes leave as one coalesced
-// 32-bit store per lane.
+// Pipeline (warp-specialised, persistent): a CTA takes tiles of kTile
+// consecutive elements. One producer warp bulk-copies the P partial tiles and
+// the f, s tiles of a tile into one stage of a kStages ring in shared memory
+// (mbarrier full[s] counts the bytes); eight consumer warps compute from
+// shared memory and release the stage on mbarrier empty[s]. A lane owns 8
+// consecutive elements of one rank; 4 lanes form a group and find its
+// maximum with two shuffles; codes leave as one coalesced 32-bit store per
+// lane.
 //
 // Algorithmic HBM bytes per element of n: P*b (partials) + 8 (f, s; each
 // element is corrected by exactly one rank) read, P*17/32 written.
@@ -28,7 +29,9 @@
 namespace echo {
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kConsumerWarps = 8;
+constexpr int kConsumers = kConsumerWarps * 32;
+constexpr int kThreads = kConsumers + 32; // + one producer warp
 
 template <int P, bool BF16, bool COMP>
 struct K1Shape {
@@ -38,7 +41,7 @@ struct K1Shape {
     static constexpr int kStages = 3;
     static constexpr int kXBytes = kTile * kEB; // one rank's partial tile
     static constexpr int kStageBytes = P * kXBytes + (COMP ? 2 * kTile * 4 : 0);
-    static constexpr int kSmem = kStages * kStageBytes + kStages * 8;
+    static constexpr int kSmem = kStages * kStageBytes + 2 * kStages * 8;
     static constexpr int kChunksPerTile = kTile / kChunk; // a multiple of 32
 };
 
@@ -63,71 +66,70 @@ __global__ void __launch_bounds__(kThreads)
     constexpr int S = Sh::kStages;
     extern __shared__ __align__(128) uint8_t smem[];
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + S * Sh::kStageBytes);
+    uint64_t *empty = full + S;
 
     const uint32_t tid = threadIdx.x;
+    const uint32_t warp = tid >> 5;
     const uint32_t lane = tid & 31u;
     const size_t e0 = static_cast<size_t>(a.chunk_begin) * kChunk;
     const size_t e1 = static_cast<size_t>(a.chunk_end) * kChunk;
     const uint32_t ntiles = static_cast<uint32_t>((e1 - e0 + Sh::kTile - 1) / Sh::kTile);
     const uint32_t mine = blockIdx.x < ntiles ? (ntiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
-    const size_t code_words = a.n / kChunk; // 32-bit code words per rank
 
     if (tid == 0) {
-        for (int s = 0; s < S; s++)
+        for (int s = 0; s < S; s++) {
             mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kConsumerWarps);
+        }
         mbar_init_fence();
     }
     __syncthreads();
 
-    // Thread 0: bulk loads of local tile i into stage i % S.
-    auto issue = [&](uint32_t i) {
-        const size_t el0 = e0 + static_cast<size_t>(blockIdx.x + i * gridDim.x) * Sh::kTile;
-        const uint32_t cnt = static_cast<uint32_t>(e1 - el0 < size_t(Sh::kTile) ? e1 - el0 : Sh::kTile);
-        uint8_t *stage = smem + (i % S) * Sh::kStageBytes;
-        uint64_t *bar = &full[i % S];
-        mbar_arrive_expect_tx(bar, P * cnt * Sh::kEB + (COMP ? 2 * cnt * 4 : 0));
+    if (warp == kConsumerWarps) { // producer
+        if (lane == 0)
+            produce_tiles<S>(full, empty, mine, a.ctl.stall, a.ctl.wait_cycles, a.ctl.status, kStatusTimeoutK1,
+                             [&](uint32_t i) {
+                                 const size_t el0 = e0 + static_cast<size_t>(blockIdx.x + i * gridDim.x) * Sh::kTile;
+                                 const uint32_t cnt = static_cast<uint32_t>(
+                                     e1 - el0 < size_t(Sh::kTile) ? e1 - el0 : Sh::kTile);
+                                 uint8_t *stage = smem + (i % S) * Sh::kStageBytes;
+                                 uint64_t *bar = &full[i % S];
+                                 mbar_arrive_expect_tx(bar, P * cnt * Sh::kEB + (COMP ? 2 * cnt * 4 : 0));
 #pragma unroll
-        for (int r = 0; r < P; r++)
-            bulk_load(stage + r * Sh::kXBytes, static_cast<const uint8_t *>(a.x.p[r]) + el0 * Sh::kEB,
-                      cnt * Sh::kEB, bar);
-        if (COMP) {
-            bulk_load(stage + P * Sh::kXBytes, a.f + el0, cnt * 4, bar);
-            bulk_load(stage + P * Sh::kXBytes + Sh::kTile * 4, a.s + el0, cnt * 4, bar);
-        }
-    };
+                                 for (int r = 0; r < P; r++)
+                                     bulk_load(stage + r * Sh::kXBytes,
+                                               static_cast<const uint8_t *>(a.x.p[r]) + el0 * Sh::kEB,
+                                               cnt * Sh::kEB, bar);
+                                 if (COMP) {
+                                     bulk_load(stage + P * Sh::kXBytes, a.f + el0, cnt * 4, bar);
+                                     bulk_load(stage + P * Sh::kXBytes + Sh::kTile * 4, a.s + el0, cnt * 4, bar);
+                                 }
+                             });
+        return;
+    }
 
-    uint32_t issued = 0; // meaningful on thread 0 only
-    if (tid == 0 && !a.ctl.stall)
-        for (; issued < mine && issued < static_cast<uint32_t>(S); issued++)
-            issue(issued);
-
+    const uint32_t code_words = static_cast<uint32_t>(a.n / kChunk); // 32-bit code words per rank
     for (uint32_t i = 0; i < mine; i++) {
-        if (!wait_tile(&full[i % S], (i / S) & 1u, a.ctl.wait_cycles, a.ctl.status, kStatusTimeoutK1)) {
-            drain_loads(full, S, i, issued, a.ctl.wait_cycles);
+        const uint32_t s = i % S;
+        if (!warp_wait(&full[s], (i / S) & 1u, a.ctl.wait_cycles, a.ctl.status, kStatusTimeoutK1))
             return;
-        }
-        // Every thread is past tile i-1, so its stage can take tile i-1+S.
-        if (tid == 0 && i >= 1 && i - 1 + S < mine) {
-            issue(i - 1 + S);
-            issued++;
-        }
-
-        const size_t el0 = e0 + static_cast<size_t>(blockIdx.x + i * gridDim.x) * Sh::kTile;
-        const uint32_t cnt = static_cast<uint32_t>(e1 - el0 < size_t(Sh::kTile) ? e1 - el0 : Sh::kTile);
-        const uint8_t *stage = smem + (i % S) * Sh::kStageBytes;
+        const uint32_t tile_chunk0 = static_cast<uint32_t>(e0 / kChunk) + (blockIdx.x + i * gridDim.x) * (Sh::kTile / kChunk);
+        const uint32_t cnt_chunks = min(static_cast<uint32_t>(Sh::kChunksPerTile), a.chunk_end - tile_chunk0);
+        const uint8_t *stage = smem + s * Sh::kStageBytes;
         const float *fs = reinterpret_cast<const float *>(stage + P * Sh::kXBytes);
 
 #pragma unroll 2
-        for (uint32_t it = tid; it < static_cast<uint32_t>(P * Sh::kChunksPerTile); it += kThreads) {
+        for (uint32_t it = tid; it < static_cast<uint32_t>(P * Sh::kChunksPerTile); it += kConsumers) {
             const uint32_t r = it / Sh::kChunksPerTile; // warp-uniform
             const uint32_t c = it % Sh::kChunksPerTile;
-            const bool active = c * kChunk < cnt;
-            const size_t chunk = el0 / kChunk + c;
-            const uint32_t g = static_cast<uint32_t>(chunk / kLanesPerGroup);
+            const bool active = c < cnt_chunks;
+            const uint32_t chunk = tile_chunk0 + c;
+            const uint32_t g = chunk / kLanesPerGroup;
 
             float v[kChunk];
             load_chunk<BF16>(stage + r * Sh::kXBytes + c * (kChunk * Sh::kEB), v);
-            if (COMP && g / a.groups_per_seg == r) {
+            // rank r owns groups [r*gps, (r+1)*gps): one unsigned range test
+            if (COMP && g - r * a.groups_per_seg < a.groups_per_seg) {
                 const float4 f0 = reinterpret_cast<const float4 *>(fs)[2 * c];
                 const float4 f1 = reinterpret_cast<const float4 *>(fs)[2 * c + 1];
                 const float4 s0 = reinterpret_cast<const float4 *>(fs + Sh::kTile)[2 * c];
@@ -140,8 +142,8 @@ __global__ void __launch_bounds__(kThreads)
                                                      __fmul_rn(a.one_minus_lambda, sv[k])));
             }
             // max |v| as a tree (fmax is exact, so the order is free)
-            float m01 = fmaxf(fabsf(v[0]), fabsf(v[1])), m23 = fmaxf(fabsf(v[2]), fabsf(v[3]));
-            float m45 = fmaxf(fabsf(v[4]), fabsf(v[5])), m67 = fmaxf(fabsf(v[6]), fabsf(v[7]));
+            const float m01 = fmaxf(fabsf(v[0]), fabsf(v[1])), m23 = fmaxf(fabsf(v[2]), fabsf(v[3]));
+            const float m45 = fmaxf(fabsf(v[4]), fabsf(v[5])), m67 = fmaxf(fabsf(v[6]), fabsf(v[7]));
             const float amax = group_absmax(fmaxf(fmaxf(m01, m23), fmaxf(m45, m67)));
             const uint32_t byte = scale_byte(amax);
             const float inv = inv_step_of(byte);
@@ -156,6 +158,9 @@ __global__ void __launch_bounds__(kThreads)
                     a.scales[static_cast<size_t>(r) * a.scale_stride + g] = static_cast<uint8_t>(byte);
             }
         }
+        __syncwarp();
+        if (lane == 0)
+            mbar_arrive(&empty[s]); // this warp is done reading stage s
     }
 }
 

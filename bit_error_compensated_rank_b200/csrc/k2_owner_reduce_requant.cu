@@ -15,10 +15,12 @@
 // err is exact: S and Y = Q*2^E differ by at most 2^(E-1) and both are
 // multiples of ulp(S).
 //
-// Pipeline: a persistent CTA takes tiles of kTile elements; thread 0
-// bulk-copies the P code tiles, the P scale tiles and the f, s tiles of a
-// tile into one stage of a kStages ring; one thread then restores one chunk
-// of 8 elements across all P ranks. On one GPU the P owners' segments are
+// Pipeline (warp-specialised, persistent): a CTA takes tiles of kTile
+// elements; one producer warp bulk-copies the P code tiles, the P scale tiles
+// and the f, s tiles of a tile into one stage of a kStages ring (mbarrier
+// full[s]); each lane of the eight consumer warps then restores one chunk of
+// 8 elements across all P ranks, and each warp releases the stage on
+// mbarrier empty[s]. On one GPU the P owners' segments are
 // contiguous slices of one index space, so a launch covers all of them.
 // Per element of n: P*17/32 bytes of wire and 8 bytes of state read, 17/32
 // bytes of wire and 8 bytes of state written.
@@ -30,17 +32,19 @@
 namespace echo {
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kConsumerWarps = 8;
+constexpr int kConsumers = kConsumerWarps * 32;
+constexpr int kThreads = kConsumers + 32; // + one producer warp
 
 template <int P, bool COMP>
 struct K2Shape {
-    static constexpr int kTile = kThreads * kChunk;     // 2048: one chunk per thread
+    static constexpr int kTile = kConsumers * kChunk;   // 2048: one chunk per consumer thread
     static constexpr int kStages = 3;
     static constexpr int kCodeBytes = kTile / 2;         // one rank's code tile
     static constexpr int kScaleBytes = kTile / kGroup;   // one rank's scale tile (64)
     static constexpr int kStateOff = P * (kCodeBytes + kScaleBytes);
     static constexpr int kStageBytes = kStateOff + (COMP ? 2 * kTile * 4 : 0);
-    static constexpr int kSmem = kStages * kStageBytes + kStages * 8;
+    static constexpr int kSmem = kStages * kStageBytes + 2 * kStages * 8;
 };
 
 __device__ __forceinline__ uint32_t round16(uint32_t x) { return (x + 15u) & ~15u; }
@@ -53,66 +57,62 @@ __global__ void __launch_bounds__(kThreads)
     constexpr int S = Sh::kStages;
     extern __shared__ __align__(128) uint8_t smem[];
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + S * Sh::kStageBytes);
+    uint64_t *empty = full + S;
 
     const uint32_t tid = threadIdx.x;
+    const uint32_t warp = tid >> 5;
     const uint32_t lane = tid & 31u;
     const size_t e0 = static_cast<size_t>(a.chunk_begin) * kChunk;
     const size_t e1 = static_cast<size_t>(a.chunk_end) * kChunk;
     const uint32_t ntiles = static_cast<uint32_t>((e1 - e0 + Sh::kTile - 1) / Sh::kTile);
     const uint32_t mine = blockIdx.x < ntiles ? (ntiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
-    const size_t code_bytes = a.n / 2; // per rank
 
     if (tid == 0) {
-        for (int s = 0; s < S; s++)
+        for (int s = 0; s < S; s++) {
             mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kConsumerWarps);
+        }
         mbar_init_fence();
     }
     __syncthreads();
 
-    // Thread 0: bulk loads of local tile i into stage i % S. The scale tile of
-    // a ragged last tile is rounded up to 16 bytes; scale rows are padded to
-    // 16 bytes, so the extra bytes stay inside the row and are never used.
-    auto issue = [&](uint32_t i) {
-        const size_t el0 = e0 + static_cast<size_t>(blockIdx.x + i * gridDim.x) * Sh::kTile;
-        const uint32_t cnt = static_cast<uint32_t>(e1 - el0 < size_t(Sh::kTile) ? e1 - el0 : Sh::kTile);
-        const uint32_t sc_bytes = round16(cnt / kGroup);
-        uint8_t *stage = smem + (i % S) * Sh::kStageBytes;
-        uint64_t *bar = &full[i % S];
-        mbar_arrive_expect_tx(bar, P * (cnt / 2 + sc_bytes) + (COMP ? 2 * cnt * 4 : 0));
+    if (warp == kConsumerWarps) { // producer
+        // The scale tile of a ragged last tile is rounded up to 16 bytes;
+        // scale rows are padded to 16 bytes, so the extra bytes stay inside
+        // the row and are never used.
+        if (lane == 0)
+            produce_tiles<S>(
+                full, empty, mine, a.ctl.stall, a.ctl.wait_cycles, a.ctl.status, kStatusTimeoutK2, [&](uint32_t i) {
+                    const size_t el0 = e0 + static_cast<size_t>(blockIdx.x + i * gridDim.x) * Sh::kTile;
+                    const uint32_t cnt = static_cast<uint32_t>(e1 - el0 < size_t(Sh::kTile) ? e1 - el0 : Sh::kTile);
+                    const uint32_t sc_bytes = round16(cnt / kGroup);
+                    uint8_t *stage = smem + (i % S) * Sh::kStageBytes;
+                    uint64_t *bar = &full[i % S];
+                    mbar_arrive_expect_tx(bar, P * (cnt / 2 + sc_bytes) + (COMP ? 2 * cnt * 4 : 0));
 #pragma unroll
-        for (int r = 0; r < P; r++) {
-            bulk_load(stage + r * Sh::kCodeBytes, a.codes + r * code_bytes + el0 / 2, cnt / 2, bar);
-            bulk_load(stage + P * Sh::kCodeBytes + r * Sh::kScaleBytes, a.scales + r * a.scale_stride + el0 / kGroup,
-                      sc_bytes, bar);
-        }
-        if (COMP) {
-            bulk_load(stage + Sh::kStateOff, a.f + el0, cnt * 4, bar);
-            bulk_load(stage + Sh::kStateOff + Sh::kTile * 4, a.s + el0, cnt * 4, bar);
-        }
-    };
-
-    uint32_t issued = 0; // meaningful on thread 0 only
-    if (tid == 0 && !a.ctl.stall)
-        for (; issued < mine && issued < static_cast<uint32_t>(S); issued++)
-            issue(issued);
+                    for (int r = 0; r < P; r++) {
+                        bulk_load(stage + r * Sh::kCodeBytes, a.codes + r * (a.n / 2) + el0 / 2, cnt / 2, bar);
+                        bulk_load(stage + P * Sh::kCodeBytes + r * Sh::kScaleBytes,
+                                  a.scales + r * a.scale_stride + el0 / kGroup, sc_bytes, bar);
+                    }
+                    if (COMP) {
+                        bulk_load(stage + Sh::kStateOff, a.f + el0, cnt * 4, bar);
+                        bulk_load(stage + Sh::kStateOff + Sh::kTile * 4, a.s + el0, cnt * 4, bar);
+                    }
+                });
+        return;
+    }
 
     for (uint32_t i = 0; i < mine; i++) {
-        if (!wait_tile(&full[i % S], (i / S) & 1u, a.ctl.wait_cycles, a.ctl.status, kStatusTimeoutK2)) {
-            drain_loads(full, S, i, issued, a.ctl.wait_cycles);
+        const uint32_t sidx = i % S;
+        if (!warp_wait(&full[sidx], (i / S) & 1u, a.ctl.wait_cycles, a.ctl.status, kStatusTimeoutK2))
             return;
-        }
-        if (tid == 0 && i >= 1 && i - 1 + S < mine) {
-            issue(i - 1 + S);
-            issued++;
-        }
-
-        const size_t el0 = e0 + static_cast<size_t>(blockIdx.x + i * gridDim.x) * Sh::kTile;
-        const uint32_t cnt = static_cast<uint32_t>(e1 - el0 < size_t(Sh::kTile) ? e1 - el0 : Sh::kTile);
-        const uint8_t *stage = smem + (i % S) * Sh::kStageBytes;
+        const uint32_t tile_chunk0 = static_cast<uint32_t>(e0 / kChunk) + (blockIdx.x + i * gridDim.x) * (Sh::kTile / kChunk);
+        const uint8_t *stage = smem + sidx * Sh::kStageBytes;
         const uint32_t c = tid; // chunk within the tile
-        const bool active = c * kChunk < cnt;
-        const size_t chunk = el0 / kChunk + c;
-        const size_t g = chunk / kLanesPerGroup;
+        const uint32_t chunk = tile_chunk0 + c;
+        const bool active = chunk < a.chunk_end;
+        const uint32_t g = chunk / kLanesPerGroup;
 
         // Restore and add, rank 0 first. The product q*2^e is exact, so
         // fma(q, 2^e, S) = RN(S + q*2^e): one rounding per addition.
@@ -163,14 +163,17 @@ __global__ void __launch_bounds__(kThreads)
                     fv[k] = __fadd_rn(__fmul_rn(a.beta_f, fv[k]), __fmul_rn(a.one_minus_beta_f, err[k]));
                     sv[k] = __fadd_rn(__fmul_rn(a.beta_s, sv[k]), __fmul_rn(a.one_minus_beta_s, err[k]));
                 }
-                float4 *fo = reinterpret_cast<float4 *>(a.f) + 2 * chunk;
-                float4 *so = reinterpret_cast<float4 *>(a.s) + 2 * chunk;
+                float4 *fo = reinterpret_cast<float4 *>(a.f) + 2 * static_cast<size_t>(chunk);
+                float4 *so = reinterpret_cast<float4 *>(a.s) + 2 * static_cast<size_t>(chunk);
                 fo[0] = make_float4(fv[0], fv[1], fv[2], fv[3]);
                 fo[1] = make_float4(fv[4], fv[5], fv[6], fv[7]);
                 so[0] = make_float4(sv[0], sv[1], sv[2], sv[3]);
                 so[1] = make_float4(sv[4], sv[5], sv[6], sv[7]);
             }
         }
+        __syncwarp();
+        if (lane == 0)
+            mbar_arrive(&empty[sidx]); // this warp is done reading the stage
     }
 }
 

@@ -6,13 +6,15 @@
 // Y = Q*2^E has at most three significant bits, so it is exact in bf16 and
 // in binary32: the restore adds no third rounding.
 //
-// Pipeline: a persistent CTA takes tiles of kTile elements. Thread 0
-// bulk-copies the tile's codes and scale bytes into a kInStages ring; the CTA
-// restores the tile once into one of kOutBufs output buffers in shared
-// memory; thread 0 then bulk-stores that buffer to all P rank outputs, so the
-// TMA engine, not the load/store units, moves the P-fold write stream. On one
-// GPU the P ranks share one requantised buffer, which is read from HBM once.
-// Per element of n: P*b bytes written, 17/32 bytes read.
+// Pipeline (warp-specialised, persistent): a CTA takes tiles of kTile
+// elements. A load warp bulk-copies the tile's codes and scale bytes into a
+// kInStages ring (mbarriers in_full / in_empty); eight consumer warps restore
+// the tile once into one of kOutBufs output buffers in shared memory
+// (mbarriers out_full / out_empty); a store warp bulk-stores each finished
+// buffer to all P rank outputs, so the TMA engine, not the load/store units,
+// moves the P-fold write stream, and hands the buffer back once the engine
+// has read it. On one GPU the P ranks share one requantised buffer, which is
+// read from HBM once. Per element of n: P*b bytes written, 17/32 bytes read.
 #include "echo_bulk.cuh"
 #include "echo_kernels.h"
 
@@ -21,21 +23,26 @@
 namespace echo {
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kConsumerWarps = 8;
+constexpr int kConsumers = kConsumerWarps * 32;
+constexpr int kLoadWarp = kConsumerWarps;
+constexpr int kStoreWarp = kConsumerWarps + 1;
+constexpr int kThreads = kConsumers + 64;
 
 template <bool BF16>
 struct K3Shape {
     static constexpr int kEB = BF16 ? 2 : 4;
     static constexpr int kTile = BF16 ? 4096 : 2048;
     static constexpr int kInStages = 4;
-    static constexpr int kOutBufs = 2;
+    static constexpr int kOutBufs = 3;
     static constexpr int kCodeBytes = kTile / 2;
     static constexpr int kScaleBytes = kTile / kGroup;
     static constexpr int kInBytes = kCodeBytes + kScaleBytes;
     static constexpr int kOutBytes = kTile * kEB;
     static constexpr int kOutOff = kInStages * kInBytes;
-    static constexpr int kSmem = kOutOff + kOutBufs * kOutBytes + kInStages * 8;
-    static constexpr int kChunksPerTile = kTile / kChunk;
+    static constexpr int kBarOff = kOutOff + kOutBufs * kOutBytes;
+    static constexpr int kSmem = kBarOff + (2 * kInStages + 2 * kOutBufs) * 8;
+    static constexpr int kChunksPerThread = kTile / kChunk / kConsumers;
 };
 
 __device__ __forceinline__ uint32_t round16(uint32_t x) { return (x + 15u) & ~15u; }
@@ -48,61 +55,92 @@ __global__ void __launch_bounds__(kThreads)
     constexpr int S = Sh::kInStages;
     constexpr int B = Sh::kOutBufs;
     extern __shared__ __align__(128) uint8_t smem[];
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + Sh::kOutOff + B * Sh::kOutBytes);
+    uint64_t *in_full = reinterpret_cast<uint64_t *>(smem + Sh::kBarOff);
+    uint64_t *in_empty = in_full + S;
+    uint64_t *out_full = in_empty + S;
+    uint64_t *out_empty = out_full + B;
 
     const uint32_t tid = threadIdx.x;
+    const uint32_t warp = tid >> 5;
+    const uint32_t lane = tid & 31u;
     const size_t e0 = static_cast<size_t>(a.chunk_begin) * kChunk;
     const size_t e1 = static_cast<size_t>(a.chunk_end) * kChunk;
     const uint32_t ntiles = static_cast<uint32_t>((e1 - e0 + Sh::kTile - 1) / Sh::kTile);
     const uint32_t mine = blockIdx.x < ntiles ? (ntiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+    auto tile_start = [&](uint32_t i) { return e0 + static_cast<size_t>(blockIdx.x + i * gridDim.x) * Sh::kTile; };
+    auto tile_count = [&](size_t el0) {
+        return static_cast<uint32_t>(e1 - el0 < size_t(Sh::kTile) ? e1 - el0 : Sh::kTile);
+    };
 
     if (tid == 0) {
-        for (int s = 0; s < S; s++)
-            mbar_init(&full[s], 1);
+        for (int s = 0; s < S; s++) {
+            mbar_init(&in_full[s], 1);
+            mbar_init(&in_empty[s], kConsumerWarps);
+        }
+        for (int b = 0; b < B; b++) {
+            mbar_init(&out_full[b], kConsumerWarps);
+            mbar_init(&out_empty[b], 1);
+        }
         mbar_init_fence();
     }
     __syncthreads();
 
-    auto issue = [&](uint32_t i) {
-        const size_t el0 = e0 + static_cast<size_t>(blockIdx.x + i * gridDim.x) * Sh::kTile;
-        const uint32_t cnt = static_cast<uint32_t>(e1 - el0 < size_t(Sh::kTile) ? e1 - el0 : Sh::kTile);
-        const uint32_t sc_bytes = round16(cnt / kGroup); // scale rows are padded to 16 bytes
-        uint8_t *stage = smem + (i % S) * Sh::kInBytes;
-        uint64_t *bar = &full[i % S];
-        mbar_arrive_expect_tx(bar, cnt / 2 + sc_bytes);
-        bulk_load(stage, a.qcodes + el0 / 2, cnt / 2, bar);
-        bulk_load(stage + Sh::kCodeBytes, a.qscales + el0 / kGroup, sc_bytes, bar);
-    };
+    if (warp == kLoadWarp) {
+        // scale rows are padded to 16 bytes, so a ragged tile's scale copy may
+        // round up to 16 bytes without leaving the row
+        if (lane == 0)
+            produce_tiles<S>(in_full, in_empty, mine, a.ctl.stall, a.ctl.wait_cycles, a.ctl.status,
+                             kStatusTimeoutK3, [&](uint32_t i) {
+                                 const size_t el0 = tile_start(i);
+                                 const uint32_t cnt = tile_count(el0);
+                                 const uint32_t sc_bytes = round16(cnt / kGroup);
+                                 uint8_t *stage = smem + (i % S) * Sh::kInBytes;
+                                 uint64_t *bar = &in_full[i % S];
+                                 mbar_arrive_expect_tx(bar, cnt / 2 + sc_bytes);
+                                 bulk_load(stage, a.qcodes + el0 / 2, cnt / 2, bar);
+                                 bulk_load(stage + Sh::kCodeBytes, a.qscales + el0 / kGroup, sc_bytes, bar);
+                             });
+        return;
+    }
 
-    uint32_t issued = 0; // meaningful on thread 0 only
-    if (tid == 0 && !a.ctl.stall)
-        for (; issued < mine && issued < static_cast<uint32_t>(S); issued++)
-            issue(issued);
+    if (warp == kStoreWarp) {
+        if (lane == 0) {
+            for (uint32_t i = 0; i < mine; i++) {
+                const uint32_t b = i % B;
+                if (!mbar_wait_bounded(&out_full[b], (i / B) & 1u, a.ctl.wait_cycles)) {
+                    atomicOr(a.ctl.status, kStatusTimeoutK3);
+                    break;
+                }
+                const size_t el0 = tile_start(i);
+                const uint32_t bytes = tile_count(el0) * Sh::kEB;
+                const uint8_t *buf = smem + Sh::kOutOff + b * Sh::kOutBytes;
+#pragma unroll
+                for (int r = 0; r < P; r++)
+                    bulk_store(static_cast<uint8_t *>(a.out.p[r]) + el0 * Sh::kEB, buf, bytes);
+                bulk_commit();
+                // at most B-1 younger groups still read: tile i-(B-1) is done
+                bulk_wait_read<B - 1>();
+                if (i >= static_cast<uint32_t>(B - 1))
+                    mbar_arrive(&out_empty[(i - (B - 1)) % B]);
+            }
+            bulk_wait_all();
+        }
+        return;
+    }
 
     for (uint32_t i = 0; i < mine; i++) {
-        // Output buffer i % B was last stored for tile i - B: make sure that
-        // store has finished reading it (at most B-1 younger groups pending).
-        if (tid == 0)
-            bulk_wait_read<B - 1>();
-        if (!wait_tile(&full[i % S], (i / S) & 1u, a.ctl.wait_cycles, a.ctl.status, kStatusTimeoutK3)) {
-            drain_loads(full, S, i, issued, a.ctl.wait_cycles);
-            if (tid == 0)
-                bulk_wait_all();
+        const uint32_t s = i % S;
+        const uint32_t b = i % B;
+        if (!warp_wait(&in_full[s], (i / S) & 1u, a.ctl.wait_cycles, a.ctl.status, kStatusTimeoutK3))
             return;
-        }
-        if (tid == 0 && i >= 1 && i - 1 + S < mine) {
-            issue(i - 1 + S);
-            issued++;
-        }
-
-        const size_t el0 = e0 + static_cast<size_t>(blockIdx.x + i * gridDim.x) * Sh::kTile;
-        const uint32_t cnt = static_cast<uint32_t>(e1 - el0 < size_t(Sh::kTile) ? e1 - el0 : Sh::kTile);
-        const uint8_t *stage = smem + (i % S) * Sh::kInBytes;
-        uint8_t *out = smem + Sh::kOutOff + (i % B) * Sh::kOutBytes;
-
+        if (i >= static_cast<uint32_t>(B) &&
+            !warp_wait(&out_empty[b], ((i / B) - 1) & 1u, a.ctl.wait_cycles, a.ctl.status, kStatusTimeoutK3))
+            return;
+        const uint8_t *stage = smem + s * Sh::kInBytes;
+        uint8_t *out = smem + Sh::kOutOff + b * Sh::kOutBytes;
 #pragma unroll
-        for (int j = 0; j < Sh::kChunksPerTile / kThreads; j++) {
-            const uint32_t c = tid + j * kThreads;
+        for (int j = 0; j < Sh::kChunksPerThread; j++) {
+            const uint32_t c = tid + j * kConsumers;
             const uint32_t w = reinterpret_cast<const uint32_t *>(stage)[c];
             const float st = step_of(stage[Sh::kCodeBytes + c / kLanesPerGroup]);
             const Unpacked u = unpack8(w);
@@ -118,16 +156,12 @@ __global__ void __launch_bounds__(kThreads)
             }
         }
         fence_proxy_async_smem(); // the restored tile is read next by the bulk stores
-        __syncthreads();
-        if (tid == 0) {
-#pragma unroll
-            for (int r = 0; r < P; r++)
-                bulk_store(static_cast<uint8_t *>(a.out.p[r]) + el0 * Sh::kEB, out, cnt * Sh::kEB);
-            bulk_commit();
+        __syncwarp();
+        if (lane == 0) {
+            mbar_arrive(&in_empty[s]);
+            mbar_arrive(&out_full[b]);
         }
     }
-    if (tid == 0)
-        bulk_wait_all();
 }
 
 template <int P, bool BF16>
