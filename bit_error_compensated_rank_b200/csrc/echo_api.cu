@@ -404,6 +404,8 @@ int persistent_grid(uint32_t tiles, int resident_per_sm)
     return g < 1 ? 1 : static_cast<int>(g);
 }
 
+int record_error(int code, const char *message) { return set_error(code, "%s", message); }
+
 cudaError_t prepare_kernel(const void *kernel, int threads, int smem_bytes, int *resident)
 {
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);

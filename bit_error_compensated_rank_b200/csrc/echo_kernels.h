@@ -77,4 +77,8 @@ int persistent_grid(uint32_t tiles, int resident_per_sm);
 // (cached by the caller per instantiation).
 cudaError_t prepare_kernel(const void *kernel, int threads, int smem_bytes, int *resident);
 
+// Record `message` as this thread's last error (echo_last_error /
+// echo_last_status) and return `code`.
+int record_error(int code, const char *message);
+
 } // namespace echo

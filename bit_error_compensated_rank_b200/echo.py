@@ -35,6 +35,7 @@ EXPORTED = (
     "echo_get_state", "echo_set_state", "echo_get_state_range", "echo_get_wire",
     "echo_get_wire_range", "echo_stats", "echo_model_bytes", "echo_set_timing",
     "echo_last_kernel_ms", "echo_kernel_ms_total", "echo_device_status",
+    "echo_allreduce_static",
 )
 
 _vp = ctypes.c_void_p
@@ -73,6 +74,8 @@ def _load():
         "echo_last_kernel_ms": (_int, [_vp, _f32p]),
         "echo_kernel_ms_total": (_int, [_vp, ctypes.POINTER(ctypes.c_double), _u64p]),
         "echo_device_status": (_int, [_vp, ctypes.POINTER(ctypes.c_int), _int]),
+        "echo_allreduce_static": (_int, [_int, _sz, _int, _vpp, _vp, _vp, ctypes.c_float, ctypes.c_float,
+                                         ctypes.c_float, _int, _vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -130,6 +133,15 @@ def echo_allreduce_out(h: int, send_ptrs, recv_ptrs, phase: int = ECHO_FWD, stre
 def echo_allreduce_host(h: int, host_send_ptrs, host_recv_ptr: int, phase: int = ECHO_FWD,
                         stream: int = 0) -> None:
     _check(_lib.echo_allreduce_host(h, _ptr_array(host_send_ptrs), host_recv_ptr, phase, stream))
+
+
+def echo_allreduce_static(P: int, n: int, dtype: int, rank_ptrs, f_ptr: int, s_ptr: int,
+                          beta_fast: float = 0.5, beta_slow: float = 0.875, lam: float = 0.5,
+                          enable: bool = True, stream: int = 0) -> None:
+    """The all-reduce without device allocation (see include/echo.h): the
+    caller passes the rank buffers and this phase's state arrays f, s."""
+    _check(_lib.echo_allreduce_static(P, n, dtype, _ptr_array(rank_ptrs), f_ptr, s_ptr, beta_fast,
+                                      beta_slow, lam, int(bool(enable)), stream))
 
 
 def echo_reset(h: int, phase_mask: int = 3) -> None:

@@ -117,6 +117,35 @@ ECHO_API int echo_allreduce_out(echo_handle *h, const void *const send_ptrs[],
 ECHO_API int echo_allreduce_host(echo_handle *h, const void *const host_send[], void *host_recv,
                         int phase, void *stream);
 
+/*
+ * echo_allreduce_static - the in-place all-reduce of echo_allreduce for
+ * callers that cannot allocate device memory (the paper has no counterpart:
+ * this is a deployment variant of the same computation). Typical callers are
+ * a serving process that reserved all of HBM for its own pool at start-up, a
+ * plugin running inside a host application that owns every allocation, and a
+ * latency-critical path where a cudaMalloc, which can synchronise the device,
+ * is not acceptable. It allocates nothing: no cudaMalloc, no cudaFree, no
+ * allocating library call.
+ *   rank_ptrs  P device pointers, n elements of dtype each, as for
+ *              echo_allreduce (read, then overwritten with the result).
+ *   f, s       the caller's compensator state for this phase: n binary32 each,
+ *              device memory, read and updated in place (ignored, and may be
+ *              NULL, when enable == 0). Zero them before the first call.
+ *   beta_fast, beta_slow, lambda, enable   as for echo_set_params.
+ * The wire buffers the kernels exchange live in one array compiled into the
+ * library, ECHO_STATIC_SCRATCH_BYTES (32 MiB) on every GPU that loads it,
+ * kept until the process exits. A call needs about (P+1)*17/32 bytes per
+ * element of n (at P = 8, n up to about 7 million elements); larger sizes are
+ * rejected with ECHO_ERR_UNSUPPORTED and nothing is enqueued. The first call
+ * on a device looks up the array's device address (cudaGetSymbolAddress) with
+ * that device current; make that first call before any stream capture. All
+ * calls share the array and it keeps the last call's contents; calls whose
+ * work overlaps on the GPU (other streams or threads at once) race on it.
+ */
+#define ECHO_STATIC_SCRATCH_BYTES (32u * 1024u * 1024u)
+ECHO_API int echo_allreduce_static(int P, size_t n, int dtype, void *const rank_ptrs[], float *f, float *s,
+                                   float beta_fast, float beta_slow, float lambda, int enable, void *stream);
+
 /* echo_reset - zero the compensator state of the phases in phase_mask
  * (bit 0 forward, bit 1 backward), enqueued on the legacy default stream and
  * completed before return. */
