@@ -13,6 +13,37 @@
 
 #include "echo_codec.cuh"
 
+// Pipeline shapes, chosen by sweeping on B200 at P = 8, 1 GiB per rank
+// (larger bulk copies win as long as two CTAs fit on an SM).
+// ECHO_K1_TILE is kernel 1's tile length in elements when a tile of all P
+// partials is at most 16 bytes per element (halved, quartered beyond).
+// ECHO_K2_CHUNKS is kernel 2's chunks of 8 elements per consumer thread per
+// tile, reduced for large P so that ECHO_K2_STAGES stages fit in shared
+// memory. ECHO_K3_TILE is kernel 3's bf16 tile (halved for binary32).
+#ifndef ECHO_K1_TILE
+#define ECHO_K1_TILE 2048
+#endif
+#ifndef ECHO_K1_STAGES
+#define ECHO_K1_STAGES 2
+#endif
+#ifndef ECHO_K2_STAGES
+#define ECHO_K2_STAGES 2
+#endif
+#ifndef ECHO_K2_CHUNKS
+#define ECHO_K2_CHUNKS 4
+#endif
+#ifndef ECHO_K3_TILE
+#define ECHO_K3_TILE 16384
+#endif
+#ifndef ECHO_K3_IN_STAGES
+#define ECHO_K3_IN_STAGES 4
+#endif
+#ifndef ECHO_K3_OUT_BUFS
+#define ECHO_K3_OUT_BUFS 2
+#endif
+// Shared memory one CTA may use (the B200 limit is 227 KB).
+#define ECHO_SMEM_BUDGET (225 * 1024)
+
 namespace echo {
 
 // Pipeline controls shared by the three kernels.

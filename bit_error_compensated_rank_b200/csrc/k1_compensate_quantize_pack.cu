@@ -37,11 +37,12 @@ template <int P, bool BF16, bool COMP>
 struct K1Shape {
     static constexpr int kEB = BF16 ? 2 : 4;
     // Tile length keeps one stage near 12-24 KB whatever P and the dtype.
-    static constexpr int kTile = (P * kEB <= 16) ? 1024 : (P * kEB <= 32 ? 512 : 256);
-    static constexpr int kStages = 3;
+    static constexpr int kTile = (P * kEB <= 16) ? ECHO_K1_TILE : (P * kEB <= 32 ? ECHO_K1_TILE / 2 : ECHO_K1_TILE / 4);
+    static constexpr int kStages = ECHO_K1_STAGES;
     static constexpr int kXBytes = kTile * kEB; // one rank's partial tile
     static constexpr int kStageBytes = P * kXBytes + (COMP ? 2 * kTile * 4 : 0);
     static constexpr int kSmem = kStages * kStageBytes + 2 * kStages * 8;
+    static_assert(kSmem <= ECHO_SMEM_BUDGET, "kernel 1 stages exceed shared memory");
     static constexpr int kChunksPerTile = kTile / kChunk; // a multiple of 32
 };
 

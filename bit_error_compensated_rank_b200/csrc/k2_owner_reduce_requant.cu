@@ -36,15 +36,34 @@ constexpr int kConsumerWarps = 8;
 constexpr int kConsumers = kConsumerWarps * 32;
 constexpr int kThreads = kConsumers + 32; // + one producer warp
 
+// Bytes of one stage for `chunks` chunks per consumer thread: P code tiles,
+// P scale tiles, and the f, s tiles.
+constexpr int k2_stage_bytes(int P, bool comp, int chunks)
+{
+    return P * (kConsumers * kChunk * chunks / 2 + kConsumers * kChunk * chunks / kGroup) +
+           (comp ? 2 * kConsumers * kChunk * chunks * 4 : 0);
+}
+
+// The largest of ECHO_K2_CHUNKS, /2, /4 whose stages fit the budget.
+constexpr int k2_chunks(int P, bool comp)
+{
+    int c = ECHO_K2_CHUNKS;
+    while (c > 1 && ECHO_K2_STAGES * k2_stage_bytes(P, comp, c) + 64 > ECHO_SMEM_BUDGET)
+        c /= 2;
+    return c;
+}
+
 template <int P, bool COMP>
 struct K2Shape {
-    static constexpr int kTile = kConsumers * kChunk;   // 2048: one chunk per consumer thread
-    static constexpr int kStages = 3;
-    static constexpr int kCodeBytes = kTile / 2;         // one rank's code tile
-    static constexpr int kScaleBytes = kTile / kGroup;   // one rank's scale tile (64)
+    static constexpr int kChunks = k2_chunks(P, COMP);    // chunks per consumer thread
+    static constexpr int kTile = kConsumers * kChunk * kChunks;
+    static constexpr int kStages = ECHO_K2_STAGES;
+    static constexpr int kCodeBytes = kTile / 2;          // one rank's code tile
+    static constexpr int kScaleBytes = kTile / kGroup;    // one rank's scale tile
     static constexpr int kStateOff = P * (kCodeBytes + kScaleBytes);
     static constexpr int kStageBytes = kStateOff + (COMP ? 2 * kTile * 4 : 0);
     static constexpr int kSmem = kStages * kStageBytes + 2 * kStages * 8;
+    static_assert(kSmem <= ECHO_SMEM_BUDGET, "kernel 2 stages exceed shared memory");
 };
 
 __device__ __forceinline__ uint32_t round16(uint32_t x) { return (x + 15u) & ~15u; }
@@ -109,7 +128,9 @@ __global__ void __launch_bounds__(kThreads)
             return;
         const uint32_t tile_chunk0 = static_cast<uint32_t>(e0 / kChunk) + (blockIdx.x + i * gridDim.x) * (Sh::kTile / kChunk);
         const uint8_t *stage = smem + sidx * Sh::kStageBytes;
-        const uint32_t c = tid; // chunk within the tile
+#pragma unroll 1
+        for (int j = 0; j < Sh::kChunks; j++) {
+        const uint32_t c = tid + j * kConsumers; // chunk within the tile
         const uint32_t chunk = tile_chunk0 + c;
         const bool active = chunk < a.chunk_end;
         const uint32_t g = chunk / kLanesPerGroup;
@@ -170,6 +191,7 @@ __global__ void __launch_bounds__(kThreads)
                 so[0] = make_float4(sv[0], sv[1], sv[2], sv[3]);
                 so[1] = make_float4(sv[4], sv[5], sv[6], sv[7]);
             }
+        }
         }
         __syncwarp();
         if (lane == 0)

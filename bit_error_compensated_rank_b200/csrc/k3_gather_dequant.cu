@@ -32,9 +32,9 @@ constexpr int kThreads = kConsumers + 64;
 template <bool BF16>
 struct K3Shape {
     static constexpr int kEB = BF16 ? 2 : 4;
-    static constexpr int kTile = BF16 ? 4096 : 2048;
-    static constexpr int kInStages = 4;
-    static constexpr int kOutBufs = 3;
+    static constexpr int kTile = BF16 ? ECHO_K3_TILE : ECHO_K3_TILE / 2;
+    static constexpr int kInStages = ECHO_K3_IN_STAGES;
+    static constexpr int kOutBufs = ECHO_K3_OUT_BUFS;
     static constexpr int kCodeBytes = kTile / 2;
     static constexpr int kScaleBytes = kTile / kGroup;
     static constexpr int kInBytes = kCodeBytes + kScaleBytes;
@@ -42,6 +42,7 @@ struct K3Shape {
     static constexpr int kOutOff = kInStages * kInBytes;
     static constexpr int kBarOff = kOutOff + kOutBufs * kOutBytes;
     static constexpr int kSmem = kBarOff + (2 * kInStages + 2 * kOutBufs) * 8;
+    static_assert(kSmem <= ECHO_SMEM_BUDGET, "kernel 3 buffers exceed shared memory");
     static constexpr int kChunksPerThread = kTile / kChunk / kConsumers;
 };
 
