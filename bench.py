@@ -243,9 +243,12 @@ def run_reference(args, rank: int, world: int) -> dict | None:
 # the CUDA path
 # ---------------------------------------------------------------------------
 # DRAM traffic per element of n for each kernel from one ncu capture
-# (dram__bytes_read.sum + dram__bytes_write.sum / n); reported only while the
-# kernel source still has the hash it had when captured.
-NCU_TRAFFIC = {}
+# ((dram__bytes_read.sum + dram__bytes_write.sum) / n, captured at P = 8,
+# n = 2^26 and scaled by n, since the traffic grows in proportion); reported
+# only while the kernel source still has the hash it had when captured.
+NCU_TRAFFIC = {
+    "k1_compensate_quantize_pack": {"bytes_per_elem": 28.08, "source_sha": "e04244497494004a"},
+}
 
 
 def _source_hash(path: str) -> str:
