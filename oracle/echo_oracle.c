@@ -130,19 +130,24 @@ static int store_output(void *out, int dtype, size_t idx, float v)
     return 0;
 }
 
-int echo_oracle_allreduce_groups(int P, int G, size_t ngroups,
-                                 const int32_t *owner, int dtype,
-                                 const void *x, void *out, float *f, float *s,
-                                 float lambda, float beta_f, float beta_s,
-                                 int enable, uint8_t *codes1, uint8_t *scales1,
-                                 uint8_t *qcodes, uint8_t *qscales,
-                                 float *c_out, float *err_out)
+int echo_oracle_allreduce_groups_ex(int P, int G, size_t ngroups,
+                                    const int32_t *owner, int dtype,
+                                    const void *x, void *out, float *f, float *s,
+                                    float *eps, float lambda, float beta_f,
+                                    float beta_s, int enable, int variant,
+                                    uint8_t *codes1, uint8_t *scales1,
+                                    uint8_t *qcodes, uint8_t *qscales,
+                                    float *c_out, float *err_out)
 {
+    const int owner_sum = (variant & ECHO_ORACLE_OWNER_SUM) != 0;
+    const int sender_ef = (variant & ECHO_ORACLE_SENDER_EF) != 0;
     if (P < 2 || P > 16 || G < 2 || (G % 2) != 0 || ngroups == 0)
         return -1;
     if (dtype != ECHO_ORACLE_BF16 && dtype != ECHO_ORACLE_FP32)
         return -1;
-    if (!owner || !x || !out || (enable && (!f || !s)))
+    if (variant & ~(ECHO_ORACLE_OWNER_SUM | ECHO_ORACLE_SENDER_EF))
+        return -1;
+    if (!owner || !x || !out || (enable && (!f || !s)) || (sender_ef && !eps))
         return -1;
     for (size_t g = 0; g < ngroups; g++)
         if (owner[g] < 0 || owner[g] >= P)
@@ -186,10 +191,15 @@ int echo_oracle_allreduce_groups(int P, int G, size_t ngroups,
                     rc = -1;
                     goto done;
                 }
-                if (enable && owner[g] == r)
-                    v[k] = xi + c[i];
+                /* Variant: the rank first adds back its own rounding-#1 error
+                 * of its previous call. */
+                float u = xi;
+                if (sender_ef)
+                    u = xi + eps[(size_t)r * m + i];
+                if (enable && !owner_sum && owner[g] == r)
+                    v[k] = u + c[i];
                 else
-                    v[k] = xi;
+                    v[k] = u;
             }
             int b = echo_oracle_quantize_group(v, G, q1 + (size_t)r * m + g * (size_t)G);
             if (b < 0) {
@@ -197,6 +207,14 @@ int echo_oracle_allreduce_groups(int P, int G, size_t ngroups,
                 goto done;
             }
             b1[(size_t)r * ngroups + g] = b;
+            /* Variant: keep this rounding's error for the rank's next call
+             * (exact in binary32, as for rounding #2). */
+            if (sender_ef)
+                for (int k = 0; k < G; k++) {
+                    size_t i = g * (size_t)G + (size_t)k;
+                    float restored = echo_oracle_dequant(q1[(size_t)r * m + i], b);
+                    eps[(size_t)r * m + i] = v[k] - restored;
+                }
         }
     }
 
@@ -211,6 +229,10 @@ int echo_oracle_allreduce_groups(int P, int G, size_t ngroups,
                 float d = echo_oracle_dequant(q1[(size_t)r * m + i], b1[(size_t)r * ngroups + g]);
                 sum = sum + d;
             }
+            /* Variant: the owner folds the correction into its sum, after
+             * the P ranks, instead of the sender adding it to its partial. */
+            if (enable && owner_sum)
+                sum = sum + c[i];
             S[k] = sum;
         }
         /* Step 4: rounding #2 of the total. */
@@ -268,11 +290,24 @@ done:
     return rc;
 }
 
-int echo_oracle_allreduce(int P, size_t n, int G, int dtype, const void *x,
-                          void *out, float *f, float *s, float lambda,
-                          float beta_f, float beta_s, int enable,
-                          uint8_t *codes1, uint8_t *scales1, uint8_t *qcodes,
-                          uint8_t *qscales, float *c_out, float *err_out)
+int echo_oracle_allreduce_groups(int P, int G, size_t ngroups,
+                                 const int32_t *owner, int dtype,
+                                 const void *x, void *out, float *f, float *s,
+                                 float lambda, float beta_f, float beta_s,
+                                 int enable, uint8_t *codes1, uint8_t *scales1,
+                                 uint8_t *qcodes, uint8_t *qscales,
+                                 float *c_out, float *err_out)
+{
+    return echo_oracle_allreduce_groups_ex(P, G, ngroups, owner, dtype, x, out, f, s, NULL,
+                                           lambda, beta_f, beta_s, enable, 0, codes1,
+                                           scales1, qcodes, qscales, c_out, err_out);
+}
+
+int echo_oracle_allreduce_ex(int P, size_t n, int G, int dtype, const void *x,
+                             void *out, float *f, float *s, float *eps, float lambda,
+                             float beta_f, float beta_s, int enable, int variant,
+                             uint8_t *codes1, uint8_t *scales1, uint8_t *qcodes,
+                             uint8_t *qscales, float *c_out, float *err_out)
 {
     if (P < 2 || G < 2 || n == 0 || n % ((size_t)P * (size_t)G) != 0)
         return -1;
@@ -283,9 +318,20 @@ int echo_oracle_allreduce(int P, size_t n, int G, int dtype, const void *x,
         return -1;
     for (size_t g = 0; g < ngroups; g++)
         owner[g] = (int32_t)((g * (size_t)G) / seg);
-    int rc = echo_oracle_allreduce_groups(P, G, ngroups, owner, dtype, x, out, f, s,
-                                          lambda, beta_f, beta_s, enable, codes1,
-                                          scales1, qcodes, qscales, c_out, err_out);
+    int rc = echo_oracle_allreduce_groups_ex(P, G, ngroups, owner, dtype, x, out, f, s, eps,
+                                             lambda, beta_f, beta_s, enable, variant, codes1,
+                                             scales1, qcodes, qscales, c_out, err_out);
     free(owner);
     return rc;
+}
+
+int echo_oracle_allreduce(int P, size_t n, int G, int dtype, const void *x,
+                          void *out, float *f, float *s, float lambda,
+                          float beta_f, float beta_s, int enable,
+                          uint8_t *codes1, uint8_t *scales1, uint8_t *qcodes,
+                          uint8_t *qscales, float *c_out, float *err_out)
+{
+    return echo_oracle_allreduce_ex(P, n, G, dtype, x, out, f, s, NULL, lambda, beta_f,
+                                    beta_s, enable, 0, codes1, scales1, qcodes, qscales,
+                                    c_out, err_out);
 }

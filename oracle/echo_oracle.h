@@ -54,6 +54,17 @@ extern "C" {
 #define ECHO_ORACLE_BF16 0
 #define ECHO_ORACLE_FP32 1
 
+/* Variants (bits of `variant` in the _ex calls; 0 is the method above):
+ *   ECHO_ORACLE_OWNER_SUM  the owner adds the correction c to its binary32
+ *                          sum, after the P restored values, instead of the
+ *                          sender adding it to its partial before rounding #1;
+ *   ECHO_ORACLE_SENDER_EF  every rank keeps its own rounding-#1 error
+ *                          eps = v - q*2^e per element (exact) and adds it to
+ *                          its partial in its next call, before the owner's
+ *                          correction: v = RN(RN(x + eps) + c). */
+#define ECHO_ORACLE_OWNER_SUM 1
+#define ECHO_ORACLE_SENDER_EF 2
+
 /* Scale choice and rounding of one group (rounding #1 at a sender, #2 at the
  * owner). v: G binary32 values. Writes G codes to q. Returns the scale byte
  * e+127 (0..253), or -1 for a non-finite value, -2 past the domain. */
@@ -88,6 +99,17 @@ int echo_oracle_allreduce_groups(int P, int G, size_t ngroups,
                                  uint8_t *qcodes, uint8_t *qscales,
                                  float *c_out, float *err_out);
 
+/* The same with a variant (see above); eps [P][m] is every rank's
+ * rounding-#1 error state, read and updated when ECHO_ORACLE_SENDER_EF. */
+int echo_oracle_allreduce_groups_ex(int P, int G, size_t ngroups,
+                                    const int32_t *owner, int dtype,
+                                    const void *x, void *out, float *f, float *s,
+                                    float *eps, float lambda, float beta_f,
+                                    float beta_s, int enable, int variant,
+                                    uint8_t *codes1, uint8_t *scales1,
+                                    uint8_t *qcodes, uint8_t *qscales,
+                                    float *c_out, float *err_out);
+
 /* Same call over n elements per rank with contiguous segments: rank r owns
  * elements [r*n/P, (r+1)*n/P). Requires n % (P*G) == 0. */
 int echo_oracle_allreduce(int P, size_t n, int G, int dtype, const void *x,
@@ -95,6 +117,12 @@ int echo_oracle_allreduce(int P, size_t n, int G, int dtype, const void *x,
                           float beta_f, float beta_s, int enable,
                           uint8_t *codes1, uint8_t *scales1, uint8_t *qcodes,
                           uint8_t *qscales, float *c_out, float *err_out);
+
+int echo_oracle_allreduce_ex(int P, size_t n, int G, int dtype, const void *x,
+                             void *out, float *f, float *s, float *eps, float lambda,
+                             float beta_f, float beta_s, int enable, int variant,
+                             uint8_t *codes1, uint8_t *scales1, uint8_t *qcodes,
+                             uint8_t *qscales, float *c_out, float *err_out);
 
 #ifdef __cplusplus
 }

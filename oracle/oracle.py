@@ -22,6 +22,8 @@ LIB_NAME = "libecho_oracle.so"
 
 BF16 = 0
 FP32 = 1
+OWNER_SUM = 1   # variant: the owner adds the correction to its sum
+SENDER_EF = 2   # variant: every rank feeds back its own rounding-#1 error
 
 _u8p = ctypes.POINTER(ctypes.c_uint8)
 _i8p = ctypes.POINTER(ctypes.c_int8)
@@ -77,6 +79,15 @@ class Oracle:
         lib.echo_oracle_allreduce.argtypes = (
             [ctypes.c_int, ctypes.c_size_t, ctypes.c_int, ctypes.c_int] + common)
         lib.echo_oracle_allreduce.restype = ctypes.c_int
+        common_ex = [ctypes.c_void_p, ctypes.c_void_p, _f32p, _f32p, _f32p,
+                     ctypes.c_float, ctypes.c_float, ctypes.c_float, ctypes.c_int, ctypes.c_int,
+                     _u8p, _u8p, _u8p, _u8p, _f32p, _f32p]
+        lib.echo_oracle_allreduce_groups_ex.argtypes = (
+            [ctypes.c_int, ctypes.c_int, ctypes.c_size_t, _i32p, ctypes.c_int] + common_ex)
+        lib.echo_oracle_allreduce_groups_ex.restype = ctypes.c_int
+        lib.echo_oracle_allreduce_ex.argtypes = (
+            [ctypes.c_int, ctypes.c_size_t, ctypes.c_int, ctypes.c_int] + common_ex)
+        lib.echo_oracle_allreduce_ex.restype = ctypes.c_int
         self.lib = lib
 
     # ---- codec -----------------------------------------------------------
@@ -105,13 +116,17 @@ class Oracle:
 
     # ---- one all-reduce call ---------------------------------------------
     def allreduce(self, x, f=None, s=None, params: Params = Params(), G: int = 32,
-                  owner=None, want_wire: bool = True, want_diag: bool = False) -> dict:
+                  owner=None, want_wire: bool = True, want_diag: bool = False,
+                  variant: int = 0, eps=None) -> dict:
         """One call on rank partials ``x`` of shape (P, m).
 
         ``x`` is uint16 (bf16 bit patterns) or float32. ``f`` and ``s`` (float32,
         length m) are updated in place when compensation is on. ``owner`` (one
         rank per group) overrides the contiguous segment layout; it lets a
         caller run any subset of groups of a larger problem.
+        ``variant`` is a bit set of OWNER_SUM and SENDER_EF; with SENDER_EF,
+        ``eps`` (float32, shape (P, m)) is every rank's rounding-#1 error state,
+        updated in place.
         Returns a dict with ``out`` and, if requested, the wire and diagnostics.
         """
         x = np.ascontiguousarray(x)
@@ -131,6 +146,10 @@ class Oracle:
             for a in (f, s):
                 if a.dtype != np.float32 or a.shape != (m,) or not a.flags.c_contiguous:
                     raise ValueError("f and s must be contiguous float32 of length m")
+        if variant & SENDER_EF:
+            if eps is None or eps.dtype != np.float32 or eps.shape != (P, m) or \
+                    not eps.flags.c_contiguous:
+                raise ValueError("SENDER_EF needs eps: contiguous float32 of shape (P, m)")
         out = np.zeros(m, dtype=x.dtype)
         res = {"out": out}
         if want_wire:
@@ -142,20 +161,22 @@ class Oracle:
             res["c"] = np.zeros(m, dtype=np.float32)
             res["err"] = np.zeros(m, dtype=np.float32)
         args = [x.ctypes.data, out.ctypes.data, _ptr(f, _f32p), _ptr(s, _f32p),
+                _ptr(eps if variant & SENDER_EF else None, _f32p),
                 params.lam, params.beta_fast, params.beta_slow, int(bool(params.enable)),
+                int(variant),
                 _ptr(res.get("codes1"), _u8p), _ptr(res.get("scales1"), _u8p),
                 _ptr(res.get("qcodes"), _u8p), _ptr(res.get("qscales"), _u8p),
                 _ptr(res.get("c"), _f32p), _ptr(res.get("err"), _f32p)]
         if owner is None:
             if m % (P * G):
                 raise ValueError("contiguous segments need m % (P*G) == 0")
-            rc = self.lib.echo_oracle_allreduce(P, m, G, dtype, *args)
+            rc = self.lib.echo_oracle_allreduce_ex(P, m, G, dtype, *args)
         else:
             owner = np.ascontiguousarray(owner, dtype=np.int32)
             if owner.shape != (ngroups,):
                 raise ValueError("owner needs one rank per group")
-            rc = self.lib.echo_oracle_allreduce_groups(P, G, ngroups, _ptr(owner, _i32p),
-                                                       dtype, *args)
+            rc = self.lib.echo_oracle_allreduce_groups_ex(P, G, ngroups, _ptr(owner, _i32p),
+                                                          dtype, *args)
         if rc != 0:
             raise ValueError(f"oracle allreduce failed ({rc})")
         return res

@@ -31,7 +31,7 @@ import numpy as np
 
 from bit_error_compensated_rank_b200.workloads import bf16_bits, bf16_to_f32, gaussian, rng
 from bruteforce import bf_quantize, value_of
-from oracle.oracle import Params
+from oracle.oracle import OWNER_SUM, SENDER_EF, Params
 
 GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
 F32 = np.float32
@@ -167,11 +167,8 @@ def pin_pack_layout(orc):
 # ---------------------------------------------------------------------------
 # whole calls
 # ---------------------------------------------------------------------------
-def pin_hand_example(orc):
-    """Four calls of the hand-worked example (fixture
-    ``hand_example_p2_g32.json``): every wire byte, output, correction, error
-    and state value, for bf16 and binary32 inputs."""
-    fx = _load("hand_example_p2_g32.json")
+def _check_hand_fixture(orc, name, variant):
+    fx = _load(name)
     n = fx["n"]
     prm = Params(lam=float(Fraction(fx["params"]["lambda"])),
                  beta_fast=float(Fraction(fx["params"]["beta_fast"])),
@@ -183,7 +180,7 @@ def pin_hand_example(orc):
         f = np.zeros(n, F32)
         s = np.zeros(n, F32)
         for call in fx["calls"]:
-            res = orc.allreduce(x, f, s, prm, want_diag=True)
+            res = orc.allreduce(x, f, s, prm, want_diag=True, variant=variant)
             for key in ("c", "err", "f", "s", "out"):
                 want = [Fraction(t) for t in call[key]] + [Fraction(0)] * (n - 4)
                 have = {"c": res["c"], "err": res["err"], "f": f, "s": s,
@@ -196,6 +193,13 @@ def pin_hand_example(orc):
             assert res["qcodes"][:2].tolist() == call["qcodes"]
             assert not res["qcodes"][2:].any()
             assert res["qscales"].tolist() == call["qscales"]
+
+
+def pin_hand_example(orc):
+    """Four calls of the hand-worked example (fixture
+    ``hand_example_p2_g32.json``): every wire byte, output, correction, error
+    and state value, for bf16 and binary32 inputs."""
+    _check_hand_fixture(orc, "hand_example_p2_g32.json", 0)
 
 
 def _grid_partials(P, ngroups, G, seed):
@@ -449,6 +453,143 @@ def pin_power_of_two_equivariance(orc):
                 assert (b["qscales"][nzq].astype(int) == a["qscales"][nzq].astype(int) + t).all()
 
 
+# ---------------------------------------------------------------------------
+# variants: the correction folded into the owner's sum; sender-side feedback
+# ---------------------------------------------------------------------------
+def pin_owner_sum_hand_example(orc):
+    """Three calls of the hand-worked owner-sum example (fixture
+    ``hand_example_owner_sum_p2_g32.json``): the senders' wire never changes,
+    the correction enters the owner's sum exactly."""
+    _check_hand_fixture(orc, "hand_example_owner_sum_p2_g32.json", OWNER_SUM)
+
+
+def pin_owner_sum_injection(orc):
+    """Owner-sum variant: zero partials and f = s = 3/4. No sender adds
+    anything (all stage-1 codes and scale bytes are 0); the owner's sum is
+    exactly 3/4 everywhere, so every rank receives 3/4 with err = 0."""
+    G, P = 32, 4
+    m = P * G * 2
+    f = np.full(m, 0.75, F32)
+    s = np.full(m, 0.75, F32)
+    res = orc.allreduce(np.zeros((P, m), np.uint16), f, s, Params(), want_diag=True,
+                        variant=OWNER_SUM)
+    assert not res["codes1"].any() and not res["scales1"].any()
+    assert (bf16_to_f32(res["out"]) == F32(0.75)).all()
+    assert (res["qscales"] == 124).all() and (res["err"] == 0).all()
+    assert (f == F32(0.375)).all() and (s == F32(0.65625)).all()
+
+
+def pin_owner_sum_order(orc):
+    """Owner-sum variant: the correction is added after the P restored values.
+    Ranks send 2^24 and -2^24 (exact) and c = 1: (2^24 - 2^24) + 1 = 1,
+    whereas starting the sum from c would give (1 + 2^24) -> 2^24, then 0."""
+    G, P = 32, 2
+    m = P * G
+    x = np.zeros((P, m), F32)
+    x[0, 0] = 2.0 ** 24
+    x[1, 0] = -(2.0 ** 24)
+    f = np.ones(m, F32)
+    s = np.ones(m, F32)
+    res = orc.allreduce(x, f, s, Params(), want_diag=True, variant=OWNER_SUM)
+    assert float(res["out"][0]) == 1.0 and float(res["err"][0]) == 0.0
+    assert (res["out"][1:G] == 1.0).all()
+
+
+def pin_owner_sum_error_feedback(orc):
+    """Owner-sum variant with lambda = 1, beta_fast = 0 (textbook error
+    feedback): c_k = err_{k-1} exactly and D_K = -err_{K-1} exactly."""
+    P, G = 4, 32
+    m = P * G * 4
+    f = np.zeros(m, F32)
+    s = np.zeros(m, F32)
+    prm = Params(lam=1.0, beta_fast=0.0, beta_slow=0.875)
+    cs, errs = [], []
+    for k in range(10):
+        res = orc.allreduce(gaussian(P, m, seed=15, call=k), f, s, prm, want_diag=True,
+                            variant=OWNER_SUM)
+        cs.append(res["c"].astype(np.float64))
+        errs.append(res["err"].astype(np.float64))
+    for k in range(1, len(cs)):
+        assert (cs[k] == errs[k - 1]).all()
+    for i in range(0, m, 11):
+        assert math.fsum([cs[k][i] - errs[k][i] for k in range(len(cs))]) == -errs[-1][i]
+
+
+def pin_sender_ef_on_grid(orc):
+    """Sender feedback on partials already on their 4-bit grid: rounding #1
+    is exact, so every rank's stored error stays exactly 0 and the results
+    equal those without the feedback."""
+    G = 32
+    for P in (2, 5, 8):
+        ngroups = 2 * P
+        m = ngroups * G
+        x32, _, _ = _grid_partials(P, ngroups, G, seed=40 + P)
+        eps = np.zeros((P, m), F32)
+        a = orc.allreduce(x32, params=Params(enable=False), want_diag=True, variant=SENDER_EF,
+                          eps=eps)
+        b = orc.allreduce(x32, params=Params(enable=False), want_diag=True)
+        assert not eps.any()
+        assert (a["out"] == b["out"]).all() and (a["codes1"] == b["codes1"]).all()
+
+
+def pin_sender_ef_per_rank(orc):
+    """Each rank keeps its own error: only the rank whose partial is off its
+    grid gets a non-zero error, equal to v - q*2^e exactly, at most half a
+    step; the next call adds it to that rank's partial only."""
+    G, P = 32, 4
+    m = P * G
+    x = np.zeros((P, m), F32)
+    x[:, 0] = 7.0          # every group's maximum: scale 2^0 on every rank
+    x[2, 1] = 0.3          # rank 2, element 1: rounds to 0, error 0.3
+    x[1, 2] = 2.0          # on the grid
+    eps = np.zeros((P, m), F32)
+    orc.allreduce(x, params=Params(enable=False), variant=SENDER_EF, eps=eps)
+    assert eps[2, 1] == F32(0.3)
+    eps_rest = eps.copy()
+    eps_rest[2, 1] = 0
+    assert not eps_rest.any()
+    # next call: rank 2 forms 0.3 + 0.3 = 0.6 (binary32), rounds to 1, error -0.4
+    res = orc.allreduce(x, params=Params(enable=False), variant=SENDER_EF, eps=eps)
+    assert eps[2, 1] == F32(F32(0.3) + F32(0.3)) - F32(1.0)
+    assert _unpack_ref(res["codes1"][2][:1])[1] == 1
+    eps_rest = eps.copy()
+    eps_rest[2, 1] = 0
+    assert not eps_rest.any()
+
+
+def pin_full_compensation_bounded(orc):
+    """With both roundings fed back (sender feedback, and the owner's
+    correction either at the sender or in the sum) the total injected error
+    telescopes: T_K = sum_k (Y_k - sum_r x_rk) = D_K - sum_r eps_r,K-1 + R_K,
+    |D_K| <= 5 max|err| (closed form), R_K the binary32 rounding of the sums
+    (at most ulp-sized per term). So T_K stays bounded however many calls, while
+    with the owner's correction alone it grows like sqrt(K) (stage-1 errors)."""
+    P, G, K = 4, 32, 96
+    m = P * G * 8
+    rms = {}
+    for variant in (SENDER_EF, SENDER_EF | OWNER_SUM, 0):
+        f = np.zeros(m, F32)
+        s = np.zeros(m, F32)
+        eps = np.zeros((P, m), F32)
+        T = np.zeros(m)
+        emax = np.zeros(m)
+        epsmax = np.zeros(m)
+        xmax = np.zeros(m)
+        for k in range(K):
+            x = gaussian(P, m, seed=13, call=k, dtype="fp32")
+            res = orc.allreduce(x, f, s, Params(), want_diag=True, variant=variant, eps=eps)
+            T += res["out"].astype(np.float64) - x.astype(np.float64).sum(axis=0)
+            emax = np.maximum(emax, np.abs(res["err"]))
+            xmax = np.maximum(xmax, np.abs(x).sum(axis=0) + 8)
+            if variant & SENDER_EF:
+                epsmax = np.maximum(epsmax, np.abs(eps).max(axis=0))
+                bound = 5 * emax + P * epsmax + (k + 1) * 4 * P * 2.0 ** -23 * xmax
+                assert (np.abs(T) <= bound).all(), (variant, k)
+        rms[variant] = math.sqrt(float(np.mean(T ** 2)))
+    assert rms[SENDER_EF] < 0.3 * rms[0], rms
+    assert rms[SENDER_EF | OWNER_SUM] < 0.3 * rms[0], rms
+
+
 ALL_PINS = [
     pin_scale_boundaries,
     pin_quantizer_bruteforce,
@@ -464,4 +605,11 @@ ALL_PINS = [
     pin_bounded_partial_sum,
     pin_two_roundings_bound,
     pin_power_of_two_equivariance,
+    pin_owner_sum_hand_example,
+    pin_owner_sum_injection,
+    pin_owner_sum_order,
+    pin_owner_sum_error_feedback,
+    pin_sender_ef_on_grid,
+    pin_sender_ef_per_rank,
+    pin_full_compensation_bounded,
 ]

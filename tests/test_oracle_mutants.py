@@ -56,8 +56,8 @@ MUTANTS = [
      "float from_fast = lambda * f[i];",
      "float from_fast = lambda * s[i];"),
     ("every_rank_injects",
-     "if (enable && owner[g] == r)",
-     "if (enable)"),
+     "if (enable && !owner_sum && owner[g] == r)",
+     "if (enable && !owner_sum)"),
     ("wrong_owner",
      "owner[g] = (int32_t)((g * (size_t)G) / seg);",
      "owner[g] = (int32_t)(((g * (size_t)G) / seg + 1) % (size_t)P);"),
@@ -74,8 +74,30 @@ MUTANTS = [
      "float Y = echo_oracle_dequant(Q[i], bq);",
      "float Y = S[k];"),
     ("correction_not_added",
-     "v[k] = xi + c[i];",
-     "v[k] = xi;"),
+     "v[k] = u + c[i];",
+     "v[k] = u;"),
+    # variants
+    ("sender_error_not_kept",
+     "eps[(size_t)r * m + i] = v[k] - restored;",
+     "eps[(size_t)r * m + i] = 0.0f;"),
+    ("sender_error_sign_flipped",
+     "eps[(size_t)r * m + i] = v[k] - restored;",
+     "eps[(size_t)r * m + i] = restored - v[k];"),
+    ("sender_error_not_added",
+     "u = xi + eps[(size_t)r * m + i];",
+     "u = xi;"),
+    ("sender_error_wrong_rank",
+     "u = xi + eps[(size_t)r * m + i];",
+     "u = xi + eps[(size_t)((r + 1) % P) * m + i];"),
+    ("owner_sum_adds_twice",
+     "sum = sum + c[i];",
+     "sum = sum + c[i] + c[i];"),
+    ("owner_sum_sender_also_adds",
+     "if (enable && !owner_sum && owner[g] == r)",
+     "if (enable && owner[g] == r)"),
+    ("owner_sum_starts_from_correction",
+     [("float sum = 0.0f;", "float sum = (enable && owner_sum) ? c[i] : 0.0f;"),
+      ("if (enable && owner_sum)\n                sum = sum + c[i];", "")]),
 ]
 
 
@@ -84,15 +106,25 @@ def mutant_dir(tmp_path_factory):
     return tmp_path_factory.mktemp("oracle_mutants")
 
 
-@pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
-def test_pins_catch_mutant(mutant_dir, name, old, new):
+def _edits(entry):
+    """A mutant is (name, old, new) or (name, [(old, new), ...])."""
+    if len(entry) == 3:
+        return [(entry[1], entry[2])]
+    return entry[1]
+
+
+@pytest.mark.parametrize("entry", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_pins_catch_mutant(mutant_dir, entry):
+    name = entry[0]
     src = open(os.path.join(ORACLE_DIR, "echo_oracle.c")).read()
-    assert src.count(old) == 1, f"mutation site for {name} not unique/present"
+    for old, new in _edits(entry):
+        assert src.count(old) == 1, f"mutation site for {name} not unique/present: {old!r}"
+        src = src.replace(old, new)
     work = os.path.join(str(mutant_dir), name)
     os.makedirs(work, exist_ok=True)
     shutil.copy(os.path.join(ORACLE_DIR, "echo_oracle.h"), work)
     with open(os.path.join(work, "echo_oracle.c"), "w") as fh:
-        fh.write(src.replace(old, new))
+        fh.write(src)
     lib = os.path.join(work, "libmutant.so")
     subprocess.run(["gcc", "-std=c99", "-O2", "-ffp-contract=off", "-fPIC", "-shared",
                     "-o", lib, os.path.join(work, "echo_oracle.c"), "-lm"], check=True)
