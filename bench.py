@@ -45,6 +45,8 @@ SEED = 0
 WORKLOAD = "echo int4 all-reduce, P=8 ranks x 1 GiB bf16 per rank (2^29 elements), group 32, " \
            "compensation on, fwd state, partials N(0,1) with 0.1% at 50x"
 HBM_FALLBACK_GBS = 6650.0  # used only when MEASURED_PEAKS.json is absent
+# where the rounding errors are fed back (see include/echo.h, echo_set_variant)
+VARIANTS = {"default": 0, "owner_sum": 1, "sender_ef": 2, "both": 3}
 # CPU baseline / reference arm samples (elements per rank, same distribution)
 CPU_SAMPLE_N = 1 << 20
 REF_SAMPLE_N = 1 << 18
@@ -184,7 +186,8 @@ def gpu_selector(local_rank: int) -> str:
 # ---------------------------------------------------------------------------
 # the CPU oracle (baseline leg and reference arm)
 # ---------------------------------------------------------------------------
-def oracle_sample_rate(n_sample: int, budget_s: float, min_calls: int, max_calls: int, seed: int):
+def oracle_sample_rate(n_sample: int, budget_s: float, min_calls: int, max_calls: int, seed: int,
+                       variant: int = 0):
     """Time the oracle on P x n_sample bf16 partials of the workload's
     distribution, call after call (state carried), until budget_s is spent."""
     import numpy as np
@@ -193,20 +196,22 @@ def oracle_sample_rate(n_sample: int, budget_s: float, min_calls: int, max_calls
     orc = Oracle()
     f = np.zeros(n_sample, np.float32)
     s = np.zeros(n_sample, np.float32)
+    eps = np.zeros((P, n_sample), np.float32)
     times = []
     t_all = time.perf_counter()
     k = 0
     while k < min_calls or (time.perf_counter() - t_all < budget_s and k < max_calls):
         x = wl.outlier_gaussian(P, n_sample, seed=seed, call=k)
         t0 = time.perf_counter()
-        orc.allreduce(x, f, s, Params(), want_wire=False)
+        orc.allreduce(x, f, s, Params(), want_wire=False, variant=variant, eps=eps)
         times.append(time.perf_counter() - t0)
         k += 1
     return times
 
 
-def cpu_baseline_leg() -> dict:
-    times = oracle_sample_rate(CPU_SAMPLE_N, budget_s=10.0, min_calls=3, max_calls=60, seed=1)
+def cpu_baseline_leg(variant: int = 0) -> dict:
+    times = oracle_sample_rate(CPU_SAMPLE_N, budget_s=10.0, min_calls=3, max_calls=60, seed=1,
+                               variant=variant)
     t = sum(times) / len(times)
     return {
         "value": round(2 * CPU_SAMPLE_N / t / 1e9, 6), "unit": UNIT, "cores": 1, "kind": "oracle",
@@ -274,8 +279,11 @@ def run_echo(args, rank: int, world: int, local: int) -> dict | None:
     recv = [torch.empty(n, dtype=torch.bfloat16, device=device) for _ in range(P)]
     for r in range(P):
         wl.torch_outlier_gaussian_(send[r], seed=SEED + 1000 * rank, call=0, rank=r)
+    variant = VARIANTS[args.variant]
     h = echo.Echo(P, n, echo.ECHO_BF16)
-    mb = echo.echo_model_bytes(P, n, echo.ECHO_BF16, True)
+    if variant:
+        h.set_variant(variant)
+    mb = echo.echo_model_bytes_variant(P, n, echo.ECHO_BF16, True, variant)
     torch.cuda.synchronize()
 
     for _ in range(args.warmup):
@@ -316,7 +324,7 @@ def run_echo(args, rank: int, world: int, local: int) -> dict | None:
     achieved = k_bytes[dom] / (k_avg[dom] * 1e-3) / 1e9
     src = os.path.join(ROOT, "bit_error_compensated_rank_b200", "csrc", names[dom] + ".cu")
     traffic = None
-    rec = NCU_TRAFFIC.get(names[dom])
+    rec = NCU_TRAFFIC.get(names[dom]) if variant == 0 else None  # captured for the default variant
     if rec and rec["source_sha"] == _source_hash(src):
         traffic = round(rec["bytes_per_elem"] * n)
 
@@ -330,7 +338,8 @@ def run_echo(args, rank: int, world: int, local: int) -> dict | None:
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": WORKLOAD, "P": P, "n_per_rank": n, "group": 32,
+        "config": {"workload": WORKLOAD + ("" if variant == 0 else f", variant {args.variant}"),
+                   "variant": args.variant, "P": P, "n_per_rank": n, "group": 32,
                    "parallelism": f"{world} independent replica(s), ranks simulated in HBM",
                    "l2": "inputs larger than L2 (8 GiB of partials per GPU vs 126 MB L2)"},
         "hbm_roofline_frac": round(call_frac, 4),
@@ -393,6 +402,8 @@ def main(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--variant", choices=sorted(VARIANTS), default="default",
+                    help="where rounding errors are fed back (default: the method as read)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -413,7 +424,7 @@ def main(argv=None):
         dist.destroy_process_group()
     if res is not None:
         if world == 1 and not args.no_cpu_baseline:
-            res["cpu_baseline"] = cpu_baseline_leg()
+            res["cpu_baseline"] = cpu_baseline_leg(VARIANTS[args.variant])
         print(json.dumps(res), flush=True)
     return 0
 

@@ -87,12 +87,16 @@ int check_shape(int P, size_t n, int group, int dtype)
     return ECHO_OK;
 }
 
-void model_bytes(int P, size_t n, int dtype, bool enable, uint64_t out[4])
+void model_bytes(int P, size_t n, int dtype, bool enable, int variant, uint64_t out[4])
 {
     const uint64_t b = elem_bytes(dtype);
     const uint64_t wire = static_cast<uint64_t>(n) / 32 * 17; // n * 17/32
     const uint64_t state = enable ? 8 * static_cast<uint64_t>(n) : 0;
-    out[0] = P * b * n + state + P * wire;           // K1
+    // the owner-sum variant reads f, s in kernel 2 only
+    const uint64_t k1_state = (variant & ECHO_VARIANT_OWNER_SUM) ? 0 : state;
+    // sender feedback: every rank reads and writes its own error (4 + 4 bytes)
+    const uint64_t eps = (variant & ECHO_VARIANT_SENDER_EF) ? 8 * static_cast<uint64_t>(P) * n : 0;
+    out[0] = P * b * n + k1_state + P * wire + eps;  // K1
     out[1] = P * wire + 2 * state + wire;            // K2
     out[2] = P * wire + P * b * n;                   // K3
     out[3] = 2 * static_cast<uint64_t>(P - 1) * wire; // link bytes
@@ -114,6 +118,8 @@ struct echo_handle {
     float *state = nullptr;     // [phase][f|s][n]
     float beta_f = 0.5f, beta_s = 0.875f, lambda = 0.5f;
     bool enable = true;
+    int variant = 0;            // ECHO_VARIANT_* bits
+    float *eps = nullptr;       // [phase][P][n]: sender errors (allocated with the variant)
     uint64_t link_bytes = 0, hbm_bytes = 0, calls = 0;
     // Kernel timing: each timed call records 4 events (before K1, after K1,
     // K2, K3) into slot (call index mod kTimingRing); a slot's durations are
@@ -278,7 +284,9 @@ int enqueue_call(echo_handle *h, const void *const send[], void *const recv[], i
     a1.one_minus_lambda = 1.0f - h->lambda;
     a1.P = h->P;
     a1.bf16 = h->dtype == ECHO_BF16;
-    a1.enable = h->enable;
+    a1.enable = h->enable && !(h->variant & ECHO_VARIANT_OWNER_SUM);
+    a1.sender_ef = (h->variant & ECHO_VARIANT_SENDER_EF) != 0;
+    a1.eps = a1.sender_ef ? h->eps + static_cast<size_t>(phase) * h->P * h->n : nullptr;
 
     a2.codes = h->codes1;
     a2.scales = h->scales1;
@@ -293,8 +301,11 @@ int enqueue_call(echo_handle *h, const void *const send[], void *const recv[], i
     a2.one_minus_beta_f = 1.0f - h->beta_f;
     a2.beta_s = h->beta_s;
     a2.one_minus_beta_s = 1.0f - h->beta_s;
+    a2.lambda = h->lambda;
+    a2.one_minus_lambda = 1.0f - h->lambda;
     a2.P = h->P;
     a2.enable = h->enable;
+    a2.owner_sum = h->enable && (h->variant & ECHO_VARIANT_OWNER_SUM);
 
     a3.qcodes = h->qcodes;
     a3.qscales = h->qscales;
@@ -340,7 +351,7 @@ int enqueue_call(echo_handle *h, const void *const send[], void *const recv[], i
 void count_call(echo_handle *h)
 {
     uint64_t mb[4];
-    model_bytes(h->P, h->n, h->dtype, h->enable, mb);
+    model_bytes(h->P, h->n, h->dtype, h->enable, h->variant, mb);
     h->hbm_bytes += mb[0] + mb[1] + mb[2];
     h->link_bytes += mb[3];
     h->calls += 1;
@@ -370,6 +381,7 @@ void free_handle(echo_handle *h)
     cudaFree(h->qscales);
     cudaFree(h->state);
     cudaFree(h->dstatus);
+    cudaFree(h->eps);
     cudaFree(h->staging);
     for (auto &slot : h->ring)
         for (cudaEvent_t e : slot)
@@ -434,8 +446,82 @@ int echo_model_bytes(int P, size_t n, int dtype, int enable, uint64_t out[4])
         return rc;
     if (!out)
         return set_error(ECHO_ERR_INVALID, "out is NULL");
-    model_bytes(P, n, dtype, enable != 0, out);
+    model_bytes(P, n, dtype, enable != 0, 0, out);
     return ECHO_OK;
+}
+
+int echo_model_bytes_variant(int P, size_t n, int dtype, int enable, int variant, uint64_t out[4])
+{
+    int rc = check_shape(P, n, ECHO_GROUP, dtype);
+    if (rc != ECHO_OK)
+        return rc;
+    if (!out)
+        return set_error(ECHO_ERR_INVALID, "out is NULL");
+    if (variant & ~(ECHO_VARIANT_OWNER_SUM | ECHO_VARIANT_SENDER_EF))
+        return set_error(ECHO_ERR_INVALID, "unknown variant bits 0x%x", variant);
+    model_bytes(P, n, dtype, enable != 0, variant, out);
+    return ECHO_OK;
+}
+
+int echo_set_variant(echo_handle *h, int variant)
+{
+    int rc;
+    if ((rc = check_handle(h)) != ECHO_OK || (rc = check_device(h)) != ECHO_OK)
+        return rc;
+    if (variant & ~(ECHO_VARIANT_OWNER_SUM | ECHO_VARIANT_SENDER_EF))
+        return set_error(ECHO_ERR_INVALID, "unknown variant bits 0x%x", variant);
+    if ((variant & ECHO_VARIANT_SENDER_EF) && !h->eps) {
+        const size_t bytes = 2 * static_cast<size_t>(h->P) * h->n * sizeof(float);
+        cudaError_t e = cudaDeviceSynchronize();
+        if (e == cudaSuccess)
+            e = cudaMalloc(&h->eps, bytes);
+        if (e != cudaSuccess) {
+            h->eps = nullptr;
+            cudaGetLastError();
+            return set_error(ECHO_ERR_OOM, "sender-error state of %zu bytes: %s", bytes, cudaGetErrorString(e));
+        }
+        e = cudaMemset(h->eps, 0, bytes);
+        if (e == cudaSuccess)
+            e = cudaDeviceSynchronize();
+        if (e != cudaSuccess)
+            return cuda_error(e, "echo_set_variant");
+    }
+    h->variant = variant;
+    return ECHO_OK;
+}
+
+int echo_get_sender_state(echo_handle *h, int phase, int rank, size_t offset, size_t count, float *host)
+{
+    int rc;
+    if ((rc = check_handle(h)) != ECHO_OK || (rc = check_phase(phase)) != ECHO_OK ||
+        (rc = check_device(h)) != ECHO_OK)
+        return rc;
+    if (!h->eps)
+        return set_error(ECHO_ERR_INVALID, "sender feedback was never switched on (echo_set_variant)");
+    if (rank < 0 || rank >= h->P || !host || offset > h->n || count > h->n - offset)
+        return set_error(ECHO_ERR_INVALID, "bad rank, range or NULL output");
+    const float *src = h->eps + (static_cast<size_t>(phase) * h->P + rank) * h->n + offset;
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e == cudaSuccess)
+        e = cudaMemcpy(host, src, count * sizeof(float), cudaMemcpyDeviceToHost);
+    return e == cudaSuccess ? ECHO_OK : cuda_error(e, "echo_get_sender_state");
+}
+
+int echo_set_sender_state(echo_handle *h, int phase, int rank, const float *host)
+{
+    int rc;
+    if ((rc = check_handle(h)) != ECHO_OK || (rc = check_phase(phase)) != ECHO_OK ||
+        (rc = check_device(h)) != ECHO_OK)
+        return rc;
+    if (!h->eps)
+        return set_error(ECHO_ERR_INVALID, "sender feedback was never switched on (echo_set_variant)");
+    if (rank < 0 || rank >= h->P || !host)
+        return set_error(ECHO_ERR_INVALID, "bad rank or NULL input");
+    float *dst = h->eps + (static_cast<size_t>(phase) * h->P + rank) * h->n;
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e == cudaSuccess)
+        e = cudaMemcpy(dst, host, h->n * sizeof(float), cudaMemcpyHostToDevice);
+    return e == cudaSuccess ? ECHO_OK : cuda_error(e, "echo_set_sender_state");
 }
 
 echo_handle *echo_create(int P, size_t n, int group, int dtype)
@@ -608,9 +694,14 @@ int echo_reset(echo_handle *h, int phase_mask)
     if (phase_mask < 0 || phase_mask > 3)
         return set_error(ECHO_ERR_INVALID, "phase_mask %d: only bits 0 (fwd) and 1 (bwd) exist", phase_mask);
     cudaError_t e = cudaDeviceSynchronize();
-    for (int p = 0; p < 2 && e == cudaSuccess; p++)
-        if (phase_mask & (1 << p))
-            e = cudaMemset(h->state + static_cast<size_t>(p) * 2 * h->n, 0, 2 * h->n * sizeof(float));
+    for (int p = 0; p < 2 && e == cudaSuccess; p++) {
+        if (!(phase_mask & (1 << p)))
+            continue;
+        e = cudaMemset(h->state + static_cast<size_t>(p) * 2 * h->n, 0, 2 * h->n * sizeof(float));
+        if (e == cudaSuccess && h->eps)
+            e = cudaMemset(h->eps + static_cast<size_t>(p) * h->P * h->n, 0,
+                           static_cast<size_t>(h->P) * h->n * sizeof(float));
+    }
     if (e == cudaSuccess)
         e = cudaDeviceSynchronize();
     return e == cudaSuccess ? ECHO_OK : cuda_error(e, "echo_reset");

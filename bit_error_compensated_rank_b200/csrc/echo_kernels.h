@@ -41,8 +41,10 @@
 #ifndef ECHO_K3_OUT_BUFS
 #define ECHO_K3_OUT_BUFS 2
 #endif
-// Shared memory one CTA may use (the B200 limit is 227 KB).
+// Shared memory one CTA may use (the B200 limit is 227 KB), and kernel 1's
+// budget per CTA so that two CTAs share an SM.
 #define ECHO_SMEM_BUDGET (225 * 1024)
+#define ECHO_K1_CTA_BUDGET (100 * 1024)
 
 namespace echo {
 
@@ -64,9 +66,11 @@ struct K1Args {
     uint32_t chunk_begin, chunk_end;
     uint32_t groups_per_seg; // n / P / 32: owner of group g is g / groups_per_seg
     float lambda, one_minus_lambda;
+    float *eps;              // sender feedback: every rank's rounding-#1 error [P][n]
     int P;
     bool bf16;
-    bool enable;
+    bool enable;             // the owner adds the correction to its partial
+    bool sender_ef;          // every rank adds back and renews its own error
     PipeCtl ctl;
 };
 
@@ -80,8 +84,10 @@ struct K2Args {
     size_t scale_stride;
     uint32_t chunk_begin, chunk_end;
     float beta_f, one_minus_beta_f, beta_s, one_minus_beta_s;
+    float lambda, one_minus_lambda;
     int P;
-    bool enable;
+    bool enable;             // read the state, capture the error, update the state
+    bool owner_sum;          // add the correction to the owner's sum
     PipeCtl ctl;
 };
 

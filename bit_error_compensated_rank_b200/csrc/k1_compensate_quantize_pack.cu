@@ -5,22 +5,26 @@
 // c = lambda*f + (1-lambda)*s built from the two smoothed error estimates
 // [rit.work "Echo 4-bit GPU communication", section "How Echo returns the
 // error to later calls": the stored error is added back in later calls].
+// With sender feedback (a variant), every rank first adds back its own
+// rounding-#1 error of its previous call and stores the new one, exact:
+// v = RN(RN(x + eps) + c), eps <- v - q*2^e.
 //
 // Layout: the rank partials are P separate buffers of n elements; the output
 // is the stage-1 wire, codes [P][n/2] (two per byte) and scale bytes
-// [P][scale_stride].
+// [P][scale_stride]; the sender errors are [P][n] binary32.
 //
 // Pipeline (warp-specialised, persistent): a CTA takes tiles of kTile
-// consecutive elements. One producer warp bulk-copies the P partial tiles and
-// the f, s tiles of a tile into one stage of a kStages ring in shared memory
-// (mbarrier full[s] counts the bytes); eight consumer warps compute from
-// shared memory and release the stage on mbarrier empty[s]. A lane owns 8
-// consecutive elements of one rank; 4 lanes form a group and find its
-// maximum with two shuffles; codes leave as one coalesced 32-bit store per
-// lane.
+// consecutive elements. One producer warp bulk-copies the P partial tiles
+// (and the f, s tiles, and the P error tiles, when used) of a tile into one
+// stage of a kStages ring in shared memory (mbarrier full[s] counts the
+// bytes); eight consumer warps compute from shared memory and release the
+// stage on mbarrier empty[s]. A lane owns 8 consecutive elements of one rank;
+// 4 lanes form a group and find its maximum with two shuffles; codes leave as
+// one coalesced 32-bit store per lane.
 //
 // Algorithmic HBM bytes per element of n: P*b (partials) + 8 (f, s; each
-// element is corrected by exactly one rank) read, P*17/32 written.
+// element is corrected by exactly one rank) read, P*17/32 written; sender
+// feedback adds 4P read and 4P written.
 #include "echo_bulk.cuh"
 #include "echo_kernels.h"
 
@@ -33,17 +37,34 @@ constexpr int kConsumerWarps = 8;
 constexpr int kConsumers = kConsumerWarps * 32;
 constexpr int kThreads = kConsumers + 32; // + one producer warp
 
-template <int P, bool BF16, bool COMP>
+// Bytes one stage holds per element of the tile.
+constexpr int k1_bytes_per_elem(int P, bool bf16, bool comp, bool ef)
+{
+    return P * (bf16 ? 2 : 4) + (comp ? 8 : 0) + (ef ? 4 * P : 0);
+}
+
+// The largest tile (ECHO_K1_TILE, /2, /4, ... down to 256 elements) whose
+// stages fit ECHO_K1_CTA_BUDGET.
+constexpr int k1_tile(int P, bool bf16, bool comp, bool ef)
+{
+    int t = ECHO_K1_TILE;
+    while (t > 256 && ECHO_K1_STAGES * t * k1_bytes_per_elem(P, bf16, comp, ef) > ECHO_K1_CTA_BUDGET)
+        t /= 2;
+    return t;
+}
+
+template <int P, bool BF16, bool COMP, bool EF>
 struct K1Shape {
     static constexpr int kEB = BF16 ? 2 : 4;
-    // Tile length keeps one stage near 12-24 KB whatever P and the dtype.
-    static constexpr int kTile = (P * kEB <= 16) ? ECHO_K1_TILE : (P * kEB <= 32 ? ECHO_K1_TILE / 2 : ECHO_K1_TILE / 4);
+    static constexpr int kTile = k1_tile(P, BF16, COMP, EF);
     static constexpr int kStages = ECHO_K1_STAGES;
-    static constexpr int kXBytes = kTile * kEB; // one rank's partial tile
-    static constexpr int kStageBytes = P * kXBytes + (COMP ? 2 * kTile * 4 : 0);
+    static constexpr int kXBytes = kTile * kEB;             // one rank's partial tile
+    static constexpr int kStateOff = P * kXBytes;           // f tile, then s tile
+    static constexpr int kEpsOff = kStateOff + (COMP ? 2 * kTile * 4 : 0); // P error tiles
+    static constexpr int kStageBytes = kEpsOff + (EF ? P * kTile * 4 : 0);
     static constexpr int kSmem = kStages * kStageBytes + 2 * kStages * 8;
+    static constexpr int kChunksPerTile = kTile / kChunk;   // a multiple of 32
     static_assert(kSmem <= ECHO_SMEM_BUDGET, "kernel 1 stages exceed shared memory");
-    static constexpr int kChunksPerTile = kTile / kChunk; // a multiple of 32
 };
 
 template <bool BF16>
@@ -59,11 +80,19 @@ __device__ __forceinline__ void load_chunk(const uint8_t *p, float (&v)[kChunk])
     }
 }
 
-template <int P, bool BF16, bool COMP>
+__device__ __forceinline__ void load_f32x8(const float *p, float (&v)[kChunk])
+{
+    const float4 a = reinterpret_cast<const float4 *>(p)[0];
+    const float4 b = reinterpret_cast<const float4 *>(p)[1];
+    v[0] = a.x, v[1] = a.y, v[2] = a.z, v[3] = a.w;
+    v[4] = b.x, v[5] = b.y, v[6] = b.z, v[7] = b.w;
+}
+
+template <int P, bool BF16, bool COMP, bool EF>
 __global__ void __launch_bounds__(kThreads)
     k1_compensate_quantize_pack(const K1Args a)
 {
-    using Sh = K1Shape<P, BF16, COMP>;
+    using Sh = K1Shape<P, BF16, COMP, EF>;
     constexpr int S = Sh::kStages;
     extern __shared__ __align__(128) uint8_t smem[];
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + S * Sh::kStageBytes);
@@ -95,15 +124,21 @@ __global__ void __launch_bounds__(kThreads)
                                      e1 - el0 < size_t(Sh::kTile) ? e1 - el0 : Sh::kTile);
                                  uint8_t *stage = smem + (i % S) * Sh::kStageBytes;
                                  uint64_t *bar = &full[i % S];
-                                 mbar_arrive_expect_tx(bar, P * cnt * Sh::kEB + (COMP ? 2 * cnt * 4 : 0));
+                                 mbar_arrive_expect_tx(bar, cnt * Sh::kStageBytes / Sh::kTile);
 #pragma unroll
                                  for (int r = 0; r < P; r++)
                                      bulk_load(stage + r * Sh::kXBytes,
                                                static_cast<const uint8_t *>(a.x.p[r]) + el0 * Sh::kEB,
                                                cnt * Sh::kEB, bar);
                                  if (COMP) {
-                                     bulk_load(stage + P * Sh::kXBytes, a.f + el0, cnt * 4, bar);
-                                     bulk_load(stage + P * Sh::kXBytes + Sh::kTile * 4, a.s + el0, cnt * 4, bar);
+                                     bulk_load(stage + Sh::kStateOff, a.f + el0, cnt * 4, bar);
+                                     bulk_load(stage + Sh::kStateOff + Sh::kTile * 4, a.s + el0, cnt * 4, bar);
+                                 }
+                                 if (EF) {
+#pragma unroll
+                                     for (int r = 0; r < P; r++)
+                                         bulk_load(stage + Sh::kEpsOff + r * Sh::kTile * 4,
+                                                   a.eps + static_cast<size_t>(r) * a.n + el0, cnt * 4, bar);
                                  }
                              });
         return;
@@ -117,7 +152,8 @@ __global__ void __launch_bounds__(kThreads)
         const uint32_t tile_chunk0 = static_cast<uint32_t>(e0 / kChunk) + (blockIdx.x + i * gridDim.x) * (Sh::kTile / kChunk);
         const uint32_t cnt_chunks = min(static_cast<uint32_t>(Sh::kChunksPerTile), a.chunk_end - tile_chunk0);
         const uint8_t *stage = smem + s * Sh::kStageBytes;
-        const float *fs = reinterpret_cast<const float *>(stage + P * Sh::kXBytes);
+        const float *fs = reinterpret_cast<const float *>(stage + Sh::kStateOff);
+        const float *es = reinterpret_cast<const float *>(stage + Sh::kEpsOff);
 
 #pragma unroll 2
         for (uint32_t it = tid; it < static_cast<uint32_t>(P * Sh::kChunksPerTile); it += kConsumers) {
@@ -129,14 +165,18 @@ __global__ void __launch_bounds__(kThreads)
 
             float v[kChunk];
             load_chunk<BF16>(stage + r * Sh::kXBytes + c * (kChunk * Sh::kEB), v);
+            if (EF) { // add back this rank's own rounding-#1 error
+                float e[kChunk];
+                load_f32x8(es + r * Sh::kTile + c * kChunk, e);
+#pragma unroll
+                for (int k = 0; k < kChunk; k++)
+                    v[k] = __fadd_rn(v[k], e[k]);
+            }
             // rank r owns groups [r*gps, (r+1)*gps): one unsigned range test
             if (COMP && g - r * a.groups_per_seg < a.groups_per_seg) {
-                const float4 f0 = reinterpret_cast<const float4 *>(fs)[2 * c];
-                const float4 f1 = reinterpret_cast<const float4 *>(fs)[2 * c + 1];
-                const float4 s0 = reinterpret_cast<const float4 *>(fs + Sh::kTile)[2 * c];
-                const float4 s1 = reinterpret_cast<const float4 *>(fs + Sh::kTile)[2 * c + 1];
-                const float fv[kChunk] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
-                const float sv[kChunk] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+                float fv[kChunk], sv[kChunk];
+                load_f32x8(fs + c * kChunk, fv);
+                load_f32x8(fs + Sh::kTile + c * kChunk, sv);
 #pragma unroll
                 for (int k = 0; k < kChunk; k++)
                     v[k] = __fadd_rn(v[k], __fadd_rn(__fmul_rn(a.lambda, fv[k]),
@@ -157,6 +197,17 @@ __global__ void __launch_bounds__(kThreads)
                 reinterpret_cast<uint32_t *>(a.codes)[static_cast<size_t>(r) * code_words + chunk] = word;
                 if ((lane & 3u) == 0)
                     a.scales[static_cast<size_t>(r) * a.scale_stride + g] = static_cast<uint8_t>(byte);
+                if (EF) { // the new error v - q*2^e, exact
+                    const float st = step_of(byte);
+                    float e[kChunk];
+#pragma unroll
+                    for (int k = 0; k < kChunk; k++)
+                        e[k] = __fmaf_rn(-code_value(qb[k]), st, v[k]);
+                    float4 *eo = reinterpret_cast<float4 *>(a.eps + static_cast<size_t>(r) * a.n) +
+                                 2 * static_cast<size_t>(chunk);
+                    eo[0] = make_float4(e[0], e[1], e[2], e[3]);
+                    eo[1] = make_float4(e[4], e[5], e[6], e[7]);
+                }
             }
         }
         __syncwarp();
@@ -165,12 +216,12 @@ __global__ void __launch_bounds__(kThreads)
     }
 }
 
-template <int P, bool BF16, bool COMP>
+template <int P, bool BF16, bool COMP, bool EF>
 cudaError_t launch_p(const K1Args &a, cudaStream_t st)
 {
-    using Sh = K1Shape<P, BF16, COMP>;
+    using Sh = K1Shape<P, BF16, COMP, EF>;
     static int resident = 0;
-    auto kern = k1_compensate_quantize_pack<P, BF16, COMP>;
+    auto kern = k1_compensate_quantize_pack<P, BF16, COMP, EF>;
     if (resident == 0) {
         cudaError_t e = prepare_kernel(reinterpret_cast<const void *>(kern), kThreads, Sh::kSmem, &resident);
         if (e != cudaSuccess)
@@ -182,12 +233,18 @@ cudaError_t launch_p(const K1Args &a, cudaStream_t st)
     return cudaGetLastError();
 }
 
+template <int P, bool BF16>
+cudaError_t dispatch_state(const K1Args &a, cudaStream_t st)
+{
+    if (a.enable)
+        return a.sender_ef ? launch_p<P, BF16, true, true>(a, st) : launch_p<P, BF16, true, false>(a, st);
+    return a.sender_ef ? launch_p<P, BF16, false, true>(a, st) : launch_p<P, BF16, false, false>(a, st);
+}
+
 template <int P>
 cudaError_t dispatch_flags(const K1Args &a, cudaStream_t st)
 {
-    if (a.bf16)
-        return a.enable ? launch_p<P, true, true>(a, st) : launch_p<P, true, false>(a, st);
-    return a.enable ? launch_p<P, false, true>(a, st) : launch_p<P, false, false>(a, st);
+    return a.bf16 ? dispatch_state<P, true>(a, st) : dispatch_state<P, false>(a, st);
 }
 
 } // namespace

@@ -9,6 +9,10 @@
 // precision at the owner, the rounding error computed from that sum, kept in
 // two smoothed estimates, separately for forward and backward].
 //
+// In the owner-sum variant the correction c = lambda*f + (1-lambda)*s is
+// added to the binary32 sum after the P restored values (one more rounding),
+// instead of being added by the owner to its partial in kernel 1.
+//
 // Every restored value q*2^e is exact, so the only roundings are the P-1
 // binary32 additions, rounding #2, and the two estimates' products and sums
 // (each rounded on its own: __fmul_rn / __fadd_rn are never contracted).
@@ -68,7 +72,7 @@ struct K2Shape {
 
 __device__ __forceinline__ uint32_t round16(uint32_t x) { return (x + 15u) & ~15u; }
 
-template <int P, bool COMP>
+template <int P, bool COMP, bool SUM>
 __global__ void __launch_bounds__(kThreads)
     k2_owner_reduce_requant(const K2Args a)
 {
@@ -130,68 +134,80 @@ __global__ void __launch_bounds__(kThreads)
         const uint8_t *stage = smem + sidx * Sh::kStageBytes;
 #pragma unroll 1
         for (int j = 0; j < Sh::kChunks; j++) {
-        const uint32_t c = tid + j * kConsumers; // chunk within the tile
-        const uint32_t chunk = tile_chunk0 + c;
-        const bool active = chunk < a.chunk_end;
-        const uint32_t g = chunk / kLanesPerGroup;
+            const uint32_t c = tid + j * kConsumers; // chunk within the tile
+            const uint32_t chunk = tile_chunk0 + c;
+            const bool active = chunk < a.chunk_end;
+            const uint32_t g = chunk / kLanesPerGroup;
 
-        // Restore and add, rank 0 first. The product q*2^e is exact, so
-        // fma(q, 2^e, S) = RN(S + q*2^e): one rounding per addition.
-        float S_[kChunk];
-#pragma unroll
-        for (int k = 0; k < kChunk; k++)
-            S_[k] = 0.f;
-#pragma unroll
-        for (int r = 0; r < P; r++) {
-            const uint32_t w = reinterpret_cast<const uint32_t *>(stage + r * Sh::kCodeBytes)[c];
-            const uint32_t b = stage[P * Sh::kCodeBytes + r * Sh::kScaleBytes + c / kLanesPerGroup];
-            const float st = step_of(b);
-            const Unpacked u = unpack8(w);
-#pragma unroll
-            for (int k = 0; k < kChunk; k++)
-                S_[k] = __fmaf_rn(code_at(u, k), st, S_[k]);
-        }
-
-        // Rounding #2 and the error it injects.
-        float m01 = fmaxf(fabsf(S_[0]), fabsf(S_[1])), m23 = fmaxf(fabsf(S_[2]), fabsf(S_[3]));
-        float m45 = fmaxf(fabsf(S_[4]), fabsf(S_[5])), m67 = fmaxf(fabsf(S_[6]), fabsf(S_[7]));
-        const float amax = group_absmax(fmaxf(fmaxf(m01, m23), fmaxf(m45, m67)));
-        const uint32_t byte = scale_byte(amax);
-        const float inv = inv_step_of(byte);
-        const float st = step_of(byte);
-        uint32_t qb[kChunk];
-        float err[kChunk];
-#pragma unroll
-        for (int k = 0; k < kChunk; k++) {
-            qb[k] = code_bits(S_[k], inv);
-            err[k] = __fmaf_rn(-code_value(qb[k]), st, S_[k]); // S - Q*2^E, exact
-        }
-
-        if (active) {
-            reinterpret_cast<uint32_t *>(a.qcodes)[chunk] = pack8_bits(qb);
-            if ((lane & 3u) == 0)
-                a.qscales[g] = static_cast<uint8_t>(byte);
+            float fv[kChunk], sv[kChunk];
             if (COMP) {
                 const float *fs = reinterpret_cast<const float *>(stage + Sh::kStateOff);
                 const float4 f0 = reinterpret_cast<const float4 *>(fs)[2 * c];
                 const float4 f1 = reinterpret_cast<const float4 *>(fs)[2 * c + 1];
                 const float4 s0 = reinterpret_cast<const float4 *>(fs + Sh::kTile)[2 * c];
                 const float4 s1 = reinterpret_cast<const float4 *>(fs + Sh::kTile)[2 * c + 1];
-                float fv[kChunk] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
-                float sv[kChunk] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
-#pragma unroll
-                for (int k = 0; k < kChunk; k++) {
-                    fv[k] = __fadd_rn(__fmul_rn(a.beta_f, fv[k]), __fmul_rn(a.one_minus_beta_f, err[k]));
-                    sv[k] = __fadd_rn(__fmul_rn(a.beta_s, sv[k]), __fmul_rn(a.one_minus_beta_s, err[k]));
-                }
-                float4 *fo = reinterpret_cast<float4 *>(a.f) + 2 * static_cast<size_t>(chunk);
-                float4 *so = reinterpret_cast<float4 *>(a.s) + 2 * static_cast<size_t>(chunk);
-                fo[0] = make_float4(fv[0], fv[1], fv[2], fv[3]);
-                fo[1] = make_float4(fv[4], fv[5], fv[6], fv[7]);
-                so[0] = make_float4(sv[0], sv[1], sv[2], sv[3]);
-                so[1] = make_float4(sv[4], sv[5], sv[6], sv[7]);
+                fv[0] = f0.x, fv[1] = f0.y, fv[2] = f0.z, fv[3] = f0.w;
+                fv[4] = f1.x, fv[5] = f1.y, fv[6] = f1.z, fv[7] = f1.w;
+                sv[0] = s0.x, sv[1] = s0.y, sv[2] = s0.z, sv[3] = s0.w;
+                sv[4] = s1.x, sv[5] = s1.y, sv[6] = s1.z, sv[7] = s1.w;
             }
-        }
+
+            // Restore and add, rank 0 first. The product q*2^e is exact, so
+            // fma(q, 2^e, S) = RN(S + q*2^e): one rounding per addition.
+            float S_[kChunk];
+#pragma unroll
+            for (int k = 0; k < kChunk; k++)
+                S_[k] = 0.f;
+#pragma unroll
+            for (int r = 0; r < P; r++) {
+                const uint32_t w = reinterpret_cast<const uint32_t *>(stage + r * Sh::kCodeBytes)[c];
+                const uint32_t b = stage[P * Sh::kCodeBytes + r * Sh::kScaleBytes + c / kLanesPerGroup];
+                const float st = step_of(b);
+                const Unpacked u = unpack8(w);
+#pragma unroll
+                for (int k = 0; k < kChunk; k++)
+                    S_[k] = __fmaf_rn(code_at(u, k), st, S_[k]);
+            }
+            if (SUM) { // variant: the correction enters the owner's sum, after the P ranks
+#pragma unroll
+                for (int k = 0; k < kChunk; k++)
+                    S_[k] = __fadd_rn(S_[k], __fadd_rn(__fmul_rn(a.lambda, fv[k]),
+                                                       __fmul_rn(a.one_minus_lambda, sv[k])));
+            }
+
+            // Rounding #2 and the error it injects.
+            const float m01 = fmaxf(fabsf(S_[0]), fabsf(S_[1])), m23 = fmaxf(fabsf(S_[2]), fabsf(S_[3]));
+            const float m45 = fmaxf(fabsf(S_[4]), fabsf(S_[5])), m67 = fmaxf(fabsf(S_[6]), fabsf(S_[7]));
+            const float amax = group_absmax(fmaxf(fmaxf(m01, m23), fmaxf(m45, m67)));
+            const uint32_t byte = scale_byte(amax);
+            const float inv = inv_step_of(byte);
+            const float st = step_of(byte);
+            uint32_t qb[kChunk];
+            float err[kChunk];
+#pragma unroll
+            for (int k = 0; k < kChunk; k++) {
+                qb[k] = code_bits(S_[k], inv);
+                err[k] = __fmaf_rn(-code_value(qb[k]), st, S_[k]); // S - Q*2^E, exact
+            }
+
+            if (active) {
+                reinterpret_cast<uint32_t *>(a.qcodes)[chunk] = pack8_bits(qb);
+                if ((lane & 3u) == 0)
+                    a.qscales[g] = static_cast<uint8_t>(byte);
+                if (COMP) {
+#pragma unroll
+                    for (int k = 0; k < kChunk; k++) {
+                        fv[k] = __fadd_rn(__fmul_rn(a.beta_f, fv[k]), __fmul_rn(a.one_minus_beta_f, err[k]));
+                        sv[k] = __fadd_rn(__fmul_rn(a.beta_s, sv[k]), __fmul_rn(a.one_minus_beta_s, err[k]));
+                    }
+                    float4 *fo = reinterpret_cast<float4 *>(a.f) + 2 * static_cast<size_t>(chunk);
+                    float4 *so = reinterpret_cast<float4 *>(a.s) + 2 * static_cast<size_t>(chunk);
+                    fo[0] = make_float4(fv[0], fv[1], fv[2], fv[3]);
+                    fo[1] = make_float4(fv[4], fv[5], fv[6], fv[7]);
+                    so[0] = make_float4(sv[0], sv[1], sv[2], sv[3]);
+                    so[1] = make_float4(sv[4], sv[5], sv[6], sv[7]);
+                }
+            }
         }
         __syncwarp();
         if (lane == 0)
@@ -199,12 +215,12 @@ __global__ void __launch_bounds__(kThreads)
     }
 }
 
-template <int P, bool COMP>
+template <int P, bool COMP, bool SUM>
 cudaError_t launch_p(const K2Args &a, cudaStream_t st)
 {
     using Sh = K2Shape<P, COMP>;
     static int resident = 0;
-    auto kern = k2_owner_reduce_requant<P, COMP>;
+    auto kern = k2_owner_reduce_requant<P, COMP, SUM>;
     if (resident == 0) {
         cudaError_t e = prepare_kernel(reinterpret_cast<const void *>(kern), kThreads, Sh::kSmem, &resident);
         if (e != cudaSuccess)
@@ -219,7 +235,9 @@ cudaError_t launch_p(const K2Args &a, cudaStream_t st)
 template <int P>
 cudaError_t dispatch_flags(const K2Args &a, cudaStream_t st)
 {
-    return a.enable ? launch_p<P, true>(a, st) : launch_p<P, false>(a, st);
+    if (!a.enable)
+        return launch_p<P, false, false>(a, st);
+    return a.owner_sum ? launch_p<P, true, true>(a, st) : launch_p<P, true, false>(a, st);
 }
 
 } // namespace

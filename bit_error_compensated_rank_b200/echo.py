@@ -28,6 +28,8 @@ ECHO_ERR_CUDA = -3
 ECHO_ERR_OOM = -4
 ECHO_MAX_RANKS = 16
 ECHO_GROUP = 32
+ECHO_VARIANT_OWNER_SUM = 1
+ECHO_VARIANT_SENDER_EF = 2
 
 EXPORTED = (
     "echo_create", "echo_allreduce", "echo_allreduce_out", "echo_allreduce_host",
@@ -35,7 +37,8 @@ EXPORTED = (
     "echo_get_state", "echo_set_state", "echo_get_state_range", "echo_get_wire",
     "echo_get_wire_range", "echo_stats", "echo_model_bytes", "echo_set_timing",
     "echo_last_kernel_ms", "echo_kernel_ms_total", "echo_device_status",
-    "echo_allreduce_static",
+    "echo_allreduce_static", "echo_set_variant", "echo_get_sender_state", "echo_set_sender_state",
+    "echo_model_bytes_variant",
 )
 
 _vp = ctypes.c_void_p
@@ -76,6 +79,10 @@ def _load():
         "echo_device_status": (_int, [_vp, ctypes.POINTER(ctypes.c_int), _int]),
         "echo_allreduce_static": (_int, [_int, _sz, _int, _vpp, _vp, _vp, ctypes.c_float, ctypes.c_float,
                                          ctypes.c_float, _int, _vp]),
+        "echo_set_variant": (_int, [_vp, _int]),
+        "echo_get_sender_state": (_int, [_vp, _int, _int, _sz, _sz, _f32p]),
+        "echo_set_sender_state": (_int, [_vp, _int, _int, _f32p]),
+        "echo_model_bytes_variant": (_int, [_int, _sz, _int, _int, _int, _u64p]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -205,6 +212,29 @@ def echo_model_bytes(P: int, n: int, dtype: int = ECHO_BF16, enable: bool = True
             "total": out[0] + out[1] + out[2]}
 
 
+def echo_model_bytes_variant(P: int, n: int, dtype: int = ECHO_BF16, enable: bool = True,
+                             variant: int = 0) -> dict:
+    out = (ctypes.c_uint64 * 4)()
+    _check(_lib.echo_model_bytes_variant(P, n, dtype, int(bool(enable)), variant, out))
+    return {"k1": out[0], "k2": out[1], "k3": out[2], "link": out[3],
+            "total": out[0] + out[1] + out[2]}
+
+
+def echo_set_variant(h: int, variant: int) -> None:
+    _check(_lib.echo_set_variant(h, variant))
+
+
+def echo_get_sender_state(h: int, phase: int, rank: int, offset: int, count: int) -> np.ndarray:
+    out = np.empty(count, np.float32)
+    _check(_lib.echo_get_sender_state(h, phase, rank, offset, count, _np(out, _f32p)))
+    return out
+
+
+def echo_set_sender_state(h: int, phase: int, rank: int, values: np.ndarray) -> None:
+    values = np.ascontiguousarray(values, np.float32)
+    _check(_lib.echo_set_sender_state(h, phase, rank, _np(values, _f32p)))
+
+
 def echo_set_timing(h: int, enable: bool = True) -> None:
     _check(_lib.echo_set_timing(h, int(bool(enable))))
 
@@ -269,6 +299,15 @@ class Echo:
 
     def reset(self, phase_mask: int = 3) -> None:
         echo_reset(self.h, phase_mask)
+
+    def set_variant(self, variant: int) -> None:
+        echo_set_variant(self.h, variant)
+
+    def get_sender_state(self, phase: int, rank: int, offset: int = 0, count: int | None = None):
+        return echo_get_sender_state(self.h, phase, rank, offset, self.n - offset if count is None else count)
+
+    def set_sender_state(self, phase: int, rank: int, values) -> None:
+        echo_set_sender_state(self.h, phase, rank, values)
 
     def get_state(self, phase: int = ECHO_FWD):
         return echo_get_state(self.h, phase, self.n)

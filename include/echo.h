@@ -146,9 +146,9 @@ ECHO_API int echo_allreduce_host(echo_handle *h, const void *const host_send[], 
 ECHO_API int echo_allreduce_static(int P, size_t n, int dtype, void *const rank_ptrs[], float *f, float *s,
                                    float beta_fast, float beta_slow, float lambda, int enable, void *stream);
 
-/* echo_reset - zero the compensator state of the phases in phase_mask
- * (bit 0 forward, bit 1 backward), enqueued on the legacy default stream and
- * completed before return. */
+/* echo_reset - zero the compensator state (and the sender errors, if
+ * allocated) of the phases in phase_mask (bit 0 forward, bit 1 backward);
+ * waits for the device first and completes before return. */
 ECHO_API int echo_reset(echo_handle *h, int phase_mask);
 
 /* echo_destroy - free everything the handle owns (synchronises the device
@@ -169,6 +169,35 @@ ECHO_API int echo_last_status(void);
  */
 ECHO_API int echo_set_params(echo_handle *h, float beta_fast, float beta_slow, float lambda,
                     int enable);
+
+/*
+ * echo_set_variant - variants of where the rounding errors are fed back, for
+ * later calls (bits; 0 is the method described above):
+ *   ECHO_VARIANT_OWNER_SUM  the owner adds c = lambda*f + (1-lambda)*s to its
+ *       binary32 sum after the P restored values, instead of adding it to its
+ *       own partial before rounding #1. The correction then passes no 4-bit
+ *       rounding, and kernel 1 reads no state (8 bytes less per element).
+ *   ECHO_VARIANT_SENDER_EF  every rank also feeds back its own rounding-#1
+ *       error: v = RN(RN(x + eps_r) + c), eps_r <- v - q*2^e (exact), one
+ *       binary32 per element per rank and phase (zeroed when first switched
+ *       on; allocated then, ECHO_ERR_OOM if that fails). With both roundings
+ *       fed back the running sum of all injected error stays bounded.
+ * The pages say the error a rounding injects is stored and added back in later
+ * calls [rit.work "Echo 4-bit GPU communication", section "How Echo returns
+ * the error to later calls"] and that the high-precision sum reveals every
+ * injected error [heraldofai.com, section "Come Echo evita che gli errori si
+ * accumulino"]; these variants are readings of where that happens.
+ */
+#define ECHO_VARIANT_OWNER_SUM 1
+#define ECHO_VARIANT_SENDER_EF 2
+ECHO_API int echo_set_variant(echo_handle *h, int variant);
+
+/* Synchronous copies of rank `rank`'s sender errors for `phase` (elements
+ * [offset, offset+count) to host; all n from host). ECHO_ERR_INVALID if sender
+ * feedback was never switched on. */
+ECHO_API int echo_get_sender_state(echo_handle *h, int phase, int rank, size_t offset, size_t count,
+                                   float *host);
+ECHO_API int echo_set_sender_state(echo_handle *h, int phase, int rank, const float *host);
 
 /* echo_get_state / echo_set_state - synchronous copies of a phase's two
  * estimates (n binary32 each) to / from host memory. A checkpoint is the pair
@@ -213,6 +242,10 @@ ECHO_API int echo_stats(echo_handle *h, uint64_t *link_bytes, uint64_t *model_hb
  * Same argument rules as echo_create.
  */
 ECHO_API int echo_model_bytes(int P, size_t n, int dtype, int enable, uint64_t out[4]);
+
+/* The same for a variant: OWNER_SUM drops kernel 1's 8 state bytes,
+ * SENDER_EF adds 8P bytes (each rank's error read and written) to kernel 1. */
+ECHO_API int echo_model_bytes_variant(int P, size_t n, int dtype, int enable, int variant, uint64_t out[4]);
 
 /*
  * Kernel timing. echo_set_timing(h, 1) starts a measurement: every later

@@ -12,7 +12,7 @@ from __future__ import annotations
 
 import numpy as np
 
-from oracle.oracle import Params
+from oracle.oracle import SENDER_EF, Params
 
 G = 32
 
@@ -63,16 +63,20 @@ class FullCompare:
     """One handle and the oracle side by side on a problem small enough to
     compare in full after every call."""
 
-    def __init__(self, oracle, P, n, dtype: str, params: Params = Params()):
+    def __init__(self, oracle, P, n, dtype: str, params: Params = Params(), variant: int = 0):
         from bit_error_compensated_rank_b200 import echo
         self.echo = echo
         self.oracle = oracle
         self.P, self.n = P, n
         self.dtype = dtype
         self.params = params
+        self.variant = variant
         self.h = echo.Echo(P, n, echo.ECHO_BF16 if dtype == "bf16" else echo.ECHO_FP32)
         self.h.set_params(*params_tuple(params))
+        if variant:
+            self.h.set_variant(variant)
         self.state = {ph: (np.zeros(n, np.float32), np.zeros(n, np.float32)) for ph in (0, 1)}
+        self.eps = {ph: np.zeros((P, n), np.float32) for ph in (0, 1)}
 
     def call(self, x: np.ndarray, phase: int = 0, out_of_place: bool = False,
              want_diag: bool = False):
@@ -87,7 +91,8 @@ class FullCompare:
             recv = dev
         t.cuda.synchronize()
         f, s = self.state[phase]
-        ref = self.oracle.allreduce(x, f, s, self.params, want_diag=want_diag)
+        ref = self.oracle.allreduce(x, f, s, self.params, want_diag=want_diag, variant=self.variant,
+                                    eps=self.eps[phase])
         got = from_device(recv)
         if out_of_place:  # the inputs are untouched
             assert_same_bits(from_device(dev), x, "send buffers")
@@ -105,6 +110,10 @@ class FullCompare:
             gf, gs = self.h.get_state(ph)
             assert_same_bits(gf, rf, f"fast estimate phase {ph}")
             assert_same_bits(gs, rs, f"slow estimate phase {ph}")
+            if self.variant & SENDER_EF:
+                for r in range(self.P):
+                    assert_same_bits(self.h.get_sender_state(ph, r), self.eps[ph][r],
+                                     f"sender error rank {r} phase {ph}")
         return ref
 
     def close(self):
@@ -121,7 +130,7 @@ class SampledCompare:
     """
 
     def __init__(self, oracle, P, n, dtype: str, params: Params = Params(), blocks=None,
-                 block_groups: int = 64, seed: int = 0):
+                 block_groups: int = 64, seed: int = 0, variant: int = 0):
         from bit_error_compensated_rank_b200 import echo
         self.echo = echo
         self.oracle = oracle
@@ -150,8 +159,12 @@ class SampledCompare:
         self.owner = (self.groups // seg_groups).astype(np.int32)
         self.h = echo.Echo(P, n, echo.ECHO_BF16 if dtype == "bf16" else echo.ECHO_FP32)
         self.h.set_params(*params_tuple(params))
+        self.variant = variant
+        if variant:
+            self.h.set_variant(variant)
         m = self.elems.size
         self.state = {ph: (np.zeros(m, np.float32), np.zeros(m, np.float32)) for ph in (0, 1)}
+        self.eps = {ph: np.zeros((P, m), np.float32) for ph in (0, 1)}
         self._idx = None
 
     def gather(self, tensors) -> np.ndarray:
@@ -169,7 +182,8 @@ class SampledCompare:
         self.h.allreduce(tensors, phase, stream)
         t.cuda.synchronize()
         f, s = self.state[phase]
-        ref = self.oracle.allreduce(x, f, s, self.params, owner=self.owner)
+        ref = self.oracle.allreduce(x, f, s, self.params, owner=self.owner, variant=self.variant,
+                                    eps=self.eps[phase])
         got = self.gather(tensors)
         for r in range(self.P):
             assert_same_bits(got[r], ref["out"], f"output rank {r}")
@@ -184,11 +198,15 @@ class SampledCompare:
             qc, qs = self.h.get_wire_range(2, 0, b, self.bg)
             assert_same_bits(qc, ref["qcodes"][csl], f"requantised codes block {b}")
             assert_same_bits(qs, ref["qscales"][sl], f"requantised scales block {b}")
+            esl = slice(bi * self.bg * G, (bi + 1) * self.bg * G)
             if self.params.enable:
-                esl = slice(bi * self.bg * G, (bi + 1) * self.bg * G)
                 gf, gs = self.h.get_state_range(phase, b * G, self.bg * G)
                 assert_same_bits(gf, f[esl], f"fast estimate block {b}")
                 assert_same_bits(gs, s[esl], f"slow estimate block {b}")
+            if self.variant & SENDER_EF:
+                for r in range(self.P):
+                    ge = self.h.get_sender_state(phase, r, b * G, self.bg * G)
+                    assert_same_bits(ge, self.eps[phase][r][esl], f"sender error rank {r} block {b}")
         return ref
 
     def close(self):
