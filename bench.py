@@ -392,8 +392,78 @@ def run_e2e(h, send, n, args, device, world) -> dict:
             "ms_per_step": round(ms, 3), "steps": steps}
 
 
+def run_sweep(args) -> None:
+    """Message-size sweep (one JSON line per size, not the benchmark line):
+    P = 8, bf16, n = 2^12 .. 2^29 elements per rank, CUDA-event time per call
+    over enough calls to fill about 50 ms, inputs resident, out of place."""
+    import torch
+    from bit_error_compensated_rank_b200 import echo
+    from bit_error_compensated_rank_b200 import workloads as wl
+    torch.cuda.set_device(0)
+    stream = torch.cuda.current_stream()
+    peak, _ = hbm_peak()
+    nmax = 1 << 29
+    send = [torch.empty(nmax, dtype=torch.bfloat16, device="cuda") for _ in range(P)]
+    recv = [torch.empty(nmax, dtype=torch.bfloat16, device="cuda") for _ in range(P)]
+    for r in range(P):
+        wl.torch_outlier_gaussian_(send[r], seed=SEED, call=0, rank=r)
+    variant = VARIANTS[args.variant]
+    for k in range(12, 30):
+        n = 1 << k
+        h = echo.Echo(P, n, echo.ECHO_BF16)
+        if variant:
+            h.set_variant(variant)
+        s_views = [t[:n] for t in send]
+        r_views = [t[:n] for t in recv]
+        for _ in range(args.warmup):
+            h.allreduce_out(s_views, r_views, 0, stream)
+        torch.cuda.synchronize()
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        h.allreduce_out(s_views, r_views, 0, stream)
+        end.record(stream)
+        torch.cuda.synchronize()
+        calls = max(5, min(2000, int(50.0 / max(start.elapsed_time(end), 1e-3))))
+        # (a) calls issued one by one from Python: includes host submission
+        start.record(stream)
+        for _ in range(calls):
+            h.allreduce_out(s_views, r_views, 0, stream)
+        end.record(stream)
+        torch.cuda.synchronize()
+        ms = start.elapsed_time(end) / calls
+        # (b) the same calls captured once in a CUDA graph and replayed: GPU time
+        per_graph = min(calls, 50)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            for _ in range(per_graph):
+                h.allreduce_out(s_views, r_views, 0, None)
+        graph.replay()
+        torch.cuda.synchronize()
+        reps = max(1, calls // per_graph)
+        start.record(stream)
+        for _ in range(reps):
+            graph.replay()
+        end.record(stream)
+        torch.cuda.synchronize()
+        ms_graph = start.elapsed_time(end) / (reps * per_graph)
+        del graph
+        mb = echo.echo_model_bytes_variant(P, n, echo.ECHO_BF16, True, variant)
+        print(json.dumps({"sweep": True, "variant": args.variant, "n_per_rank": n,
+                          "msg_bytes": 2 * n, "calls": calls,
+                          "us_per_call": round(ms * 1e3, 2),
+                          "us_per_call_graph": round(ms_graph * 1e3, 2),
+                          "algbw_GBs": round(2 * n / (ms * 1e-3) / 1e9, 2),
+                          "algbw_graph_GBs": round(2 * n / (ms_graph * 1e-3) / 1e9, 2),
+                          "roofline_frac_graph": round(mb["total"] / (ms_graph * 1e-3) / (peak * 1e9), 4)}),
+              flush=True)
+        h.close()
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--sweep", action="store_true",
+                    help="print one line per message size (2^12..2^29 elements) instead of the benchmark")
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
@@ -415,6 +485,10 @@ def main(argv=None):
         res = run_reference(args, rank, world)
         if res is not None:
             print(json.dumps(res), flush=True)
+        return 0
+    if args.sweep:
+        if rank == 0:
+            run_sweep(args)
         return 0
 
     res = run_echo(args, rank, world, local)

@@ -400,7 +400,7 @@ void free_handle(echo_handle *h)
 
 namespace echo {
 
-int persistent_grid(uint32_t tiles, int resident_per_sm)
+static int sm_count()
 {
     static int sms = 0;
     if (sms == 0) {
@@ -411,12 +411,29 @@ int persistent_grid(uint32_t tiles, int resident_per_sm)
         else
             sms = 148;
     }
-    const long full = static_cast<long>(sms) * (resident_per_sm > 0 ? resident_per_sm : 1);
+    return sms;
+}
+
+int persistent_grid(uint32_t tiles, int resident_per_sm)
+{
+    const long full = static_cast<long>(sm_count()) * (resident_per_sm > 0 ? resident_per_sm : 1);
     const long g = static_cast<long>(tiles) < full ? static_cast<long>(tiles) : full;
     return g < 1 ? 1 : static_cast<int>(g);
 }
 
 int record_error(int code, const char *message) { return set_error(code, "%s", message); }
+
+uint32_t pick_tile_log2(size_t elems, int max_tile, int min_tile, int resident_per_sm)
+{
+    const size_t ctas = static_cast<size_t>(sm_count()) * (resident_per_sm > 0 ? resident_per_sm : 1);
+    size_t t = static_cast<size_t>(max_tile);
+    while (t > static_cast<size_t>(min_tile) && elems / t < 4 * ctas)
+        t /= 2;
+    uint32_t lg = 0;
+    while ((size_t(1) << lg) < t)
+        lg++;
+    return lg;
+}
 
 cudaError_t prepare_kernel(const void *kernel, int threads, int smem_bytes, int *resident)
 {

@@ -104,6 +104,22 @@ __device__ __forceinline__ void fence_proxy_async_smem()
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// Programmatic dependent launch. Each kernel is launched allowed to start
+// before its predecessor in the stream has finished; it sets up its own
+// barriers, then waits here until every prerequisite grid has completed and
+// its memory is visible, before it touches any global memory. Right after,
+// it lets its own successor start launching (that successor waits the same
+// way). Without the launch attribute both are no-ops.
+__device__ __forceinline__ void wait_for_predecessor()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+__device__ __forceinline__ void allow_successor()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ void mbar_arrive(uint64_t *bar)
 {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");

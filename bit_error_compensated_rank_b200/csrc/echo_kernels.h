@@ -64,6 +64,7 @@ struct K1Args {
     size_t n;
     size_t scale_stride;     // bytes between ranks' scale rows (n/32 rounded up to 16)
     uint32_t chunk_begin, chunk_end;
+    uint32_t tile, tile_log2; // set by the launcher: this launch's tile length
     uint32_t groups_per_seg; // n / P / 32: owner of group g is g / groups_per_seg
     float lambda, one_minus_lambda;
     float *eps;              // sender feedback: every rank's rounding-#1 error [P][n]
@@ -83,6 +84,7 @@ struct K2Args {
     size_t n;
     size_t scale_stride;
     uint32_t chunk_begin, chunk_end;
+    uint32_t tile, tile_log2; // set by the launcher: this launch's tile length
     float beta_f, one_minus_beta_f, beta_s, one_minus_beta_s;
     float lambda, one_minus_lambda;
     int P;
@@ -97,6 +99,7 @@ struct K3Args {
     RankOutPtrs out;         // P rank outputs (bf16 or binary32)
     size_t n;
     uint32_t chunk_begin, chunk_end;
+    uint32_t tile, tile_log2; // set by the launcher: this launch's tile length
     int P;
     bool bf16;
     PipeCtl ctl;
@@ -110,6 +113,11 @@ cudaError_t launch_k3_gather_dequant(const K3Args &a, cudaStream_t st);
 // Persistent grid: one CTA per tile up to (SMs x resident CTAs per SM).
 int persistent_grid(uint32_t tiles, int resident_per_sm);
 
+// log2 of a launch's tile length: the largest power of two in
+// [min_tile, max_tile] that still gives every CTA of a full persistent grid
+// about four tiles, so mid-sized tensors keep the pipelines fed and balanced.
+uint32_t pick_tile_log2(size_t elems, int max_tile, int min_tile, int resident_per_sm);
+
 // Set a kernel's dynamic shared memory and return its resident CTAs per SM
 // (cached by the caller per instantiation).
 cudaError_t prepare_kernel(const void *kernel, int threads, int smem_bytes, int *resident);
@@ -117,5 +125,24 @@ cudaError_t prepare_kernel(const void *kernel, int threads, int smem_bytes, int 
 // Record `message` as this thread's last error (echo_last_error /
 // echo_last_status) and return `code`.
 int record_error(int code, const char *message);
+
+// Launch `kern` with programmatic stream serialisation: it may begin (set up
+// its barriers) while the previous kernel in the stream finishes; the kernel
+// itself waits (wait_for_predecessor) before touching global memory.
+template <typename Arg>
+cudaError_t launch_chained(void (*kern)(Arg), int grid, int threads, int smem, cudaStream_t st, const Arg &a)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cfg.blockDim = dim3(static_cast<unsigned>(threads));
+    cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, a);
+}
 
 } // namespace echo

@@ -63,7 +63,6 @@ struct K1Shape {
     static constexpr int kEpsOff = kStateOff + (COMP ? 2 * kTile * 4 : 0); // P error tiles
     static constexpr int kStageBytes = kEpsOff + (EF ? P * kTile * 4 : 0);
     static constexpr int kSmem = kStages * kStageBytes + 2 * kStages * 8;
-    static constexpr int kChunksPerTile = kTile / kChunk;   // a multiple of 32
     static_assert(kSmem <= ECHO_SMEM_BUDGET, "kernel 1 stages exceed shared memory");
 };
 
@@ -103,7 +102,10 @@ __global__ void __launch_bounds__(kThreads)
     const uint32_t lane = tid & 31u;
     const size_t e0 = static_cast<size_t>(a.chunk_begin) * kChunk;
     const size_t e1 = static_cast<size_t>(a.chunk_end) * kChunk;
-    const uint32_t ntiles = static_cast<uint32_t>((e1 - e0 + Sh::kTile - 1) / Sh::kTile);
+    // the tile length of this launch: a power of two <= Sh::kTile (smem strides keep Sh::kTile)
+    const uint32_t tile = a.tile;
+    const uint32_t cpt_log2 = a.tile_log2 - 3; // chunks per tile = 2^cpt_log2
+    const uint32_t ntiles = static_cast<uint32_t>((e1 - e0 + tile - 1) >> a.tile_log2);
     const uint32_t mine = blockIdx.x < ntiles ? (ntiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
 
     if (tid == 0) {
@@ -114,14 +116,15 @@ __global__ void __launch_bounds__(kThreads)
         mbar_init_fence();
     }
     __syncthreads();
+    wait_for_predecessor(); // nothing above touches global memory
+    allow_successor();
 
     if (warp == kConsumerWarps) { // producer
         if (lane == 0)
             produce_tiles<S>(full, empty, mine, a.ctl.stall, a.ctl.wait_cycles, a.ctl.status, kStatusTimeoutK1,
                              [&](uint32_t i) {
-                                 const size_t el0 = e0 + static_cast<size_t>(blockIdx.x + i * gridDim.x) * Sh::kTile;
-                                 const uint32_t cnt = static_cast<uint32_t>(
-                                     e1 - el0 < size_t(Sh::kTile) ? e1 - el0 : Sh::kTile);
+                                 const size_t el0 = e0 + static_cast<size_t>(blockIdx.x + i * gridDim.x) * tile;
+                                 const uint32_t cnt = static_cast<uint32_t>(e1 - el0 < size_t(tile) ? e1 - el0 : tile);
                                  uint8_t *stage = smem + (i % S) * Sh::kStageBytes;
                                  uint64_t *bar = &full[i % S];
                                  mbar_arrive_expect_tx(bar, cnt * Sh::kStageBytes / Sh::kTile);
@@ -149,16 +152,16 @@ __global__ void __launch_bounds__(kThreads)
         const uint32_t s = i % S;
         if (!warp_wait(&full[s], (i / S) & 1u, a.ctl.wait_cycles, a.ctl.status, kStatusTimeoutK1))
             return;
-        const uint32_t tile_chunk0 = static_cast<uint32_t>(e0 / kChunk) + (blockIdx.x + i * gridDim.x) * (Sh::kTile / kChunk);
-        const uint32_t cnt_chunks = min(static_cast<uint32_t>(Sh::kChunksPerTile), a.chunk_end - tile_chunk0);
+        const uint32_t tile_chunk0 = static_cast<uint32_t>(e0 / kChunk) + ((blockIdx.x + i * gridDim.x) << cpt_log2);
+        const uint32_t cnt_chunks = min(1u << cpt_log2, a.chunk_end - tile_chunk0);
         const uint8_t *stage = smem + s * Sh::kStageBytes;
         const float *fs = reinterpret_cast<const float *>(stage + Sh::kStateOff);
         const float *es = reinterpret_cast<const float *>(stage + Sh::kEpsOff);
 
 #pragma unroll 2
-        for (uint32_t it = tid; it < static_cast<uint32_t>(P * Sh::kChunksPerTile); it += kConsumers) {
-            const uint32_t r = it / Sh::kChunksPerTile; // warp-uniform
-            const uint32_t c = it % Sh::kChunksPerTile;
+        for (uint32_t it = tid; it < (static_cast<uint32_t>(P) << cpt_log2); it += kConsumers) {
+            const uint32_t r = it >> cpt_log2; // warp-uniform (a tile has >= 32 chunks)
+            const uint32_t c = it & ((1u << cpt_log2) - 1u);
             const bool active = c < cnt_chunks;
             const uint32_t chunk = tile_chunk0 + c;
             const uint32_t g = chunk / kLanesPerGroup;
@@ -228,9 +231,11 @@ cudaError_t launch_p(const K1Args &a, cudaStream_t st)
             return e;
     }
     const size_t elems = static_cast<size_t>(a.chunk_end - a.chunk_begin) * kChunk;
-    const uint32_t tiles = static_cast<uint32_t>((elems + Sh::kTile - 1) / Sh::kTile);
-    kern<<<persistent_grid(tiles, resident), kThreads, Sh::kSmem, st>>>(a);
-    return cudaGetLastError();
+    K1Args b = a;
+    b.tile_log2 = pick_tile_log2(elems, Sh::kTile, 256, resident);
+    b.tile = 1u << b.tile_log2;
+    const uint32_t tiles = static_cast<uint32_t>((elems + b.tile - 1) >> b.tile_log2);
+    return launch_chained(kern, persistent_grid(tiles, resident), kThreads, Sh::kSmem, st, b);
 }
 
 template <int P, bool BF16>

@@ -87,7 +87,9 @@ __global__ void __launch_bounds__(kThreads)
     const uint32_t lane = tid & 31u;
     const size_t e0 = static_cast<size_t>(a.chunk_begin) * kChunk;
     const size_t e1 = static_cast<size_t>(a.chunk_end) * kChunk;
-    const uint32_t ntiles = static_cast<uint32_t>((e1 - e0 + Sh::kTile - 1) / Sh::kTile);
+    // the tile length of this launch: a power of two <= Sh::kTile (smem strides keep Sh::kTile)
+    const uint32_t tile = a.tile;
+    const uint32_t ntiles = static_cast<uint32_t>((e1 - e0 + tile - 1) >> a.tile_log2);
     const uint32_t mine = blockIdx.x < ntiles ? (ntiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
 
     if (tid == 0) {
@@ -98,6 +100,8 @@ __global__ void __launch_bounds__(kThreads)
         mbar_init_fence();
     }
     __syncthreads();
+    wait_for_predecessor(); // nothing above touches global memory
+    allow_successor();
 
     if (warp == kConsumerWarps) { // producer
         // The scale tile of a ragged last tile is rounded up to 16 bytes;
@@ -106,8 +110,8 @@ __global__ void __launch_bounds__(kThreads)
         if (lane == 0)
             produce_tiles<S>(
                 full, empty, mine, a.ctl.stall, a.ctl.wait_cycles, a.ctl.status, kStatusTimeoutK2, [&](uint32_t i) {
-                    const size_t el0 = e0 + static_cast<size_t>(blockIdx.x + i * gridDim.x) * Sh::kTile;
-                    const uint32_t cnt = static_cast<uint32_t>(e1 - el0 < size_t(Sh::kTile) ? e1 - el0 : Sh::kTile);
+                    const size_t el0 = e0 + static_cast<size_t>(blockIdx.x + i * gridDim.x) * tile;
+                    const uint32_t cnt = static_cast<uint32_t>(e1 - el0 < size_t(tile) ? e1 - el0 : tile);
                     const uint32_t sc_bytes = round16(cnt / kGroup);
                     uint8_t *stage = smem + (i % S) * Sh::kStageBytes;
                     uint64_t *bar = &full[i % S];
@@ -130,10 +134,10 @@ __global__ void __launch_bounds__(kThreads)
         const uint32_t sidx = i % S;
         if (!warp_wait(&full[sidx], (i / S) & 1u, a.ctl.wait_cycles, a.ctl.status, kStatusTimeoutK2))
             return;
-        const uint32_t tile_chunk0 = static_cast<uint32_t>(e0 / kChunk) + (blockIdx.x + i * gridDim.x) * (Sh::kTile / kChunk);
+        const uint32_t tile_chunk0 = static_cast<uint32_t>(e0 / kChunk) + (blockIdx.x + i * gridDim.x) * (tile / kChunk);
         const uint8_t *stage = smem + sidx * Sh::kStageBytes;
 #pragma unroll 1
-        for (int j = 0; j < Sh::kChunks; j++) {
+        for (uint32_t j = 0; j < tile / (kChunk * kConsumers); j++) {
             const uint32_t c = tid + j * kConsumers; // chunk within the tile
             const uint32_t chunk = tile_chunk0 + c;
             const bool active = chunk < a.chunk_end;
@@ -227,9 +231,11 @@ cudaError_t launch_p(const K2Args &a, cudaStream_t st)
             return e;
     }
     const size_t elems = static_cast<size_t>(a.chunk_end - a.chunk_begin) * kChunk;
-    const uint32_t tiles = static_cast<uint32_t>((elems + Sh::kTile - 1) / Sh::kTile);
-    kern<<<persistent_grid(tiles, resident), kThreads, Sh::kSmem, st>>>(a);
-    return cudaGetLastError();
+    K2Args b = a;
+    b.tile_log2 = pick_tile_log2(elems, Sh::kTile, kConsumers * kChunk, resident);
+    b.tile = 1u << b.tile_log2;
+    const uint32_t tiles = static_cast<uint32_t>((elems + b.tile - 1) >> b.tile_log2);
+    return launch_chained(kern, persistent_grid(tiles, resident), kThreads, Sh::kSmem, st, b);
 }
 
 template <int P>

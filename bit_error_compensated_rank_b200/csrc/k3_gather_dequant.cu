@@ -43,7 +43,6 @@ struct K3Shape {
     static constexpr int kBarOff = kOutOff + kOutBufs * kOutBytes;
     static constexpr int kSmem = kBarOff + (2 * kInStages + 2 * kOutBufs) * 8;
     static_assert(kSmem <= ECHO_SMEM_BUDGET, "kernel 3 buffers exceed shared memory");
-    static constexpr int kChunksPerThread = kTile / kChunk / kConsumers;
 };
 
 __device__ __forceinline__ uint32_t round16(uint32_t x) { return (x + 15u) & ~15u; }
@@ -66,11 +65,13 @@ __global__ void __launch_bounds__(kThreads)
     const uint32_t lane = tid & 31u;
     const size_t e0 = static_cast<size_t>(a.chunk_begin) * kChunk;
     const size_t e1 = static_cast<size_t>(a.chunk_end) * kChunk;
-    const uint32_t ntiles = static_cast<uint32_t>((e1 - e0 + Sh::kTile - 1) / Sh::kTile);
+    // the tile length of this launch: a power of two <= Sh::kTile (smem strides keep Sh::kTile)
+    const uint32_t tile = a.tile;
+    const uint32_t ntiles = static_cast<uint32_t>((e1 - e0 + tile - 1) >> a.tile_log2);
     const uint32_t mine = blockIdx.x < ntiles ? (ntiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
-    auto tile_start = [&](uint32_t i) { return e0 + static_cast<size_t>(blockIdx.x + i * gridDim.x) * Sh::kTile; };
+    auto tile_start = [&](uint32_t i) { return e0 + static_cast<size_t>(blockIdx.x + i * gridDim.x) * tile; };
     auto tile_count = [&](size_t el0) {
-        return static_cast<uint32_t>(e1 - el0 < size_t(Sh::kTile) ? e1 - el0 : Sh::kTile);
+        return static_cast<uint32_t>(e1 - el0 < size_t(tile) ? e1 - el0 : tile);
     };
 
     if (tid == 0) {
@@ -85,6 +86,8 @@ __global__ void __launch_bounds__(kThreads)
         mbar_init_fence();
     }
     __syncthreads();
+    wait_for_predecessor(); // nothing above touches global memory
+    allow_successor();
 
     if (warp == kLoadWarp) {
         // scale rows are padded to 16 bytes, so a ragged tile's scale copy may
@@ -139,8 +142,8 @@ __global__ void __launch_bounds__(kThreads)
             return;
         const uint8_t *stage = smem + s * Sh::kInBytes;
         uint8_t *out = smem + Sh::kOutOff + b * Sh::kOutBytes;
-#pragma unroll
-        for (int j = 0; j < Sh::kChunksPerThread; j++) {
+#pragma unroll 2
+        for (uint32_t j = 0; j < tile / (kChunk * kConsumers); j++) {
             const uint32_t c = tid + j * kConsumers;
             const uint32_t w = reinterpret_cast<const uint32_t *>(stage)[c];
             const float st = step_of(stage[Sh::kCodeBytes + c / kLanesPerGroup]);
@@ -177,9 +180,11 @@ cudaError_t launch_p(const K3Args &a, cudaStream_t st)
             return e;
     }
     const size_t elems = static_cast<size_t>(a.chunk_end - a.chunk_begin) * kChunk;
-    const uint32_t tiles = static_cast<uint32_t>((elems + Sh::kTile - 1) / Sh::kTile);
-    kern<<<persistent_grid(tiles, resident), kThreads, Sh::kSmem, st>>>(a);
-    return cudaGetLastError();
+    K3Args b = a;
+    b.tile_log2 = pick_tile_log2(elems, Sh::kTile, kConsumers * kChunk, resident);
+    b.tile = 1u << b.tile_log2;
+    const uint32_t tiles = static_cast<uint32_t>((elems + b.tile - 1) >> b.tile_log2);
+    return launch_chained(kern, persistent_grid(tiles, resident), kThreads, Sh::kSmem, st, b);
 }
 
 template <int P>

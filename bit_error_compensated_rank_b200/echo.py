@@ -281,14 +281,27 @@ class Echo:
 
     def __init__(self, P: int, n: int, dtype: int = ECHO_BF16, group: int = ECHO_GROUP):
         self.P, self.n, self.dtype = P, n, dtype
+        self._arrays = {}
         self.h = echo_create(P, n, group, dtype)
 
+    def _ptrs(self, tensors) -> ctypes.Array:
+        """The tensors' device addresses as a C array, kept for reuse: a
+        layer that reduces the same buffers every step pays the marshalling
+        once."""
+        key = tuple(t.data_ptr() for t in tensors)
+        arr = self._arrays.get(key)
+        if arr is None:
+            if len(self._arrays) >= 64:
+                self._arrays.clear()
+            arr = self._arrays[key] = _ptr_array(key)
+        return arr
+
     def allreduce(self, tensors, phase: int = ECHO_FWD, stream=None) -> None:
-        echo_allreduce(self.h, [t.data_ptr() for t in tensors], phase, _stream(stream))
+        _check(_lib.echo_allreduce(self.h, self._ptrs(tensors), phase, _stream(stream)))
 
     def allreduce_out(self, send, recv, phase: int = ECHO_FWD, stream=None) -> None:
-        echo_allreduce_out(self.h, [t.data_ptr() for t in send], [t.data_ptr() for t in recv],
-                           phase, _stream(stream))
+        _check(_lib.echo_allreduce_out(self.h, self._ptrs(send), self._ptrs(recv), phase,
+                                       _stream(stream)))
 
     def allreduce_host(self, host_send, host_recv, phase: int = ECHO_FWD, stream=None) -> None:
         echo_allreduce_host(self.h, [t.data_ptr() for t in host_send], host_recv.data_ptr(),
