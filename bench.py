@@ -256,6 +256,11 @@ NCU_TRAFFIC = {
 }
 
 
+def workload_name(args) -> str:
+    name = WORKLOAD if args.group == 32 else WORKLOAD.replace("group 32", f"group {args.group}")
+    return name if args.variant == "default" else f"{name}, variant {args.variant}"
+
+
 def _source_hash(path: str) -> str:
     import hashlib
     with open(path, "rb") as fh:
@@ -280,10 +285,10 @@ def run_echo(args, rank: int, world: int, local: int) -> dict | None:
     for r in range(P):
         wl.torch_outlier_gaussian_(send[r], seed=SEED + 1000 * rank, call=0, rank=r)
     variant = VARIANTS[args.variant]
-    h = echo.Echo(P, n, echo.ECHO_BF16)
+    h = echo.Echo(P, n, echo.ECHO_BF16, args.group)
     if variant:
         h.set_variant(variant)
-    mb = echo.echo_model_bytes_variant(P, n, echo.ECHO_BF16, True, variant)
+    mb = echo.echo_model_bytes_ex(P, n, args.group, echo.ECHO_BF16, True, variant)
     torch.cuda.synchronize()
 
     for _ in range(args.warmup):
@@ -324,7 +329,8 @@ def run_echo(args, rank: int, world: int, local: int) -> dict | None:
     achieved = k_bytes[dom] / (k_avg[dom] * 1e-3) / 1e9
     src = os.path.join(ROOT, "bit_error_compensated_rank_b200", "csrc", names[dom] + ".cu")
     traffic = None
-    rec = NCU_TRAFFIC.get(names[dom]) if variant == 0 else None  # captured for the default variant
+    # captured for the default variant and group
+    rec = NCU_TRAFFIC.get(names[dom]) if variant == 0 and args.group == 32 else None
     if rec and rec["source_sha"] == _source_hash(src):
         traffic = round(rec["bytes_per_elem"] * n)
 
@@ -338,8 +344,8 @@ def run_echo(args, rank: int, world: int, local: int) -> dict | None:
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": WORKLOAD + ("" if variant == 0 else f", variant {args.variant}"),
-                   "variant": args.variant, "P": P, "n_per_rank": n, "group": 32,
+        "config": {"workload": workload_name(args),
+                   "variant": args.variant, "P": P, "n_per_rank": n, "group": args.group,
                    "parallelism": f"{world} independent replica(s), ranks simulated in HBM",
                    "l2": "inputs larger than L2 (8 GiB of partials per GPU vs 126 MB L2)"},
         "hbm_roofline_frac": round(call_frac, 4),
@@ -410,7 +416,7 @@ def run_sweep(args) -> None:
     variant = VARIANTS[args.variant]
     for k in range(12, 30):
         n = 1 << k
-        h = echo.Echo(P, n, echo.ECHO_BF16)
+        h = echo.Echo(P, n, echo.ECHO_BF16, args.group)
         if variant:
             h.set_variant(variant)
         s_views = [t[:n] for t in send]
@@ -448,8 +454,8 @@ def run_sweep(args) -> None:
         torch.cuda.synchronize()
         ms_graph = start.elapsed_time(end) / (reps * per_graph)
         del graph
-        mb = echo.echo_model_bytes_variant(P, n, echo.ECHO_BF16, True, variant)
-        print(json.dumps({"sweep": True, "variant": args.variant, "n_per_rank": n,
+        mb = echo.echo_model_bytes_ex(P, n, args.group, echo.ECHO_BF16, True, variant)
+        print(json.dumps({"sweep": True, "variant": args.variant, "group": args.group, "n_per_rank": n,
                           "msg_bytes": 2 * n, "calls": calls,
                           "us_per_call": round(ms * 1e3, 2),
                           "us_per_call_graph": round(ms_graph * 1e3, 2),
@@ -474,6 +480,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--variant", choices=sorted(VARIANTS), default="default",
                     help="where rounding errors are fed back (default: the method as read)")
+    ap.add_argument("--group", type=int, choices=[16, 32, 64, 128], default=32,
+                    help="elements per scale (default 32, the method as read)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -80,17 +80,21 @@ int check_shape(int P, size_t n, int group, int dtype)
     if (n == 0 || n % (static_cast<size_t>(P) * static_cast<size_t>(group)) != 0)
         return set_error(ECHO_ERR_INVALID, "n = %zu must be a positive multiple of P*group = %d", n,
                          P * group);
-    if (group != ECHO_GROUP)
-        return set_error(ECHO_ERR_UNSUPPORTED, "group = %d: only %d is built", group, ECHO_GROUP);
+    if (group != 16 && group != 32 && group != 64 && group != 128)
+        return set_error(ECHO_ERR_UNSUPPORTED, "group = %d: the built group sizes are 16, 32, 64 and 128", group);
+    // Every rank's code row (n/2 bytes) must start on a 16-byte boundary for
+    // the bulk copies; only group 16 with an odd P can miss it.
+    if (n % 32 != 0)
+        return set_error(ECHO_ERR_UNSUPPORTED, "n = %zu: code rows need n to be a multiple of 32", n);
     if (n > kMaxN)
         return set_error(ECHO_ERR_UNSUPPORTED, "n = %zu exceeds the supported maximum %zu", n, kMaxN);
     return ECHO_OK;
 }
 
-void model_bytes(int P, size_t n, int dtype, bool enable, int variant, uint64_t out[4])
+void model_bytes(int P, size_t n, int group, int dtype, bool enable, int variant, uint64_t out[4])
 {
     const uint64_t b = elem_bytes(dtype);
-    const uint64_t wire = static_cast<uint64_t>(n) / 32 * 17; // n * 17/32
+    const uint64_t wire = static_cast<uint64_t>(n) / 2 + static_cast<uint64_t>(n) / group; // n * (1/2 + 1/G)
     const uint64_t state = enable ? 8 * static_cast<uint64_t>(n) : 0;
     // the owner-sum variant reads f, s in kernel 2 only
     const uint64_t k1_state = (variant & ECHO_VARIANT_OWNER_SUM) ? 0 : state;
@@ -108,12 +112,14 @@ struct echo_handle {
     int P = 0;
     size_t n = 0;
     int dtype = ECHO_BF16;
+    int group = ECHO_GROUP;     // elements per scale
+    uint32_t lanes_log2 = 2;    // log2(group / 8)
     int device = 0;
     uint8_t *codes1 = nullptr;  // [P][n/2]
-    uint8_t *scales1 = nullptr; // [P][scale_stride]
+    uint8_t *scales1 = nullptr; // [P][scale_stride], n/group bytes used per rank
     uint8_t *qcodes = nullptr;  // [n/2]
     uint8_t *qscales = nullptr; // [scale_stride]
-    size_t scale_stride = 0;    // n/32 rounded up to 16 bytes (bulk-copy alignment)
+    size_t scale_stride = 0;    // n/group rounded up to 16 bytes (bulk-copy alignment)
     int *dstatus = nullptr;     // device status word written by timed-out waits
     float *state = nullptr;     // [phase][f|s][n]
     float beta_f = 0.5f, beta_s = 0.875f, lambda = 0.5f;
@@ -246,10 +252,10 @@ int fold_timings(echo_handle *h, uint64_t upto)
 int enqueue_call(echo_handle *h, const void *const send[], void *const recv[], int phase, cudaStream_t st,
                  uint32_t cb, uint32_t ce, bool record_events)
 {
-    // Tiles start at multiples of 512 elements from the range start, so every
-    // bulk copy (partials, codes, 16-byte scale rows, state) is 16-byte aligned.
-    if (cb % 64 != 0 || ce < cb)
-        return set_error(ECHO_ERR_INVALID, "internal: element range must start at a multiple of 512");
+    // The range starts at a multiple of 16 groups, so every bulk copy
+    // (partials, codes, 16-byte scale rows, state) is 16-byte aligned.
+    if ((static_cast<size_t>(cb) * echo::kChunk) % (16 * static_cast<size_t>(h->group)) != 0 || ce < cb)
+        return set_error(ECHO_ERR_INVALID, "internal: element range must start at a multiple of 16 groups");
     cudaEvent_t *ev = nullptr;
     if (record_events) {
         if (h->ring_calls >= static_cast<uint64_t>(kTimingRing)) {
@@ -279,7 +285,8 @@ int enqueue_call(echo_handle *h, const void *const send[], void *const recv[], i
     a1.n = h->n;
     a1.chunk_begin = cb;
     a1.chunk_end = ce;
-    a1.groups_per_seg = static_cast<uint32_t>(h->n / h->P / ECHO_GROUP);
+    a1.groups_per_seg = static_cast<uint32_t>(h->n / h->P / h->group);
+    a1.lanes_log2 = a2.lanes_log2 = a3.lanes_log2 = h->lanes_log2;
     a1.lambda = h->lambda;
     a1.one_minus_lambda = 1.0f - h->lambda;
     a1.P = h->P;
@@ -351,7 +358,7 @@ int enqueue_call(echo_handle *h, const void *const send[], void *const recv[], i
 void count_call(echo_handle *h)
 {
     uint64_t mb[4];
-    model_bytes(h->P, h->n, h->dtype, h->enable, h->variant, mb);
+    model_bytes(h->P, h->n, h->group, h->dtype, h->enable, h->variant, mb);
     h->hbm_bytes += mb[0] + mb[1] + mb[2];
     h->link_bytes += mb[3];
     h->calls += 1;
@@ -463,20 +470,20 @@ int echo_model_bytes(int P, size_t n, int dtype, int enable, uint64_t out[4])
         return rc;
     if (!out)
         return set_error(ECHO_ERR_INVALID, "out is NULL");
-    model_bytes(P, n, dtype, enable != 0, 0, out);
+    model_bytes(P, n, ECHO_GROUP, dtype, enable != 0, 0, out);
     return ECHO_OK;
 }
 
-int echo_model_bytes_variant(int P, size_t n, int dtype, int enable, int variant, uint64_t out[4])
+int echo_model_bytes_ex(int P, size_t n, int group, int dtype, int enable, int variant, uint64_t out[4])
 {
-    int rc = check_shape(P, n, ECHO_GROUP, dtype);
+    int rc = check_shape(P, n, group, dtype);
     if (rc != ECHO_OK)
         return rc;
     if (!out)
         return set_error(ECHO_ERR_INVALID, "out is NULL");
     if (variant & ~(ECHO_VARIANT_OWNER_SUM | ECHO_VARIANT_SENDER_EF))
         return set_error(ECHO_ERR_INVALID, "unknown variant bits 0x%x", variant);
-    model_bytes(P, n, dtype, enable != 0, variant, out);
+    model_bytes(P, n, group, dtype, enable != 0, variant, out);
     return ECHO_OK;
 }
 
@@ -557,7 +564,11 @@ echo_handle *echo_create(int P, size_t n, int group, int dtype)
     h->P = P;
     h->n = n;
     h->dtype = dtype;
-    h->scale_stride = (n / ECHO_GROUP + 15) / 16 * 16;
+    h->group = group;
+    h->lanes_log2 = 0; // group = 8 << lanes_log2 (a power of two in [16, 128])
+    while ((8u << h->lanes_log2) != static_cast<uint32_t>(group))
+        h->lanes_log2++;
+    h->scale_stride = (n / group + 15) / 16 * 16;
     cudaError_t e = cudaGetDevice(&h->device);
     if (e != cudaSuccess) {
         cuda_error(e, "cudaGetDevice");
@@ -790,7 +801,7 @@ int echo_get_wire_range(echo_handle *h, int stage, int rank, size_t group_offset
     int rc;
     if ((rc = check_handle(h)) != ECHO_OK || (rc = check_device(h)) != ECHO_OK)
         return rc;
-    const size_t groups = h->n / ECHO_GROUP;
+    const size_t groups = h->n / h->group;
     if (stage != 1 && stage != 2)
         return set_error(ECHO_ERR_INVALID, "stage %d is neither 1 (per-rank wire) nor 2 (requantised)", stage);
     if (stage == 1 && (rank < 0 || rank >= h->P))
@@ -801,7 +812,7 @@ int echo_get_wire_range(echo_handle *h, int stage, int rank, size_t group_offset
     const uint8_t *scales = stage == 1 ? h->scales1 + static_cast<size_t>(rank) * h->scale_stride : h->qscales;
     cudaError_t e = cudaDeviceSynchronize();
     if (e == cudaSuccess && codes_host)
-        e = cudaMemcpy(codes_host, codes + group_offset * (ECHO_GROUP / 2), ngroups * (ECHO_GROUP / 2),
+        e = cudaMemcpy(codes_host, codes + group_offset * (h->group / 2), ngroups * (h->group / 2),
                        cudaMemcpyDeviceToHost);
     if (e == cudaSuccess && scales_host)
         e = cudaMemcpy(scales_host, scales + group_offset, ngroups, cudaMemcpyDeviceToHost);
@@ -813,7 +824,7 @@ int echo_get_wire(echo_handle *h, int stage, int rank, uint8_t *codes_host, uint
     int rc = check_handle(h);
     if (rc != ECHO_OK)
         return rc;
-    return echo_get_wire_range(h, stage, rank, 0, h->n / ECHO_GROUP, codes_host, scales_host);
+    return echo_get_wire_range(h, stage, rank, 0, h->n / h->group, codes_host, scales_host);
 }
 
 int echo_stats(echo_handle *h, uint64_t *link_bytes, uint64_t *model_hbm_bytes, uint64_t *calls)

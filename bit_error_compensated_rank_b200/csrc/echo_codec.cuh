@@ -2,23 +2,24 @@
 //
 // Format (fixed readings of the 4-bit segments on [rit.work "Echo 4-bit GPU
 // communication", section "How Echo returns the error to later calls"]):
-// groups of 32 consecutive elements share a power-of-two scale 2^e, stored
+// groups of G consecutive elements (32 by default; 16, 64 and 128 are the
+// group-size variants) share a power-of-two scale 2^e, stored
 // as the byte e+127, e the smallest integer >= -127 with max|v| <= 7*2^e;
 // codes are round(v/2^e), halves to even, in [-7, 7]; two codes per byte,
 // element 2j in the low nibble, two's complement.
 //
 // Every helper here is exact integer or power-of-two arithmetic; the only
-// rounding is the conversion to the nearest code (cvt.rni), which rounds
-// halves to even.
+// rounding is the choice of the nearest code (code_bits), which rounds halves
+// to even.
 #pragma once
 
 #include <cstdint>
 
 namespace echo {
 
-constexpr int kGroup = 32;          // elements per scale
 constexpr int kChunk = 8;           // elements per thread (one 32-bit code word)
-constexpr int kLanesPerGroup = kGroup / kChunk;
+constexpr int kMinGroup = 16;       // elements per scale: 16, 32, 64 or 128
+constexpr int kMaxGroup = 128;      // (a group spans 2, 4, 8 or 16 lanes)
 constexpr int kMaxRanks = 16;
 
 struct RankPtrs {
@@ -112,12 +113,13 @@ __device__ __forceinline__ float code_at(const Unpacked &u, int k)
     return __fsub_rn(__uint_as_float(bits), kRoundPlus8);
 }
 
-// Absolute maximum over the 4 lanes (32 elements) of a group. The lanes of a
-// group are 4 consecutive lanes of the warp; every lane of the warp calls it.
-__device__ __forceinline__ float group_absmax(float a)
+// Absolute maximum over the 2^lanes_log2 consecutive lanes (8 elements each)
+// that form a group. Every lane of the warp calls it with the same
+// lanes_log2.
+__device__ __forceinline__ float group_absmax(float a, uint32_t lanes_log2)
 {
-    a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, 1));
-    a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, 2));
+    for (uint32_t d = 1; d < (1u << lanes_log2); d <<= 1)
+        a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, d));
     return a;
 }
 

@@ -60,12 +60,13 @@ struct K1Args {
     const float *f;          // phase state, fast estimate [n]
     const float *s;          // phase state, slow estimate [n]
     uint8_t *codes;          // stage-1 wire codes [P][n/2]
-    uint8_t *scales;         // stage-1 wire scale bytes [P][scale_stride]
+    uint8_t *scales;         // stage-1 wire scale bytes [P][scale_stride], n/G per rank
     size_t n;
     size_t scale_stride;     // bytes between ranks' scale rows (n/32 rounded up to 16)
     uint32_t chunk_begin, chunk_end;
     uint32_t tile, tile_log2; // set by the launcher: this launch's tile length
-    uint32_t groups_per_seg; // n / P / 32: owner of group g is g / groups_per_seg
+    uint32_t lanes_log2;     // log2(G / 8): lanes per group
+    uint32_t groups_per_seg; // n / P / G: owner of group g is g / groups_per_seg
     float lambda, one_minus_lambda;
     float *eps;              // sender feedback: every rank's rounding-#1 error [P][n]
     int P;
@@ -85,6 +86,7 @@ struct K2Args {
     size_t scale_stride;
     uint32_t chunk_begin, chunk_end;
     uint32_t tile, tile_log2; // set by the launcher: this launch's tile length
+    uint32_t lanes_log2;     // log2(G / 8): lanes per group
     float beta_f, one_minus_beta_f, beta_s, one_minus_beta_s;
     float lambda, one_minus_lambda;
     int P;
@@ -100,6 +102,7 @@ struct K3Args {
     size_t n;
     uint32_t chunk_begin, chunk_end;
     uint32_t tile, tile_log2; // set by the launcher: this launch's tile length
+    uint32_t lanes_log2;     // log2(G / 8): lanes per group
     int P;
     bool bf16;
     PipeCtl ctl;

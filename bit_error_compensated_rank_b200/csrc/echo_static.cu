@@ -167,6 +167,7 @@ extern "C" int echo_allreduce_static(int P, size_t n, int dtype, void *const ran
     a1.chunk_begin = 0;
     a1.chunk_end = chunks;
     a1.groups_per_seg = static_cast<uint32_t>(n / P / ECHO_GROUP);
+    a1.lanes_log2 = a2.lanes_log2 = a3.lanes_log2 = 2; // groups of 32: 4 lanes
     a1.lambda = lambda;
     a1.one_minus_lambda = 1.0f - lambda;
     a1.P = P;

@@ -11,7 +11,7 @@
 //
 // Layout: the rank partials are P separate buffers of n elements; the output
 // is the stage-1 wire, codes [P][n/2] (two per byte) and scale bytes
-// [P][scale_stride]; the sender errors are [P][n] binary32.
+// [P][scale_stride] (n/G per rank); the sender errors are [P][n] binary32.
 //
 // Pipeline (warp-specialised, persistent): a CTA takes tiles of kTile
 // consecutive elements. One producer warp bulk-copies the P partial tiles
@@ -19,8 +19,8 @@
 // stage of a kStages ring in shared memory (mbarrier full[s] counts the
 // bytes); eight consumer warps compute from shared memory and release the
 // stage on mbarrier empty[s]. A lane owns 8 consecutive elements of one rank;
-// 4 lanes form a group and find its maximum with two shuffles; codes leave as
-// one coalesced 32-bit store per lane.
+// G/8 lanes form a group and find its maximum with log2(G/8) shuffles; codes
+// leave as one coalesced 32-bit store per lane.
 //
 // Algorithmic HBM bytes per element of n: P*b (partials) + 8 (f, s; each
 // element is corrected by exactly one rank) read, P*17/32 written; sender
@@ -164,7 +164,7 @@ __global__ void __launch_bounds__(kThreads)
             const uint32_t c = it & ((1u << cpt_log2) - 1u);
             const bool active = c < cnt_chunks;
             const uint32_t chunk = tile_chunk0 + c;
-            const uint32_t g = chunk / kLanesPerGroup;
+            const uint32_t g = chunk >> a.lanes_log2;
 
             float v[kChunk];
             load_chunk<BF16>(stage + r * Sh::kXBytes + c * (kChunk * Sh::kEB), v);
@@ -188,7 +188,7 @@ __global__ void __launch_bounds__(kThreads)
             // max |v| as a tree (fmax is exact, so the order is free)
             const float m01 = fmaxf(fabsf(v[0]), fabsf(v[1])), m23 = fmaxf(fabsf(v[2]), fabsf(v[3]));
             const float m45 = fmaxf(fabsf(v[4]), fabsf(v[5])), m67 = fmaxf(fabsf(v[6]), fabsf(v[7]));
-            const float amax = group_absmax(fmaxf(fmaxf(m01, m23), fmaxf(m45, m67)));
+            const float amax = group_absmax(fmaxf(fmaxf(m01, m23), fmaxf(m45, m67)), a.lanes_log2);
             const uint32_t byte = scale_byte(amax);
             const float inv = inv_step_of(byte);
             uint32_t qb[kChunk];
@@ -198,7 +198,7 @@ __global__ void __launch_bounds__(kThreads)
             const uint32_t word = pack8_bits(qb);
             if (active) {
                 reinterpret_cast<uint32_t *>(a.codes)[static_cast<size_t>(r) * code_words + chunk] = word;
-                if ((lane & 3u) == 0)
+                if ((lane & ((1u << a.lanes_log2) - 1u)) == 0) // the group's first lane
                     a.scales[static_cast<size_t>(r) * a.scale_stride + g] = static_cast<uint8_t>(byte);
                 if (EF) { // the new error v - q*2^e, exact
                     const float st = step_of(byte);

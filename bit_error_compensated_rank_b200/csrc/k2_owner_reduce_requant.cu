@@ -44,7 +44,7 @@ constexpr int kThreads = kConsumers + 32; // + one producer warp
 // P scale tiles, and the f, s tiles.
 constexpr int k2_stage_bytes(int P, bool comp, int chunks)
 {
-    return P * (kConsumers * kChunk * chunks / 2 + kConsumers * kChunk * chunks / kGroup) +
+    return P * (kConsumers * kChunk * chunks / 2 + kConsumers * kChunk * chunks / kMinGroup) +
            (comp ? 2 * kConsumers * kChunk * chunks * 4 : 0);
 }
 
@@ -63,7 +63,7 @@ struct K2Shape {
     static constexpr int kTile = kConsumers * kChunk * kChunks;
     static constexpr int kStages = ECHO_K2_STAGES;
     static constexpr int kCodeBytes = kTile / 2;          // one rank's code tile
-    static constexpr int kScaleBytes = kTile / kGroup;    // one rank's scale tile
+    static constexpr int kScaleBytes = kTile / kMinGroup; // room for one rank's scale tile
     static constexpr int kStateOff = P * (kCodeBytes + kScaleBytes);
     static constexpr int kStageBytes = kStateOff + (COMP ? 2 * kTile * 4 : 0);
     static constexpr int kSmem = kStages * kStageBytes + 2 * kStages * 8;
@@ -112,7 +112,7 @@ __global__ void __launch_bounds__(kThreads)
                 full, empty, mine, a.ctl.stall, a.ctl.wait_cycles, a.ctl.status, kStatusTimeoutK2, [&](uint32_t i) {
                     const size_t el0 = e0 + static_cast<size_t>(blockIdx.x + i * gridDim.x) * tile;
                     const uint32_t cnt = static_cast<uint32_t>(e1 - el0 < size_t(tile) ? e1 - el0 : tile);
-                    const uint32_t sc_bytes = round16(cnt / kGroup);
+                    const uint32_t sc_bytes = round16(cnt >> (a.lanes_log2 + 3));
                     uint8_t *stage = smem + (i % S) * Sh::kStageBytes;
                     uint64_t *bar = &full[i % S];
                     mbar_arrive_expect_tx(bar, P * (cnt / 2 + sc_bytes) + (COMP ? 2 * cnt * 4 : 0));
@@ -120,7 +120,7 @@ __global__ void __launch_bounds__(kThreads)
                     for (int r = 0; r < P; r++) {
                         bulk_load(stage + r * Sh::kCodeBytes, a.codes + r * (a.n / 2) + el0 / 2, cnt / 2, bar);
                         bulk_load(stage + P * Sh::kCodeBytes + r * Sh::kScaleBytes,
-                                  a.scales + r * a.scale_stride + el0 / kGroup, sc_bytes, bar);
+                                  a.scales + r * a.scale_stride + (el0 >> (a.lanes_log2 + 3)), sc_bytes, bar);
                     }
                     if (COMP) {
                         bulk_load(stage + Sh::kStateOff, a.f + el0, cnt * 4, bar);
@@ -141,7 +141,7 @@ __global__ void __launch_bounds__(kThreads)
             const uint32_t c = tid + j * kConsumers; // chunk within the tile
             const uint32_t chunk = tile_chunk0 + c;
             const bool active = chunk < a.chunk_end;
-            const uint32_t g = chunk / kLanesPerGroup;
+            const uint32_t g = chunk >> a.lanes_log2;
 
             float fv[kChunk], sv[kChunk];
             if (COMP) {
@@ -165,7 +165,7 @@ __global__ void __launch_bounds__(kThreads)
 #pragma unroll
             for (int r = 0; r < P; r++) {
                 const uint32_t w = reinterpret_cast<const uint32_t *>(stage + r * Sh::kCodeBytes)[c];
-                const uint32_t b = stage[P * Sh::kCodeBytes + r * Sh::kScaleBytes + c / kLanesPerGroup];
+                const uint32_t b = stage[P * Sh::kCodeBytes + r * Sh::kScaleBytes + (c >> a.lanes_log2)];
                 const float st = step_of(b);
                 const Unpacked u = unpack8(w);
 #pragma unroll
@@ -182,7 +182,7 @@ __global__ void __launch_bounds__(kThreads)
             // Rounding #2 and the error it injects.
             const float m01 = fmaxf(fabsf(S_[0]), fabsf(S_[1])), m23 = fmaxf(fabsf(S_[2]), fabsf(S_[3]));
             const float m45 = fmaxf(fabsf(S_[4]), fabsf(S_[5])), m67 = fmaxf(fabsf(S_[6]), fabsf(S_[7]));
-            const float amax = group_absmax(fmaxf(fmaxf(m01, m23), fmaxf(m45, m67)));
+            const float amax = group_absmax(fmaxf(fmaxf(m01, m23), fmaxf(m45, m67)), a.lanes_log2);
             const uint32_t byte = scale_byte(amax);
             const float inv = inv_step_of(byte);
             const float st = step_of(byte);
@@ -196,7 +196,7 @@ __global__ void __launch_bounds__(kThreads)
 
             if (active) {
                 reinterpret_cast<uint32_t *>(a.qcodes)[chunk] = pack8_bits(qb);
-                if ((lane & 3u) == 0)
+                if ((lane & ((1u << a.lanes_log2) - 1u)) == 0) // the group's first lane
                     a.qscales[g] = static_cast<uint8_t>(byte);
                 if (COMP) {
 #pragma unroll

@@ -36,7 +36,7 @@ struct K3Shape {
     static constexpr int kInStages = ECHO_K3_IN_STAGES;
     static constexpr int kOutBufs = ECHO_K3_OUT_BUFS;
     static constexpr int kCodeBytes = kTile / 2;
-    static constexpr int kScaleBytes = kTile / kGroup;
+    static constexpr int kScaleBytes = kTile / kMinGroup; // room for the tile's scale bytes
     static constexpr int kInBytes = kCodeBytes + kScaleBytes;
     static constexpr int kOutBytes = kTile * kEB;
     static constexpr int kOutOff = kInStages * kInBytes;
@@ -97,12 +97,12 @@ __global__ void __launch_bounds__(kThreads)
                              kStatusTimeoutK3, [&](uint32_t i) {
                                  const size_t el0 = tile_start(i);
                                  const uint32_t cnt = tile_count(el0);
-                                 const uint32_t sc_bytes = round16(cnt / kGroup);
+                                 const uint32_t sc_bytes = round16(cnt >> (a.lanes_log2 + 3));
                                  uint8_t *stage = smem + (i % S) * Sh::kInBytes;
                                  uint64_t *bar = &in_full[i % S];
                                  mbar_arrive_expect_tx(bar, cnt / 2 + sc_bytes);
                                  bulk_load(stage, a.qcodes + el0 / 2, cnt / 2, bar);
-                                 bulk_load(stage + Sh::kCodeBytes, a.qscales + el0 / kGroup, sc_bytes, bar);
+                                 bulk_load(stage + Sh::kCodeBytes, a.qscales + (el0 >> (a.lanes_log2 + 3)), sc_bytes, bar);
                              });
         return;
     }
@@ -146,7 +146,7 @@ __global__ void __launch_bounds__(kThreads)
         for (uint32_t j = 0; j < tile / (kChunk * kConsumers); j++) {
             const uint32_t c = tid + j * kConsumers;
             const uint32_t w = reinterpret_cast<const uint32_t *>(stage)[c];
-            const float st = step_of(stage[Sh::kCodeBytes + c / kLanesPerGroup]);
+            const float st = step_of(stage[Sh::kCodeBytes + (c >> a.lanes_log2)]);
             const Unpacked u = unpack8(w);
             float y[kChunk];
 #pragma unroll

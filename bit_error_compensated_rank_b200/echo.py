@@ -38,7 +38,7 @@ EXPORTED = (
     "echo_get_wire_range", "echo_stats", "echo_model_bytes", "echo_set_timing",
     "echo_last_kernel_ms", "echo_kernel_ms_total", "echo_device_status",
     "echo_allreduce_static", "echo_set_variant", "echo_get_sender_state", "echo_set_sender_state",
-    "echo_model_bytes_variant",
+    "echo_model_bytes_ex",
 )
 
 _vp = ctypes.c_void_p
@@ -82,7 +82,7 @@ def _load():
         "echo_set_variant": (_int, [_vp, _int]),
         "echo_get_sender_state": (_int, [_vp, _int, _int, _sz, _sz, _f32p]),
         "echo_set_sender_state": (_int, [_vp, _int, _int, _f32p]),
-        "echo_model_bytes_variant": (_int, [_int, _sz, _int, _int, _int, _u64p]),
+        "echo_model_bytes_ex": (_int, [_int, _sz, _int, _int, _int, _int, _u64p]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -184,15 +184,16 @@ def echo_get_state_range(h: int, phase: int, offset: int, count: int):
     return f, s
 
 
-def echo_get_wire(h: int, stage: int, rank: int, n: int):
+def echo_get_wire(h: int, stage: int, rank: int, n: int, group: int = ECHO_GROUP):
     codes = np.empty(n // 2, np.uint8)
-    scales = np.empty(n // ECHO_GROUP, np.uint8)
+    scales = np.empty(n // group, np.uint8)
     _check(_lib.echo_get_wire(h, stage, rank, _np(codes, _u8p), _np(scales, _u8p)))
     return codes, scales
 
 
-def echo_get_wire_range(h: int, stage: int, rank: int, group_offset: int, ngroups: int):
-    codes = np.empty(ngroups * ECHO_GROUP // 2, np.uint8)
+def echo_get_wire_range(h: int, stage: int, rank: int, group_offset: int, ngroups: int,
+                        group: int = ECHO_GROUP):
+    codes = np.empty(ngroups * group // 2, np.uint8)
     scales = np.empty(ngroups, np.uint8)
     _check(_lib.echo_get_wire_range(h, stage, rank, group_offset, ngroups,
                                     _np(codes, _u8p), _np(scales, _u8p)))
@@ -212,10 +213,10 @@ def echo_model_bytes(P: int, n: int, dtype: int = ECHO_BF16, enable: bool = True
             "total": out[0] + out[1] + out[2]}
 
 
-def echo_model_bytes_variant(P: int, n: int, dtype: int = ECHO_BF16, enable: bool = True,
-                             variant: int = 0) -> dict:
+def echo_model_bytes_ex(P: int, n: int, group: int = ECHO_GROUP, dtype: int = ECHO_BF16,
+                        enable: bool = True, variant: int = 0) -> dict:
     out = (ctypes.c_uint64 * 4)()
-    _check(_lib.echo_model_bytes_variant(P, n, dtype, int(bool(enable)), variant, out))
+    _check(_lib.echo_model_bytes_ex(P, n, group, dtype, int(bool(enable)), variant, out))
     return {"k1": out[0], "k2": out[1], "k3": out[2], "link": out[3],
             "total": out[0] + out[1] + out[2]}
 
@@ -280,7 +281,7 @@ class Echo:
     :meth:`allreduce` with P device tensors (torch) of n elements each."""
 
     def __init__(self, P: int, n: int, dtype: int = ECHO_BF16, group: int = ECHO_GROUP):
-        self.P, self.n, self.dtype = P, n, dtype
+        self.P, self.n, self.dtype, self.group = P, n, dtype, group
         self._arrays = {}
         self.h = echo_create(P, n, group, dtype)
 
@@ -332,10 +333,10 @@ class Echo:
         return echo_get_state_range(self.h, phase, offset, count)
 
     def get_wire(self, stage: int, rank: int = 0):
-        return echo_get_wire(self.h, stage, rank, self.n)
+        return echo_get_wire(self.h, stage, rank, self.n, self.group)
 
     def get_wire_range(self, stage: int, rank: int, group_offset: int, ngroups: int):
-        return echo_get_wire_range(self.h, stage, rank, group_offset, ngroups)
+        return echo_get_wire_range(self.h, stage, rank, group_offset, ngroups, self.group)
 
     def stats(self) -> dict:
         return echo_stats(self.h)

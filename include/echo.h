@@ -73,11 +73,15 @@ enum {
 /*
  * echo_create - a handle for all-reduces of P ranks x n elements of dtype.
  *   P      number of simulated tensor-parallel ranks, 2..16.
- *   n      elements per rank; n % (P*group) == 0 and n <= 2^34.
- *   group  elements per scale; only 32 is built (else ECHO_ERR_UNSUPPORTED).
+ *   n      elements per rank; n % (P*group) == 0 and n <= 2^34; also
+ *          n % 32 == 0 (16-byte code rows), which only group 16 with an
+ *          odd P can miss (ECHO_ERR_UNSUPPORTED).
+ *   group  elements per scale: 32 (the default reading) or, as group-size
+ *          variants, 16, 64 or 128; anything else ECHO_ERR_UNSUPPORTED. The
+ *          wire then costs 1/2 + 1/group bytes per element.
  *   dtype  ECHO_BF16 or ECHO_FP32: the element type of the rank buffers.
  * Allocates on the current device: stage-1 wire (P x n/2 code bytes and
- * P x n/32 scale bytes), the requantised wire (n/2 + n/32 bytes) and the
+ * P x n/group scale bytes), the requantised wire (n/2 + n/group bytes) and the
  * compensator state (2 phases x 2 estimates x n binary32, zeroed).
  * Returns NULL on any error (see echo_last_error). The handle is bound to the
  * device that was current at creation.
@@ -211,7 +215,7 @@ ECHO_API int echo_get_state_range(echo_handle *h, int phase, size_t offset, size
 
 /*
  * echo_get_wire - synchronous copy of the wire left by the last call.
- *   stage 1: rank's packed codes (n/2 bytes) and scale bytes (n/32);
+ *   stage 1: rank's packed codes (n/2 bytes) and scale bytes (n/group);
  *   stage 2: the requantised total (rank ignored).
  * Either output pointer may be NULL to skip it.
  */
@@ -219,7 +223,7 @@ ECHO_API int echo_get_wire(echo_handle *h, int stage, int rank, uint8_t *codes_h
                   uint8_t *scales_host);
 
 /* Range variant over groups [group_offset, group_offset+ngroups):
- * 16*ngroups code bytes and ngroups scale bytes. */
+ * group/2 * ngroups code bytes and ngroups scale bytes. */
 ECHO_API int echo_get_wire_range(echo_handle *h, int stage, int rank, size_t group_offset,
                         size_t ngroups, uint8_t *codes_host, uint8_t *scales_host);
 
@@ -243,9 +247,11 @@ ECHO_API int echo_stats(echo_handle *h, uint64_t *link_bytes, uint64_t *model_hb
  */
 ECHO_API int echo_model_bytes(int P, size_t n, int dtype, int enable, uint64_t out[4]);
 
-/* The same for a variant: OWNER_SUM drops kernel 1's 8 state bytes,
- * SENDER_EF adds 8P bytes (each rank's error read and written) to kernel 1. */
-ECHO_API int echo_model_bytes_variant(int P, size_t n, int dtype, int enable, int variant, uint64_t out[4]);
+/* The same for any group size and variant: the wire is 1/2 + 1/group bytes
+ * per element; OWNER_SUM drops kernel 1's 8 state bytes; SENDER_EF adds 8P
+ * bytes (each rank's error read and written) to kernel 1. */
+ECHO_API int echo_model_bytes_ex(int P, size_t n, int group, int dtype, int enable, int variant,
+                                 uint64_t out[4]);
 
 /*
  * Kernel timing. echo_set_timing(h, 1) starts a measurement: every later

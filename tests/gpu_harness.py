@@ -63,7 +63,8 @@ class FullCompare:
     """One handle and the oracle side by side on a problem small enough to
     compare in full after every call."""
 
-    def __init__(self, oracle, P, n, dtype: str, params: Params = Params(), variant: int = 0):
+    def __init__(self, oracle, P, n, dtype: str, params: Params = Params(), variant: int = 0,
+                 group: int = G):
         from bit_error_compensated_rank_b200 import echo
         self.echo = echo
         self.oracle = oracle
@@ -71,7 +72,8 @@ class FullCompare:
         self.dtype = dtype
         self.params = params
         self.variant = variant
-        self.h = echo.Echo(P, n, echo.ECHO_BF16 if dtype == "bf16" else echo.ECHO_FP32)
+        self.group = group
+        self.h = echo.Echo(P, n, echo.ECHO_BF16 if dtype == "bf16" else echo.ECHO_FP32, group)
         self.h.set_params(*params_tuple(params))
         if variant:
             self.h.set_variant(variant)
@@ -91,8 +93,8 @@ class FullCompare:
             recv = dev
         t.cuda.synchronize()
         f, s = self.state[phase]
-        ref = self.oracle.allreduce(x, f, s, self.params, want_diag=want_diag, variant=self.variant,
-                                    eps=self.eps[phase])
+        ref = self.oracle.allreduce(x, f, s, self.params, G=self.group, want_diag=want_diag,
+                                    variant=self.variant, eps=self.eps[phase])
         got = from_device(recv)
         if out_of_place:  # the inputs are untouched
             assert_same_bits(from_device(dev), x, "send buffers")
@@ -130,12 +132,13 @@ class SampledCompare:
     """
 
     def __init__(self, oracle, P, n, dtype: str, params: Params = Params(), blocks=None,
-                 block_groups: int = 64, seed: int = 0, variant: int = 0):
+                 block_groups: int = 64, seed: int = 0, variant: int = 0, group: int = G):
         from bit_error_compensated_rank_b200 import echo
         self.echo = echo
         self.oracle = oracle
         self.P, self.n, self.dtype, self.params = P, n, dtype, params
-        ngroups = n // G
+        self.group = group
+        ngroups = n // group
         seg_groups = ngroups // P
         if blocks is None:
             starts = {0, max(0, ngroups - block_groups)}
@@ -155,9 +158,9 @@ class SampledCompare:
         self.blocks = merged
         self.bg = bg
         self.groups = np.concatenate([np.arange(b, b + bg) for b in self.blocks])
-        self.elems = (self.groups[:, None] * G + np.arange(G)[None, :]).reshape(-1)
+        self.elems = (self.groups[:, None] * group + np.arange(group)[None, :]).reshape(-1)
         self.owner = (self.groups // seg_groups).astype(np.int32)
-        self.h = echo.Echo(P, n, echo.ECHO_BF16 if dtype == "bf16" else echo.ECHO_FP32)
+        self.h = echo.Echo(P, n, echo.ECHO_BF16 if dtype == "bf16" else echo.ECHO_FP32, group)
         self.h.set_params(*params_tuple(params))
         self.variant = variant
         if variant:
@@ -182,8 +185,9 @@ class SampledCompare:
         self.h.allreduce(tensors, phase, stream)
         t.cuda.synchronize()
         f, s = self.state[phase]
-        ref = self.oracle.allreduce(x, f, s, self.params, owner=self.owner, variant=self.variant,
-                                    eps=self.eps[phase])
+        G = self.group
+        ref = self.oracle.allreduce(x, f, s, self.params, G=G, owner=self.owner,
+                                    variant=self.variant, eps=self.eps[phase])
         got = self.gather(tensors)
         for r in range(self.P):
             assert_same_bits(got[r], ref["out"], f"output rank {r}")

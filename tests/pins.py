@@ -130,7 +130,7 @@ def _random_groups(count, G, seed):
 def pin_quantizer_bruteforce(orc):
     """Scale byte and every code equal an exhaustive search over exponents and
     codes (ties to even), over ties, subnormals, boundaries and wide ranges."""
-    for G in (32, 8, 2):
+    for G in (32, 16, 64, 128, 8, 2):
         for v in _random_groups(60 if G == 32 else 24, G, seed=G):
             b, q = orc.quantize_group(v)
             bb, bq = bf_quantize(v.tolist())
@@ -223,9 +223,10 @@ def pin_exact_sums_on_grid(orc):
     """With partials already on their 4-bit grid, rounding #1 is exact, the sum
     is exact, and the result equals the exhaustive quantiser applied to the
     exact sum; err = exact sum - result. Covers P from 2 to 16, both dtypes,
-    compensation off and a first call with it on (zero state)."""
-    G = 32
-    for P in (2, 3, 4, 8, 16):
+    compensation off and a first call with it on (zero state); the group-size
+    variants 16, 64 and 128 at P = 2 and 8."""
+    cases = [(P, 32) for P in (2, 3, 4, 8, 16)] + [(P, G) for G in (16, 64, 128) for P in (2, 8)]
+    for P, G in cases:
         ngroups = 2 * P
         m = ngroups * G
         x32, k, e = _grid_partials(P, ngroups, G, seed=P)
@@ -239,7 +240,7 @@ def pin_exact_sums_on_grid(orc):
             for enable in (False, True):
                 f = np.zeros(m, F32)
                 s = np.zeros(m, F32)
-                res = orc.allreduce(x, f, s, Params(enable=enable), want_diag=True)
+                res = orc.allreduce(x, f, s, Params(enable=enable), G=G, want_diag=True)
                 assert res["scales1"].tolist() == (e + 127).tolist()
                 for r in range(P):
                     assert _unpack_ref(res["codes1"][r]) == k[r].reshape(-1).tolist()

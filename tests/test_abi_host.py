@@ -58,9 +58,23 @@ def test_model_bytes_per_element(echo):
     assert abs(f32["total"] / 65536 - (2 * 8 * 4 + 25 * w + 24)) < 1e-12
 
 
+@pytest.mark.parametrize("group", [16, 32, 64, 128])
+def test_model_bytes_group_sizes(echo, group):
+    # the wire costs 1/2 + 1/group bytes per element, the rest is unchanged
+    P, n = 8, 1 << 29
+    mb = echo.echo_model_bytes_ex(P, n, group, echo.ECHO_BF16, True, 0)
+    w = 0.5 + 1 / group
+    assert mb["k1"] == round((P * 2 + 8 + P * w) * n)
+    assert mb["k2"] == round((P * w + 16 + w) * n)
+    assert mb["k3"] == round((P * w + P * 2) * n)
+    assert mb["link"] == round(2 * (P - 1) * w * n)
+
+
 @pytest.mark.parametrize("P,n,group,dtype,status", [
     (1, 64, 32, 0, -1), (17, 17 * 32, 32, 0, -1), (2, 0, 32, 0, -1), (2, 96, 32, 0, -1),
-    (4, 4 * 32 * 3 + 32, 32, 0, -1), (2, 64, 32, 7, -1), (2, 128, 64, 0, -2),
+    (4, 4 * 32 * 3 + 32, 32, 0, -1), (2, 64, 32, 7, -1), (2, 192, 48, 0, -2),
+    (2, 512, 256, 0, -2), (2, 64, 8, 0, -2), (4, 4 * 64 * 3 + 64, 64, 0, -1),
+    (5, 5 * 16, 16, 0, -2),
     (2, 1 << 35, 32, 0, -2), (2, 64, 0, 0, -1),
 ])
 def test_create_rejects_bad_shapes(echo, P, n, group, dtype, status):

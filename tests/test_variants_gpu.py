@@ -80,9 +80,9 @@ def test_sender_state_checkpoint_and_reset(oracle):
 def test_variant_bytes_model():
     from bit_error_compensated_rank_b200 import echo
     P, n = 8, 1 << 29
-    base = echo.echo_model_bytes_variant(P, n, echo.ECHO_BF16, True, 0)
-    osum = echo.echo_model_bytes_variant(P, n, echo.ECHO_BF16, True, OWNER_SUM)
-    ef = echo.echo_model_bytes_variant(P, n, echo.ECHO_BF16, True, SENDER_EF)
+    base = echo.echo_model_bytes_ex(P, n, echo.ECHO_GROUP, echo.ECHO_BF16, True, 0)
+    osum = echo.echo_model_bytes_ex(P, n, echo.ECHO_GROUP, echo.ECHO_BF16, True, OWNER_SUM)
+    ef = echo.echo_model_bytes_ex(P, n, echo.ECHO_GROUP, echo.ECHO_BF16, True, SENDER_EF)
     assert base == echo.echo_model_bytes(P, n, echo.ECHO_BF16, True)
     assert base["total"] - osum["total"] == 8 * n
     assert ef["total"] - base["total"] == 8 * P * n
