@@ -64,16 +64,25 @@ static int choose_exponent(double A)
     return e;
 }
 
-int echo_oracle_quantize_group(const float *v, int G, int8_t *q)
+/* Largest magnitude of a group, exact in binary64; -1 for a non-finite value. */
+static double group_absmax(const float *v, int G)
 {
     double A = 0.0;
     for (int k = 0; k < G; k++) {
         if (!isfinite(v[k]))
-            return -1;
+            return -1.0;
         double a = fabs((double)v[k]);
         if (a > A)
             A = a;
     }
+    return A;
+}
+
+int echo_oracle_quantize_group(const float *v, int G, int8_t *q)
+{
+    double A = group_absmax(v, G);
+    if (A < 0)
+        return -1;
     int e = choose_exponent(A);
     if (e > 126)
         return -2;
@@ -91,6 +100,95 @@ int echo_oracle_quantize_group(const float *v, int G, int8_t *q)
 float echo_oracle_dequant(int q, int b)
 {
     return (float)ldexp((double)q, b - 127);
+}
+
+/* ---- binary16-scale variant ------------------------------------------- */
+
+/* Value of a binary16 bit pattern (finite values only), exact in binary64:
+ * sign, 5 exponent bits (bias 15), 10 fraction bits; exponent 0 holds the
+ * subnormals frac * 2^-24. */
+double echo_oracle_half_value(uint16_t h)
+{
+    int ex = (h >> 10) & 0x1F;
+    int frac = h & 0x3FF;
+    double v = ex == 0 ? ldexp((double)frac, -24) : ldexp((double)(frac | 0x400), ex - 25);
+    return (h & 0x8000u) ? -v : v;
+}
+
+/* Smallest positive finite binary16 s with 7*s >= A (7*s is exact in
+ * binary64); 0 when A == 0; the largest finite binary16, 65504, when no
+ * binary16 is large enough (the codes then saturate at +-7). Positive
+ * binary16 values grow with their bit patterns, so a bisection over the
+ * patterns 0x0001..0x7BFF finds it. */
+static uint16_t choose_half_scale(double A)
+{
+    if (A == 0.0)
+        return 0;
+    uint16_t lo = 1, hi = 0x7BFF;
+    if (7.0 * echo_oracle_half_value(hi) < A)
+        return hi;
+    while (lo < hi) {
+        uint16_t mid = (uint16_t)(lo + (hi - lo) / 2);
+        if (7.0 * echo_oracle_half_value(mid) >= A)
+            hi = mid;
+        else
+            lo = (uint16_t)(mid + 1);
+    }
+    return lo;
+}
+
+/* The code in [-7, 7] nearest to v/s, a tie going to the even code. |v| is
+ * compared with the midpoints (k + 1/2)*s, which binary64 holds exactly
+ * (at most 15 significant bits), so no quotient is rounded. */
+static int nearest_code(double v, double s)
+{
+    double a = fabs(v);
+    int k = 0;
+    while (k < 7 && a > (k + 0.5) * s)
+        k = k + 1;
+    if (k < 7 && a == (k + 0.5) * s && (k % 2) == 1)
+        k = k + 1;
+    return v < 0 ? -k : k;
+}
+
+int echo_oracle_quantize_group_f16(const float *v, int G, int8_t *q, uint16_t *scale)
+{
+    double A = group_absmax(v, G);
+    if (A < 0)
+        return -1;
+    uint16_t h = choose_half_scale(A);
+    double sv = echo_oracle_half_value(h);
+    for (int k = 0; k < G; k++)
+        q[k] = (int8_t)nearest_code((double)v[k], sv);
+    *scale = h;
+    return 0;
+}
+
+float echo_oracle_dequant_f16(int q, uint16_t h)
+{
+    return (float)((double)q * echo_oracle_half_value(h)); /* <= 14 significant bits: exact */
+}
+
+/* v rounded to the nearest bf16 (8 significant bits), a tie going to the
+ * even last bit; v is finite with |v| < 2^127. */
+float echo_oracle_round_bf16(float v)
+{
+    double a = fabs((double)v);
+    if (a == 0.0)
+        return v;
+    int e;
+    frexp(a, &e);                             /* 2^(e-1) <= a < 2^e */
+    double step = ldexp(1.0, (e - 8 < -133) ? -133 : e - 8);
+    double lo = floor(a / step) * step;       /* power-of-two scaling: exact */
+    double hi = lo + step;
+    double r;
+    if (a - lo < hi - a)
+        r = lo;
+    else if (a - lo > hi - a)
+        r = hi;
+    else
+        r = (fmod(lo / step, 2.0) == 0.0) ? lo : hi;
+    return (float)(v < 0 ? -r : r);
 }
 
 void echo_oracle_pack(const int8_t *q, size_t count, uint8_t *out)
@@ -130,6 +228,23 @@ static int store_output(void *out, int dtype, size_t idx, float v)
     return 0;
 }
 
+/* Restored value of code q under a scale byte (power of two) or a binary16
+ * scale pattern. */
+static float restore(int q, int scale, int half_scale)
+{
+    return half_scale ? echo_oracle_dequant_f16(q, (uint16_t)scale) : echo_oracle_dequant(q, scale);
+}
+
+static void put_scale(uint8_t *out, size_t t, int scale, int half_scale)
+{
+    if (half_scale) {
+        out[2 * t] = (uint8_t)(scale & 0xFF);
+        out[2 * t + 1] = (uint8_t)((scale >> 8) & 0xFF);
+    } else {
+        out[t] = (uint8_t)scale;
+    }
+}
+
 int echo_oracle_allreduce_groups_ex(int P, int G, size_t ngroups,
                                     const int32_t *owner, int dtype,
                                     const void *x, void *out, float *f, float *s,
@@ -141,11 +256,12 @@ int echo_oracle_allreduce_groups_ex(int P, int G, size_t ngroups,
 {
     const int owner_sum = (variant & ECHO_ORACLE_OWNER_SUM) != 0;
     const int sender_ef = (variant & ECHO_ORACLE_SENDER_EF) != 0;
+    const int half_scale = (variant & ECHO_ORACLE_FP16_SCALE) != 0;
     if (P < 2 || P > 16 || G < 2 || (G % 2) != 0 || ngroups == 0)
         return -1;
     if (dtype != ECHO_ORACLE_BF16 && dtype != ECHO_ORACLE_FP32)
         return -1;
-    if (variant & ~(ECHO_ORACLE_OWNER_SUM | ECHO_ORACLE_SENDER_EF))
+    if (variant & ~(ECHO_ORACLE_OWNER_SUM | ECHO_ORACLE_SENDER_EF | ECHO_ORACLE_FP16_SCALE))
         return -1;
     if (!owner || !x || !out || (enable && (!f || !s)) || (sender_ef && !eps))
         return -1;
@@ -201,18 +317,27 @@ int echo_oracle_allreduce_groups_ex(int P, int G, size_t ngroups,
                 else
                     v[k] = u;
             }
-            int b = echo_oracle_quantize_group(v, G, q1 + (size_t)r * m + g * (size_t)G);
+            int b;
+            if (half_scale) {
+                uint16_t h = 0;
+                b = echo_oracle_quantize_group_f16(v, G, q1 + (size_t)r * m + g * (size_t)G, &h);
+                if (b == 0)
+                    b = h;
+            } else {
+                b = echo_oracle_quantize_group(v, G, q1 + (size_t)r * m + g * (size_t)G);
+            }
             if (b < 0) {
                 rc = b;
                 goto done;
             }
             b1[(size_t)r * ngroups + g] = b;
             /* Variant: keep this rounding's error for the rank's next call
-             * (exact in binary32, as for rounding #2). */
+             * (exact in binary32, as for rounding #2, unless a binary16
+             * scale saturated). */
             if (sender_ef)
                 for (int k = 0; k < G; k++) {
                     size_t i = g * (size_t)G + (size_t)k;
-                    float restored = echo_oracle_dequant(q1[(size_t)r * m + i], b);
+                    float restored = restore(q1[(size_t)r * m + i], b, half_scale);
                     eps[(size_t)r * m + i] = v[k] - restored;
                 }
         }
@@ -226,7 +351,7 @@ int echo_oracle_allreduce_groups_ex(int P, int G, size_t ngroups,
             size_t i = g * (size_t)G + (size_t)k;
             float sum = 0.0f;
             for (int r = 0; r < P; r++) {
-                float d = echo_oracle_dequant(q1[(size_t)r * m + i], b1[(size_t)r * ngroups + g]);
+                float d = restore(q1[(size_t)r * m + i], b1[(size_t)r * ngroups + g], half_scale);
                 sum = sum + d;
             }
             /* Variant: the owner folds the correction into its sum, after
@@ -236,7 +361,15 @@ int echo_oracle_allreduce_groups_ex(int P, int G, size_t ngroups,
             S[k] = sum;
         }
         /* Step 4: rounding #2 of the total. */
-        int bq = echo_oracle_quantize_group(S, G, Q + g * (size_t)G);
+        int bq;
+        if (half_scale) {
+            uint16_t h = 0;
+            bq = echo_oracle_quantize_group_f16(S, G, Q + g * (size_t)G, &h);
+            if (bq == 0)
+                bq = h;
+        } else {
+            bq = echo_oracle_quantize_group(S, G, Q + g * (size_t)G);
+        }
         if (bq < 0) {
             rc = bq;
             goto done;
@@ -244,8 +377,13 @@ int echo_oracle_allreduce_groups_ex(int P, int G, size_t ngroups,
         bQ[g] = bq;
         for (int k = 0; k < G; k++) {
             size_t i = g * (size_t)G + (size_t)k;
-            float Y = echo_oracle_dequant(Q[i], bq);
-            /* Step 5: the error rounding #2 injected (exact in binary32). */
+            float Y = restore(Q[i], bq, half_scale);
+            /* Variant: a binary16 scale makes Y a 14-bit value, which a bf16
+             * output rounds once more; every rank receives that value. */
+            if (half_scale && dtype == ECHO_ORACLE_BF16)
+                Y = echo_oracle_round_bf16(Y);
+            /* Step 5: the error injected into what the ranks receive (exact
+             * in binary32). */
             float err = S[k] - Y;
             if (enable) {
                 float f_keep = beta_f * f[i];
@@ -270,14 +408,16 @@ int echo_oracle_allreduce_groups_ex(int P, int G, size_t ngroups,
     if (codes1)
         for (int r = 0; r < P; r++)
             echo_oracle_pack(q1 + (size_t)r * m, m, codes1 + (size_t)r * (m / 2));
+    /* Scale bytes: one per group, or a little-endian binary16 (two bytes)
+     * per group under the binary16-scale variant. */
     if (scales1)
         for (size_t t = 0; t < (size_t)P * ngroups; t++)
-            scales1[t] = (uint8_t)b1[t];
+            put_scale(scales1, t, b1[t], half_scale);
     if (qcodes)
         echo_oracle_pack(Q, m, qcodes);
     if (qscales)
         for (size_t g = 0; g < ngroups; g++)
-            qscales[g] = (uint8_t)bQ[g];
+            put_scale(qscales, g, bQ[g], half_scale);
 
 done:
     free(c);

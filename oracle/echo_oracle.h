@@ -64,6 +64,18 @@ extern "C" {
  *                          correction: v = RN(RN(x + eps) + c). */
 #define ECHO_ORACLE_OWNER_SUM 1
 #define ECHO_ORACLE_SENDER_EF 2
+/*   ECHO_ORACLE_FP16_SCALE every group (both roundings) takes a binary16
+ *                          scale s instead of a power of two: s is the
+ *                          smallest positive finite binary16 with
+ *                          7*s >= max|v| (0 for an all-zero group; 65504,
+ *                          with saturated codes, past 7*65504); each code is
+ *                          the integer in [-7, 7] nearest to v/s, ties to
+ *                          even. Restored values q*s are exact in binary32;
+ *                          bf16 outputs are q*s rounded to the nearest bf16
+ *                          (ties to even), and the captured error is taken
+ *                          against that received value. Wire scales are
+ *                          little-endian binary16, two bytes per group. */
+#define ECHO_ORACLE_FP16_SCALE 4
 
 /* Scale choice and rounding of one group (rounding #1 at a sender, #2 at the
  * owner). v: G binary32 values. Writes G codes to q. Returns the scale byte
@@ -72,6 +84,15 @@ int echo_oracle_quantize_group(const float *v, int G, int8_t *q);
 
 /* Value of code q under scale byte b: q * 2^(b-127), exact in binary32. */
 float echo_oracle_dequant(int q, int b);
+
+/* Binary16-scale codec (variant ECHO_ORACLE_FP16_SCALE): scale pattern and
+ * codes of one group (returns 0, or -1 for a non-finite value); the value of
+ * code q under scale pattern h; the value of a binary16 pattern; a binary32
+ * rounded to the nearest bf16, ties to even. */
+int echo_oracle_quantize_group_f16(const float *v, int G, int8_t *q, uint16_t *scale);
+float echo_oracle_dequant_f16(int q, uint16_t h);
+double echo_oracle_half_value(uint16_t h);
+float echo_oracle_round_bf16(float v);
 
 /* Pack count codes (count even) two per byte; unpack the reverse. */
 void echo_oracle_pack(const int8_t *q, size_t count, uint8_t *out);
@@ -86,8 +107,10 @@ void echo_oracle_unpack(const uint8_t *in, size_t count, int8_t *q);
  * f, s     the phase's compensator state, m binary32 each, read and updated
  *          in place (untouched when enable == 0).
  * out      m elements of dtype: the value every rank receives.
- * codes1   optional [P][m/2] stage-1 packed codes, scales1 [P][ngroups].
- * qcodes   optional [m/2] requantised codes, qscales [ngroups].
+ * codes1   optional [P][m/2] stage-1 packed codes, scales1 [P][ngroups]
+ *          (bytes; [P][2*ngroups] under ECHO_ORACLE_FP16_SCALE).
+ * qcodes   optional [m/2] requantised codes, qscales [ngroups] (bytes;
+ *          [2*ngroups] under ECHO_ORACLE_FP16_SCALE).
  * c_out    optional [m] correction the owner added (0 when off).
  * err_out  optional [m] captured error S - Y.
  */

@@ -24,11 +24,13 @@ BF16 = 0
 FP32 = 1
 OWNER_SUM = 1   # variant: the owner adds the correction to its sum
 SENDER_EF = 2   # variant: every rank feeds back its own rounding-#1 error
+FP16_SCALE = 4  # variant: binary16 scales (rounded up) instead of powers of two
 
 _u8p = ctypes.POINTER(ctypes.c_uint8)
 _i8p = ctypes.POINTER(ctypes.c_int8)
 _f32p = ctypes.POINTER(ctypes.c_float)
 _i32p = ctypes.POINTER(ctypes.c_int32)
+_u16p = ctypes.POINTER(ctypes.c_uint16)
 
 
 def build(src_dir: str = HERE) -> str:
@@ -70,6 +72,14 @@ class Oracle:
         lib.echo_oracle_pack.restype = None
         lib.echo_oracle_unpack.argtypes = [_u8p, ctypes.c_size_t, _i8p]
         lib.echo_oracle_unpack.restype = None
+        lib.echo_oracle_quantize_group_f16.argtypes = [_f32p, ctypes.c_int, _i8p, _u16p]
+        lib.echo_oracle_quantize_group_f16.restype = ctypes.c_int
+        lib.echo_oracle_dequant_f16.argtypes = [ctypes.c_int, ctypes.c_uint16]
+        lib.echo_oracle_dequant_f16.restype = ctypes.c_float
+        lib.echo_oracle_half_value.argtypes = [ctypes.c_uint16]
+        lib.echo_oracle_half_value.restype = ctypes.c_double
+        lib.echo_oracle_round_bf16.argtypes = [ctypes.c_float]
+        lib.echo_oracle_round_bf16.restype = ctypes.c_float
         common = [ctypes.c_void_p, ctypes.c_void_p, _f32p, _f32p,
                   ctypes.c_float, ctypes.c_float, ctypes.c_float, ctypes.c_int,
                   _u8p, _u8p, _u8p, _u8p, _f32p, _f32p]
@@ -102,6 +112,26 @@ class Oracle:
     def dequant(self, q: int, b: int) -> float:
         return float(np.float32(self.lib.echo_oracle_dequant(int(q), int(b))))
 
+    def quantize_group_f16(self, v) -> tuple[int, np.ndarray]:
+        """Binary16 scale pattern and codes of one group (variant FP16_SCALE)."""
+        v = np.ascontiguousarray(v, dtype=np.float32)
+        q = np.zeros(v.shape[0], dtype=np.int8)
+        h = ctypes.c_uint16(0)
+        rc = self.lib.echo_oracle_quantize_group_f16(_ptr(v, _f32p), v.shape[0], _ptr(q, _i8p),
+                                                     ctypes.byref(h))
+        if rc < 0:
+            raise ValueError(f"oracle quantize_group_f16 failed ({rc})")
+        return int(h.value), q
+
+    def dequant_f16(self, q: int, h: int) -> float:
+        return float(np.float32(self.lib.echo_oracle_dequant_f16(int(q), int(h))))
+
+    def half_value(self, h: int) -> float:
+        return float(self.lib.echo_oracle_half_value(int(h)))
+
+    def round_bf16(self, v: float) -> float:
+        return float(np.float32(self.lib.echo_oracle_round_bf16(float(np.float32(v)))))
+
     def pack(self, q) -> np.ndarray:
         q = np.ascontiguousarray(q, dtype=np.int8)
         out = np.zeros(q.shape[0] // 2, dtype=np.uint8)
@@ -124,9 +154,10 @@ class Oracle:
         length m) are updated in place when compensation is on. ``owner`` (one
         rank per group) overrides the contiguous segment layout; it lets a
         caller run any subset of groups of a larger problem.
-        ``variant`` is a bit set of OWNER_SUM and SENDER_EF; with SENDER_EF,
-        ``eps`` (float32, shape (P, m)) is every rank's rounding-#1 error state,
-        updated in place.
+        ``variant`` is a bit set of OWNER_SUM, SENDER_EF and FP16_SCALE; with
+        SENDER_EF, ``eps`` (float32, shape (P, m)) is every rank's rounding-#1
+        error state, updated in place; with FP16_SCALE the scale arrays hold
+        binary16 bit patterns (uint16) instead of scale bytes.
         Returns a dict with ``out`` and, if requested, the wire and diagnostics.
         """
         x = np.ascontiguousarray(x)
@@ -154,9 +185,10 @@ class Oracle:
         res = {"out": out}
         if want_wire:
             res["codes1"] = np.zeros((P, m // 2), dtype=np.uint8)
-            res["scales1"] = np.zeros((P, ngroups), dtype=np.uint8)
+            sdt = np.uint16 if variant & FP16_SCALE else np.uint8
+            res["scales1"] = np.zeros((P, ngroups), dtype=sdt)
             res["qcodes"] = np.zeros(m // 2, dtype=np.uint8)
-            res["qscales"] = np.zeros(ngroups, dtype=np.uint8)
+            res["qscales"] = np.zeros(ngroups, dtype=sdt)
         if want_diag:
             res["c"] = np.zeros(m, dtype=np.float32)
             res["err"] = np.zeros(m, dtype=np.float32)

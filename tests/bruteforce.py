@@ -42,3 +42,55 @@ def bf_quantize(values) -> tuple[int, list[int]]:
 def value_of(code: int, byte: int) -> Fraction:
     """Exact value of a code under a scale byte."""
     return code * Fraction(2) ** (byte - 127)
+
+
+# ---- binary16-scale variant ------------------------------------------------
+def _half_table():
+    """Every positive finite binary16 value in increasing order, decoded by
+    numpy (not by the oracle), with its bit pattern."""
+    import numpy as np
+    bits = np.arange(1, 0x7C00, dtype=np.uint16)
+    return bits, bits.view(np.float16).astype(np.float64)
+
+
+def bf_quantize_f16(values) -> tuple[int, list[int]]:
+    """Binary16 scale pattern and codes of one group by exhaustive search.
+
+    The scale is the first positive finite binary16, in increasing order, whose
+    7-fold covers the largest magnitude (the largest finite one, 65504, when
+    none does; 0 for an all-zero group). Every code in [-7, 7] is tried per
+    value with exact rational distances; a tie goes to the even code.
+    """
+    import numpy as np
+    vals = [Fraction(float(v)) for v in values]
+    A = max(abs(v) for v in vals)
+    if A == 0:
+        return 0, [0] * len(vals)
+    bits, table = _half_table()
+    ok = np.flatnonzero(7 * table >= float(A))  # 7*s and A are exact in binary64
+    i = int(ok[0]) if ok.size else len(table) - 1
+    h, s = int(bits[i]), Fraction(float(table[i]))
+    codes = []
+    for v in vals:
+        best_k, best_d = None, None
+        for k in range(CODE_MIN, CODE_MAX + 1):
+            d = abs(v - k * s)
+            if best_d is None or d < best_d or (d == best_d and k % 2 == 0):
+                best_k, best_d = k, d
+        codes.append(best_k)
+    return h, codes
+
+
+def half_fraction(h: int) -> Fraction:
+    """Exact value of a binary16 bit pattern, decoded by numpy."""
+    import numpy as np
+    return Fraction(float(np.array([h], dtype=np.uint16).view(np.float16)[0]))
+
+
+def bf16_round_bits(x: float) -> float:
+    """Nearest bf16 to a binary32 value, ties to even, by integer arithmetic on
+    the bit pattern: add 0x7FFF plus the lowest kept bit, drop the low half."""
+    import struct
+    u = struct.unpack("<I", struct.pack("<f", x))[0]
+    u = (u + 0x7FFF + ((u >> 16) & 1)) & 0xFFFF0000
+    return struct.unpack("<f", struct.pack("<I", u))[0]

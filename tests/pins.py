@@ -30,8 +30,8 @@ from fractions import Fraction
 import numpy as np
 
 from bit_error_compensated_rank_b200.workloads import bf16_bits, bf16_to_f32, gaussian, rng
-from bruteforce import bf_quantize, value_of
-from oracle.oracle import OWNER_SUM, SENDER_EF, Params
+from bruteforce import bf16_round_bits, bf_quantize, bf_quantize_f16, half_fraction, value_of
+from oracle.oracle import FP16_SCALE, OWNER_SUM, SENDER_EF, Params
 
 GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
 F32 = np.float32
@@ -591,6 +591,171 @@ def pin_full_compensation_bounded(orc):
     assert rms[SENDER_EF | OWNER_SUM] < 0.3 * rms[0], rms
 
 
+# ---------------------------------------------------------------------------
+# binary16-scale variant (scale = the smallest binary16 s with 7*s >= max|v|)
+# ---------------------------------------------------------------------------
+def _f16_groups(count, G, seed):
+    """Random groups plus the cases the binary16 rule turns on: 7*s exactly
+    at the maximum, one ulp past it, the subnormal binary16 range, below the
+    smallest binary16 step, past the largest scale (saturation), zero."""
+    groups = _random_groups(count, G, seed)
+    g = rng(seed, 16)
+    for h in (0x3C00, 0x0001, 0x0200, 0x03FF, 0x0400, 0x2E66, 0x7BFF, 0x5A5A):
+        sv = float(half_fraction(h))
+        v = g.uniform(-7, 7, G) * sv
+        v[0] = 7 * sv                                   # exactly 7*s: s itself
+        groups.append(v.astype(F32))
+        w = v.astype(F32)
+        w[1] = np.nextafter(F32(7 * sv), F32(np.inf))   # just past: the next binary16
+        groups.append(w)
+        t = (g.integers(-7, 8, G) + 0.5) * sv           # exact ties k + 1/2
+        t[0] = 7 * sv
+        groups.append(t.astype(F32))
+    groups.append((g.standard_normal(G) * 1e6).astype(F32))      # saturates at 65504
+    groups.append((g.standard_normal(G) * 2.0 ** -30).astype(F32))  # below 2^-24
+    groups.append(np.zeros(G, F32))
+    return groups
+
+
+def pin_f16_quantizer_bruteforce(orc):
+    """Binary16 scale pattern and every code equal an exhaustive search over
+    all binary16 scales (decoded by numpy) and all codes, with exact
+    distances; ties go to the even code."""
+    for G in (32, 16, 2):
+        for v in _f16_groups(36 if G == 32 else 12, G, seed=200 + G):
+            h, q = orc.quantize_group_f16(v)
+            bh, bq = bf_quantize_f16(v.tolist())
+            assert h == bh, (v, h, bh)
+            assert q.tolist() == bq, (v, q.tolist(), bq)
+
+
+def pin_f16_values(orc):
+    """Restored values are q*s exactly (numpy's binary16 decoding); the bf16
+    rounding of outputs agrees with the bit-pattern rule add-0x7FFF-plus-odd;
+    a restored q*s is within s/2 of v unless the scale saturated, and s is
+    within one binary16 step of max|v|/7."""
+    for h in list(range(1, 0x7C00, 97)) + [0x7BFF, 1, 0x3FF, 0x400]:
+        sv = half_fraction(h)
+        assert Fraction(orc.half_value(h)) == sv
+        for q in range(-7, 8):
+            y = orc.dequant_f16(q, h)
+            assert Fraction(y) == q * sv
+            assert orc.round_bf16(y) == bf16_round_bits(y), (q, h)
+    g = rng(5, 16)
+    for x in np.concatenate([g.standard_normal(4000) * 2.0 ** g.integers(-30, 20, 4000),
+                             (g.integers(0, 2 ** 16, 500) * 2.0 + 1) * 2.0 ** -16]).astype(F32):
+        assert orc.round_bf16(float(x)) == bf16_round_bits(float(x)), x
+    for v in _f16_groups(12, 32, seed=7):
+        h, q = orc.quantize_group_f16(v)
+        A = max(abs(Fraction(float(t))) for t in v)
+        if A == 0:
+            continue
+        sv = half_fraction(h)
+        if A <= 7 * Fraction(65504):
+            assert 7 * sv >= A and (h == 1 or 7 * half_fraction(h - 1) < A)
+            for t, k in zip(v, q.tolist()):
+                assert abs(Fraction(float(t)) - k * sv) <= sv / 2
+
+
+def _f16_grid_partials(P, ngroups, G, seed):
+    """Partials k*s with s a binary16 and one |k| = 7 per group, so that
+    rounding #1 reproduces them exactly with scale s. The scales stay within a
+    narrow range so that binary32 sums are exact."""
+    g = rng(seed, 161, P)
+    k = g.integers(-7, 8, (P, ngroups, G))
+    lead = g.integers(0, G, (P, ngroups))
+    h = g.integers(0x3800, 0x3C00, (P, ngroups)).astype(np.uint16)   # s in [0.5, 1)
+    for r in range(P):
+        for j in range(ngroups):
+            k[r, j, lead[r, j]] = 7 if g.random() < 0.5 else -7
+    sv = h.view(np.float16).astype(np.float64)
+    x = (k * sv[:, :, None]).astype(F32)
+    return x.reshape(P, ngroups * G), k, h
+
+
+def pin_f16_exact_sums_on_grid(orc):
+    """Binary16 scales with partials on their grid: rounding #1 is exact, the
+    binary32 sum is exact, the total is the exhaustive quantiser's result on
+    the exact sum; a binary32 output is q*s exactly, a bf16 output is that
+    rounded to the nearest bf16 (ties to even), and the captured error is the
+    exact sum minus what the ranks receive."""
+    for P, G in [(2, 32), (5, 32), (8, 16), (3, 128)]:
+        ngroups = 2 * P
+        m = ngroups * G
+        x32, k, h = _f16_grid_partials(P, ngroups, G, seed=P * G)
+        exact = [sum(Fraction(float(x32[r, i])) for r in range(P)) for i in range(m)]
+        want_h, want_Y = [], []
+        for j in range(ngroups):
+            bh, bq = bf_quantize_f16([float(t) for t in exact[j * G:(j + 1) * G]])
+            want_h.append(bh)
+            want_Y += [c * half_fraction(bh) for c in bq]
+        for x, bf in ((x32, False), (bf16_bits(x32), True)):
+            if bf and not (bf16_to_f32(x) == x32).all():
+                continue   # k*s is not always a bf16: that input would round first
+            for enable in (False, True):
+                f = np.zeros(m, F32)
+                s = np.zeros(m, F32)
+                res = orc.allreduce(x, f, s, Params(enable=enable), G=G, want_diag=True,
+                                    variant=FP16_SCALE)
+                assert res["scales1"].tolist() == h.tolist()
+                for r in range(P):
+                    assert _unpack_ref(res["codes1"][r]) == k[r].reshape(-1).tolist()
+                assert res["qscales"].tolist() == want_h
+                Y = [Fraction(bf16_round_bits(float(y))) if bf else y for y in want_Y]
+                out = [Fraction(float(t)) for t in _values(res["out"])]
+                assert out == Y
+                err = [Fraction(float(t)) for t in res["err"]]
+                assert err == [a - b for a, b in zip(exact, Y)]
+        # bf16 inputs that are on a bf16 grid: k*s with s = 2^j * (1 + i/8)
+        hb = (0x3800 + (np.arange(ngroups * P) % 8) * 128).astype(np.uint16).reshape(P, ngroups)
+        xb = (k * hb.view(np.float16).astype(np.float64)[:, :, None]).astype(F32).reshape(P, m)
+        assert (bf16_to_f32(bf16_bits(xb)) == xb).all()
+        res = orc.allreduce(bf16_bits(xb), params=Params(enable=False), G=G, want_diag=True,
+                            variant=FP16_SCALE)
+        assert res["scales1"].tolist() == hb.tolist()
+        exact = [sum(Fraction(float(xb[r, i])) for r in range(P)) for i in range(m)]
+        for j in range(ngroups):
+            bh, bq = bf_quantize_f16([float(t) for t in exact[j * G:(j + 1) * G]])
+            assert res["qscales"][j] == bh
+            for t in range(G):
+                y = Fraction(bf16_round_bits(float(bq[t] * half_fraction(bh))))
+                i = j * G + t
+                assert Fraction(float(_values(res["out"])[i])) == y
+                assert Fraction(float(res["err"][i])) == exact[i] - y
+
+
+def pin_f16_feedback(orc):
+    """The compensator and both feedback variants run unchanged over binary16
+    scales: with lambda = 1, beta_fast = 0 the correction of call k is
+    exactly the error of call k-1; sender feedback on grid partials keeps
+    every stored error at 0; the closed-form bound |D_K| <= 5 max|err| holds."""
+    P, G = 4, 32
+    m = P * G * 4
+    f = np.zeros(m, F32)
+    s = np.zeros(m, F32)
+    prev = None
+    for k in range(8):
+        res = orc.allreduce(gaussian(P, m, seed=6, call=k), f, s, Params(lam=1.0, beta_fast=0.0),
+                            want_diag=True, variant=FP16_SCALE)
+        if prev is not None:
+            assert (res["c"] == prev).all()
+        prev = res["err"].copy()
+    x32, _, _ = _f16_grid_partials(P, 2 * P, G, seed=77)
+    eps = np.zeros((P, x32.shape[1]), F32)
+    orc.allreduce(x32, params=Params(enable=False), variant=FP16_SCALE | SENDER_EF, eps=eps)
+    assert not eps.any()
+    f = np.zeros(m, F32)
+    s = np.zeros(m, F32)
+    D = np.zeros(m)
+    emax = np.zeros(m)
+    for k in range(48):
+        res = orc.allreduce(gaussian(P, m, seed=8, call=k), f, s, Params(), want_diag=True,
+                            variant=FP16_SCALE)
+        D += res["c"].astype(np.float64) - res["err"].astype(np.float64)
+        emax = np.maximum(emax, np.abs(res["err"].astype(np.float64)))
+        assert (np.abs(D) <= 5.0 * emax * (1 + 1e-4) + 1e-30).all(), k
+
+
 ALL_PINS = [
     pin_scale_boundaries,
     pin_quantizer_bruteforce,
@@ -613,4 +778,8 @@ ALL_PINS = [
     pin_sender_ef_on_grid,
     pin_sender_ef_per_rank,
     pin_full_compensation_bounded,
+    pin_f16_quantizer_bruteforce,
+    pin_f16_values,
+    pin_f16_exact_sums_on_grid,
+    pin_f16_feedback,
 ]

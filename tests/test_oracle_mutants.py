@@ -41,8 +41,8 @@ MUTANTS = [
      "for (int r = 0; r < P; r++) {\n                float d",
      "for (int r = 1; r < P; r++) {\n                float d"),
     ("sum_reversed_order",
-     "float d = echo_oracle_dequant(q1[(size_t)r * m + i], b1[(size_t)r * ngroups + g]);",
-     "float d = echo_oracle_dequant(q1[(size_t)(P - 1 - r) * m + i], b1[(size_t)(P - 1 - r) * ngroups + g]);"),
+     "float d = restore(q1[(size_t)r * m + i], b1[(size_t)r * ngroups + g], half_scale);",
+     "float d = restore(q1[(size_t)(P - 1 - r) * m + i], b1[(size_t)(P - 1 - r) * ngroups + g], half_scale);"),
     ("sum_in_binary64",
      "float sum = 0.0f;",
      "double sum = 0.0;"),
@@ -71,7 +71,7 @@ MUTANTS = [
      "f[i] = f_keep + f_new;",
      "f[i] = f[i];"),
     ("captures_stage1_error_instead",
-     "float Y = echo_oracle_dequant(Q[i], bq);",
+     "float Y = restore(Q[i], bq, half_scale);",
      "float Y = S[k];"),
     ("correction_not_added",
      "v[k] = u + c[i];",
@@ -98,6 +98,39 @@ MUTANTS = [
     ("owner_sum_starts_from_correction",
      [("float sum = 0.0f;", "float sum = (enable && owner_sum) ? c[i] : 0.0f;"),
       ("if (enable && owner_sum)\n                sum = sum + c[i];", "")]),
+    # binary16-scale variant
+    ("f16_scale_strict_boundary",
+     "if (7.0 * echo_oracle_half_value(mid) >= A)",
+     "if (7.0 * echo_oracle_half_value(mid) > A)"),
+    ("f16_scale_range_8",
+     "if (7.0 * echo_oracle_half_value(mid) >= A)",
+     "if (8.0 * echo_oracle_half_value(mid) >= A)"),
+    ("f16_saturates_to_infinity",
+     "if (7.0 * echo_oracle_half_value(hi) < A)\n        return hi;",
+     "if (7.0 * echo_oracle_half_value(hi) < A)\n        return 0x7C00;"),
+    ("f16_ties_to_odd",
+     "(k + 0.5) * s && (k % 2) == 1)",
+     "(k + 0.5) * s && (k % 2) == 0)"),
+    ("f16_ties_away_from_zero",
+     "(k + 0.5) * s && (k % 2) == 1)",
+     "(k + 0.5) * s)"),
+    ("f16_codes_truncated",
+     "while (k < 7 && a > (k + 0.5) * s)",
+     "while (k < 7 && a >= (k + 1) * s)"),
+    ("f16_subnormal_scale_decoded_wrong",
+     "ldexp((double)frac, -24)",
+     "ldexp((double)frac, -25)"),
+    ("f16_bf16_output_ties_up",
+     "r = (fmod(lo / step, 2.0) == 0.0) ? lo : hi;",
+     "r = hi;"),
+    ("f16_error_against_unrounded_output",
+     [("Y = echo_oracle_round_bf16(Y);", ";"),
+      ("int so = store_output(out, dtype, i, Y);",
+       "int so = store_output(out, dtype, i, (half_scale && dtype == ECHO_ORACLE_BF16) ? "
+       "echo_oracle_round_bf16(Y) : Y);")]),
+    ("f16_wire_big_endian",
+     "out[2 * t] = (uint8_t)(scale & 0xFF);\n        out[2 * t + 1] = (uint8_t)((scale >> 8) & 0xFF);",
+     "out[2 * t + 1] = (uint8_t)(scale & 0xFF);\n        out[2 * t] = (uint8_t)((scale >> 8) & 0xFF);"),
 ]
 
 
