@@ -45,8 +45,9 @@ SEED = 0
 WORKLOAD = "echo int4 all-reduce, P=8 ranks x 1 GiB bf16 per rank (2^29 elements), group 32, " \
            "compensation on, fwd state, partials N(0,1) with 0.1% at 50x"
 HBM_FALLBACK_GBS = 6650.0  # used only when MEASURED_PEAKS.json is absent
-# where the rounding errors are fed back (see include/echo.h, echo_set_variant)
-VARIANTS = {"default": 0, "owner_sum": 1, "sender_ef": 2, "both": 3}
+# where the rounding errors are fed back, and the scale format (see
+# include/echo.h, echo_set_variant)
+VARIANTS = {"default": 0, "owner_sum": 1, "sender_ef": 2, "both": 3, "fp16_scale": 4}
 # CPU baseline / reference arm samples (elements per rank, same distribution)
 CPU_SAMPLE_N = 1 << 20
 REF_SAMPLE_N = 1 << 18

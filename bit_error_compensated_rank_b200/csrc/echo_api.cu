@@ -65,6 +65,7 @@ constexpr size_t kMaxN = size_t(1) << 34;  // chunk indices stay 32-bit
 constexpr long long kWaitCycles = 1LL << 31;
 constexpr long long kStallWaitCycles = 1LL << 20;
 constexpr size_t kHostPiece = size_t(1) << 22; // elements per pipelined host transfer
+constexpr int kVariantBits = ECHO_VARIANT_OWNER_SUM | ECHO_VARIANT_SENDER_EF | ECHO_VARIANT_FP16_SCALE;
 constexpr int kTimingRing = 32;                 // event sets of timed calls in flight
 
 size_t elem_bytes(int dtype) { return dtype == ECHO_BF16 ? 2 : 4; }
@@ -94,7 +95,9 @@ int check_shape(int P, size_t n, int group, int dtype)
 void model_bytes(int P, size_t n, int group, int dtype, bool enable, int variant, uint64_t out[4])
 {
     const uint64_t b = elem_bytes(dtype);
-    const uint64_t wire = static_cast<uint64_t>(n) / 2 + static_cast<uint64_t>(n) / group; // n * (1/2 + 1/G)
+    // n * (1/2 + 1/G) bytes, or n * (1/2 + 2/G) with binary16 scales
+    const uint64_t scale_bytes = (variant & ECHO_VARIANT_FP16_SCALE) ? 2 : 1;
+    const uint64_t wire = static_cast<uint64_t>(n) / 2 + scale_bytes * static_cast<uint64_t>(n) / group;
     const uint64_t state = enable ? 8 * static_cast<uint64_t>(n) : 0;
     // the owner-sum variant reads f, s in kernel 2 only
     const uint64_t k1_state = (variant & ECHO_VARIANT_OWNER_SUM) ? 0 : state;
@@ -119,7 +122,7 @@ struct echo_handle {
     uint8_t *scales1 = nullptr; // [P][scale_stride], n/group bytes used per rank
     uint8_t *qcodes = nullptr;  // [n/2]
     uint8_t *qscales = nullptr; // [scale_stride]
-    size_t scale_stride = 0;    // n/group rounded up to 16 bytes (bulk-copy alignment)
+    size_t scale_stride = 0;    // 2n/group rounded up to 16 bytes (bulk-copy alignment)
     int *dstatus = nullptr;     // device status word written by timed-out waits
     float *state = nullptr;     // [phase][f|s][n]
     float beta_f = 0.5f, beta_s = 0.875f, lambda = 0.5f;
@@ -293,6 +296,8 @@ int enqueue_call(echo_handle *h, const void *const send[], void *const recv[], i
     a1.bf16 = h->dtype == ECHO_BF16;
     a1.enable = h->enable && !(h->variant & ECHO_VARIANT_OWNER_SUM);
     a1.sender_ef = (h->variant & ECHO_VARIANT_SENDER_EF) != 0;
+    a1.fp16_scale = a2.fp16_scale = a3.fp16_scale = (h->variant & ECHO_VARIANT_FP16_SCALE) != 0;
+    a2.bf16 = h->dtype == ECHO_BF16;
     a1.eps = a1.sender_ef ? h->eps + static_cast<size_t>(phase) * h->P * h->n : nullptr;
 
     a2.codes = h->codes1;
@@ -481,7 +486,7 @@ int echo_model_bytes_ex(int P, size_t n, int group, int dtype, int enable, int v
         return rc;
     if (!out)
         return set_error(ECHO_ERR_INVALID, "out is NULL");
-    if (variant & ~(ECHO_VARIANT_OWNER_SUM | ECHO_VARIANT_SENDER_EF))
+    if (variant & ~kVariantBits)
         return set_error(ECHO_ERR_INVALID, "unknown variant bits 0x%x", variant);
     model_bytes(P, n, group, dtype, enable != 0, variant, out);
     return ECHO_OK;
@@ -492,7 +497,7 @@ int echo_set_variant(echo_handle *h, int variant)
     int rc;
     if ((rc = check_handle(h)) != ECHO_OK || (rc = check_device(h)) != ECHO_OK)
         return rc;
-    if (variant & ~(ECHO_VARIANT_OWNER_SUM | ECHO_VARIANT_SENDER_EF))
+    if (variant & ~kVariantBits)
         return set_error(ECHO_ERR_INVALID, "unknown variant bits 0x%x", variant);
     if ((variant & ECHO_VARIANT_SENDER_EF) && !h->eps) {
         const size_t bytes = 2 * static_cast<size_t>(h->P) * h->n * sizeof(float);
@@ -568,7 +573,7 @@ echo_handle *echo_create(int P, size_t n, int group, int dtype)
     h->lanes_log2 = 0; // group = 8 << lanes_log2 (a power of two in [16, 128])
     while ((8u << h->lanes_log2) != static_cast<uint32_t>(group))
         h->lanes_log2++;
-    h->scale_stride = (n / group + 15) / 16 * 16;
+    h->scale_stride = (2 * (n / group) + 15) / 16 * 16; // room for binary16 scales
     cudaError_t e = cudaGetDevice(&h->device);
     if (e != cudaSuccess) {
         cuda_error(e, "cudaGetDevice");
@@ -810,12 +815,13 @@ int echo_get_wire_range(echo_handle *h, int stage, int rank, size_t group_offset
         return set_error(ECHO_ERR_INVALID, "group range exceeds %zu groups", groups);
     const uint8_t *codes = stage == 1 ? h->codes1 + static_cast<size_t>(rank) * (h->n / 2) : h->qcodes;
     const uint8_t *scales = stage == 1 ? h->scales1 + static_cast<size_t>(rank) * h->scale_stride : h->qscales;
+    const size_t sb = (h->variant & ECHO_VARIANT_FP16_SCALE) ? 2 : 1; // bytes per scale
     cudaError_t e = cudaDeviceSynchronize();
     if (e == cudaSuccess && codes_host)
         e = cudaMemcpy(codes_host, codes + group_offset * (h->group / 2), ngroups * (h->group / 2),
                        cudaMemcpyDeviceToHost);
     if (e == cudaSuccess && scales_host)
-        e = cudaMemcpy(scales_host, scales + group_offset, ngroups, cudaMemcpyDeviceToHost);
+        e = cudaMemcpy(scales_host, scales + sb * group_offset, sb * ngroups, cudaMemcpyDeviceToHost);
     return e == cudaSuccess ? ECHO_OK : cuda_error(e, "echo_get_wire");
 }
 

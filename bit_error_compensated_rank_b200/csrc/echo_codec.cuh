@@ -11,9 +11,17 @@
 // Every helper here is exact integer or power-of-two arithmetic; the only
 // rounding is the choice of the nearest code (code_bits), which rounds halves
 // to even.
+//
+// Binary16-scale variant: the scale is the smallest positive finite binary16
+// s with 7*s >= max|v| (0 for an all-zero group, 65504 with saturated codes
+// beyond 7*65504), stored as its two-byte pattern; codes are the integers in
+// [-7, 7] nearest to v/s, ties to even (code_bits_near). Restored values q*s
+// have at most 14 significant bits and are exact in binary32.
 #pragma once
 
 #include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 namespace echo {
 
@@ -77,6 +85,67 @@ __device__ __forceinline__ uint32_t code_bits(float v, float inv)
 __device__ __forceinline__ float code_value(uint32_t bits)
 {
     return __fsub_rn(__uint_as_float(bits), kRound);
+}
+
+// ---- binary16 scales --------------------------------------------------------
+// Value of a binary16 scale pattern (exact conversion).
+__device__ __forceinline__ float half_step(uint32_t h)
+{
+    return __half2float(__ushort_as_half(static_cast<unsigned short>(h)));
+}
+
+// Smallest positive finite binary16 s with 7*s >= A (A finite, >= 0), as its
+// pattern; 0 for A == 0; 0x7BFF (65504) when 7*65504 < A. An estimate, A/7
+// rounded up to binary16 from a binary32 product, lies within one binary16
+// step of the answer (the product's relative error is about 2^-23, the
+// binary16 spacing 2^-10), and one exact test on each side settles it: 7*s
+// has at most 14 significant bits, so the binary32 product is exact.
+__device__ __forceinline__ uint32_t half_scale_bits(float A)
+{
+    constexpr float kSeventh = 0.142857142857142857f;
+    if (A == 0.f)
+        return 0u;
+    uint32_t h = __half_as_ushort(__float2half_ru(__fmul_rn(A, kSeventh)));
+    h = min(h, 0x7BFFu);
+    if (__fmul_rn(7.f, half_step(h)) < A)
+        h = min(h + 1u, 0x7BFFu);
+    else if (h > 1u && __fmul_rn(7.f, half_step(h - 1u)) >= A)
+        h = h - 1u;
+    return h;
+}
+
+// Bit pattern kRoundBits + q of the code q in [-7, 7] nearest to v/step, a
+// tie going to the even code, for any step >= 0 (inv an estimate of 1/step,
+// 0 when step is 0). The estimate k = nearest integer to v*inv can only miss
+// by one, next to a midpoint; the remainder r = v - k*step is exact there
+// (|r| <= step/2 needs at most 24 significant bits), so comparing |r| with
+// the exact step/2 moves k to the nearest code, or off an odd code on a tie.
+// A saturated group (v/step beyond 7.5) ends at +-7 after the clamp.
+__device__ __forceinline__ uint32_t code_bits_near(float v, float step, float inv)
+{
+    const float y = fminf(fmaxf(__fmul_rn(v, inv), -8.f), 8.f);
+    float k = __fsub_rn(__fadd_rn(y, kRound), kRound);
+    const float r = __fmaf_rn(-k, step, v);
+    const float half = __fmul_rn(0.5f, step);
+    const float ar = fabsf(r);
+    const bool odd = (__float_as_uint(__fadd_rn(k, kRound)) & 1u) != 0u;
+    if (ar > half || (ar == half && odd))
+        k = __fadd_rn(k, r < 0.f ? -1.f : 1.f);
+    k = fminf(fmaxf(k, -7.f), 7.f);
+    return __float_as_uint(__fadd_rn(k, kRound));
+}
+
+// Reciprocal estimate used by code_bits_near (0 for a zero step).
+__device__ __forceinline__ float half_inv(float step)
+{
+    return step > 0.f ? __frcp_rn(step) : 0.f;
+}
+
+// Nearest bf16 to a binary32 (ties to even), as the upper half of a binary32:
+// the value every rank receives under binary16 scales with bf16 outputs.
+__device__ __forceinline__ float round_bf16(float y)
+{
+    return __bfloat162float(__float2bfloat16_rn(y));
 }
 
 // Pack the codes of 8 rounded bit patterns (element k = low byte of b[k])

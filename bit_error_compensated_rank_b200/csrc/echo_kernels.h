@@ -60,9 +60,9 @@ struct K1Args {
     const float *f;          // phase state, fast estimate [n]
     const float *s;          // phase state, slow estimate [n]
     uint8_t *codes;          // stage-1 wire codes [P][n/2]
-    uint8_t *scales;         // stage-1 wire scale bytes [P][scale_stride], n/G per rank
+    uint8_t *scales;         // stage-1 wire scales [P][scale_stride]: n/G bytes or binary16s per rank
     size_t n;
-    size_t scale_stride;     // bytes between ranks' scale rows (n/32 rounded up to 16)
+    size_t scale_stride;     // bytes between ranks' scale rows (2n/G rounded up to 16)
     uint32_t chunk_begin, chunk_end;
     uint32_t tile, tile_log2; // set by the launcher: this launch's tile length
     uint32_t lanes_log2;     // log2(G / 8): lanes per group
@@ -73,6 +73,7 @@ struct K1Args {
     bool bf16;
     bool enable;             // the owner adds the correction to its partial
     bool sender_ef;          // every rank adds back and renews its own error
+    bool fp16_scale;         // binary16 scales (rounded up) instead of powers of two
     PipeCtl ctl;
 };
 
@@ -92,6 +93,9 @@ struct K2Args {
     int P;
     bool enable;             // read the state, capture the error, update the state
     bool owner_sum;          // add the correction to the owner's sum
+    bool fp16_scale;         // binary16 scales
+    bool bf16;               // bf16 outputs: under binary16 scales the error is
+                             // taken against the bf16-rounded value ranks receive
     PipeCtl ctl;
 };
 
@@ -105,6 +109,7 @@ struct K3Args {
     uint32_t lanes_log2;     // log2(G / 8): lanes per group
     int P;
     bool bf16;
+    bool fp16_scale;         // binary16 scales: outputs q*s rounded to bf16 when bf16
     PipeCtl ctl;
 };
 

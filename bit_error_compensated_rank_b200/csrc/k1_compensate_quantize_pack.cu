@@ -10,8 +10,13 @@
 // v = RN(RN(x + eps) + c), eps <- v - q*2^e.
 //
 // Layout: the rank partials are P separate buffers of n elements; the output
-// is the stage-1 wire, codes [P][n/2] (two per byte) and scale bytes
-// [P][scale_stride] (n/G per rank); the sender errors are [P][n] binary32.
+// is the stage-1 wire, codes [P][n/2] (two per byte) and scales
+// [P][scale_stride] (n/G bytes per rank, or n/G binary16 patterns under the
+// binary16-scale variant); the sender errors are [P][n] binary32.
+//
+// Two builds of the kernel body: the default one (groups of 32, power-of-two
+// scales, both fixed at compile time) and a general one that takes the group
+// size and the scale format at run time for the variants.
 //
 // Pipeline (warp-specialised, persistent): a CTA takes tiles of kTile
 // consecutive elements. One producer warp bulk-copies the P partial tiles
@@ -87,10 +92,14 @@ __device__ __forceinline__ void load_f32x8(const float *p, float (&v)[kChunk])
     v[4] = b.x, v[5] = b.y, v[6] = b.z, v[7] = b.w;
 }
 
-template <int P, bool BF16, bool COMP, bool EF>
+template <int P, bool BF16, bool COMP, bool EF, bool GEN>
 __global__ void __launch_bounds__(kThreads)
     k1_compensate_quantize_pack(const K1Args a)
 {
+    // group = 8 << lanes_log2 elements; the default build fixes 32 and
+    // power-of-two scales
+    const uint32_t lanes_log2 = GEN ? a.lanes_log2 : 2u;
+    const bool f16 = GEN && a.fp16_scale;
     using Sh = K1Shape<P, BF16, COMP, EF>;
     constexpr int S = Sh::kStages;
     extern __shared__ __align__(128) uint8_t smem[];
@@ -164,7 +173,7 @@ __global__ void __launch_bounds__(kThreads)
             const uint32_t c = it & ((1u << cpt_log2) - 1u);
             const bool active = c < cnt_chunks;
             const uint32_t chunk = tile_chunk0 + c;
-            const uint32_t g = chunk >> a.lanes_log2;
+            const uint32_t g = chunk >> lanes_log2;
 
             float v[kChunk];
             load_chunk<BF16>(stage + r * Sh::kXBytes + c * (kChunk * Sh::kEB), v);
@@ -188,20 +197,36 @@ __global__ void __launch_bounds__(kThreads)
             // max |v| as a tree (fmax is exact, so the order is free)
             const float m01 = fmaxf(fabsf(v[0]), fabsf(v[1])), m23 = fmaxf(fabsf(v[2]), fabsf(v[3]));
             const float m45 = fmaxf(fabsf(v[4]), fabsf(v[5])), m67 = fmaxf(fabsf(v[6]), fabsf(v[7]));
-            const float amax = group_absmax(fmaxf(fmaxf(m01, m23), fmaxf(m45, m67)), a.lanes_log2);
-            const uint32_t byte = scale_byte(amax);
-            const float inv = inv_step_of(byte);
+            const float amax = group_absmax(fmaxf(fmaxf(m01, m23), fmaxf(m45, m67)), lanes_log2);
             uint32_t qb[kChunk];
+            uint32_t scale; // scale byte, or binary16 pattern
+            float st;       // the step q is restored with
+            if (f16) {
+                scale = half_scale_bits(amax);
+                st = half_step(scale);
+                const float inv = half_inv(st);
 #pragma unroll
-            for (int k = 0; k < kChunk; k++)
-                qb[k] = code_bits(v[k], inv);
+                for (int k = 0; k < kChunk; k++)
+                    qb[k] = code_bits_near(v[k], st, inv);
+            } else {
+                scale = scale_byte(amax);
+                st = step_of(scale);
+                const float inv = inv_step_of(scale);
+#pragma unroll
+                for (int k = 0; k < kChunk; k++)
+                    qb[k] = code_bits(v[k], inv);
+            }
             const uint32_t word = pack8_bits(qb);
             if (active) {
                 reinterpret_cast<uint32_t *>(a.codes)[static_cast<size_t>(r) * code_words + chunk] = word;
-                if ((lane & ((1u << a.lanes_log2) - 1u)) == 0) // the group's first lane
-                    a.scales[static_cast<size_t>(r) * a.scale_stride + g] = static_cast<uint8_t>(byte);
-                if (EF) { // the new error v - q*2^e, exact
-                    const float st = step_of(byte);
+                if ((lane & ((1u << lanes_log2) - 1u)) == 0) { // the group's first lane
+                    uint8_t *row = a.scales + static_cast<size_t>(r) * a.scale_stride;
+                    if (f16)
+                        reinterpret_cast<uint16_t *>(row)[g] = static_cast<uint16_t>(scale);
+                    else
+                        row[g] = static_cast<uint8_t>(scale);
+                }
+                if (EF) { // the new error v - q*step (exact unless a binary16 scale saturated)
                     float e[kChunk];
 #pragma unroll
                     for (int k = 0; k < kChunk; k++)
@@ -219,12 +244,12 @@ __global__ void __launch_bounds__(kThreads)
     }
 }
 
-template <int P, bool BF16, bool COMP, bool EF>
+template <int P, bool BF16, bool COMP, bool EF, bool GEN>
 cudaError_t launch_p(const K1Args &a, cudaStream_t st)
 {
     using Sh = K1Shape<P, BF16, COMP, EF>;
     static int resident = 0;
-    auto kern = k1_compensate_quantize_pack<P, BF16, COMP, EF>;
+    auto kern = k1_compensate_quantize_pack<P, BF16, COMP, EF, GEN>;
     if (resident == 0) {
         cudaError_t e = prepare_kernel(reinterpret_cast<const void *>(kern), kThreads, Sh::kSmem, &resident);
         if (e != cudaSuccess)
@@ -238,18 +263,20 @@ cudaError_t launch_p(const K1Args &a, cudaStream_t st)
     return launch_chained(kern, persistent_grid(tiles, resident), kThreads, Sh::kSmem, st, b);
 }
 
-template <int P, bool BF16>
+template <int P, bool BF16, bool GEN>
 cudaError_t dispatch_state(const K1Args &a, cudaStream_t st)
 {
     if (a.enable)
-        return a.sender_ef ? launch_p<P, BF16, true, true>(a, st) : launch_p<P, BF16, true, false>(a, st);
-    return a.sender_ef ? launch_p<P, BF16, false, true>(a, st) : launch_p<P, BF16, false, false>(a, st);
+        return a.sender_ef ? launch_p<P, BF16, true, true, GEN>(a, st) : launch_p<P, BF16, true, false, GEN>(a, st);
+    return a.sender_ef ? launch_p<P, BF16, false, true, GEN>(a, st) : launch_p<P, BF16, false, false, GEN>(a, st);
 }
 
 template <int P>
 cudaError_t dispatch_flags(const K1Args &a, cudaStream_t st)
 {
-    return a.bf16 ? dispatch_state<P, true>(a, st) : dispatch_state<P, false>(a, st);
+    if (a.lanes_log2 != 2u || a.fp16_scale) // a group-size or scale-format variant
+        return a.bf16 ? dispatch_state<P, true, true>(a, st) : dispatch_state<P, false, true>(a, st);
+    return a.bf16 ? dispatch_state<P, true, false>(a, st) : dispatch_state<P, false, false>(a, st);
 }
 
 } // namespace

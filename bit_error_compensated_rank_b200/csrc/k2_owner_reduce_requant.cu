@@ -19,6 +19,12 @@
 // err is exact: S and Y = Q*2^E differ by at most 2^(E-1) and both are
 // multiples of ulp(S).
 //
+// Binary16-scale variant (F16): scales are binary16 patterns (two bytes per
+// group), restored values q*s are still exact, and with bf16 outputs the
+// value every rank receives is q*s rounded to bf16; err is measured against
+// that received value (still exact in binary32: it is a multiple of ulp(S)
+// below 2^(exponent of S)).
+//
 // Pipeline (warp-specialised, persistent): a CTA takes tiles of kTile
 // elements; one producer warp bulk-copies the P code tiles, the P scale tiles
 // and the f, s tiles of a tile into one stage of a kStages ring (mbarrier
@@ -41,29 +47,30 @@ constexpr int kConsumers = kConsumerWarps * 32;
 constexpr int kThreads = kConsumers + 32; // + one producer warp
 
 // Bytes of one stage for `chunks` chunks per consumer thread: P code tiles,
-// P scale tiles, and the f, s tiles.
-constexpr int k2_stage_bytes(int P, bool comp, int chunks)
+// P scale tiles (1 or 2 bytes per group of at least kMinGroup), and the f, s
+// tiles.
+constexpr int k2_stage_bytes(int P, bool comp, bool f16, int chunks)
 {
-    return P * (kConsumers * kChunk * chunks / 2 + kConsumers * kChunk * chunks / kMinGroup) +
+    return P * (kConsumers * kChunk * chunks / 2 + kConsumers * kChunk * chunks / kMinGroup * (f16 ? 2 : 1)) +
            (comp ? 2 * kConsumers * kChunk * chunks * 4 : 0);
 }
 
 // The largest of ECHO_K2_CHUNKS, /2, /4 whose stages fit the budget.
-constexpr int k2_chunks(int P, bool comp)
+constexpr int k2_chunks(int P, bool comp, bool f16)
 {
     int c = ECHO_K2_CHUNKS;
-    while (c > 1 && ECHO_K2_STAGES * k2_stage_bytes(P, comp, c) + 64 > ECHO_SMEM_BUDGET)
+    while (c > 1 && ECHO_K2_STAGES * k2_stage_bytes(P, comp, f16, c) + 64 > ECHO_SMEM_BUDGET)
         c /= 2;
     return c;
 }
 
-template <int P, bool COMP>
+template <int P, bool COMP, bool F16>
 struct K2Shape {
-    static constexpr int kChunks = k2_chunks(P, COMP);    // chunks per consumer thread
+    static constexpr int kChunks = k2_chunks(P, COMP, F16); // chunks per consumer thread
     static constexpr int kTile = kConsumers * kChunk * kChunks;
     static constexpr int kStages = ECHO_K2_STAGES;
     static constexpr int kCodeBytes = kTile / 2;          // one rank's code tile
-    static constexpr int kScaleBytes = kTile / kMinGroup; // room for one rank's scale tile
+    static constexpr int kScaleBytes = kTile / kMinGroup * (F16 ? 2 : 1); // room for one rank's scale tile
     static constexpr int kStateOff = P * (kCodeBytes + kScaleBytes);
     static constexpr int kStageBytes = kStateOff + (COMP ? 2 * kTile * 4 : 0);
     static constexpr int kSmem = kStages * kStageBytes + 2 * kStages * 8;
@@ -72,11 +79,12 @@ struct K2Shape {
 
 __device__ __forceinline__ uint32_t round16(uint32_t x) { return (x + 15u) & ~15u; }
 
-template <int P, bool COMP, bool SUM>
+template <int P, bool COMP, bool SUM, bool F16>
 __global__ void __launch_bounds__(kThreads)
     k2_owner_reduce_requant(const K2Args a)
 {
-    using Sh = K2Shape<P, COMP>;
+    using Sh = K2Shape<P, COMP, F16>;
+    constexpr uint32_t kScaleLog2 = F16 ? 1u : 0u; // log2 of the bytes per scale
     constexpr int S = Sh::kStages;
     extern __shared__ __align__(128) uint8_t smem[];
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + S * Sh::kStageBytes);
@@ -112,7 +120,7 @@ __global__ void __launch_bounds__(kThreads)
                 full, empty, mine, a.ctl.stall, a.ctl.wait_cycles, a.ctl.status, kStatusTimeoutK2, [&](uint32_t i) {
                     const size_t el0 = e0 + static_cast<size_t>(blockIdx.x + i * gridDim.x) * tile;
                     const uint32_t cnt = static_cast<uint32_t>(e1 - el0 < size_t(tile) ? e1 - el0 : tile);
-                    const uint32_t sc_bytes = round16(cnt >> (a.lanes_log2 + 3));
+                    const uint32_t sc_bytes = round16((cnt >> (a.lanes_log2 + 3)) << kScaleLog2);
                     uint8_t *stage = smem + (i % S) * Sh::kStageBytes;
                     uint64_t *bar = &full[i % S];
                     mbar_arrive_expect_tx(bar, P * (cnt / 2 + sc_bytes) + (COMP ? 2 * cnt * 4 : 0));
@@ -120,7 +128,8 @@ __global__ void __launch_bounds__(kThreads)
                     for (int r = 0; r < P; r++) {
                         bulk_load(stage + r * Sh::kCodeBytes, a.codes + r * (a.n / 2) + el0 / 2, cnt / 2, bar);
                         bulk_load(stage + P * Sh::kCodeBytes + r * Sh::kScaleBytes,
-                                  a.scales + r * a.scale_stride + (el0 >> (a.lanes_log2 + 3)), sc_bytes, bar);
+                                  a.scales + r * a.scale_stride + ((el0 >> (a.lanes_log2 + 3)) << kScaleLog2),
+                                  sc_bytes, bar);
                     }
                     if (COMP) {
                         bulk_load(stage + Sh::kStateOff, a.f + el0, cnt * 4, bar);
@@ -156,8 +165,8 @@ __global__ void __launch_bounds__(kThreads)
                 sv[4] = s1.x, sv[5] = s1.y, sv[6] = s1.z, sv[7] = s1.w;
             }
 
-            // Restore and add, rank 0 first. The product q*2^e is exact, so
-            // fma(q, 2^e, S) = RN(S + q*2^e): one rounding per addition.
+            // Restore and add, rank 0 first. The product q*step is exact, so
+            // fma(q, step, S) = RN(S + q*step): one rounding per addition.
             float S_[kChunk];
 #pragma unroll
             for (int k = 0; k < kChunk; k++)
@@ -165,8 +174,9 @@ __global__ void __launch_bounds__(kThreads)
 #pragma unroll
             for (int r = 0; r < P; r++) {
                 const uint32_t w = reinterpret_cast<const uint32_t *>(stage + r * Sh::kCodeBytes)[c];
-                const uint32_t b = stage[P * Sh::kCodeBytes + r * Sh::kScaleBytes + (c >> a.lanes_log2)];
-                const float st = step_of(b);
+                const uint8_t *srow = stage + P * Sh::kCodeBytes + r * Sh::kScaleBytes;
+                const float st = F16 ? half_step(reinterpret_cast<const uint16_t *>(srow)[c >> a.lanes_log2])
+                                     : step_of(srow[c >> a.lanes_log2]);
                 const Unpacked u = unpack8(w);
 #pragma unroll
                 for (int k = 0; k < kChunk; k++)
@@ -183,21 +193,38 @@ __global__ void __launch_bounds__(kThreads)
             const float m01 = fmaxf(fabsf(S_[0]), fabsf(S_[1])), m23 = fmaxf(fabsf(S_[2]), fabsf(S_[3]));
             const float m45 = fmaxf(fabsf(S_[4]), fabsf(S_[5])), m67 = fmaxf(fabsf(S_[6]), fabsf(S_[7]));
             const float amax = group_absmax(fmaxf(fmaxf(m01, m23), fmaxf(m45, m67)), a.lanes_log2);
-            const uint32_t byte = scale_byte(amax);
-            const float inv = inv_step_of(byte);
-            const float st = step_of(byte);
             uint32_t qb[kChunk];
             float err[kChunk];
+            uint32_t scale;
+            if (F16) {
+                scale = half_scale_bits(amax);
+                const float st = half_step(scale);
+                const float inv = half_inv(st);
 #pragma unroll
-            for (int k = 0; k < kChunk; k++) {
-                qb[k] = code_bits(S_[k], inv);
-                err[k] = __fmaf_rn(-code_value(qb[k]), st, S_[k]); // S - Q*2^E, exact
+                for (int k = 0; k < kChunk; k++) {
+                    qb[k] = code_bits_near(S_[k], st, inv);
+                    const float y = __fmul_rn(code_value(qb[k]), st); // exact
+                    err[k] = __fsub_rn(S_[k], a.bf16 ? round_bf16(y) : y);
+                }
+            } else {
+                scale = scale_byte(amax);
+                const float inv = inv_step_of(scale);
+                const float st = step_of(scale);
+#pragma unroll
+                for (int k = 0; k < kChunk; k++) {
+                    qb[k] = code_bits(S_[k], inv);
+                    err[k] = __fmaf_rn(-code_value(qb[k]), st, S_[k]); // S - Q*2^E, exact
+                }
             }
 
             if (active) {
                 reinterpret_cast<uint32_t *>(a.qcodes)[chunk] = pack8_bits(qb);
-                if ((lane & ((1u << a.lanes_log2) - 1u)) == 0) // the group's first lane
-                    a.qscales[g] = static_cast<uint8_t>(byte);
+                if ((lane & ((1u << a.lanes_log2) - 1u)) == 0) { // the group's first lane
+                    if (F16)
+                        reinterpret_cast<uint16_t *>(a.qscales)[g] = static_cast<uint16_t>(scale);
+                    else
+                        a.qscales[g] = static_cast<uint8_t>(scale);
+                }
                 if (COMP) {
 #pragma unroll
                     for (int k = 0; k < kChunk; k++) {
@@ -219,12 +246,12 @@ __global__ void __launch_bounds__(kThreads)
     }
 }
 
-template <int P, bool COMP, bool SUM>
+template <int P, bool COMP, bool SUM, bool F16>
 cudaError_t launch_p(const K2Args &a, cudaStream_t st)
 {
-    using Sh = K2Shape<P, COMP>;
+    using Sh = K2Shape<P, COMP, F16>;
     static int resident = 0;
-    auto kern = k2_owner_reduce_requant<P, COMP, SUM>;
+    auto kern = k2_owner_reduce_requant<P, COMP, SUM, F16>;
     if (resident == 0) {
         cudaError_t e = prepare_kernel(reinterpret_cast<const void *>(kern), kThreads, Sh::kSmem, &resident);
         if (e != cudaSuccess)
@@ -238,12 +265,18 @@ cudaError_t launch_p(const K2Args &a, cudaStream_t st)
     return launch_chained(kern, persistent_grid(tiles, resident), kThreads, Sh::kSmem, st, b);
 }
 
+template <int P, bool F16>
+cudaError_t dispatch_state(const K2Args &a, cudaStream_t st)
+{
+    if (!a.enable)
+        return launch_p<P, false, false, F16>(a, st);
+    return a.owner_sum ? launch_p<P, true, true, F16>(a, st) : launch_p<P, true, false, F16>(a, st);
+}
+
 template <int P>
 cudaError_t dispatch_flags(const K2Args &a, cudaStream_t st)
 {
-    if (!a.enable)
-        return launch_p<P, false, false>(a, st);
-    return a.owner_sum ? launch_p<P, true, true>(a, st) : launch_p<P, true, false>(a, st);
+    return a.fp16_scale ? dispatch_state<P, true>(a, st) : dispatch_state<P, false>(a, st);
 }
 
 } // namespace

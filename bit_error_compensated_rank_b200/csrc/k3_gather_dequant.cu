@@ -4,7 +4,10 @@
 // [rit.work "Echo 4-bit GPU communication", section "How Echo returns the
 // error to later calls": the compressed total is sent back to every rank].
 // Y = Q*2^E has at most three significant bits, so it is exact in bf16 and
-// in binary32: the restore adds no third rounding.
+// in binary32: the restore adds no third rounding. Under the binary16-scale
+// variant (F16) Y = Q*s has up to 14 significant bits: exact in binary32,
+// rounded to the nearest bf16 (ties to even) for bf16 outputs, the value
+// kernel 2 measured its error against.
 //
 // Pipeline (warp-specialised, persistent): a CTA takes tiles of kTile
 // elements. A load warp bulk-copies the tile's codes and scale bytes into a
@@ -29,14 +32,14 @@ constexpr int kLoadWarp = kConsumerWarps;
 constexpr int kStoreWarp = kConsumerWarps + 1;
 constexpr int kThreads = kConsumers + 64;
 
-template <bool BF16>
+template <bool BF16, bool F16>
 struct K3Shape {
     static constexpr int kEB = BF16 ? 2 : 4;
     static constexpr int kTile = BF16 ? ECHO_K3_TILE : ECHO_K3_TILE / 2;
     static constexpr int kInStages = ECHO_K3_IN_STAGES;
     static constexpr int kOutBufs = ECHO_K3_OUT_BUFS;
     static constexpr int kCodeBytes = kTile / 2;
-    static constexpr int kScaleBytes = kTile / kMinGroup; // room for the tile's scale bytes
+    static constexpr int kScaleBytes = kTile / kMinGroup * (F16 ? 2 : 1); // room for the tile's scales
     static constexpr int kInBytes = kCodeBytes + kScaleBytes;
     static constexpr int kOutBytes = kTile * kEB;
     static constexpr int kOutOff = kInStages * kInBytes;
@@ -47,11 +50,12 @@ struct K3Shape {
 
 __device__ __forceinline__ uint32_t round16(uint32_t x) { return (x + 15u) & ~15u; }
 
-template <int P, bool BF16>
+template <int P, bool BF16, bool F16>
 __global__ void __launch_bounds__(kThreads)
     k3_gather_dequant(const K3Args a)
 {
-    using Sh = K3Shape<BF16>;
+    using Sh = K3Shape<BF16, F16>;
+    constexpr uint32_t kScaleLog2 = F16 ? 1u : 0u; // log2 of the bytes per scale
     constexpr int S = Sh::kInStages;
     constexpr int B = Sh::kOutBufs;
     extern __shared__ __align__(128) uint8_t smem[];
@@ -97,12 +101,13 @@ __global__ void __launch_bounds__(kThreads)
                              kStatusTimeoutK3, [&](uint32_t i) {
                                  const size_t el0 = tile_start(i);
                                  const uint32_t cnt = tile_count(el0);
-                                 const uint32_t sc_bytes = round16(cnt >> (a.lanes_log2 + 3));
+                                 const uint32_t sc_bytes = round16((cnt >> (a.lanes_log2 + 3)) << kScaleLog2);
                                  uint8_t *stage = smem + (i % S) * Sh::kInBytes;
                                  uint64_t *bar = &in_full[i % S];
                                  mbar_arrive_expect_tx(bar, cnt / 2 + sc_bytes);
                                  bulk_load(stage, a.qcodes + el0 / 2, cnt / 2, bar);
-                                 bulk_load(stage + Sh::kCodeBytes, a.qscales + (el0 >> (a.lanes_log2 + 3)), sc_bytes, bar);
+                                 bulk_load(stage + Sh::kCodeBytes,
+                                           a.qscales + ((el0 >> (a.lanes_log2 + 3)) << kScaleLog2), sc_bytes, bar);
                              });
         return;
     }
@@ -146,13 +151,22 @@ __global__ void __launch_bounds__(kThreads)
         for (uint32_t j = 0; j < tile / (kChunk * kConsumers); j++) {
             const uint32_t c = tid + j * kConsumers;
             const uint32_t w = reinterpret_cast<const uint32_t *>(stage)[c];
-            const float st = step_of(stage[Sh::kCodeBytes + (c >> a.lanes_log2)]);
+            const float st =
+                F16 ? half_step(reinterpret_cast<const uint16_t *>(stage + Sh::kCodeBytes)[c >> a.lanes_log2])
+                    : step_of(stage[Sh::kCodeBytes + (c >> a.lanes_log2)]);
             const Unpacked u = unpack8(w);
             float y[kChunk];
 #pragma unroll
             for (int k = 0; k < kChunk; k++)
                 y[k] = __fmul_rn(code_at(u, k), st);
-            if (BF16) {
+            if (BF16 && F16) { // round to the nearest bf16
+                uint32_t w2[4];
+#pragma unroll
+                for (int j = 0; j < 4; j++)
+                    w2[j] = __float_as_uint(round_bf16(y[2 * j])) >> 16 |
+                            (__float_as_uint(round_bf16(y[2 * j + 1])) & 0xFFFF0000u);
+                reinterpret_cast<uint4 *>(out)[c] = make_uint4(w2[0], w2[1], w2[2], w2[3]);
+            } else if (BF16) {
                 reinterpret_cast<uint4 *>(out)[c] = f32x8_to_bf16_exact(y);
             } else {
                 reinterpret_cast<float4 *>(out)[2 * c] = make_float4(y[0], y[1], y[2], y[3]);
@@ -168,12 +182,12 @@ __global__ void __launch_bounds__(kThreads)
     }
 }
 
-template <int P, bool BF16>
+template <int P, bool BF16, bool F16>
 cudaError_t launch_p(const K3Args &a, cudaStream_t st)
 {
-    using Sh = K3Shape<BF16>;
+    using Sh = K3Shape<BF16, F16>;
     static int resident = 0;
-    auto kern = k3_gather_dequant<P, BF16>;
+    auto kern = k3_gather_dequant<P, BF16, F16>;
     if (resident == 0) {
         cudaError_t e = prepare_kernel(reinterpret_cast<const void *>(kern), kThreads, Sh::kSmem, &resident);
         if (e != cudaSuccess)
@@ -190,7 +204,9 @@ cudaError_t launch_p(const K3Args &a, cudaStream_t st)
 template <int P>
 cudaError_t dispatch_flags(const K3Args &a, cudaStream_t st)
 {
-    return a.bf16 ? launch_p<P, true>(a, st) : launch_p<P, false>(a, st);
+    if (a.fp16_scale)
+        return a.bf16 ? launch_p<P, true, true>(a, st) : launch_p<P, false, true>(a, st);
+    return a.bf16 ? launch_p<P, true, false>(a, st) : launch_p<P, false, false>(a, st);
 }
 
 } // namespace

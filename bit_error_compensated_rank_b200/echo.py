@@ -30,6 +30,7 @@ ECHO_MAX_RANKS = 16
 ECHO_GROUP = 32
 ECHO_VARIANT_OWNER_SUM = 1
 ECHO_VARIANT_SENDER_EF = 2
+ECHO_VARIANT_FP16_SCALE = 4
 
 EXPORTED = (
     "echo_create", "echo_allreduce", "echo_allreduce_out", "echo_allreduce_host",
@@ -184,17 +185,20 @@ def echo_get_state_range(h: int, phase: int, offset: int, count: int):
     return f, s
 
 
-def echo_get_wire(h: int, stage: int, rank: int, n: int, group: int = ECHO_GROUP):
+def echo_get_wire(h: int, stage: int, rank: int, n: int, group: int = ECHO_GROUP,
+                  fp16_scale: bool = False):
+    """Codes (uint8) and scales: uint8 bytes, or uint16 binary16 patterns
+    when the handle runs ECHO_VARIANT_FP16_SCALE (say so with fp16_scale)."""
     codes = np.empty(n // 2, np.uint8)
-    scales = np.empty(n // group, np.uint8)
+    scales = np.empty(n // group, np.uint16 if fp16_scale else np.uint8)
     _check(_lib.echo_get_wire(h, stage, rank, _np(codes, _u8p), _np(scales, _u8p)))
     return codes, scales
 
 
 def echo_get_wire_range(h: int, stage: int, rank: int, group_offset: int, ngroups: int,
-                        group: int = ECHO_GROUP):
+                        group: int = ECHO_GROUP, fp16_scale: bool = False):
     codes = np.empty(ngroups * group // 2, np.uint8)
-    scales = np.empty(ngroups, np.uint8)
+    scales = np.empty(ngroups, np.uint16 if fp16_scale else np.uint8)
     _check(_lib.echo_get_wire_range(h, stage, rank, group_offset, ngroups,
                                     _np(codes, _u8p), _np(scales, _u8p)))
     return codes, scales
@@ -282,6 +286,7 @@ class Echo:
 
     def __init__(self, P: int, n: int, dtype: int = ECHO_BF16, group: int = ECHO_GROUP):
         self.P, self.n, self.dtype, self.group = P, n, dtype, group
+        self.variant = 0
         self._arrays = {}
         self.h = echo_create(P, n, group, dtype)
 
@@ -316,6 +321,7 @@ class Echo:
 
     def set_variant(self, variant: int) -> None:
         echo_set_variant(self.h, variant)
+        self.variant = variant
 
     def get_sender_state(self, phase: int, rank: int, offset: int = 0, count: int | None = None):
         return echo_get_sender_state(self.h, phase, rank, offset, self.n - offset if count is None else count)
@@ -333,10 +339,12 @@ class Echo:
         return echo_get_state_range(self.h, phase, offset, count)
 
     def get_wire(self, stage: int, rank: int = 0):
-        return echo_get_wire(self.h, stage, rank, self.n, self.group)
+        return echo_get_wire(self.h, stage, rank, self.n, self.group,
+                             bool(self.variant & ECHO_VARIANT_FP16_SCALE))
 
     def get_wire_range(self, stage: int, rank: int, group_offset: int, ngroups: int):
-        return echo_get_wire_range(self.h, stage, rank, group_offset, ngroups, self.group)
+        return echo_get_wire_range(self.h, stage, rank, group_offset, ngroups, self.group,
+                                   bool(self.variant & ECHO_VARIANT_FP16_SCALE))
 
     def stats(self) -> dict:
         return echo_stats(self.h)

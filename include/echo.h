@@ -81,8 +81,9 @@ enum {
  *          wire then costs 1/2 + 1/group bytes per element.
  *   dtype  ECHO_BF16 or ECHO_FP32: the element type of the rank buffers.
  * Allocates on the current device: stage-1 wire (P x n/2 code bytes and
- * P x n/group scale bytes), the requantised wire (n/2 + n/group bytes) and the
- * compensator state (2 phases x 2 estimates x n binary32, zeroed).
+ * P x 2n/group scale bytes, room for binary16 scales), the requantised wire
+ * (n/2 + 2n/group bytes) and the compensator state (2 phases x 2 estimates x
+ * n binary32, zeroed).
  * Returns NULL on any error (see echo_last_error). The handle is bound to the
  * device that was current at creation.
  */
@@ -186,6 +187,15 @@ ECHO_API int echo_set_params(echo_handle *h, float beta_fast, float beta_slow, f
  *       binary32 per element per rank and phase (zeroed when first switched
  *       on; allocated then, ECHO_ERR_OOM if that fails). With both roundings
  *       fed back the running sum of all injected error stays bounded.
+ *   ECHO_VARIANT_FP16_SCALE  a scale format variant for both roundings: each
+ *       group's scale is the smallest positive finite binary16 s with
+ *       7*s >= max|v| (0 for an all-zero group; 65504 past 7*65504, where
+ *       codes saturate at +-7), stored as two little-endian bytes; each code
+ *       is the integer in [-7, 7] nearest to v/s, ties to even. Restored
+ *       values q*s are exact in binary32; bf16 outputs are q*s rounded to the
+ *       nearest bf16 (ties to even), and the owner's captured error is taken
+ *       against that received value. The wire costs 1/2 + 2/group bytes per
+ *       element; steps follow max|v| within 2^-10 instead of a factor of 2.
  * The pages say the error a rounding injects is stored and added back in later
  * calls [rit.work "Echo 4-bit GPU communication", section "How Echo returns
  * the error to later calls"] and that the high-precision sum reveals every
@@ -194,6 +204,7 @@ ECHO_API int echo_set_params(echo_handle *h, float beta_fast, float beta_slow, f
  */
 #define ECHO_VARIANT_OWNER_SUM 1
 #define ECHO_VARIANT_SENDER_EF 2
+#define ECHO_VARIANT_FP16_SCALE 4
 ECHO_API int echo_set_variant(echo_handle *h, int variant);
 
 /* Synchronous copies of rank `rank`'s sender errors for `phase` (elements
@@ -215,7 +226,9 @@ ECHO_API int echo_get_state_range(echo_handle *h, int phase, size_t offset, size
 
 /*
  * echo_get_wire - synchronous copy of the wire left by the last call.
- *   stage 1: rank's packed codes (n/2 bytes) and scale bytes (n/group);
+ *   stage 1: rank's packed codes (n/2 bytes) and scales (n/group bytes, or
+ *            n/group little-endian binary16 patterns under
+ *            ECHO_VARIANT_FP16_SCALE: 2n/group bytes);
  *   stage 2: the requantised total (rank ignored).
  * Either output pointer may be NULL to skip it.
  */
@@ -223,7 +236,7 @@ ECHO_API int echo_get_wire(echo_handle *h, int stage, int rank, uint8_t *codes_h
                   uint8_t *scales_host);
 
 /* Range variant over groups [group_offset, group_offset+ngroups):
- * group/2 * ngroups code bytes and ngroups scale bytes. */
+ * group/2 * ngroups code bytes and ngroups scales (1 or 2 bytes each). */
 ECHO_API int echo_get_wire_range(echo_handle *h, int stage, int rank, size_t group_offset,
                         size_t ngroups, uint8_t *codes_host, uint8_t *scales_host);
 
@@ -248,8 +261,9 @@ ECHO_API int echo_stats(echo_handle *h, uint64_t *link_bytes, uint64_t *model_hb
 ECHO_API int echo_model_bytes(int P, size_t n, int dtype, int enable, uint64_t out[4]);
 
 /* The same for any group size and variant: the wire is 1/2 + 1/group bytes
- * per element; OWNER_SUM drops kernel 1's 8 state bytes; SENDER_EF adds 8P
- * bytes (each rank's error read and written) to kernel 1. */
+ * per element (1/2 + 2/group with FP16_SCALE); OWNER_SUM drops kernel 1's 8
+ * state bytes; SENDER_EF adds 8P bytes (each rank's error read and written)
+ * to kernel 1. */
 ECHO_API int echo_model_bytes_ex(int P, size_t n, int group, int dtype, int enable, int variant,
                                  uint64_t out[4]);
 

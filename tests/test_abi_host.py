@@ -58,12 +58,15 @@ def test_model_bytes_per_element(echo):
     assert abs(f32["total"] / 65536 - (2 * 8 * 4 + 25 * w + 24)) < 1e-12
 
 
+@pytest.mark.parametrize("fp16", [False, True])
 @pytest.mark.parametrize("group", [16, 32, 64, 128])
-def test_model_bytes_group_sizes(echo, group):
-    # the wire costs 1/2 + 1/group bytes per element, the rest is unchanged
+def test_model_bytes_group_sizes(echo, group, fp16):
+    # the wire costs 1/2 + 1/group bytes per element (2/group with binary16
+    # scales), the rest is unchanged
     P, n = 8, 1 << 29
-    mb = echo.echo_model_bytes_ex(P, n, group, echo.ECHO_BF16, True, 0)
-    w = 0.5 + 1 / group
+    mb = echo.echo_model_bytes_ex(P, n, group, echo.ECHO_BF16, True,
+                                  echo.ECHO_VARIANT_FP16_SCALE if fp16 else 0)
+    w = 0.5 + (2 if fp16 else 1) / group
     assert mb["k1"] == round((P * 2 + 8 + P * w) * n)
     assert mb["k2"] == round((P * w + 16 + w) * n)
     assert mb["k3"] == round((P * w + P * 2) * n)
