@@ -45,6 +45,7 @@ SEED = 0
 WORKLOAD = "echo int4 all-reduce, P=8 ranks x 1 GiB bf16 per rank (2^29 elements), group 32, " \
            "compensation on, fwd state, partials N(0,1) with 0.1% at 50x"
 HBM_FALLBACK_GBS = 6650.0  # used only when MEASURED_PEAKS.json is absent
+L2_BYTES = 126 * 10 ** 6
 # where the rounding errors are fed back, and the scale format (see
 # include/echo.h, echo_set_variant)
 VARIANTS = {"default": 0, "owner_sum": 1, "sender_ef": 2, "both": 3, "fp16_scale": 4}
@@ -210,23 +211,68 @@ def oracle_sample_rate(n_sample: int, budget_s: float, min_calls: int, max_calls
     return times
 
 
+def host_info() -> dict:
+    """CPU model, logical cores and RAM of the host the oracle runs on."""
+    info = {"nproc": os.cpu_count(), "cpu_model": None, "ram_gb": None}
+    try:
+        with open("/proc/cpuinfo") as fh:
+            for line in fh:
+                if line.startswith("model name"):
+                    info["cpu_model"] = line.split(":", 1)[1].strip()
+                    break
+        with open("/proc/meminfo") as fh:
+            for line in fh:
+                if line.startswith("MemTotal"):
+                    info["ram_gb"] = round(int(line.split()[1]) / 2 ** 20, 1)
+                    break
+    except OSError:
+        pass
+    return info
+
+
+class one_core:
+    """Pin this process to one core (the first it may use) while timing the
+    single-threaded oracle; restore the previous set afterwards."""
+
+    def __enter__(self):
+        self.prev = None
+        if hasattr(os, "sched_getaffinity"):
+            try:
+                self.prev = os.sched_getaffinity(0)
+                os.sched_setaffinity(0, {min(self.prev)})
+            except OSError:
+                self.prev = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.prev is not None:
+            try:
+                os.sched_setaffinity(0, self.prev)
+            except OSError:
+                pass
+        return False
+
+
 def cpu_baseline_leg(variant: int = 0) -> dict:
-    times = oracle_sample_rate(CPU_SAMPLE_N, budget_s=10.0, min_calls=3, max_calls=60, seed=1,
-                               variant=variant)
+    with one_core():
+        times = oracle_sample_rate(CPU_SAMPLE_N, budget_s=15.0, min_calls=3, max_calls=80, seed=1,
+                                   variant=variant)
     t = sum(times) / len(times)
     return {
         "value": round(2 * CPU_SAMPLE_N / t / 1e9, 6), "unit": UNIT, "cores": 1, "kind": "oracle",
         "sample": f"P=8 x 2^20 bf16 elements per rank (2 MiB), same distribution, compensation on, "
-                  f"{len(times)} sequential calls, {sum(times):.1f} s single-threaded; "
-                  f"value = 2*n/t per call (bf16-equivalent)",
+                  f"{len(times)} sequential calls, {sum(times):.1f} s single-threaded on one pinned "
+                  f"core; value = 2*n/t per call (bf16-equivalent)",
+        "host": host_info(),
     }
 
 
 def run_reference(args, rank: int, world: int) -> dict | None:
     if rank != 0:
         return None
-    times = oracle_sample_rate(REF_SAMPLE_N, budget_s=0.0, min_calls=args.warmup + args.steps,
-                               max_calls=args.warmup + args.steps, seed=2)
+    with one_core():
+        times = oracle_sample_rate(REF_SAMPLE_N, budget_s=0.0, min_calls=args.warmup + args.steps,
+                                   max_calls=args.warmup + args.steps, seed=2)
     timed = times[args.warmup:]
     t = sum(timed) / len(timed)
     value = 2 * REF_SAMPLE_N / t / 1e9
@@ -240,7 +286,7 @@ def run_reference(args, rank: int, world: int) -> dict | None:
         "config": {"workload": WORKLOAD, "P": P, "n_per_rank": N_ELEMS, "sample_n_per_rank": REF_SAMPLE_N,
                    "parallelism": f"{world} independent replica(s)"},
         "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": 1, "kind": "oracle",
-                         "sample": sample},
+                         "sample": sample, "host": host_info()},
         "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
@@ -263,9 +309,15 @@ def workload_name(args) -> str:
 
 
 def _source_hash(path: str) -> str:
+    """First 16 hex digits of the sha256 of a kernel's .cu file followed by
+    its .cuh body, when it has one."""
     import hashlib
-    with open(path, "rb") as fh:
-        return hashlib.sha256(fh.read()).hexdigest()[:16]
+    h = hashlib.sha256()
+    for p in (path, path[:-3] + ".cuh"):
+        if os.path.exists(p):
+            with open(p, "rb") as fh:
+                h.update(fh.read())
+    return h.hexdigest()[:16]
 
 
 def run_echo(args, rank: int, world: int, local: int) -> dict | None:
@@ -439,6 +491,15 @@ def run_sweep(args) -> None:
         end.record(stream)
         torch.cuda.synchronize()
         ms = start.elapsed_time(end) / calls
+        # (a') 16 calls timed one by one (events around each): the median
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(16)]
+        for e_start, e_end in evs:
+            e_start.record(stream)
+            h.allreduce_out(s_views, r_views, 0, stream)
+            e_end.record(stream)
+        torch.cuda.synchronize()
+        ms_median = statistics.median(a.elapsed_time(b) for a, b in evs)
         # (b) the same calls captured once in a CUDA graph and replayed: GPU time
         per_graph = min(calls, 50)
         graph = torch.cuda.CUDAGraph()
@@ -459,6 +520,9 @@ def run_sweep(args) -> None:
         print(json.dumps({"sweep": True, "variant": args.variant, "group": args.group, "n_per_rank": n,
                           "msg_bytes": 2 * n, "calls": calls,
                           "us_per_call": round(ms * 1e3, 2),
+                          "us_per_call_median16": round(ms_median * 1e3, 2),
+                          # the call's bytes fit the 126 MB L2: may read above the HBM roofline
+                          "l2_resident": mb["total"] < L2_BYTES,
                           "us_per_call_graph": round(ms_graph * 1e3, 2),
                           "algbw_GBs": round(2 * n / (ms * 1e-3) / 1e9, 2),
                           "algbw_graph_GBs": round(2 * n / (ms_graph * 1e-3) / 1e9, 2),

@@ -116,23 +116,24 @@ __device__ __forceinline__ uint32_t half_scale_bits(float A)
 
 // Bit pattern kRoundBits + q of the code q in [-7, 7] nearest to v/step, a
 // tie going to the even code, for any step >= 0 (inv an estimate of 1/step,
-// 0 when step is 0). The estimate k = nearest integer to v*inv can only miss
-// by one, next to a midpoint; the remainder r = v - k*step is exact there
-// (|r| <= step/2 needs at most 24 significant bits), so comparing |r| with
-// the exact step/2 moves k to the nearest code, or off an odd code on a tie.
-// A saturated group (v/step beyond 7.5) ends at +-7 after the clamp.
-__device__ __forceinline__ uint32_t code_bits_near(float v, float step, float inv)
+// 0 when step is 0; half = step/2, exact). The estimate k = nearest integer
+// to v*inv can only miss by one, next to a midpoint; the remainder
+// r = v - k*step is exact there (|r| <= step/2 needs at most 24 significant
+// bits), so comparing |r| with half moves k to the nearest code, or off an
+// odd code on a tie. The pattern kRound + k has k's parity in its last bit
+// and moves by one per code. A saturated group (v/step beyond 7.5) ends at
+// +-7 after the clamp.
+__device__ __forceinline__ uint32_t code_bits_near(float v, float step, float inv, float half)
 {
     const float y = fminf(fmaxf(__fmul_rn(v, inv), -8.f), 8.f);
-    float k = __fsub_rn(__fadd_rn(y, kRound), kRound);
-    const float r = __fmaf_rn(-k, step, v);
-    const float half = __fmul_rn(0.5f, step);
+    const float t = __fadd_rn(y, kRound);
+    const float r = __fmaf_rn(-__fsub_rn(t, kRound), step, v);
     const float ar = fabsf(r);
-    const bool odd = (__float_as_uint(__fadd_rn(k, kRound)) & 1u) != 0u;
-    if (ar > half || (ar == half && odd))
-        k = __fadd_rn(k, r < 0.f ? -1.f : 1.f);
-    k = fminf(fmaxf(k, -7.f), 7.f);
-    return __float_as_uint(__fadd_rn(k, kRound));
+    int bits = __float_as_int(t);
+    if (ar > half || (ar == half && (bits & 1)))
+        bits += r < 0.f ? -1 : 1;
+    bits = min(max(bits, static_cast<int>(kRoundBits) - 7), static_cast<int>(kRoundBits) + 7);
+    return static_cast<uint32_t>(bits);
 }
 
 // Reciprocal estimate used by code_bits_near (0 for a zero step).

@@ -115,6 +115,13 @@ struct K3Args {
 
 // Each returns the launch's cudaError_t (cudaSuccess when enqueued).
 cudaError_t launch_k1_compensate_quantize_pack(const K1Args &a, cudaStream_t st);
+// The general build of kernel 1 (group size and scale format at run time),
+// one function per element type and sender-feedback setting; called by
+// launch_k1_compensate_quantize_pack for the variants.
+cudaError_t launch_k1_variant_bf16(const K1Args &a, cudaStream_t st);
+cudaError_t launch_k1_variant_bf16_ef(const K1Args &a, cudaStream_t st);
+cudaError_t launch_k1_variant_fp32(const K1Args &a, cudaStream_t st);
+cudaError_t launch_k1_variant_fp32_ef(const K1Args &a, cudaStream_t st);
 cudaError_t launch_k2_owner_reduce_requant(const K2Args &a, cudaStream_t st);
 cudaError_t launch_k3_gather_dequant(const K3Args &a, cudaStream_t st);
 

@@ -1,0 +1,330 @@
+// k1_compensate_quantize_pack.cuh - kernel 1 of the Echo all-reduce (body).
+//
+// Every rank rounds its partial to 4-bit codes per group of 32 (rounding #1);
+// on its own segment the owner first adds the correction
+// c = lambda*f + (1-lambda)*s built from the two smoothed error estimates
+// [rit.work "Echo 4-bit GPU communication", section "How Echo returns the
+// error to later calls": the stored error is added back in later calls].
+// With sender feedback (a variant), every rank first adds back its own
+// rounding-#1 error of its previous call and stores the new one, exact:
+// v = RN(RN(x + eps) + c), eps <- v - q*2^e.
+//
+// Layout: the rank partials are P separate buffers of n elements; the output
+// is the stage-1 wire, codes [P][n/2] (two per byte) and scales
+// [P][scale_stride] (n/G bytes per rank, or n/G binary16 patterns under the
+// binary16-scale variant); the sender errors are [P][n] binary32.
+//
+// Two builds of the kernel: the default one (groups of 32, power-of-two
+// scales) and a general one for the variants, which selects once per launch
+// a consumer body compiled for the launch's group size and scale format.
+//
+// Pipeline (warp-specialised, persistent): a CTA takes tiles of kTile
+// consecutive elements. One producer warp bulk-copies the P partial tiles
+// (and the f, s tiles, and the P error tiles, when used) of a tile into one
+// stage of a kStages ring in shared memory (mbarrier full[s] counts the
+// bytes); eight consumer warps compute from shared memory and release the
+// stage on mbarrier empty[s]. A lane owns 8 consecutive elements of one rank;
+// G/8 lanes form a group and find its maximum with log2(G/8) shuffles; codes
+// leave as one coalesced 32-bit store per lane.
+//
+// Algorithmic HBM bytes per element of n: P*b (partials) + 8 (f, s; each
+// element is corrected by exactly one rank) read, P*17/32 written; sender
+// feedback adds 4P read and 4P written.
+#pragma once
+
+#include "echo_bulk.cuh"
+#include "echo_kernels.h"
+
+#include <cuda_runtime.h>
+
+// Included by k1_compensate_quantize_pack.cu (the default build) and by the
+// k1_variants_*.cu files (the general build, split by element type and
+// feedback setting so that they compile in parallel). Everything here has
+// internal linkage in each of them.
+namespace echo {
+namespace {
+
+constexpr int kConsumerWarps = 8;
+constexpr int kConsumers = kConsumerWarps * 32;
+constexpr int kThreads = kConsumers + 32; // + one producer warp
+
+// Bytes one stage holds per element of the tile.
+constexpr int k1_bytes_per_elem(int P, bool bf16, bool comp, bool ef)
+{
+    return P * (bf16 ? 2 : 4) + (comp ? 8 : 0) + (ef ? 4 * P : 0);
+}
+
+// The largest tile (ECHO_K1_TILE, /2, /4, ... down to 256 elements) whose
+// stages fit ECHO_K1_CTA_BUDGET.
+constexpr int k1_tile(int P, bool bf16, bool comp, bool ef)
+{
+    int t = ECHO_K1_TILE;
+    while (t > 256 && ECHO_K1_STAGES * t * k1_bytes_per_elem(P, bf16, comp, ef) > ECHO_K1_CTA_BUDGET)
+        t /= 2;
+    return t;
+}
+
+template <int P, bool BF16, bool COMP, bool EF>
+struct K1Shape {
+    static constexpr int kEB = BF16 ? 2 : 4;
+    static constexpr int kTile = k1_tile(P, BF16, COMP, EF);
+    static constexpr int kStages = ECHO_K1_STAGES;
+    static constexpr int kXBytes = kTile * kEB;             // one rank's partial tile
+    static constexpr int kStateOff = P * kXBytes;           // f tile, then s tile
+    static constexpr int kEpsOff = kStateOff + (COMP ? 2 * kTile * 4 : 0); // P error tiles
+    static constexpr int kStageBytes = kEpsOff + (EF ? P * kTile * 4 : 0);
+    static constexpr int kSmem = kStages * kStageBytes + 2 * kStages * 8;
+    static_assert(kSmem <= ECHO_SMEM_BUDGET, "kernel 1 stages exceed shared memory");
+};
+
+template <bool BF16>
+__device__ __forceinline__ void load_chunk(const uint8_t *p, float (&v)[kChunk])
+{
+    if (BF16) {
+        bf16x8_to_f32(*reinterpret_cast<const uint4 *>(p), v);
+    } else {
+        const float4 a = reinterpret_cast<const float4 *>(p)[0];
+        const float4 b = reinterpret_cast<const float4 *>(p)[1];
+        v[0] = a.x, v[1] = a.y, v[2] = a.z, v[3] = a.w;
+        v[4] = b.x, v[5] = b.y, v[6] = b.z, v[7] = b.w;
+    }
+}
+
+__device__ __forceinline__ void load_f32x8(const float *p, float (&v)[kChunk])
+{
+    const float4 a = reinterpret_cast<const float4 *>(p)[0];
+    const float4 b = reinterpret_cast<const float4 *>(p)[1];
+    v[0] = a.x, v[1] = a.y, v[2] = a.z, v[3] = a.w;
+    v[4] = b.x, v[5] = b.y, v[6] = b.z, v[7] = b.w;
+}
+
+// The consumer warps' part of kernel 1 for a group of 8 << LANES elements and
+// one scale format (F16: binary16 scales), both fixed at compile time.
+template <int P, bool BF16, bool COMP, bool EF, uint32_t LANES, bool F16>
+__device__ __forceinline__ void k1_consume(const K1Args &a, const uint8_t *smem, uint64_t *full, uint64_t *empty,
+                                           uint32_t mine, uint32_t cpt_log2, size_t e0)
+{
+    using Sh = K1Shape<P, BF16, COMP, EF>;
+    constexpr int S = Sh::kStages;
+    constexpr uint32_t lanes_log2 = LANES;
+    constexpr bool f16 = F16;
+    const uint32_t tid = threadIdx.x;
+    const uint32_t lane = tid & 31u;
+    const uint32_t code_words = static_cast<uint32_t>(a.n / kChunk); // 32-bit code words per rank
+    for (uint32_t i = 0; i < mine; i++) {
+        const uint32_t s = i % S;
+        if (!warp_wait(&full[s], (i / S) & 1u, a.ctl.wait_cycles, a.ctl.status, kStatusTimeoutK1))
+            return;
+        const uint32_t tile_chunk0 = static_cast<uint32_t>(e0 / kChunk) + ((blockIdx.x + i * gridDim.x) << cpt_log2);
+        const uint32_t cnt_chunks = min(1u << cpt_log2, a.chunk_end - tile_chunk0);
+        const uint8_t *stage = smem + s * Sh::kStageBytes;
+        const float *fs = reinterpret_cast<const float *>(stage + Sh::kStateOff);
+        const float *es = reinterpret_cast<const float *>(stage + Sh::kEpsOff);
+
+#pragma unroll 2
+        for (uint32_t it = tid; it < (static_cast<uint32_t>(P) << cpt_log2); it += kConsumers) {
+            const uint32_t r = it >> cpt_log2; // warp-uniform (a tile has >= 32 chunks)
+            const uint32_t c = it & ((1u << cpt_log2) - 1u);
+            const bool active = c < cnt_chunks;
+            const uint32_t chunk = tile_chunk0 + c;
+            const uint32_t g = chunk >> lanes_log2;
+
+            float v[kChunk];
+            load_chunk<BF16>(stage + r * Sh::kXBytes + c * (kChunk * Sh::kEB), v);
+            if (EF) { // add back this rank's own rounding-#1 error
+                float e[kChunk];
+                load_f32x8(es + r * Sh::kTile + c * kChunk, e);
+#pragma unroll
+                for (int k = 0; k < kChunk; k++)
+                    v[k] = __fadd_rn(v[k], e[k]);
+            }
+            // rank r owns groups [r*gps, (r+1)*gps): one unsigned range test
+            if (COMP && g - r * a.groups_per_seg < a.groups_per_seg) {
+                float fv[kChunk], sv[kChunk];
+                load_f32x8(fs + c * kChunk, fv);
+                load_f32x8(fs + Sh::kTile + c * kChunk, sv);
+#pragma unroll
+                for (int k = 0; k < kChunk; k++)
+                    v[k] = __fadd_rn(v[k], __fadd_rn(__fmul_rn(a.lambda, fv[k]),
+                                                     __fmul_rn(a.one_minus_lambda, sv[k])));
+            }
+            // max |v| as a tree (fmax is exact, so the order is free)
+            const float m01 = fmaxf(fabsf(v[0]), fabsf(v[1])), m23 = fmaxf(fabsf(v[2]), fabsf(v[3]));
+            const float m45 = fmaxf(fabsf(v[4]), fabsf(v[5])), m67 = fmaxf(fabsf(v[6]), fabsf(v[7]));
+            const float amax = group_absmax(fmaxf(fmaxf(m01, m23), fmaxf(m45, m67)), lanes_log2);
+            uint32_t qb[kChunk];
+            uint32_t scale; // scale byte, or binary16 pattern
+            float st;       // the step q is restored with
+            if (f16) {
+                scale = half_scale_bits(amax);
+                st = half_step(scale);
+                const float inv = half_inv(st);
+                const float half = __fmul_rn(0.5f, st);
+#pragma unroll
+                for (int k = 0; k < kChunk; k++)
+                    qb[k] = code_bits_near(v[k], st, inv, half);
+            } else {
+                scale = scale_byte(amax);
+                st = step_of(scale);
+                const float inv = inv_step_of(scale);
+#pragma unroll
+                for (int k = 0; k < kChunk; k++)
+                    qb[k] = code_bits(v[k], inv);
+            }
+            const uint32_t word = pack8_bits(qb);
+            if (active) {
+                reinterpret_cast<uint32_t *>(a.codes)[static_cast<size_t>(r) * code_words + chunk] = word;
+                if ((lane & ((1u << lanes_log2) - 1u)) == 0) { // the group's first lane
+                    uint8_t *row = a.scales + static_cast<size_t>(r) * a.scale_stride;
+                    if (f16)
+                        reinterpret_cast<uint16_t *>(row)[g] = static_cast<uint16_t>(scale);
+                    else
+                        row[g] = static_cast<uint8_t>(scale);
+                }
+                if (EF) { // the new error v - q*step (exact unless a binary16 scale saturated)
+                    float e[kChunk];
+#pragma unroll
+                    for (int k = 0; k < kChunk; k++)
+                        e[k] = __fmaf_rn(-code_value(qb[k]), st, v[k]);
+                    float4 *eo = reinterpret_cast<float4 *>(a.eps + static_cast<size_t>(r) * a.n) +
+                                 2 * static_cast<size_t>(chunk);
+                    eo[0] = make_float4(e[0], e[1], e[2], e[3]);
+                    eo[1] = make_float4(e[4], e[5], e[6], e[7]);
+                }
+            }
+        }
+        __syncwarp();
+        if (lane == 0)
+            mbar_arrive(&empty[s]); // this warp is done reading stage s
+    }
+}
+
+template <int P, bool BF16, bool COMP, bool EF, bool GEN>
+__global__ void __launch_bounds__(kThreads)
+    k1_compensate_quantize_pack(const K1Args a)
+{
+    using Sh = K1Shape<P, BF16, COMP, EF>;
+    constexpr int S = Sh::kStages;
+    extern __shared__ __align__(128) uint8_t smem[];
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + S * Sh::kStageBytes);
+    uint64_t *empty = full + S;
+
+    const uint32_t tid = threadIdx.x;
+    const uint32_t warp = tid >> 5;
+    const uint32_t lane = tid & 31u;
+    const size_t e0 = static_cast<size_t>(a.chunk_begin) * kChunk;
+    const size_t e1 = static_cast<size_t>(a.chunk_end) * kChunk;
+    // the tile length of this launch: a power of two <= Sh::kTile (smem strides keep Sh::kTile)
+    const uint32_t tile = a.tile;
+    const uint32_t cpt_log2 = a.tile_log2 - 3; // chunks per tile = 2^cpt_log2
+    const uint32_t ntiles = static_cast<uint32_t>((e1 - e0 + tile - 1) >> a.tile_log2);
+    const uint32_t mine = blockIdx.x < ntiles ? (ntiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+
+    if (tid == 0) {
+        for (int s = 0; s < S; s++) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kConsumerWarps);
+        }
+        mbar_init_fence();
+    }
+    __syncthreads();
+    wait_for_predecessor(); // nothing above touches global memory
+    allow_successor();
+
+    if (warp == kConsumerWarps) { // producer
+        if (lane == 0)
+            produce_tiles<S>(full, empty, mine, a.ctl.stall, a.ctl.wait_cycles, a.ctl.status, kStatusTimeoutK1,
+                             [&](uint32_t i) {
+                                 const size_t el0 = e0 + static_cast<size_t>(blockIdx.x + i * gridDim.x) * tile;
+                                 const uint32_t cnt = static_cast<uint32_t>(e1 - el0 < size_t(tile) ? e1 - el0 : tile);
+                                 uint8_t *stage = smem + (i % S) * Sh::kStageBytes;
+                                 uint64_t *bar = &full[i % S];
+                                 mbar_arrive_expect_tx(bar, cnt * Sh::kStageBytes / Sh::kTile);
+#pragma unroll
+                                 for (int r = 0; r < P; r++)
+                                     bulk_load(stage + r * Sh::kXBytes,
+                                               static_cast<const uint8_t *>(a.x.p[r]) + el0 * Sh::kEB,
+                                               cnt * Sh::kEB, bar);
+                                 if (COMP) {
+                                     bulk_load(stage + Sh::kStateOff, a.f + el0, cnt * 4, bar);
+                                     bulk_load(stage + Sh::kStateOff + Sh::kTile * 4, a.s + el0, cnt * 4, bar);
+                                 }
+                                 if (EF) {
+#pragma unroll
+                                     for (int r = 0; r < P; r++)
+                                         bulk_load(stage + Sh::kEpsOff + r * Sh::kTile * 4,
+                                                   a.eps + static_cast<size_t>(r) * a.n + el0, cnt * 4, bar);
+                                 }
+                             });
+        return;
+    }
+
+    if (!GEN) {
+        k1_consume<P, BF16, COMP, EF, 2u, false>(a, smem, full, empty, mine, cpt_log2, e0);
+        return;
+    }
+    // variants: one switch per launch selects the compile-time group size
+    // and scale format (group = 8 << lanes_log2)
+    switch (a.lanes_log2 | (a.fp16_scale ? 8u : 0u)) {
+    case 1u: k1_consume<P, BF16, COMP, EF, 1u, false>(a, smem, full, empty, mine, cpt_log2, e0); break;
+    case 3u: k1_consume<P, BF16, COMP, EF, 3u, false>(a, smem, full, empty, mine, cpt_log2, e0); break;
+    case 4u: k1_consume<P, BF16, COMP, EF, 4u, false>(a, smem, full, empty, mine, cpt_log2, e0); break;
+    case 9u: k1_consume<P, BF16, COMP, EF, 1u, true>(a, smem, full, empty, mine, cpt_log2, e0); break;
+    case 10u: k1_consume<P, BF16, COMP, EF, 2u, true>(a, smem, full, empty, mine, cpt_log2, e0); break;
+    case 11u: k1_consume<P, BF16, COMP, EF, 3u, true>(a, smem, full, empty, mine, cpt_log2, e0); break;
+    case 12u: k1_consume<P, BF16, COMP, EF, 4u, true>(a, smem, full, empty, mine, cpt_log2, e0); break;
+    default: break; // the host accepts no other group size
+    }
+}
+
+template <int P, bool BF16, bool COMP, bool EF, bool GEN>
+cudaError_t launch_p(const K1Args &a, cudaStream_t st)
+{
+    using Sh = K1Shape<P, BF16, COMP, EF>;
+    static int resident = 0;
+    auto kern = k1_compensate_quantize_pack<P, BF16, COMP, EF, GEN>;
+    if (resident == 0) {
+        cudaError_t e = prepare_kernel(reinterpret_cast<const void *>(kern), kThreads, Sh::kSmem, &resident);
+        if (e != cudaSuccess)
+            return e;
+    }
+    const size_t elems = static_cast<size_t>(a.chunk_end - a.chunk_begin) * kChunk;
+    K1Args b = a;
+    b.tile_log2 = pick_tile_log2(elems, Sh::kTile, 256, resident);
+    b.tile = 1u << b.tile_log2;
+    const uint32_t tiles = static_cast<uint32_t>((elems + b.tile - 1) >> b.tile_log2);
+    return launch_chained(kern, persistent_grid(tiles, resident), kThreads, Sh::kSmem, st, b);
+}
+
+template <int P, bool BF16, bool EF, bool GEN>
+cudaError_t dispatch_state(const K1Args &a, cudaStream_t st)
+{
+    return a.enable ? launch_p<P, BF16, true, EF, GEN>(a, st) : launch_p<P, BF16, false, EF, GEN>(a, st);
+}
+
+// One element type, feedback setting and build of the kernel, over P.
+template <bool BF16, bool EF, bool GEN>
+cudaError_t dispatch_ranks(const K1Args &a, cudaStream_t st)
+{
+    switch (a.P) {
+    case 2: return dispatch_state<2, BF16, EF, GEN>(a, st);
+    case 3: return dispatch_state<3, BF16, EF, GEN>(a, st);
+    case 4: return dispatch_state<4, BF16, EF, GEN>(a, st);
+    case 5: return dispatch_state<5, BF16, EF, GEN>(a, st);
+    case 6: return dispatch_state<6, BF16, EF, GEN>(a, st);
+    case 7: return dispatch_state<7, BF16, EF, GEN>(a, st);
+    case 8: return dispatch_state<8, BF16, EF, GEN>(a, st);
+    case 9: return dispatch_state<9, BF16, EF, GEN>(a, st);
+    case 10: return dispatch_state<10, BF16, EF, GEN>(a, st);
+    case 11: return dispatch_state<11, BF16, EF, GEN>(a, st);
+    case 12: return dispatch_state<12, BF16, EF, GEN>(a, st);
+    case 13: return dispatch_state<13, BF16, EF, GEN>(a, st);
+    case 14: return dispatch_state<14, BF16, EF, GEN>(a, st);
+    case 15: return dispatch_state<15, BF16, EF, GEN>(a, st);
+    case 16: return dispatch_state<16, BF16, EF, GEN>(a, st);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+} // namespace
+} // namespace echo

@@ -9,7 +9,8 @@ import numpy as np
 import pytest
 
 from bit_error_compensated_rank_b200.workloads import bf16_bits, gaussian, outlier_gaussian, rng
-from gpu_harness import FullCompare, assert_same_bits, from_device, to_device
+from bit_error_compensated_rank_b200 import workloads as wl
+from gpu_harness import FullCompare, SampledCompare, assert_same_bits, from_device, to_device
 from oracle.oracle import Params
 
 pytestmark = pytest.mark.gpu
@@ -273,3 +274,25 @@ def test_host_end_to_end(oracle):
             assert_same_bits(gs, s, "slow estimate")
     finally:
         h.close()
+
+
+def test_largest_tensor_sampled(oracle):
+    """More than 2^31 elements per rank (P = 2, n = 3 * 2^30 + 64, ragged
+    against every tile length): byte offsets past 2^32 in the partials, the
+    state and the wire, 32-bit chunk indices near their top. About 70 GB of
+    device memory; sampled blocks at both ends, the segment boundary and
+    random places, compared exactly after each of two calls."""
+    import torch
+    torch.cuda.empty_cache()
+    P, n = 2, 3 * (1 << 30) + 64
+    sc = SampledCompare(oracle, P, n, "bf16", block_groups=32)
+    try:
+        bufs = [torch.empty(n, device="cuda", dtype=torch.bfloat16) for _ in range(P)]
+        for k in range(2):
+            for r in range(P):
+                wl.torch_outlier_gaussian_(bufs[r], seed=21, call=k, rank=r)
+            sc.call(bufs, phase=k)
+    finally:
+        sc.close()
+        del bufs
+        torch.cuda.empty_cache()
