@@ -12,6 +12,7 @@
 #include "echo_kernels.h"
 
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <cstdarg>
 #include <cstdio>
@@ -250,6 +251,13 @@ int fold_timings(echo_handle *h, uint64_t upto)
     return ECHO_OK;
 }
 
+struct NvtxRange {
+    explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange &) = delete;
+    NvtxRange &operator=(const NvtxRange &) = delete;
+};
+
 // Enqueue K1, K2, K3 over chunks [cb, ce) (multiples of 4) of the tensor.
 // With record_events the call takes the next timing slot.
 int enqueue_call(echo_handle *h, const void *const send[], void *const recv[], int phase, cudaStream_t st,
@@ -334,20 +342,32 @@ int enqueue_call(echo_handle *h, const void *const send[], void *const recv[], i
     a1.ctl = a2.ctl = a3.ctl = ctl;
     a1.scale_stride = a2.scale_stride = h->scale_stride;
 
+    // NVTX ranges (no-ops unless a profiler is attached) mark the call and
+    // each kernel's enqueue, so a timeline tool can attribute the launches.
+    NvtxRange call_range("echo_allreduce");
     cudaError_t e = cudaSuccess;
     const char *what = "cudaEventRecord";
     if (ev)
         e = cudaEventRecord(ev[0], st);
-    if (e == cudaSuccess && (e = echo::launch_k1_compensate_quantize_pack(a1, st)) != cudaSuccess)
-        what = "launch k1_compensate_quantize_pack";
+    if (e == cudaSuccess) {
+        NvtxRange r("k1_compensate_quantize_pack");
+        if ((e = echo::launch_k1_compensate_quantize_pack(a1, st)) != cudaSuccess)
+            what = "launch k1_compensate_quantize_pack";
+    }
     if (e == cudaSuccess && ev)
         e = cudaEventRecord(ev[1], st);
-    if (e == cudaSuccess && (e = echo::launch_k2_owner_reduce_requant(a2, st)) != cudaSuccess)
-        what = "launch k2_owner_reduce_requant";
+    if (e == cudaSuccess) {
+        NvtxRange r("k2_owner_reduce_requant");
+        if ((e = echo::launch_k2_owner_reduce_requant(a2, st)) != cudaSuccess)
+            what = "launch k2_owner_reduce_requant";
+    }
     if (e == cudaSuccess && ev)
         e = cudaEventRecord(ev[2], st);
-    if (e == cudaSuccess && (e = echo::launch_k3_gather_dequant(a3, st)) != cudaSuccess)
-        what = "launch k3_gather_dequant";
+    if (e == cudaSuccess) {
+        NvtxRange r("k3_gather_dequant");
+        if ((e = echo::launch_k3_gather_dequant(a3, st)) != cudaSuccess)
+            what = "launch k3_gather_dequant";
+    }
     if (e == cudaSuccess && ev)
         e = cudaEventRecord(ev[3], st);
     if (e != cudaSuccess) {
