@@ -1,6 +1,11 @@
 """Build ``libecho.so`` in-tree with nvcc for sm_100a.
 
-    python -m bit_error_compensated_rank_b200.build [--verbose]
+    python -m bit_error_compensated_rank_b200.build [--verbose] [--debug | --all]
+
+``--debug`` builds ``libecho_debug.so`` instead: the same sources with
+``ECHO_DEBUG=1`` (device-side bounds checks on every computed index and copy
+range, guard bytes around every library buffer, both reported through the
+device status word). ``--all`` builds both.
 
 Each ``csrc/*.cu`` compiles to an object under ``_build/`` (in parallel), then
 nvcc links them into ``bit_error_compensated_rank_b200/lib/libecho.so`` with the
@@ -25,6 +30,8 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB_DIR = os.path.join(PKG, "lib")
 LIB = os.path.join(LIB_DIR, "libecho.so")
 OBJ_DIR = os.path.join(ROOT, "_build", "echo")
+LIB_DEBUG = os.path.join(LIB_DIR, "libecho_debug.so")
+OBJ_DIR_DEBUG = os.path.join(ROOT, "_build", "echo_debug")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ARCH + [
@@ -58,8 +65,8 @@ def _stale(target: str, deps: list[str]) -> bool:
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def _compile(src: str, obj: str, verbose: bool) -> str:
-    cmd = [nvcc()] + NVCC_FLAGS + ["-c", src, "-o", obj]
+def _compile(src: str, obj: str, verbose: bool, debug: bool = False) -> str:
+    cmd = [nvcc()] + NVCC_FLAGS + (["-DECHO_DEBUG=1"] if debug else []) + ["-c", src, "-o", obj]
     if verbose:
         cmd += ["-Xptxas", "-v"]
     res = subprocess.run(cmd, capture_output=True, text=True)
@@ -68,37 +75,50 @@ def _compile(src: str, obj: str, verbose: bool) -> str:
     return res.stdout + res.stderr
 
 
-def build(verbose: bool = False, force: bool = False) -> str:
-    """Compile what changed and link ``libecho.so``; return its path."""
-    os.makedirs(OBJ_DIR, exist_ok=True)
+def build(verbose: bool = False, force: bool = False, debug: bool = False) -> str:
+    """Compile what changed and link ``libecho.so`` (``libecho_debug.so``
+    with debug); return its path."""
+    obj_dir = OBJ_DIR_DEBUG if debug else OBJ_DIR
+    lib = LIB_DEBUG if debug else LIB
+    os.makedirs(obj_dir, exist_ok=True)
     os.makedirs(LIB_DIR, exist_ok=True)
     hdrs = headers()
     jobs = []
     objs = []
     for src in sources():
-        obj = os.path.join(OBJ_DIR, os.path.basename(src)[:-3] + ".o")
+        obj = os.path.join(obj_dir, os.path.basename(src)[:-3] + ".o")
         objs.append(obj)
         if force or verbose or _stale(obj, [src] + hdrs):
             jobs.append((src, obj))
     logs = []
     if jobs:
         with cf.ThreadPoolExecutor(max_workers=min(len(jobs), os.cpu_count() or 4)) as ex:
-            futs = [ex.submit(_compile, s, o, verbose) for s, o in jobs]
+            futs = [ex.submit(_compile, s, o, verbose, debug) for s, o in jobs]
             for f in futs:
                 logs.append(f.result())
-    if jobs or _stale(LIB, objs):
-        cmd = [nvcc()] + ARCH + ["-shared", "-cudart", "static", "-o", LIB] + objs + ["-ldl"]
+    if jobs or _stale(lib, objs):
+        cmd = [nvcc()] + ARCH + ["-shared", "-cudart", "static", "-o", lib] + objs + ["-ldl"]
         res = subprocess.run(cmd, capture_output=True, text=True)
         if res.returncode != 0:
             raise RuntimeError(f"link failed:\n{res.stdout}\n{res.stderr}")
     if verbose:
         sys.stdout.write("".join(logs))
-    return LIB
+    return lib
+
+
+def build_all(verbose: bool = False, force: bool = False) -> list[str]:
+    """The release library and the debug library."""
+    return [build(verbose, force, debug=False), build(verbose, force, debug=True)]
 
 
 if __name__ == "__main__":
     ap = argparse.ArgumentParser(description=__doc__)
     ap.add_argument("--verbose", action="store_true", help="print ptxas resource usage")
     ap.add_argument("--force", action="store_true")
+    ap.add_argument("--debug", action="store_true", help="build libecho_debug.so instead")
+    ap.add_argument("--all", action="store_true", help="build both libraries")
     args = ap.parse_args()
-    print(build(verbose=args.verbose, force=args.force))
+    if args.all:
+        print("\n".join(build_all(verbose=args.verbose, force=args.force)))
+    else:
+        print(build(verbose=args.verbose, force=args.force, debug=args.debug))

@@ -148,9 +148,47 @@ struct echo_handle {
     // pointers that already passed the device-memory check
     const void *checked[2 * ECHO_MAX_RANKS] = {};
     bool checked_valid = false;
+    // debug build: the guard regions around every buffer above
+    echo::GuardList guards = {};
 };
 
 namespace {
+
+#ifndef ECHO_DEBUG
+#define ECHO_DEBUG 0
+#endif
+
+// Device allocation of every library buffer. The debug build puts
+// kGuardBytes of kGuardByte on both sides of each buffer and records the two
+// regions in the handle; the release build allocates exactly `bytes`.
+cudaError_t dev_alloc(echo_handle *h, void **p, size_t bytes)
+{
+    if (!ECHO_DEBUG)
+        return cudaMalloc(p, bytes);
+    if (h->guards.count + 2 > echo::kMaxGuards)
+        return cudaErrorInvalidValue;
+    uint8_t *base = nullptr;
+    cudaError_t e = cudaMalloc(reinterpret_cast<void **>(&base), bytes + 2 * echo::kGuardBytes);
+    if (e != cudaSuccess)
+        return e;
+    e = cudaMemset(base, echo::kGuardByte, echo::kGuardBytes);
+    if (e == cudaSuccess)
+        e = cudaMemset(base + echo::kGuardBytes + bytes, echo::kGuardByte, echo::kGuardBytes);
+    if (e != cudaSuccess) {
+        cudaFree(base);
+        return e;
+    }
+    h->guards.region[h->guards.count++] = base;
+    h->guards.region[h->guards.count++] = base + echo::kGuardBytes + bytes;
+    *p = base + echo::kGuardBytes;
+    return cudaSuccess;
+}
+
+void dev_free(void *p)
+{
+    if (p)
+        cudaFree(ECHO_DEBUG ? static_cast<uint8_t *>(p) - echo::kGuardBytes : p);
+}
 
 int check_handle(const echo_handle *h)
 {
@@ -340,7 +378,7 @@ int enqueue_call(echo_handle *h, const void *const send[], void *const recv[], i
     const bool stall = fault_injected("stall");
     const echo::PipeCtl ctl{h->dstatus, stall ? kStallWaitCycles : kWaitCycles, stall};
     a1.ctl = a2.ctl = a3.ctl = ctl;
-    a1.scale_stride = a2.scale_stride = h->scale_stride;
+    a1.scale_stride = a2.scale_stride = a3.scale_stride = h->scale_stride;
 
     // NVTX ranges (no-ops unless a profiler is attached) mark the call and
     // each kernel's enqueue, so a timeline tool can attribute the launches.
@@ -370,6 +408,8 @@ int enqueue_call(echo_handle *h, const void *const send[], void *const recv[], i
     }
     if (e == cudaSuccess && ev)
         e = cudaEventRecord(ev[3], st);
+    if (ECHO_DEBUG && e == cudaSuccess && (e = echo::launch_check_guards(h->guards, h->dstatus, st)) != cudaSuccess)
+        what = "launch check_guards";
     if (e != cudaSuccess) {
         if (ev) { // the slot was not fully recorded: give it back
             h->ring_calls -= 1;
@@ -407,14 +447,14 @@ int allreduce_impl(echo_handle *h, const void *const send[], void *const recv[],
 
 void free_handle(echo_handle *h)
 {
-    cudaFree(h->codes1);
-    cudaFree(h->scales1);
-    cudaFree(h->qcodes);
-    cudaFree(h->qscales);
-    cudaFree(h->state);
-    cudaFree(h->dstatus);
-    cudaFree(h->eps);
-    cudaFree(h->staging);
+    dev_free(h->codes1);
+    dev_free(h->scales1);
+    dev_free(h->qcodes);
+    dev_free(h->qscales);
+    dev_free(h->state);
+    dev_free(h->dstatus);
+    dev_free(h->eps);
+    dev_free(h->staging);
     for (auto &slot : h->ring)
         for (cudaEvent_t e : slot)
             if (e)
@@ -523,7 +563,7 @@ int echo_set_variant(echo_handle *h, int variant)
         const size_t bytes = 2 * static_cast<size_t>(h->P) * h->n * sizeof(float);
         cudaError_t e = cudaDeviceSynchronize();
         if (e == cudaSuccess)
-            e = cudaMalloc(&h->eps, bytes);
+            e = dev_alloc(h, reinterpret_cast<void **>(&h->eps), bytes);
         if (e != cudaSuccess) {
             h->eps = nullptr;
             cudaGetLastError();
@@ -612,7 +652,7 @@ echo_handle *echo_create(int P, size_t n, int group, int dtype)
         {reinterpret_cast<void **>(&h->dstatus), sizeof(int)},
     };
     for (auto &a : allocs) {
-        e = cudaMalloc(a.p, a.bytes);
+        e = dev_alloc(h, a.p, a.bytes);
         if (e != cudaSuccess) {
             if (e == cudaErrorMemoryAllocation)
                 set_error(ECHO_ERR_OOM, "cudaMalloc of %zu bytes failed: %s", a.bytes, cudaGetErrorString(e));
@@ -679,7 +719,8 @@ int echo_allreduce_host(echo_handle *h, const void *const host_send[], void *hos
     const size_t eb = elem_bytes(h->dtype);
     cudaError_t e;
     if (!h->staging) {
-        if ((e = cudaMalloc(&h->staging, static_cast<size_t>(h->P) * h->n * eb)) != cudaSuccess) {
+        if ((e = dev_alloc(h, reinterpret_cast<void **>(&h->staging), static_cast<size_t>(h->P) * h->n * eb)) !=
+            cudaSuccess) {
             h->staging = nullptr;
             cudaGetLastError();
             return set_error(ECHO_ERR_OOM, "staging allocation failed: %s", cudaGetErrorString(e));
@@ -924,6 +965,24 @@ int echo_device_status(echo_handle *h, int *status, int clear)
     if (e == cudaSuccess && clear)
         e = cudaDeviceSynchronize();
     return e == cudaSuccess ? ECHO_OK : cuda_error(e, "echo_device_status");
+}
+
+int echo_debug_build(void) { return ECHO_DEBUG ? 1 : 0; }
+
+int echo_debug_touch_guard(echo_handle *h)
+{
+    int rc;
+    if ((rc = check_handle(h)) != ECHO_OK || (rc = check_device(h)) != ECHO_OK)
+        return rc;
+    if (!ECHO_DEBUG || h->guards.count < 2)
+        return set_error(ECHO_ERR_UNSUPPORTED, "guard bytes exist only in the debug build");
+    // the first byte after the stage-1 code buffer (the first buffer allocated)
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e == cudaSuccess)
+        e = cudaMemset(const_cast<uint8_t *>(h->guards.region[1]), 0, 1);
+    if (e == cudaSuccess)
+        e = cudaDeviceSynchronize();
+    return e == cudaSuccess ? ECHO_OK : cuda_error(e, "echo_debug_touch_guard");
 }
 
 int echo_kernel_ms_total(echo_handle *h, double ms[3], uint64_t *timed_calls)

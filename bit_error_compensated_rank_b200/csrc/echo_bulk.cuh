@@ -21,6 +21,29 @@ namespace echo {
 constexpr int kStatusTimeoutK1 = 1;
 constexpr int kStatusTimeoutK2 = 2;
 constexpr int kStatusTimeoutK3 = 4;
+constexpr int kStatusBounds = 8;  // debug build: an access would leave its buffer
+constexpr int kStatusCanary = 16; // debug build: a guard byte around a buffer changed
+
+#ifndef ECHO_DEBUG
+#define ECHO_DEBUG 0
+#endif
+
+// In the debug build (ECHO_DEBUG=1), a failed check of an index or a copy
+// range against its buffer records kStatusBounds and returns false, so the
+// caller skips the access; the release build checks nothing and returns true.
+__device__ __forceinline__ bool in_bounds(bool ok, int *status)
+{
+#if ECHO_DEBUG
+    if (!ok) {
+        atomicOr(status, kStatusBounds);
+        return false;
+    }
+#else
+    (void)ok;
+    (void)status;
+#endif
+    return true;
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p)
 {

@@ -104,6 +104,7 @@ struct K3Args {
     const uint8_t *qscales;  // [scale_stride]
     RankOutPtrs out;         // P rank outputs (bf16 or binary32)
     size_t n;
+    size_t scale_stride;
     uint32_t chunk_begin, chunk_end;
     uint32_t tile, tile_log2; // set by the launcher: this launch's tile length
     uint32_t lanes_log2;     // log2(G / 8): lanes per group
@@ -112,6 +113,16 @@ struct K3Args {
     bool fp16_scale;         // binary16 scales: outputs q*s rounded to bf16 when bf16
     PipeCtl ctl;
 };
+
+// Guard bytes around the library's device buffers (debug build only).
+constexpr size_t kGuardBytes = 256;
+constexpr uint8_t kGuardByte = 0xA5;
+constexpr int kMaxGuards = 16;
+struct GuardList {
+    const uint8_t *region[kMaxGuards]; // kGuardBytes each
+    int count;
+};
+cudaError_t launch_check_guards(const GuardList &g, int *status, cudaStream_t st);
 
 // Each returns the launch's cudaError_t (cudaSuccess when enqueued).
 cudaError_t launch_k1_compensate_quantize_pack(const K1Args &a, cudaStream_t st);

@@ -196,6 +196,7 @@ extern "C" int echo_allreduce_static(int P, size_t n, int dtype, void *const ran
     a3.qcodes = qcodes;
     a3.qscales = qscales;
     a3.n = n;
+    a3.scale_stride = scale_stride;
     a3.chunk_begin = 0;
     a3.chunk_end = chunks;
     a3.P = P;

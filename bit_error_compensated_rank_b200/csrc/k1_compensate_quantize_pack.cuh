@@ -172,7 +172,8 @@ __device__ __forceinline__ void k1_consume(const K1Args &a, const uint8_t *smem,
                     qb[k] = code_bits(v[k], inv);
             }
             const uint32_t word = pack8_bits(qb);
-            if (active) {
+            if (active && in_bounds(chunk < code_words && (g + 1) * (f16 ? 2u : 1u) <= a.scale_stride,
+                                    a.ctl.status)) {
                 reinterpret_cast<uint32_t *>(a.codes)[static_cast<size_t>(r) * code_words + chunk] = word;
                 if ((lane & ((1u << lanes_log2) - 1u)) == 0) { // the group's first lane
                     uint8_t *row = a.scales + static_cast<size_t>(r) * a.scale_stride;
@@ -239,7 +240,11 @@ __global__ void __launch_bounds__(kThreads)
                                  const uint32_t cnt = static_cast<uint32_t>(e1 - el0 < size_t(tile) ? e1 - el0 : tile);
                                  uint8_t *stage = smem + (i % S) * Sh::kStageBytes;
                                  uint64_t *bar = &full[i % S];
-                                 mbar_arrive_expect_tx(bar, cnt * Sh::kStageBytes / Sh::kTile);
+                                 // every copy below covers elements [el0, el0 + cnt) of an n-element row
+                                 const bool ok = in_bounds(el0 + cnt <= a.n && cnt <= Sh::kTile, a.ctl.status);
+                                 mbar_arrive_expect_tx(bar, ok ? cnt * Sh::kStageBytes / Sh::kTile : 0u);
+                                 if (!ok)
+                                     return;
 #pragma unroll
                                  for (int r = 0; r < P; r++)
                                      bulk_load(stage + r * Sh::kXBytes,

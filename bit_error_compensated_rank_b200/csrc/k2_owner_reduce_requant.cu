@@ -123,7 +123,14 @@ __global__ void __launch_bounds__(kThreads)
                     const uint32_t sc_bytes = round16((cnt >> (a.lanes_log2 + 3)) << kScaleLog2);
                     uint8_t *stage = smem + (i % S) * Sh::kStageBytes;
                     uint64_t *bar = &full[i % S];
-                    mbar_arrive_expect_tx(bar, P * (cnt / 2 + sc_bytes) + (COMP ? 2 * cnt * 4 : 0));
+                    // code, state and scale copies against their rows
+                    const bool ok = in_bounds(el0 + cnt <= a.n && cnt <= Sh::kTile && sc_bytes <= Sh::kScaleBytes &&
+                                                  ((el0 >> (a.lanes_log2 + 3)) << kScaleLog2) + sc_bytes <=
+                                                      a.scale_stride,
+                                              a.ctl.status);
+                    mbar_arrive_expect_tx(bar, ok ? P * (cnt / 2 + sc_bytes) + (COMP ? 2 * cnt * 4 : 0) : 0u);
+                    if (!ok)
+                        return;
 #pragma unroll
                     for (int r = 0; r < P; r++) {
                         bulk_load(stage + r * Sh::kCodeBytes, a.codes + r * (a.n / 2) + el0 / 2, cnt / 2, bar);
@@ -218,7 +225,8 @@ __global__ void __launch_bounds__(kThreads)
                 }
             }
 
-            if (active) {
+            if (active && in_bounds(chunk < a.n / kChunk && (g + 1) * (F16 ? 2u : 1u) <= a.scale_stride,
+                                    a.ctl.status)) {
                 reinterpret_cast<uint32_t *>(a.qcodes)[chunk] = pack8_bits(qb);
                 if ((lane & ((1u << a.lanes_log2) - 1u)) == 0) { // the group's first lane
                     if (F16)

@@ -104,7 +104,15 @@ __global__ void __launch_bounds__(kThreads)
                                  const uint32_t sc_bytes = round16((cnt >> (a.lanes_log2 + 3)) << kScaleLog2);
                                  uint8_t *stage = smem + (i % S) * Sh::kInBytes;
                                  uint64_t *bar = &in_full[i % S];
-                                 mbar_arrive_expect_tx(bar, cnt / 2 + sc_bytes);
+                                 // the requantised scales have room for 2n/G bytes
+                                 const bool ok = in_bounds(el0 + cnt <= a.n && cnt <= Sh::kTile &&
+                                                               sc_bytes <= Sh::kScaleBytes &&
+                                                               ((el0 >> (a.lanes_log2 + 3)) << kScaleLog2) +
+                                                                       sc_bytes <= a.scale_stride,
+                                                           a.ctl.status);
+                                 mbar_arrive_expect_tx(bar, ok ? cnt / 2 + sc_bytes : 0u);
+                                 if (!ok)
+                                     return;
                                  bulk_load(stage, a.qcodes + el0 / 2, cnt / 2, bar);
                                  bulk_load(stage + Sh::kCodeBytes,
                                            a.qscales + ((el0 >> (a.lanes_log2 + 3)) << kScaleLog2), sc_bytes, bar);
@@ -123,9 +131,11 @@ __global__ void __launch_bounds__(kThreads)
                 const size_t el0 = tile_start(i);
                 const uint32_t bytes = tile_count(el0) * Sh::kEB;
                 const uint8_t *buf = smem + Sh::kOutOff + b * Sh::kOutBytes;
+                if (in_bounds(el0 + tile_count(el0) <= a.n, a.ctl.status)) {
 #pragma unroll
-                for (int r = 0; r < P; r++)
-                    bulk_store(static_cast<uint8_t *>(a.out.p[r]) + el0 * Sh::kEB, buf, bytes);
+                    for (int r = 0; r < P; r++)
+                        bulk_store(static_cast<uint8_t *>(a.out.p[r]) + el0 * Sh::kEB, buf, bytes);
+                }
                 bulk_commit();
                 // at most B-1 younger groups still read: tile i-(B-1) is done
                 bulk_wait_read<B - 1>();

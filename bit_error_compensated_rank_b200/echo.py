@@ -7,6 +7,10 @@ every failing call raises :class:`EchoError` with the library's message.
 
 Device buffers are passed as integer addresses; the helpers that take torch
 tensors read ``data_ptr()`` and the current stream's handle, nothing more.
+
+``ECHO_LIB=debug`` in the environment loads the debug build
+(``libecho_debug.so``: device-side bounds checks and guard bytes, reported in
+the device status word) instead of the release build.
 """
 from __future__ import annotations
 
@@ -15,7 +19,8 @@ import os
 
 import numpy as np
 
-LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib", "libecho.so")
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib",
+                        "libecho_debug.so" if os.environ.get("ECHO_LIB") == "debug" else "libecho.so")
 
 ECHO_BF16 = 0
 ECHO_FP32 = 1
@@ -31,6 +36,11 @@ ECHO_GROUP = 32
 ECHO_VARIANT_OWNER_SUM = 1
 ECHO_VARIANT_SENDER_EF = 2
 ECHO_VARIANT_FP16_SCALE = 4
+ECHO_STATUS_TIMEOUT_K1 = 1
+ECHO_STATUS_TIMEOUT_K2 = 2
+ECHO_STATUS_TIMEOUT_K3 = 4
+ECHO_STATUS_BOUNDS = 8
+ECHO_STATUS_CANARY = 16
 
 EXPORTED = (
     "echo_create", "echo_allreduce", "echo_allreduce_out", "echo_allreduce_host",
@@ -39,7 +49,7 @@ EXPORTED = (
     "echo_get_wire_range", "echo_stats", "echo_model_bytes", "echo_set_timing",
     "echo_last_kernel_ms", "echo_kernel_ms_total", "echo_device_status",
     "echo_allreduce_static", "echo_set_variant", "echo_get_sender_state", "echo_set_sender_state",
-    "echo_model_bytes_ex",
+    "echo_model_bytes_ex", "echo_debug_build", "echo_debug_touch_guard",
 )
 
 _vp = ctypes.c_void_p
@@ -84,6 +94,8 @@ def _load():
         "echo_get_sender_state": (_int, [_vp, _int, _int, _sz, _sz, _f32p]),
         "echo_set_sender_state": (_int, [_vp, _int, _int, _f32p]),
         "echo_model_bytes_ex": (_int, [_int, _sz, _int, _int, _int, _int, _u64p]),
+        "echo_debug_build": (_int, []),
+        "echo_debug_touch_guard": (_int, [_vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -215,6 +227,14 @@ def echo_model_bytes(P: int, n: int, dtype: int = ECHO_BF16, enable: bool = True
     _check(_lib.echo_model_bytes(P, n, dtype, int(bool(enable)), out))
     return {"k1": out[0], "k2": out[1], "k3": out[2], "link": out[3],
             "total": out[0] + out[1] + out[2]}
+
+
+def echo_debug_build() -> bool:
+    return bool(_lib.echo_debug_build())
+
+
+def echo_debug_touch_guard(h: int) -> None:
+    _check(_lib.echo_debug_touch_guard(h))
 
 
 def echo_model_bytes_ex(P: int, n: int, group: int = ECHO_GROUP, dtype: int = ECHO_BF16,
@@ -360,6 +380,9 @@ class Echo:
 
     def device_status(self, clear: bool = False) -> int:
         return echo_device_status(self.h, clear)
+
+    def debug_touch_guard(self) -> None:
+        echo_debug_touch_guard(self.h)
 
     def close(self) -> None:
         if self.h:

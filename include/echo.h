@@ -278,12 +278,33 @@ ECHO_API int echo_model_bytes_ex(int P, size_t n, int group, int dtype, int enab
  */
 /*
  * echo_device_status - the handle's device status word (synchronous): 0, or
- * bits 1/2/4 when a wait inside kernel 1/2/3 ran out of its time bound (about
- * a second). The kernels never spin without bound; a CTA whose tile did not
- * arrive in time records the bit and returns, leaving that call's outputs
- * incomplete. clear != 0 resets the word after reading it.
+ * bits 1/2/4 (ECHO_STATUS_TIMEOUT_K1..K3) when a wait inside kernel 1/2/3 ran
+ * out of its time bound (about a second). The kernels never spin without
+ * bound; a CTA whose tile did not arrive in time records the bit and returns,
+ * leaving that call's outputs incomplete. The debug build adds
+ * ECHO_STATUS_BOUNDS (an index or copy range would have left its buffer; the
+ * access was skipped) and ECHO_STATUS_CANARY (a guard byte around one of the
+ * library's buffers changed). clear != 0 resets the word after reading it.
  */
+#define ECHO_STATUS_TIMEOUT_K1 1
+#define ECHO_STATUS_TIMEOUT_K2 2
+#define ECHO_STATUS_TIMEOUT_K3 4
+#define ECHO_STATUS_BOUNDS 8
+#define ECHO_STATUS_CANARY 16
 ECHO_API int echo_device_status(echo_handle *h, int *status, int clear);
+
+/*
+ * Debug build (libecho_debug.so, compiled with ECHO_DEBUG=1): every kernel
+ * checks each computed index and bulk-copy range against its buffer, and
+ * every device buffer the library allocates carries 256 guard bytes on each
+ * side, checked after each call. echo_debug_build returns 1 in that build and
+ * 0 in the release build. echo_debug_touch_guard overwrites one guard byte
+ * (the first after the stage-1 code buffer) so that a test can see the next
+ * call report ECHO_STATUS_CANARY; it returns ECHO_ERR_UNSUPPORTED in the
+ * release build.
+ */
+ECHO_API int echo_debug_build(void);
+ECHO_API int echo_debug_touch_guard(echo_handle *h);
 
 ECHO_API int echo_set_timing(echo_handle *h, int enable);
 ECHO_API int echo_last_kernel_ms(echo_handle *h, float ms[3]);

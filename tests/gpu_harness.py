@@ -96,6 +96,8 @@ class FullCompare:
         ref = self.oracle.allreduce(x, f, s, self.params, G=self.group, want_diag=want_diag,
                                     variant=self.variant, eps=self.eps[phase])
         got = from_device(recv)
+        # no wait ran out; in the debug build also no bounds or guard failure
+        assert self.h.device_status(clear=True) == 0, "device status"
         if out_of_place:  # the inputs are untouched
             assert_same_bits(from_device(dev), x, "send buffers")
         for r in range(self.P):
@@ -189,6 +191,7 @@ class SampledCompare:
         ref = self.oracle.allreduce(x, f, s, self.params, G=G, owner=self.owner,
                                     variant=self.variant, eps=self.eps[phase])
         got = self.gather(tensors)
+        assert self.h.device_status(clear=True) == 0, "device status"
         for r in range(self.P):
             assert_same_bits(got[r], ref["out"], f"output rank {r}")
         half = G // 2

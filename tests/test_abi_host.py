@@ -32,6 +32,22 @@ def test_header_declares_the_boundary():
         assert required in names
 
 
+def test_debug_library_exports_the_same_symbols(echo):
+    from bit_error_compensated_rank_b200 import build
+    path = build.build(debug=True)
+    out = subprocess.run(["nm", "-D", "--defined-only", path], capture_output=True,
+                         text=True, check=True).stdout
+    assert set(re.findall(r"\bT (echo_\w+)", out)) == set(declared_symbols())
+
+
+def test_build_flavour_is_reported(echo):
+    assert echo.echo_debug_build() is False
+    code = ("from bit_error_compensated_rank_b200 import echo; "
+            "assert echo.LIB_PATH.endswith('libecho_debug.so'); assert echo.echo_debug_build()")
+    env = dict(os.environ, ECHO_LIB="debug")
+    subprocess.run([sys.executable, "-c", code], cwd=ROOT, env=env, check=True)
+
+
 def test_library_exports_every_declared_symbol(echo):
     out = subprocess.run(["nm", "-D", "--defined-only", echo.LIB_PATH], capture_output=True,
                          text=True, check=True).stdout
