@@ -136,6 +136,29 @@ __device__ __forceinline__ uint32_t code_bits_near(float v, float step, float in
     return static_cast<uint32_t>(bits);
 }
 
+// The same result with a shortcut for groups whose scale did not saturate
+// (max|v| <= 7*65504, so |v/step| <= 7): y = v*inv is within 2^-20 of v/step
+// (two binary32 roundings of a value at most 7.5), so when y lies farther
+// than 2^-19 from a midpoint, the nearest integer to y (from the same kRound
+// addition, |y - k| exact) is already the nearest code. Only the rare values
+// next to a midpoint take the exact path.
+__device__ __forceinline__ uint32_t code_bits_near_unsaturated(float v, float step, float inv, float half)
+{
+    constexpr float kSafe = 0.5f - 0.0000019073486328125f; // 1/2 - 2^-19
+    const float y = __fmul_rn(v, inv);
+    const float t = __fadd_rn(y, kRound);
+    if (fabsf(__fsub_rn(y, __fsub_rn(t, kRound))) < kSafe)
+        return __float_as_uint(t);
+    return code_bits_near(v, step, inv, half);
+}
+
+// True when a group with maximum A gets the saturated scale 65504 and codes
+// clamped at +-7.
+__device__ __forceinline__ bool half_scale_saturates(float A)
+{
+    return A > 458528.f; // 7 * 65504
+}
+
 // Reciprocal estimate used by code_bits_near (0 for a zero step).
 __device__ __forceinline__ float half_inv(float step)
 {
