@@ -103,15 +103,10 @@ __device__ __forceinline__ float half_step(uint32_t h)
 __device__ __forceinline__ uint32_t half_scale_bits(float A)
 {
     constexpr float kSeventh = 0.142857142857142857f;
-    if (A == 0.f)
-        return 0u;
-    uint32_t h = __half_as_ushort(__float2half_ru(__fmul_rn(A, kSeventh)));
-    h = min(h, 0x7BFFu);
-    if (__fmul_rn(7.f, half_step(h)) < A)
-        h = min(h + 1u, 0x7BFFu);
-    else if (h > 1u && __fmul_rn(7.f, half_step(h - 1u)) >= A)
-        h = h - 1u;
-    return h;
+    const uint32_t h = min(static_cast<uint32_t>(__half_as_ushort(__float2half_ru(__fmul_rn(A, kSeventh)))), 0x7BFFu);
+    const bool up = __fmul_rn(7.f, half_step(h)) < A && h < 0x7BFFu;
+    const bool down = !up && h > 1u && __fmul_rn(7.f, half_step(h - 1u)) >= A;
+    return A == 0.f ? 0u : h + (up ? 1u : 0u) - (down ? 1u : 0u);
 }
 
 // Bit pattern kRoundBits + q of the code q in [-7, 7] nearest to v/step, a
@@ -136,27 +131,38 @@ __device__ __forceinline__ uint32_t code_bits_near(float v, float step, float in
     return static_cast<uint32_t>(bits);
 }
 
-// The same result with a shortcut for groups whose scale did not saturate
-// (max|v| <= 7*65504, so |v/step| <= 7): y = v*inv is within 2^-20 of v/step
-// (two binary32 roundings of a value at most 7.5), so when y lies farther
-// than 2^-19 from a midpoint, the nearest integer to y (from the same kRound
-// addition, |y - k| exact) is already the nearest code. Only the rare values
-// next to a midpoint take the exact path.
-__device__ __forceinline__ uint32_t code_bits_near_unsaturated(float v, float step, float inv, float half)
-{
-    constexpr float kSafe = 0.5f - 0.0000019073486328125f; // 1/2 - 2^-19
-    const float y = __fmul_rn(v, inv);
-    const float t = __fadd_rn(y, kRound);
-    if (fabsf(__fsub_rn(y, __fsub_rn(t, kRound))) < kSafe)
-        return __float_as_uint(t);
-    return code_bits_near(v, step, inv, half);
-}
-
 // True when a group with maximum A gets the saturated scale 65504 and codes
 // clamped at +-7.
 __device__ __forceinline__ bool half_scale_saturates(float A)
 {
     return A > 458528.f; // 7 * 65504
+}
+
+// The 8 codes of one lane under a binary16 step (the results of
+// code_bits_near), with a shortcut. In a group whose scale did not saturate,
+// |v/step| <= 7 and y = v*inv is within 2^-20 of v/step (two binary32
+// roundings of a value at most 7.5); when every y of the lane lies farther
+// than 2^-19 from a midpoint, the nearest integer to each y (from the kRound
+// addition; |y - k| is exact) is already the nearest code. Otherwise, or when
+// the group saturated, the lane takes the exact path for all 8 values: one
+// branch per lane, taken rarely.
+__device__ __forceinline__ void codes8_half(const float (&v)[kChunk], float step, float inv, float half, bool sat,
+                                            uint32_t (&qb)[kChunk])
+{
+    constexpr float kSafe = 0.5f - 0.0000019073486328125f; // 1/2 - 2^-19
+    float worst = 0.f;
+#pragma unroll
+    for (int k = 0; k < kChunk; k++) {
+        const float y = __fmul_rn(v[k], inv);
+        const float t = __fadd_rn(y, kRound);
+        qb[k] = __float_as_uint(t);
+        worst = fmaxf(worst, fabsf(__fsub_rn(y, __fsub_rn(t, kRound))));
+    }
+    if (sat || !(worst < kSafe)) {
+#pragma unroll
+        for (int k = 0; k < kChunk; k++)
+            qb[k] = code_bits_near(v[k], step, inv, half);
+    }
 }
 
 // Reciprocal estimate used by code_bits_near (0 for a zero step).

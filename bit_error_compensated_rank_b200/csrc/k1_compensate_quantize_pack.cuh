@@ -160,15 +160,7 @@ __device__ __forceinline__ void k1_consume(const K1Args &a, const uint8_t *smem,
                 st = half_step(scale);
                 const float inv = half_inv(st);
                 const float half = __fmul_rn(0.5f, st);
-                if (half_scale_saturates(amax)) {
-#pragma unroll
-                    for (int k = 0; k < kChunk; k++)
-                        qb[k] = code_bits_near(v[k], st, inv, half);
-                } else {
-#pragma unroll
-                    for (int k = 0; k < kChunk; k++)
-                        qb[k] = code_bits_near_unsaturated(v[k], st, inv, half);
-                }
+                codes8_half(v, st, inv, half, half_scale_saturates(amax), qb);
             } else {
                 scale = scale_byte(amax);
                 st = step_of(scale);

@@ -208,11 +208,9 @@ __global__ void __launch_bounds__(kThreads)
                 const float st = half_step(scale);
                 const float inv = half_inv(st);
                 const float half = __fmul_rn(0.5f, st);
-                const bool sat = half_scale_saturates(amax);
+                codes8_half(S_, st, inv, half, half_scale_saturates(amax), qb);
 #pragma unroll
                 for (int k = 0; k < kChunk; k++) {
-                    qb[k] = sat ? code_bits_near(S_[k], st, inv, half)
-                                : code_bits_near_unsaturated(S_[k], st, inv, half);
                     const float y = __fmul_rn(code_value(qb[k]), st); // exact
                     err[k] = __fsub_rn(S_[k], a.bf16 ? round_bf16(y) : y);
                 }
