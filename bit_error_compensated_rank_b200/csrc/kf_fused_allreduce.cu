@@ -36,7 +36,8 @@
 namespace echo {
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 512;
+constexpr int kCtasPerSm = 2; // few CTAs at the barrier, enough threads for one item each up to 2^21 elements
 
 __device__ __forceinline__ uint32_t ld_acquire(const uint32_t *p)
 {
@@ -78,7 +79,6 @@ __device__ bool grid_barrier(uint32_t *bar, long long limit, bool stall, int *st
                     ok = 0;
                     break;
                 }
-                __nanosleep(64);
             }
         }
     }
@@ -166,6 +166,8 @@ __device__ __forceinline__ void store_scale(uint8_t *row, size_t g, bool f16, ui
 
 __global__ void __launch_bounds__(kThreads) kf_fused_allreduce(const FusedArgs a)
 {
+    wait_for_predecessor(); // launched early (programmatic launch): wait for the previous call's writes
+    allow_successor();
     if (__ldcg(a.ctl.status) & kStatusTimeoutFused)
         return; // an earlier launch lost its barrier: do nothing until the host clears the word
     const uint32_t lane = threadIdx.x & 31u;
@@ -328,7 +330,7 @@ int fused_max_grid()
             cudaGetDevice(&dev) != cudaSuccess ||
             cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
             return 0;
-        grid = per_sm * sms;
+        grid = (per_sm < kCtasPerSm ? per_sm : kCtasPerSm) * sms;
     }
     return grid;
 }
@@ -350,12 +352,24 @@ cudaError_t launch_kf_fused_allreduce(const FusedArgs &a, cudaStream_t st)
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    // cooperative (every CTA resident, for the barrier) and, where the driver
+    // takes both, programmatic (launched while the previous call drains)
+    static bool programmatic = true;
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeCooperative;
     attr[0].val.cooperative = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kf_fused_allreduce, a);
+    cfg.numAttrs = programmatic ? 2 : 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kf_fused_allreduce, a);
+    if (e != cudaSuccess && programmatic) {
+        cudaGetLastError();
+        programmatic = false;
+        cfg.numAttrs = 1;
+        e = cudaLaunchKernelEx(&cfg, kf_fused_allreduce, a);
+    }
+    return e;
 }
 
 } // namespace echo
