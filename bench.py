@@ -49,8 +49,6 @@ L2_BYTES = 126 * 10 ** 6
 # where the rounding errors are fed back, and the scale format (see
 # include/echo.h, echo_set_variant)
 VARIANTS = {"default": 0, "owner_sum": 1, "sender_ef": 2, "both": 3, "fp16_scale": 4}
-# how a call runs (see include/echo.h, echo_set_path)
-PATHS = {"auto": 0, "pipelined": 1, "fused": 2}
 # CPU baseline / reference arm samples (elements per rank, same distribution)
 CPU_SAMPLE_N = 1 << 20
 REF_SAMPLE_N = 1 << 18
@@ -341,7 +339,6 @@ def run_echo(args, rank: int, world: int, local: int) -> dict | None:
         wl.torch_outlier_gaussian_(send[r], seed=SEED + 1000 * rank, call=0, rank=r)
     variant = VARIANTS[args.variant]
     h = echo.Echo(P, n, echo.ECHO_BF16, args.group)
-    h.set_path(PATHS[args.path])
     if variant:
         h.set_variant(variant)
     mb = echo.echo_model_bytes_ex(P, n, args.group, echo.ECHO_BF16, True, variant)
@@ -379,14 +376,8 @@ def run_echo(args, rank: int, world: int, local: int) -> dict | None:
     call_frac = call_bytes / (ms_step * 1e-3) / (peak * 1e9)
 
     k_avg = [t / timed_calls for t in kern_ms]
-    one_launch = args.path == "fused" or (args.path == "auto" and P * n <= 1 << 21)
-    if one_launch:  # the whole call is one kernel, timed in the first slot
-        names = ["kf_fused_allreduce"]
-        k_bytes = [mb["total"]]
-        k_avg = k_avg[:1]
-    else:
-        names = ["k1_compensate_quantize_pack", "k2_owner_reduce_requant", "k3_gather_dequant"]
-        k_bytes = [mb["k1"], mb["k2"], mb["k3"]]
+    names = ["k1_compensate_quantize_pack", "k2_owner_reduce_requant", "k3_gather_dequant"]
+    k_bytes = [mb["k1"], mb["k2"], mb["k3"]]
     dom = max(range(len(names)), key=lambda i: k_bytes[i])
     achieved = k_bytes[dom] / (k_avg[dom] * 1e-3) / 1e9
     src = os.path.join(ROOT, "bit_error_compensated_rank_b200", "csrc", names[dom] + ".cu")
@@ -407,7 +398,7 @@ def run_echo(args, rank: int, world: int, local: int) -> dict | None:
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
         "config": {"workload": workload_name(args),
-                   "variant": args.variant, "P": P, "n_per_rank": n, "group": args.group, "path": args.path,
+                   "variant": args.variant, "P": P, "n_per_rank": n, "group": args.group,
                    "parallelism": f"{world} independent replica(s), ranks simulated in HBM",
                    "l2": "inputs larger than L2 (8 GiB of partials per GPU vs 126 MB L2)"},
         "hbm_roofline_frac": round(call_frac, 4),
@@ -423,7 +414,7 @@ def run_echo(args, rank: int, world: int, local: int) -> dict | None:
         "roofline": {"kernel": names[dom], "bound": "hbm", "achieved": round(achieved, 1),
                      "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
                      "traffic": traffic, "peak_kind": peak_kind},
-        "gpu_launches": (1 if one_launch else 3) * args.steps,
+        "gpu_launches": 3 * args.steps,
         "clocks": clk,
     }
     if e2e is not None:
@@ -480,8 +471,6 @@ def run_sweep(args) -> None:
     for k in range(12, 30):
         n = 1 << k
         h = echo.Echo(P, n, echo.ECHO_BF16, args.group)
-        if args.path != "fused" or P * n <= 1 << 30:
-            h.set_path(PATHS[args.path])
         if variant:
             h.set_variant(variant)
         s_views = [t[:n] for t in send]
@@ -529,8 +518,7 @@ def run_sweep(args) -> None:
         ms_graph = start.elapsed_time(end) / (reps * per_graph)
         del graph
         mb = echo.echo_model_bytes_ex(P, n, args.group, echo.ECHO_BF16, True, variant)
-        print(json.dumps({"sweep": True, "variant": args.variant, "group": args.group, "path": args.path,
-                          "n_per_rank": n,
+        print(json.dumps({"sweep": True, "variant": args.variant, "group": args.group, "n_per_rank": n,
                           "msg_bytes": 2 * n, "calls": calls,
                           "us_per_call": round(ms * 1e3, 2),
                           "us_per_call_median16": round(ms_median * 1e3, 2),
@@ -560,8 +548,6 @@ def main(argv=None):
                     help="where rounding errors are fed back (default: the method as read)")
     ap.add_argument("--group", type=int, choices=[16, 32, 64, 128], default=32,
                     help="elements per scale (default 32, the method as read)")
-    ap.add_argument("--path", choices=sorted(PATHS), default="auto",
-                    help="auto (one launch for small calls, three kernels above), pipelined or fused")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -67,11 +67,6 @@ constexpr long long kWaitCycles = 1LL << 31;
 constexpr long long kStallWaitCycles = 1LL << 20;
 constexpr size_t kHostPiece = size_t(1) << 22; // elements per pipelined host transfer
 constexpr int kVariantBits = ECHO_VARIANT_OWNER_SUM | ECHO_VARIANT_SENDER_EF | ECHO_VARIANT_FP16_SCALE;
-// Ranges of at most this many elements over all ranks take the one-launch
-// path by default (ECHO_PATH_AUTO).
-constexpr size_t kFusedAutoElems = size_t(1) << 21;
-// The one-launch path indexes items in 32 bits: at most 2^30 elements over all ranks.
-constexpr size_t kFusedMaxElems = size_t(1) << 30;
 constexpr int kTimingRing = 32;                 // event sets of timed calls in flight
 
 size_t elem_bytes(int dtype) { return dtype == ECHO_BF16 ? 2 : 4; }
@@ -142,7 +137,6 @@ struct echo_handle {
     // timed loop of calls never waits on the device.
     bool timing = false;
     cudaEvent_t ring[kTimingRing][4] = {};
-    bool ring_fused[kTimingRing] = {}; // the slot timed a one-launch call (events 0 and 1 only)
     uint64_t ring_calls = 0; // timed calls since timing was switched on
     uint64_t folded = 0;     // timed calls already added to total_ms
     double total_ms[3] = {};
@@ -156,9 +150,6 @@ struct echo_handle {
     bool checked_valid = false;
     // debug build: the guard regions around every buffer above
     echo::GuardList guards = {};
-    // the one-launch path: its grid barrier [count, generation] and the choice
-    uint32_t *barrier = nullptr;
-    int path = ECHO_PATH_AUTO;
 };
 
 namespace {
@@ -286,9 +277,8 @@ int fold_timings(echo_handle *h, uint64_t upto)
 {
     for (; h->folded < upto; h->folded++) {
         cudaEvent_t *ev = h->ring[h->folded % kTimingRing];
-        const int kernels = h->ring_fused[h->folded % kTimingRing] ? 1 : 3;
-        cudaError_t e = cudaEventSynchronize(ev[kernels]);
-        for (int k = 0; k < kernels && e == cudaSuccess; k++) {
+        cudaError_t e = cudaEventSynchronize(ev[3]);
+        for (int k = 0; k < 3 && e == cudaSuccess; k++) {
             float ms = 0.f;
             e = cudaEventElapsedTime(&ms, ev[k], ev[k + 1]);
             h->total_ms[k] += ms;
@@ -305,79 +295,6 @@ struct NvtxRange {
     NvtxRange(const NvtxRange &) = delete;
     NvtxRange &operator=(const NvtxRange &) = delete;
 };
-
-// Whether a range goes through the one-launch path: always when chosen, never
-// when the pipelined path is chosen or the stall injection is on (it tests the
-// pipeline's waits), and by default for ranges of at most kFusedAutoElems
-// elements over all ranks.
-bool use_fused(const echo_handle *h, uint32_t cb, uint32_t ce, bool stall)
-{
-    if (h->path == ECHO_PATH_PIPELINED || (stall && h->path != ECHO_PATH_FUSED))
-        return false;
-    if (h->path == ECHO_PATH_FUSED)
-        return true;
-    return static_cast<size_t>(ce - cb) * echo::kChunk * static_cast<size_t>(h->P) <= kFusedAutoElems;
-}
-
-// The one-launch path over the same arguments as the three kernels. A timed
-// call records its events around the one kernel: kernel 1's slot gets the
-// whole duration, kernels 2 and 3 get zero.
-int enqueue_fused(echo_handle *h, const echo::K1Args &a1, const echo::K2Args &a2, const echo::K3Args &a3,
-                  cudaStream_t st, cudaEvent_t *ev)
-{
-    echo::FusedArgs fa{};
-    fa.x = a1.x;
-    fa.out = a3.out;
-    fa.f = const_cast<float *>(a1.f);
-    fa.s = const_cast<float *>(a1.s);
-    fa.eps = a1.eps;
-    fa.codes1 = h->codes1;
-    fa.scales1 = h->scales1;
-    fa.qcodes = h->qcodes;
-    fa.qscales = h->qscales;
-    fa.n = h->n;
-    fa.scale_stride = h->scale_stride;
-    fa.chunk_begin = a1.chunk_begin;
-    fa.chunk_end = a1.chunk_end;
-    fa.lanes_log2 = h->lanes_log2;
-    fa.groups_per_seg = a1.groups_per_seg;
-    fa.lambda = a1.lambda;
-    fa.one_minus_lambda = a1.one_minus_lambda;
-    fa.beta_f = a2.beta_f;
-    fa.one_minus_beta_f = a2.one_minus_beta_f;
-    fa.beta_s = a2.beta_s;
-    fa.one_minus_beta_s = a2.one_minus_beta_s;
-    fa.P = h->P;
-    fa.bf16 = h->dtype == ECHO_BF16;
-    fa.enable = h->enable;
-    fa.owner_sum = a2.owner_sum;
-    fa.sender_ef = a1.sender_ef;
-    fa.fp16_scale = a1.fp16_scale;
-    fa.barrier = h->barrier;
-    fa.ctl = a1.ctl;
-
-    NvtxRange call_range("echo_allreduce (one launch)");
-    cudaError_t e = cudaSuccess;
-    const char *what = "cudaEventRecord";
-    if (ev)
-        e = cudaEventRecord(ev[0], st);
-    if (e == cudaSuccess && (e = echo::launch_kf_fused_allreduce(fa, st)) != cudaSuccess)
-        what = "launch kf_fused_allreduce";
-    if (e == cudaSuccess && ev) {
-        e = cudaEventRecord(ev[1], st);
-        h->ring_fused[h->last_slot] = true;
-    }
-    if (ECHO_DEBUG && e == cudaSuccess && (e = echo::launch_check_guards(h->guards, h->dstatus, st)) != cudaSuccess)
-        what = "launch check_guards";
-    if (e != cudaSuccess) {
-        if (ev) {
-            h->ring_calls -= 1;
-            h->last_slot = -1;
-        }
-        return cuda_error(e, what);
-    }
-    return ECHO_OK;
-}
 
 // Enqueue K1, K2, K3 over chunks [cb, ce) (multiples of 4) of the tensor.
 // With record_events the call takes the next timing slot.
@@ -463,11 +380,6 @@ int enqueue_call(echo_handle *h, const void *const send[], void *const recv[], i
     a1.ctl = a2.ctl = a3.ctl = ctl;
     a1.scale_stride = a2.scale_stride = a3.scale_stride = h->scale_stride;
 
-    if (use_fused(h, cb, ce, stall))
-        return enqueue_fused(h, a1, a2, a3, st, ev);
-
-    if (ev)
-        h->ring_fused[h->last_slot] = false;
     // NVTX ranges (no-ops unless a profiler is attached) mark the call and
     // each kernel's enqueue, so a timeline tool can attribute the launches.
     NvtxRange call_range("echo_allreduce");
@@ -543,7 +455,6 @@ void free_handle(echo_handle *h)
     dev_free(h->dstatus);
     dev_free(h->eps);
     dev_free(h->staging);
-    dev_free(h->barrier);
     for (auto &slot : h->ring)
         for (cudaEvent_t e : slot)
             if (e)
@@ -739,7 +650,6 @@ echo_handle *echo_create(int P, size_t n, int group, int dtype)
         {reinterpret_cast<void **>(&h->qscales), h->scale_stride},
         {reinterpret_cast<void **>(&h->state), 4 * n * sizeof(float)},
         {reinterpret_cast<void **>(&h->dstatus), sizeof(int)},
-        {reinterpret_cast<void **>(&h->barrier), 2 * sizeof(uint32_t)},
     };
     for (auto &a : allocs) {
         e = dev_alloc(h, a.p, a.bytes);
@@ -756,8 +666,6 @@ echo_handle *echo_create(int P, size_t n, int group, int dtype)
     e = cudaMemset(h->state, 0, 4 * n * sizeof(float));
     if (e == cudaSuccess)
         e = cudaMemset(h->dstatus, 0, sizeof(int));
-    if (e == cudaSuccess)
-        e = cudaMemset(h->barrier, 0, 2 * sizeof(uint32_t));
     if (e == cudaSuccess)
         e = cudaDeviceSynchronize();
     if (e != cudaSuccess) {
@@ -1036,13 +944,9 @@ int echo_last_kernel_ms(echo_handle *h, float ms[3])
     if (h->last_slot < 0)
         return set_error(ECHO_ERR_INVALID, "the last call was not timed (echo_set_timing)");
     cudaEvent_t *ev = h->ring[h->last_slot];
-    const int kernels = h->ring_fused[h->last_slot] ? 1 : 3;
-    cudaError_t e = cudaEventSynchronize(ev[kernels]);
-    for (int k = 0; k < 3 && e == cudaSuccess; k++) {
-        ms[k] = 0.f;
-        if (k < kernels)
-            e = cudaEventElapsedTime(&ms[k], ev[k], ev[k + 1]);
-    }
+    cudaError_t e = cudaEventSynchronize(ev[3]);
+    for (int k = 0; k < 3 && e == cudaSuccess; k++)
+        e = cudaEventElapsedTime(&ms[k], ev[k], ev[k + 1]);
     return e == cudaSuccess ? ECHO_OK : cuda_error(e, "echo_last_kernel_ms");
 }
 
@@ -1058,25 +962,9 @@ int echo_device_status(echo_handle *h, int *status, int clear)
         e = cudaMemcpy(status, h->dstatus, sizeof(int), cudaMemcpyDeviceToHost);
     if (e == cudaSuccess && clear)
         e = cudaMemset(h->dstatus, 0, sizeof(int));
-    if (e == cudaSuccess && clear) // a lost grid barrier leaves its words anywhere
-        e = cudaMemset(h->barrier, 0, 2 * sizeof(uint32_t));
     if (e == cudaSuccess && clear)
         e = cudaDeviceSynchronize();
     return e == cudaSuccess ? ECHO_OK : cuda_error(e, "echo_device_status");
-}
-
-int echo_set_path(echo_handle *h, int path)
-{
-    int rc = check_handle(h);
-    if (rc != ECHO_OK)
-        return rc;
-    if (path != ECHO_PATH_AUTO && path != ECHO_PATH_PIPELINED && path != ECHO_PATH_FUSED)
-        return set_error(ECHO_ERR_INVALID, "unknown path %d", path);
-    if (path == ECHO_PATH_FUSED && static_cast<size_t>(h->P) * h->n > kFusedMaxElems)
-        return set_error(ECHO_ERR_UNSUPPORTED, "the one-launch path takes at most %zu elements over all ranks",
-                         kFusedMaxElems);
-    h->path = path;
-    return ECHO_OK;
 }
 
 int echo_debug_build(void) { return ECHO_DEBUG ? 1 : 0; }

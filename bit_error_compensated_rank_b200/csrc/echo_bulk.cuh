@@ -23,7 +23,6 @@ constexpr int kStatusTimeoutK2 = 2;
 constexpr int kStatusTimeoutK3 = 4;
 constexpr int kStatusBounds = 8;  // debug build: an access would leave its buffer
 constexpr int kStatusCanary = 16; // debug build: a guard byte around a buffer changed
-constexpr int kStatusTimeoutFused = 32; // the one-launch path lost its grid barrier
 
 #ifndef ECHO_DEBUG
 #define ECHO_DEBUG 0

@@ -114,35 +114,6 @@ struct K3Args {
     PipeCtl ctl;
 };
 
-// The one-launch path for small messages (kf_fused_allreduce.cu): the three
-// steps of kernels 1-3 over chunks [chunk_begin, chunk_end), separated by a
-// grid-wide barrier.
-struct FusedArgs {
-    RankPtrs x;              // P rank partials
-    RankOutPtrs out;         // P rank outputs (may equal the partials)
-    float *f, *s;            // phase state
-    float *eps;              // sender errors [P][n] (sender feedback only)
-    uint8_t *codes1, *scales1, *qcodes, *qscales; // the wire, as for kernels 1-3
-    size_t n;
-    size_t scale_stride;
-    uint32_t chunk_begin, chunk_end;
-    uint32_t lanes_log2;     // log2(G / 8)
-    uint32_t groups_per_seg; // n / P / G
-    float lambda, one_minus_lambda;
-    float beta_f, one_minus_beta_f, beta_s, one_minus_beta_s;
-    int P;
-    bool bf16;
-    bool enable;             // compensation on
-    bool owner_sum;          // the correction enters the owner's sum
-    bool sender_ef;          // sender feedback
-    bool fp16_scale;         // binary16 scales
-    uint32_t *barrier;       // [count, generation], zero at rest
-    PipeCtl ctl;
-};
-cudaError_t launch_kf_fused_allreduce(const FusedArgs &a, cudaStream_t st);
-// The largest cooperative grid of the fused kernel on this device (0 on error).
-int fused_max_grid();
-
 // Guard bytes around the library's device buffers (debug build only).
 constexpr size_t kGuardBytes = 256;
 constexpr uint8_t kGuardByte = 0xA5;

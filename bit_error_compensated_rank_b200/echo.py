@@ -41,10 +41,6 @@ ECHO_STATUS_TIMEOUT_K2 = 2
 ECHO_STATUS_TIMEOUT_K3 = 4
 ECHO_STATUS_BOUNDS = 8
 ECHO_STATUS_CANARY = 16
-ECHO_STATUS_TIMEOUT_FUSED = 32
-ECHO_PATH_AUTO = 0
-ECHO_PATH_PIPELINED = 1
-ECHO_PATH_FUSED = 2
 
 EXPORTED = (
     "echo_create", "echo_allreduce", "echo_allreduce_out", "echo_allreduce_host",
@@ -53,7 +49,7 @@ EXPORTED = (
     "echo_get_wire_range", "echo_stats", "echo_model_bytes", "echo_set_timing",
     "echo_last_kernel_ms", "echo_kernel_ms_total", "echo_device_status",
     "echo_allreduce_static", "echo_set_variant", "echo_get_sender_state", "echo_set_sender_state",
-    "echo_model_bytes_ex", "echo_debug_build", "echo_debug_touch_guard", "echo_set_path",
+    "echo_model_bytes_ex", "echo_debug_build", "echo_debug_touch_guard",
 )
 
 _vp = ctypes.c_void_p
@@ -100,7 +96,6 @@ def _load():
         "echo_model_bytes_ex": (_int, [_int, _sz, _int, _int, _int, _int, _u64p]),
         "echo_debug_build": (_int, []),
         "echo_debug_touch_guard": (_int, [_vp]),
-        "echo_set_path": (_int, [_vp, _int]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -232,10 +227,6 @@ def echo_model_bytes(P: int, n: int, dtype: int = ECHO_BF16, enable: bool = True
     _check(_lib.echo_model_bytes(P, n, dtype, int(bool(enable)), out))
     return {"k1": out[0], "k2": out[1], "k3": out[2], "link": out[3],
             "total": out[0] + out[1] + out[2]}
-
-
-def echo_set_path(h: int, path: int) -> None:
-    _check(_lib.echo_set_path(h, path))
 
 
 def echo_debug_build() -> bool:
@@ -392,9 +383,6 @@ class Echo:
 
     def debug_touch_guard(self) -> None:
         echo_debug_touch_guard(self.h)
-
-    def set_path(self, path: int) -> None:
-        echo_set_path(self.h, path)
 
     def close(self) -> None:
         if self.h:

@@ -276,15 +276,16 @@ ECHO_API int echo_model_bytes_ex(int P, size_t n, int group, int dtype, int enab
  * the measurement started, and how many calls that was (waiting for the last).
  * echo_set_timing(h, 0) stops recording; the totals stay readable.
  */
+ECHO_API int echo_set_timing(echo_handle *h, int enable);
+ECHO_API int echo_last_kernel_ms(echo_handle *h, float ms[3]);
+ECHO_API int echo_kernel_ms_total(echo_handle *h, double ms[3], uint64_t *timed_calls);
+
 /*
  * echo_device_status - the handle's device status word (synchronous): 0, or
  * bits 1/2/4 (ECHO_STATUS_TIMEOUT_K1..K3) when a wait inside kernel 1/2/3 ran
  * out of its time bound (about a second). The kernels never spin without
  * bound; a CTA whose tile did not arrive in time records the bit and returns,
- * leaving that call's outputs incomplete. ECHO_STATUS_TIMEOUT_FUSED (32): a
- * CTA of the one-launch path waited too long at its grid barrier; while the
- * bit is set, later one-launch calls do nothing. Clearing the word also
- * resets that barrier. The debug build adds
+ * leaving that call's outputs incomplete. The debug build adds
  * ECHO_STATUS_BOUNDS (an index or copy range would have left its buffer; the
  * access was skipped) and ECHO_STATUS_CANARY (a guard byte around one of the
  * library's buffers changed). clear != 0 resets the word after reading it.
@@ -294,7 +295,6 @@ ECHO_API int echo_model_bytes_ex(int P, size_t n, int group, int dtype, int enab
 #define ECHO_STATUS_TIMEOUT_K3 4
 #define ECHO_STATUS_BOUNDS 8
 #define ECHO_STATUS_CANARY 16
-#define ECHO_STATUS_TIMEOUT_FUSED 32
 ECHO_API int echo_device_status(echo_handle *h, int *status, int clear);
 
 /*
@@ -308,31 +308,7 @@ ECHO_API int echo_device_status(echo_handle *h, int *status, int clear);
  * release build.
  */
 ECHO_API int echo_debug_build(void);
-
-/*
- * echo_set_path - how later calls run.
- *   ECHO_PATH_AUTO (default): the one-launch path for calls of at most 2^21
- *       elements over all ranks (P*n), the three pipelined kernels above that.
- *   ECHO_PATH_PIPELINED: always the three kernels (compensate + quantise +
- *       pack, owner reduce + requantise, gather + dequantise).
- *   ECHO_PATH_FUSED: always one cooperative launch that runs the same three
- *       steps with a grid-wide barrier between them (bounded waits); the wire
- *       still goes through device memory. At most 2^30 elements over all
- *       ranks (else ECHO_ERR_UNSUPPORTED).
- * Both paths compute the same bits. Under the one-launch path the kernel
- * timing (echo_last_kernel_ms) puts the whole call in kernel 1's slot and 0
- * in the others. Small messages are bound by launch latency, which the
- * one-launch path cuts to one launch.
- */
-#define ECHO_PATH_AUTO 0
-#define ECHO_PATH_PIPELINED 1
-#define ECHO_PATH_FUSED 2
-ECHO_API int echo_set_path(echo_handle *h, int path);
 ECHO_API int echo_debug_touch_guard(echo_handle *h);
-
-ECHO_API int echo_set_timing(echo_handle *h, int enable);
-ECHO_API int echo_last_kernel_ms(echo_handle *h, float ms[3]);
-ECHO_API int echo_kernel_ms_total(echo_handle *h, double ms[3], uint64_t *timed_calls);
 
 #ifdef __cplusplus
 }

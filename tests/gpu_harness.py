@@ -15,10 +15,6 @@ import numpy as np
 from oracle.oracle import SENDER_EF, Params
 
 G = 32
-# which path a comparison runs: the three pipelined kernels (the default here,
-# so each test keeps covering them at every size), the one-launch kernel, or
-# the library's own choice
-PATHS = {"auto": 0, "pipelined": 1, "fused": 2}
 
 
 def torch():
@@ -68,7 +64,7 @@ class FullCompare:
     compare in full after every call."""
 
     def __init__(self, oracle, P, n, dtype: str, params: Params = Params(), variant: int = 0,
-                 group: int = G, path: str = "pipelined"):
+                 group: int = G):
         from bit_error_compensated_rank_b200 import echo
         self.echo = echo
         self.oracle = oracle
@@ -78,7 +74,6 @@ class FullCompare:
         self.variant = variant
         self.group = group
         self.h = echo.Echo(P, n, echo.ECHO_BF16 if dtype == "bf16" else echo.ECHO_FP32, group)
-        self.h.set_path(PATHS[path])
         self.h.set_params(*params_tuple(params))
         if variant:
             self.h.set_variant(variant)
@@ -139,8 +134,7 @@ class SampledCompare:
     """
 
     def __init__(self, oracle, P, n, dtype: str, params: Params = Params(), blocks=None,
-                 block_groups: int = 64, seed: int = 0, variant: int = 0, group: int = G,
-                 path: str = "pipelined"):
+                 block_groups: int = 64, seed: int = 0, variant: int = 0, group: int = G):
         from bit_error_compensated_rank_b200 import echo
         self.echo = echo
         self.oracle = oracle
@@ -169,7 +163,6 @@ class SampledCompare:
         self.elems = (self.groups[:, None] * group + np.arange(group)[None, :]).reshape(-1)
         self.owner = (self.groups // seg_groups).astype(np.int32)
         self.h = echo.Echo(P, n, echo.ECHO_BF16 if dtype == "bf16" else echo.ECHO_FP32, group)
-        self.h.set_path(PATHS[path])
         self.h.set_params(*params_tuple(params))
         self.variant = variant
         if variant:
