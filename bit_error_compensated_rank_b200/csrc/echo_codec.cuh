@@ -140,23 +140,23 @@ __device__ __forceinline__ bool half_scale_saturates(float A)
 
 // The 8 codes of one lane under a binary16 step (the results of
 // code_bits_near), with a shortcut. In a group whose scale did not saturate,
-// |v/step| <= 7 and y = v*inv is within 2^-20 of v/step (two binary32
-// roundings of a value at most 7.5); when every y of the lane lies farther
-// than 2^-19 from a midpoint, the nearest integer to each y (from the kRound
-// addition; |y - k| is exact) is already the nearest code. Otherwise, or when
-// the group saturated, the lane takes the exact path for all 8 values: one
-// branch per lane, taken rarely.
+// |v/step| <= 7, and the exact product v*inv lies within 2^-19 of v/step
+// (inv has a relative error of at most about 2^-23; see half_inv). The
+// kRound addition fused with the product, t = RN(v*inv + kRound), gives the
+// nearest integer k to v*inv, and d = RN(v*inv - k) its distance. When every
+// |d| of the lane is below 1/2 - 2^-18, each k is the nearest code to v/step.
+// Otherwise, or when the group saturated, the lane takes the exact path for
+// all 8 values: one branch per lane, taken rarely.
 __device__ __forceinline__ void codes8_half(const float (&v)[kChunk], float step, float inv, float half, bool sat,
                                             uint32_t (&qb)[kChunk])
 {
-    constexpr float kSafe = 0.5f - 0.0000019073486328125f; // 1/2 - 2^-19
+    constexpr float kSafe = 0.5f - 0.000003814697265625f; // 1/2 - 2^-18
     float worst = 0.f;
 #pragma unroll
     for (int k = 0; k < kChunk; k++) {
-        const float y = __fmul_rn(v[k], inv);
-        const float t = __fadd_rn(y, kRound);
+        const float t = __fmaf_rn(v[k], inv, kRound);
         qb[k] = __float_as_uint(t);
-        worst = fmaxf(worst, fabsf(__fsub_rn(y, __fsub_rn(t, kRound))));
+        worst = fmaxf(worst, fabsf(__fmaf_rn(v[k], inv, -__fsub_rn(t, kRound))));
     }
     if (sat || !(worst < kSafe)) {
 #pragma unroll
@@ -165,10 +165,15 @@ __device__ __forceinline__ void codes8_half(const float (&v)[kChunk], float step
     }
 }
 
-// Reciprocal estimate used by code_bits_near (0 for a zero step).
+// Reciprocal estimate used by code_bits_near and codes8_half (0 for a zero
+// step): the hardware approximation (rcp.approx, at most 1 ulp off, so a
+// relative error of at most 2^-23; steps are normal binary32 values). Both
+// users settle every code exactly, so the estimate only has to be close.
 __device__ __forceinline__ float half_inv(float step)
 {
-    return step > 0.f ? __frcp_rn(step) : 0.f;
+    float r;
+    asm("rcp.approx.f32 %0, %1;" : "=f"(r) : "f"(step));
+    return step > 0.f ? r : 0.f;
 }
 
 // Nearest bf16 to a binary32 (ties to even), as the upper half of a binary32:
