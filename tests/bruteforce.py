@@ -94,3 +94,56 @@ def bf16_round_bits(x: float) -> float:
     u = struct.unpack("<I", struct.pack("<f", x))[0]
     u = (u + 0x7FFF + ((u >> 16) & 1)) & 0xFFFF0000
     return struct.unpack("<f", struct.pack("<I", u))[0]
+
+
+# ---- vectorised versions for many random groups -----------------------------
+def bf_quantize_many(v):
+    """Scale bytes and codes of many groups (rows of v, binary32 values) by
+    the same search, vectorised: the exponent is the first e >= -127 with
+    every |v| <= 7*2^e (found from an estimate and settled by exact tests on
+    both sides), and each code is the k in [-7, 7] at the least distance
+    |v - k*2^e|, a tie going to the even k. Everything is exact in binary64."""
+    import numpy as np
+    x = np.asarray(v, dtype=np.float64)
+    A = np.abs(x).max(axis=1)
+    e = np.full(A.shape, -127, dtype=np.int64)
+    nz = A > 0
+    _, ex = np.frexp(A[nz] / 7.0)
+    e[nz] = np.maximum(ex - 1, -127)
+    for _ in range(3):  # settle: smallest e with A <= 7*2^e
+        up = A > 7.0 * np.ldexp(1.0, e)
+        e = np.where(up, e + 1, e)
+        down = (e > -127) & (A <= 7.0 * np.ldexp(1.0, e - 1))
+        e = np.where(down, e - 1, e)
+    step = np.ldexp(1.0, e)[:, None]
+    best_k = np.zeros(x.shape, dtype=np.int64)
+    best_d = np.full(x.shape, np.inf)
+    for k in range(CODE_MIN, CODE_MAX + 1):
+        d = np.abs(x - k * step)
+        better = (d < best_d) | ((d == best_d) & (k % 2 == 0))
+        best_k = np.where(better, k, best_k)
+        best_d = np.where(better, d, best_d)
+    return (e + 127).astype(np.int64), best_k
+
+
+def bf_quantize_f16_many(v):
+    """The binary16-scale quantiser for many groups: the scale is the first
+    binary16 (numpy's table) whose 7-fold covers the group's maximum, found
+    by a search over the sorted table (65504 past it, 0 for a zero group);
+    codes as in bf_quantize_many."""
+    import numpy as np
+    x = np.asarray(v, dtype=np.float64)
+    A = np.abs(x).max(axis=1)
+    bits, table = _half_table()
+    i = np.searchsorted(7.0 * table, A, side="left")  # first index with 7*s >= A
+    i = np.minimum(i, len(table) - 1)
+    h = np.where(A == 0, 0, bits[i].astype(np.int64))
+    s = np.where(A == 0, 0.0, table[i])[:, None]
+    best_k = np.zeros(x.shape, dtype=np.int64)
+    best_d = np.full(x.shape, np.inf)
+    for k in range(CODE_MIN, CODE_MAX + 1):
+        d = np.abs(x - k * s)
+        better = (d < best_d) | ((d == best_d) & (k % 2 == 0))
+        best_k = np.where(better, k, best_k)
+        best_d = np.where(better, d, best_d)
+    return h, np.where((A == 0)[:, None], 0, best_k)  # a zero group has no step: codes 0

@@ -30,7 +30,8 @@ from fractions import Fraction
 import numpy as np
 
 from bit_error_compensated_rank_b200.workloads import bf16_bits, bf16_to_f32, gaussian, rng
-from bruteforce import bf16_round_bits, bf_quantize, bf_quantize_f16, half_fraction, value_of
+from bruteforce import (bf16_round_bits, bf_quantize, bf_quantize_f16, bf_quantize_f16_many,
+                        bf_quantize_many, half_fraction, value_of)
 from oracle.oracle import FP16_SCALE, OWNER_SUM, SENDER_EF, Params
 
 GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
@@ -756,6 +757,51 @@ def pin_f16_feedback(orc):
         assert (np.abs(D) <= 5.0 * emax * (1 + 1e-4) + 1e-30).all(), k
 
 
+def _many_random_groups(ngroups, G, seed):
+    """Groups of random magnitudes (2^-140 .. 2^100 per group, with
+    subnormals, ties on a power-of-two grid and bf16 values mixed in)."""
+    g = rng(seed, 77, ngroups)
+    x = g.standard_normal((ngroups, G)) * np.exp2(g.integers(-140, 100, (ngroups, 1)).astype(np.float64))
+    tie_rows = g.random(ngroups) < 0.2     # halves on a power-of-two grid
+    e = g.integers(-120, 100, (ngroups, 1)).astype(np.float64)
+    ties = (g.integers(-7, 7, (ngroups, G)) + 0.5) * np.exp2(e)
+    ties[:, 0] = 7 * np.exp2(e[:, 0])
+    x = np.where(tie_rows[:, None], ties, x)
+    x = x.astype(np.float32)
+    bf_rows = g.random(ngroups) < 0.2
+    x[bf_rows] = bf16_to_f32(bf16_bits(x[bf_rows]))
+    return x
+
+
+def _quantise_rows_with_oracle(orc, x, G, variant):
+    """Stage-1 codes and scales of rank 0 for the rows of x (compensation off,
+    so rank 0 rounds exactly its own values), through one oracle call."""
+    ngroups = x.shape[0]
+    P = 2
+    xs = np.stack([x.reshape(-1), np.zeros(ngroups * G, np.float32)])
+    owner = np.zeros(ngroups, np.int32)
+    res = orc.allreduce(xs, params=Params(enable=False), G=G, owner=owner, variant=variant)
+    codes = np.array(_unpack_ref(res["codes1"][0])).reshape(ngroups, G)
+    return res["scales1"][0].astype(np.int64), codes
+
+
+def pin_quantizer_many_groups(orc):
+    """About a million random groups through the oracle's rounding #1 against
+    the vectorised exhaustive search: every scale byte and every code; and a
+    quarter of that many through the binary16-scale rounding."""
+    x = _many_random_groups(1 << 20, 32, seed=1)
+    b, q = _quantise_rows_with_oracle(orc, x, 32, 0)
+    bb, bq = bf_quantize_many(x)
+    bad = np.flatnonzero((b != bb) | (q != bq).any(axis=1))
+    assert bad.size == 0, (bad[:5], x[bad[:1]], b[bad[:1]], bb[bad[:1]])
+    x = _many_random_groups(1 << 18, 32, seed=2)
+    x = np.clip(x, -1e6, 1e6).astype(np.float32)  # include saturated groups, stay finite
+    h, q = _quantise_rows_with_oracle(orc, x, 32, FP16_SCALE)
+    bh, bq = bf_quantize_f16_many(x)
+    bad = np.flatnonzero((h != bh) | (q != bq).any(axis=1))
+    assert bad.size == 0, (bad[:5], x[bad[:1]], h[bad[:1]], bh[bad[:1]])
+
+
 ALL_PINS = [
     pin_scale_boundaries,
     pin_quantizer_bruteforce,
@@ -782,4 +828,5 @@ ALL_PINS = [
     pin_f16_values,
     pin_f16_exact_sums_on_grid,
     pin_f16_feedback,
+    pin_quantizer_many_groups,
 ]
