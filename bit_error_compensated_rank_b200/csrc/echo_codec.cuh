@@ -26,8 +26,7 @@
 namespace echo {
 
 constexpr int kChunk = 8;           // elements per thread (one 32-bit code word)
-constexpr int kMinGroup = 16;       // elements per scale: 16, 32, 64 or 128
-constexpr int kMaxGroup = 128;      // (a group spans 2, 4, 8 or 16 lanes)
+constexpr int kMinGroup = 16;       // elements per scale: 16, 32, 64 or 128 (2, 4, 8 or 16 lanes)
 constexpr int kMaxRanks = 16;
 
 struct RankPtrs {

@@ -19,7 +19,8 @@
  * cross a link are counted (echo_stats), not sent.
  *
  * Fixed readings of what the pages leave open (every entry point follows
- * them): group of G = 32 consecutive elements; scale 2^e stored as the byte
+ * them; echo_create's group and echo_set_variant select the variants listed
+ * there): group of G = 32 consecutive elements; scale 2^e stored as the byte
  * e+127, e the smallest integer >= -127 with max|v| <= 7*2^e; codes
  * round(v/2^e) with halves to even, in [-7, 7], two per byte (element 2j in
  * the low nibble); rank s owns the contiguous segment [s*n/P, (s+1)*n/P) and
@@ -62,7 +63,7 @@ typedef enum { ECHO_FWD = 0, ECHO_BWD = 1 } echo_phase;
 enum {
     ECHO_OK = 0,
     ECHO_ERR_INVALID = -1,     /* bad argument: nothing enqueued */
-    ECHO_ERR_UNSUPPORTED = -2, /* valid but not built (group != 32, n too large) */
+    ECHO_ERR_UNSUPPORTED = -2, /* valid but not built (group not 16/32/64/128, n too large) */
     ECHO_ERR_CUDA = -3,        /* a CUDA runtime call failed; message has its string */
     ECHO_ERR_OOM = -4          /* device allocation failed */
 };
@@ -98,7 +99,8 @@ ECHO_API echo_handle *echo_create(int P, size_t n, int group, int dtype);
  * Enqueues three kernels (compensate+quantise+pack, owner reduce+requantise,
  * gather+dequantise) and returns. When the stream reaches the end, every
  * rank_ptrs[r] holds the same value Y = Q*2^E, exactly representable in the
- * dtype, and the phase's state holds the updated estimates.
+ * dtype (Q*s under ECHO_VARIANT_FP16_SCALE, rounded to the nearest bf16 for
+ * bf16 buffers), and the phase's state holds the updated estimates.
  */
 ECHO_API int echo_allreduce(echo_handle *h, void *const rank_ptrs[], int phase, void *stream);
 
@@ -242,7 +244,8 @@ ECHO_API int echo_get_wire_range(echo_handle *h, int stage, int rank, size_t gro
 
 /*
  * echo_stats - counters since creation: bytes that would cross links
- * (reduce-scatter + all-gather, 2(P-1) * n * 17/32 per call), modelled HBM
+ * (reduce-scatter + all-gather, 2(P-1) * n * w per call, with w the wire
+ * bytes per element: 17/32 at the default group of 32), modelled HBM
  * bytes (sum of the three kernels' algorithmic bytes), and calls made. Any
  * output pointer may be NULL.
  */
@@ -252,9 +255,9 @@ ECHO_API int echo_stats(echo_handle *h, uint64_t *link_bytes, uint64_t *model_hb
 /*
  * echo_model_bytes - algorithmic bytes of one call, host-only arithmetic:
  *   out[0..2]  HBM bytes read + written by kernels 1, 2, 3
- *              (P*b + 8 + P*w, P*w + 16 + w, P*w + P*b per element, w = 17/32,
- *               b = element bytes; the 8/16 state terms vanish with
- *               compensation off),
+ *              (P*b + 8 + P*w, P*w + 16 + w, P*w + P*b per element, w = 17/32
+ *               at group 32, b = element bytes; the 8/16 state terms vanish
+ *               with compensation off),
  *   out[3]     link bytes of one call, 2(P-1) * n * w.
  * Same argument rules as echo_create.
  */
