@@ -143,3 +143,22 @@ def test_config5_deep_residual(oracle):
     finally:
         on.close()
         off.close()
+
+
+@pytest.mark.parametrize("variant", [0, 3, 4], ids=["default", "owner_sum+sender_ef", "fp16_scale"])
+def test_sixteen_ranks_large(oracle, variant):
+    """The most ranks the library takes (P = 16) at 256 MiB of bf16 per rank,
+    sampled blocks at every segment boundary, two calls."""
+    import torch
+    P, n = 16, 1 << 27
+    sc = SampledCompare(oracle, P, n, "bf16", variant=variant, block_groups=32)
+    try:
+        bufs = _bf16_buffers(P, n)
+        for k in range(2):
+            for r in range(P):
+                wl.torch_outlier_gaussian_(bufs[r], seed=44, call=k, rank=r)
+            sc.call(bufs, phase=k)
+    finally:
+        sc.close()
+        del bufs
+        torch.cuda.empty_cache()
