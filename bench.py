@@ -282,8 +282,9 @@ def run_reference(args, rank: int, world: int) -> dict | None:
         "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": UNIT,
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(t * 1e3, 3), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {"workload": WORKLOAD, "P": P, "n_per_rank": N_ELEMS, "sample_n_per_rank": REF_SAMPLE_N,
+                   "element_dtype": "bf16", "wire": "int4 codes + scales",
                    "parallelism": f"{world} independent replica(s)"},
         "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": 1, "kind": "oracle",
                          "sample": sample, "host": host_info()},
@@ -395,10 +396,13 @@ def run_echo(args, rank: int, world: int, local: int) -> dict | None:
     result = {
         "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        # arithmetic in binary32 (restores, sums, estimates) on bf16 partials and
+        # outputs with 4-bit codes on the wire
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic",
         "config": {"workload": workload_name(args),
                    "variant": args.variant, "P": P, "n_per_rank": n, "group": args.group,
+                   "element_dtype": "bf16", "wire": "int4 codes + scales",
                    "parallelism": f"{world} independent replica(s), ranks simulated in HBM",
                    "l2": "inputs larger than L2 (8 GiB of partials per GPU vs 126 MB L2)"},
         "hbm_roofline_frac": round(call_frac, 4),
