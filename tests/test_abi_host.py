@@ -74,6 +74,16 @@ def test_model_bytes_per_element(echo):
     assert abs(f32["total"] / 65536 - (2 * 8 * 4 + 25 * w + 24)) < 1e-12
 
 
+def test_link_bytes_are_17_64_of_a_16_bit_exchange(echo):
+    """The pages' "almost four times" less volume [rit.work "Echo 4-bit GPU
+    communication", first section]: the counted link bytes of one call are
+    17/64 of those of the same reduce-scatter + all-gather in 16 bits."""
+    from fractions import Fraction
+    for P, n in [(2, 4096), (4, 2048 * 4096), (8, 1 << 29), (16, 16 * 32 * 1000)]:
+        mb = echo.echo_model_bytes(P, n, echo.ECHO_BF16, True)
+        assert Fraction(mb["link"], 2 * (P - 1) * n * 2) == Fraction(17, 64)
+
+
 @pytest.mark.parametrize("fp16", [False, True])
 @pytest.mark.parametrize("group", [16, 32, 64, 128])
 def test_model_bytes_group_sizes(echo, group, fp16):
