@@ -313,14 +313,28 @@ class Echo:
     def _ptrs(self, tensors) -> ctypes.Array:
         """The tensors' device addresses as a C array, kept for reuse: a
         layer that reduces the same buffers every step pays the marshalling
-        once."""
-        key = tuple(t.data_ptr() for t in tensors)
+        once. The C ABI sees plain pointers and cannot know a buffer's size,
+        so a new set of tensors is checked here first: P contiguous CUDA
+        tensors of the handle's dtype with at least n elements each."""
+        key = tuple((t.data_ptr(), t.numel(), t.dtype) for t in tensors)
         arr = self._arrays.get(key)
         if arr is None:
+            self._check_tensors(tensors)
             if len(self._arrays) >= 64:
                 self._arrays.clear()
-            arr = self._arrays[key] = _ptr_array(key)
+            arr = self._arrays[key] = _ptr_array([k[0] for k in key])
         return arr
+
+    def _check_tensors(self, tensors) -> None:
+        if len(tensors) != self.P:
+            raise EchoError(ECHO_ERR_INVALID, f"{len(tensors)} tensors for P = {self.P} ranks")
+        for r, t in enumerate(tensors):
+            if not t.is_cuda or not t.is_contiguous():
+                raise EchoError(ECHO_ERR_INVALID, f"rank {r}: tensor must be a contiguous CUDA tensor")
+            if _dtype_code(t) != self.dtype:
+                raise EchoError(ECHO_ERR_INVALID, f"rank {r}: dtype {t.dtype} does not match the handle")
+            if t.numel() < self.n:
+                raise EchoError(ECHO_ERR_INVALID, f"rank {r}: {t.numel()} elements, the handle needs {self.n}")
 
     def allreduce(self, tensors, phase: int = ECHO_FWD, stream=None) -> None:
         _check(_lib.echo_allreduce(self.h, self._ptrs(tensors), phase, _stream(stream)))
@@ -330,6 +344,12 @@ class Echo:
                                        _stream(stream)))
 
     def allreduce_host(self, host_send, host_recv, phase: int = ECHO_FWD, stream=None) -> None:
+        if len(host_send) != self.P:
+            raise EchoError(ECHO_ERR_INVALID, f"{len(host_send)} tensors for P = {self.P} ranks")
+        for t in list(host_send) + [host_recv]:
+            if t.is_cuda or not t.is_contiguous() or _dtype_code(t) != self.dtype or t.numel() < self.n:
+                raise EchoError(ECHO_ERR_INVALID, "host tensors must be contiguous CPU tensors of the "
+                                                  f"handle's dtype with at least {self.n} elements")
         echo_allreduce_host(self.h, [t.data_ptr() for t in host_send], host_recv.data_ptr(),
                             phase, _stream(stream))
 

@@ -192,6 +192,18 @@ def test_rejects_bad_buffers_without_launching():
             echo.echo_allreduce(h.h, [t.data_ptr() for t in x], 2, 0)
         with pytest.raises(echo.EchoError):
             h.set_params(1.0, 0.5, 0.5, True)
+        # the torch wrapper checks what the C ABI cannot see: count, size, dtype, layout
+        wrapper_cases = {
+            "count": x[:-1],
+            "short": x[:-1] + [torch.zeros(n - 32, device="cuda", dtype=torch.bfloat16)],
+            "dtype": x[:-1] + [torch.zeros(n, device="cuda", dtype=torch.float32)],
+            "strided": x[:-1] + [torch.zeros(2 * n, device="cuda", dtype=torch.bfloat16)[::2]],
+            "cpu": x[:-1] + [torch.zeros(n, dtype=torch.bfloat16)],
+        }
+        for name, tensors in wrapper_cases.items():
+            with pytest.raises(echo.EchoError) as ei:
+                h.allreduce(tensors)
+            assert ei.value.code == echo.ECHO_ERR_INVALID, name
         assert h.stats()["calls"] == 1
         torch.cuda.synchronize()
     finally:
