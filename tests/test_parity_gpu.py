@@ -308,3 +308,44 @@ def test_largest_tensor_sampled(oracle):
         sc.close()
         del bufs
         torch.cuda.empty_cache()
+
+
+def test_cuda_graph_replay(oracle):
+    """Calls captured once in a CUDA graph and replayed: every replay is a
+    correct call (the kernels read their launch shape from the arguments, and
+    the state moves on device), bit for bit the oracle's sequence."""
+    import torch
+    from bit_error_compensated_rank_b200 import echo
+    P, n, per_graph, replays = 8, 8 * 32 * 1024, 3, 3
+    h = echo.Echo(P, n)
+    try:
+        x = gaussian(P, n, seed=95, call=0)
+        send = to_device(x)
+        recv = [torch.empty_like(t) for t in send]
+        stream = torch.cuda.Stream()
+        with torch.cuda.stream(stream):
+            h.allreduce_out(send, recv, 0, stream)  # warm-up outside the capture
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            for _ in range(per_graph):
+                h.allreduce_out(send, recv, 0, stream)
+        torch.cuda.synchronize()
+        h.reset()
+        f = np.zeros(n, np.float32)
+        s = np.zeros(n, np.float32)
+        for _ in range(replays):
+            graph.replay()
+            torch.cuda.synchronize()
+            for _ in range(per_graph):
+                ref = oracle.allreduce(x, f, s, Params())
+            assert h.device_status(clear=True) == 0
+            got = from_device(recv)
+            for r in range(P):
+                assert_same_bits(got[r], ref["out"], f"output rank {r}")
+            gf, gs = h.get_state(0)
+            assert_same_bits(gf, f, "fast estimate")
+            assert_same_bits(gs, s, "slow estimate")
+        del graph
+    finally:
+        h.close()
