@@ -246,8 +246,9 @@ ECHO_API int echo_get_wire_range(echo_handle *h, int stage, int rank, size_t gro
  * echo_stats - counters since creation: bytes that would cross links
  * (reduce-scatter + all-gather, 2(P-1) * n * w per call, with w the wire
  * bytes per element: 17/32 at the default group of 32), modelled HBM
- * bytes (sum of the three kernels' algorithmic bytes), and calls made. Any
- * output pointer may be NULL.
+ * bytes (sum of the three kernels' algorithmic bytes), and calls made through
+ * the API (replays of a captured CUDA graph are not counted). Any output
+ * pointer may be NULL.
  */
 ECHO_API int echo_stats(echo_handle *h, uint64_t *link_bytes, uint64_t *model_hbm_bytes,
                uint64_t *calls);

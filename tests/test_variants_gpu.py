@@ -142,3 +142,34 @@ def test_full_compensation_stops_error_growth(oracle):
             fc.close()
     assert rel["both"][256] < 1.3 * rel["both"][16], rel     # flat with depth
     assert rel["both"][256] < 0.7 * rel["default"][256], rel
+
+
+@pytest.mark.parametrize("variant", VARIANTS, ids=VIDS)
+def test_variant_host_end_to_end(oracle, variant):
+    """Host buffers in, host result out, over several pipelined pieces: the
+    sender errors and the state follow the pieces."""
+    import torch
+    from bit_error_compensated_rank_b200 import echo
+    P, n = 4, 4 * 32 * 80000  # 10.24 M elements per rank: three pieces
+    h = echo.Echo(P, n)
+    h.set_variant(variant)
+    try:
+        f = np.zeros(n, np.float32)
+        s = np.zeros(n, np.float32)
+        eps = np.zeros((P, n), np.float32)
+        for k in range(2):
+            x = gaussian(P, n, seed=17, call=k)
+            host_in = [torch.from_numpy(x[r].view(np.int16)).view(torch.bfloat16).pin_memory()
+                       for r in range(P)]
+            host_out = torch.empty(n, dtype=torch.bfloat16).pin_memory()
+            h.allreduce_host(host_in, host_out)
+            ref = oracle.allreduce(x, f, s, Params(), variant=variant, eps=eps)
+            assert_same_bits(host_out.view(torch.int16).numpy().view(np.uint16), ref["out"], "host result")
+            gf, gs = h.get_state(0)
+            assert_same_bits(gf, f, "fast estimate")
+            assert_same_bits(gs, s, "slow estimate")
+            if variant & SENDER_EF:
+                for r in range(P):
+                    assert_same_bits(h.get_sender_state(0, r), eps[r], f"sender error rank {r}")
+    finally:
+        h.close()
