@@ -1,0 +1,499 @@
+// echo_dist.cu - the all-reduce with one process per rank (echo_dist_* in
+// include/echo.h).
+//
+// Each process holds one rank's partial, its own stage-1 wire row, the
+// requantised segment it owns and the compensator state of that segment. The
+// three kernels run as three stages with the wire exchanged between the
+// processes in between [rit.work "Echo 4-bit GPU communication", section "How
+// Echo returns the error to later calls": segments go to their owner, the
+// owner's compressed total goes back to every rank]:
+//   stage 1  kernel 1 on this rank's partial (one rank, owner mapping of the
+//            whole group): the stage-1 row of all n elements, in this
+//            process's exported buffer;
+//   stage 2  segment `rank` of every rank's stage-1 row is copied into this
+//            process (device-to-device copies from the other processes'
+//            exported buffers, opened with CUDA IPC), then kernel 2 reduces
+//            and requantises the owned segment and updates its state;
+//   stage 3  every owner's requantised segment is copied in, then kernel 3
+//            restores the whole tensor into this rank's output.
+// The copies read other processes' memory into this GPU's memory and the
+// kernels then read local memory only. No kernel waits on another process:
+// the caller orders the stages across processes (synchronise, then a host
+// barrier, between stages and after stage 3). Every operation is the
+// single-process path's, so the results are bit for bit the same.
+#include "echo.h"
+#include "echo_kernels.h"
+
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <new>
+#include <set>
+
+struct echo_dist {
+    int world = 0, rank = 0;
+    size_t n = 0, seg = 0;
+    int group = ECHO_GROUP;
+    uint32_t lanes_log2 = 2;
+    int dtype = ECHO_BF16;
+    int device = 0;
+    int variant = 0;
+    float beta_f = 0.5f, beta_s = 0.875f, lambda = 0.5f;
+    bool enable = true;
+    // exported block: stage-1 row (codes, scales), owned requantised segment (codes, scales)
+    uint8_t *xbuf = nullptr;
+    size_t off_row_scales = 0, off_q_codes = 0, off_q_scales = 0;
+    size_t row_scale_stride = 0, seg_scale_stride = 0; // 2n/G and 2seg/G rounded up to 16
+    // local: the owned segment from every rank, the gathered requantised tensor, state
+    uint8_t *recv_codes = nullptr, *recv_scales = nullptr;
+    uint8_t *q_codes = nullptr, *q_scales = nullptr;
+    float *state = nullptr; // [phase][f|s][n]; only the owned segment moves
+    float *eps = nullptr;   // [phase][n], sender feedback
+    int *dstatus = nullptr;
+    const uint8_t *peer[ECHO_MAX_RANKS] = {}; // every rank's exported block (own included)
+    bool connected = false;
+    uint64_t calls = 0;
+};
+
+namespace {
+
+std::mutex g_mu;
+std::set<const echo_dist *> g_live;
+
+constexpr long long kWaitCycles = 1LL << 31;
+
+int fail(int code, const char *fmt, ...) __attribute__((format(printf, 2, 3)));
+int fail(int code, const char *fmt, ...)
+{
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    return echo::record_error(code, buf);
+}
+
+int cuda_fail(cudaError_t e, const char *what)
+{
+    return fail(ECHO_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorString(e), cudaGetErrorName(e));
+}
+
+size_t round16(size_t x) { return (x + 15) / 16 * 16; }
+size_t round256(size_t x) { return (x + 255) / 256 * 256; }
+
+int check(const echo_dist *d)
+{
+    if (!d)
+        return fail(ECHO_ERR_INVALID, "handle is NULL");
+    {
+        std::lock_guard<std::mutex> lock(g_mu);
+        if (!g_live.count(d))
+            return fail(ECHO_ERR_INVALID, "distributed handle %p is unknown or destroyed",
+                        static_cast<const void *>(d));
+    }
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "cudaGetDevice");
+    if (dev != d->device)
+        return fail(ECHO_ERR_INVALID, "the handle belongs to device %d, the current device is %d", d->device, dev);
+    return ECHO_OK;
+}
+
+int check_user_buffer(const void *p, int device, const char *what)
+{
+    if (!p)
+        return fail(ECHO_ERR_INVALID, "%s is NULL", what);
+    if (reinterpret_cast<uintptr_t>(p) % 16 != 0)
+        return fail(ECHO_ERR_INVALID, "%s is not 16-byte aligned", what);
+    cudaPointerAttributes attr;
+    cudaError_t e = cudaPointerGetAttributes(&attr, p);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return fail(ECHO_ERR_INVALID, "%s is not CUDA memory (%s)", what, cudaGetErrorString(e));
+    }
+    if ((attr.type != cudaMemoryTypeDevice && attr.type != cudaMemoryTypeManaged) || attr.device != device)
+        return fail(ECHO_ERR_INVALID, "%s is not memory of device %d", what, device);
+    return ECHO_OK;
+}
+
+void free_dist(echo_dist *d)
+{
+    for (int p = 0; p < d->world; p++)
+        if (p != d->rank && d->peer[p])
+            cudaIpcCloseMemHandle(const_cast<uint8_t *>(d->peer[p]));
+    for (void *p : {static_cast<void *>(d->xbuf), static_cast<void *>(d->recv_codes),
+                    static_cast<void *>(d->recv_scales), static_cast<void *>(d->q_codes),
+                    static_cast<void *>(d->q_scales), static_cast<void *>(d->state), static_cast<void *>(d->eps),
+                    static_cast<void *>(d->dstatus)})
+        if (p)
+            cudaFree(p);
+    delete d;
+}
+
+echo::PipeCtl ctl_of(const echo_dist *d) { return echo::PipeCtl{d->dstatus, kWaitCycles, false}; }
+
+int stage1(echo_dist *d, const void *x, int phase, cudaStream_t st)
+{
+    echo::K1Args a{};
+    a.x.p[0] = x;
+    a.f = d->state + static_cast<size_t>(phase) * 2 * d->n;
+    a.s = a.f + d->n;
+    a.codes = d->xbuf;
+    a.scales = d->xbuf + d->off_row_scales;
+    a.n = d->n;
+    a.scale_stride = d->row_scale_stride;
+    a.chunk_begin = 0;
+    a.chunk_end = static_cast<uint32_t>(d->n / echo::kChunk);
+    a.lanes_log2 = d->lanes_log2;
+    a.groups_per_seg = static_cast<uint32_t>(d->seg / d->group);
+    a.rank_base = static_cast<uint32_t>(d->rank);
+    a.lambda = d->lambda;
+    a.one_minus_lambda = 1.0f - d->lambda;
+    a.eps = (d->variant & ECHO_VARIANT_SENDER_EF) ? d->eps + static_cast<size_t>(phase) * d->n : nullptr;
+    a.P = 1;
+    a.bf16 = d->dtype == ECHO_BF16;
+    a.enable = d->enable && !(d->variant & ECHO_VARIANT_OWNER_SUM);
+    a.sender_ef = (d->variant & ECHO_VARIANT_SENDER_EF) != 0;
+    a.fp16_scale = (d->variant & ECHO_VARIANT_FP16_SCALE) != 0;
+    a.ctl = ctl_of(d);
+    cudaError_t e = echo::launch_k1_compensate_quantize_pack(a, st);
+    return e == cudaSuccess ? ECHO_OK : cuda_fail(e, "launch k1_compensate_quantize_pack");
+}
+
+int stage2(echo_dist *d, int phase, cudaStream_t st)
+{
+    const size_t sb = (d->variant & ECHO_VARIANT_FP16_SCALE) ? 2 : 1; // bytes per scale
+    const size_t seg_codes = d->seg / 2, seg_scales = d->seg / d->group * sb;
+    for (int p = 0; p < d->world; p++) {
+        const uint8_t *row = d->peer[p];
+        cudaError_t e = cudaMemcpyAsync(d->recv_codes + p * seg_codes, row + d->rank * seg_codes, seg_codes,
+                                        cudaMemcpyDeviceToDevice, st);
+        if (e == cudaSuccess)
+            e = cudaMemcpyAsync(d->recv_scales + p * d->seg_scale_stride,
+                                row + d->off_row_scales + d->rank * seg_scales, seg_scales, cudaMemcpyDeviceToDevice,
+                                st);
+        if (e != cudaSuccess)
+            return cuda_fail(e, "stage 2 copy from a rank's stage-1 row");
+    }
+    float *f = d->state + static_cast<size_t>(phase) * 2 * d->n + d->rank * d->seg;
+    echo::K2Args a{};
+    a.codes = d->recv_codes;
+    a.scales = d->recv_scales;
+    a.qcodes = d->xbuf + d->off_q_codes;
+    a.qscales = d->xbuf + d->off_q_scales;
+    a.f = f;
+    a.s = f + d->n;
+    a.n = d->seg;
+    a.scale_stride = d->seg_scale_stride;
+    a.chunk_begin = 0;
+    a.chunk_end = static_cast<uint32_t>(d->seg / echo::kChunk);
+    a.lanes_log2 = d->lanes_log2;
+    a.beta_f = d->beta_f;
+    a.one_minus_beta_f = 1.0f - d->beta_f;
+    a.beta_s = d->beta_s;
+    a.one_minus_beta_s = 1.0f - d->beta_s;
+    a.lambda = d->lambda;
+    a.one_minus_lambda = 1.0f - d->lambda;
+    a.P = d->world;
+    a.enable = d->enable;
+    a.owner_sum = d->enable && (d->variant & ECHO_VARIANT_OWNER_SUM);
+    a.fp16_scale = (d->variant & ECHO_VARIANT_FP16_SCALE) != 0;
+    a.bf16 = d->dtype == ECHO_BF16;
+    a.ctl = ctl_of(d);
+    cudaError_t e = echo::launch_k2_owner_reduce_requant(a, st);
+    return e == cudaSuccess ? ECHO_OK : cuda_fail(e, "launch k2_owner_reduce_requant");
+}
+
+int stage3(echo_dist *d, void *out, cudaStream_t st)
+{
+    const size_t sb = (d->variant & ECHO_VARIANT_FP16_SCALE) ? 2 : 1;
+    const size_t seg_codes = d->seg / 2, seg_scales = d->seg / d->group * sb;
+    for (int p = 0; p < d->world; p++) {
+        const uint8_t *blk = d->peer[p];
+        cudaError_t e = cudaMemcpyAsync(d->q_codes + p * seg_codes, blk + d->off_q_codes, seg_codes,
+                                        cudaMemcpyDeviceToDevice, st);
+        if (e == cudaSuccess)
+            e = cudaMemcpyAsync(d->q_scales + p * seg_scales, blk + d->off_q_scales, seg_scales,
+                                cudaMemcpyDeviceToDevice, st);
+        if (e != cudaSuccess)
+            return cuda_fail(e, "stage 3 copy from an owner's requantised segment");
+    }
+    echo::K3Args a{};
+    a.qcodes = d->q_codes;
+    a.qscales = d->q_scales;
+    a.out.p[0] = out;
+    a.n = d->n;
+    a.scale_stride = d->row_scale_stride;
+    a.chunk_begin = 0;
+    a.chunk_end = static_cast<uint32_t>(d->n / echo::kChunk);
+    a.lanes_log2 = d->lanes_log2;
+    a.P = 1;
+    a.bf16 = d->dtype == ECHO_BF16;
+    a.fp16_scale = (d->variant & ECHO_VARIANT_FP16_SCALE) != 0;
+    a.ctl = ctl_of(d);
+    cudaError_t e = echo::launch_k3_gather_dequant(a, st);
+    return e == cudaSuccess ? ECHO_OK : cuda_fail(e, "launch k3_gather_dequant");
+}
+
+} // namespace
+
+extern "C" {
+
+echo_dist *echo_dist_create(int world, int rank, size_t n, int group, int dtype)
+{
+    if (world < 2 || world > ECHO_MAX_RANKS) {
+        fail(ECHO_ERR_INVALID, "world = %d is outside [2, %d]", world, ECHO_MAX_RANKS);
+        return nullptr;
+    }
+    if (rank < 0 || rank >= world) {
+        fail(ECHO_ERR_INVALID, "rank %d outside [0, %d)", rank, world);
+        return nullptr;
+    }
+    if (dtype != ECHO_BF16 && dtype != ECHO_FP32) {
+        fail(ECHO_ERR_INVALID, "unknown dtype %d", dtype);
+        return nullptr;
+    }
+    if (group != 16 && group != 32 && group != 64 && group != 128) {
+        fail(ECHO_ERR_UNSUPPORTED, "group = %d: the built group sizes are 16, 32, 64 and 128", group);
+        return nullptr;
+    }
+    // segments of whole groups whose code rows start on 16 bytes
+    const size_t unit = static_cast<size_t>(world) * (group > 32 ? group : 32);
+    if (n == 0 || n % unit != 0) {
+        fail(ECHO_ERR_INVALID, "n = %zu must be a positive multiple of %zu (world x max(group, 32))", n, unit);
+        return nullptr;
+    }
+    if (n > (size_t(1) << 34)) {
+        fail(ECHO_ERR_UNSUPPORTED, "n = %zu exceeds the supported maximum 2^34", n);
+        return nullptr;
+    }
+    echo_dist *d = new (std::nothrow) echo_dist();
+    if (!d) {
+        fail(ECHO_ERR_OOM, "host allocation of the handle failed");
+        return nullptr;
+    }
+    d->world = world;
+    d->rank = rank;
+    d->n = n;
+    d->seg = n / world;
+    d->group = group;
+    d->lanes_log2 = 0; // group = 8 << lanes_log2
+    while ((8u << d->lanes_log2) != static_cast<uint32_t>(group))
+        d->lanes_log2++;
+    d->dtype = dtype;
+    d->row_scale_stride = round16(2 * (n / group));
+    d->seg_scale_stride = round16(2 * (d->seg / group));
+    d->off_row_scales = round256(n / 2);
+    d->off_q_codes = d->off_row_scales + round256(d->row_scale_stride);
+    d->off_q_scales = d->off_q_codes + round256(d->seg / 2);
+    const size_t xbytes = d->off_q_scales + round256(d->seg_scale_stride);
+    cudaError_t e = cudaGetDevice(&d->device);
+    struct {
+        void **p;
+        size_t bytes;
+    } allocs[] = {
+        {reinterpret_cast<void **>(&d->xbuf), xbytes},
+        {reinterpret_cast<void **>(&d->recv_codes), static_cast<size_t>(world) * (d->seg / 2)},
+        {reinterpret_cast<void **>(&d->recv_scales), static_cast<size_t>(world) * d->seg_scale_stride},
+        {reinterpret_cast<void **>(&d->q_codes), n / 2},
+        {reinterpret_cast<void **>(&d->q_scales), d->row_scale_stride},
+        {reinterpret_cast<void **>(&d->state), 4 * n * sizeof(float)},
+        {reinterpret_cast<void **>(&d->dstatus), sizeof(int)},
+    };
+    for (auto &a : allocs) {
+        if (e == cudaSuccess)
+            e = cudaMalloc(a.p, a.bytes);
+    }
+    if (e == cudaSuccess)
+        e = cudaMemset(d->state, 0, 4 * n * sizeof(float));
+    if (e == cudaSuccess)
+        e = cudaMemset(d->dstatus, 0, sizeof(int));
+    if (e == cudaSuccess)
+        e = cudaMemset(d->xbuf, 0, xbytes);
+    if (e == cudaSuccess)
+        e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) {
+        if (e == cudaErrorMemoryAllocation)
+            fail(ECHO_ERR_OOM, "device allocation failed: %s", cudaGetErrorString(e));
+        else
+            cuda_fail(e, "echo_dist_create");
+        cudaGetLastError();
+        free_dist(d);
+        return nullptr;
+    }
+    d->peer[rank] = d->xbuf;
+    std::lock_guard<std::mutex> lock(g_mu);
+    g_live.insert(d);
+    return d;
+}
+
+int echo_dist_export(echo_dist *d, uint8_t handle[ECHO_IPC_HANDLE_BYTES])
+{
+    int rc = check(d);
+    if (rc != ECHO_OK)
+        return rc;
+    if (!handle)
+        return fail(ECHO_ERR_INVALID, "handle buffer is NULL");
+    cudaIpcMemHandle_t h;
+    static_assert(sizeof(h) == ECHO_IPC_HANDLE_BYTES, "CUDA IPC handle size");
+    cudaError_t e = cudaIpcGetMemHandle(&h, d->xbuf);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "cudaIpcGetMemHandle");
+    std::memcpy(handle, &h, sizeof h);
+    return ECHO_OK;
+}
+
+int echo_dist_connect(echo_dist *d, const uint8_t *handles)
+{
+    int rc = check(d);
+    if (rc != ECHO_OK)
+        return rc;
+    if (!handles)
+        return fail(ECHO_ERR_INVALID, "handles is NULL");
+    if (d->connected)
+        return fail(ECHO_ERR_INVALID, "already connected");
+    for (int p = 0; p < d->world; p++) {
+        if (p == d->rank)
+            continue;
+        cudaIpcMemHandle_t h;
+        std::memcpy(&h, handles + static_cast<size_t>(p) * ECHO_IPC_HANDLE_BYTES, sizeof h);
+        void *ptr = nullptr;
+        cudaError_t e = cudaIpcOpenMemHandle(&ptr, h, cudaIpcMemLazyEnablePeerAccess);
+        if (e != cudaSuccess) {
+            cudaGetLastError();
+            for (int q = 0; q < p; q++)
+                if (q != d->rank && d->peer[q]) {
+                    cudaIpcCloseMemHandle(const_cast<uint8_t *>(d->peer[q]));
+                    d->peer[q] = nullptr;
+                }
+            return cuda_fail(e, "cudaIpcOpenMemHandle");
+        }
+        d->peer[p] = static_cast<const uint8_t *>(ptr);
+    }
+    d->connected = true;
+    return ECHO_OK;
+}
+
+int echo_dist_stage(echo_dist *d, int stage, const void *x, void *out, int phase, void *stream)
+{
+    int rc = check(d);
+    if (rc != ECHO_OK)
+        return rc;
+    if (!d->connected)
+        return fail(ECHO_ERR_INVALID, "not connected (echo_dist_connect)");
+    if (phase != ECHO_FWD && phase != ECHO_BWD)
+        return fail(ECHO_ERR_INVALID, "phase %d is neither ECHO_FWD (0) nor ECHO_BWD (1)", phase);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    switch (stage) {
+    case 1:
+        if ((rc = check_user_buffer(x, d->device, "x")) != ECHO_OK)
+            return rc;
+        return stage1(d, x, phase, st);
+    case 2:
+        return stage2(d, phase, st);
+    case 3:
+        if ((rc = check_user_buffer(out, d->device, "out")) != ECHO_OK)
+            return rc;
+        rc = stage3(d, out, st);
+        if (rc == ECHO_OK)
+            d->calls += 1;
+        return rc;
+    default:
+        return fail(ECHO_ERR_INVALID, "stage %d is not 1, 2 or 3", stage);
+    }
+}
+
+int echo_dist_set_params(echo_dist *d, float beta_fast, float beta_slow, float lambda, int enable)
+{
+    int rc = check(d);
+    if (rc != ECHO_OK)
+        return rc;
+    if (!(beta_fast >= 0.f && beta_fast < 1.f) || !(beta_slow >= 0.f && beta_slow < 1.f) ||
+        !(lambda >= 0.f && lambda <= 1.f) || (enable != 0 && enable != 1))
+        return fail(ECHO_ERR_INVALID, "parameters out of range (beta in [0,1), lambda in [0,1], enable 0/1)");
+    d->beta_f = beta_fast;
+    d->beta_s = beta_slow;
+    d->lambda = lambda;
+    d->enable = enable != 0;
+    return ECHO_OK;
+}
+
+int echo_dist_set_variant(echo_dist *d, int variant)
+{
+    int rc = check(d);
+    if (rc != ECHO_OK)
+        return rc;
+    if (variant & ~(ECHO_VARIANT_OWNER_SUM | ECHO_VARIANT_SENDER_EF | ECHO_VARIANT_FP16_SCALE))
+        return fail(ECHO_ERR_INVALID, "unknown variant bits 0x%x", variant);
+    if ((variant & ECHO_VARIANT_SENDER_EF) && !d->eps) {
+        const size_t bytes = 2 * d->n * sizeof(float);
+        cudaError_t e = cudaMalloc(&d->eps, bytes);
+        if (e == cudaSuccess)
+            e = cudaMemset(d->eps, 0, bytes);
+        if (e == cudaSuccess)
+            e = cudaDeviceSynchronize();
+        if (e != cudaSuccess) {
+            cudaGetLastError();
+            if (d->eps)
+                cudaFree(d->eps);
+            d->eps = nullptr;
+            return fail(ECHO_ERR_OOM, "sender-error state of %zu bytes: %s", bytes, cudaGetErrorString(e));
+        }
+    }
+    d->variant = variant;
+    return ECHO_OK;
+}
+
+int echo_dist_get_state(echo_dist *d, int phase, float *f_host, float *s_host)
+{
+    int rc = check(d);
+    if (rc != ECHO_OK)
+        return rc;
+    if (phase != ECHO_FWD && phase != ECHO_BWD)
+        return fail(ECHO_ERR_INVALID, "phase %d is neither ECHO_FWD (0) nor ECHO_BWD (1)", phase);
+    const float *f = d->state + static_cast<size_t>(phase) * 2 * d->n + d->rank * d->seg;
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e == cudaSuccess && f_host)
+        e = cudaMemcpy(f_host, f, d->seg * sizeof(float), cudaMemcpyDeviceToHost);
+    if (e == cudaSuccess && s_host)
+        e = cudaMemcpy(s_host, f + d->n, d->seg * sizeof(float), cudaMemcpyDeviceToHost);
+    return e == cudaSuccess ? ECHO_OK : cuda_fail(e, "echo_dist_get_state");
+}
+
+int echo_dist_device_status(echo_dist *d, int *status, int clear)
+{
+    int rc = check(d);
+    if (rc != ECHO_OK)
+        return rc;
+    if (!status)
+        return fail(ECHO_ERR_INVALID, "status is NULL");
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e == cudaSuccess)
+        e = cudaMemcpy(status, d->dstatus, sizeof(int), cudaMemcpyDeviceToHost);
+    if (e == cudaSuccess && clear)
+        e = cudaMemset(d->dstatus, 0, sizeof(int));
+    if (e == cudaSuccess && clear)
+        e = cudaDeviceSynchronize();
+    return e == cudaSuccess ? ECHO_OK : cuda_fail(e, "echo_dist_device_status");
+}
+
+int echo_dist_destroy(echo_dist *d)
+{
+    if (!d)
+        return ECHO_OK;
+    {
+        std::lock_guard<std::mutex> lock(g_mu);
+        if (!g_live.erase(d))
+            return fail(ECHO_ERR_INVALID, "distributed handle %p is unknown or destroyed",
+                        static_cast<const void *>(d));
+    }
+    cudaDeviceSynchronize();
+    free_dist(d);
+    return ECHO_OK;
+}
+
+} // extern "C"

@@ -67,6 +67,8 @@ struct K1Args {
     uint32_t tile, tile_log2; // set by the launcher: this launch's tile length
     uint32_t lanes_log2;     // log2(G / 8): lanes per group
     uint32_t groups_per_seg; // n / P / G: owner of group g is g / groups_per_seg
+    uint32_t rank_base;      // global rank of partial 0 (a one-rank launch of a process
+                             // that holds one rank of a larger group; 0 otherwise)
     float lambda, one_minus_lambda;
     float *eps;              // sender feedback: every rank's rounding-#1 error [P][n]
     int P;

@@ -10,7 +10,7 @@ cudaError_t launch_k1_compensate_quantize_pack(const K1Args &a, cudaStream_t st)
 {
     if (a.chunk_end <= a.chunk_begin)
         return cudaSuccess;
-    if (a.P < 2 || a.P > kMaxRanks)
+    if (a.P < 1 || a.P > kMaxRanks)
         return cudaErrorInvalidValue;
     if (a.lanes_log2 != 2u || a.fp16_scale) { // a group-size or scale-format variant
         if (a.bf16)

@@ -139,7 +139,7 @@ __device__ __forceinline__ void k1_consume(const K1Args &a, const uint8_t *smem,
                     v[k] = __fadd_rn(v[k], e[k]);
             }
             // rank r owns groups [r*gps, (r+1)*gps): one unsigned range test
-            if (COMP && g - r * a.groups_per_seg < a.groups_per_seg) {
+            if (COMP && g - (r + a.rank_base) * a.groups_per_seg < a.groups_per_seg) {
                 float fv[kChunk], sv[kChunk];
                 load_f32x8(fs + c * kChunk, fv);
                 load_f32x8(fs + Sh::kTile + c * kChunk, sv);
@@ -310,6 +310,7 @@ template <bool BF16, bool EF, bool GEN>
 cudaError_t dispatch_ranks(const K1Args &a, cudaStream_t st)
 {
     switch (a.P) {
+    case 1: return dispatch_state<1, BF16, EF, GEN>(a, st); // one rank per process
     case 2: return dispatch_state<2, BF16, EF, GEN>(a, st);
     case 3: return dispatch_state<3, BF16, EF, GEN>(a, st);
     case 4: return dispatch_state<4, BF16, EF, GEN>(a, st);

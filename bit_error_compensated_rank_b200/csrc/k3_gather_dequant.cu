@@ -226,6 +226,7 @@ cudaError_t launch_k3_gather_dequant(const K3Args &a, cudaStream_t st)
     if (a.chunk_end <= a.chunk_begin)
         return cudaSuccess;
     switch (a.P) {
+    case 1: return dispatch_flags<1>(a, st); // one output per process
     case 2: return dispatch_flags<2>(a, st);
     case 3: return dispatch_flags<3>(a, st);
     case 4: return dispatch_flags<4>(a, st);

@@ -50,7 +50,11 @@ EXPORTED = (
     "echo_last_kernel_ms", "echo_kernel_ms_total", "echo_device_status",
     "echo_allreduce_static", "echo_set_variant", "echo_get_sender_state", "echo_set_sender_state",
     "echo_model_bytes_ex", "echo_debug_build", "echo_debug_touch_guard",
+    "echo_dist_create", "echo_dist_export", "echo_dist_connect", "echo_dist_stage",
+    "echo_dist_set_params", "echo_dist_set_variant", "echo_dist_get_state",
+    "echo_dist_device_status", "echo_dist_destroy",
 )
+ECHO_IPC_HANDLE_BYTES = 64
 
 _vp = ctypes.c_void_p
 _sz = ctypes.c_size_t
@@ -96,6 +100,15 @@ def _load():
         "echo_model_bytes_ex": (_int, [_int, _sz, _int, _int, _int, _int, _u64p]),
         "echo_debug_build": (_int, []),
         "echo_debug_touch_guard": (_int, [_vp]),
+        "echo_dist_create": (_vp, [_int, _int, _sz, _int, _int]),
+        "echo_dist_export": (_int, [_vp, _u8p]),
+        "echo_dist_connect": (_int, [_vp, _u8p]),
+        "echo_dist_stage": (_int, [_vp, _int, _vp, _vp, _int, _vp]),
+        "echo_dist_set_params": (_int, [_vp, ctypes.c_float, ctypes.c_float, ctypes.c_float, _int]),
+        "echo_dist_set_variant": (_int, [_vp, _int]),
+        "echo_dist_get_state": (_int, [_vp, _int, _f32p, _f32p]),
+        "echo_dist_device_status": (_int, [_vp, ctypes.POINTER(ctypes.c_int), _int]),
+        "echo_dist_destroy": (_int, [_vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -414,6 +427,86 @@ class Echo:
 
     def __exit__(self, *exc):
         self.close()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+# ---- one process per rank ---------------------------------------------------
+class DistEcho:
+    """One rank of an all-reduce whose ranks are separate processes (the
+    echo_dist_* entry points): ``DistEcho(world, rank, n, dtype)``, exchange
+    the IPC handles (``export`` on every rank, then ``connect`` with all of
+    them in rank order), then :meth:`allreduce`. ``barrier`` is a callable
+    that returns when every rank has called it (``torch.distributed.barrier``
+    in practice); the stages are ordered across processes with it."""
+
+    def __init__(self, world: int, rank: int, n: int, dtype: int = ECHO_BF16, group: int = ECHO_GROUP):
+        self.world, self.rank, self.n, self.dtype, self.group = world, rank, n, dtype, group
+        self.seg = n // world
+        h = _lib.echo_dist_create(world, rank, n, group, dtype)
+        if not h:
+            raise EchoError(_lib.echo_last_status(), echo_last_error())
+        self.h = h
+
+    def export(self) -> bytes:
+        buf = (ctypes.c_uint8 * ECHO_IPC_HANDLE_BYTES)()
+        _check(_lib.echo_dist_export(self.h, buf))
+        return bytes(buf)
+
+    def connect(self, handles) -> None:
+        if len(handles) != self.world or any(len(b) != ECHO_IPC_HANDLE_BYTES for b in handles):
+            raise EchoError(ECHO_ERR_INVALID, f"need {self.world} handles of {ECHO_IPC_HANDLE_BYTES} bytes")
+        blob = (ctypes.c_uint8 * (self.world * ECHO_IPC_HANDLE_BYTES)).from_buffer_copy(b"".join(handles))
+        _check(_lib.echo_dist_connect(self.h, blob))
+
+    def _check_tensor(self, t, what: str) -> None:
+        if not t.is_cuda or not t.is_contiguous() or _dtype_code(t) != self.dtype or t.numel() < self.n:
+            raise EchoError(ECHO_ERR_INVALID, f"{what}: a contiguous CUDA tensor of the handle's dtype "
+                                              f"with at least {self.n} elements is needed")
+
+    def stage(self, stage: int, x=None, out=None, phase: int = ECHO_FWD, stream=None) -> None:
+        if stage == 1:
+            self._check_tensor(x, "x")
+        if stage == 3:
+            self._check_tensor(out, "out")
+        _check(_lib.echo_dist_stage(self.h, stage, x.data_ptr() if stage == 1 else None,
+                                    out.data_ptr() if stage == 3 else None, phase, _stream(stream)))
+
+    def allreduce(self, x, out, barrier, phase: int = ECHO_FWD, stream=None) -> None:
+        """One call: each stage, then wait for this rank's stream and for
+        every rank (the next stage reads the others' buffers)."""
+        import torch
+        st = stream if stream is not None else torch.cuda.current_stream()
+        for k in (1, 2, 3):
+            self.stage(k, x, out, phase, st)
+            st.synchronize()
+            barrier()
+
+    def set_params(self, beta_fast=0.5, beta_slow=0.875, lam=0.5, enable=True) -> None:
+        _check(_lib.echo_dist_set_params(self.h, beta_fast, beta_slow, lam, int(bool(enable))))
+
+    def set_variant(self, variant: int) -> None:
+        _check(_lib.echo_dist_set_variant(self.h, variant))
+
+    def get_state(self, phase: int = ECHO_FWD):
+        f = np.empty(self.seg, np.float32)
+        s = np.empty(self.seg, np.float32)
+        _check(_lib.echo_dist_get_state(self.h, phase, _np(f, _f32p), _np(s, _f32p)))
+        return f, s
+
+    def device_status(self, clear: bool = False) -> int:
+        st = ctypes.c_int()
+        _check(_lib.echo_dist_device_status(self.h, ctypes.byref(st), int(bool(clear))))
+        return st.value
+
+    def close(self) -> None:
+        if self.h:
+            _check(_lib.echo_dist_destroy(self.h))
+            self.h = None
 
     def __del__(self):
         try:

@@ -314,6 +314,56 @@ ECHO_API int echo_device_status(echo_handle *h, int *status, int clear);
 ECHO_API int echo_debug_build(void);
 ECHO_API int echo_debug_touch_guard(echo_handle *h);
 
+/*
+ * One process per rank (echo_dist_*). The same all-reduce when each of the
+ * world ranks is its own process holding only its own partial; every rank
+ * keeps the compensator state of the segment it owns, [rank*n/world,
+ * (rank+1)*n/world). A call runs in three stages:
+ *   stage 1  this rank's partial x is rounded into its stage-1 wire row
+ *            (kernel 1 for one rank, the owner mapping of the whole group);
+ *   stage 2  segment `rank` of every rank's row is copied into this process,
+ *            then kernel 2 sums, requantises and updates the owned state;
+ *   stage 3  every owner's requantised segment is copied in, then kernel 3
+ *            writes the result (n elements, identical on every rank) to out.
+ * The copies read the other processes' exported buffers (CUDA IPC; on
+ * several GPUs, peer reads over NVLink) into this GPU's memory; the kernels
+ * read local memory only, and no kernel waits on another process. The caller
+ * orders the stages across processes: after each stage, synchronise the
+ * stream, then a host barrier over all ranks (also after stage 3, before the
+ * next call's stage 1). The results are bit for bit those of echo_allreduce
+ * on the same partials.
+ *
+ * echo_dist_create(world, rank, n, group, dtype): world in [2, 16], rank in
+ *   [0, world), n a positive multiple of world x max(group, 32) (segments of
+ *   whole groups whose code rows start on 16 bytes), group and dtype as for
+ *   echo_create. Allocates on the current device, NULL on error.
+ * echo_dist_export: the CUDA IPC handle (ECHO_IPC_HANDLE_BYTES bytes) of this
+ *   rank's exported buffer (its stage-1 row and its requantised segment).
+ * echo_dist_connect: handles = world handles in rank order (this rank's own
+ *   entry is ignored); opens the others' buffers. Once per handle.
+ * echo_dist_stage(d, stage, x, out, phase, stream): x (stage 1) and out
+ *   (stage 3) are device pointers to n elements of dtype, 16-byte aligned
+ *   (unused in the other stages; out may equal x).
+ * echo_dist_set_params / echo_dist_set_variant: as echo_set_params and
+ *   echo_set_variant, for this rank (every rank must use the same settings).
+ * echo_dist_get_state: the owned segment's two estimates (n/world binary32
+ *   each) of a phase, synchronous.
+ * echo_dist_device_status: as echo_device_status.
+ * echo_dist_destroy: closes the peers' buffers and frees this rank's (call
+ *   on every rank after a final barrier).
+ */
+#define ECHO_IPC_HANDLE_BYTES 64
+typedef struct echo_dist echo_dist; /* opaque */
+ECHO_API echo_dist *echo_dist_create(int world, int rank, size_t n, int group, int dtype);
+ECHO_API int echo_dist_export(echo_dist *d, uint8_t handle[ECHO_IPC_HANDLE_BYTES]);
+ECHO_API int echo_dist_connect(echo_dist *d, const uint8_t *handles);
+ECHO_API int echo_dist_stage(echo_dist *d, int stage, const void *x, void *out, int phase, void *stream);
+ECHO_API int echo_dist_set_params(echo_dist *d, float beta_fast, float beta_slow, float lambda, int enable);
+ECHO_API int echo_dist_set_variant(echo_dist *d, int variant);
+ECHO_API int echo_dist_get_state(echo_dist *d, int phase, float *f_host, float *s_host);
+ECHO_API int echo_dist_device_status(echo_dist *d, int *status, int clear);
+ECHO_API int echo_dist_destroy(echo_dist *d);
+
 #ifdef __cplusplus
 }
 #endif

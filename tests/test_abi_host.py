@@ -114,6 +114,16 @@ def test_create_rejects_bad_shapes(echo, P, n, group, dtype, status):
     assert echo.echo_last_error()
 
 
+@pytest.mark.parametrize("world,rank,n,group,dtype,status", [
+    (1, 0, 64, 32, 0, -1), (17, 0, 17 * 32, 32, 0, -1), (2, 2, 64, 32, 0, -1), (2, -1, 64, 32, 0, -1),
+    (2, 0, 96, 32, 0, -1), (2, 0, 2 * 48, 48, 0, -2), (2, 0, 64, 32, 9, -1), (3, 0, 3 * 16, 16, 0, -1),
+])
+def test_dist_create_rejects_bad_shapes(echo, world, rank, n, group, dtype, status):
+    assert not echo._lib.echo_dist_create(world, rank, n, group, dtype)
+    assert echo.echo_last_status() == status
+    assert echo.echo_last_error()
+
+
 def test_null_and_unknown_handles(echo):
     for fn, args in [(echo._lib.echo_allreduce, (None, None, 0, None)),
                      (echo._lib.echo_reset, (None, 1)),
