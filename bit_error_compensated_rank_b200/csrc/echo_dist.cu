@@ -1,26 +1,27 @@
 // echo_dist.cu - the all-reduce with one process per rank (echo_dist_* in
 // include/echo.h).
 //
-// Each process holds one rank's partial, its own stage-1 wire row, the
-// requantised segment it owns and the compensator state of that segment. The
-// three kernels run as three stages with the wire exchanged between the
-// processes in between [rit.work "Echo 4-bit GPU communication", section "How
+// Each process holds one rank's partial, the compensator state of the segment
+// it owns, and an exported block that the other processes write into (opened
+// with CUDA IPC): a receive slot per rank for the owned segment's stage-1
+// wire, and the gathered requantised tensor. The three kernels run as three
+// stages, and the wire moves inside them as plain stores into the other
+// processes' blocks [rit.work "Echo 4-bit GPU communication", section "How
 // Echo returns the error to later calls": segments go to their owner, the
 // owner's compressed total goes back to every rank]:
 //   stage 1  kernel 1 on this rank's partial (one rank, owner mapping of the
-//            whole group): the stage-1 row of all n elements, in this
-//            process's exported buffer;
-//   stage 2  segment `rank` of every rank's stage-1 row is copied into this
-//            process (device-to-device copies from the other processes'
-//            exported buffers, opened with CUDA IPC), then kernel 2 reduces
-//            and requantises the owned segment and updates its state;
-//   stage 3  every owner's requantised segment is copied in, then kernel 3
-//            restores the whole tensor into this rank's output.
-// The copies read other processes' memory into this GPU's memory and the
-// kernels then read local memory only. No kernel waits on another process:
-// the caller orders the stages across processes (synchronise, then a host
-// barrier, between stages and after stage 3). Every operation is the
-// single-process path's, so the results are bit for bit the same.
+//            whole group) stores each segment's codes and scales straight
+//            into its owner's receive slot for this rank;
+//   stage 2  kernel 2 reduces and requantises the owned segment from the
+//            local receive slots, updates its state, and stores the
+//            requantised segment into every rank's gathered tensor;
+//   stage 3  kernel 3 restores the local gathered tensor into this rank's
+//            output.
+// On several GPUs the stores cross NVLink as peer stores; the kernels read
+// local memory only. No kernel waits on another process: the caller orders
+// the stages across processes (synchronise, then a host barrier, after each
+// stage). Every operation is the single-process path's, so the results are
+// bit for bit the same.
 #include "echo.h"
 #include "echo_kernels.h"
 
@@ -43,13 +44,12 @@ struct echo_dist {
     int variant = 0;
     float beta_f = 0.5f, beta_s = 0.875f, lambda = 0.5f;
     bool enable = true;
-    // exported block: stage-1 row (codes, scales), owned requantised segment (codes, scales)
+    // exported block: receive slots [world][seg/2] codes and [world][seg scale
+    // stride] scales for the owned segment, then the gathered requantised
+    // tensor ([n/2] codes, [2n/G rounded up] scales)
     uint8_t *xbuf = nullptr;
-    size_t off_row_scales = 0, off_q_codes = 0, off_q_scales = 0;
+    size_t off_recv_scales = 0, off_q_codes = 0, off_q_scales = 0;
     size_t row_scale_stride = 0, seg_scale_stride = 0; // 2n/G and 2seg/G rounded up to 16
-    // local: the owned segment from every rank, the gathered requantised tensor, state
-    uint8_t *recv_codes = nullptr, *recv_scales = nullptr;
-    uint8_t *q_codes = nullptr, *q_scales = nullptr;
     float *state = nullptr; // [phase][f|s][n]; only the owned segment moves
     float *eps = nullptr;   // [phase][n], sender feedback
     int *dstatus = nullptr;
@@ -125,9 +125,7 @@ void free_dist(echo_dist *d)
     for (int p = 0; p < d->world; p++)
         if (p != d->rank && d->peer[p])
             cudaIpcCloseMemHandle(const_cast<uint8_t *>(d->peer[p]));
-    for (void *p : {static_cast<void *>(d->xbuf), static_cast<void *>(d->recv_codes),
-                    static_cast<void *>(d->recv_scales), static_cast<void *>(d->q_codes),
-                    static_cast<void *>(d->q_scales), static_cast<void *>(d->state), static_cast<void *>(d->eps),
+    for (void *p : {static_cast<void *>(d->xbuf), static_cast<void *>(d->state), static_cast<void *>(d->eps),
                     static_cast<void *>(d->dstatus)})
         if (p)
             cudaFree(p);
@@ -142,8 +140,12 @@ int stage1(echo_dist *d, const void *x, int phase, cudaStream_t st)
     a.x.p[0] = x;
     a.f = d->state + static_cast<size_t>(phase) * 2 * d->n;
     a.s = a.f + d->n;
-    a.codes = d->xbuf;
-    a.scales = d->xbuf + d->off_row_scales;
+    a.to_owners = true;
+    for (int p = 0; p < d->world; p++)
+        a.owners.p[p] = const_cast<uint8_t *>(d->peer[p]);
+    a.seg_code_bytes = d->seg / 2;
+    a.recv_scales_off = d->off_recv_scales;
+    a.seg_scale_stride = d->seg_scale_stride;
     a.n = d->n;
     a.scale_stride = d->row_scale_stride;
     a.chunk_begin = 0;
@@ -166,25 +168,10 @@ int stage1(echo_dist *d, const void *x, int phase, cudaStream_t st)
 
 int stage2(echo_dist *d, int phase, cudaStream_t st)
 {
-    const size_t sb = (d->variant & ECHO_VARIANT_FP16_SCALE) ? 2 : 1; // bytes per scale
-    const size_t seg_codes = d->seg / 2, seg_scales = d->seg / d->group * sb;
-    for (int p = 0; p < d->world; p++) {
-        const uint8_t *row = d->peer[p];
-        cudaError_t e = cudaMemcpyAsync(d->recv_codes + p * seg_codes, row + d->rank * seg_codes, seg_codes,
-                                        cudaMemcpyDeviceToDevice, st);
-        if (e == cudaSuccess)
-            e = cudaMemcpyAsync(d->recv_scales + p * d->seg_scale_stride,
-                                row + d->off_row_scales + d->rank * seg_scales, seg_scales, cudaMemcpyDeviceToDevice,
-                                st);
-        if (e != cudaSuccess)
-            return cuda_fail(e, "stage 2 copy from a rank's stage-1 row");
-    }
     float *f = d->state + static_cast<size_t>(phase) * 2 * d->n + d->rank * d->seg;
     echo::K2Args a{};
-    a.codes = d->recv_codes;
-    a.scales = d->recv_scales;
-    a.qcodes = d->xbuf + d->off_q_codes;
-    a.qscales = d->xbuf + d->off_q_scales;
+    a.codes = d->xbuf; // the receive slots, one per rank
+    a.scales = d->xbuf + d->off_recv_scales;
     a.f = f;
     a.s = f + d->n;
     a.n = d->seg;
@@ -203,6 +190,13 @@ int stage2(echo_dist *d, int phase, cudaStream_t st)
     a.owner_sum = d->enable && (d->variant & ECHO_VARIANT_OWNER_SUM);
     a.fp16_scale = (d->variant & ECHO_VARIANT_FP16_SCALE) != 0;
     a.bf16 = d->dtype == ECHO_BF16;
+    a.to_ranks = true;
+    for (int p = 0; p < d->world; p++)
+        a.ranks.p[p] = const_cast<uint8_t *>(d->peer[p]) + d->off_q_codes;
+    a.q_chunk0 = static_cast<uint32_t>(d->rank * (d->seg / echo::kChunk));
+    a.q_group0 = static_cast<uint32_t>(d->rank * (d->seg / d->group));
+    a.q_scales_off = d->off_q_scales - d->off_q_codes;
+    a.q_scale_bytes = d->row_scale_stride;
     a.ctl = ctl_of(d);
     cudaError_t e = echo::launch_k2_owner_reduce_requant(a, st);
     return e == cudaSuccess ? ECHO_OK : cuda_fail(e, "launch k2_owner_reduce_requant");
@@ -210,21 +204,9 @@ int stage2(echo_dist *d, int phase, cudaStream_t st)
 
 int stage3(echo_dist *d, void *out, cudaStream_t st)
 {
-    const size_t sb = (d->variant & ECHO_VARIANT_FP16_SCALE) ? 2 : 1;
-    const size_t seg_codes = d->seg / 2, seg_scales = d->seg / d->group * sb;
-    for (int p = 0; p < d->world; p++) {
-        const uint8_t *blk = d->peer[p];
-        cudaError_t e = cudaMemcpyAsync(d->q_codes + p * seg_codes, blk + d->off_q_codes, seg_codes,
-                                        cudaMemcpyDeviceToDevice, st);
-        if (e == cudaSuccess)
-            e = cudaMemcpyAsync(d->q_scales + p * seg_scales, blk + d->off_q_scales, seg_scales,
-                                cudaMemcpyDeviceToDevice, st);
-        if (e != cudaSuccess)
-            return cuda_fail(e, "stage 3 copy from an owner's requantised segment");
-    }
     echo::K3Args a{};
-    a.qcodes = d->q_codes;
-    a.qscales = d->q_scales;
+    a.qcodes = d->xbuf + d->off_q_codes; // written by every owner in stage 2
+    a.qscales = d->xbuf + d->off_q_scales;
     a.out.p[0] = out;
     a.n = d->n;
     a.scale_stride = d->row_scale_stride;
@@ -287,20 +269,16 @@ echo_dist *echo_dist_create(int world, int rank, size_t n, int group, int dtype)
     d->dtype = dtype;
     d->row_scale_stride = round16(2 * (n / group));
     d->seg_scale_stride = round16(2 * (d->seg / group));
-    d->off_row_scales = round256(n / 2);
-    d->off_q_codes = d->off_row_scales + round256(d->row_scale_stride);
-    d->off_q_scales = d->off_q_codes + round256(d->seg / 2);
-    const size_t xbytes = d->off_q_scales + round256(d->seg_scale_stride);
+    d->off_recv_scales = round256(static_cast<size_t>(world) * (d->seg / 2));
+    d->off_q_codes = d->off_recv_scales + round256(static_cast<size_t>(world) * d->seg_scale_stride);
+    d->off_q_scales = d->off_q_codes + round256(n / 2);
+    const size_t xbytes = d->off_q_scales + round256(d->row_scale_stride);
     cudaError_t e = cudaGetDevice(&d->device);
     struct {
         void **p;
         size_t bytes;
     } allocs[] = {
         {reinterpret_cast<void **>(&d->xbuf), xbytes},
-        {reinterpret_cast<void **>(&d->recv_codes), static_cast<size_t>(world) * (d->seg / 2)},
-        {reinterpret_cast<void **>(&d->recv_scales), static_cast<size_t>(world) * d->seg_scale_stride},
-        {reinterpret_cast<void **>(&d->q_codes), n / 2},
-        {reinterpret_cast<void **>(&d->q_scales), d->row_scale_stride},
         {reinterpret_cast<void **>(&d->state), 4 * n * sizeof(float)},
         {reinterpret_cast<void **>(&d->dstatus), sizeof(int)},
     };

@@ -69,6 +69,14 @@ struct K1Args {
     uint32_t groups_per_seg; // n / P / G: owner of group g is g / groups_per_seg
     uint32_t rank_base;      // global rank of partial 0 (a one-rank launch of a process
                              // that holds one rank of a larger group; 0 otherwise)
+    // One process per rank (P == 1 launches only): the stage-1 row goes
+    // straight to the owners. Segment s lands in owner s's receive block
+    // owners.p[s], in the slot of rank rank_base: codes at
+    // rank_base * seg_code_bytes, scales at recv_scales_off + rank_base *
+    // seg_scale_stride.
+    bool to_owners;
+    RankOutPtrs owners;
+    size_t seg_code_bytes, recv_scales_off, seg_scale_stride;
     float lambda, one_minus_lambda;
     float *eps;              // sender feedback: every rank's rounding-#1 error [P][n]
     int P;
@@ -98,6 +106,13 @@ struct K2Args {
     bool fp16_scale;         // binary16 scales
     bool bf16;               // bf16 outputs: under binary16 scales the error is
                              // taken against the bf16-rounded value ranks receive
+    // One process per rank: the requantised segment goes straight to every
+    // rank's gathered buffer ranks.p[r] (codes from word q_chunk0, scales at
+    // q_scales_off + q_group0 scales), instead of qcodes / qscales.
+    bool to_ranks;
+    RankOutPtrs ranks;
+    uint32_t q_chunk0, q_group0;
+    size_t q_scales_off, q_scale_bytes; // where the scales start, and their room
     PipeCtl ctl;
 };
 

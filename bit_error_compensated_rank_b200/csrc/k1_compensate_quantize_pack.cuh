@@ -170,8 +170,26 @@ __device__ __forceinline__ void k1_consume(const K1Args &a, const uint8_t *smem,
                     qb[k] = code_bits(v[k], inv);
             }
             const uint32_t word = pack8_bits(qb);
-            if (active && in_bounds(chunk < code_words && (g + 1) * (f16 ? 2u : 1u) <= a.scale_stride,
-                                    a.ctl.status)) {
+            if (P == 1 && a.to_owners) {
+                // one process per rank: straight into the owner's receive block
+                const uint32_t owner = g / a.groups_per_seg;
+                const uint32_t gl = g - owner * a.groups_per_seg;               // group in the segment
+                const uint32_t cl = chunk - ((owner * a.groups_per_seg) << lanes_log2); // chunk in the segment
+                if (active && in_bounds(owner < kMaxRanks && (size_t(gl) + 1) * (f16 ? 2u : 1u) <= a.seg_scale_stride &&
+                                            (size_t(cl) + 1) * 4u <= a.seg_code_bytes,
+                                        a.ctl.status)) {
+                    uint8_t *blk = static_cast<uint8_t *>(a.owners.p[owner]);
+                    reinterpret_cast<uint32_t *>(blk + a.rank_base * a.seg_code_bytes)[cl] = word;
+                    if ((lane & ((1u << lanes_log2) - 1u)) == 0) { // the group's first lane
+                        uint8_t *row = blk + a.recv_scales_off + a.rank_base * a.seg_scale_stride;
+                        if (f16)
+                            reinterpret_cast<uint16_t *>(row)[gl] = static_cast<uint16_t>(scale);
+                        else
+                            row[gl] = static_cast<uint8_t>(scale);
+                    }
+                }
+            } else if (active && in_bounds(chunk < code_words && (g + 1) * (f16 ? 2u : 1u) <= a.scale_stride,
+                                           a.ctl.status)) {
                 reinterpret_cast<uint32_t *>(a.codes)[static_cast<size_t>(r) * code_words + chunk] = word;
                 if ((lane & ((1u << lanes_log2) - 1u)) == 0) { // the group's first lane
                     uint8_t *row = a.scales + static_cast<size_t>(r) * a.scale_stride;
@@ -180,16 +198,17 @@ __device__ __forceinline__ void k1_consume(const K1Args &a, const uint8_t *smem,
                     else
                         row[g] = static_cast<uint8_t>(scale);
                 }
-                if (EF) { // the new error v - q*step (exact unless a binary16 scale saturated)
-                    float e[kChunk];
+            }
+            if (EF && active && in_bounds(chunk < code_words, a.ctl.status)) {
+                // the new error v - q*step (exact unless a binary16 scale saturated)
+                float e[kChunk];
 #pragma unroll
-                    for (int k = 0; k < kChunk; k++)
-                        e[k] = __fmaf_rn(-code_value(qb[k]), st, v[k]);
-                    float4 *eo = reinterpret_cast<float4 *>(a.eps + static_cast<size_t>(r) * a.n) +
-                                 2 * static_cast<size_t>(chunk);
-                    eo[0] = make_float4(e[0], e[1], e[2], e[3]);
-                    eo[1] = make_float4(e[4], e[5], e[6], e[7]);
-                }
+                for (int k = 0; k < kChunk; k++)
+                    e[k] = __fmaf_rn(-code_value(qb[k]), st, v[k]);
+                float4 *eo = reinterpret_cast<float4 *>(a.eps + static_cast<size_t>(r) * a.n) +
+                             2 * static_cast<size_t>(chunk);
+                eo[0] = make_float4(e[0], e[1], e[2], e[3]);
+                eo[1] = make_float4(e[4], e[5], e[6], e[7]);
             }
         }
         __syncwarp();

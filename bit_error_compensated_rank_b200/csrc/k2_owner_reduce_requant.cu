@@ -225,14 +225,36 @@ __global__ void __launch_bounds__(kThreads)
                 }
             }
 
+            if (active && a.to_ranks &&
+                in_bounds(chunk < a.n / kChunk && (size_t(a.q_chunk0) + chunk + 1) * 4u <= a.q_scales_off &&
+                              (size_t(a.q_group0) + g + 1) * (F16 ? 2u : 1u) <= a.q_scale_bytes,
+                          a.ctl.status)) {
+                // one process per rank: the owned segment straight into every rank's gathered buffer
+                const uint32_t word = pack8_bits(qb);
+                const bool first = (lane & ((1u << a.lanes_log2) - 1u)) == 0;
+#pragma unroll
+                for (int p = 0; p < P; p++) {
+                    uint8_t *blk = static_cast<uint8_t *>(a.ranks.p[p]);
+                    reinterpret_cast<uint32_t *>(blk)[a.q_chunk0 + chunk] = word;
+                    if (first) {
+                        if (F16)
+                            reinterpret_cast<uint16_t *>(blk + a.q_scales_off)[a.q_group0 + g] =
+                                static_cast<uint16_t>(scale);
+                        else
+                            blk[a.q_scales_off + a.q_group0 + g] = static_cast<uint8_t>(scale);
+                    }
+                }
+            }
             if (active && in_bounds(chunk < a.n / kChunk && (g + 1) * (F16 ? 2u : 1u) <= a.scale_stride,
                                     a.ctl.status)) {
-                reinterpret_cast<uint32_t *>(a.qcodes)[chunk] = pack8_bits(qb);
-                if ((lane & ((1u << a.lanes_log2) - 1u)) == 0) { // the group's first lane
-                    if (F16)
-                        reinterpret_cast<uint16_t *>(a.qscales)[g] = static_cast<uint16_t>(scale);
-                    else
-                        a.qscales[g] = static_cast<uint8_t>(scale);
+                if (!a.to_ranks) {
+                    reinterpret_cast<uint32_t *>(a.qcodes)[chunk] = pack8_bits(qb);
+                    if ((lane & ((1u << a.lanes_log2) - 1u)) == 0) { // the group's first lane
+                        if (F16)
+                            reinterpret_cast<uint16_t *>(a.qscales)[g] = static_cast<uint16_t>(scale);
+                        else
+                            a.qscales[g] = static_cast<uint8_t>(scale);
+                    }
                 }
                 if (COMP) {
 #pragma unroll

@@ -318,16 +318,19 @@ ECHO_API int echo_debug_touch_guard(echo_handle *h);
  * One process per rank (echo_dist_*). The same all-reduce when each of the
  * world ranks is its own process holding only its own partial; every rank
  * keeps the compensator state of the segment it owns, [rank*n/world,
- * (rank+1)*n/world). A call runs in three stages:
- *   stage 1  this rank's partial x is rounded into its stage-1 wire row
- *            (kernel 1 for one rank, the owner mapping of the whole group);
- *   stage 2  segment `rank` of every rank's row is copied into this process,
- *            then kernel 2 sums, requantises and updates the owned state;
- *   stage 3  every owner's requantised segment is copied in, then kernel 3
- *            writes the result (n elements, identical on every rank) to out.
- * The copies read the other processes' exported buffers (CUDA IPC; on
- * several GPUs, peer reads over NVLink) into this GPU's memory; the kernels
- * read local memory only, and no kernel waits on another process. The caller
+ * (rank+1)*n/world). Every rank exports a block (CUDA IPC) that the others
+ * write into: a receive slot per rank for the owned segment's stage-1 wire,
+ * and the gathered requantised tensor. A call runs in three stages:
+ *   stage 1  kernel 1 rounds this rank's partial x and stores each segment's
+ *            codes and scales straight into its owner's receive slot;
+ *   stage 2  kernel 2 sums the owned segment from the receive slots,
+ *            requantises it, updates the owned state, and stores the
+ *            requantised segment into every rank's gathered tensor;
+ *   stage 3  kernel 3 writes the result (n elements, identical on every rank)
+ *            from the local gathered tensor to out.
+ * The wire moves as plain stores into the other processes' blocks (on
+ * several GPUs, peer stores over NVLink); the kernels read local memory only,
+ * and no kernel waits on another process. The caller
  * orders the stages across processes: after each stage, synchronise the
  * stream, then a host barrier over all ranks (also after stage 3, before the
  * next call's stage 1). The results are bit for bit those of echo_allreduce
@@ -338,7 +341,7 @@ ECHO_API int echo_debug_touch_guard(echo_handle *h);
  *   whole groups whose code rows start on 16 bytes), group and dtype as for
  *   echo_create. Allocates on the current device, NULL on error.
  * echo_dist_export: the CUDA IPC handle (ECHO_IPC_HANDLE_BYTES bytes) of this
- *   rank's exported buffer (its stage-1 row and its requantised segment).
+ *   rank's exported block (its receive slots and its gathered tensor).
  * echo_dist_connect: handles = world handles in rank order (this rank's own
  *   entry is ignored); opens the others' buffers. Once per handle.
  * echo_dist_stage(d, stage, x, out, phase, stream): x (stage 1) and out

@@ -1,8 +1,8 @@
 """The all-reduce with one process per rank (echo_dist_*), several processes
 on one GPU: each holds only its own partial and the state of the segment it
-owns, the wire crosses processes through CUDA IPC copies, and every rank's
-result and owned state must equal the oracle's bit for bit, call after call,
-for both phases, in place and out of place.
+owns, the kernels store the wire straight into the other processes' blocks
+(CUDA IPC), and every rank's result and owned state must equal the oracle's
+bit for bit, call after call, for both phases, in place and out of place.
 
 No kernel waits on another process: the stages are ordered by host barriers
 (gloo), so the processes can share one GPU."""
