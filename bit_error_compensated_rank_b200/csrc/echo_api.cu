@@ -14,6 +14,7 @@
 #include <cuda_runtime.h>
 #include <nvtx3/nvToolsExt.h>
 
+#include <atomic>
 #include <cstdarg>
 #include <cstdio>
 #include <cstdlib>
@@ -474,7 +475,8 @@ namespace echo {
 
 static int sm_count()
 {
-    static int sms = 0;
+    static std::atomic<int> cached{0}; // threads that race here compute the same value
+    int sms = cached.load(std::memory_order_relaxed);
     if (sms == 0) {
         int dev = 0, v = 0;
         if (cudaGetDevice(&dev) == cudaSuccess &&
@@ -482,6 +484,7 @@ static int sm_count()
             sms = v;
         else
             sms = 148;
+        cached.store(sms, std::memory_order_relaxed);
     }
     return sms;
 }

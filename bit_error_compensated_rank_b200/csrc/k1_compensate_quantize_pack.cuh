@@ -37,6 +37,8 @@
 
 #include <cuda_runtime.h>
 
+#include <atomic>
+
 // Included by k1_compensate_quantize_pack.cu (the default build) and by the
 // k1_variants_*.cu files (the general build, split by element type and
 // feedback setting so that they compile in parallel). Everything here has
@@ -303,12 +305,16 @@ template <int P, bool BF16, bool COMP, bool EF, bool GEN>
 cudaError_t launch_p(const K1Args &a, cudaStream_t st)
 {
     using Sh = K1Shape<P, BF16, COMP, EF>;
-    static int resident = 0;
+    // CTAs per SM of this instantiation, found once (threads that race here
+    // compute the same value)
+    static std::atomic<int> cached{0};
+    int resident = cached.load(std::memory_order_relaxed);
     auto kern = k1_compensate_quantize_pack<P, BF16, COMP, EF, GEN>;
     if (resident == 0) {
         cudaError_t e = prepare_kernel(reinterpret_cast<const void *>(kern), kThreads, Sh::kSmem, &resident);
         if (e != cudaSuccess)
             return e;
+        cached.store(resident, std::memory_order_relaxed);
     }
     const size_t elems = static_cast<size_t>(a.chunk_end - a.chunk_begin) * kChunk;
     K1Args b = a;

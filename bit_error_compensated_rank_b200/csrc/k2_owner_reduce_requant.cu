@@ -39,6 +39,8 @@
 
 #include <cuda_runtime.h>
 
+#include <atomic>
+
 namespace echo {
 namespace {
 
@@ -281,12 +283,16 @@ template <int P, bool COMP, bool SUM, bool F16>
 cudaError_t launch_p(const K2Args &a, cudaStream_t st)
 {
     using Sh = K2Shape<P, COMP, F16>;
-    static int resident = 0;
+    // CTAs per SM of this instantiation, found once (threads that race here
+    // compute the same value)
+    static std::atomic<int> cached{0};
+    int resident = cached.load(std::memory_order_relaxed);
     auto kern = k2_owner_reduce_requant<P, COMP, SUM, F16>;
     if (resident == 0) {
         cudaError_t e = prepare_kernel(reinterpret_cast<const void *>(kern), kThreads, Sh::kSmem, &resident);
         if (e != cudaSuccess)
             return e;
+        cached.store(resident, std::memory_order_relaxed);
     }
     const size_t elems = static_cast<size_t>(a.chunk_end - a.chunk_begin) * kChunk;
     K2Args b = a;

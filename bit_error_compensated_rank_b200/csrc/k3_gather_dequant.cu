@@ -23,6 +23,8 @@
 
 #include <cuda_runtime.h>
 
+#include <atomic>
+
 namespace echo {
 namespace {
 
@@ -196,12 +198,16 @@ template <int P, bool BF16, bool F16>
 cudaError_t launch_p(const K3Args &a, cudaStream_t st)
 {
     using Sh = K3Shape<BF16, F16>;
-    static int resident = 0;
+    // CTAs per SM of this instantiation, found once (threads that race here
+    // compute the same value)
+    static std::atomic<int> cached{0};
+    int resident = cached.load(std::memory_order_relaxed);
     auto kern = k3_gather_dequant<P, BF16, F16>;
     if (resident == 0) {
         cudaError_t e = prepare_kernel(reinterpret_cast<const void *>(kern), kThreads, Sh::kSmem, &resident);
         if (e != cudaSuccess)
             return e;
+        cached.store(resident, std::memory_order_relaxed);
     }
     const size_t elems = static_cast<size_t>(a.chunk_end - a.chunk_begin) * kChunk;
     K3Args b = a;
