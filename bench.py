@@ -260,7 +260,7 @@ def cpu_baseline_leg(variant: int = 0) -> dict:
     t = sum(times) / len(times)
     return {
         "value": round(2 * CPU_SAMPLE_N / t / 1e9, 6), "unit": UNIT, "cores": 1, "kind": "oracle",
-        "sample": f"P=8 x 2^20 bf16 elements per rank (2 MiB), same distribution, compensation on, "
+        "sample": f"P={P} x 2^20 bf16 elements per rank (2 MiB), same distribution, compensation on, "
                   f"{len(times)} sequential calls, {sum(times):.1f} s single-threaded on one pinned "
                   f"core; value = 2*n/t per call (bf16-equivalent)",
         "host": host_info(),
@@ -276,7 +276,7 @@ def run_reference(args, rank: int, world: int) -> dict | None:
     timed = times[args.warmup:]
     t = sum(timed) / len(timed)
     value = 2 * REF_SAMPLE_N / t / 1e9
-    sample = (f"P=8 x 2^18 bf16 elements per rank per step (512 KiB), same distribution as the "
+    sample = (f"P={P} x 2^18 bf16 elements per rank per step (512 KiB), same distribution as the "
               f"1 GiB workload, compensation on; oracle single-threaded on the host")
     return {
         "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": UNIT,
@@ -306,6 +306,8 @@ NCU_TRAFFIC = {
 
 def workload_name(args) -> str:
     name = WORKLOAD if args.group == 32 else WORKLOAD.replace("group 32", f"group {args.group}")
+    if P != 8:
+        name = name.replace("P=8 ranks", f"P={P} ranks")
     return name if args.variant == "default" else f"{name}, variant {args.variant}"
 
 
@@ -384,7 +386,7 @@ def run_echo(args, rank: int, world: int, local: int) -> dict | None:
     src = os.path.join(ROOT, "bit_error_compensated_rank_b200", "csrc", names[dom] + ".cu")
     traffic = None
     # captured for the default variant and group
-    rec = NCU_TRAFFIC.get(names[dom]) if variant == 0 and args.group == 32 else None
+    rec = NCU_TRAFFIC.get(names[dom]) if variant == 0 and args.group == 32 and P == 8 else None
     if rec and rec["source_sha"] == _source_hash(src):
         traffic = round(rec["bytes_per_elem"] * n)
 
@@ -552,7 +554,11 @@ def main(argv=None):
                     help="where rounding errors are fed back (default: the method as read)")
     ap.add_argument("--group", type=int, choices=[16, 32, 64, 128], default=32,
                     help="elements per scale (default 32, the method as read)")
+    ap.add_argument("--ranks", type=int, default=8, choices=range(2, 17), metavar="P",
+                    help="simulated ranks per GPU, 2..16 (default 8, the benchmark's workload)")
     args = ap.parse_args(argv)
+    global P
+    P = args.ranks
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     rank, world, local = dist_env()
