@@ -44,17 +44,17 @@
 namespace echo {
 namespace {
 
-// Consumer warps of a CTA: 8, or 16 from P = 12 ranks on, where each chunk
-// restores so many ranks that one CTA per SM needs more warps in flight.
-constexpr int k2_warps(int P) { return P >= 12 ? 16 : 8; }
+constexpr int kConsumerWarps = 8;
+constexpr int kConsumers = kConsumerWarps * 32;
+constexpr int kThreads = kConsumers + 32; // + one producer warp
 
 // Bytes of one stage for `chunks` chunks per consumer thread: P code tiles,
 // P scale tiles (1 or 2 bytes per group of at least kMinGroup), and the f, s
 // tiles.
 constexpr int k2_stage_bytes(int P, bool comp, bool f16, int chunks)
 {
-    const int tile = k2_warps(P) * 32 * kChunk * chunks;
-    return P * (tile / 2 + tile / kMinGroup * (f16 ? 2 : 1)) + (comp ? 2 * tile * 4 : 0);
+    return P * (kConsumers * kChunk * chunks / 2 + kConsumers * kChunk * chunks / kMinGroup * (f16 ? 2 : 1)) +
+           (comp ? 2 * kConsumers * kChunk * chunks * 4 : 0);
 }
 
 // The largest of ECHO_K2_CHUNKS, /2, /4 whose stages fit the budget.
@@ -69,9 +69,6 @@ constexpr int k2_chunks(int P, bool comp, bool f16)
 template <int P, bool COMP, bool F16>
 struct K2Shape {
     static constexpr int kChunks = k2_chunks(P, COMP, F16); // chunks per consumer thread
-    static constexpr int kConsumerWarps = k2_warps(P);
-    static constexpr int kConsumers = kConsumerWarps * 32;
-    static constexpr int kThreads = kConsumers + 32; // + one producer warp
     static constexpr int kTile = kConsumers * kChunk * kChunks;
     static constexpr int kStages = ECHO_K2_STAGES;
     static constexpr int kCodeBytes = kTile / 2;          // one rank's code tile
@@ -85,12 +82,10 @@ struct K2Shape {
 __device__ __forceinline__ uint32_t round16(uint32_t x) { return (x + 15u) & ~15u; }
 
 template <int P, bool COMP, bool SUM, bool F16>
-__global__ void __launch_bounds__(K2Shape<P, COMP, F16>::kThreads)
+__global__ void __launch_bounds__(kThreads)
     k2_owner_reduce_requant(const K2Args a)
 {
     using Sh = K2Shape<P, COMP, F16>;
-    constexpr int kConsumerWarps = Sh::kConsumerWarps;
-    constexpr int kConsumers = Sh::kConsumers;
     constexpr uint32_t kScaleLog2 = F16 ? 1u : 0u; // log2 of the bytes per scale
     constexpr int S = Sh::kStages;
     extern __shared__ __align__(128) uint8_t smem[];
@@ -294,17 +289,17 @@ cudaError_t launch_p(const K2Args &a, cudaStream_t st)
     int resident = cached.load(std::memory_order_relaxed);
     auto kern = k2_owner_reduce_requant<P, COMP, SUM, F16>;
     if (resident == 0) {
-        cudaError_t e = prepare_kernel(reinterpret_cast<const void *>(kern), Sh::kThreads, Sh::kSmem, &resident);
+        cudaError_t e = prepare_kernel(reinterpret_cast<const void *>(kern), kThreads, Sh::kSmem, &resident);
         if (e != cudaSuccess)
             return e;
         cached.store(resident, std::memory_order_relaxed);
     }
     const size_t elems = static_cast<size_t>(a.chunk_end - a.chunk_begin) * kChunk;
     K2Args b = a;
-    b.tile_log2 = pick_tile_log2(elems, Sh::kTile, Sh::kConsumers * kChunk, resident);
+    b.tile_log2 = pick_tile_log2(elems, Sh::kTile, kConsumers * kChunk, resident);
     b.tile = 1u << b.tile_log2;
     const uint32_t tiles = static_cast<uint32_t>((elems + b.tile - 1) >> b.tile_log2);
-    return launch_chained(kern, persistent_grid(tiles, resident), Sh::kThreads, Sh::kSmem, st, b);
+    return launch_chained(kern, persistent_grid(tiles, resident), kThreads, Sh::kSmem, st, b);
 }
 
 template <int P, bool F16>
