@@ -331,7 +331,8 @@ def run_echo(args, rank: int, world: int, local: int) -> dict | None:
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
     dist = init_dist(world, "nccl")
-    n = args.n
+    # whole groups on every rank: round down to a multiple of P * max(group, 32)
+    n = args.n - args.n % (P * max(args.group, 32))
     stream = torch.cuda.current_stream(device)
 
     # inputs resident in HBM before timing; outputs to separate buffers so
@@ -475,7 +476,7 @@ def run_sweep(args) -> None:
         wl.torch_outlier_gaussian_(send[r], seed=SEED, call=0, rank=r)
     variant = VARIANTS[args.variant]
     for k in range(12, 30):
-        n = 1 << k
+        n = (1 << k) - (1 << k) % (P * max(args.group, 32))
         h = echo.Echo(P, n, echo.ECHO_BF16, args.group)
         if variant:
             h.set_variant(variant)
