@@ -185,4 +185,40 @@ __device__ __forceinline__ void produce_tiles(uint64_t *full, uint64_t *empty, u
         mbar_wait_bounded(&full[t % S], (t / S) & 1u, limit);
 }
 
+// The same ring fed by the whole producer warp: for local tile i, lane 0
+// arms full[i % S] (arm(i): arrive with the tile's byte count), then the
+// tile's ncopies bulk copies are issued by the 32 lanes in parallel
+// (copy(i, k) for k = lane, lane + 32, ...), so a tile made of many small
+// copies does not wait on one thread issuing them in turn. Every lane of the
+// warp must call it. The stage waits and the final drain are as in
+// produce_tiles, and bounded the same way.
+template <int S, typename Arm, typename Copy>
+__device__ __forceinline__ void produce_tiles_warp(uint64_t *full, uint64_t *empty, uint32_t tiles, bool stall,
+                                                   long long limit, int *status, int status_bit, uint32_t ncopies,
+                                                   Arm arm, Copy copy)
+{
+    const uint32_t lane = threadIdx.x & 31u;
+    uint32_t i = 0;
+    if (!stall) {
+        for (; i < tiles; i++) {
+            const uint32_t s = i % S;
+            if (i >= static_cast<uint32_t>(S) &&
+                !__all_sync(0xFFFFFFFFu, mbar_wait_bounded(&empty[s], ((i / S) - 1) & 1u, limit))) {
+                if (lane == 0)
+                    atomicOr(status, status_bit);
+                break;
+            }
+            if (lane == 0)
+                arm(i);
+            __syncwarp();
+            for (uint32_t k = lane; k < ncopies; k += 32)
+                copy(i, k);
+        }
+    }
+    if (lane == 0)
+        for (uint32_t t = i > static_cast<uint32_t>(S) ? i - S : 0; t < i; t++)
+            mbar_wait_bounded(&full[t % S], (t / S) & 1u, limit);
+    __syncwarp();
+}
+
 } // namespace echo

@@ -117,34 +117,50 @@ __global__ void __launch_bounds__(kThreads)
         // The scale tile of a ragged last tile is rounded up to 16 bytes;
         // scale rows are padded to 16 bytes, so the extra bytes stay inside
         // the row and are never used.
-        if (lane == 0)
-            produce_tiles<S>(
-                full, empty, mine, a.ctl.stall, a.ctl.wait_cycles, a.ctl.status, kStatusTimeoutK2, [&](uint32_t i) {
-                    const size_t el0 = e0 + static_cast<size_t>(blockIdx.x + i * gridDim.x) * tile;
-                    const uint32_t cnt = static_cast<uint32_t>(e1 - el0 < size_t(tile) ? e1 - el0 : tile);
-                    const uint32_t sc_bytes = round16((cnt >> (a.lanes_log2 + 3)) << kScaleLog2);
-                    uint8_t *stage = smem + (i % S) * Sh::kStageBytes;
-                    uint64_t *bar = &full[i % S];
-                    // code, state and scale copies against their rows
-                    const bool ok = in_bounds(el0 + cnt <= a.n && cnt <= Sh::kTile && sc_bytes <= Sh::kScaleBytes &&
-                                                  ((el0 >> (a.lanes_log2 + 3)) << kScaleLog2) + sc_bytes <=
-                                                      a.scale_stride,
-                                              a.ctl.status);
-                    mbar_arrive_expect_tx(bar, ok ? P * (cnt / 2 + sc_bytes) + (COMP ? 2 * cnt * 4 : 0) : 0u);
-                    if (!ok)
-                        return;
-#pragma unroll
-                    for (int r = 0; r < P; r++) {
-                        bulk_load(stage + r * Sh::kCodeBytes, a.codes + r * (a.n / 2) + el0 / 2, cnt / 2, bar);
-                        bulk_load(stage + P * Sh::kCodeBytes + r * Sh::kScaleBytes,
-                                  a.scales + r * a.scale_stride + ((el0 >> (a.lanes_log2 + 3)) << kScaleLog2),
-                                  sc_bytes, bar);
-                    }
-                    if (COMP) {
-                        bulk_load(stage + Sh::kStateOff, a.f + el0, cnt * 4, bar);
-                        bulk_load(stage + Sh::kStateOff + Sh::kTile * 4, a.s + el0, cnt * 4, bar);
-                    }
-                });
+        // A tile is 2P + 2 copies (P code slices, P scale slices, f, s),
+        // issued by the warp's lanes in parallel.
+        struct Tile {
+            size_t el0;
+            uint32_t cnt, sc_bytes;
+            bool ok;
+        };
+        auto tile_of = [&](uint32_t i) {
+            Tile t;
+            t.el0 = e0 + static_cast<size_t>(blockIdx.x + i * gridDim.x) * tile;
+            t.cnt = static_cast<uint32_t>(e1 - t.el0 < size_t(tile) ? e1 - t.el0 : tile);
+            t.sc_bytes = round16((t.cnt >> (a.lanes_log2 + 3)) << kScaleLog2);
+            // code, state and scale copies against their rows
+            t.ok = in_bounds(t.el0 + t.cnt <= a.n && t.cnt <= Sh::kTile && t.sc_bytes <= Sh::kScaleBytes &&
+                                 ((t.el0 >> (a.lanes_log2 + 3)) << kScaleLog2) + t.sc_bytes <= a.scale_stride,
+                             a.ctl.status);
+            return t;
+        };
+        produce_tiles_warp<S>(
+            full, empty, mine, a.ctl.stall, a.ctl.wait_cycles, a.ctl.status, kStatusTimeoutK2,
+            2 * P + (COMP ? 2 : 0),
+            [&](uint32_t i) {
+                const Tile t = tile_of(i);
+                mbar_arrive_expect_tx(&full[i % S],
+                                      t.ok ? P * (t.cnt / 2 + t.sc_bytes) + (COMP ? 2 * t.cnt * 4 : 0) : 0u);
+            },
+            [&](uint32_t i, uint32_t k) {
+                const Tile t = tile_of(i);
+                if (!t.ok)
+                    return;
+                uint8_t *stage = smem + (i % S) * Sh::kStageBytes;
+                uint64_t *bar = &full[i % S];
+                if (k < static_cast<uint32_t>(P)) {
+                    bulk_load(stage + k * Sh::kCodeBytes, a.codes + k * (a.n / 2) + t.el0 / 2, t.cnt / 2, bar);
+                } else if (k < 2u * P) {
+                    const uint32_t r = k - P;
+                    bulk_load(stage + P * Sh::kCodeBytes + r * Sh::kScaleBytes,
+                              a.scales + r * a.scale_stride + ((t.el0 >> (a.lanes_log2 + 3)) << kScaleLog2),
+                              t.sc_bytes, bar);
+                } else if (COMP) {
+                    const uint32_t j = k - 2 * P; // 0: f, 1: s
+                    bulk_load(stage + Sh::kStateOff + j * Sh::kTile * 4, (j ? a.s : a.f) + t.el0, t.cnt * 4, bar);
+                }
+            });
         return;
     }
 
