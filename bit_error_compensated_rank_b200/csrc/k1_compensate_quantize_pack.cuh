@@ -252,42 +252,34 @@ __global__ void __launch_bounds__(kThreads)
     allow_successor();
 
     if (warp == kConsumerWarps) { // producer
-        // A tile is P partial slices, f and s, and the P error slices with
-        // sender feedback: copies issued by the warp's lanes in parallel.
-        auto tile_at = [&](uint32_t i, size_t &el0, uint32_t &cnt) {
-            el0 = e0 + static_cast<size_t>(blockIdx.x + i * gridDim.x) * tile;
-            cnt = static_cast<uint32_t>(e1 - el0 < size_t(tile) ? e1 - el0 : tile);
-            // every copy covers elements [el0, el0 + cnt) of an n-element row
-            return in_bounds(el0 + cnt <= a.n && cnt <= Sh::kTile, a.ctl.status);
-        };
-        produce_tiles_warp<S>(
-            full, empty, mine, a.ctl.stall, a.ctl.wait_cycles, a.ctl.status, kStatusTimeoutK1,
-            P + (COMP ? 2 : 0) + (EF ? P : 0),
-            [&](uint32_t i) {
-                size_t el0;
-                uint32_t cnt;
-                const bool ok = tile_at(i, el0, cnt);
-                mbar_arrive_expect_tx(&full[i % S], ok ? cnt * Sh::kStageBytes / Sh::kTile : 0u);
-            },
-            [&](uint32_t i, uint32_t k) {
-                size_t el0;
-                uint32_t cnt;
-                if (!tile_at(i, el0, cnt))
-                    return;
-                uint8_t *stage = smem + (i % S) * Sh::kStageBytes;
-                uint64_t *bar = &full[i % S];
-                if (k < static_cast<uint32_t>(P)) {
-                    bulk_load(stage + k * Sh::kXBytes, static_cast<const uint8_t *>(a.x.p[k]) + el0 * Sh::kEB,
-                              cnt * Sh::kEB, bar);
-                } else if (COMP && k < static_cast<uint32_t>(P) + 2) {
-                    const uint32_t j = k - P; // 0: f, 1: s
-                    bulk_load(stage + Sh::kStateOff + j * Sh::kTile * 4, (j ? a.s : a.f) + el0, cnt * 4, bar);
-                } else if (EF) {
-                    const uint32_t r = k - P - (COMP ? 2 : 0);
-                    bulk_load(stage + Sh::kEpsOff + r * Sh::kTile * 4, a.eps + static_cast<size_t>(r) * a.n + el0,
-                              cnt * 4, bar);
-                }
-            });
+        if (lane == 0)
+            produce_tiles<S>(full, empty, mine, a.ctl.stall, a.ctl.wait_cycles, a.ctl.status, kStatusTimeoutK1,
+                             [&](uint32_t i) {
+                                 const size_t el0 = e0 + static_cast<size_t>(blockIdx.x + i * gridDim.x) * tile;
+                                 const uint32_t cnt = static_cast<uint32_t>(e1 - el0 < size_t(tile) ? e1 - el0 : tile);
+                                 uint8_t *stage = smem + (i % S) * Sh::kStageBytes;
+                                 uint64_t *bar = &full[i % S];
+                                 // every copy below covers elements [el0, el0 + cnt) of an n-element row
+                                 const bool ok = in_bounds(el0 + cnt <= a.n && cnt <= Sh::kTile, a.ctl.status);
+                                 mbar_arrive_expect_tx(bar, ok ? cnt * Sh::kStageBytes / Sh::kTile : 0u);
+                                 if (!ok)
+                                     return;
+#pragma unroll
+                                 for (int r = 0; r < P; r++)
+                                     bulk_load(stage + r * Sh::kXBytes,
+                                               static_cast<const uint8_t *>(a.x.p[r]) + el0 * Sh::kEB,
+                                               cnt * Sh::kEB, bar);
+                                 if (COMP) {
+                                     bulk_load(stage + Sh::kStateOff, a.f + el0, cnt * 4, bar);
+                                     bulk_load(stage + Sh::kStateOff + Sh::kTile * 4, a.s + el0, cnt * 4, bar);
+                                 }
+                                 if (EF) {
+#pragma unroll
+                                     for (int r = 0; r < P; r++)
+                                         bulk_load(stage + Sh::kEpsOff + r * Sh::kTile * 4,
+                                                   a.eps + static_cast<size_t>(r) * a.n + el0, cnt * 4, bar);
+                                 }
+                             });
         return;
     }
 
