@@ -349,3 +349,29 @@ def test_cuda_graph_replay(oracle):
         del graph
     finally:
         h.close()
+
+
+def test_host_end_to_end_fp32_backward(oracle):
+    """The host path with binary32 partials, in the backward phase, over a
+    ragged last piece; the forward state stays untouched."""
+    import torch
+    from bit_error_compensated_rank_b200 import echo
+    P, n = 2, 2 * 32 * 70001  # 4.48 M elements per rank: a full piece and a ragged one
+    h = echo.Echo(P, n, echo.ECHO_FP32)
+    try:
+        f = np.zeros(n, np.float32)
+        s = np.zeros(n, np.float32)
+        for k in range(2):
+            x = gaussian(P, n, seed=18, call=k, dtype="fp32")
+            host_in = [torch.from_numpy(np.ascontiguousarray(x[r])).pin_memory() for r in range(P)]
+            host_out = torch.empty(n, dtype=torch.float32).pin_memory()
+            h.allreduce_host(host_in, host_out, echo.ECHO_BWD)
+            ref = oracle.allreduce(x, f, s, Params())
+            assert_same_bits(host_out.numpy(), ref["out"], "host result")
+            gf, gs = h.get_state(echo.ECHO_BWD)
+            assert_same_bits(gf, f, "fast estimate")
+            assert_same_bits(gs, s, "slow estimate")
+            ff, fs = h.get_state(echo.ECHO_FWD)
+            assert not ff.any() and not fs.any()
+    finally:
+        h.close()
