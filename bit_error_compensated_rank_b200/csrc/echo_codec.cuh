@@ -94,18 +94,18 @@ __device__ __forceinline__ float half_step(uint32_t h)
 }
 
 // Smallest positive finite binary16 s with 7*s >= A (A finite, >= 0), as its
-// pattern; 0 for A == 0; 0x7BFF (65504) when 7*65504 < A. An estimate, A/7
-// rounded up to binary16 from a binary32 product, lies within one binary16
-// step of the answer (the product's relative error is about 2^-23, the
-// binary16 spacing 2^-10), and one exact test on each side settles it: 7*s
-// has at most 14 significant bits, so the binary32 product is exact.
+// pattern; 0 for A == 0; 0x7BFF (65504) when 7*65504 < A. The estimate
+// u = A * RU(1/7), rounded up, is at least A/7 and within a relative 2^-22
+// of it; rounded up to binary16 it is therefore never below the answer and
+// at most one binary16 step above it (the binary16 spacing is 2^-10
+// relative). One exact test on the step below settles it: 7*s has at most
+// 14 significant bits, so the binary32 product is exact.
 __device__ __forceinline__ uint32_t half_scale_bits(float A)
 {
-    constexpr float kSeventh = 0.142857142857142857f;
-    const uint32_t h = min(static_cast<uint32_t>(__half_as_ushort(__float2half_ru(__fmul_rn(A, kSeventh)))), 0x7BFFu);
-    const bool up = __fmul_rn(7.f, half_step(h)) < A && h < 0x7BFFu;
-    const bool down = !up && h > 1u && __fmul_rn(7.f, half_step(h - 1u)) >= A;
-    return A == 0.f ? 0u : h + (up ? 1u : 0u) - (down ? 1u : 0u);
+    const float u = __fmul_ru(A, __uint_as_float(0x3E124925u)); // RU(1/7) = 0.14285715
+    const uint32_t h = min(static_cast<uint32_t>(__half_as_ushort(__float2half_ru(u))), 0x7BFFu);
+    const bool down = h > 1u && __fmul_rn(7.f, half_step(h - 1u)) >= A;
+    return h - (down ? 1u : 0u);
 }
 
 // Bit pattern kRoundBits + q of the code q in [-7, 7] nearest to v/step, a
@@ -138,29 +138,55 @@ __device__ __forceinline__ bool half_scale_saturates(float A)
 }
 
 // The 8 codes of one lane under a binary16 step (the results of
-// code_bits_near), with a shortcut. In a group whose scale did not saturate,
-// |v/step| <= 7, and the exact product v*inv lies within 2^-19 of v/step
-// (inv has a relative error of at most about 2^-23; see half_inv). The
-// kRound addition fused with the product, t = RN(v*inv + kRound), gives the
-// nearest integer k to v*inv, and d = RN(v*inv - k) its distance. When every
-// |d| of the lane is below 1/2 - 2^-18, each k is the nearest code to v/step.
-// Otherwise, or when the group saturated, the lane takes the exact path for
-// all 8 values: one branch per lane, taken rarely.
-__device__ __forceinline__ void codes8_half(const float (&v)[kChunk], float step, float inv, float half, bool sat,
-                                            uint32_t (&qb)[kChunk])
+// code_bits_near), in z-form: the bit pattern z of the binary32
+// RN(v*inv + kZ), kZ = 192 + 1/2 + 2*2^-16. In a group whose scale did not
+// saturate, |v/step| <= 7, so z stays in the binade [128, 256), where the
+// spacing is 2^-16 and z = 0x43400000 + Z with the integer
+// Z = RN(2^16*(v*inv + 1/2) + 2). Then z >> 16 = 0x4340 + floor(Z / 2^16),
+// and byte 2 of z holds that code as 0x40 + q (its low nibble is q in two's
+// complement). inv has a relative error of at most about 2^-23 (half_inv),
+// so Z lies within 0.56 of 2^16*(v/step + 1/2) + 2. When the low 16 bits of
+// Z are at least 3, 2^16*(v/step + 1/2) is then strictly between two
+// multiples of 2^16 and floor(Z / 2^16) is the nearest code to v/step, not a
+// tie. The lane takes the minimum of its 8 low halves two at a time (a 16x2
+// minimum); if one is below 3, or the group saturated, the lane takes the exact path for all 8
+// values: one branch per lane, taken rarely.
+constexpr float kZ = 192.500030517578125f; // 192 + 1/2 + 2*2^-16, bits 0x43408002
+constexpr uint32_t kZMargin = 3;
+
+__device__ __forceinline__ uint32_t min_u16x2(uint32_t a, uint32_t b)
 {
-    constexpr float kSafe = 0.5f - 0.000003814697265625f; // 1/2 - 2^-18
-    float worst = 0.f;
+    uint32_t d;
+    asm("min.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+// z-form of the rounded pattern kRoundBits + q (for the exact path).
+__device__ __forceinline__ uint32_t zcode_of_bits(uint32_t bits)
+{
+    return ((bits - kRoundBits) << 16) + 0x43408000u;
+}
+
+// The rounded pattern kRoundBits + q of a z-form code (code_value, pack8_bits).
+__device__ __forceinline__ uint32_t zcode_bits(uint32_t z)
+{
+    return (z >> 16) + (kRoundBits - 0x4340u);
+}
+
+__device__ __forceinline__ void codes8_half(const float (&v)[kChunk], float step, float inv, float half, bool sat,
+                                            uint32_t (&z)[kChunk])
+{
 #pragma unroll
-    for (int k = 0; k < kChunk; k++) {
-        const float t = __fmaf_rn(v[k], inv, kRound);
-        qb[k] = __float_as_uint(t);
-        worst = fmaxf(worst, fabsf(__fmaf_rn(v[k], inv, -__fsub_rn(t, kRound))));
-    }
-    if (sat || !(worst < kSafe)) {
+    for (int k = 0; k < kChunk; k++)
+        z[k] = __float_as_uint(__fmaf_rn(v[k], inv, kZ));
+    const uint32_t lo = min_u16x2(min_u16x2(__byte_perm(z[0], z[1], 0x5410), __byte_perm(z[2], z[3], 0x5410)),
+                                  min_u16x2(__byte_perm(z[4], z[5], 0x5410), __byte_perm(z[6], z[7], 0x5410)));
+    // a half below kZMargin (<= 0x8000) borrows into its own top bit, which
+    // was clear: the usual SIMD test for a lane below a bound
+    if (sat || ((lo - kZMargin * 0x00010001u) & ~lo & 0x80008000u)) {
 #pragma unroll
         for (int k = 0; k < kChunk; k++)
-            qb[k] = code_bits_near(v[k], step, inv, half);
+            z[k] = zcode_of_bits(code_bits_near(v[k], step, inv, half));
     }
 }
 
@@ -193,6 +219,14 @@ __device__ __forceinline__ uint32_t pack8_bits(const uint32_t (&b)[kChunk])
     return (even & 0x0F0F0F0Fu) | ((odd << 4) & 0xF0F0F0F0u);
 }
 
+// pack8_bits for z-form codes: the same interleave from byte 2 of each.
+__device__ __forceinline__ uint32_t pack8_zcodes(const uint32_t (&z)[kChunk])
+{
+    const uint32_t even = __byte_perm(__byte_perm(z[0], z[2], 0x0062), __byte_perm(z[4], z[6], 0x0062), 0x5410);
+    const uint32_t odd = __byte_perm(__byte_perm(z[1], z[3], 0x0062), __byte_perm(z[5], z[7], 0x0062), 0x5410);
+    return (even & 0x0F0F0F0Fu) | ((odd << 4) & 0xF0F0F0F0u);
+}
+
 // ---- restoring codes --------------------------------------------------------
 // A packed word holds 8 two's-complement nibbles. Flipping bit 3 of each
 // nibble turns q in [-8, 7] into q + 8 in [0, 15]; placing that byte in the
@@ -214,6 +248,21 @@ __device__ __forceinline__ float code_at(const Unpacked &u, int k)
     const uint32_t src = (k & 1) ? u.odd : u.even;
     const uint32_t bits = __byte_perm(src, kRoundBits, 0x7650 + (k >> 1));
     return __fsub_rn(__uint_as_float(bits), kRoundPlus8);
+}
+
+// max(|a|, |b|, |c|): the three-input maximum of absolute values that sm_100
+// adds to PTX (max.abs.f32 with three sources); exact, like every maximum.
+__device__ __forceinline__ float max3_abs(float a, float b, float c)
+{
+    float r;
+    asm("max.abs.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+// Absolute maximum of one lane's 8 values (finite), as a tree.
+__device__ __forceinline__ float absmax8(const float (&v)[kChunk])
+{
+    return fmaxf(max3_abs(v[0], v[1], v[2]), max3_abs(v[3], v[4], max3_abs(v[5], v[6], v[7])));
 }
 
 // Absolute maximum over the 2^lanes_log2 consecutive lanes (8 elements each)

@@ -19,7 +19,8 @@
 // partials is at most 16 bytes per element (halved, quartered beyond).
 // ECHO_K2_CHUNKS is kernel 2's chunks of 8 elements per consumer thread per
 // tile, reduced for large P so that ECHO_K2_STAGES stages fit in shared
-// memory. ECHO_K3_TILE is kernel 3's bf16 tile (halved for binary32).
+// memory; a reduced tile then takes as many stages as fit, up to
+// ECHO_K2_MAX_STAGES. ECHO_K3_TILE is kernel 3's bf16 tile (halved for binary32).
 #ifndef ECHO_K1_TILE
 #define ECHO_K1_TILE 2048
 #endif
@@ -31,6 +32,9 @@
 #endif
 #ifndef ECHO_K2_CHUNKS
 #define ECHO_K2_CHUNKS 4
+#endif
+#ifndef ECHO_K2_MAX_STAGES
+#define ECHO_K2_MAX_STAGES 3
 #endif
 #ifndef ECHO_K3_TILE
 #define ECHO_K3_TILE 16384

@@ -151,9 +151,7 @@ __device__ __forceinline__ void k1_consume(const K1Args &a, const uint8_t *smem,
                                                      __fmul_rn(a.one_minus_lambda, sv[k])));
             }
             // max |v| as a tree (fmax is exact, so the order is free)
-            const float m01 = fmaxf(fabsf(v[0]), fabsf(v[1])), m23 = fmaxf(fabsf(v[2]), fabsf(v[3]));
-            const float m45 = fmaxf(fabsf(v[4]), fabsf(v[5])), m67 = fmaxf(fabsf(v[6]), fabsf(v[7]));
-            const float amax = group_absmax(fmaxf(fmaxf(m01, m23), fmaxf(m45, m67)), lanes_log2);
+            const float amax = group_absmax(absmax8(v), lanes_log2);
             uint32_t qb[kChunk];
             uint32_t scale; // scale byte, or binary16 pattern
             float st;       // the step q is restored with
@@ -171,7 +169,7 @@ __device__ __forceinline__ void k1_consume(const K1Args &a, const uint8_t *smem,
                 for (int k = 0; k < kChunk; k++)
                     qb[k] = code_bits(v[k], inv);
             }
-            const uint32_t word = pack8_bits(qb);
+            const uint32_t word = f16 ? pack8_zcodes(qb) : pack8_bits(qb); // binary16: z-form codes
             if (P == 1 && a.to_owners) {
                 // one process per rank: straight into the owner's receive block
                 const uint32_t owner = g / a.groups_per_seg;
@@ -206,7 +204,7 @@ __device__ __forceinline__ void k1_consume(const K1Args &a, const uint8_t *smem,
                 float e[kChunk];
 #pragma unroll
                 for (int k = 0; k < kChunk; k++)
-                    e[k] = __fmaf_rn(-code_value(qb[k]), st, v[k]);
+                    e[k] = __fmaf_rn(-code_value(f16 ? zcode_bits(qb[k]) : qb[k]), st, v[k]);
                 float4 *eo = reinterpret_cast<float4 *>(a.eps + static_cast<size_t>(r) * a.n) +
                              2 * static_cast<size_t>(chunk);
                 eo[0] = make_float4(e[0], e[1], e[2], e[3]);

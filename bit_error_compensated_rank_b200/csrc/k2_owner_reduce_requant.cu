@@ -66,11 +66,23 @@ constexpr int k2_chunks(int P, bool comp, bool f16)
     return c;
 }
 
+// Stages of the ring: ECHO_K2_STAGES, or, when the tile had to shrink, as
+// many of the smaller stages as fit, up to ECHO_K2_MAX_STAGES.
+constexpr int k2_stages(int P, bool comp, bool f16)
+{
+    const int c = k2_chunks(P, comp, f16);
+    int s = ECHO_K2_STAGES;
+    if (c < ECHO_K2_CHUNKS)
+        while (s < ECHO_K2_MAX_STAGES && (s + 1) * (k2_stage_bytes(P, comp, f16, c) + 16) <= ECHO_SMEM_BUDGET)
+            s++;
+    return s;
+}
+
 template <int P, bool COMP, bool F16>
 struct K2Shape {
     static constexpr int kChunks = k2_chunks(P, COMP, F16); // chunks per consumer thread
     static constexpr int kTile = kConsumers * kChunk * kChunks;
-    static constexpr int kStages = ECHO_K2_STAGES;
+    static constexpr int kStages = k2_stages(P, COMP, F16);
     static constexpr int kCodeBytes = kTile / 2;          // one rank's code tile
     static constexpr int kScaleBytes = kTile / kMinGroup * (F16 ? 2 : 1); // room for one rank's scale tile
     static constexpr int kStateOff = P * (kCodeBytes + kScaleBytes);
@@ -215,9 +227,7 @@ __global__ void __launch_bounds__(kThreads)
             }
 
             // Rounding #2 and the error it injects.
-            const float m01 = fmaxf(fabsf(S_[0]), fabsf(S_[1])), m23 = fmaxf(fabsf(S_[2]), fabsf(S_[3]));
-            const float m45 = fmaxf(fabsf(S_[4]), fabsf(S_[5])), m67 = fmaxf(fabsf(S_[6]), fabsf(S_[7]));
-            const float amax = group_absmax(fmaxf(fmaxf(m01, m23), fmaxf(m45, m67)), a.lanes_log2);
+            const float amax = group_absmax(absmax8(S_), a.lanes_log2);
             uint32_t qb[kChunk];
             float err[kChunk];
             uint32_t scale;
@@ -229,6 +239,7 @@ __global__ void __launch_bounds__(kThreads)
                 codes8_half(S_, st, inv, half, half_scale_saturates(amax), qb);
 #pragma unroll
                 for (int k = 0; k < kChunk; k++) {
+                    qb[k] = zcode_bits(qb[k]);
                     const float y = __fmul_rn(code_value(qb[k]), st); // exact
                     err[k] = __fsub_rn(S_[k], a.bf16 ? round_bf16(y) : y);
                 }

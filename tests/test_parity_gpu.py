@@ -375,3 +375,20 @@ def test_host_end_to_end_fp32_backward(oracle):
             assert not ff.any() and not fs.any()
     finally:
         h.close()
+
+
+@pytest.mark.parametrize("variant", [0, 4], ids=["default", "fp16_scale"])
+@pytest.mark.parametrize("P", [11, 12, 13, 16])
+def test_many_ranks_full_tiles(oracle, P, variant):
+    """From P = 11 on, kernel 2's stages no longer fit two full tiles, so the
+    tile halves and the ring deepens to three stages. About 4 Mi elements per
+    rank give full-size tiles, several turns of the ring per CTA and a ragged
+    last tile; compared in full over two calls, the second corrected by the
+    state the first left."""
+    n = P * 32 * ((1 << 22) // (P * 32) + 3)
+    fc = FullCompare(oracle, P, n, "bf16", variant=variant)
+    try:
+        for k in range(2):
+            fc.call(outlier_gaussian(P, n, seed=60 + P, call=k), phase=0)
+    finally:
+        fc.close()
