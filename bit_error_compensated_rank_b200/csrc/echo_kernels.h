@@ -48,7 +48,9 @@
 // Shared memory one CTA may use (the B200 limit is 227 KB), and kernel 1's
 // budget per CTA so that two CTAs share an SM.
 #define ECHO_SMEM_BUDGET (225 * 1024)
+#ifndef ECHO_K1_CTA_BUDGET
 #define ECHO_K1_CTA_BUDGET (100 * 1024)
+#endif
 
 namespace echo {
 

@@ -68,6 +68,15 @@ def _edge(kind, P, n, G):
         k = g.integers(-7, 7, (P, n)) + 0.5
         k[:, ::G] = 7
         x = k * s
+    elif kind == "near_ties":    # up to 6 binary32 ulps either side of the midpoints (k + 1/2) * s
+        h = g.integers(0x2000, 0x5000, (P, n // G)).astype(np.uint16)
+        s = np.repeat(h.view(np.float16).astype(np.float64), G, axis=1)
+        k = g.integers(-7, 7, (P, n)) + 0.5
+        k[:, ::G] = 7
+        x = (k * s).astype(np.float32)
+        off = g.integers(-6, 7, (P, n)).astype(np.int32)
+        off[:, ::G] = 0  # keeps each group's maximum at exactly 7*s
+        x = (x.view(np.int32) + off).view(np.float32)
     elif kind == "boundary":     # max|v| exactly 7*s and one ulp past it
         h = g.integers(0x0400, 0x7000, (P, n // G)).astype(np.uint16)
         s = np.repeat(h.view(np.float16).astype(np.float64), G, axis=1)
@@ -82,7 +91,7 @@ def _edge(kind, P, n, G):
     return np.asarray(x, np.float64).astype(np.float32)
 
 
-@pytest.mark.parametrize("kind", ["saturating", "tiny", "subnormal", "ties", "boundary", "zeros"])
+@pytest.mark.parametrize("kind", ["saturating", "tiny", "subnormal", "ties", "near_ties", "boundary", "zeros"])
 @pytest.mark.parametrize("dtype", ["bf16", "fp32"])
 def test_fp16_scale_edge_values(oracle, kind, dtype):
     P, G = 4, 32
