@@ -265,6 +265,17 @@ __device__ __forceinline__ float absmax8(const float (&v)[kChunk])
     return fmaxf(max3_abs(v[0], v[1], v[2]), max3_abs(v[3], v[4], max3_abs(v[5], v[6], v[7])));
 }
 
+// Codes of elements 2j and 2j+1 as a pair of floats, by one packed
+// subtraction (sm_100's f32x2 forms round each component exactly as the
+// scalar __fadd_rn, __fmul_rn and __fmaf_rn do); j is a constant after
+// unrolling.
+__device__ __forceinline__ float2 code_pair(const Unpacked &u, int j)
+{
+    const float a = __uint_as_float(__byte_perm(u.even, kRoundBits, 0x7650 + j));
+    const float b = __uint_as_float(__byte_perm(u.odd, kRoundBits, 0x7650 + j));
+    return __fadd2_rn(make_float2(a, b), make_float2(-kRoundPlus8, -kRoundPlus8));
+}
+
 // Absolute maximum over the 2^lanes_log2 consecutive lanes (8 elements each)
 // that form a group. Every lane of the warp calls it with the same
 // lanes_log2.

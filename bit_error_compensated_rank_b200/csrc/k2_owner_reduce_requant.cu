@@ -99,6 +99,12 @@ __global__ void __launch_bounds__(kThreads)
 {
     using Sh = K2Shape<P, COMP, F16>;
     constexpr uint32_t kScaleLog2 = F16 ? 1u : 0u; // log2 of the bytes per scale
+    // From P = 11 on the kernel issues more instructions than its bytes
+    // hide, so the restore-and-add and the codes of rounding #2 use sm_100's
+    // packed f32x2 FMA (two elements per instruction, each rounded as the
+    // scalar __fmaf_rn). At P <= 8 the scalar form measured faster. No
+    // product feeds a separate addition here, so nothing can be contracted.
+    constexpr bool kPacked = P >= 11;
     constexpr int S = Sh::kStages;
     extern __shared__ __align__(128) uint8_t smem[];
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + S * Sh::kStageBytes);
@@ -215,9 +221,19 @@ __global__ void __launch_bounds__(kThreads)
                 const float st = F16 ? half_step(reinterpret_cast<const uint16_t *>(srow)[c >> a.lanes_log2])
                                      : step_of(srow[c >> a.lanes_log2]);
                 const Unpacked u = unpack8(w);
+                if (kPacked) {
+                    const float2 st2 = make_float2(st, st);
 #pragma unroll
-                for (int k = 0; k < kChunk; k++)
-                    S_[k] = __fmaf_rn(code_at(u, k), st, S_[k]);
+                    for (int j = 0; j < kChunk / 2; j++) { // two elements per packed FMA
+                        const float2 acc =
+                            __ffma2_rn(code_pair(u, j), st2, make_float2(S_[2 * j], S_[2 * j + 1]));
+                        S_[2 * j] = acc.x, S_[2 * j + 1] = acc.y;
+                    }
+                } else {
+#pragma unroll
+                    for (int k = 0; k < kChunk; k++)
+                        S_[k] = __fmaf_rn(code_at(u, k), st, S_[k]);
+                }
             }
             if (SUM) { // variant: the correction enters the owner's sum, after the P ranks
 #pragma unroll
@@ -247,10 +263,23 @@ __global__ void __launch_bounds__(kThreads)
                 scale = scale_byte(amax);
                 const float inv = inv_step_of(scale);
                 const float st = step_of(scale);
+                if (kPacked) {
 #pragma unroll
-                for (int k = 0; k < kChunk; k++) {
-                    qb[k] = code_bits(S_[k], inv);
-                    err[k] = __fmaf_rn(-code_value(qb[k]), st, S_[k]); // S - Q*2^E, exact
+                    for (int j = 0; j < kChunk / 2; j++) {
+                        const float2 S2 = make_float2(S_[2 * j], S_[2 * j + 1]);
+                        const float2 t = __ffma2_rn(S2, make_float2(inv, inv), make_float2(kRound, kRound));
+                        qb[2 * j] = __float_as_uint(t.x), qb[2 * j + 1] = __float_as_uint(t.y);
+                        // S - Q*2^E, exact: Q = t - kRound, then Q*(-2^E) + S
+                        const float2 e2 =
+                            __ffma2_rn(__fadd2_rn(t, make_float2(-kRound, -kRound)), make_float2(-st, -st), S2);
+                        err[2 * j] = e2.x, err[2 * j + 1] = e2.y;
+                    }
+                } else {
+#pragma unroll
+                    for (int k = 0; k < kChunk; k++) {
+                        qb[k] = code_bits(S_[k], inv);
+                        err[k] = __fmaf_rn(-code_value(qb[k]), st, S_[k]); // S - Q*2^E, exact
+                    }
                 }
             }
 
@@ -286,6 +315,10 @@ __global__ void __launch_bounds__(kThreads)
                     }
                 }
                 if (COMP) {
+                    // Scalar on purpose: packed f32x2 multiplies followed by a
+                    // packed add did not match the oracle on B200 (one element
+                    // of the slow estimate in millions, as if fused into one
+                    // FMA), so the estimates keep the scalar roundings.
 #pragma unroll
                     for (int k = 0; k < kChunk; k++) {
                         fv[k] = __fadd_rn(__fmul_rn(a.beta_f, fv[k]), __fmul_rn(a.one_minus_beta_f, err[k]));
