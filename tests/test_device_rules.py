@@ -1,0 +1,130 @@
+"""The binary16-scale codec's device shortcuts, modelled on the CPU and held
+against the oracle's rounding (no GPU needed).
+
+The kernels do not compute a binary16 scale or code the way the oracle does
+(bisection over binary16 values, exact midpoint comparison in binary64).
+They take shortcuts whose exactness rests on an argument, written beside
+them in ``echo_codec.cuh``:
+
+* scale: u = A * RU(1/7), rounded up, then rounded up again to binary16, is
+  never below the answer and at most one binary16 step above it, so one exact
+  test of the step below settles it;
+* code: z = RN(v * inv + kZ) keeps the code in byte 2 and a 16-bit fraction
+  below it; when that fraction is at least kZMargin units of 2^-16 from a
+  midpoint, the code is the exact nearest one, whatever error up to 2^-23
+  the reciprocal estimate inv carries.
+
+This test restates both in binary64 and long double, with the constants read
+from the header, and checks them against the oracle on groups with ties,
+near-ties, bf16 partials, subnormals and wide ranges. It reads the header as
+text only; nothing of the CUDA path runs.
+"""
+from __future__ import annotations
+
+import os
+import re
+
+import numpy as np
+
+from bit_error_compensated_rank_b200.workloads import bf16_to_f32, outlier_gaussian
+from oracle.oracle import FP16_SCALE
+from pins import _many_random_groups, _quantise_rows_with_oracle
+
+CODEC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                     "bit_error_compensated_rank_b200", "csrc", "echo_codec.cuh")
+G = 32
+
+
+def _constants():
+    text = open(CODEC).read()
+    kz = float(re.search(r"constexpr float kZ = ([0-9.]+)f;", text).group(1))
+    margin = int(re.search(r"constexpr uint32_t kZMargin = (\d+);", text).group(1))
+    seventh = int(re.search(r"__fmul_ru\(A, __uint_as_float\((0x[0-9A-Fa-f]+)u\)\)", text).group(1), 16)
+    return np.float32(kz), margin, np.uint32(seventh).view(np.float32)
+
+
+def _ru32(x: np.ndarray) -> np.ndarray:
+    """Exact binary64 values rounded up to binary32."""
+    f = x.astype(np.float32)
+    lo = f.astype(np.float64) < x
+    f[lo] = np.nextafter(f[lo], np.float32(np.inf))
+    return f
+
+
+def _ru16(x: np.ndarray) -> np.ndarray:
+    """binary32 values rounded up to binary16 (beyond 65504: infinity)."""
+    with np.errstate(over="ignore"):
+        h = x.astype(np.float16)
+        lo = h.astype(np.float64) < x.astype(np.float64)
+        h[lo] = np.nextafter(h[lo], np.float16(np.inf))
+    return h
+
+
+def _device_scale(A: np.ndarray, seventh: np.float32) -> np.ndarray:
+    u = _ru32(A.astype(np.float64) * np.float64(seventh))  # the product is exact in binary64
+    h = np.minimum(_ru16(u).view(np.uint16).astype(np.int64), 0x7BFF)
+    below = np.maximum(h - 1, 0).astype(np.uint16).view(np.float16).astype(np.float64)
+    down = (h > 1) & (7.0 * below >= A.astype(np.float64))
+    return h - down
+
+
+def _device_codes(v: np.ndarray, h: np.ndarray, kz: np.float32, margin: int, eta: float):
+    """z-form codes of rows v under binary16 steps h, with the reciprocal off
+    by the relative error eta; returns (codes, lane flagged for the exact path)."""
+    s = h.astype(np.uint16).view(np.float16).astype(np.float32)
+    inv = np.where(s > 0, np.float32(1) / np.where(s > 0, s, 1), 0).astype(np.float64) * (1 + eta)
+    z = (v.astype(np.longdouble) * inv[:, None].astype(np.longdouble) + np.longdouble(kz)).astype(np.float32)
+    bits = z.view(np.uint32).astype(np.int64)
+    codes = (bits >> 16) - 0x4340
+    flagged = ((bits & 0xFFFF) < margin).reshape(v.shape[0], -1, 8).any(axis=2)  # per lane of 8
+    return codes, np.repeat(flagged, 8, axis=1)
+
+
+def _rows():
+    mixed = _many_random_groups(1 << 15, G, seed=9)
+    mixed = np.clip(mixed, -4e5, 4e5).astype(np.float32)  # below saturation (7 * 65504)
+    partials = bf16_to_f32(outlier_gaussian(1, (1 << 15) * G, seed=3, call=0)).reshape(-1, G)
+    g = np.random.default_rng(11)  # near ties: a few binary32 ulps around (k + 1/2) * s
+    hs = g.integers(0x0400, 0x7000, (1 << 14, 1)).astype(np.uint16).view(np.float16).astype(np.float64)
+    k = g.integers(-7, 7, (1 << 14, G)) + 0.5
+    k[:, 0] = 7
+    near = (k * hs).astype(np.float32)
+    off = g.integers(-3, 4, near.shape).astype(np.int32)
+    off[:, 0] = 0
+    near = (near.view(np.int32) + off).view(np.float32)
+    return np.concatenate([mixed, partials, near]).astype(np.float32)
+
+
+def test_binary16_scale_one_test_rule(oracle):
+    _, _, seventh = _constants()
+    x = _rows()
+    h_oracle, _ = _quantise_rows_with_oracle(oracle, x, G, FP16_SCALE)
+    A = np.abs(x).max(axis=1)
+    assert np.array_equal(_device_scale(A, seventh), h_oracle)
+    # every boundary 7*s of the rule and a few ulps either side
+    s = np.arange(1, 0x7C00, dtype=np.uint16).view(np.float16).astype(np.float64)
+    b = (7.0 * s).astype(np.float32)
+    for d in range(-2, 3):
+        Ab = (b.view(np.int32) + d).view(np.float32)
+        rows = np.zeros((Ab.size, G), np.float32)
+        rows[:, 0] = Ab
+        h_b, _ = _quantise_rows_with_oracle(oracle, rows, G, FP16_SCALE)
+        assert np.array_equal(_device_scale(Ab, seventh), h_b), d
+
+
+def test_binary16_zform_codes_exact_when_not_flagged(oracle):
+    kz, margin, _ = _constants()
+    assert kz.view(np.uint32) == 0x43408002 and margin >= 1
+    x = _rows()
+    h, q = _quantise_rows_with_oracle(oracle, x, G, FP16_SCALE)
+    for eta in (0.0, 2.0 ** -23, -(2.0 ** -23)):
+        codes, flagged = _device_codes(x, h, kz, margin, eta)
+        wrong = codes != q
+        assert not (wrong & ~flagged).any(), (eta, np.argwhere(wrong & ~flagged)[:4])
+        # exact ties are flagged, so the exact path sees every one of them
+        s = h.astype(np.uint16).view(np.float16).astype(np.float64)
+        ratio = x.astype(np.float64) / np.where(s > 0, s, 1)[:, None]
+        ties = (s[:, None] > 0) & (ratio - np.floor(ratio) == 0.5)
+        assert ties.any() and flagged[ties].all()
+    # bf16 partials hold exact ties often enough to matter for the kernel's cost
+    assert ties.mean() > 1e-4
