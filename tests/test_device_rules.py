@@ -1,10 +1,13 @@
-"""The binary16-scale codec's device shortcuts, modelled on the CPU and held
-against the oracle's rounding (no GPU needed).
+"""The codec's device shortcuts, modelled on the CPU and held against the
+oracle's rounding (no GPU needed).
 
-The kernels do not compute a binary16 scale or code the way the oracle does
-(bisection over binary16 values, exact midpoint comparison in binary64).
-They take shortcuts whose exactness rests on an argument, written beside
-them in ``echo_codec.cuh``:
+The kernels do not compute a scale or a code the way the oracle does (a
+search over e or over binary16 values, rounding in binary64). They take
+shortcuts whose exactness rests on an argument, written beside them in
+``echo_codec.cuh``:
+
+* power-of-two scale: the byte is read from the exponent and mantissa fields
+  of the maximum, and the code is one fused fma(v, 2^-e, 1.5 * 2^23);
 
 * scale: u = A * RU(1/7), rounded up, then rounded up again to binary16, is
   never below the answer and at most one binary16 step above it, so one exact
@@ -14,7 +17,7 @@ them in ``echo_codec.cuh``:
   midpoint, the code is the exact nearest one, whatever error up to 2^-23
   the reciprocal estimate inv carries.
 
-This test restates both in binary64 and long double, with the constants read
+This test restates them in binary64 and long double, with the constants read
 from the header, and checks them against the oracle on groups with ties,
 near-ties, bf16 partials, subnormals and wide ranges. It reads the header as
 text only; nothing of the CUDA path runs.
@@ -128,3 +131,34 @@ def test_binary16_zform_codes_exact_when_not_flagged(oracle):
         assert ties.any() and flagged[ties].all()
     # bf16 partials hold exact ties often enough to matter for the kernel's cost
     assert ties.mean() > 1e-4
+
+
+def _device_scale_byte(A: np.ndarray) -> np.ndarray:
+    """The kernels' closed form: byte = max(0, E - 2 + [M > 0x600000])."""
+    u = A.astype(np.float32).view(np.uint32).astype(np.int64)
+    b = (u >> 23) - 2 + ((u & 0x7FFFFF) > 0x600000)
+    return np.maximum(b, 0)
+
+
+def test_power_of_two_scale_closed_form_and_fused_codes(oracle):
+    """Default format: the scale byte read from the bits of the maximum, and
+    the code from one fused fma(v, 2^-e, 1.5 * 2^23), against the oracle's
+    search over e and its binary64 rounding."""
+    x = _rows()
+    # every exponent field up to the oracle's domain (|x| < 2^120), mantissas
+    # around the 7/4 boundary
+    g = np.random.default_rng(12)
+    E = np.repeat(np.arange(0, 246), 16)
+    M = np.clip(0x600000 + g.integers(-3, 4, E.size), 0, 0x7FFFFF)
+    A = ((E << 23) | M).astype(np.uint32).view(np.float32)
+    edge = np.zeros((A.size, G), np.float32)
+    edge[:, 0] = A
+    edge[:, 1:] = A[:, None] * g.uniform(-1, 1, (A.size, G - 1)).astype(np.float32)
+    x = np.concatenate([x, edge])
+    b_oracle, q_oracle = _quantise_rows_with_oracle(oracle, x, G, 0)
+    b = _device_scale_byte(np.abs(x).max(axis=1))
+    assert np.array_equal(b, b_oracle)
+    inv = np.ldexp(1.0, 127 - b)  # 2^-e, a normal binary32 for every byte the rule gives
+    t = (x.astype(np.longdouble) * inv[:, None].astype(np.longdouble) + np.longdouble(1.5 * 2 ** 23)).astype(np.float32)
+    codes = t.view(np.uint32).astype(np.int64) - 0x4B400000
+    assert np.array_equal(codes, q_oracle)
