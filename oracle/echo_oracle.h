@@ -35,7 +35,11 @@
  *   - the captured error is err = S - Y with Y the requantised total;
  *   - f <- beta_f*f + (1-beta_f)*err, s <- beta_s*s + (1-beta_s)*err and
  *     c = lambda*f + (1-lambda)*s, every product and sum rounded to binary32
- *     on its own (no fused multiply-add), subnormals kept.
+ *     on its own (no fused multiply-add), 1-lambda and 1-beta themselves
+ *     formed in binary32, subnormals kept; with sender feedback the owner's
+ *     value is (x + eps) + c, rounded after each add. The tests pin this order
+ *     with hand-worked cases where a fused or regrouped form gives another
+ *     binary32 value (tests/golden/rounding_order_p3_g32.json).
  *
  * Status codes: 0 on success, -1 on an invalid argument or a non-finite
  * value, -2 when a value leaves the domain (output not exactly

@@ -203,6 +203,118 @@ def pin_hand_example(orc):
     _check_hand_fixture(orc, "hand_example_p2_g32.json", 0)
 
 
+def _dyadic(expr: str) -> Fraction:
+    """``n*2^k``, ``n`` or ``p/q`` as an exact rational."""
+    expr = expr.strip()
+    if "*2^" in expr:
+        coef, _, power = expr.partition("*2^")
+        return Fraction(int(coef)) * Fraction(2) ** int(power)
+    return Fraction(expr)
+
+
+def _assert_nearest_binary32(exact: Fraction, rounded: Fraction, what: str):
+    """``rounded`` is a binary32 value and no binary32 value lies nearer to
+    ``exact``; on a tie the last significand bit of ``rounded`` is 0."""
+    r = F32(float(rounded))
+    assert Fraction(float(r)) == rounded, f"{what}: {rounded} is not a binary32 value"
+    d = abs(exact - rounded)
+    for nb in (np.nextafter(r, F32(-np.inf)), np.nextafter(r, F32(np.inf))):
+        dn = abs(exact - Fraction(float(nb)))
+        assert d <= dn, f"{what}: {float(nb)!r} is nearer to {exact} than {rounded}"
+        if d == dn and d != 0:
+            assert int(np.array(r).view(np.uint32)) & 1 == 0, f"{what}: tie not to even"
+
+
+def _check_derivation(steps, vals, what):
+    """Re-check each written step: its exact result from its operands, and
+    its binary32 rounding. Adds every step's rounded result to ``vals``."""
+    for st in steps:
+        a = [vals[t] if t in vals else _dyadic(t) for t in st["args"]]
+        exact = {"mul": lambda: a[0] * a[1], "add": lambda: a[0] + a[1],
+                 "sub": lambda: a[0] - a[1], "fma": lambda: a[0] * a[1] + a[2]}[st["op"]]()
+        assert exact == _dyadic(st["exact"]), (what, st)
+        _assert_nearest_binary32(exact, _dyadic(st["rounded"]), f"{what}/{st['name']}")
+        vals[st["name"]] = _dyadic(st["rounded"])
+
+
+def pin_rounding_order(orc):
+    """Hand-worked operation order (fixture ``rounding_order_p3_g32.json``):
+    the correction c = RN(RN(lambda f) + RN((1-lambda) s)), each estimate
+    RN(RN(beta z) + RN((1-beta) err)), and with sender feedback the owner's
+    RN(RN(x + eps) + c), each product and sum rounded on its own. The probes
+    are chosen so that fusing a product into the add, or reassociating the
+    adds, changes the binary32 result; the fixture lists each such value. The
+    pin re-checks every written step of the derivation (exact rational,
+    nearest binary32), then requires the oracle's c, err, f, s, output and
+    rank 0's new sender error at each probe, for bf16 and binary32 partials,
+    under dyadic coefficients (5/8, 3/4, 7/8) and the binary32 values of
+    0.25, 0.3, 0.95."""
+    fx = _load("rounding_order_p3_g32.json")
+    P, G = 3, 32
+    m = P * G
+    for case in fx["cases"]:
+        prm = {k: _dyadic(v) for k, v in case["params"].items()}
+        params = Params(lam=float(prm["lambda"]), beta_fast=float(prm["beta_fast"]),
+                        beta_slow=float(prm["beta_slow"]))
+        for k, v in prm.items():  # the coefficients themselves are binary32 values
+            assert Fraction(float(F32(float(v)))) == v, (case["name"], k)
+        variant = SENDER_EF if case["variant"] == "SENDER_EF" else 0
+        x32 = np.zeros((P, m), F32)
+        x32[0, 2] = 7.0
+        x32[2, 0] = 12.0
+        f0 = np.zeros(m, F32)
+        s0 = np.zeros(m, F32)
+        eps0 = np.zeros((P, m), F32)
+        for p in case["probes"]:
+            e = p["element"]
+            assert 3 <= e < G
+            x32[0, e] = 1.0
+            x32[1, e] = 7.0 * 2.0 ** -10
+            f0[e] = float(_dyadic(p["f"]))
+            s0[e] = float(_dyadic(p["s"]))
+            if "eps_rank0" in p:
+                eps0[0, e] = float(_dyadic(p["eps_rank0"]))
+        for p in case["probes"]:
+            vals = {"lambda": prm["lambda"], "beta_fast": prm["beta_fast"],
+                    "beta_slow": prm["beta_slow"], "f": _dyadic(p["f"]), "s": _dyadic(p["s"]),
+                    "err": Fraction(-1017, 1024), "x": Fraction(1)}
+            if "eps_rank0" in p:
+                vals["eps"] = _dyadic(p["eps_rank0"])
+            what = f"{case['name']}/{p['element']}"
+            _check_derivation(p["steps"], vals, what)
+            want = {k: _dyadic(v) for k, v in p["expect"].items()}
+            assert want["err"] == vals["err"] and want["c"] == vals["c"]
+            if "f" in want:
+                assert want["f"] == vals["f_next"] and want["s"] == vals["s_next"]
+            if "eps_rank0" in want:
+                assert want["eps_rank0"] == vals["eps_next"]
+            for alt in p["alternatives"]:
+                avals = dict(vals)
+                _check_derivation(alt["steps"], avals, f"{what}/{alt['mutant']}")
+                assert _dyadic(alt["value"]) == avals[alt["steps"][-1]["name"]]
+                key = "eps_rank0" if alt["of"] == "eps" else alt["of"]
+                assert _dyadic(alt["value"]) != want[key], (what, alt["mutant"])
+        for x in (x32, bf16_bits(x32)):
+            f, s, eps = f0.copy(), s0.copy(), eps0.copy()
+            res = orc.allreduce(x, f, s, params, want_diag=True, variant=variant,
+                                eps=eps if variant else None)
+            assert res["scales1"][:, 0].tolist() == [127, 117, 128]
+            assert res["qscales"].tolist() == [128, 0, 0]
+            q = _unpack_ref(res["qcodes"][:G // 2])
+            assert q[0] == 6 and q[2] == 4
+            for p in case["probes"]:
+                e = p["element"]
+                want = {k: _dyadic(v) for k, v in p["expect"].items()}
+                assert _unpack_ref(res["codes1"][0][:G // 2])[e] == 1
+                assert _unpack_ref(res["codes1"][1][:G // 2])[e] == 7
+                assert q[e] == 1
+                have = {"c": res["c"][e], "err": res["err"][e], "out": _values(res["out"])[e],
+                        "f": f[e], "s": s[e], "eps_rank0": eps[0, e]}
+                for key, w in want.items():
+                    assert Fraction(float(have[key])) == w, (case["name"], e, key,
+                                                             float(have[key]), float(w))
+
+
 def _grid_partials(P, ngroups, G, seed):
     """Partials that rounding #1 reproduces exactly: each group is k*2^e_rg,
     |k| <= 7, with one |k| in 4..7 so that e_rg is the group's scale. Exponents
@@ -808,6 +920,7 @@ ALL_PINS = [
     pin_roundtrip_bound,
     pin_pack_layout,
     pin_hand_example,
+    pin_rounding_order,
     pin_exact_sums_on_grid,
     pin_p2_enumeration,
     pin_rank_order,

@@ -76,6 +76,41 @@ MUTANTS = [
     ("correction_not_added",
      "v[k] = u + c[i];",
      "v[k] = u;"),
+    # operation order: a product fused into the following add, or the adds
+    # regrouped (each is the same real-number expression, rounded differently)
+    ("combine_fma",
+     "c[i] = from_fast + from_slow;",
+     "c[i] = fmaf(lambda, f[i], from_slow);"),
+    ("combine_fma_slow",
+     "c[i] = from_fast + from_slow;",
+     "c[i] = fmaf(one_minus_lambda, s[i], from_fast);"),
+    ("combine_increment",
+     "c[i] = from_fast + from_slow;",
+     "c[i] = s[i] + lambda * (f[i] - s[i]);"),
+    ("ema_fast_fma",
+     "f[i] = f_keep + f_new;",
+     "f[i] = fmaf(beta_f, f[i], f_new);"),
+    ("ema_fast_fma_new",
+     "f[i] = f_keep + f_new;",
+     "f[i] = fmaf(one_minus_beta_f, err, f_keep);"),
+    ("ema_fast_increment",
+     "f[i] = f_keep + f_new;",
+     "f[i] = f[i] + one_minus_beta_f * (err - f[i]);"),
+    ("ema_slow_fma",
+     "s[i] = s_keep + s_new;",
+     "s[i] = fmaf(beta_s, s[i], s_new);"),
+    ("ema_slow_fma_new",
+     "s[i] = s_keep + s_new;",
+     "s[i] = fmaf(one_minus_beta_s, err, s_keep);"),
+    ("ema_slow_increment",
+     "s[i] = s_keep + s_new;",
+     "s[i] = s[i] + one_minus_beta_s * (err - s[i]);"),
+    ("sender_reassoc",
+     "v[k] = u + c[i];",
+     "v[k] = sender_ef ? xi + (eps[(size_t)r * m + i] + c[i]) : u + c[i];"),
+    ("sender_correction_first",
+     "v[k] = u + c[i];",
+     "v[k] = sender_ef ? (xi + c[i]) + eps[(size_t)r * m + i] : u + c[i];"),
     # variants
     ("sender_error_not_kept",
      "eps[(size_t)r * m + i] = v[k] - restored;",
