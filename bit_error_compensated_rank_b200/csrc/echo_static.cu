@@ -8,15 +8,20 @@
 // them: the caller passes its rank buffers and the compensator state, and the
 // wire buffers the three kernels exchange live in a fixed scratch array
 // compiled into the library (ECHO_STATIC_SCRATCH_BYTES, 32 MiB, held on every
-// GPU that loads the library until the process exits).
+// GPU where it has been set up until the process exits).
 //
 // In host code the array's name is only a host-side stand-in, not a device
 // address, so the device address is looked up with cudaGetSymbolAddress, once
-// per device, on the first call made with that device current. That first
-// call should come before any stream capture. Every call shares the one
-// array and leaves its contents behind; the device status word at its start
-// is cleared at the start of each call. Calls whose work overlaps on the GPU
-// (two streams, or two host threads, at once) race on the array.
+// per device, by the first call of echo_allreduce_static or
+// echo_static_status made with that device current. Under CUDA's lazy module
+// loading that lookup is also when the 32 MiB are taken from the device, so a
+// caller that reserves the rest of HBM for its own pool, or captures streams
+// into graphs, makes one such call first. The set-up also zeroes the device
+// status word at the start of the array. The kernels only ever OR bits into
+// that word (bounded waits that ran out), so it keeps them across calls until
+// echo_static_status clears it. Every call shares the one array and leaves
+// its contents behind; calls whose work overlaps on the GPU (two streams, or
+// two host threads, at once) race on the array.
 #include "echo.h"
 #include "echo_bulk.cuh"
 #include "echo_kernels.h"
@@ -25,6 +30,8 @@
 
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
+#include <cstring>
 #include <mutex>
 
 namespace {
@@ -32,7 +39,9 @@ namespace {
 static __device__ __align__(256) uint8_t g_static_scratch[ECHO_STATIC_SCRATCH_BYTES];
 
 constexpr int kMaxDevices = 64;
-constexpr long long kWaitCycles = 1LL << 31; // about a second at B200 clocks
+constexpr size_t kMaxN = size_t(1) << 34;          // as echo_create: chunk indices stay 32-bit
+constexpr long long kWaitCycles = 1LL << 31;      // about a second at B200 clocks
+constexpr long long kStallWaitCycles = 1LL << 20; // the injected stall (tests)
 
 std::mutex g_addr_mu;
 uint8_t *g_addr[kMaxDevices] = {}; // device address of the array, per device
@@ -73,7 +82,64 @@ int check_device_pointer(const void *p, int device, const char *what, int index)
     return ECHO_OK;
 }
 
+// Test hook shared with the handle path: ECHO_FAULT=stall launches the
+// kernels with no loads issued and a short wait bound, so every CTA's first
+// wait runs out and records its bit in the status word.
+bool stall_injected()
+{
+    const char *e = std::getenv("ECHO_FAULT");
+    return e && std::strcmp(e, "stall") == 0;
+}
+
+// The array's device address on the current device. The first lookup on a
+// device also zeroes the status word (synchronously).
+int static_base(uint8_t **base)
+{
+    int device = -1;
+    cudaError_t e = cudaGetDevice(&device);
+    if (e != cudaSuccess)
+        return fail(ECHO_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    if (device < 0 || device >= kMaxDevices)
+        return fail(ECHO_ERR_UNSUPPORTED, "device %d is beyond the %d devices this entry point tracks", device,
+                    kMaxDevices);
+    std::lock_guard<std::mutex> lock(g_addr_mu);
+    if (!g_addr[device]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_static_scratch);
+        if (e != cudaSuccess)
+            return fail(ECHO_ERR_CUDA, "cudaGetSymbolAddress of the static scratch: %s", cudaGetErrorString(e));
+        e = cudaMemset(p, 0, sizeof(int));
+        if (e == cudaSuccess)
+            e = cudaDeviceSynchronize();
+        if (e != cudaSuccess)
+            return fail(ECHO_ERR_CUDA, "clearing the static status word: %s", cudaGetErrorString(e));
+        g_addr[device] = static_cast<uint8_t *>(p);
+    }
+    *base = g_addr[device];
+    return ECHO_OK;
+}
+
 } // namespace
+
+extern "C" int echo_static_status(int *status, int clear)
+{
+    if (!status)
+        return fail(ECHO_ERR_INVALID, "status is NULL");
+    uint8_t *base = nullptr;
+    int rc = static_base(&base);
+    if (rc != ECHO_OK)
+        return rc;
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e == cudaSuccess)
+        e = cudaMemcpy(status, base, sizeof(int), cudaMemcpyDeviceToHost);
+    if (e == cudaSuccess && clear)
+        e = cudaMemset(base, 0, sizeof(int));
+    if (e == cudaSuccess && clear)
+        e = cudaDeviceSynchronize();
+    if (e != cudaSuccess)
+        return fail(ECHO_ERR_CUDA, "echo_static_status: %s", cudaGetErrorString(e));
+    return ECHO_OK;
+}
 
 extern "C" int echo_allreduce_static(int P, size_t n, int dtype, void *const rank_ptrs[], float *f, float *s,
                                      float beta_fast, float beta_slow, float lambda, int enable, void *stream)
@@ -85,6 +151,9 @@ extern "C" int echo_allreduce_static(int P, size_t n, int dtype, void *const ran
         return fail(ECHO_ERR_INVALID, "unknown dtype %d", dtype);
     if (n == 0 || n % (static_cast<size_t>(P) * ECHO_GROUP) != 0)
         return fail(ECHO_ERR_INVALID, "n = %zu must be a positive multiple of P*32 = %d", n, P * ECHO_GROUP);
+    // Before any size arithmetic, so that nothing below can wrap around.
+    if (n > kMaxN)
+        return fail(ECHO_ERR_UNSUPPORTED, "n = %zu exceeds the supported maximum %zu", n, kMaxN);
     if (!(beta_fast >= 0.f && beta_fast < 1.f) || !(beta_slow >= 0.f && beta_slow < 1.f) ||
         !(lambda >= 0.f && lambda <= 1.f) || (enable != 0 && enable != 1))
         return fail(ECHO_ERR_INVALID, "parameters out of range (beta in [0,1), lambda in [0,1], enable 0/1)");
@@ -103,9 +172,6 @@ extern "C" int echo_allreduce_static(int P, size_t n, int dtype, void *const ran
     cudaError_t e = cudaGetDevice(&device);
     if (e != cudaSuccess)
         return fail(ECHO_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
-    if (device < 0 || device >= kMaxDevices)
-        return fail(ECHO_ERR_UNSUPPORTED, "device %d is beyond the %d devices this entry point tracks", device,
-                    kMaxDevices);
     if (!rank_ptrs)
         return fail(ECHO_ERR_INVALID, "rank pointer array is NULL");
     const size_t bytes = n * (dtype == ECHO_BF16 ? 2 : 4);
@@ -130,18 +196,9 @@ extern "C" int echo_allreduce_static(int P, size_t n, int dtype, void *const ran
     }
 
     // ---- the array's device address on this device (looked up once) ----
-    uint8_t *base;
-    {
-        std::lock_guard<std::mutex> lock(g_addr_mu);
-        if (!g_addr[device]) {
-            void *p = nullptr;
-            e = cudaGetSymbolAddress(&p, g_static_scratch);
-            if (e != cudaSuccess)
-                return fail(ECHO_ERR_CUDA, "cudaGetSymbolAddress of the static scratch: %s", cudaGetErrorString(e));
-            g_addr[device] = static_cast<uint8_t *>(p);
-        }
-        base = g_addr[device];
-    }
+    uint8_t *base = nullptr;
+    if ((rc = static_base(&base)) != ECHO_OK)
+        return rc;
 
     // ---- the three kernels, as echo_allreduce enqueues them ----
     cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -149,7 +206,8 @@ extern "C" int echo_allreduce_static(int P, size_t n, int dtype, void *const ran
     uint8_t *codes1 = base + off_codes1, *scales1 = base + off_scales1;
     uint8_t *qcodes = base + off_qcodes, *qscales = base + off_qscales;
     const uint32_t chunks = static_cast<uint32_t>(n / echo::kChunk);
-    const echo::PipeCtl ctl{status, kWaitCycles, false};
+    const bool stall = stall_injected();
+    const echo::PipeCtl ctl{status, stall ? kStallWaitCycles : kWaitCycles, stall};
 
     echo::K1Args a1{};
     echo::K2Args a2{};
@@ -203,10 +261,8 @@ extern "C" int echo_allreduce_static(int P, size_t n, int dtype, void *const ran
     a3.bf16 = dtype == ECHO_BF16;
     a3.ctl = ctl;
 
-    const char *what = "cudaMemsetAsync of the status word";
-    e = cudaMemsetAsync(status, 0, sizeof(int), st); // must start at zero
-    if (e == cudaSuccess && (e = echo::launch_k1_compensate_quantize_pack(a1, st)) != cudaSuccess)
-        what = "launch k1_compensate_quantize_pack";
+    const char *what = "launch k1_compensate_quantize_pack";
+    e = echo::launch_k1_compensate_quantize_pack(a1, st);
     if (e == cudaSuccess && (e = echo::launch_k2_owner_reduce_requant(a2, st)) != cudaSuccess)
         what = "launch k2_owner_reduce_requant";
     if (e == cudaSuccess && (e = echo::launch_k3_gather_dequant(a3, st)) != cudaSuccess)

@@ -48,7 +48,7 @@ EXPORTED = (
     "echo_get_state", "echo_set_state", "echo_get_state_range", "echo_get_wire",
     "echo_get_wire_range", "echo_stats", "echo_model_bytes", "echo_set_timing",
     "echo_last_kernel_ms", "echo_kernel_ms_total", "echo_device_status",
-    "echo_allreduce_static", "echo_set_variant", "echo_get_sender_state", "echo_set_sender_state",
+    "echo_allreduce_static", "echo_static_status", "echo_set_variant", "echo_get_sender_state", "echo_set_sender_state",
     "echo_model_bytes_ex", "echo_debug_build", "echo_debug_touch_guard",
     "echo_dist_create", "echo_dist_export", "echo_dist_connect", "echo_dist_stage",
     "echo_dist_set_params", "echo_dist_set_variant", "echo_dist_get_state",
@@ -94,6 +94,7 @@ def _load():
         "echo_device_status": (_int, [_vp, ctypes.POINTER(ctypes.c_int), _int]),
         "echo_allreduce_static": (_int, [_int, _sz, _int, _vpp, _vp, _vp, ctypes.c_float, ctypes.c_float,
                                          ctypes.c_float, _int, _vp]),
+        "echo_static_status": (_int, [ctypes.POINTER(ctypes.c_int), _int]),
         "echo_set_variant": (_int, [_vp, _int]),
         "echo_get_sender_state": (_int, [_vp, _int, _int, _sz, _sz, _f32p]),
         "echo_set_sender_state": (_int, [_vp, _int, _int, _f32p]),
@@ -175,6 +176,14 @@ def echo_allreduce_static(P: int, n: int, dtype: int, rank_ptrs, f_ptr: int, s_p
     caller passes the rank buffers and this phase's state arrays f, s."""
     _check(_lib.echo_allreduce_static(P, n, dtype, _ptr_array(rank_ptrs), f_ptr, s_ptr, beta_fast,
                                       beta_slow, lam, int(bool(enable)), stream))
+
+
+def echo_static_status(clear: bool = False) -> int:
+    """The static path's device status word on the current device (waits for
+    the device); ``clear`` zeroes it after reading."""
+    st = ctypes.c_int(0)
+    _check(_lib.echo_static_status(ctypes.byref(st), int(bool(clear))))
+    return st.value
 
 
 def echo_reset(h: int, phase_mask: int = 3) -> None:

@@ -73,6 +73,10 @@ enum {
 
 /*
  * echo_create - a handle for all-reduces of P ranks x n elements of dtype.
+ * Defined by [rit.work "Echo 4-bit GPU communication", section "How Echo
+ * returns the error to later calls"]: P tensor-parallel ranks each hold a
+ * partial sum of the same tensor, cut into P segments with one owner each;
+ * the handle holds the wire those ranks exchange and the compensator state.
  *   P      number of simulated tensor-parallel ranks, 2..16.
  *   n      elements per rank; n % (P*group) == 0 and n <= 2^34; also
  *          n % 32 == 0 (16-byte code rows), which only group 16 with an
@@ -92,6 +96,13 @@ ECHO_API echo_handle *echo_create(int P, size_t n, int group, int dtype);
 
 /*
  * echo_allreduce - in-place Echo all-reduce of P rank buffers.
+ * Defined by [rit.work "Echo 4-bit GPU communication", section "How Echo
+ * returns the error to later calls"]: every rank rounds its partial to 4-bit
+ * integers (the owner of a segment first adds the correction to its own part
+ * of it), each owner restores and adds the P segments in high precision,
+ * rounds the total to 4 bits once more and sends it back to every rank, so
+ * each element is rounded at most twice; the owner's rounding error updates
+ * the fast and slow estimates of the call's phase.
  *   rank_ptrs  P device pointers, each n elements of the handle's dtype,
  *              16-byte aligned, pairwise non-overlapping. Caller-owned.
  *   phase      ECHO_FWD or ECHO_BWD: which compensator state is read and
@@ -140,22 +151,45 @@ ECHO_API int echo_allreduce_host(echo_handle *h, const void *const host_send[], 
  *              NULL, when enable == 0). Zero them before the first call.
  *   beta_fast, beta_slow, lambda, enable   as for echo_set_params.
  * The wire buffers the kernels exchange live in one array compiled into the
- * library, ECHO_STATIC_SCRATCH_BYTES (32 MiB) on every GPU that loads it,
- * kept until the process exits. A call needs about (P+1)*17/32 bytes per
- * element of n (at P = 8, n up to about 7 million elements); larger sizes are
- * rejected with ECHO_ERR_UNSUPPORTED and nothing is enqueued. The first call
- * on a device looks up the array's device address (cudaGetSymbolAddress) with
- * that device current; make that first call before any stream capture. All
- * calls share the array and it keeps the last call's contents; calls whose
- * work overlaps on the GPU (other streams or threads at once) race on it.
+ * library, ECHO_STATIC_SCRATCH_BYTES (32 MiB) per GPU, kept until the process
+ * exits. A call needs about (P+1)*17/32 bytes per element of n (at P = 8, n
+ * up to about 7 million elements); larger sizes, and n > 2^34, are rejected
+ * with ECHO_ERR_UNSUPPORTED and nothing is enqueued. Argument errors (P, n,
+ * dtype, parameters, NULL, misaligned, non-device, other-device or
+ * overlapping pointers, state overlapping a rank buffer) return
+ * ECHO_ERR_INVALID with nothing enqueued.
+ * Set-up: the first call of echo_allreduce_static or echo_static_status on a
+ * device, with that device current, looks up the array's device address
+ * (cudaGetSymbolAddress) and zeroes its status word, synchronously. Under
+ * CUDA's lazy module loading that is also when the 32 MiB are taken from the
+ * device. So make one such call (echo_static_status is the cheap one) at
+ * start-up: before reserving the rest of HBM for a memory pool, and before
+ * any stream capture.
+ * All calls share the array and it keeps the last call's contents; calls
+ * whose work overlaps on the GPU (other streams or threads at once) race on
+ * it.
  */
 #define ECHO_STATIC_SCRATCH_BYTES (32u * 1024u * 1024u)
 ECHO_API int echo_allreduce_static(int P, size_t n, int dtype, void *const rank_ptrs[], float *f, float *s,
                                    float beta_fast, float beta_slow, float lambda, int enable, void *stream);
 
+/*
+ * echo_static_status - the static path's device status word on the current
+ * device (synchronous: waits for the device first), with the bits of
+ * echo_device_status. Every echo_allreduce_static call on the device ORs
+ * into the same word, so it gathers the timeouts of all calls since it was
+ * last cleared; clear != 0 zeroes it after reading. The first use on a
+ * device sets up the static array (see echo_allreduce_static) and allocates
+ * nothing else.
+ */
+ECHO_API int echo_static_status(int *status, int clear);
+
 /* echo_reset - zero the compensator state (and the sender errors, if
  * allocated) of the phases in phase_mask (bit 0 forward, bit 1 backward);
- * waits for the device first and completes before return. */
+ * waits for the device first and completes before return. The forward and
+ * the backward pass keep separate estimates [rit.work "Echo 4-bit GPU
+ * communication", end of section "How Echo returns the error to later
+ * calls"]. */
 ECHO_API int echo_reset(echo_handle *h, int phase_mask);
 
 /* echo_destroy - free everything the handle owns (synchronises the device
@@ -218,7 +252,9 @@ ECHO_API int echo_set_sender_state(echo_handle *h, int phase, int rank, const fl
 
 /* echo_get_state / echo_set_state - synchronous copies of a phase's two
  * estimates (n binary32 each) to / from host memory. A checkpoint is the pair
- * for both phases. */
+ * for both phases. The two smoothed estimates, one fast and one slow, per
+ * phase: [rit.work "Echo 4-bit GPU communication", end of section "How Echo
+ * returns the error to later calls"]. */
 ECHO_API int echo_get_state(echo_handle *h, int phase, float *f_host, float *s_host);
 ECHO_API int echo_set_state(echo_handle *h, int phase, const float *f_host, const float *s_host);
 
@@ -227,7 +263,10 @@ ECHO_API int echo_get_state_range(echo_handle *h, int phase, size_t offset, size
                          float *f_host, float *s_host);
 
 /*
- * echo_get_wire - synchronous copy of the wire left by the last call.
+ * echo_get_wire - synchronous copy of the wire left by the last call: the
+ * 4-bit segments every rank sends to the owners, and the 4-bit total the
+ * owners send back [rit.work "Echo 4-bit GPU communication", section "How
+ * Echo returns the error to later calls"].
  *   stage 1: rank's packed codes (n/2 bytes) and scales (n/group bytes, or
  *            n/group little-endian binary16 patterns under
  *            ECHO_VARIANT_FP16_SCALE: 2n/group bytes);
@@ -243,7 +282,10 @@ ECHO_API int echo_get_wire_range(echo_handle *h, int stage, int rank, size_t gro
                         size_t ngroups, uint8_t *codes_host, uint8_t *scales_host);
 
 /*
- * echo_stats - counters since creation: bytes that would cross links
+ * echo_stats - counters since creation (the exchanged volume is the pages'
+ * point: 4-bit words make it almost four times smaller than 16-bit ones,
+ * [rit.work "Echo 4-bit GPU communication", section "Why plain 4-bit
+ * summation damages the model"]): bytes that would cross links
  * (reduce-scatter + all-gather, 2(P-1) * n * w per call, with w the wire
  * bytes per element: 17/32 at the default group of 32), modelled HBM
  * bytes (sum of the three kernels' algorithmic bytes), and calls made through

@@ -170,3 +170,37 @@ def test_binding_fails_loudly_without_library(tmp_path):
     copy.write_text(open(os.path.join(ROOT, "bit_error_compensated_rank_b200", "echo.py")).read())
     res = subprocess.run([sys.executable, "-c", code, str(copy)], capture_output=True, text=True)
     assert res.returncode == 0, res.stderr
+
+
+@pytest.mark.parametrize("P,n,dtype,params,status,words", [
+    (1, 64, 0, (0.5, 0.875, 0.5, 1), -1, "outside"),
+    (17, 17 * 32, 0, (0.5, 0.875, 0.5, 1), -1, "outside"),
+    (2, 64, 5, (0.5, 0.875, 0.5, 1), -1, "dtype"),
+    (2, 0, 0, (0.5, 0.875, 0.5, 1), -1, "multiple"),
+    (4, 4 * 32 * 3 + 32, 0, (0.5, 0.875, 0.5, 1), -1, "multiple"),
+    (2, 64, 0, (1.0, 0.875, 0.5, 1), -1, "parameters"),
+    (2, 64, 0, (0.5, -0.1, 0.5, 1), -1, "parameters"),
+    (2, 64, 0, (0.5, 0.875, 1.5, 1), -1, "parameters"),
+    (2, 64, 0, (0.5, 0.875, 0.5, 2), -1, "parameters"),
+    # larger than the fixed scratch array
+    (8, 8 * 32 * 65536, 0, (0.5, 0.875, 0.5, 1), -2, "static scratch"),
+    # past 2^34, including a size whose scratch arithmetic would wrap around
+    # 64 bits: rejected before any of it is computed
+    (16, (1 << 34) + 512, 0, (0.5, 0.875, 0.5, 1), -2, "maximum"),
+    (16, (1 << 64) - 512, 1, (0.5, 0.875, 0.5, 1), -2, "maximum"),
+])
+def test_static_rejects_bad_arguments_before_cuda(echo, P, n, dtype, params, status, words):
+    """echo_allreduce_static checks its shape and parameters on the host,
+    before any CUDA call, so these run without a GPU; pointer checks need one
+    and run in the GPU suite."""
+    bf, bs, lam, en = params
+    ptrs = echo._ptr_array([0] * max(P, 1))
+    rc = echo._lib.echo_allreduce_static(P, n, dtype, ptrs, None, None, bf, bs, lam, en, None)
+    assert rc == status, echo.echo_last_error()
+    assert echo.echo_last_status() == status
+    assert words in echo.echo_last_error()
+
+
+def test_static_status_needs_an_output(echo):
+    assert echo._lib.echo_static_status(None, 0) == echo.ECHO_ERR_INVALID
+    assert "NULL" in echo.echo_last_error()
