@@ -1,6 +1,7 @@
 """Benchmark of the Echo error-compensated 4-bit all-reduce on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl echo|reference]
+                    [--mode simulated|sharded|replicas] [--config 1|2|4|5] [--sweep]
 
 Workload (one step = one all-reduce call, the whole hot path: compensate +
 quantise + pack, owner reduce + requantise, gather + dequantise): P = 8
@@ -13,9 +14,24 @@ nccl-tests definition), and the call's fraction of the HBM roofline, where
 the roofline time is the three kernels' algorithmic bytes divided by the
 measured HBM copy bandwidth.
 
-With N > 1 (one process per GPU under torchrun) every GPU runs its own
-independent 8-rank problem (weak scaling, no collective on the data path);
-the value is the sum of all GPUs' work divided by the slowest GPU's time.
+Modes (``--mode``; the default is ``simulated`` at N = 1, ``sharded`` at
+N > 1):
+
+* ``simulated``: one handle, the P ranks are P buffers in one GPU's HBM.
+* ``sharded``: the same P-rank all-reduce with one handle per rank
+  (echo_dist_*), the P ranks spread over the N processes (P/N each, one
+  process per GPU), the wire stored straight into the other ranks' blocks
+  (peer stores over NVLink between GPUs) and the stages ordered by events.
+  The problem is fixed as N grows (strong scaling) and the value is the
+  all-reduce's algbw; at N = 8 it is the P = 8, 1 GiB all-reduce over NVLink.
+* ``replicas``: every GPU runs its own independent P-rank simulated problem
+  (weak scaling, nothing crosses GPUs); the value is the sum of all GPUs'
+  work divided by the slowest GPU's time.
+
+``--config 1|2|4|5`` prints one line for another of the five workloads
+(per-call time issued one by one and replayed from a CUDA graph, algbw,
+roofline fraction; for the deep residual stream also the distance to the
+exact sum by depth) instead of the benchmark line.
 
 ``--impl reference`` times the plain CPU oracle instead (the slow reference
 program this library is checked against), on a bounded sample of the same
@@ -300,7 +316,7 @@ def run_reference(args, rank: int, world: int) -> dict | None:
 # n = 2^26 and scaled by n, since the traffic grows in proportion); reported
 # only while the kernel source still has the hash it had when captured.
 NCU_TRAFFIC = {
-    "k1_compensate_quantize_pack": {"bytes_per_elem": 28.06, "source_sha": "766fbf51be35dcc8"},
+    "k1_compensate_quantize_pack": {"bytes_per_elem": 28.062, "source_sha": "4b0571337a1e501c"},
 }
 
 
@@ -378,6 +394,10 @@ def run_echo(args, rank: int, world: int, local: int) -> dict | None:
     peak, peak_kind = hbm_peak()
     call_bytes = mb["total"]
     call_frac = call_bytes / (ms_step * 1e-3) / (peak * 1e9)
+    # On one GPU the P simulated ranks share one requantised buffer, which
+    # kernel 3 reads once instead of once per rank: (P-1) wire reads fewer
+    # than the P-GPU model above, whose fraction can therefore pass 1.
+    min_bytes = call_bytes - mb["link"] // 2
 
     k_avg = [t / timed_calls for t in kern_ms]
     names = ["k1_compensate_quantize_pack", "k2_owner_reduce_requant", "k3_gather_dequant"]
@@ -406,13 +426,17 @@ def run_echo(args, rank: int, world: int, local: int) -> dict | None:
         "config": {"workload": workload_name(args),
                    "variant": args.variant, "P": P, "n_per_rank": n, "group": args.group,
                    "element_dtype": "bf16", "wire": "int4 codes + scales",
+                   "mode": "simulated" if world == 1 else "replicas",
                    "parallelism": f"{world} independent replica(s), ranks simulated in HBM",
                    "l2": "inputs larger than L2 (8 GiB of partials per GPU vs 126 MB L2)"},
         "hbm_roofline_frac": round(call_frac, 4),
         "hbm_roofline": {"model_bytes_per_call": call_bytes,
                          "bytes_per_elem": round(call_bytes / n, 5),
                          "peak_gbs": peak, "peak_kind": peak_kind,
-                         "ideal_ms": round(call_bytes / (peak * 1e9) * 1e3, 4)},
+                         "ideal_ms": round(call_bytes / (peak * 1e9) * 1e3, 4),
+                         "model": "P-GPU: every rank reads its own copy of the requantised wire"},
+        "single_gpu_min_bytes_per_elem": round(min_bytes / n, 5),
+        "single_gpu_min_frac": round(min_bytes / (ms_step * 1e-3) / (peak * 1e9), 4),
         "busbw": round(value * 2 * (P - 1) / P, 3),
         "kernel_ms": {names[i]: round(k_avg[i], 4) for i in range(len(names))},
         "kernel_frac": {names[i]: round(k_bytes[i] / (k_avg[i] * 1e-3) / 1e9 / peak, 4)
@@ -428,6 +452,383 @@ def run_echo(args, rank: int, world: int, local: int) -> dict | None:
         result["e2e"] = e2e
     h.close()
     return result if rank == 0 else None
+
+
+# Peer copy bandwidth per direction per GPU measured on this machine's B200s over
+# NVLink 5 (the denominator of the sharded mode's link fraction; nominal 900).
+NVLINK_PEER_GBS = 770.0
+
+
+def shard_ranks(P: int, world: int, rank: int) -> list[int]:
+    """The all-reduce ranks that process ``rank`` of ``world`` holds: P/world
+    consecutive ranks."""
+    if P % world:
+        raise ValueError(f"{P} ranks do not split evenly over {world} processes")
+    per = P // world
+    return list(range(rank * per, (rank + 1) * per))
+
+
+def cross_gpu_link_bytes(P: int, n_gpus: int, link_bytes: int) -> int:
+    """Wire bytes one GPU sends to the other GPUs per call when the P ranks
+    are spread L = P/N per GPU. ``link_bytes`` is the P-GPU figure 2(P-1)*W,
+    W the wire bytes of a whole message, so a segment's wire is W/P. Each of a
+    GPU's L ranks sends its segments for the P - L owners on other GPUs, and
+    each of its L owners sends its requantised segment to those P - L ranks:
+    2 L (P - L) W / P, which is 2(P-1)/P * W at one rank per GPU."""
+    if n_gpus <= 1:
+        return 0
+    L = P // n_gpus
+    W = link_bytes // (2 * (P - 1))
+    return 2 * L * (P - L) * W // P
+
+
+def run_sharded(args, rank: int, world: int, local: int) -> dict | None:
+    """The P-rank all-reduce with one handle per rank (echo_dist_*), the
+    ranks spread over the processes (P/world each); strong scaling."""
+    import torch
+    from bit_error_compensated_rank_b200 import echo
+    from bit_error_compensated_rank_b200 import workloads as wl
+
+    dev_index = 0 if args.one_gpu else local
+    torch.cuda.set_device(dev_index)
+    device = torch.device("cuda", dev_index)
+    dist = init_dist(world, "gloo")  # host barriers and the handle exchange only: no data
+    mine = shard_ranks(P, world, rank)
+    n = args.n - args.n % (P * max(args.group, 32))
+    stream = torch.cuda.current_stream(device)
+    xs = [torch.empty(n, dtype=torch.bfloat16, device=device) for _ in mine]
+    outs = [torch.empty(n, dtype=torch.bfloat16, device=device) for _ in mine]
+    for x, r in zip(xs, mine):
+        wl.torch_outlier_gaussian_(x, seed=SEED, call=0, rank=r)
+    variant = VARIANTS[args.variant]
+    ds = [echo.DistEcho(P, r, n, echo.ECHO_BF16, args.group) for r in mine]
+    for d in ds:
+        if variant:
+            d.set_variant(variant)
+    blobs = [d.export() for d in ds]
+    if world > 1:
+        gathered = [None] * world
+        dist.all_gather_object(gathered, blobs)
+        blobs = [b for part in gathered for b in part]
+    for d in ds:
+        d.connect(blobs)
+
+    def bar():
+        barrier(world)
+
+    def call():
+        echo.dist_allreduce(ds, xs, outs, bar, echo.ECHO_FWD, stream, sync=args.host_ordered)
+
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize()
+    bar()
+    clocks = ClockSampler(gpu_selector(dev_index))
+    clocks.start()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    bar()
+    start.record(stream)
+    for _ in range(args.steps):
+        call()
+    end.record(stream)
+    torch.cuda.synchronize()
+    bar()
+    clk = clocks.stop()
+    ms_step = max_over_ranks(start.elapsed_time(end) / args.steps, world)
+    stage_ms = sharded_stage_ms(ds, xs, outs, bar, stream, args)
+
+    mb = echo.echo_model_bytes_ex(P, n, args.group, echo.ECHO_BF16, True, variant)
+    n_gpus = 1 if args.one_gpu else world
+    peak, peak_kind = hbm_peak()
+    gpu_bytes = mb["total"] * len(mine) // P  # the model is the same for every rank
+    hbm_achieved = gpu_bytes / (ms_step * 1e-3) / 1e9
+    link = cross_gpu_link_bytes(P, n_gpus, mb["link"])
+    value = 2.0 * n / (ms_step * 1e-3) / 1e9
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_sharded_e2e(ds, xs, outs, n, args, device, world, bar)
+    result = {
+        "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": n_gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": workload_name(args), "mode": "sharded", "variant": args.variant, "P": P,
+                   "n_per_rank": n, "group": args.group, "element_dtype": "bf16",
+                   "wire": "int4 codes + scales",
+                   "parallelism": f"{P} ranks as one handle each, {len(mine)} per process, {world} "
+                                  f"process(es) on {n_gpus} GPU(s); wire stored into the other ranks' "
+                                  f"blocks, stages ordered by "
+                                  f"{'host synchronisation' if args.host_ordered else 'events'}",
+                   "l2": "inputs larger than L2" if P // n_gpus * n * 2 > L2_BYTES else "inputs fit in L2"},
+        "busbw": round(value * 2 * (P - 1) / P, 3),
+        "hbm_roofline_frac": round(hbm_achieved / peak, 4),
+        "roofline": {"kernel": "whole call (three stages)", "bound": "hbm", "achieved": round(hbm_achieved, 1),
+                     "peak": peak, "unit": "GB/s", "frac": round(hbm_achieved / peak, 4), "traffic": None,
+                     "peak_kind": peak_kind, "bytes_per_gpu_per_call": gpu_bytes},
+        "link_bytes_per_gpu_per_call": link,
+        # after the timed region: each stage of this process's ranks, the
+        # waits on the other ranks' events included (rank 0's process)
+        "stage_ms": stage_ms,
+        "gpu_launches": 3 * len(mine) * args.steps,
+        "clocks": clk,
+    }
+    if link:
+        result["link"] = {"achieved_gbs": round(link / (ms_step * 1e-3) / 1e9, 1),
+                          "peak_gbs": NVLINK_PEER_GBS, "peak_kind": "measured peer copy per direction",
+                          "frac": round(link / (ms_step * 1e-3) / 1e9 / NVLINK_PEER_GBS, 4)}
+    if e2e is not None:
+        result["e2e"] = e2e
+    torch.cuda.synchronize()
+    bar()
+    for d in ds:
+        d.close()
+    return result if rank == 0 else None
+
+
+def sharded_stage_ms(ds, xs, outs, bar, stream, args) -> list[float]:
+    """Mean time of each of the three stages over ``args.steps`` more calls,
+    from CUDA events recorded between the stages on the launching stream."""
+    import torch
+    from bit_error_compensated_rank_b200 import echo
+    calls = []
+    for _ in range(args.steps):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        ev[0].record(stream)
+        for k in (1, 2, 3):
+            for d, x, out in zip(ds, xs, outs):
+                d.stage(k, x, out, echo.ECHO_FWD, stream)
+            ev[k].record(stream)
+            if k < 3:
+                bar()
+        calls.append(ev)
+    torch.cuda.synchronize()
+    bar()
+    return [round(statistics.mean(ev[k - 1].elapsed_time(ev[k]) for ev in calls), 4) for k in (1, 2, 3)]
+
+
+def run_sharded_e2e(ds, xs, outs, n, args, device, world, bar) -> dict:
+    """Per step: every local rank's partial from pinned host memory to the
+    device, the all-reduce, and the result back to pinned host memory."""
+    import torch
+    from bit_error_compensated_rank_b200 import echo
+    steps = max(1, min(args.steps, args.e2e_steps))
+    try:
+        host_in = [torch.empty(n, dtype=torch.bfloat16, pin_memory=True) for _ in xs]
+        host_out = torch.empty(n, dtype=torch.bfloat16, pin_memory=True)
+    except RuntimeError as exc:
+        return {"value": None, "unit": UNIT, "error": f"pinned host allocation failed: {exc}"}
+    for h, x in zip(host_in, xs):
+        h.copy_(x)
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        for x, h in zip(xs, host_in):
+            x.copy_(h, non_blocking=True)
+        echo.dist_allreduce(ds, xs, outs, bar, echo.ECHO_FWD, stream, sync=args.host_ordered)
+        host_out.copy_(outs[0], non_blocking=True)
+
+    step()
+    torch.cuda.synchronize()
+    bar()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for _ in range(steps):
+        step()
+    end.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(start.elapsed_time(end) / steps, world)
+    return {"value": round(2.0 * n / (ms * 1e-3) / 1e9, 3), "unit": UNIT,
+            "h2d_bytes_per_step": int(sum_over_ranks(2.0 * n * len(xs), world)),
+            "d2h_bytes_per_step": int(sum_over_ranks(2.0 * n, world)),
+            "ms_per_step": round(ms, 3), "steps": steps}
+
+
+# The other four workloads: shape and inputs (the headline is the third).
+CONFIG_DESC = {
+    1: "P=2, one 4096-element bf16 partial per rank (1 token x hidden 4096), N(0,1), group 32, "
+       "8 calls, compensation on, seed 0",
+    2: "Qwen3-8B-shaped inference: P=4, 2048 tokens x 4096 hidden bf16, 72 calls, channel-scaled "
+       "partials (sigma_c log-uniform [0.1,1], 1% channels x20), forward state only",
+    4: "Llama-3-8B-shaped training step: P=4, 2 x 4096 tokens x 4096 hidden bf16, 64 forward calls "
+       "(channel-scaled) then 64 backward calls (1e-3 Student-t nu=3), separate state",
+    5: "deep residual stream: P=8, 64 tokens x hidden 1024 binary32, 256 layers, pre-norm partials "
+       "(x/rms(x)) W_r / sqrt(1024 P); compensation on vs off vs sender feedback vs exact sum",
+}
+
+
+def time_sequence(h, seq, outs, stream, min_ms: float = 60.0) -> tuple[float, float, int]:
+    """Per-call time of a sequence of out-of-place calls ``seq`` = [(inputs,
+    phase), ...] on handle ``h``: (a) issued one by one from Python, and (b)
+    captured once in a CUDA graph and replayed (the GPU time). Returns
+    (eager ms, graph ms, repetitions of the sequence)."""
+    import torch
+
+    def run_once(st):
+        for xs, phase in seq:
+            h.allreduce_out(xs, outs, phase, st)
+
+    run_once(stream)
+    torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    run_once(stream)
+    end.record(stream)
+    torch.cuda.synchronize()
+    reps = max(2, min(2000, int(min_ms / max(start.elapsed_time(end), 1e-3)) + 1))
+    start.record(stream)
+    for _ in range(reps):
+        run_once(stream)
+    end.record(stream)
+    torch.cuda.synchronize()
+    eager = start.elapsed_time(end) / (reps * len(seq))
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        run_once(None)
+    graph.replay()
+    torch.cuda.synchronize()
+    start.record(stream)
+    for _ in range(reps):
+        graph.replay()
+    end.record(stream)
+    torch.cuda.synchronize()
+    replayed = start.elapsed_time(end) / (reps * len(seq))
+    del graph
+    return eager, replayed, reps
+
+
+def residual_partials(x, layer: int, P: int, hidden: int, seed: int):
+    """Pre-norm tensor-parallel partials of one layer of the deep residual
+    stream: (x / rms(x)) W_{layer,r} / sqrt(hidden * P), r = 0..P-1."""
+    import torch
+    from bit_error_compensated_rank_b200 import workloads as wl
+    xn = x / torch.sqrt(torch.mean(x.double() ** 2, dim=1, keepdim=True)).float()
+    scale = 1.0 / math.sqrt(hidden * P)
+    return [(xn @ wl.residual_weight(layer, r, hidden, seed, device=x.device)) * scale for r in range(P)]
+
+
+def residual_errors(P: int, tokens: int, hidden: int, layers: int, seed: int) -> dict:
+    """The deep residual stream run three ways through the CUDA path
+    (compensation on, off, and on with sender feedback) beside the exact sum
+    of the partials (binary64), from the same start: |x - x_exact| / |x_exact|
+    and |x - x_exact| per layer, reported at layers 1, 2, 4, ..., ``layers``."""
+    import torch
+    from bit_error_compensated_rank_b200 import echo
+    from bit_error_compensated_rank_b200 import workloads as wl
+    torch.backends.cuda.matmul.allow_tf32 = False
+    n = tokens * hidden
+    x0 = torch.from_numpy(wl.residual_init(tokens, hidden, seed)).cuda()
+    runs = {"on": (True, 0), "off": (False, 0), "sender_ef": (True, echo.ECHO_VARIANT_SENDER_EF)}
+    handles = {}
+    for key, (enable, variant) in runs.items():
+        h = echo.Echo(P, n, echo.ECHO_FP32)
+        h.set_params(enable=enable)
+        if variant:
+            h.set_variant(variant)
+        handles[key] = h
+    x = {k: x0.clone() for k in list(runs) + ["exact"]}
+    marks = [2 ** k for k in range(int(math.log2(layers)) + 1)]
+    out = {"layers": marks, "rel": {k: [] for k in runs}, "abs": {k: [] for k in runs}}
+    for layer in range(layers):
+        pe = residual_partials(x["exact"], layer, P, hidden, seed)
+        x["exact"] = (x["exact"].double() + torch.stack(pe).double().sum(0)).float()
+        for key, h in handles.items():
+            parts = [t.reshape(-1).contiguous() for t in residual_partials(x[key], layer, P, hidden, seed)]
+            h.allreduce(parts, 0)
+            x[key] = x[key] + parts[0].reshape(tokens, hidden)
+        if layer + 1 in marks:
+            ref = float(torch.linalg.norm(x["exact"].double()))
+            for key in runs:
+                d = float(torch.linalg.norm((x[key] - x["exact"]).double()))
+                out["abs"][key].append(round(d, 6))
+                out["rel"][key].append(round(d / ref, 6))
+    for h in handles.values():
+        h.close()
+    return out
+
+
+def run_config(args) -> dict:
+    """One line for workload ``args.config`` (1, 2, 4 or 5)."""
+    import numpy as np
+    import torch
+    from bit_error_compensated_rank_b200 import echo
+    from bit_error_compensated_rank_b200 import workloads as wl
+
+    torch.cuda.set_device(0)
+    stream = torch.cuda.current_stream()
+    peak, peak_kind = hbm_peak()
+    cfg = args.config
+    if cfg == 1:
+        Pc, n, code = 2, 4096, echo.ECHO_BF16
+        seq_inputs = []
+        for k in range(8):
+            x = torch.from_numpy(wl.gaussian(Pc, n, seed=0, call=k).view(np.int16)).cuda()
+            seq_inputs.append(([x[r].view(torch.bfloat16) for r in range(Pc)], 0))
+    elif cfg in (2, 4):
+        Pc, hidden, code = 4, 4096, echo.ECHO_BF16
+        tokens = 2048 if cfg == 2 else 2 * 4096
+        n = tokens * hidden
+        sigma = torch.from_numpy(wl.channel_scale(hidden, seed=0 if cfg == 2 else 1)).cuda()
+        pool = 72 if cfg == 2 else 8  # distinct input sets (config 4 cycles 8 per phase)
+        fwd = []
+        for k in range(pool):
+            bufs = [torch.empty(n, dtype=torch.bfloat16, device="cuda") for _ in range(Pc)]
+            for r in range(Pc):
+                wl.torch_channel_scaled_(bufs[r], sigma, seed=cfg, call=k, rank=r)
+            fwd.append(bufs)
+        if cfg == 2:
+            seq_inputs = [(fwd[k], 0) for k in range(72)]
+        else:
+            bwd = []
+            for k in range(pool):
+                bufs = [torch.empty(n, dtype=torch.bfloat16, device="cuda") for _ in range(Pc)]
+                for r in range(Pc):
+                    wl.torch_student_t_(bufs[r], seed=cfg, call=k, rank=r)
+                bwd.append(bufs)
+            seq_inputs = [(fwd[k % pool], 0) for k in range(64)] + [(bwd[k % pool], 1) for k in range(64)]
+    elif cfg == 5:
+        Pc, hidden, tokens, code = 8, 1024, 64, echo.ECHO_FP32
+        n = hidden * tokens
+        x0 = torch.from_numpy(wl.residual_init(tokens, hidden, 0)).cuda()
+        seq_inputs = [([t.reshape(-1).contiguous() for t in residual_partials(x0, layer, Pc, hidden, 0)], 0)
+                      for layer in range(8)]
+    else:
+        raise ValueError(f"no workload {cfg}")
+    ebytes = 2 if code == echo.ECHO_BF16 else 4
+    outs = [torch.empty(n, dtype=torch.bfloat16 if code == echo.ECHO_BF16 else torch.float32, device="cuda")
+            for _ in range(Pc)]
+    h = echo.Echo(Pc, n, code)
+    clocks = ClockSampler(gpu_selector(0))
+    clocks.start()
+    eager, graph, reps = time_sequence(h, seq_inputs, outs, stream)
+    clk = clocks.stop()
+    h.close()
+    mb = echo.echo_model_bytes(Pc, n, code, True)
+    frac_graph = mb["total"] / (graph * 1e-3) / (peak * 1e9)
+    line = {
+        "config_line": cfg, "workload": CONFIG_DESC[cfg], "P": Pc, "n_per_rank": n,
+        "element_dtype": "bf16" if code == echo.ECHO_BF16 else "fp32",
+        "calls_per_sequence": len(seq_inputs), "sequence_repetitions": reps,
+        "us_per_call_eager": round(eager * 1e3, 2), "us_per_call_graph": round(graph * 1e3, 2),
+        "algbw_GBs_eager": round(ebytes * n / (eager * 1e-3) / 1e9, 2),
+        "algbw_GBs_graph": round(ebytes * n / (graph * 1e-3) / 1e9, 2),
+        "model_bytes_per_call": mb["total"],
+        "roofline_frac_eager": round(mb["total"] / (eager * 1e-3) / (peak * 1e9), 4),
+        "roofline_frac_graph": round(frac_graph, 4), "peak_gbs": peak, "peak_kind": peak_kind,
+        "l2_resident": mb["total"] < L2_BYTES,
+        "regime": "launch-bound" if frac_graph < 0.5 else "hbm-bound",
+        "link_bytes_per_call": mb["link"],
+        "clocks": clk,
+    }
+    if cfg == 4:
+        line["inputs"] = "8 distinct input sets per phase, cycled over the 64 calls of each phase"
+    if cfg == 5:
+        line["inputs"] = "timing: 8 layers' partials from the start point, cycled"
+        line["residual_error_vs_depth"] = residual_errors(Pc, tokens, hidden, 256, 0)
+    return line
 
 
 def run_e2e(h, send, n, args, device, world) -> dict:
@@ -547,7 +948,9 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["echo", "reference"], default="echo")
-    ap.add_argument("--n", type=int, default=N_ELEMS, help="elements per rank (default 2^29)")
+    ap.add_argument("--n", "--elems", dest="n", type=int, default=N_ELEMS,
+                    help="elements per rank (default 2^29); under torchrun spell it --elems, which "
+                         "torchrun's own options do not abbreviate")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -556,15 +959,36 @@ def main(argv=None):
     ap.add_argument("--group", type=int, choices=[16, 32, 64, 128], default=32,
                     help="elements per scale (default 32, the method as read)")
     ap.add_argument("--ranks", type=int, default=8, choices=range(2, 17), metavar="P",
-                    help="simulated ranks per GPU, 2..16 (default 8, the benchmark's workload)")
+                    help="ranks of the all-reduce, 2..16 (default 8, the benchmark's workload)")
+    ap.add_argument("--mode", choices=["auto", "simulated", "sharded", "replicas"], default="auto",
+                    help="simulated: one handle, ranks in one GPU's HBM; sharded: one handle per rank, "
+                         "ranks spread over the processes; replicas: an independent simulated problem "
+                         "per GPU (auto: simulated at one process, sharded at more)")
+    ap.add_argument("--config", type=int, choices=[1, 2, 4, 5], default=None,
+                    help="print one line for this workload instead of the benchmark line")
+    ap.add_argument("--one-gpu", action="store_true",
+                    help="sharded mode: every process uses GPU 0 (with --gpus 1)")
+    ap.add_argument("--host-ordered", action="store_true",
+                    help="sharded mode: synchronise the stream before each stage barrier instead of "
+                         "ordering the stages with events")
     args = ap.parse_args(argv)
     global P
     P = args.ranks
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     rank, world, local = dist_env()
-    if world != args.gpus:
+    if args.one_gpu:
+        if args.gpus != 1:
+            ap.error("--one-gpu runs every process on GPU 0: use it with --gpus 1")
+    elif world != args.gpus:
         ap.error(f"--gpus {args.gpus} but WORLD_SIZE is {world}")
+    mode = args.mode if args.mode != "auto" else ("simulated" if world == 1 else "sharded")
+    if mode == "simulated" and world > 1:
+        ap.error("simulated mode runs one process; use --mode replicas or sharded")
+    if mode == "sharded" and P % world:
+        ap.error(f"--ranks {P} does not split evenly over {world} processes")
+    if mode != "sharded" and (args.one_gpu or args.host_ordered):
+        ap.error("--one-gpu and --host-ordered belong to the sharded mode")
 
     if args.impl == "reference":
         res = run_reference(args, rank, world)
@@ -575,14 +999,21 @@ def main(argv=None):
         if rank == 0:
             run_sweep(args)
         return 0
+    if args.config is not None:
+        if rank == 0:
+            print(json.dumps(run_config(args)), flush=True)
+        return 0
 
-    res = run_echo(args, rank, world, local)
+    if mode == "sharded":
+        res = run_sharded(args, rank, world, local)
+    else:
+        res = run_echo(args, rank, world, local)
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
         dist.destroy_process_group()
     if res is not None:
-        if world == 1 and not args.no_cpu_baseline:
+        if world == 1 and mode == "simulated" and not args.no_cpu_baseline:
             res["cpu_baseline"] = cpu_baseline_leg(VARIANTS[args.variant])
         print(json.dumps(res), flush=True)
     return 0

@@ -151,8 +151,22 @@ __device__ __forceinline__ bool half_scale_saturates(float A)
 // tie. The lane takes the minimum of its 8 low halves two at a time (a 16x2
 // minimum); if one is below 3, or the group saturated, the lane takes the exact path for all 8
 // values: one branch per lane, taken rarely.
+//
+// Values of 8 significant bits (bf16 partials that carry no correction)
+// need no exact path. With v = a*2^p (|a| < 2^8) and the step s = b*2^q
+// (b < 2^11, any binary16), a non-zero distance from v/s to a midpoint,
+// |v/s - (j + 1/2)| = |2a*2^p - (2j+1)*b*2^q| / (2b*2^q), is at least
+// 2^(min(p,q)-q) / (2b): more than 2^-12 when p >= q; when p < q, a |v|
+// that reaches a midpoint (>= s/2) has 2^(p-q) >= b/(2|a|), so more than
+// 2^-10. That is at least 16 units of 2^-16 against the estimate's 0.06, so
+// floor(Z / 2^16) is the nearest code unless v/s is exactly a midpoint. An
+// exact midpoint lands on a fraction of exactly 2 and floor(Z / 2^16) is the
+// code above it; the tie goes to the even code, so an odd code moves down
+// by one. A fraction below kZTie flags those values: no 8-bit value reaches
+// [0, kZTie) otherwise.
 constexpr float kZ = 192.500030517578125f; // 192 + 1/2 + 2*2^-16, bits 0x43408002
 constexpr uint32_t kZMargin = 3;
+constexpr uint32_t kZTie = 4;
 
 __device__ __forceinline__ uint32_t min_u16x2(uint32_t a, uint32_t b)
 {
@@ -173,20 +187,32 @@ __device__ __forceinline__ uint32_t zcode_bits(uint32_t z)
     return (z >> 16) + (kRoundBits - 0x4340u);
 }
 
+// Whether either 16-bit half of x is below bound (<= 0x8000): such a half
+// borrows into its own top bit, which was clear.
+__device__ __forceinline__ bool half_below(uint32_t x, uint32_t bound)
+{
+    return ((x - bound * 0x00010001u) & ~x & 0x80008000u) != 0;
+}
+
+// short_vals: every v[k] has at most 8 significant bits (see kZTie).
 __device__ __forceinline__ void codes8_half(const float (&v)[kChunk], float step, float inv, float half, bool sat,
-                                            uint32_t (&z)[kChunk])
+                                            bool short_vals, uint32_t (&z)[kChunk])
 {
 #pragma unroll
     for (int k = 0; k < kChunk; k++)
         z[k] = __float_as_uint(__fmaf_rn(v[k], inv, kZ));
     const uint32_t lo = min_u16x2(min_u16x2(__byte_perm(z[0], z[1], 0x5410), __byte_perm(z[2], z[3], 0x5410)),
                                   min_u16x2(__byte_perm(z[4], z[5], 0x5410), __byte_perm(z[6], z[7], 0x5410)));
-    // a half below kZMargin (<= 0x8000) borrows into its own top bit, which
-    // was clear: the usual SIMD test for a lane below a bound
-    if (sat || ((lo - kZMargin * 0x00010001u) & ~lo & 0x80008000u)) {
+    if (sat || (!short_vals && half_below(lo, kZMargin))) {
 #pragma unroll
         for (int k = 0; k < kChunk; k++)
             z[k] = zcode_of_bits(code_bits_near(v[k], step, inv, half));
+    } else if (short_vals && half_below(lo, kZTie)) {
+        // exact midpoints: an odd code (bit 16, the parity of byte 2) moves down
+#pragma unroll
+        for (int k = 0; k < kChunk; k++)
+            if ((z[k] & 0x1FFFFu) - 0x10000u < kZTie)
+                z[k] -= 0x10000u;
     }
 }
 

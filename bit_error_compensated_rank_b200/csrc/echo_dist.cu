@@ -18,15 +18,33 @@
 //   stage 3  kernel 3 restores the local gathered tensor into this rank's
 //            output.
 // On several GPUs the stores cross NVLink as peer stores; the kernels read
-// local memory only. No kernel waits on another process: the caller orders
-// the stages across processes (synchronise, then a host barrier, after each
-// stage). Every operation is the single-process path's, so the results are
-// bit for bit the same.
+// local memory only. No kernel waits on another process or spins on a flag.
+// The stages are ordered on the GPU by events: every rank records one
+// interprocess event after each of its stages, and before a stage each rank's
+// stream waits for the events of the stages it depends on on every rank:
+//   stage 1 (call k) writes the owners' receive slots, which stage 2 of call
+//            k-1 read: it waits for every rank's stage-2 event;
+//   stage 2 reads the receive slots every rank's stage 1 wrote, and writes
+//            the gathered tensors that stage 3 of call k-1 read: it waits for
+//            every rank's stage-1 and stage-3 events;
+//   stage 3 reads the gathered tensor every rank's stage 2 wrote: it waits
+//            for every rank's stage-2 event.
+// A wait takes the event's latest record at the time it is enqueued, so the
+// caller puts a host barrier over all ranks after stage 1 and after stage 2
+// of every call (each rank has enqueued its record before any rank enqueues
+// the waits that need it). The host never waits for the GPU, and the next
+// record of each event comes only after the following barrier. Ranks in one
+// process use each other's buffers and events directly; ranks in other
+// processes through CUDA IPC. Every operation is the single-process path's,
+// so the results are bit for bit the same.
 #include "echo.h"
 #include "echo_kernels.h"
 
 #include <cuda_runtime.h>
 
+#include <unistd.h>
+
+#include <chrono>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -50,10 +68,13 @@ struct echo_dist {
     uint8_t *xbuf = nullptr;
     size_t off_recv_scales = 0, off_q_codes = 0, off_q_scales = 0;
     size_t row_scale_stride = 0, seg_scale_stride = 0; // 2n/G and 2seg/G rounded up to 16
-    float *state = nullptr; // [phase][f|s][n]; only the owned segment moves
+    float *state = nullptr; // [phase][f|s][seg]: the owned segment's estimates
     float *eps = nullptr;   // [phase][n], sender feedback
     int *dstatus = nullptr;
     const uint8_t *peer[ECHO_MAX_RANKS] = {}; // every rank's exported block (own included)
+    bool peer_ipc[ECHO_MAX_RANKS] = {};       // opened through CUDA IPC (closed at destroy)
+    cudaEvent_t done[3] = {};                 // recorded after this rank's stage 1, 2, 3
+    cudaEvent_t peer_done[ECHO_MAX_RANKS][3] = {}; // every rank's (own included)
     bool connected = false;
     uint64_t calls = 0;
 };
@@ -64,6 +85,33 @@ std::mutex g_mu;
 std::set<const echo_dist *> g_live;
 
 constexpr long long kWaitCycles = 1LL << 31;
+
+// Layout of the blob echo_dist_export writes (ECHO_DIST_HANDLE_BYTES):
+//   [0, 64)     CUDA IPC handle of the exported block
+//   [64, 256)   CUDA IPC handles of the three stage events
+//   [256, 264)  token of the exporting process
+//   [264, 272)  the exporting handle (used only inside that process)
+//   [272, 280)  n;  [280, 284) world;  [284, 288) rank;  [288, 292) group;
+//   [292, 296)  dtype;  the rest zero
+struct Blob {
+    cudaIpcMemHandle_t mem;
+    cudaIpcEventHandle_t ev[3];
+    uint64_t token;
+    uint64_t self;
+    uint64_t n;
+    int32_t world, rank, group, dtype;
+};
+static_assert(sizeof(cudaIpcMemHandle_t) == 64 && sizeof(cudaIpcEventHandle_t) == 64, "CUDA IPC handle size");
+static_assert(sizeof(Blob) <= ECHO_DIST_HANDLE_BYTES, "exported blob size");
+
+// Identifies this process in exported blobs: the pid and the start time.
+uint64_t process_token()
+{
+    static const uint64_t token =
+        (static_cast<uint64_t>(getpid()) << 32) ^
+        static_cast<uint64_t>(std::chrono::steady_clock::now().time_since_epoch().count());
+    return token;
+}
 
 int fail(int code, const char *fmt, ...) __attribute__((format(printf, 2, 3)));
 int fail(int code, const char *fmt, ...)
@@ -122,9 +170,18 @@ int check_user_buffer(const void *p, int device, const char *what)
 
 void free_dist(echo_dist *d)
 {
-    for (int p = 0; p < d->world; p++)
-        if (p != d->rank && d->peer[p])
+    for (int p = 0; p < d->world; p++) {
+        if (!d->peer_ipc[p])
+            continue;
+        if (d->peer[p])
             cudaIpcCloseMemHandle(const_cast<uint8_t *>(d->peer[p]));
+        for (int k = 0; k < 3; k++)
+            if (d->peer_done[p][k])
+                cudaEventDestroy(d->peer_done[p][k]);
+    }
+    for (int k = 0; k < 3; k++)
+        if (d->done[k])
+            cudaEventDestroy(d->done[k]);
     for (void *p : {static_cast<void *>(d->xbuf), static_cast<void *>(d->state), static_cast<void *>(d->eps),
                     static_cast<void *>(d->dstatus)})
         if (p)
@@ -138,8 +195,8 @@ int stage1(echo_dist *d, const void *x, int phase, cudaStream_t st)
 {
     echo::K1Args a{};
     a.x.p[0] = x;
-    a.f = d->state + static_cast<size_t>(phase) * 2 * d->n;
-    a.s = a.f + d->n;
+    a.f = d->state + static_cast<size_t>(phase) * 2 * d->seg; // the owned segment's estimates
+    a.s = a.f + d->seg;
     a.to_owners = true;
     for (int p = 0; p < d->world; p++)
         a.owners.p[p] = const_cast<uint8_t *>(d->peer[p]);
@@ -162,18 +219,41 @@ int stage1(echo_dist *d, const void *x, int phase, cudaStream_t st)
     a.sender_ef = (d->variant & ECHO_VARIANT_SENDER_EF) != 0;
     a.fp16_scale = (d->variant & ECHO_VARIANT_FP16_SCALE) != 0;
     a.ctl = ctl_of(d);
-    cudaError_t e = echo::launch_k1_compensate_quantize_pack(a, st);
-    return e == cudaSuccess ? ECHO_OK : cuda_fail(e, "launch k1_compensate_quantize_pack");
+    // Only the owned segment carries the correction: with compensation on,
+    // one launch covers it with the state, and the rest of the row goes in
+    // launches that stage no state (their tiles hold partials only, so they
+    // are long enough to keep HBM busy).
+    const uint32_t s0 = static_cast<uint32_t>(d->rank * (d->seg / echo::kChunk));
+    const uint32_t s1 = s0 + static_cast<uint32_t>(d->seg / echo::kChunk);
+    struct Range {
+        uint32_t begin, end;
+        bool comp;
+    } ranges[3] = {{s0, s1, true}, {0, s0, false}, {s1, a.chunk_end, false}};
+    const int nranges = a.enable ? 3 : 1;
+    if (!a.enable)
+        ranges[0] = {0, a.chunk_end, false};
+    for (int i = 0; i < nranges; i++) {
+        if (ranges[i].end <= ranges[i].begin)
+            continue;
+        echo::K1Args b = a;
+        b.chunk_begin = ranges[i].begin;
+        b.chunk_end = ranges[i].end;
+        b.enable = a.enable && ranges[i].comp;
+        cudaError_t e = echo::launch_k1_compensate_quantize_pack(b, st);
+        if (e != cudaSuccess)
+            return cuda_fail(e, "launch k1_compensate_quantize_pack");
+    }
+    return ECHO_OK;
 }
 
 int stage2(echo_dist *d, int phase, cudaStream_t st)
 {
-    float *f = d->state + static_cast<size_t>(phase) * 2 * d->n + d->rank * d->seg;
+    float *f = d->state + static_cast<size_t>(phase) * 2 * d->seg;
     echo::K2Args a{};
     a.codes = d->xbuf; // the receive slots, one per rank
     a.scales = d->xbuf + d->off_recv_scales;
     a.f = f;
-    a.s = f + d->n;
+    a.s = f + d->seg;
     a.n = d->seg;
     a.scale_stride = d->seg_scale_stride;
     a.chunk_begin = 0;
@@ -279,15 +359,17 @@ echo_dist *echo_dist_create(int world, int rank, size_t n, int group, int dtype)
         size_t bytes;
     } allocs[] = {
         {reinterpret_cast<void **>(&d->xbuf), xbytes},
-        {reinterpret_cast<void **>(&d->state), 4 * n * sizeof(float)},
+        {reinterpret_cast<void **>(&d->state), 4 * d->seg * sizeof(float)},
         {reinterpret_cast<void **>(&d->dstatus), sizeof(int)},
     };
     for (auto &a : allocs) {
         if (e == cudaSuccess)
             e = cudaMalloc(a.p, a.bytes);
     }
+    for (int k = 0; k < 3 && e == cudaSuccess; k++)
+        e = cudaEventCreateWithFlags(&d->done[k], cudaEventDisableTiming | cudaEventInterprocess);
     if (e == cudaSuccess)
-        e = cudaMemset(d->state, 0, 4 * n * sizeof(float));
+        e = cudaMemset(d->state, 0, 4 * d->seg * sizeof(float));
     if (e == cudaSuccess)
         e = cudaMemset(d->dstatus, 0, sizeof(int));
     if (e == cudaSuccess)
@@ -304,26 +386,61 @@ echo_dist *echo_dist_create(int world, int rank, size_t n, int group, int dtype)
         return nullptr;
     }
     d->peer[rank] = d->xbuf;
+    for (int k = 0; k < 3; k++)
+        d->peer_done[rank][k] = d->done[k];
     std::lock_guard<std::mutex> lock(g_mu);
     g_live.insert(d);
     return d;
 }
 
-int echo_dist_export(echo_dist *d, uint8_t handle[ECHO_IPC_HANDLE_BYTES])
+int echo_dist_export(echo_dist *d, uint8_t handle[ECHO_DIST_HANDLE_BYTES])
 {
     int rc = check(d);
     if (rc != ECHO_OK)
         return rc;
     if (!handle)
         return fail(ECHO_ERR_INVALID, "handle buffer is NULL");
-    cudaIpcMemHandle_t h;
-    static_assert(sizeof(h) == ECHO_IPC_HANDLE_BYTES, "CUDA IPC handle size");
-    cudaError_t e = cudaIpcGetMemHandle(&h, d->xbuf);
+    Blob b;
+    std::memset(&b, 0, sizeof b);
+    cudaError_t e = cudaIpcGetMemHandle(&b.mem, d->xbuf);
+    for (int k = 0; k < 3 && e == cudaSuccess; k++)
+        e = cudaIpcGetEventHandle(&b.ev[k], d->done[k]);
     if (e != cudaSuccess)
-        return cuda_fail(e, "cudaIpcGetMemHandle");
-    std::memcpy(handle, &h, sizeof h);
+        return cuda_fail(e, "cudaIpcGetMemHandle / cudaIpcGetEventHandle");
+    b.token = process_token();
+    b.self = reinterpret_cast<uintptr_t>(d);
+    b.n = d->n;
+    b.world = d->world;
+    b.rank = d->rank;
+    b.group = d->group;
+    b.dtype = d->dtype;
+    std::memset(handle, 0, ECHO_DIST_HANDLE_BYTES);
+    std::memcpy(handle, &b, sizeof b);
     return ECHO_OK;
 }
+
+namespace {
+
+void disconnect(echo_dist *d)
+{
+    for (int q = 0; q < d->world; q++) {
+        if (q == d->rank)
+            continue;
+        if (d->peer_ipc[q]) {
+            if (d->peer[q])
+                cudaIpcCloseMemHandle(const_cast<uint8_t *>(d->peer[q]));
+            for (int k = 0; k < 3; k++)
+                if (d->peer_done[q][k])
+                    cudaEventDestroy(d->peer_done[q][k]);
+        }
+        d->peer[q] = nullptr;
+        d->peer_ipc[q] = false;
+        for (int k = 0; k < 3; k++)
+            d->peer_done[q][k] = nullptr;
+    }
+}
+
+} // namespace
 
 int echo_dist_connect(echo_dist *d, const uint8_t *handles)
 {
@@ -334,23 +451,66 @@ int echo_dist_connect(echo_dist *d, const uint8_t *handles)
         return fail(ECHO_ERR_INVALID, "handles is NULL");
     if (d->connected)
         return fail(ECHO_ERR_INVALID, "already connected");
+    Blob b[ECHO_MAX_RANKS];
+    for (int p = 0; p < d->world; p++) {
+        std::memcpy(&b[p], handles + static_cast<size_t>(p) * ECHO_DIST_HANDLE_BYTES, sizeof(Blob));
+        if (b[p].world != d->world || b[p].rank != p || b[p].n != d->n || b[p].group != d->group ||
+            b[p].dtype != d->dtype)
+            return fail(ECHO_ERR_INVALID,
+                        "handle %d is from rank %d of world %d (n = %llu, group %d, dtype %d); expected rank %d of "
+                        "world %d (n = %zu, group %d, dtype %d)",
+                        p, b[p].rank, b[p].world, static_cast<unsigned long long>(b[p].n), b[p].group, b[p].dtype, p,
+                        d->world, d->n, d->group, d->dtype);
+    }
+    const uint64_t me = process_token();
     for (int p = 0; p < d->world; p++) {
         if (p == d->rank)
             continue;
-        cudaIpcMemHandle_t h;
-        std::memcpy(&h, handles + static_cast<size_t>(p) * ECHO_IPC_HANDLE_BYTES, sizeof h);
+        cudaError_t e = cudaSuccess;
+        if (b[p].token == me) {
+            // a rank of this process: its buffers and events directly
+            echo_dist *o = reinterpret_cast<echo_dist *>(static_cast<uintptr_t>(b[p].self));
+            bool live;
+            {
+                std::lock_guard<std::mutex> lock(g_mu);
+                live = g_live.count(o) != 0;
+            }
+            if (!live) {
+                disconnect(d);
+                return fail(ECHO_ERR_INVALID, "handle %d names a rank of this process that no longer exists", p);
+            }
+            if (o->device != d->device) {
+                e = cudaDeviceEnablePeerAccess(o->device, 0);
+                if (e == cudaErrorPeerAccessAlreadyEnabled) {
+                    cudaGetLastError();
+                    e = cudaSuccess;
+                }
+                if (e != cudaSuccess) {
+                    cudaGetLastError();
+                    disconnect(d);
+                    return cuda_fail(e, "cudaDeviceEnablePeerAccess");
+                }
+            }
+            d->peer[p] = o->xbuf;
+            for (int k = 0; k < 3; k++)
+                d->peer_done[p][k] = o->done[k];
+            continue;
+        }
         void *ptr = nullptr;
-        cudaError_t e = cudaIpcOpenMemHandle(&ptr, h, cudaIpcMemLazyEnablePeerAccess);
+        e = cudaIpcOpenMemHandle(&ptr, b[p].mem, cudaIpcMemLazyEnablePeerAccess);
+        if (e == cudaSuccess) {
+            d->peer[p] = static_cast<const uint8_t *>(ptr);
+            d->peer_ipc[p] = true;
+            for (int k = 0; k < 3 && e == cudaSuccess; k++)
+                e = cudaIpcOpenEventHandle(&d->peer_done[p][k], b[p].ev[k]);
+        }
         if (e != cudaSuccess) {
             cudaGetLastError();
-            for (int q = 0; q < p; q++)
-                if (q != d->rank && d->peer[q]) {
-                    cudaIpcCloseMemHandle(const_cast<uint8_t *>(d->peer[q]));
-                    d->peer[q] = nullptr;
-                }
-            return cuda_fail(e, "cudaIpcOpenMemHandle");
+            if (ptr && !d->peer_ipc[p])
+                cudaIpcCloseMemHandle(ptr);
+            disconnect(d);
+            return cuda_fail(e, "cudaIpcOpenMemHandle / cudaIpcOpenEventHandle");
         }
-        d->peer[p] = static_cast<const uint8_t *>(ptr);
     }
     d->connected = true;
     return ECHO_OK;
@@ -366,23 +526,33 @@ int echo_dist_stage(echo_dist *d, int stage, const void *x, void *out, int phase
     if (phase != ECHO_FWD && phase != ECHO_BWD)
         return fail(ECHO_ERR_INVALID, "phase %d is neither ECHO_FWD (0) nor ECHO_BWD (1)", phase);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    switch (stage) {
-    case 1:
-        if ((rc = check_user_buffer(x, d->device, "x")) != ECHO_OK)
-            return rc;
-        return stage1(d, x, phase, st);
-    case 2:
-        return stage2(d, phase, st);
-    case 3:
-        if ((rc = check_user_buffer(out, d->device, "out")) != ECHO_OK)
-            return rc;
-        rc = stage3(d, out, st);
-        if (rc == ECHO_OK)
-            d->calls += 1;
-        return rc;
-    default:
+    if (stage < 1 || stage > 3)
         return fail(ECHO_ERR_INVALID, "stage %d is not 1, 2 or 3", stage);
+    if (stage == 1 && (rc = check_user_buffer(x, d->device, "x")) != ECHO_OK)
+        return rc;
+    if (stage == 3 && (rc = check_user_buffer(out, d->device, "out")) != ECHO_OK)
+        return rc;
+    // the events of the stages this one depends on, on every rank
+    const int deps[3][2] = {{2, 0}, {1, 3}, {2, 0}}; // stage numbers, 0 = none
+    for (int j = 0; j < 2; j++) {
+        const int dep = deps[stage - 1][j];
+        if (!dep)
+            continue;
+        for (int p = 0; p < d->world; p++) {
+            cudaError_t e = cudaStreamWaitEvent(st, d->peer_done[p][dep - 1], 0);
+            if (e != cudaSuccess)
+                return cuda_fail(e, "cudaStreamWaitEvent");
+        }
     }
+    rc = stage == 1 ? stage1(d, x, phase, st) : stage == 2 ? stage2(d, phase, st) : stage3(d, out, st);
+    if (rc != ECHO_OK)
+        return rc;
+    cudaError_t e = cudaEventRecord(d->done[stage - 1], st);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "cudaEventRecord");
+    if (stage == 3)
+        d->calls += 1;
+    return ECHO_OK;
 }
 
 int echo_dist_set_params(echo_dist *d, float beta_fast, float beta_slow, float lambda, int enable)
@@ -433,12 +603,12 @@ int echo_dist_get_state(echo_dist *d, int phase, float *f_host, float *s_host)
         return rc;
     if (phase != ECHO_FWD && phase != ECHO_BWD)
         return fail(ECHO_ERR_INVALID, "phase %d is neither ECHO_FWD (0) nor ECHO_BWD (1)", phase);
-    const float *f = d->state + static_cast<size_t>(phase) * 2 * d->n + d->rank * d->seg;
+    const float *f = d->state + static_cast<size_t>(phase) * 2 * d->seg;
     cudaError_t e = cudaDeviceSynchronize();
     if (e == cudaSuccess && f_host)
         e = cudaMemcpy(f_host, f, d->seg * sizeof(float), cudaMemcpyDeviceToHost);
     if (e == cudaSuccess && s_host)
-        e = cudaMemcpy(s_host, f + d->n, d->seg * sizeof(float), cudaMemcpyDeviceToHost);
+        e = cudaMemcpy(s_host, f + d->seg, d->seg * sizeof(float), cudaMemcpyDeviceToHost);
     return e == cudaSuccess ? ECHO_OK : cuda_fail(e, "echo_dist_get_state");
 }
 

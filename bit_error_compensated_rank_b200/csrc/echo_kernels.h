@@ -15,8 +15,9 @@
 
 // Pipeline shapes, chosen by sweeping on B200 at P = 8, 1 GiB per rank
 // (larger bulk copies win as long as two CTAs fit on an SM).
-// ECHO_K1_TILE is kernel 1's tile length in elements when a tile of all P
-// partials is at most 16 bytes per element (halved, quartered beyond).
+// ECHO_K1_TILE is kernel 1's tile length in elements when the P partials of
+// an element take 16 bytes (longer below, shorter beyond, within the CTA's
+// shared-memory budget).
 // ECHO_K2_CHUNKS is kernel 2's chunks of 8 elements per consumer thread per
 // tile, reduced for large P so that ECHO_K2_STAGES stages fit in shared
 // memory; a reduced tile then takes as many stages as fit, up to
@@ -26,6 +27,20 @@
 #endif
 #ifndef ECHO_K1_STAGES
 #define ECHO_K1_STAGES 2
+#endif
+// Kernel 1's consumer warps: the default build (bound by HBM; 16 warps
+// measured 7 % slower), the power-of-two group-size variants, and the
+// binary16-scale variants. The last two have longer dependency chains per
+// item (more shuffles for large groups; the binary16 scale, reciprocal and
+// code settling) and want more warps per SM to hide them.
+#ifndef ECHO_K1_WARPS
+#define ECHO_K1_WARPS 8
+#endif
+#ifndef ECHO_K1_WARPS_GROUPS
+#define ECHO_K1_WARPS_GROUPS 16
+#endif
+#ifndef ECHO_K1_WARPS_HALF_SCALE
+#define ECHO_K1_WARPS_HALF_SCALE 16
 #endif
 #ifndef ECHO_K2_STAGES
 #define ECHO_K2_STAGES 2
@@ -63,8 +78,8 @@ struct PipeCtl {
 
 struct K1Args {
     RankPtrs x;              // P rank partials (bf16 or binary32), n elements each
-    const float *f;          // phase state, fast estimate [n]
-    const float *s;          // phase state, slow estimate [n]
+    const float *f;          // phase state, fast estimate, of the elements the launch's ranks
+    const float *s;          // own, from rank_base's segment on: [n] for P ranks, [n/P] for one
     uint8_t *codes;          // stage-1 wire codes [P][n/2]
     uint8_t *scales;         // stage-1 wire scales [P][scale_stride]: n/G bytes or binary16s per rank
     size_t n;

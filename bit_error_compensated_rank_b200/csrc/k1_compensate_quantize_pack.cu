@@ -18,8 +18,10 @@ cudaError_t launch_k1_compensate_quantize_pack(const K1Args &a, cudaStream_t st)
         return a.sender_ef ? launch_k1_variant_fp32_ef(a, st) : launch_k1_variant_fp32(a, st);
     }
     if (a.bf16)
-        return a.sender_ef ? dispatch_ranks<true, true, false>(a, st) : dispatch_ranks<true, false, false>(a, st);
-    return a.sender_ef ? dispatch_ranks<false, true, false>(a, st) : dispatch_ranks<false, false, false>(a, st);
+        return a.sender_ef ? dispatch_ranks<true, true, kDefaultBuild>(a, st)
+                         : dispatch_ranks<true, false, kDefaultBuild>(a, st);
+    return a.sender_ef ? dispatch_ranks<false, true, kDefaultBuild>(a, st)
+                     : dispatch_ranks<false, false, kDefaultBuild>(a, st);
 }
 
 } // namespace echo

@@ -22,14 +22,16 @@
 // consecutive elements. One producer warp bulk-copies the P partial tiles
 // (and the f, s tiles, and the P error tiles, when used) of a tile into one
 // stage of a kStages ring in shared memory (mbarrier full[s] counts the
-// bytes); eight consumer warps compute from shared memory and release the
-// stage on mbarrier empty[s]. A lane owns 8 consecutive elements of one rank;
-// G/8 lanes form a group and find its maximum with log2(G/8) shuffles; codes
-// leave as one coalesced 32-bit store per lane.
+// bytes); consumer warps (8 in the default build, 16 in the variants' builds,
+// whose longer dependency chains want more warps to hide them) compute from
+// shared memory and release the stage on mbarrier empty[s]. A lane owns 8 consecutive
+// elements of one rank; G/8 lanes form a group and find its maximum with
+// log2(G/8) shuffles; codes leave as one coalesced 32-bit store per lane.
 //
 // Algorithmic HBM bytes per element of n: P*b (partials) + 8 (f, s; each
 // element is corrected by exactly one rank) read, P*17/32 written; sender
-// feedback adds 4P read and 4P written.
+// feedback adds 4P read and 4P written. A one-rank launch (one handle per
+// rank) reads the state of its own segment only: 8/P bytes per element.
 #pragma once
 
 #include "echo_bulk.cuh"
@@ -46,9 +48,19 @@
 namespace echo {
 namespace {
 
-constexpr int kConsumerWarps = 8;
-constexpr int kConsumers = kConsumerWarps * 32;
-constexpr int kThreads = kConsumers + 32; // + one producer warp
+// The kernel's three builds: the default one (groups of 32, power-of-two
+// scales) and the general one, split into its power-of-two group sizes and
+// its binary16-scale bodies, which get their own count of consumer warps.
+enum K1Build { kDefaultBuild = 0, kGroupsBuild = 1, kHalfScaleBuild = 2 };
+
+template <int B>
+struct K1Warps {
+    static constexpr int kConsumerWarps = B == kHalfScaleBuild  ? ECHO_K1_WARPS_HALF_SCALE
+                                          : B == kGroupsBuild   ? ECHO_K1_WARPS_GROUPS
+                                                                : ECHO_K1_WARPS;
+    static constexpr int kConsumers = kConsumerWarps * 32;
+    static constexpr int kThreads = kConsumers + 32; // + one producer warp
+};
 
 // Bytes one stage holds per element of the tile.
 constexpr int k1_bytes_per_elem(int P, bool bf16, bool comp, bool ef)
@@ -56,11 +68,14 @@ constexpr int k1_bytes_per_elem(int P, bool bf16, bool comp, bool ef)
     return P * (bf16 ? 2 : 4) + (comp ? 8 : 0) + (ef ? 4 * P : 0);
 }
 
-// The largest tile (ECHO_K1_TILE, /2, /4, ... down to 256 elements) whose
-// stages fit ECHO_K1_CTA_BUDGET.
+// The largest tile whose stages fit ECHO_K1_CTA_BUDGET, from ECHO_K1_TILE
+// (times 16 / (P * element bytes) when the P partials of an element take
+// fewer than 16 bytes, so that a tile holds about as many partial bytes at
+// small P) down to 256 elements.
 constexpr int k1_tile(int P, bool bf16, bool comp, bool ef)
 {
-    int t = ECHO_K1_TILE;
+    const int xb = P * (bf16 ? 2 : 4);
+    int t = xb < 16 ? ECHO_K1_TILE * (16 / xb) : ECHO_K1_TILE;
     while (t > 256 && ECHO_K1_STAGES * t * k1_bytes_per_elem(P, bf16, comp, ef) > ECHO_K1_CTA_BUDGET)
         t /= 2;
     return t;
@@ -101,8 +116,9 @@ __device__ __forceinline__ void load_f32x8(const float *p, float (&v)[kChunk])
 }
 
 // The consumer warps' part of kernel 1 for a group of 8 << LANES elements and
-// one scale format (F16: binary16 scales), both fixed at compile time.
-template <int P, bool BF16, bool COMP, bool EF, uint32_t LANES, bool F16>
+// one scale format (F16: binary16 scales), both fixed at compile time, run by
+// NC consumer threads.
+template <int P, bool BF16, bool COMP, bool EF, uint32_t LANES, bool F16, int NC>
 __device__ __forceinline__ void k1_consume(const K1Args &a, const uint8_t *smem, uint64_t *full, uint64_t *empty,
                                            uint32_t mine, uint32_t cpt_log2, size_t e0)
 {
@@ -124,7 +140,7 @@ __device__ __forceinline__ void k1_consume(const K1Args &a, const uint8_t *smem,
         const float *es = reinterpret_cast<const float *>(stage + Sh::kEpsOff);
 
 #pragma unroll 2
-        for (uint32_t it = tid; it < (static_cast<uint32_t>(P) << cpt_log2); it += kConsumers) {
+        for (uint32_t it = tid; it < (static_cast<uint32_t>(P) << cpt_log2); it += NC) {
             const uint32_t r = it >> cpt_log2; // warp-uniform (a tile has >= 32 chunks)
             const uint32_t c = it & ((1u << cpt_log2) - 1u);
             const bool active = c < cnt_chunks;
@@ -140,8 +156,11 @@ __device__ __forceinline__ void k1_consume(const K1Args &a, const uint8_t *smem,
                 for (int k = 0; k < kChunk; k++)
                     v[k] = __fadd_rn(v[k], e[k]);
             }
+            // bf16 partials keep 8 significant bits unless something is added
+            bool short_vals = BF16 && !EF;
             // rank r owns groups [r*gps, (r+1)*gps): one unsigned range test
             if (COMP && g - (r + a.rank_base) * a.groups_per_seg < a.groups_per_seg) {
+                short_vals = false;
                 float fv[kChunk], sv[kChunk];
                 load_f32x8(fs + c * kChunk, fv);
                 load_f32x8(fs + Sh::kTile + c * kChunk, sv);
@@ -160,7 +179,7 @@ __device__ __forceinline__ void k1_consume(const K1Args &a, const uint8_t *smem,
                 st = half_step(scale);
                 const float inv = half_inv(st);
                 const float half = __fmul_rn(0.5f, st);
-                codes8_half(v, st, inv, half, half_scale_saturates(amax), qb);
+                codes8_half(v, st, inv, half, half_scale_saturates(amax), short_vals, qb);
             } else {
                 scale = scale_byte(amax);
                 st = step_of(scale);
@@ -201,14 +220,14 @@ __device__ __forceinline__ void k1_consume(const K1Args &a, const uint8_t *smem,
             }
             if (EF && active && in_bounds(chunk < code_words, a.ctl.status)) {
                 // the new error v - q*step (exact unless a binary16 scale saturated)
-                float e[kChunk];
+                float en[kChunk];
 #pragma unroll
                 for (int k = 0; k < kChunk; k++)
-                    e[k] = __fmaf_rn(-code_value(f16 ? zcode_bits(qb[k]) : qb[k]), st, v[k]);
+                    en[k] = __fmaf_rn(-code_value(f16 ? zcode_bits(qb[k]) : qb[k]), st, v[k]);
                 float4 *eo = reinterpret_cast<float4 *>(a.eps + static_cast<size_t>(r) * a.n) +
                              2 * static_cast<size_t>(chunk);
-                eo[0] = make_float4(e[0], e[1], e[2], e[3]);
-                eo[1] = make_float4(e[4], e[5], e[6], e[7]);
+                __stcs(eo, make_float4(en[0], en[1], en[2], en[3]));
+                __stcs(eo + 1, make_float4(en[4], en[5], en[6], en[7]));
             }
         }
         __syncwarp();
@@ -217,11 +236,13 @@ __device__ __forceinline__ void k1_consume(const K1Args &a, const uint8_t *smem,
     }
 }
 
-template <int P, bool BF16, bool COMP, bool EF, bool GEN>
-__global__ void __launch_bounds__(kThreads)
+template <int P, bool BF16, bool COMP, bool EF, int B>
+__global__ void __launch_bounds__(K1Warps<B>::kThreads, 2)
     k1_compensate_quantize_pack(const K1Args a)
 {
     using Sh = K1Shape<P, BF16, COMP, EF>;
+    constexpr int kConsumerWarps = K1Warps<B>::kConsumerWarps;
+    constexpr int NC = K1Warps<B>::kConsumers;
     constexpr int S = Sh::kStages;
     extern __shared__ __align__(128) uint8_t smem[];
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + S * Sh::kStageBytes);
@@ -250,6 +271,12 @@ __global__ void __launch_bounds__(kThreads)
     allow_successor();
 
     if (warp == kConsumerWarps) { // producer
+        // The state holds the elements this launch's ranks own, [state_lo,
+        // state_lo + P*seg): all n for P simulated ranks, one segment for a
+        // one-rank launch. Only the part of a tile inside it is loaded.
+        const size_t seg = static_cast<size_t>(a.groups_per_seg) << (a.lanes_log2 + 3);
+        const size_t state_lo = static_cast<size_t>(a.rank_base) * seg;
+        const size_t state_hi = state_lo + static_cast<size_t>(P) * seg;
         if (lane == 0)
             produce_tiles<S>(full, empty, mine, a.ctl.stall, a.ctl.wait_cycles, a.ctl.status, kStatusTimeoutK1,
                              [&](uint32_t i) {
@@ -257,9 +284,14 @@ __global__ void __launch_bounds__(kThreads)
                                  const uint32_t cnt = static_cast<uint32_t>(e1 - el0 < size_t(tile) ? e1 - el0 : tile);
                                  uint8_t *stage = smem + (i % S) * Sh::kStageBytes;
                                  uint64_t *bar = &full[i % S];
-                                 // every copy below covers elements [el0, el0 + cnt) of an n-element row
+                                 // the partial and error copies cover elements [el0, el0 + cnt) of an
+                                 // n-element row; the state copies [lo, hi), its part inside the state
+                                 const size_t lo = el0 > state_lo ? el0 : state_lo;
+                                 const size_t hi = el0 + cnt < state_hi ? el0 + cnt : state_hi;
+                                 const uint32_t sn = COMP && hi > lo ? static_cast<uint32_t>(hi - lo) : 0u;
                                  const bool ok = in_bounds(el0 + cnt <= a.n && cnt <= Sh::kTile, a.ctl.status);
-                                 mbar_arrive_expect_tx(bar, ok ? cnt * Sh::kStageBytes / Sh::kTile : 0u);
+                                 mbar_arrive_expect_tx(
+                                     bar, ok ? cnt * (P * Sh::kEB + (EF ? 4u * P : 0u)) + 8u * sn : 0u);
                                  if (!ok)
                                      return;
 #pragma unroll
@@ -267,9 +299,11 @@ __global__ void __launch_bounds__(kThreads)
                                      bulk_load(stage + r * Sh::kXBytes,
                                                static_cast<const uint8_t *>(a.x.p[r]) + el0 * Sh::kEB,
                                                cnt * Sh::kEB, bar);
-                                 if (COMP) {
-                                     bulk_load(stage + Sh::kStateOff, a.f + el0, cnt * 4, bar);
-                                     bulk_load(stage + Sh::kStateOff + Sh::kTile * 4, a.s + el0, cnt * 4, bar);
+                                 if (COMP && sn) {
+                                     const size_t off = (lo - el0) * 4;
+                                     bulk_load(stage + Sh::kStateOff + off, a.f + (lo - state_lo), sn * 4, bar);
+                                     bulk_load(stage + Sh::kStateOff + Sh::kTile * 4 + off, a.s + (lo - state_lo),
+                                               sn * 4, bar);
                                  }
                                  if (EF) {
 #pragma unroll
@@ -281,33 +315,37 @@ __global__ void __launch_bounds__(kThreads)
         return;
     }
 
-    if (!GEN) {
-        k1_consume<P, BF16, COMP, EF, 2u, false>(a, smem, full, empty, mine, cpt_log2, e0);
-        return;
-    }
-    // variants: one switch per launch selects the compile-time group size
-    // and scale format (group = 8 << lanes_log2)
-    switch (a.lanes_log2 | (a.fp16_scale ? 8u : 0u)) {
-    case 1u: k1_consume<P, BF16, COMP, EF, 1u, false>(a, smem, full, empty, mine, cpt_log2, e0); break;
-    case 3u: k1_consume<P, BF16, COMP, EF, 3u, false>(a, smem, full, empty, mine, cpt_log2, e0); break;
-    case 4u: k1_consume<P, BF16, COMP, EF, 4u, false>(a, smem, full, empty, mine, cpt_log2, e0); break;
-    case 9u: k1_consume<P, BF16, COMP, EF, 1u, true>(a, smem, full, empty, mine, cpt_log2, e0); break;
-    case 10u: k1_consume<P, BF16, COMP, EF, 2u, true>(a, smem, full, empty, mine, cpt_log2, e0); break;
-    case 11u: k1_consume<P, BF16, COMP, EF, 3u, true>(a, smem, full, empty, mine, cpt_log2, e0); break;
-    case 12u: k1_consume<P, BF16, COMP, EF, 4u, true>(a, smem, full, empty, mine, cpt_log2, e0); break;
-    default: break; // the host accepts no other group size
+    if constexpr (B == kDefaultBuild) {
+        k1_consume<P, BF16, COMP, EF, 2u, false, NC>(a, smem, full, empty, mine, cpt_log2, e0);
+    } else if constexpr (B == kGroupsBuild) {
+        // one switch per launch selects the compile-time group size (8 << lanes_log2)
+        switch (a.lanes_log2) {
+        case 1u: k1_consume<P, BF16, COMP, EF, 1u, false, NC>(a, smem, full, empty, mine, cpt_log2, e0); break;
+        case 3u: k1_consume<P, BF16, COMP, EF, 3u, false, NC>(a, smem, full, empty, mine, cpt_log2, e0); break;
+        case 4u: k1_consume<P, BF16, COMP, EF, 4u, false, NC>(a, smem, full, empty, mine, cpt_log2, e0); break;
+        default: break; // the host accepts no other group size
+        }
+    } else {
+        switch (a.lanes_log2) {
+        case 1u: k1_consume<P, BF16, COMP, EF, 1u, true, NC>(a, smem, full, empty, mine, cpt_log2, e0); break;
+        case 2u: k1_consume<P, BF16, COMP, EF, 2u, true, NC>(a, smem, full, empty, mine, cpt_log2, e0); break;
+        case 3u: k1_consume<P, BF16, COMP, EF, 3u, true, NC>(a, smem, full, empty, mine, cpt_log2, e0); break;
+        case 4u: k1_consume<P, BF16, COMP, EF, 4u, true, NC>(a, smem, full, empty, mine, cpt_log2, e0); break;
+        default: break;
+        }
     }
 }
 
-template <int P, bool BF16, bool COMP, bool EF, bool GEN>
+template <int P, bool BF16, bool COMP, bool EF, int B>
 cudaError_t launch_p(const K1Args &a, cudaStream_t st)
 {
     using Sh = K1Shape<P, BF16, COMP, EF>;
+    constexpr int kThreads = K1Warps<B>::kThreads;
     // CTAs per SM of this instantiation, found once (threads that race here
     // compute the same value)
     static std::atomic<int> cached{0};
     int resident = cached.load(std::memory_order_relaxed);
-    auto kern = k1_compensate_quantize_pack<P, BF16, COMP, EF, GEN>;
+    auto kern = k1_compensate_quantize_pack<P, BF16, COMP, EF, B>;
     if (resident == 0) {
         cudaError_t e = prepare_kernel(reinterpret_cast<const void *>(kern), kThreads, Sh::kSmem, &resident);
         if (e != cudaSuccess)
@@ -322,35 +360,43 @@ cudaError_t launch_p(const K1Args &a, cudaStream_t st)
     return launch_chained(kern, persistent_grid(tiles, resident), kThreads, Sh::kSmem, st, b);
 }
 
-template <int P, bool BF16, bool EF, bool GEN>
+template <int P, bool BF16, bool EF, int B>
 cudaError_t dispatch_state(const K1Args &a, cudaStream_t st)
 {
-    return a.enable ? launch_p<P, BF16, true, EF, GEN>(a, st) : launch_p<P, BF16, false, EF, GEN>(a, st);
+    return a.enable ? launch_p<P, BF16, true, EF, B>(a, st) : launch_p<P, BF16, false, EF, B>(a, st);
 }
 
 // One element type, feedback setting and build of the kernel, over P.
-template <bool BF16, bool EF, bool GEN>
+template <bool BF16, bool EF, int B>
 cudaError_t dispatch_ranks(const K1Args &a, cudaStream_t st)
 {
     switch (a.P) {
-    case 1: return dispatch_state<1, BF16, EF, GEN>(a, st); // one rank per process
-    case 2: return dispatch_state<2, BF16, EF, GEN>(a, st);
-    case 3: return dispatch_state<3, BF16, EF, GEN>(a, st);
-    case 4: return dispatch_state<4, BF16, EF, GEN>(a, st);
-    case 5: return dispatch_state<5, BF16, EF, GEN>(a, st);
-    case 6: return dispatch_state<6, BF16, EF, GEN>(a, st);
-    case 7: return dispatch_state<7, BF16, EF, GEN>(a, st);
-    case 8: return dispatch_state<8, BF16, EF, GEN>(a, st);
-    case 9: return dispatch_state<9, BF16, EF, GEN>(a, st);
-    case 10: return dispatch_state<10, BF16, EF, GEN>(a, st);
-    case 11: return dispatch_state<11, BF16, EF, GEN>(a, st);
-    case 12: return dispatch_state<12, BF16, EF, GEN>(a, st);
-    case 13: return dispatch_state<13, BF16, EF, GEN>(a, st);
-    case 14: return dispatch_state<14, BF16, EF, GEN>(a, st);
-    case 15: return dispatch_state<15, BF16, EF, GEN>(a, st);
-    case 16: return dispatch_state<16, BF16, EF, GEN>(a, st);
+    case 1: return dispatch_state<1, BF16, EF, B>(a, st); // one rank per process
+    case 2: return dispatch_state<2, BF16, EF, B>(a, st);
+    case 3: return dispatch_state<3, BF16, EF, B>(a, st);
+    case 4: return dispatch_state<4, BF16, EF, B>(a, st);
+    case 5: return dispatch_state<5, BF16, EF, B>(a, st);
+    case 6: return dispatch_state<6, BF16, EF, B>(a, st);
+    case 7: return dispatch_state<7, BF16, EF, B>(a, st);
+    case 8: return dispatch_state<8, BF16, EF, B>(a, st);
+    case 9: return dispatch_state<9, BF16, EF, B>(a, st);
+    case 10: return dispatch_state<10, BF16, EF, B>(a, st);
+    case 11: return dispatch_state<11, BF16, EF, B>(a, st);
+    case 12: return dispatch_state<12, BF16, EF, B>(a, st);
+    case 13: return dispatch_state<13, BF16, EF, B>(a, st);
+    case 14: return dispatch_state<14, BF16, EF, B>(a, st);
+    case 15: return dispatch_state<15, BF16, EF, B>(a, st);
+    case 16: return dispatch_state<16, BF16, EF, B>(a, st);
     default: return cudaErrorInvalidValue;
     }
+}
+
+// The general build: the power-of-two group sizes or the binary16 bodies.
+template <bool BF16, bool EF>
+cudaError_t dispatch_variant(const K1Args &a, cudaStream_t st)
+{
+    return a.fp16_scale ? dispatch_ranks<BF16, EF, kHalfScaleBuild>(a, st)
+                        : dispatch_ranks<BF16, EF, kGroupsBuild>(a, st);
 }
 
 } // namespace

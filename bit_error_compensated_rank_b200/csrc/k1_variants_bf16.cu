@@ -6,7 +6,7 @@ namespace echo {
 
 cudaError_t launch_k1_variant_bf16(const K1Args &a, cudaStream_t st)
 {
-    return dispatch_ranks<true, false, true>(a, st);
+    return dispatch_variant<true, false>(a, st);
 }
 
 } // namespace echo

@@ -6,7 +6,7 @@ namespace echo {
 
 cudaError_t launch_k1_variant_bf16_ef(const K1Args &a, cudaStream_t st)
 {
-    return dispatch_ranks<true, true, true>(a, st);
+    return dispatch_variant<true, true>(a, st);
 }
 
 } // namespace echo

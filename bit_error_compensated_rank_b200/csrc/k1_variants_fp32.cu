@@ -6,7 +6,7 @@ namespace echo {
 
 cudaError_t launch_k1_variant_fp32(const K1Args &a, cudaStream_t st)
 {
-    return dispatch_ranks<false, false, true>(a, st);
+    return dispatch_variant<false, false>(a, st);
 }
 
 } // namespace echo

@@ -6,7 +6,7 @@ namespace echo {
 
 cudaError_t launch_k1_variant_fp32_ef(const K1Args &a, cudaStream_t st)
 {
-    return dispatch_ranks<false, true, true>(a, st);
+    return dispatch_variant<false, true>(a, st);
 }
 
 } // namespace echo

@@ -252,7 +252,7 @@ __global__ void __launch_bounds__(kThreads)
                 const float st = half_step(scale);
                 const float inv = half_inv(st);
                 const float half = __fmul_rn(0.5f, st);
-                codes8_half(S_, st, inv, half, half_scale_saturates(amax), qb);
+                codes8_half(S_, st, inv, half, half_scale_saturates(amax), false, qb);
 #pragma unroll
                 for (int k = 0; k < kChunk; k++) {
                     qb[k] = zcode_bits(qb[k]);

@@ -54,7 +54,7 @@ EXPORTED = (
     "echo_dist_set_params", "echo_dist_set_variant", "echo_dist_get_state",
     "echo_dist_device_status", "echo_dist_destroy",
 )
-ECHO_IPC_HANDLE_BYTES = 64
+ECHO_DIST_HANDLE_BYTES = 320
 
 _vp = ctypes.c_void_p
 _sz = ctypes.c_size_t
@@ -444,14 +444,34 @@ class Echo:
             pass
 
 
-# ---- one process per rank ---------------------------------------------------
+# ---- one rank per handle (several processes, or several ranks per process) ----
+def dist_allreduce(handles, xs, outs, barrier, phase: int = ECHO_FWD, stream=None, sync: bool = False) -> None:
+    """One call of the ranks ``handles`` held by this process (one or more),
+    with their partials ``xs`` and outputs ``outs``: every local rank's stage
+    1, ``barrier()``, every local rank's stage 2, ``barrier()``, every local
+    rank's stage 3. The library orders the stages on the GPU with events;
+    the two barriers only make sure every rank, in every process, has enqueued
+    a stage before any enqueues the next, so the host never waits for the
+    GPU. ``sync=True`` is the host-ordered form kept for comparison: it waits
+    for the stream before each barrier and adds one after stage 3."""
+    import torch
+    st = stream if stream is not None else torch.cuda.current_stream()
+    for k in (1, 2, 3):
+        for d, x, out in zip(handles, xs, outs):
+            d.stage(k, x, out, phase, st)
+        if sync:
+            st.synchronize()
+        if k < 3 or sync:
+            barrier()
+
+
 class DistEcho:
-    """One rank of an all-reduce whose ranks are separate processes (the
+    """One rank of an all-reduce whose ranks are separate handles (the
     echo_dist_* entry points): ``DistEcho(world, rank, n, dtype)``, exchange
-    the IPC handles (``export`` on every rank, then ``connect`` with all of
-    them in rank order), then :meth:`allreduce`. ``barrier`` is a callable
-    that returns when every rank has called it (``torch.distributed.barrier``
-    in practice); the stages are ordered across processes with it."""
+    the blobs (``export`` on every rank, then ``connect`` with all of them in
+    rank order), then :meth:`allreduce`. ``barrier`` is a callable that
+    returns when every rank has called it (``torch.distributed.barrier`` on a
+    gloo group, in practice)."""
 
     def __init__(self, world: int, rank: int, n: int, dtype: int = ECHO_BF16, group: int = ECHO_GROUP):
         self.world, self.rank, self.n, self.dtype, self.group = world, rank, n, dtype, group
@@ -462,14 +482,14 @@ class DistEcho:
         self.h = h
 
     def export(self) -> bytes:
-        buf = (ctypes.c_uint8 * ECHO_IPC_HANDLE_BYTES)()
+        buf = (ctypes.c_uint8 * ECHO_DIST_HANDLE_BYTES)()
         _check(_lib.echo_dist_export(self.h, buf))
         return bytes(buf)
 
     def connect(self, handles) -> None:
-        if len(handles) != self.world or any(len(b) != ECHO_IPC_HANDLE_BYTES for b in handles):
-            raise EchoError(ECHO_ERR_INVALID, f"need {self.world} handles of {ECHO_IPC_HANDLE_BYTES} bytes")
-        blob = (ctypes.c_uint8 * (self.world * ECHO_IPC_HANDLE_BYTES)).from_buffer_copy(b"".join(handles))
+        if len(handles) != self.world or any(len(b) != ECHO_DIST_HANDLE_BYTES for b in handles):
+            raise EchoError(ECHO_ERR_INVALID, f"need {self.world} blobs of {ECHO_DIST_HANDLE_BYTES} bytes")
+        blob = (ctypes.c_uint8 * (self.world * ECHO_DIST_HANDLE_BYTES)).from_buffer_copy(b"".join(handles))
         _check(_lib.echo_dist_connect(self.h, blob))
 
     def _check_tensor(self, t, what: str) -> None:
@@ -485,15 +505,9 @@ class DistEcho:
         _check(_lib.echo_dist_stage(self.h, stage, x.data_ptr() if stage == 1 else None,
                                     out.data_ptr() if stage == 3 else None, phase, _stream(stream)))
 
-    def allreduce(self, x, out, barrier, phase: int = ECHO_FWD, stream=None) -> None:
-        """One call: each stage, then wait for this rank's stream and for
-        every rank (the next stage reads the others' buffers)."""
-        import torch
-        st = stream if stream is not None else torch.cuda.current_stream()
-        for k in (1, 2, 3):
-            self.stage(k, x, out, phase, st)
-            st.synchronize()
-            barrier()
+    def allreduce(self, x, out, barrier, phase: int = ECHO_FWD, stream=None, sync: bool = False) -> None:
+        """One call of this rank (see :func:`dist_allreduce`)."""
+        dist_allreduce([self], [x], [out], barrier, phase, stream, sync)
 
     def set_params(self, beta_fast=0.5, beta_slow=0.875, lam=0.5, enable=True) -> None:
         _check(_lib.echo_dist_set_params(self.h, beta_fast, beta_slow, lam, int(bool(enable))))

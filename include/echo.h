@@ -357,12 +357,18 @@ ECHO_API int echo_debug_build(void);
 ECHO_API int echo_debug_touch_guard(echo_handle *h);
 
 /*
- * One process per rank (echo_dist_*). The same all-reduce when each of the
- * world ranks is its own process holding only its own partial; every rank
- * keeps the compensator state of the segment it owns, [rank*n/world,
- * (rank+1)*n/world). Every rank exports a block (CUDA IPC) that the others
- * write into: a receive slot per rank for the owned segment's stage-1 wire,
- * and the gathered requantised tensor. A call runs in three stages:
+ * One rank per handle (echo_dist_*): the same all-reduce when each of the
+ * world ranks holds only its own partial, as on a real tensor-parallel
+ * group [rit.work "Echo 4-bit GPU communication", sections "How Echo returns
+ * the error to later calls" (segments go to their owner, the owner's 4-bit
+ * total goes back to every rank) and "When the gain changes the
+ * infrastructure plan" (the exchange crosses NVLink, PCIe or the network)].
+ * Ranks may be separate processes (one per GPU, or several sharing a GPU) or
+ * several handles in one process. Every rank keeps the compensator state of
+ * the segment it owns, [rank*n/world, (rank+1)*n/world), and exports a block
+ * that the others write into: a receive slot per rank for the owned segment's
+ * stage-1 wire, and the gathered requantised tensor. A call runs in three
+ * stages:
  *   stage 1  kernel 1 rounds this rank's partial x and stores each segment's
  *            codes and scales straight into its owner's receive slot;
  *   stage 2  kernel 2 sums the owned segment from the receive slots,
@@ -370,37 +376,49 @@ ECHO_API int echo_debug_touch_guard(echo_handle *h);
  *            requantised segment into every rank's gathered tensor;
  *   stage 3  kernel 3 writes the result (n elements, identical on every rank)
  *            from the local gathered tensor to out.
- * The wire moves as plain stores into the other processes' blocks (on
- * several GPUs, peer stores over NVLink); the kernels read local memory only,
- * and no kernel waits on another process. The caller
- * orders the stages across processes: after each stage, synchronise the
- * stream, then a host barrier over all ranks (also after stage 3, before the
- * next call's stage 1). The results are bit for bit those of echo_allreduce
- * on the same partials.
+ * The wire moves as plain stores into the other ranks' blocks (on several
+ * GPUs, peer stores over NVLink); the kernels read local memory only, and no
+ * kernel waits on another rank or spins on a flag.
+ * Ordering: every rank records an event after each of its stages (CUDA IPC
+ * events across processes), and each stage first makes its stream wait for
+ * the events it depends on, on every rank (stage 1 on the stage-2 events of
+ * the previous call, stage 2 on the stage-1 and the previous call's stage-3
+ * events, stage 3 on the stage-2 events). A wait takes an event's latest
+ * record when it is enqueued, so the caller puts a host barrier over all
+ * ranks after every rank has enqueued stage 1, and again after stage 2,
+ * of every call. Nothing waits for the GPU: the stream of each rank carries
+ * the ordering. The results are bit for bit those of echo_allreduce on the
+ * same partials.
  *
  * echo_dist_create(world, rank, n, group, dtype): world in [2, 16], rank in
  *   [0, world), n a positive multiple of world x max(group, 32) (segments of
  *   whole groups whose code rows start on 16 bytes), group and dtype as for
  *   echo_create. Allocates on the current device, NULL on error.
- * echo_dist_export: the CUDA IPC handle (ECHO_IPC_HANDLE_BYTES bytes) of this
- *   rank's exported block (its receive slots and its gathered tensor).
- * echo_dist_connect: handles = world handles in rank order (this rank's own
- *   entry is ignored); opens the others' buffers. Once per handle.
+ * echo_dist_export: writes ECHO_DIST_HANDLE_BYTES bytes that describe this
+ *   rank to the others: the CUDA IPC handles of its block and of its three
+ *   stage events, its process, its rank, world, n, group and dtype.
+ * echo_dist_connect: handles = world such blobs in rank order (this rank's
+ *   own entry is ignored). Blobs from this process are used directly (their
+ *   handles must stay alive while this one is used); the others are opened
+ *   through CUDA IPC. A blob whose rank, world, n, group or dtype does not
+ *   match is rejected with ECHO_ERR_INVALID. Once per handle.
  * echo_dist_stage(d, stage, x, out, phase, stream): x (stage 1) and out
  *   (stage 3) are device pointers to n elements of dtype, 16-byte aligned
- *   (unused in the other stages; out may equal x).
+ *   (unused in the other stages; out may equal x). The three stages of a
+ *   rank's call go on one stream, or on streams the caller orders.
  * echo_dist_set_params / echo_dist_set_variant: as echo_set_params and
  *   echo_set_variant, for this rank (every rank must use the same settings).
  * echo_dist_get_state: the owned segment's two estimates (n/world binary32
  *   each) of a phase, synchronous.
  * echo_dist_device_status: as echo_device_status.
- * echo_dist_destroy: closes the peers' buffers and frees this rank's (call
- *   on every rank after a final barrier).
+ * echo_dist_destroy: closes the peers' buffers and events and frees this
+ *   rank's (call on every rank after its stream is idle and after a final
+ *   barrier).
  */
-#define ECHO_IPC_HANDLE_BYTES 64
+#define ECHO_DIST_HANDLE_BYTES 320
 typedef struct echo_dist echo_dist; /* opaque */
 ECHO_API echo_dist *echo_dist_create(int world, int rank, size_t n, int group, int dtype);
-ECHO_API int echo_dist_export(echo_dist *d, uint8_t handle[ECHO_IPC_HANDLE_BYTES]);
+ECHO_API int echo_dist_export(echo_dist *d, uint8_t handle[ECHO_DIST_HANDLE_BYTES]);
 ECHO_API int echo_dist_connect(echo_dist *d, const uint8_t *handles);
 ECHO_API int echo_dist_stage(echo_dist *d, int stage, const void *x, void *out, int phase, void *stream);
 ECHO_API int echo_dist_set_params(echo_dist *d, float beta_fast, float beta_slow, float lambda, int enable);

@@ -1,7 +1,8 @@
-"""One rank of the one-process-per-rank tests (tests/test_dist_gpu.py): run
-as a spawned process, it all-reduces its own partial with the others through
-the echo_dist_* entry points and checks its result and its owned state
-against the oracle, computed here from the same seeded inputs."""
+"""Ranks of the one-rank-per-handle tests (tests/test_dist_gpu.py): run as a
+spawned process (or called directly for a single process), it holds one or
+more consecutive ranks, all-reduces their partials with the other ranks
+through the echo_dist_* entry points and checks every held rank's result and
+owned state against the oracle, computed here from the same seeded inputs."""
 from __future__ import annotations
 
 import datetime
@@ -9,7 +10,8 @@ import datetime
 import numpy as np
 
 
-def run(rank: int, world: int, port: int, n: int, dtype: str, variant: int, calls: int, group: int):
+def run(proc: int, nprocs: int, port: int, world: int, n: int, dtype: str, variant: int, calls: int,
+        group: int, sync: bool = False):
     import torch
     import torch.distributed as dist
 
@@ -18,44 +20,65 @@ def run(rank: int, world: int, port: int, n: int, dtype: str, variant: int, call
     from gpu_harness import assert_same_bits
     from oracle.oracle import Oracle, Params
 
-    dist.init_process_group("gloo", rank=rank, world_size=world, init_method=f"tcp://127.0.0.1:{port}",
-                            timeout=datetime.timedelta(seconds=120))
+    if nprocs > 1:
+        dist.init_process_group("gloo", rank=proc, world_size=nprocs, init_method=f"tcp://127.0.0.1:{port}",
+                                timeout=datetime.timedelta(seconds=120))
+        barrier = dist.barrier
+    else:
+        def barrier():
+            return None
     try:
         torch.cuda.set_device(0)
-        d = echo.DistEcho(world, rank, n, echo.ECHO_BF16 if dtype == "bf16" else echo.ECHO_FP32, group)
-        if variant:
-            d.set_variant(variant)
-        handles = [None] * world
-        dist.all_gather_object(handles, d.export())
-        d.connect(handles)
+        per = world // nprocs
+        mine = list(range(proc * per, (proc + 1) * per))
+        code = echo.ECHO_BF16 if dtype == "bf16" else echo.ECHO_FP32
+        ds = [echo.DistEcho(world, r, n, code, group) for r in mine]
+        for d in ds:
+            if variant:
+                d.set_variant(variant)
+        blobs = [d.export() for d in ds]
+        if nprocs > 1:
+            gathered = [None] * nprocs
+            dist.all_gather_object(gathered, blobs)
+            blobs = [b for part in gathered for b in part]
+        for d in ds:
+            d.connect(blobs)
         orc = Oracle()
         f = {ph: np.zeros(n, np.float32) for ph in (0, 1)}
         s = {ph: np.zeros(n, np.float32) for ph in (0, 1)}
         eps = {ph: np.zeros((world, n), np.float32) for ph in (0, 1)}
-        seg = slice(rank * (n // world), (rank + 1) * (n // world))
         for k in range(calls):
             phase = (k // 2) & 1
             xs = wl.outlier_gaussian(world, n, seed=60 + world, call=k, dtype=dtype)  # every rank's partial
-            mine = np.ascontiguousarray(xs[rank])
-            if dtype == "bf16":
-                x = torch.from_numpy(mine.view(np.int16)).cuda().view(torch.bfloat16)
-            else:
-                x = torch.from_numpy(mine).cuda()
-            out = torch.empty_like(x) if k % 3 else x  # in place every third call
-            d.allreduce(x, out, dist.barrier, phase=phase)
+            xt, outs = [], []
+            for r in mine:
+                part = np.ascontiguousarray(xs[r])
+                if dtype == "bf16":
+                    x = torch.from_numpy(part.view(np.int16)).cuda().view(torch.bfloat16)
+                else:
+                    x = torch.from_numpy(part).cuda()
+                xt.append(x)
+                outs.append(torch.empty_like(x) if k % 3 else x)  # in place every third call
+            echo.dist_allreduce(ds, xt, outs, barrier, phase=phase, sync=sync)
             ref = orc.allreduce(xs, f[phase], s[phase], Params(), G=group, variant=variant, eps=eps[phase])
-            got = out.view(torch.int16).cpu().numpy().view(np.uint16) if dtype == "bf16" else out.cpu().numpy()
-            assert_same_bits(got, ref["out"], f"rank {rank} call {k} output")
-            for ph in (0, 1):
-                gf, gs = d.get_state(ph)
-                assert_same_bits(gf, f[ph][seg], f"rank {rank} call {k} fast estimate phase {ph}")
-                assert_same_bits(gs, s[ph][seg], f"rank {rank} call {k} slow estimate phase {ph}")
-            assert d.device_status(clear=True) == 0
-        dist.barrier()
-        d.close()
+            for r, d, out in zip(mine, ds, outs):
+                got = out.view(torch.int16).cpu().numpy().view(np.uint16) if dtype == "bf16" \
+                    else out.cpu().numpy()
+                assert_same_bits(got, ref["out"], f"rank {r} call {k} output")
+                seg = slice(r * (n // world), (r + 1) * (n // world))
+                for ph in (0, 1):
+                    gf, gs = d.get_state(ph)
+                    assert_same_bits(gf, f[ph][seg], f"rank {r} call {k} fast estimate phase {ph}")
+                    assert_same_bits(gs, s[ph][seg], f"rank {r} call {k} slow estimate phase {ph}")
+                assert d.device_status(clear=True) == 0
+        torch.cuda.synchronize()
+        barrier()
+        for d in ds:
+            d.close()
     finally:
-        dist.barrier()
-        dist.destroy_process_group()
+        if nprocs > 1:
+            dist.barrier()
+            dist.destroy_process_group()
 
 
 def free_port() -> int:
@@ -63,4 +86,3 @@ def free_port() -> int:
     with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as sock:
         sock.bind(("127.0.0.1", 0))
         return sock.getsockname()[1]
-

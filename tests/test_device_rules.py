@@ -15,7 +15,10 @@ shortcuts whose exactness rests on an argument, written beside them in
 * code: z = RN(v * inv + kZ) keeps the code in byte 2 and a 16-bit fraction
   below it; when that fraction is at least kZMargin units of 2^-16 from a
   midpoint, the code is the exact nearest one, whatever error up to 2^-23
-  the reciprocal estimate inv carries.
+  the reciprocal estimate inv carries;
+* code of a value with 8 significant bits (a bf16 partial that carries no
+  correction): the nearest code unless the fraction is below kZTie, which
+  only an exact midpoint reaches, and then an odd code moves down by one.
 
 This test restates them in binary64 and long double, with the constants read
 from the header, and checks them against the oracle on groups with ties,
@@ -30,7 +33,7 @@ import re
 import numpy as np
 import pytest
 
-from bit_error_compensated_rank_b200.workloads import bf16_to_f32, outlier_gaussian
+from bit_error_compensated_rank_b200.workloads import bf16_bits, bf16_to_f32, outlier_gaussian
 from oracle.oracle import FP16_SCALE
 from pins import _many_random_groups, _quantise_rows_with_oracle
 
@@ -89,6 +92,40 @@ def _device_codes(v: np.ndarray, h: np.ndarray, kz: np.float32, margin: int, eta
     return codes, np.repeat(flagged, 8, axis=1)
 
 
+def _zbits(v: np.ndarray, h: np.ndarray, kz: np.float32, eta: float) -> np.ndarray:
+    """Bit patterns of z = RN(v * inv + kZ) for rows v under binary16 steps h,
+    the reciprocal off by the relative error eta."""
+    s = h.astype(np.uint16).view(np.float16).astype(np.float32)
+    inv = np.where(s > 0, np.float32(1) / np.where(s > 0, s, 1), 0).astype(np.float64) * (1 + eta)
+    z = (v.astype(np.longdouble) * inv[:, None].astype(np.longdouble) + np.longdouble(kz)).astype(np.float32)
+    return z.view(np.uint32).astype(np.int64)
+
+
+def _bf16_rows():
+    """Rows of bf16 values below saturation: the benchmark's partials, bf16
+    roundings of wide-range groups, rows of exact midpoints (k + 1/2) * s of
+    few-bit binary16 steps s, and the bf16 values nearest to the midpoints of
+    random binary16 steps (each an exact tie or a near one)."""
+    partials = bf16_to_f32(outlier_gaussian(1, (1 << 15) * G, seed=5, call=0)).reshape(-1, G)
+    mixed = np.clip(_many_random_groups(1 << 14, G, seed=19), -4e5, 4e5).astype(np.float32)
+    mixed = bf16_to_f32(bf16_bits(mixed))
+    g = np.random.default_rng(21)
+    rows = 1 << 14
+    m = g.integers(1, 16, (rows, 1))
+    q = g.integers(-24, 13, (rows, 1))
+    s = m * np.exp2(q.astype(np.float64))          # a binary16 value: 4 bits, 2^-24 .. 61440
+    k = g.integers(-7, 7, (rows, G)) + 0.5          # midpoints -6.5 .. 6.5: 8 bits or fewer
+    mid = k * s
+    mid[:, 0] = 7 * s[:, 0]                         # the maximum makes s the group's step
+    hs = g.integers(0x0001, 0x7800, (rows, 1)).astype(np.uint16).view(np.float16).astype(np.float64)
+    near = (g.integers(-7, 7, (rows, G)) + 0.5) * hs
+    near[:, 0] = 7 * hs[:, 0]
+    near = bf16_to_f32(bf16_bits(near.astype(np.float32)))
+    out = np.concatenate([partials, mixed, mid.astype(np.float32), near]).astype(np.float32)
+    assert np.array_equal(bf16_to_f32(bf16_bits(out)), out)  # every value is a bf16
+    return out
+
+
 def _rows():
     mixed = _many_random_groups(1 << 15, G, seed=9)
     mixed = np.clip(mixed, -4e5, 4e5).astype(np.float32)  # below saturation (7 * 65504)
@@ -137,6 +174,29 @@ def test_binary16_zform_codes_exact_when_not_flagged(oracle):
         assert ties.any() and flagged[ties].all()
     # bf16 partials hold exact ties often enough to matter for the kernel's cost
     assert ties.mean() > 1e-4
+
+
+def test_binary16_codes_of_bf16_values_settle_ties_without_the_exact_path(oracle):
+    """Values of 8 significant bits: the fast code, with an odd code moved
+    down by one where the fraction is below kZTie (exact midpoints only), is
+    the oracle's nearest code for every value, whatever reciprocal error up
+    to 2^-23; and no value other than an exact midpoint reaches kZTie."""
+    kz, margin, _ = _constants()
+    tie_bound = int(re.search(r"constexpr uint32_t kZTie = (\d+);", open(CODEC).read()).group(1))
+    x = _bf16_rows()
+    h, q = _quantise_rows_with_oracle(oracle, x, G, FP16_SCALE)
+    assert (h < 0x7BFF).all()  # no saturated group: those take the exact path
+    s = h.astype(np.uint16).view(np.float16).astype(np.float64)
+    ratio = x.astype(np.float64) / np.where(s > 0, s, 1)[:, None]
+    ties = (s[:, None] > 0) & (ratio - np.floor(ratio) == 0.5)
+    assert ties.sum() > 10000
+    for eta in (0.0, 2.0 ** -23, -(2.0 ** -23)):
+        bits = _zbits(x, h, kz, eta)
+        codes = (bits >> 16) - 0x4340
+        low = bits & 0xFFFF
+        assert np.array_equal(low < tie_bound, ties), eta
+        fixed = codes - ((low < tie_bound) & (codes % 2 != 0))
+        assert np.array_equal(fixed, q), (eta, np.argwhere(fixed != q)[:4])
 
 
 def _device_scale_byte(A: np.ndarray) -> np.ndarray:
