@@ -29,15 +29,19 @@
 #define ECHO_K1_STAGES 2
 #endif
 // Kernel 1's consumer warps: the default build (bound by HBM; 16 warps
-// measured 7 % slower), the power-of-two group-size variants, and the
-// binary16-scale variants. The last two have longer dependency chains per
-// item (more shuffles for large groups; the binary16 scale, reciprocal and
-// code settling) and want more warps per SM to hide them.
+// measured 1 to 7 % slower), the power-of-two group-size variants, the
+// binary16-scale variants, and the default group with sender feedback. The
+// last three have longer chains per item (more shuffles for large groups; the
+// binary16 scale, reciprocal and code settling; the error tiles' loads and
+// stores) and want more warps per SM to hide them.
 #ifndef ECHO_K1_WARPS
 #define ECHO_K1_WARPS 8
 #endif
 #ifndef ECHO_K1_WARPS_GROUPS
 #define ECHO_K1_WARPS_GROUPS 16
+#endif
+#ifndef ECHO_K1_WARPS_SENDER_EF
+#define ECHO_K1_WARPS_SENDER_EF 16
 #endif
 #ifndef ECHO_K1_WARPS_HALF_SCALE
 #define ECHO_K1_WARPS_HALF_SCALE 16

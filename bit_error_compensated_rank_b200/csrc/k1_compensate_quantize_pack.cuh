@@ -22,9 +22,10 @@
 // consecutive elements. One producer warp bulk-copies the P partial tiles
 // (and the f, s tiles, and the P error tiles, when used) of a tile into one
 // stage of a kStages ring in shared memory (mbarrier full[s] counts the
-// bytes); consumer warps (8 in the default build, 16 in the variants' builds,
-// whose longer dependency chains want more warps to hide them) compute from
-// shared memory and release the stage on mbarrier empty[s]. A lane owns 8 consecutive
+// bytes); consumer warps (8 in the default build, 16 in the variants' builds
+// and with sender feedback, whose longer dependency chains want more warps to
+// hide them) compute from shared memory and release the stage on mbarrier
+// empty[s]. A lane owns 8 consecutive
 // elements of one rank; G/8 lanes form a group and find its maximum with
 // log2(G/8) shuffles; codes leave as one coalesced 32-bit store per lane.
 //
@@ -53,10 +54,11 @@ namespace {
 // its binary16-scale bodies, which get their own count of consumer warps.
 enum K1Build { kDefaultBuild = 0, kGroupsBuild = 1, kHalfScaleBuild = 2 };
 
-template <int B>
+template <int B, bool EF>
 struct K1Warps {
     static constexpr int kConsumerWarps = B == kHalfScaleBuild  ? ECHO_K1_WARPS_HALF_SCALE
                                           : B == kGroupsBuild   ? ECHO_K1_WARPS_GROUPS
+                                          : EF                  ? ECHO_K1_WARPS_SENDER_EF
                                                                 : ECHO_K1_WARPS;
     static constexpr int kConsumers = kConsumerWarps * 32;
     static constexpr int kThreads = kConsumers + 32; // + one producer warp
@@ -237,12 +239,12 @@ __device__ __forceinline__ void k1_consume(const K1Args &a, const uint8_t *smem,
 }
 
 template <int P, bool BF16, bool COMP, bool EF, int B>
-__global__ void __launch_bounds__(K1Warps<B>::kThreads, 2)
+__global__ void __launch_bounds__(K1Warps<B, EF>::kThreads, 2)
     k1_compensate_quantize_pack(const K1Args a)
 {
     using Sh = K1Shape<P, BF16, COMP, EF>;
-    constexpr int kConsumerWarps = K1Warps<B>::kConsumerWarps;
-    constexpr int NC = K1Warps<B>::kConsumers;
+    constexpr int kConsumerWarps = K1Warps<B, EF>::kConsumerWarps;
+    constexpr int NC = K1Warps<B, EF>::kConsumers;
     constexpr int S = Sh::kStages;
     extern __shared__ __align__(128) uint8_t smem[];
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + S * Sh::kStageBytes);
@@ -340,7 +342,7 @@ template <int P, bool BF16, bool COMP, bool EF, int B>
 cudaError_t launch_p(const K1Args &a, cudaStream_t st)
 {
     using Sh = K1Shape<P, BF16, COMP, EF>;
-    constexpr int kThreads = K1Warps<B>::kThreads;
+    constexpr int kThreads = K1Warps<B, EF>::kThreads;
     // CTAs per SM of this instantiation, found once (threads that race here
     // compute the same value)
     static std::atomic<int> cached{0};

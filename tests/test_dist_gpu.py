@@ -45,3 +45,36 @@ def test_ranks_in_one_process(world, n, dtype, variant):
     used directly, with no CUDA IPC."""
     import dist_worker
     dist_worker.run(0, 1, 0, world, n, dtype, variant, 6, 32)
+
+
+def test_connect_checks_the_blobs():
+    """echo_dist_connect refuses blobs of another shape or in the wrong rank
+    order, with nothing opened, and accepts the right ones afterwards."""
+    import torch
+
+    from bit_error_compensated_rank_b200 import echo
+    torch.cuda.set_device(0)
+    n = 2 * 32 * 64
+    d0 = echo.DistEcho(2, 0, n)
+    d1 = echo.DistEcho(2, 1, n)
+    other = echo.DistEcho(2, 1, 2 * n)
+    try:
+        for blobs, words in [([d0.export(), other.export()], "expected rank 1"),
+                             ([d1.export(), d0.export()], "expected rank 0")]:
+            with pytest.raises(echo.EchoError) as ei:
+                d0.connect(blobs)
+            assert ei.value.code == echo.ECHO_ERR_INVALID and words in str(ei.value)
+        blobs = [d0.export(), d1.export()]
+        d0.connect(blobs)
+        d1.connect(blobs)
+        with pytest.raises(echo.EchoError):
+            d0.connect(blobs)  # once per handle
+        x = [torch.randn(n, device="cuda").to(torch.bfloat16) for _ in range(2)]
+        out = [torch.empty_like(t) for t in x]
+        echo.dist_allreduce([d0, d1], x, out, lambda: None)
+        torch.cuda.synchronize()
+        assert torch.equal(out[0].view(torch.int16), out[1].view(torch.int16))
+    finally:
+        torch.cuda.synchronize()
+        for d in (d0, d1, other):
+            d.close()

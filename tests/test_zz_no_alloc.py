@@ -19,6 +19,7 @@ tests cover its argument rejections (nothing enqueued) and its status word.
 This file sorts last so a run that stops at the first failure has already
 run everything else; it also passes alone in a fresh process.
 """
+import gc
 import os
 import subprocess
 import sys
@@ -144,16 +145,23 @@ def test_static_calls_allocate_nothing():
 
     call()  # set-up (and first launch of each kernel) happens here
     torch.cuda.synchronize()
-    free0, _ = torch.cuda.mem_get_info()
-    alloc0 = torch.cuda.memory_allocated()
-    reserved0 = torch.cuda.memory_reserved()
-    for _ in range(5):
-        call()
-    torch.cuda.synchronize()
-    free1, _ = torch.cuda.mem_get_info()
-    assert free1 == free0, (free0, free1)
-    assert torch.cuda.memory_allocated() == alloc0
-    assert torch.cuda.memory_reserved() == reserved0
+    # Tensors that earlier tests left in reference cycles would otherwise be
+    # freed whenever the garbage collector runs, moving torch's counters.
+    gc.collect()
+    gc.disable()
+    try:
+        free0, _ = torch.cuda.mem_get_info()
+        alloc0 = torch.cuda.memory_allocated()
+        reserved0 = torch.cuda.memory_reserved()
+        for _ in range(5):
+            call()
+        torch.cuda.synchronize()
+        free1, _ = torch.cuda.mem_get_info()
+        assert free1 == free0, (free0, free1)
+        assert torch.cuda.memory_allocated() == alloc0
+        assert torch.cuda.memory_reserved() == reserved0
+    finally:
+        gc.enable()
     assert echo.echo_static_status() == 0
 
 
