@@ -1,12 +1,12 @@
-// echo_dist.cu - the all-reduce with one process per rank (echo_dist_* in
+// echo_dist.cu - the all-reduce with one handle per rank (echo_dist_* in
 // include/echo.h).
 //
-// Each process holds one rank's partial, the compensator state of the segment
-// it owns, and an exported block that the other processes write into (opened
-// with CUDA IPC): a receive slot per rank for the owned segment's stage-1
-// wire, and the gathered requantised tensor. The three kernels run as three
-// stages, and the wire moves inside them as plain stores into the other
-// processes' blocks [rit.work "Echo 4-bit GPU communication", section "How
+// Each rank (a process, or one of several handles in a process) holds its own
+// partial, the compensator state of the segment it owns, and an exported
+// block that the other ranks write into (through CUDA IPC across processes):
+// a receive slot per rank for the owned segment's stage-1 wire, and the
+// gathered requantised tensor. The three kernels run as three stages, and the
+// wire moves inside them as plain stores into the other ranks' blocks [rit.work "Echo 4-bit GPU communication", section "How
 // Echo returns the error to later calls": segments go to their owner, the
 // owner's compressed total goes back to every rank]:
 //   stage 1  kernel 1 on this rank's partial (one rank, owner mapping of the

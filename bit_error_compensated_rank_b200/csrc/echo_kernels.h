@@ -94,7 +94,7 @@ struct K1Args {
     uint32_t groups_per_seg; // n / P / G: owner of group g is g / groups_per_seg
     uint32_t rank_base;      // global rank of partial 0 (a one-rank launch of a process
                              // that holds one rank of a larger group; 0 otherwise)
-    // One process per rank (P == 1 launches only): the stage-1 row goes
+    // One handle per rank (P == 1 launches only): the stage-1 row goes
     // straight to the owners. Segment s lands in owner s's receive block
     // owners.p[s], in the slot of rank rank_base: codes at
     // rank_base * seg_code_bytes, scales at recv_scales_off + rank_base *
@@ -131,7 +131,7 @@ struct K2Args {
     bool fp16_scale;         // binary16 scales
     bool bf16;               // bf16 outputs: under binary16 scales the error is
                              // taken against the bf16-rounded value ranks receive
-    // One process per rank: the requantised segment goes straight to every
+    // One handle per rank: the requantised segment goes straight to every
     // rank's gathered buffer ranks.p[r] (codes from word q_chunk0, scales at
     // q_scales_off + q_group0 scales), instead of qcodes / qscales.
     bool to_ranks;

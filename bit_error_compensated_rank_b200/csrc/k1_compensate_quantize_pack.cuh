@@ -192,7 +192,7 @@ __device__ __forceinline__ void k1_consume(const K1Args &a, const uint8_t *smem,
             }
             const uint32_t word = f16 ? pack8_zcodes(qb) : pack8_bits(qb); // binary16: z-form codes
             if (P == 1 && a.to_owners) {
-                // one process per rank: straight into the owner's receive block
+                // one handle per rank: straight into the owner's receive block
                 const uint32_t owner = g / a.groups_per_seg;
                 const uint32_t gl = g - owner * a.groups_per_seg;               // group in the segment
                 const uint32_t cl = chunk - ((owner * a.groups_per_seg) << lanes_log2); // chunk in the segment

@@ -287,7 +287,7 @@ __global__ void __launch_bounds__(kThreads)
                 in_bounds(chunk < a.n / kChunk && (size_t(a.q_chunk0) + chunk + 1) * 4u <= a.q_scales_off &&
                               (size_t(a.q_group0) + g + 1) * (F16 ? 2u : 1u) <= a.q_scale_bytes,
                           a.ctl.status)) {
-                // one process per rank: the owned segment straight into every rank's gathered buffer
+                // one handle per rank: the owned segment straight into every rank's gathered buffer
                 const uint32_t word = pack8_bits(qb);
                 const bool first = (lane & ((1u << a.lanes_log2) - 1u)) == 0;
 #pragma unroll
