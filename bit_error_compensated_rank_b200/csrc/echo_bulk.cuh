@@ -185,6 +185,52 @@ __device__ __forceinline__ void produce_tiles(uint64_t *full, uint64_t *empty, u
         mbar_wait_bounded(&full[t % S], (t / S) & 1u, limit);
 }
 
+// produce_tiles with a write-back: the consumers leave results in a stage
+// (written to shared memory, then fence.proxy.async, then their release on
+// empty[s]), and writeback(t) bulk-stores them for local tile t. A stage is
+// refilled only after the stores of its previous tile have read it. After
+// the last tile the producer waits (bounded) for the consumers to release
+// each tile not yet written back, writes it back, and waits until every store
+// has completed before returning. If a consumer wait runs out, the remaining
+// tiles are not written back (the status bit says why) and the producer only
+// waits for their loads to land.
+template <int S, typename Issue, typename WriteBack>
+__device__ __forceinline__ void produce_tiles_writeback(uint64_t *full, uint64_t *empty, uint32_t tiles, bool stall,
+                                                        long long limit, int *status, int status_bit, Issue issue,
+                                                        WriteBack writeback)
+{
+    uint32_t i = 0;
+    bool ok = true;
+    if (!stall) {
+        for (; i < tiles; i++) {
+            const uint32_t s = i % S;
+            if (i >= static_cast<uint32_t>(S)) {
+                if (!mbar_wait_bounded(&empty[s], ((i / S) - 1) & 1u, limit)) {
+                    atomicOr(status, status_bit);
+                    ok = false;
+                    break;
+                }
+                writeback(i - S);
+                bulk_commit();
+                bulk_wait_read<0>(); // the stores have read the stage: it may be refilled
+            }
+            issue(i);
+        }
+    }
+    for (uint32_t t = i > static_cast<uint32_t>(S) ? i - S : 0; t < i; t++) {
+        if (ok && mbar_wait_bounded(&empty[t % S], (t / S) & 1u, limit)) {
+            writeback(t);
+            bulk_commit();
+        } else {
+            if (ok)
+                atomicOr(status, status_bit);
+            ok = false;
+            mbar_wait_bounded(&full[t % S], (t / S) & 1u, limit);
+        }
+    }
+    bulk_wait_all();
+}
+
 // The same ring fed by the whole producer warp: for local tile i, lane 0
 // arms full[i % S] (arm(i): arrive with the tile's byte count), then the
 // tile's ncopies bulk copies are issued by the 32 lanes in parallel

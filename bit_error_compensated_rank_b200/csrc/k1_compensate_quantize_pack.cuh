@@ -28,6 +28,10 @@
 // empty[s]. A lane owns 8 consecutive
 // elements of one rank; G/8 lanes form a group and find its maximum with
 // log2(G/8) shuffles; codes leave as one coalesced 32-bit store per lane.
+// With sender feedback each lane writes its 8 new errors over the old ones
+// in the stage, and the producer bulk-stores the P error tiles once every
+// consumer warp has released the stage, before it refills it: the TMA engine,
+// not the load/store units, carries that 4P bytes per element of writes.
 //
 // Algorithmic HBM bytes per element of n: P*b (partials) + 8 (f, s; each
 // element is corrected by exactly one rank) read, P*17/32 written; sender
@@ -139,7 +143,9 @@ __device__ __forceinline__ void k1_consume(const K1Args &a, const uint8_t *smem,
         const uint32_t cnt_chunks = min(1u << cpt_log2, a.chunk_end - tile_chunk0);
         const uint8_t *stage = smem + s * Sh::kStageBytes;
         const float *fs = reinterpret_cast<const float *>(stage + Sh::kStateOff);
-        const float *es = reinterpret_cast<const float *>(stage + Sh::kEpsOff);
+        // the error tiles: read, then overwritten in place with the new errors,
+        // which the producer bulk-stores once the stage is released
+        float *es = reinterpret_cast<float *>(const_cast<uint8_t *>(stage) + Sh::kEpsOff);
 
 #pragma unroll 2
         for (uint32_t it = tid; it < (static_cast<uint32_t>(P) << cpt_log2); it += NC) {
@@ -220,21 +226,23 @@ __device__ __forceinline__ void k1_consume(const K1Args &a, const uint8_t *smem,
                         row[g] = static_cast<uint8_t>(scale);
                 }
             }
-            if (EF && active && in_bounds(chunk < code_words, a.ctl.status)) {
-                // the new error v - q*step (exact unless a binary16 scale saturated)
+            if (EF && active) {
+                // the new error v - q*step (exact unless a binary16 scale saturated),
+                // over the old one in the stage
                 float en[kChunk];
 #pragma unroll
                 for (int k = 0; k < kChunk; k++)
                     en[k] = __fmaf_rn(-code_value(f16 ? zcode_bits(qb[k]) : qb[k]), st, v[k]);
-                float4 *eo = reinterpret_cast<float4 *>(a.eps + static_cast<size_t>(r) * a.n) +
-                             2 * static_cast<size_t>(chunk);
-                __stcs(eo, make_float4(en[0], en[1], en[2], en[3]));
-                __stcs(eo + 1, make_float4(en[4], en[5], en[6], en[7]));
+                float4 *eo = reinterpret_cast<float4 *>(es + r * Sh::kTile + c * kChunk);
+                eo[0] = make_float4(en[0], en[1], en[2], en[3]);
+                eo[1] = make_float4(en[4], en[5], en[6], en[7]);
             }
         }
+        if (EF)
+            fence_proxy_async_smem(); // the new errors are read next by the producer's bulk stores
         __syncwarp();
         if (lane == 0)
-            mbar_arrive(&empty[s]); // this warp is done reading stage s
+            mbar_arrive(&empty[s]); // this warp is done with stage s
     }
 }
 
@@ -279,41 +287,61 @@ __global__ void __launch_bounds__(K1Warps<B, EF>::kThreads, 2)
         const size_t seg = static_cast<size_t>(a.groups_per_seg) << (a.lanes_log2 + 3);
         const size_t state_lo = static_cast<size_t>(a.rank_base) * seg;
         const size_t state_hi = state_lo + static_cast<size_t>(P) * seg;
-        if (lane == 0)
-            produce_tiles<S>(full, empty, mine, a.ctl.stall, a.ctl.wait_cycles, a.ctl.status, kStatusTimeoutK1,
-                             [&](uint32_t i) {
-                                 const size_t el0 = e0 + static_cast<size_t>(blockIdx.x + i * gridDim.x) * tile;
-                                 const uint32_t cnt = static_cast<uint32_t>(e1 - el0 < size_t(tile) ? e1 - el0 : tile);
-                                 uint8_t *stage = smem + (i % S) * Sh::kStageBytes;
-                                 uint64_t *bar = &full[i % S];
-                                 // the partial and error copies cover elements [el0, el0 + cnt) of an
-                                 // n-element row; the state copies [lo, hi), its part inside the state
-                                 const size_t lo = el0 > state_lo ? el0 : state_lo;
-                                 const size_t hi = el0 + cnt < state_hi ? el0 + cnt : state_hi;
-                                 const uint32_t sn = COMP && hi > lo ? static_cast<uint32_t>(hi - lo) : 0u;
-                                 const bool ok = in_bounds(el0 + cnt <= a.n && cnt <= Sh::kTile, a.ctl.status);
-                                 mbar_arrive_expect_tx(
-                                     bar, ok ? cnt * (P * Sh::kEB + (EF ? 4u * P : 0u)) + 8u * sn : 0u);
-                                 if (!ok)
-                                     return;
+        auto issue = [&](uint32_t i) {
+            const size_t el0 = e0 + static_cast<size_t>(blockIdx.x + i * gridDim.x) * tile;
+            const uint32_t cnt = static_cast<uint32_t>(e1 - el0 < size_t(tile) ? e1 - el0 : tile);
+            uint8_t *stage = smem + (i % S) * Sh::kStageBytes;
+            uint64_t *bar = &full[i % S];
+            // the partial and error copies cover elements [el0, el0 + cnt) of an
+            // n-element row; the state copies [lo, hi), its part inside the state
+            const size_t lo = el0 > state_lo ? el0 : state_lo;
+            const size_t hi = el0 + cnt < state_hi ? el0 + cnt : state_hi;
+            const uint32_t sn = COMP && hi > lo ? static_cast<uint32_t>(hi - lo) : 0u;
+            const bool ok = in_bounds(el0 + cnt <= a.n && cnt <= Sh::kTile, a.ctl.status);
+            mbar_arrive_expect_tx(
+                bar, ok ? cnt * (P * Sh::kEB + (EF ? 4u * P : 0u)) + 8u * sn : 0u);
+            if (!ok)
+                return;
 #pragma unroll
-                                 for (int r = 0; r < P; r++)
-                                     bulk_load(stage + r * Sh::kXBytes,
-                                               static_cast<const uint8_t *>(a.x.p[r]) + el0 * Sh::kEB,
-                                               cnt * Sh::kEB, bar);
-                                 if (COMP && sn) {
-                                     const size_t off = (lo - el0) * 4;
-                                     bulk_load(stage + Sh::kStateOff + off, a.f + (lo - state_lo), sn * 4, bar);
-                                     bulk_load(stage + Sh::kStateOff + Sh::kTile * 4 + off, a.s + (lo - state_lo),
-                                               sn * 4, bar);
-                                 }
-                                 if (EF) {
+            for (int r = 0; r < P; r++)
+                bulk_load(stage + r * Sh::kXBytes,
+                          static_cast<const uint8_t *>(a.x.p[r]) + el0 * Sh::kEB,
+                          cnt * Sh::kEB, bar);
+            if (COMP && sn) {
+                const size_t off = (lo - el0) * 4;
+                bulk_load(stage + Sh::kStateOff + off, a.f + (lo - state_lo), sn * 4, bar);
+                bulk_load(stage + Sh::kStateOff + Sh::kTile * 4 + off, a.s + (lo - state_lo),
+                          sn * 4, bar);
+            }
+            if (EF) {
 #pragma unroll
-                                     for (int r = 0; r < P; r++)
-                                         bulk_load(stage + Sh::kEpsOff + r * Sh::kTile * 4,
-                                                   a.eps + static_cast<size_t>(r) * a.n + el0, cnt * 4, bar);
-                                 }
-                             });
+                for (int r = 0; r < P; r++)
+                    bulk_load(stage + Sh::kEpsOff + r * Sh::kTile * 4,
+                              a.eps + static_cast<size_t>(r) * a.n + el0, cnt * 4, bar);
+            }
+        };
+        if (lane == 0) {
+            if constexpr (EF) {
+                // the new errors go back to global memory by bulk stores from
+                // the released stage, not by the consumers' own stores
+                produce_tiles_writeback<S>(
+                    full, empty, mine, a.ctl.stall, a.ctl.wait_cycles, a.ctl.status, kStatusTimeoutK1, issue,
+                    [&](uint32_t t) {
+                        const size_t el0 = e0 + static_cast<size_t>(blockIdx.x + t * gridDim.x) * tile;
+                        const uint32_t cnt = static_cast<uint32_t>(e1 - el0 < size_t(tile) ? e1 - el0 : tile);
+                        const uint8_t *stage = smem + (t % S) * Sh::kStageBytes;
+                        if (!in_bounds(el0 + cnt <= a.n && cnt <= Sh::kTile, a.ctl.status))
+                            return;
+#pragma unroll
+                        for (int r = 0; r < P; r++)
+                            bulk_store(a.eps + static_cast<size_t>(r) * a.n + el0,
+                                       stage + Sh::kEpsOff + r * Sh::kTile * 4, cnt * 4);
+                    });
+            } else {
+                produce_tiles<S>(full, empty, mine, a.ctl.stall, a.ctl.wait_cycles, a.ctl.status, kStatusTimeoutK1,
+                                 issue);
+            }
+        }
         return;
     }
 
