@@ -66,7 +66,10 @@ constexpr size_t kMaxN = size_t(1) << 34;  // chunk indices stay 32-bit
 // lands in microseconds); the injected stall uses about half a millisecond.
 constexpr long long kWaitCycles = 1LL << 31;
 constexpr long long kStallWaitCycles = 1LL << 20;
-constexpr size_t kHostPiece = size_t(1) << 22; // elements per pipelined host transfer
+#ifndef ECHO_HOST_PIECE_LOG2
+#define ECHO_HOST_PIECE_LOG2 22
+#endif
+constexpr size_t kHostPiece = size_t(1) << ECHO_HOST_PIECE_LOG2; // elements per pipelined host transfer
 constexpr int kVariantBits = ECHO_VARIANT_OWNER_SUM | ECHO_VARIANT_SENDER_EF | ECHO_VARIANT_FP16_SCALE;
 constexpr int kTimingRing = 32;                 // event sets of timed calls in flight
 

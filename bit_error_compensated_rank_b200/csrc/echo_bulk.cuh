@@ -5,7 +5,9 @@
 // issues whole-tile copies, completion is tracked by an mbarrier's
 // transaction count ("full"), consumer warps compute from shared memory and
 // hand each stage back on a second mbarrier ("empty"). No copy uses cluster
-// multicast, and every copy reads or writes only this GPU's memory.
+// multicast, and every bulk load reads this GPU's memory only; the only bulk
+// stores into another rank's memory are kernel 1's code words with one handle
+// per rank and sender feedback (a peer's receive block, on several GPUs).
 //
 // Every wait is bounded in time: a warp that does not see its barrier phase
 // complete within the limit records the failure in the device status word

@@ -31,7 +31,9 @@
 // With sender feedback each lane writes its 8 new errors over the old ones
 // in the stage, and the producer bulk-stores the P error tiles once every
 // consumer warp has released the stage, before it refills it: the TMA engine,
-// not the load/store units, carries that 4P bytes per element of writes.
+// not the load/store units, carries that 4P bytes per element of writes. A
+// one-rank launch (one handle per rank) with sender feedback sends its code
+// words to the owners the same way.
 //
 // Algorithmic HBM bytes per element of n: P*b (partials) + 8 (f, s; each
 // element is corrected by exactly one rank) read, P*17/32 written; sender
@@ -82,7 +84,10 @@ constexpr int k1_tile(int P, bool bf16, bool comp, bool ef)
 {
     const int xb = P * (bf16 ? 2 : 4);
     int t = xb < 16 ? ECHO_K1_TILE * (16 / xb) : ECHO_K1_TILE;
-    while (t > 256 && ECHO_K1_STAGES * t * k1_bytes_per_elem(P, bf16, comp, ef) > ECHO_K1_CTA_BUDGET)
+    // a one-rank tile with sender feedback also holds its code words (half a
+    // byte per element)
+    while (t > 256 && ECHO_K1_STAGES * (t * k1_bytes_per_elem(P, bf16, comp, ef) + (P == 1 && ef ? t / 2 : 0)) >
+                          ECHO_K1_CTA_BUDGET)
         t /= 2;
     return t;
 }
@@ -95,7 +100,8 @@ struct K1Shape {
     static constexpr int kXBytes = kTile * kEB;             // one rank's partial tile
     static constexpr int kStateOff = P * kXBytes;           // f tile, then s tile
     static constexpr int kEpsOff = kStateOff + (COMP ? 2 * kTile * 4 : 0); // P error tiles
-    static constexpr int kStageBytes = kEpsOff + (EF ? P * kTile * 4 : 0);
+    static constexpr int kCodeOff = kEpsOff + (EF ? P * kTile * 4 : 0); // one rank, feedback: code words
+    static constexpr int kStageBytes = kCodeOff + (P == 1 && EF ? kTile / 2 : 0);
     static constexpr int kSmem = kStages * kStageBytes + 2 * kStages * 8;
     static_assert(kSmem <= ECHO_SMEM_BUDGET, "kernel 1 stages exceed shared memory");
 };
@@ -198,15 +204,22 @@ __device__ __forceinline__ void k1_consume(const K1Args &a, const uint8_t *smem,
             }
             const uint32_t word = f16 ? pack8_zcodes(qb) : pack8_bits(qb); // binary16: z-form codes
             if (P == 1 && a.to_owners) {
-                // one handle per rank: straight into the owner's receive block
+                // one handle per rank: into the owner's receive block. With
+                // sender feedback the producer already bulk-stores the error
+                // tiles from the released stage, so the code words go that way
+                // too; otherwise each lane stores its own (a stage waiting for
+                // its stores measured slower there).
                 const uint32_t owner = g / a.groups_per_seg;
                 const uint32_t gl = g - owner * a.groups_per_seg;               // group in the segment
                 const uint32_t cl = chunk - ((owner * a.groups_per_seg) << lanes_log2); // chunk in the segment
+                if (EF && active)
+                    reinterpret_cast<uint32_t *>(const_cast<uint8_t *>(stage) + Sh::kCodeOff)[c] = word;
                 if (active && in_bounds(owner < kMaxRanks && (size_t(gl) + 1) * (f16 ? 2u : 1u) <= a.seg_scale_stride &&
                                             (size_t(cl) + 1) * 4u <= a.seg_code_bytes,
                                         a.ctl.status)) {
                     uint8_t *blk = static_cast<uint8_t *>(a.owners.p[owner]);
-                    reinterpret_cast<uint32_t *>(blk + a.rank_base * a.seg_code_bytes)[cl] = word;
+                    if (!EF)
+                        reinterpret_cast<uint32_t *>(blk + a.rank_base * a.seg_code_bytes)[cl] = word;
                     if ((lane & ((1u << lanes_log2) - 1u)) == 0) { // the group's first lane
                         uint8_t *row = blk + a.recv_scales_off + a.rank_base * a.seg_scale_stride;
                         if (f16)
@@ -239,7 +252,7 @@ __device__ __forceinline__ void k1_consume(const K1Args &a, const uint8_t *smem,
             }
         }
         if (EF)
-            fence_proxy_async_smem(); // the new errors are read next by the producer's bulk stores
+            fence_proxy_async_smem(); // read next by the producer's bulk stores
         __syncwarp();
         if (lane == 0)
             mbar_arrive(&empty[s]); // this warp is done with stage s
@@ -320,27 +333,45 @@ __global__ void __launch_bounds__(K1Warps<B, EF>::kThreads, 2)
                               a.eps + static_cast<size_t>(r) * a.n + el0, cnt * 4, bar);
             }
         };
-        if (lane == 0) {
+        // With sender feedback, what the consumers leave in a released stage
+        // goes out by bulk stores: the new errors, and with one handle per
+        // rank the code words, into each owner's receive block for the part of
+        // the tile in its segment (segment bounds are multiples of 32
+        // elements, so every piece starts on 16 bytes).
+        auto writeback = [&](uint32_t t) {
+            const size_t el0 = e0 + static_cast<size_t>(blockIdx.x + t * gridDim.x) * tile;
+            const uint32_t cnt = static_cast<uint32_t>(e1 - el0 < size_t(tile) ? e1 - el0 : tile);
+            const uint8_t *stage = smem + (t % S) * Sh::kStageBytes;
+            if (!in_bounds(el0 + cnt <= a.n && cnt <= Sh::kTile, a.ctl.status))
+                return;
             if constexpr (EF) {
-                // the new errors go back to global memory by bulk stores from
-                // the released stage, not by the consumers' own stores
-                produce_tiles_writeback<S>(
-                    full, empty, mine, a.ctl.stall, a.ctl.wait_cycles, a.ctl.status, kStatusTimeoutK1, issue,
-                    [&](uint32_t t) {
-                        const size_t el0 = e0 + static_cast<size_t>(blockIdx.x + t * gridDim.x) * tile;
-                        const uint32_t cnt = static_cast<uint32_t>(e1 - el0 < size_t(tile) ? e1 - el0 : tile);
-                        const uint8_t *stage = smem + (t % S) * Sh::kStageBytes;
-                        if (!in_bounds(el0 + cnt <= a.n && cnt <= Sh::kTile, a.ctl.status))
-                            return;
 #pragma unroll
-                        for (int r = 0; r < P; r++)
-                            bulk_store(a.eps + static_cast<size_t>(r) * a.n + el0,
-                                       stage + Sh::kEpsOff + r * Sh::kTile * 4, cnt * 4);
-                    });
-            } else {
+                for (int r = 0; r < P; r++)
+                    bulk_store(a.eps + static_cast<size_t>(r) * a.n + el0, stage + Sh::kEpsOff + r * Sh::kTile * 4,
+                               cnt * 4);
+            }
+            if constexpr (P == 1 && EF) {
+                if (a.to_owners) {
+                    for (size_t lo = el0; lo < el0 + cnt;) {
+                        const size_t owner = lo / seg;
+                        const size_t hi = el0 + cnt < (owner + 1) * seg ? el0 + cnt : (owner + 1) * seg;
+                        if (in_bounds(owner < kMaxRanks && (lo - owner * seg + (hi - lo)) / 2 <= a.seg_code_bytes,
+                                      a.ctl.status))
+                            bulk_store(static_cast<uint8_t *>(a.owners.p[owner]) + a.rank_base * a.seg_code_bytes +
+                                           (lo - owner * seg) / 2,
+                                       stage + Sh::kCodeOff + (lo - el0) / 2, static_cast<uint32_t>(hi - lo) / 2);
+                        lo = hi;
+                    }
+                }
+            }
+        };
+        if (lane == 0) {
+            if constexpr (EF)
+                produce_tiles_writeback<S>(full, empty, mine, a.ctl.stall, a.ctl.wait_cycles, a.ctl.status,
+                                           kStatusTimeoutK1, issue, writeback);
+            else
                 produce_tiles<S>(full, empty, mine, a.ctl.stall, a.ctl.wait_cycles, a.ctl.status, kStatusTimeoutK1,
                                  issue);
-            }
         }
         return;
     }
