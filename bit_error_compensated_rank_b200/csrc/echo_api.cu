@@ -66,8 +66,11 @@ constexpr size_t kMaxN = size_t(1) << 34;  // chunk indices stay 32-bit
 // lands in microseconds); the injected stall uses about half a millisecond.
 constexpr long long kWaitCycles = 1LL << 31;
 constexpr long long kStallWaitCycles = 1LL << 20;
+// Host-path pieces: 2^25 elements per rank measured best at 1 GiB (159 ms per
+// step, against 168 at 2^22, whose 1024 copies per step each cost set-up,
+// and 161 at 2^26, whose first and last pieces take longer to fill and drain).
 #ifndef ECHO_HOST_PIECE_LOG2
-#define ECHO_HOST_PIECE_LOG2 22
+#define ECHO_HOST_PIECE_LOG2 25
 #endif
 constexpr size_t kHostPiece = size_t(1) << ECHO_HOST_PIECE_LOG2; // elements per pipelined host transfer
 constexpr int kVariantBits = ECHO_VARIANT_OWNER_SUM | ECHO_VARIANT_SENDER_EF | ECHO_VARIANT_FP16_SCALE;

@@ -356,7 +356,7 @@ def test_host_end_to_end_fp32_backward(oracle):
     ragged last piece; the forward state stays untouched."""
     import torch
     from bit_error_compensated_rank_b200 import echo
-    P, n = 2, 2 * 32 * 70001  # 4.48 M elements per rank: a full piece and a ragged one
+    P, n = 2, 2 * 32 * ((1 << 19) + 1)  # 2^25 + 64 elements per rank: a full piece and a ragged one
     h = echo.Echo(P, n, echo.ECHO_FP32)
     try:
         f = np.zeros(n, np.float32)
