@@ -195,24 +195,35 @@ __device__ __forceinline__ bool half_below(uint32_t x, uint32_t bound)
 }
 
 // short_vals: every v[k] has at most 8 significant bits (see kZTie).
+// The z-form products go two at a time through sm_100's packed f32x2 FMA,
+// which rounds each component exactly as the scalar __fmaf_rn does. One
+// test sends a lane off the common path: a saturated scale, or a fraction
+// below the margin (below kZTie for short values); there a saturated or
+// long-valued lane takes the exact path and a short-valued one settles its
+// exact midpoints.
 __device__ __forceinline__ void codes8_half(const float (&v)[kChunk], float step, float inv, float half, bool sat,
                                             bool short_vals, uint32_t (&z)[kChunk])
 {
 #pragma unroll
-    for (int k = 0; k < kChunk; k++)
-        z[k] = __float_as_uint(__fmaf_rn(v[k], inv, kZ));
+    for (int j = 0; j < kChunk / 2; j++) {
+        const float2 p = __ffma2_rn(make_float2(v[2 * j], v[2 * j + 1]), make_float2(inv, inv), make_float2(kZ, kZ));
+        z[2 * j] = __float_as_uint(p.x);
+        z[2 * j + 1] = __float_as_uint(p.y);
+    }
     const uint32_t lo = min_u16x2(min_u16x2(__byte_perm(z[0], z[1], 0x5410), __byte_perm(z[2], z[3], 0x5410)),
                                   min_u16x2(__byte_perm(z[4], z[5], 0x5410), __byte_perm(z[6], z[7], 0x5410)));
-    if (sat || (!short_vals && half_below(lo, kZMargin))) {
+    if (sat || half_below(lo, short_vals ? kZTie : kZMargin)) {
+        if (sat || !short_vals) {
 #pragma unroll
-        for (int k = 0; k < kChunk; k++)
-            z[k] = zcode_of_bits(code_bits_near(v[k], step, inv, half));
-    } else if (short_vals && half_below(lo, kZTie)) {
-        // exact midpoints: an odd code (bit 16, the parity of byte 2) moves down
+            for (int k = 0; k < kChunk; k++)
+                z[k] = zcode_of_bits(code_bits_near(v[k], step, inv, half));
+        } else {
+            // exact midpoints: an odd code (bit 16, the parity of byte 2) moves down
 #pragma unroll
-        for (int k = 0; k < kChunk; k++)
-            if ((z[k] & 0x1FFFFu) - 0x10000u < kZTie)
-                z[k] -= 0x10000u;
+            for (int k = 0; k < kChunk; k++)
+                if ((z[k] & 0x1FFFFu) - 0x10000u < kZTie)
+                    z[k] -= 0x10000u;
+        }
     }
 }
 
@@ -289,6 +300,14 @@ __device__ __forceinline__ float max3_abs(float a, float b, float c)
 __device__ __forceinline__ float absmax8(const float (&v)[kChunk])
 {
     return fmaxf(max3_abs(v[0], v[1], v[2]), max3_abs(v[3], v[4], max3_abs(v[5], v[6], v[7])));
+}
+
+// The same over 16 values in two rows of 8 (8 three-input maxima).
+__device__ __forceinline__ float absmax16(const float (&a)[kChunk], const float (&b)[kChunk])
+{
+    const float m0 = max3_abs(a[0], a[1], a[2]), m1 = max3_abs(a[3], a[4], a[5]), m2 = max3_abs(a[6], a[7], b[0]);
+    const float m3 = max3_abs(b[1], b[2], b[3]), m4 = max3_abs(b[4], b[5], b[6]);
+    return fmaxf(max3_abs(m0, m1, m2), max3_abs(m3, m4, b[7]));
 }
 
 // Codes of elements 2j and 2j+1 as a pair of floats, by one packed

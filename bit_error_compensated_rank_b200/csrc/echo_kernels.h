@@ -33,7 +33,9 @@
 // binary16-scale variants, and the default group with sender feedback. The
 // last three have longer chains per item (more shuffles for large groups; the
 // binary16 scale, reciprocal and code settling; the error tiles' loads and
-// stores) and want more warps per SM to hide them.
+// stores) and want more warps per SM to hide them. The binary16 body for bf16
+// partials without sender feedback (16 elements per lane) has twice the work
+// per item, and 8 warps measured as fast as 12 and faster than 16.
 #ifndef ECHO_K1_WARPS
 #define ECHO_K1_WARPS 8
 #endif
@@ -45,6 +47,9 @@
 #endif
 #ifndef ECHO_K1_WARPS_HALF_SCALE
 #define ECHO_K1_WARPS_HALF_SCALE 16
+#endif
+#ifndef ECHO_K1_WARPS_HALF_WIDE
+#define ECHO_K1_WARPS_HALF_WIDE 8
 #endif
 #ifndef ECHO_K2_STAGES
 #define ECHO_K2_STAGES 2

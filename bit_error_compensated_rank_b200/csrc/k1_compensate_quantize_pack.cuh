@@ -28,6 +28,8 @@
 // empty[s]. A lane owns 8 consecutive
 // elements of one rank; G/8 lanes form a group and find its maximum with
 // log2(G/8) shuffles; codes leave as one coalesced 32-bit store per lane.
+// The binary16-scale body for bf16 partials without sender feedback, bound
+// by instruction issue, gives a lane 16 elements instead (k1_consume_wide).
 // With sender feedback each lane writes its 8 new errors over the old ones
 // in the stage, and the producer bulk-stores the P error tiles once every
 // consumer warp has released the stage, before it refills it: the TMA engine,
@@ -60,12 +62,16 @@ namespace {
 // its binary16-scale bodies, which get their own count of consumer warps.
 enum K1Build { kDefaultBuild = 0, kGroupsBuild = 1, kHalfScaleBuild = 2 };
 
-template <int B, bool EF>
+// Whether a build runs the wide binary16 body (k1_consume_wide).
+__host__ __device__ constexpr bool k1_wide(int B, bool bf16, bool ef) { return B == kHalfScaleBuild && bf16 && !ef; }
+
+template <int B, bool BF16, bool EF>
 struct K1Warps {
-    static constexpr int kConsumerWarps = B == kHalfScaleBuild  ? ECHO_K1_WARPS_HALF_SCALE
-                                          : B == kGroupsBuild   ? ECHO_K1_WARPS_GROUPS
-                                          : EF                  ? ECHO_K1_WARPS_SENDER_EF
-                                                                : ECHO_K1_WARPS;
+    static constexpr int kConsumerWarps = k1_wide(B, BF16, EF) ? ECHO_K1_WARPS_HALF_WIDE
+                                          : B == kHalfScaleBuild ? ECHO_K1_WARPS_HALF_SCALE
+                                          : B == kGroupsBuild    ? ECHO_K1_WARPS_GROUPS
+                                          : EF                   ? ECHO_K1_WARPS_SENDER_EF
+                                                                 : ECHO_K1_WARPS;
     static constexpr int kConsumers = kConsumerWarps * 32;
     static constexpr int kThreads = kConsumers + 32; // + one producer warp
 };
@@ -259,13 +265,113 @@ __device__ __forceinline__ void k1_consume(const K1Args &a, const uint8_t *smem,
     }
 }
 
+// The consumer body for binary16 scales with bf16 partials and no sender
+// feedback. That body is bound by instruction issue, not by HBM, so here a
+// lane owns 16 consecutive elements (two code words) of one rank, and the
+// work a lane does once per unit (its indices, the group maximum's shuffles,
+// the scale with its step and reciprocal, the stores) is spent once per 16
+// elements instead of once per 8. A group of 8 << LANES elements spans
+// 2^LANES / 2 lanes. The lane reads its 32 bytes of partials as two 16-byte
+// halves, half sw = (lane >> 2) & 1 first, so the 8 lanes of each
+// shared-memory phase cover the 32 banks once; row 0 of its values (and of
+// the state it adds) is chunk c + sw of the unit, row 1 the other chunk, and
+// the two code words are put back in element order for one 8-byte store.
+template <int P, bool COMP, uint32_t LANES, int NC>
+__device__ __forceinline__ void k1_consume_wide(const K1Args &a, const uint8_t *smem, uint64_t *full,
+                                                uint64_t *empty, uint32_t mine, uint32_t cpt_log2, size_t e0)
+{
+    using Sh = K1Shape<P, true, COMP, false>;
+    constexpr int S = Sh::kStages;
+    constexpr uint32_t lanes_log2 = LANES;     // log2(G / 8)
+    constexpr uint32_t glanes = (1u << LANES) / 2; // lanes per group
+    const uint32_t tid = threadIdx.x;
+    const uint32_t lane = tid & 31u;
+    const uint32_t sw = (lane >> 2) & 1u;
+    const uint32_t upt_log2 = cpt_log2 - 1; // 16-element units per tile = 2^upt_log2
+    const uint32_t code_words = static_cast<uint32_t>(a.n / kChunk);
+    for (uint32_t i = 0; i < mine; i++) {
+        const uint32_t s = i % S;
+        if (!warp_wait(&full[s], (i / S) & 1u, a.ctl.wait_cycles, a.ctl.status, kStatusTimeoutK1))
+            return;
+        const uint32_t tile_chunk0 = static_cast<uint32_t>(e0 / kChunk) + ((blockIdx.x + i * gridDim.x) << cpt_log2);
+        const uint32_t cnt_chunks = min(1u << cpt_log2, a.chunk_end - tile_chunk0); // even
+        const uint8_t *stage = smem + s * Sh::kStageBytes;
+        const float *fs = reinterpret_cast<const float *>(stage + Sh::kStateOff);
+
+#pragma unroll 1 // an item is 16 elements: unrolling by 2 measured the same
+        for (uint32_t it = tid; it < (static_cast<uint32_t>(P) << upt_log2); it += NC) {
+            const uint32_t r = it >> upt_log2; // warp-uniform (a tile has >= 32 units)
+            const uint32_t c = (it & ((1u << upt_log2) - 1u)) << 1; // the unit's first chunk
+            const bool active = c < cnt_chunks;
+            const uint32_t chunk = tile_chunk0 + c;
+            const uint32_t g = chunk >> lanes_log2;
+
+            const uint8_t *xp = stage + r * Sh::kXBytes + c * (kChunk * 2);
+            float v[2][kChunk];
+            bf16x8_to_f32(*reinterpret_cast<const uint4 *>(xp + 16u * sw), v[0]);
+            bf16x8_to_f32(*reinterpret_cast<const uint4 *>(xp + 16u * (sw ^ 1u)), v[1]);
+            bool short_vals = true; // bf16 partials keep 8 significant bits unless corrected
+            if (COMP && g - (r + a.rank_base) * a.groups_per_seg < a.groups_per_seg) {
+                short_vals = false;
+#pragma unroll
+                for (uint32_t h = 0; h < 2; h++) {
+                    float fv[kChunk], sv[kChunk];
+                    load_f32x8(fs + (c + (sw ^ h)) * kChunk, fv);
+                    load_f32x8(fs + Sh::kTile + (c + (sw ^ h)) * kChunk, sv);
+#pragma unroll
+                    for (int k = 0; k < kChunk; k++)
+                        v[h][k] = __fadd_rn(v[h][k], __fadd_rn(__fmul_rn(a.lambda, fv[k]),
+                                                               __fmul_rn(a.one_minus_lambda, sv[k])));
+                }
+            }
+            const float amax = group_absmax(absmax16(v[0], v[1]), lanes_log2 - 1);
+            const uint32_t scale = half_scale_bits(amax);
+            const float st = half_step(scale);
+            const float inv = half_inv(st);
+            const float half = __fmul_rn(0.5f, st);
+            const bool sat = half_scale_saturates(amax);
+            uint32_t z[kChunk];
+            codes8_half(v[0], st, inv, half, sat, short_vals, z);
+            const uint32_t w0 = pack8_zcodes(z);
+            codes8_half(v[1], st, inv, half, sat, short_vals, z);
+            const uint32_t w1 = pack8_zcodes(z);
+            const uint2 words = sw ? make_uint2(w1, w0) : make_uint2(w0, w1); // chunks c, c + 1
+            const bool first = (lane & (glanes - 1u)) == 0; // the group's first lane
+            if (P == 1 && a.to_owners) {
+                // one handle per rank: into the owner's receive block
+                const uint32_t owner = g / a.groups_per_seg;
+                const uint32_t gl = g - owner * a.groups_per_seg;               // group in the segment
+                const uint32_t cl = chunk - ((owner * a.groups_per_seg) << lanes_log2); // chunk in the segment
+                if (active && in_bounds(owner < kMaxRanks && (size_t(gl) + 1) * 2u <= a.seg_scale_stride &&
+                                            (size_t(cl) + 2) * 4u <= a.seg_code_bytes,
+                                        a.ctl.status)) {
+                    uint8_t *blk = static_cast<uint8_t *>(a.owners.p[owner]);
+                    reinterpret_cast<uint2 *>(blk + a.rank_base * a.seg_code_bytes)[cl / 2] = words;
+                    if (first)
+                        reinterpret_cast<uint16_t *>(blk + a.recv_scales_off +
+                                                     a.rank_base * a.seg_scale_stride)[gl] =
+                            static_cast<uint16_t>(scale);
+                }
+            } else if (active && in_bounds(chunk + 2 <= code_words && (g + 1) * 2u <= a.scale_stride, a.ctl.status)) {
+                reinterpret_cast<uint2 *>(a.codes)[(static_cast<size_t>(r) * code_words + chunk) / 2] = words;
+                if (first)
+                    reinterpret_cast<uint16_t *>(a.scales + static_cast<size_t>(r) * a.scale_stride)[g] =
+                        static_cast<uint16_t>(scale);
+            }
+        }
+        __syncwarp();
+        if (lane == 0)
+            mbar_arrive(&empty[s]); // this warp is done with stage s
+    }
+}
+
 template <int P, bool BF16, bool COMP, bool EF, int B>
-__global__ void __launch_bounds__(K1Warps<B, EF>::kThreads, 2)
+__global__ void __launch_bounds__(K1Warps<B, BF16, EF>::kThreads, 2)
     k1_compensate_quantize_pack(const K1Args a)
 {
     using Sh = K1Shape<P, BF16, COMP, EF>;
-    constexpr int kConsumerWarps = K1Warps<B, EF>::kConsumerWarps;
-    constexpr int NC = K1Warps<B, EF>::kConsumers;
+    constexpr int kConsumerWarps = K1Warps<B, BF16, EF>::kConsumerWarps;
+    constexpr int NC = K1Warps<B, BF16, EF>::kConsumers;
     constexpr int S = Sh::kStages;
     extern __shared__ __align__(128) uint8_t smem[];
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + S * Sh::kStageBytes);
@@ -386,6 +492,14 @@ __global__ void __launch_bounds__(K1Warps<B, EF>::kThreads, 2)
         case 4u: k1_consume<P, BF16, COMP, EF, 4u, false, NC>(a, smem, full, empty, mine, cpt_log2, e0); break;
         default: break; // the host accepts no other group size
         }
+    } else if constexpr (k1_wide(B, BF16, EF)) {
+        switch (a.lanes_log2) {
+        case 1u: k1_consume_wide<P, COMP, 1u, NC>(a, smem, full, empty, mine, cpt_log2, e0); break;
+        case 2u: k1_consume_wide<P, COMP, 2u, NC>(a, smem, full, empty, mine, cpt_log2, e0); break;
+        case 3u: k1_consume_wide<P, COMP, 3u, NC>(a, smem, full, empty, mine, cpt_log2, e0); break;
+        case 4u: k1_consume_wide<P, COMP, 4u, NC>(a, smem, full, empty, mine, cpt_log2, e0); break;
+        default: break;
+        }
     } else {
         switch (a.lanes_log2) {
         case 1u: k1_consume<P, BF16, COMP, EF, 1u, true, NC>(a, smem, full, empty, mine, cpt_log2, e0); break;
@@ -401,7 +515,12 @@ template <int P, bool BF16, bool COMP, bool EF, int B>
 cudaError_t launch_p(const K1Args &a, cudaStream_t st)
 {
     using Sh = K1Shape<P, BF16, COMP, EF>;
-    constexpr int kThreads = K1Warps<B, EF>::kThreads;
+    constexpr int kThreads = K1Warps<B, BF16, EF>::kThreads;
+    // Every consumer loop runs over a whole warp's items or none, so that the
+    // group shuffles see all 32 lanes: a tile holds at least 32 items of each
+    // rank (chunks of 8 elements; units of 16 in the wide binary16 body).
+    constexpr int kMinTile = k1_wide(B, BF16, EF) ? 512 : 256;
+    static_assert(Sh::kTile >= kMinTile, "kernel 1 tile below a warp's items");
     // CTAs per SM of this instantiation, found once (threads that race here
     // compute the same value)
     static std::atomic<int> cached{0};
@@ -415,7 +534,7 @@ cudaError_t launch_p(const K1Args &a, cudaStream_t st)
     }
     const size_t elems = static_cast<size_t>(a.chunk_end - a.chunk_begin) * kChunk;
     K1Args b = a;
-    b.tile_log2 = pick_tile_log2(elems, Sh::kTile, 256, resident);
+    b.tile_log2 = pick_tile_log2(elems, Sh::kTile, kMinTile, resident);
     b.tile = 1u << b.tile_log2;
     const uint32_t tiles = static_cast<uint32_t>((elems + b.tile - 1) >> b.tile_log2);
     return launch_chained(kern, persistent_grid(tiles, resident), kThreads, Sh::kSmem, st, b);

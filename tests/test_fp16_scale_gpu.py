@@ -30,7 +30,7 @@ def _n(P, G, k):
 
 @pytest.mark.parametrize("dtype", ["bf16", "fp32"])
 @pytest.mark.parametrize("P,k", [(2, 37), (8, 41), (16, 9), (5, 3)])
-@pytest.mark.parametrize("G", [32, 16, 128])
+@pytest.mark.parametrize("G", [32, 16, 64, 128])
 def test_fp16_scale_sequences(oracle, G, P, k, dtype):
     n = _n(P, G, k)
     fc = FullCompare(oracle, P, n, dtype, group=G, variant=FP16_SCALE)
