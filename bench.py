@@ -316,7 +316,7 @@ def run_reference(args, rank: int, world: int) -> dict | None:
 # n = 2^26 and scaled by n, since the traffic grows in proportion); reported
 # only while the kernel source still has the hash it had when captured.
 NCU_TRAFFIC = {
-    "k1_compensate_quantize_pack": {"bytes_per_elem": 28.065, "source_sha": "1fa44d7bb3d48ddc"},
+    "k1_compensate_quantize_pack": {"bytes_per_elem": 28.056, "source_sha": "c222c7e4f7240425"},
 }
 
 
@@ -750,6 +750,23 @@ def residual_errors(P: int, tokens: int, hidden: int, layers: int, seed: int) ->
     return out
 
 
+def fused_bytes(Pc: int, n: int, ebytes: int, group: int = 32, enable: bool = True, variant: int = 0) -> int:
+    """Algorithmic HBM bytes of one call run as one kernel: the P partials and
+    the state read; both wires, the state and the P outputs written; sender
+    feedback's errors read and written. Nothing is read back."""
+    wire = n // 2 + n // group * (2 if variant & 4 else 1)
+    b = Pc * ebytes * n + (Pc + 1) * wire + Pc * ebytes * n
+    if enable:
+        b += 16 * n
+    if variant & 2:
+        b += 8 * Pc * n
+    return b
+
+
+def call_path(h, n: int) -> str:
+    return "one kernel" if n <= h.fused_limit() else "three kernels"
+
+
 def run_config(args) -> dict:
     """One line for workload ``args.config`` (1, 2, 4 or 5)."""
     import numpy as np
@@ -801,28 +818,42 @@ def run_config(args) -> dict:
     outs = [torch.empty(n, dtype=torch.bfloat16 if code == echo.ECHO_BF16 else torch.float32, device="cuda")
             for _ in range(Pc)]
     h = echo.Echo(Pc, n, code)
+    if args.fused_limit is not None:
+        h.set_fused_limit(args.fused_limit)
+    path = call_path(h, n)
     clocks = ClockSampler(gpu_selector(0))
     clocks.start()
     eager, graph, reps = time_sequence(h, seq_inputs, outs, stream)
+    three = None
+    if path == "one kernel":  # the three pipelined kernels on the same sequence, for comparison
+        h.set_fused_limit(0)
+        three = time_sequence(h, seq_inputs, outs, stream)
     clk = clocks.stop()
     h.close()
     mb = echo.echo_model_bytes(Pc, n, code, True)
-    frac_graph = mb["total"] / (graph * 1e-3) / (peak * 1e9)
+    # the bytes of the path that ran: the one-kernel path reads no wire back
+    path_bytes = fused_bytes(Pc, n, ebytes) if path == "one kernel" else mb["total"]
+    frac_graph = path_bytes / (graph * 1e-3) / (peak * 1e9)
     line = {
         "config_line": cfg, "workload": CONFIG_DESC[cfg], "P": Pc, "n_per_rank": n,
         "element_dtype": "bf16" if code == echo.ECHO_BF16 else "fp32",
+        "path": path,
         "calls_per_sequence": len(seq_inputs), "sequence_repetitions": reps,
         "us_per_call_eager": round(eager * 1e3, 2), "us_per_call_graph": round(graph * 1e3, 2),
         "algbw_GBs_eager": round(ebytes * n / (eager * 1e-3) / 1e9, 2),
         "algbw_GBs_graph": round(ebytes * n / (graph * 1e-3) / 1e9, 2),
-        "model_bytes_per_call": mb["total"],
-        "roofline_frac_eager": round(mb["total"] / (eager * 1e-3) / (peak * 1e9), 4),
+        "bytes_per_call": path_bytes, "model_bytes_per_call_three_kernels": mb["total"],
+        "roofline_frac_eager": round(path_bytes / (eager * 1e-3) / (peak * 1e9), 4),
         "roofline_frac_graph": round(frac_graph, 4), "peak_gbs": peak, "peak_kind": peak_kind,
         "l2_resident": mb["total"] < L2_BYTES,
         "regime": "launch-bound" if frac_graph < 0.5 else "hbm-bound",
         "link_bytes_per_call": mb["link"],
         "clocks": clk,
     }
+    if three is not None:
+        line["three_kernels"] = {"us_per_call_eager": round(three[0] * 1e3, 2),
+                                 "us_per_call_graph": round(three[1] * 1e3, 2),
+                                 "roofline_frac_graph": round(mb["total"] / (three[1] * 1e-3) / (peak * 1e9), 4)}
     if cfg == 4:
         line["inputs"] = "8 distinct input sets per phase, cycled over the 64 calls of each phase"
     if cfg == 5:
@@ -862,7 +893,7 @@ def run_e2e(h, send, n, args, device, world) -> dict:
 
 def run_sweep(args) -> None:
     """Message-size sweep (one JSON line per size, not the benchmark line):
-    P = 8, bf16, n = 2^12 .. 2^29 elements per rank, CUDA-event time per call
+    P = 8, bf16, n = 2^12 .. 2^sweep_max (default 2^29) elements per rank, CUDA-event time per call
     over enough calls to fill about 50 ms, inputs resident, out of place."""
     import torch
     from bit_error_compensated_rank_b200 import echo
@@ -870,17 +901,20 @@ def run_sweep(args) -> None:
     torch.cuda.set_device(0)
     stream = torch.cuda.current_stream()
     peak, _ = hbm_peak()
-    nmax = 1 << 29
+    nmax = 1 << args.sweep_max
     send = [torch.empty(nmax, dtype=torch.bfloat16, device="cuda") for _ in range(P)]
     recv = [torch.empty(nmax, dtype=torch.bfloat16, device="cuda") for _ in range(P)]
     for r in range(P):
         wl.torch_outlier_gaussian_(send[r], seed=SEED, call=0, rank=r)
     variant = VARIANTS[args.variant]
-    for k in range(12, 30):
+    for k in range(12, args.sweep_max + 1):
         n = (1 << k) - (1 << k) % (P * max(args.group, 32))
         h = echo.Echo(P, n, echo.ECHO_BF16, args.group)
         if variant:
             h.set_variant(variant)
+        if args.fused_limit is not None:
+            h.set_fused_limit(args.fused_limit)
+        path = call_path(h, n)
         s_views = [t[:n] for t in send]
         r_views = [t[:n] for t in recv]
         for _ in range(args.warmup):
@@ -926,8 +960,9 @@ def run_sweep(args) -> None:
         ms_graph = start.elapsed_time(end) / (reps * per_graph)
         del graph
         mb = echo.echo_model_bytes_ex(P, n, args.group, echo.ECHO_BF16, True, variant)
+        path_bytes = fused_bytes(P, n, 2, args.group, True, variant) if path == "one kernel" else mb["total"]
         print(json.dumps({"sweep": True, "variant": args.variant, "group": args.group, "n_per_rank": n,
-                          "msg_bytes": 2 * n, "calls": calls,
+                          "msg_bytes": 2 * n, "calls": calls, "path": path, "bytes_per_call": path_bytes,
                           "us_per_call": round(ms * 1e3, 2),
                           "us_per_call_median16": round(ms_median * 1e3, 2),
                           # the call's bytes fit the 126 MB L2: may read above the HBM roofline
@@ -935,7 +970,7 @@ def run_sweep(args) -> None:
                           "us_per_call_graph": round(ms_graph * 1e3, 2),
                           "algbw_GBs": round(2 * n / (ms * 1e-3) / 1e9, 2),
                           "algbw_graph_GBs": round(2 * n / (ms_graph * 1e-3) / 1e9, 2),
-                          "roofline_frac_graph": round(mb["total"] / (ms_graph * 1e-3) / (peak * 1e9), 4)}),
+                          "roofline_frac_graph": round(path_bytes / (ms_graph * 1e-3) / (peak * 1e9), 4)}),
               flush=True)
         h.close()
 
@@ -944,6 +979,8 @@ def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--sweep", action="store_true",
                     help="print one line per message size (2^12..2^29 elements) instead of the benchmark")
+    ap.add_argument("--sweep-max", type=int, default=29, choices=range(12, 30), metavar="K",
+                    help="with --sweep: the largest size, 2^K elements per rank (default 29)")
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
@@ -966,6 +1003,9 @@ def main(argv=None):
                          "per GPU (auto: simulated at one process, sharded at more)")
     ap.add_argument("--config", type=int, choices=[1, 2, 4, 5], default=None,
                     help="print one line for this workload instead of the benchmark line")
+    ap.add_argument("--fused-limit", type=int, default=None, metavar="N",
+                    help="with --config or --sweep: calls with n <= N elements per rank run as one kernel "
+                         "(0: never; default: the library's 2^20)")
     ap.add_argument("--one-gpu", action="store_true",
                     help="sharded mode: every process uses GPU 0 (with --gpus 1)")
     ap.add_argument("--host-ordered", action="store_true",

@@ -75,6 +75,14 @@ constexpr long long kStallWaitCycles = 1LL << 20;
 constexpr size_t kHostPiece = size_t(1) << ECHO_HOST_PIECE_LOG2; // elements per pipelined host transfer
 constexpr int kVariantBits = ECHO_VARIANT_OWNER_SUM | ECHO_VARIANT_SENDER_EF | ECHO_VARIANT_FP16_SCALE;
 constexpr int kTimingRing = 32;                 // event sets of timed calls in flight
+// Largest n per rank whose calls run as one kernel (kf_fused_allreduce) by
+// default; larger calls run the three pipelined kernels. At P = 8, bf16, the
+// one kernel took 4.1 to 6.7 us per call up to 2^19 elements per rank against
+// 6.7 to 12.9, and 15.2 against 18.2 us at 2^20; at 2^21 both took 29.5 us,
+// and beyond it the pipelined kernels are faster.
+#ifndef ECHO_FUSED_LIMIT
+#define ECHO_FUSED_LIMIT (size_t(1) << 20)
+#endif
 
 size_t elem_bytes(int dtype) { return dtype == ECHO_BF16 ? 2 : 4; }
 
@@ -137,6 +145,7 @@ struct echo_handle {
     bool enable = true;
     int variant = 0;            // ECHO_VARIANT_* bits
     float *eps = nullptr;       // [phase][P][n]: sender errors (allocated with the variant)
+    size_t fused_limit = ECHO_FUSED_LIMIT; // calls with n <= this run as one kernel
     uint64_t link_bytes = 0, hbm_bytes = 0, calls = 0;
     // Kernel timing: each timed call records 4 events (before K1, after K1,
     // K2, K3) into slot (call index mod kTimingRing); a slot's durations are
@@ -144,6 +153,7 @@ struct echo_handle {
     // timed loop of calls never waits on the device.
     bool timing = false;
     cudaEvent_t ring[kTimingRing][4] = {};
+    bool ring_fused[kTimingRing] = {}; // the slot's call ran as one kernel: events 0 and 1 only
     uint64_t ring_calls = 0; // timed calls since timing was switched on
     uint64_t folded = 0;     // timed calls already added to total_ms
     double total_ms[3] = {};
@@ -280,18 +290,31 @@ int check_buffers(echo_handle *h, const void *const send[], void *const recv[])
 }
 
 // Add the kernel durations of timed calls [h->folded, upto) to the totals.
+// The three kernel durations of timing slot `slot` (waiting for its events).
+// A call that ran as one kernel recorded events 0 and 1 only: its whole time
+// is kernel 1's, and kernels 2 and 3 are 0.
+cudaError_t slot_ms(const echo_handle *h, int slot, float ms[3])
+{
+    const cudaEvent_t *ev = h->ring[slot];
+    const int kernels = h->ring_fused[slot] ? 1 : 3;
+    cudaError_t e = cudaEventSynchronize(ev[kernels]);
+    for (int k = 0; k < 3 && e == cudaSuccess; k++) {
+        ms[k] = 0.f;
+        if (k < kernels)
+            e = cudaEventElapsedTime(&ms[k], ev[k], ev[k + 1]);
+    }
+    return e;
+}
+
 int fold_timings(echo_handle *h, uint64_t upto)
 {
     for (; h->folded < upto; h->folded++) {
-        cudaEvent_t *ev = h->ring[h->folded % kTimingRing];
-        cudaError_t e = cudaEventSynchronize(ev[3]);
-        for (int k = 0; k < 3 && e == cudaSuccess; k++) {
-            float ms = 0.f;
-            e = cudaEventElapsedTime(&ms, ev[k], ev[k + 1]);
-            h->total_ms[k] += ms;
-        }
+        float ms[3];
+        cudaError_t e = slot_ms(h, static_cast<int>(h->folded % kTimingRing), ms);
         if (e != cudaSuccess)
             return cuda_error(e, "kernel timing events");
+        for (int k = 0; k < 3; k++)
+            h->total_ms[k] += ms[k];
     }
     return ECHO_OK;
 }
@@ -312,6 +335,12 @@ int enqueue_call(echo_handle *h, const void *const send[], void *const recv[], i
     // (partials, codes, 16-byte scale rows, state) is 16-byte aligned.
     if ((static_cast<size_t>(cb) * echo::kChunk) % (16 * static_cast<size_t>(h->group)) != 0 || ce < cb)
         return set_error(ECHO_ERR_INVALID, "internal: element range must start at a multiple of 16 groups");
+    // Every wait in the kernels is bounded; ECHO_FAULT=stall (tests) issues no
+    // loads at all and shortens the bound, so each wait runs out quickly.
+    const bool stall = fault_injected("stall");
+    // Small calls run as one kernel (the injected stall exercises the three
+    // kernels' bounded waits, so it always runs them).
+    const bool fused = !stall && h->n <= h->fused_limit;
     cudaEvent_t *ev = nullptr;
     if (record_events) {
         if (h->ring_calls >= static_cast<uint64_t>(kTimingRing)) {
@@ -321,6 +350,7 @@ int enqueue_call(echo_handle *h, const void *const send[], void *const recv[], i
         }
         h->last_slot = static_cast<int>(h->ring_calls % kTimingRing);
         ev = h->ring[h->last_slot];
+        h->ring_fused[h->last_slot] = fused;
         h->ring_calls += 1;
     } else {
         h->last_slot = -1;
@@ -380,9 +410,6 @@ int enqueue_call(echo_handle *h, const void *const send[], void *const recv[], i
     a3.P = h->P;
     a3.bf16 = h->dtype == ECHO_BF16;
 
-    // Every wait in the kernels is bounded; ECHO_FAULT=stall (tests) issues no
-    // loads at all and shortens the bound, so each wait runs out quickly.
-    const bool stall = fault_injected("stall");
     const echo::PipeCtl ctl{h->dstatus, stall ? kStallWaitCycles : kWaitCycles, stall};
     a1.ctl = a2.ctl = a3.ctl = ctl;
     a1.scale_stride = a2.scale_stride = a3.scale_stride = h->scale_stride;
@@ -394,26 +421,64 @@ int enqueue_call(echo_handle *h, const void *const send[], void *const recv[], i
     const char *what = "cudaEventRecord";
     if (ev)
         e = cudaEventRecord(ev[0], st);
-    if (e == cudaSuccess) {
+    if (e == cudaSuccess && fused) {
+        echo::KFArgs af{};
+        for (int r = 0; r < h->P; r++) {
+            af.x.p[r] = send[r];
+            af.out.p[r] = recv[r];
+        }
+        af.f = f;
+        af.s = s;
+        af.eps = a1.eps;
+        af.codes = h->codes1;
+        af.scales = h->scales1;
+        af.qcodes = h->qcodes;
+        af.qscales = h->qscales;
+        af.n = h->n;
+        af.scale_stride = h->scale_stride;
+        af.chunk_begin = cb;
+        af.chunk_end = ce;
+        af.lanes_log2 = h->lanes_log2;
+        af.groups_per_seg = a1.groups_per_seg;
+        af.lambda = a1.lambda;
+        af.one_minus_lambda = a1.one_minus_lambda;
+        af.beta_f = a2.beta_f;
+        af.one_minus_beta_f = a2.one_minus_beta_f;
+        af.beta_s = a2.beta_s;
+        af.one_minus_beta_s = a2.one_minus_beta_s;
+        af.P = h->P;
+        af.bf16 = h->dtype == ECHO_BF16;
+        af.enable = h->enable;
+        af.owner_sum = a2.owner_sum;
+        af.sender_ef = a1.sender_ef;
+        af.fp16_scale = a1.fp16_scale;
+        af.ctl = ctl;
+        NvtxRange r("kf_fused_allreduce");
+        if ((e = echo::launch_kf_fused_allreduce(af, st)) != cudaSuccess)
+            what = "launch kf_fused_allreduce";
+        if (e == cudaSuccess && ev) // the whole call counts as kernel 1's time
+            e = cudaEventRecord(ev[1], st);
+    }
+    if (e == cudaSuccess && !fused) {
         NvtxRange r("k1_compensate_quantize_pack");
         if ((e = echo::launch_k1_compensate_quantize_pack(a1, st)) != cudaSuccess)
             what = "launch k1_compensate_quantize_pack";
     }
-    if (e == cudaSuccess && ev)
+    if (e == cudaSuccess && !fused && ev)
         e = cudaEventRecord(ev[1], st);
-    if (e == cudaSuccess) {
+    if (e == cudaSuccess && !fused) {
         NvtxRange r("k2_owner_reduce_requant");
         if ((e = echo::launch_k2_owner_reduce_requant(a2, st)) != cudaSuccess)
             what = "launch k2_owner_reduce_requant";
     }
-    if (e == cudaSuccess && ev)
+    if (e == cudaSuccess && !fused && ev)
         e = cudaEventRecord(ev[2], st);
-    if (e == cudaSuccess) {
+    if (e == cudaSuccess && !fused) {
         NvtxRange r("k3_gather_dequant");
         if ((e = echo::launch_k3_gather_dequant(a3, st)) != cudaSuccess)
             what = "launch k3_gather_dequant";
     }
-    if (e == cudaSuccess && ev)
+    if (e == cudaSuccess && !fused && ev)
         e = cudaEventRecord(ev[3], st);
     if (ECHO_DEBUG && e == cudaSuccess && (e = echo::launch_check_guards(h->guards, h->dstatus, st)) != cudaSuccess)
         what = "launch check_guards";
@@ -917,6 +982,26 @@ int echo_stats(echo_handle *h, uint64_t *link_bytes, uint64_t *model_hbm_bytes, 
     return ECHO_OK;
 }
 
+int echo_set_fused_limit(echo_handle *h, size_t max_n)
+{
+    int rc = check_handle(h);
+    if (rc != ECHO_OK)
+        return rc;
+    h->fused_limit = max_n;
+    return ECHO_OK;
+}
+
+int echo_get_fused_limit(echo_handle *h, size_t *max_n)
+{
+    int rc = check_handle(h);
+    if (rc != ECHO_OK)
+        return rc;
+    if (!max_n)
+        return set_error(ECHO_ERR_INVALID, "max_n is NULL");
+    *max_n = h->fused_limit;
+    return ECHO_OK;
+}
+
 int echo_set_timing(echo_handle *h, int enable)
 {
     int rc = check_handle(h);
@@ -952,10 +1037,7 @@ int echo_last_kernel_ms(echo_handle *h, float ms[3])
         return set_error(ECHO_ERR_INVALID, "ms is NULL");
     if (h->last_slot < 0)
         return set_error(ECHO_ERR_INVALID, "the last call was not timed (echo_set_timing)");
-    cudaEvent_t *ev = h->ring[h->last_slot];
-    cudaError_t e = cudaEventSynchronize(ev[3]);
-    for (int k = 0; k < 3 && e == cudaSuccess; k++)
-        e = cudaEventElapsedTime(&ms[k], ev[k], ev[k + 1]);
+    cudaError_t e = slot_ms(h, h->last_slot, ms);
     return e == cudaSuccess ? ECHO_OK : cuda_error(e, "echo_last_kernel_ms");
 }
 

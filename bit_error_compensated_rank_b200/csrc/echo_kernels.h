@@ -161,6 +161,33 @@ struct K3Args {
     PipeCtl ctl;
 };
 
+// The whole call as one kernel (small messages): every argument of the three
+// kernels' simulated-rank launches, over one element range.
+struct KFArgs {
+    RankPtrs x;              // P rank partials (bf16 or binary32), n elements each
+    RankOutPtrs out;         // P rank outputs (may equal x: in place)
+    float *f, *s;            // phase state [n], read and updated in place
+    float *eps;              // sender feedback: every rank's rounding-#1 error [P][n]
+    uint8_t *codes;          // stage-1 wire codes [P][n/2]
+    uint8_t *scales;         // stage-1 wire scales [P][scale_stride]
+    uint8_t *qcodes;         // requantised total [n/2]
+    uint8_t *qscales;        // [scale_stride]
+    size_t n;
+    size_t scale_stride;
+    uint32_t chunk_begin, chunk_end;
+    uint32_t lanes_log2;     // log2(G / 8): lanes per group
+    uint32_t groups_per_seg; // n / P / G: owner of group g is g / groups_per_seg
+    float lambda, one_minus_lambda;
+    float beta_f, one_minus_beta_f, beta_s, one_minus_beta_s;
+    int P;
+    bool bf16;
+    bool enable;             // compensation: state read, error captured, state updated
+    bool owner_sum;          // the correction enters the owner's sum (else the owner's partial)
+    bool sender_ef;          // every rank adds back and renews its own rounding-#1 error
+    bool fp16_scale;         // binary16 scales
+    PipeCtl ctl;
+};
+
 // Guard bytes around the library's device buffers (debug build only).
 constexpr size_t kGuardBytes = 256;
 constexpr uint8_t kGuardByte = 0xA5;
@@ -182,6 +209,7 @@ cudaError_t launch_k1_variant_fp32(const K1Args &a, cudaStream_t st);
 cudaError_t launch_k1_variant_fp32_ef(const K1Args &a, cudaStream_t st);
 cudaError_t launch_k2_owner_reduce_requant(const K2Args &a, cudaStream_t st);
 cudaError_t launch_k3_gather_dequant(const K3Args &a, cudaStream_t st);
+cudaError_t launch_kf_fused_allreduce(const KFArgs &a, cudaStream_t st);
 
 // Persistent grid: one CTA per tile up to (SMs x resident CTAs per SM).
 int persistent_grid(uint32_t tiles, int resident_per_sm);

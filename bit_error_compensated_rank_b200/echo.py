@@ -49,6 +49,7 @@ EXPORTED = (
     "echo_get_wire_range", "echo_stats", "echo_model_bytes", "echo_set_timing",
     "echo_last_kernel_ms", "echo_kernel_ms_total", "echo_device_status",
     "echo_allreduce_static", "echo_static_status", "echo_set_variant", "echo_get_sender_state", "echo_set_sender_state",
+    "echo_set_fused_limit", "echo_get_fused_limit",
     "echo_model_bytes_ex", "echo_debug_build", "echo_debug_touch_guard",
     "echo_dist_create", "echo_dist_export", "echo_dist_connect", "echo_dist_stage",
     "echo_dist_set_params", "echo_dist_set_variant", "echo_dist_get_state",
@@ -96,6 +97,8 @@ def _load():
                                          ctypes.c_float, _int, _vp]),
         "echo_static_status": (_int, [ctypes.POINTER(ctypes.c_int), _int]),
         "echo_set_variant": (_int, [_vp, _int]),
+        "echo_set_fused_limit": (_int, [_vp, _sz]),
+        "echo_get_fused_limit": (_int, [_vp, ctypes.POINTER(ctypes.c_size_t)]),
         "echo_get_sender_state": (_int, [_vp, _int, _int, _sz, _sz, _f32p]),
         "echo_set_sender_state": (_int, [_vp, _int, _int, _f32p]),
         "echo_model_bytes_ex": (_int, [_int, _sz, _int, _int, _int, _int, _u64p]),
@@ -271,6 +274,16 @@ def echo_set_variant(h: int, variant: int) -> None:
     _check(_lib.echo_set_variant(h, variant))
 
 
+def echo_set_fused_limit(h: int, max_n: int) -> None:
+    _check(_lib.echo_set_fused_limit(h, max_n))
+
+
+def echo_get_fused_limit(h: int) -> int:
+    v = ctypes.c_size_t()
+    _check(_lib.echo_get_fused_limit(h, ctypes.byref(v)))
+    return v.value
+
+
 def echo_get_sender_state(h: int, phase: int, rank: int, offset: int, count: int) -> np.ndarray:
     out = np.empty(count, np.float32)
     _check(_lib.echo_get_sender_state(h, phase, rank, offset, count, _np(out, _f32p)))
@@ -384,6 +397,13 @@ class Echo:
     def set_variant(self, variant: int) -> None:
         echo_set_variant(self.h, variant)
         self.variant = variant
+
+    def set_fused_limit(self, max_n: int) -> None:
+        """Calls with n <= max_n run as one kernel (0: never)."""
+        echo_set_fused_limit(self.h, max_n)
+
+    def fused_limit(self) -> int:
+        return echo_get_fused_limit(self.h)
 
     def get_sender_state(self, phase: int, rank: int, offset: int = 0, count: int | None = None):
         return echo_get_sender_state(self.h, phase, rank, offset, self.n - offset if count is None else count)

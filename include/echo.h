@@ -243,6 +243,26 @@ ECHO_API int echo_set_params(echo_handle *h, float beta_fast, float beta_slow, f
 #define ECHO_VARIANT_FP16_SCALE 4
 ECHO_API int echo_set_variant(echo_handle *h, int variant);
 
+/*
+ * echo_set_fused_limit - calls of this handle with n <= max_n (elements per
+ * rank) run as one kernel instead of the three: every step of the method
+ * works on one group of G elements at a time [rit.work "Echo 4-bit GPU
+ * communication", section "How Echo returns the error to later calls": a
+ * rank's segment rounded, the owner's high-precision sum rounded again, the
+ * total sent back], so one lane can take its 8 elements through all three
+ * steps. Up to about 2 MiB per rank the three dependent launches, not the
+ * bytes, set the time of a call. The fused call computes the same results bit
+ * for bit and writes the same buffers (both wires, state, sender errors,
+ * outputs); it does not read the stage-1 wire back. Every variant and group
+ * size runs fused. 0 turns it off; the default is 2^20. It applies to
+ * echo_allreduce, echo_allreduce_out and echo_allreduce_host, not to the
+ * static or per-rank entry points. echo_stats still counts the three kernels'
+ * model bytes. echo_get_fused_limit reads the setting (max_n non-NULL, else
+ * ECHO_ERR_INVALID).
+ */
+ECHO_API int echo_set_fused_limit(echo_handle *h, size_t max_n);
+ECHO_API int echo_get_fused_limit(echo_handle *h, size_t *max_n);
+
 /* Synchronous copies of rank `rank`'s sender errors for `phase` (elements
  * [offset, offset+count) to host; all n from host). ECHO_ERR_INVALID if sender
  * feedback was never switched on. */
@@ -324,6 +344,8 @@ ECHO_API int echo_model_bytes_ex(int P, size_t n, int group, int dtype, int enab
  */
 ECHO_API int echo_set_timing(echo_handle *h, int enable);
 ECHO_API int echo_last_kernel_ms(echo_handle *h, float ms[3]);
+/* (A call that ran as one kernel, see echo_set_fused_limit, reports its whole
+ * time as kernel 1's and 0 for kernels 2 and 3.) */
 ECHO_API int echo_kernel_ms_total(echo_handle *h, double ms[3], uint64_t *timed_calls);
 
 /*

@@ -61,10 +61,15 @@ def params_tuple(p: Params):
 
 class FullCompare:
     """One handle and the oracle side by side on a problem small enough to
-    compare in full after every call."""
+    compare in full after every call.
+
+    fused: run every call as the one-kernel path (True) or as the three
+    pipelined kernels (False, the default here, so that the small problems
+    these tests use keep covering the pipelined kernels; the one-kernel path
+    has its own tests)."""
 
     def __init__(self, oracle, P, n, dtype: str, params: Params = Params(), variant: int = 0,
-                 group: int = G):
+                 group: int = G, fused: bool = False):
         from bit_error_compensated_rank_b200 import echo
         self.echo = echo
         self.oracle = oracle
@@ -74,6 +79,7 @@ class FullCompare:
         self.variant = variant
         self.group = group
         self.h = echo.Echo(P, n, echo.ECHO_BF16 if dtype == "bf16" else echo.ECHO_FP32, group)
+        self.h.set_fused_limit(n if fused else 0)
         self.h.set_params(*params_tuple(params))
         if variant:
             self.h.set_variant(variant)

@@ -129,7 +129,9 @@ def test_null_and_unknown_handles(echo):
                      (echo._lib.echo_reset, (None, 1)),
                      (echo._lib.echo_set_params, (None, 0.5, 0.875, 0.5, 1)),
                      (echo._lib.echo_stats, (None, None, None, None)),
-                     (echo._lib.echo_set_timing, (None, 1))]:
+                     (echo._lib.echo_set_timing, (None, 1)),
+                     (echo._lib.echo_set_fused_limit, (None, 0)),
+                     (echo._lib.echo_get_fused_limit, (None, None))]:
         assert fn(*args) == echo.ECHO_ERR_INVALID
         assert "NULL" in echo.echo_last_error()
     bogus = 0x1000

@@ -29,6 +29,7 @@ def test_parity_suites_under_the_debug_build():
     res = _run_debug(["-m", "pytest", "-q", "-x", "-p", "no:cacheprovider",
                       "tests/test_parity_gpu.py", "tests/test_variants_gpu.py",
                       "tests/test_groups_gpu.py", "tests/test_fp16_scale_gpu.py", "tests/test_dist_gpu.py",
+                      "tests/test_fused_gpu.py",
                       "-k", "not one_gib and not largest and not error_growth and not timing"])
     assert res.returncode == 0, res.stdout[-4000:] + res.stderr[-2000:]
 
