@@ -361,6 +361,10 @@ def run_echo(args, rank: int, world: int, local: int) -> dict | None:
     h = echo.Echo(P, n, echo.ECHO_BF16, args.group)
     if variant:
         h.set_variant(variant)
+    # the three pipelined kernels at any --n, unless --fused-limit lets this
+    # size run as one kernel
+    h.set_fused_limit(0 if args.fused_limit is None else args.fused_limit)
+    fused = call_path(h, n) == "one kernel"
     mb = echo.echo_model_bytes_ex(P, n, args.group, echo.ECHO_BF16, True, variant)
     torch.cuda.synchronize()
 
@@ -402,6 +406,11 @@ def run_echo(args, rank: int, world: int, local: int) -> dict | None:
     k_avg = [t / timed_calls for t in kern_ms]
     names = ["k1_compensate_quantize_pack", "k2_owner_reduce_requant", "k3_gather_dequant"]
     k_bytes = [mb["k1"], mb["k2"], mb["k3"]]
+    if fused:  # one kernel, timed as kernel 1, with its own bytes
+        names, k_avg, k_bytes = ["kf_fused_allreduce"], k_avg[:1], [fused_bytes(P, n, 2, args.group, True, variant)]
+        call_bytes = k_bytes[0]
+        call_frac = call_bytes / (ms_step * 1e-3) / (peak * 1e9)
+        min_bytes = call_bytes
     dom = max(range(len(names)), key=lambda i: k_bytes[i])
     achieved = k_bytes[dom] / (k_avg[dom] * 1e-3) / 1e9
     src = os.path.join(ROOT, "bit_error_compensated_rank_b200", "csrc", names[dom] + ".cu")
@@ -434,7 +443,9 @@ def run_echo(args, rank: int, world: int, local: int) -> dict | None:
                          "bytes_per_elem": round(call_bytes / n, 5),
                          "peak_gbs": peak, "peak_kind": peak_kind,
                          "ideal_ms": round(call_bytes / (peak * 1e9) * 1e3, 4),
-                         "model": "P-GPU: every rank reads its own copy of the requantised wire"},
+                         "model": "one kernel: partials and state read, both wires, state and outputs written"
+                                  if fused else "P-GPU: every rank reads its own copy of the requantised wire"},
+        "path": "one kernel" if fused else "three kernels",
         "single_gpu_min_bytes_per_elem": round(min_bytes / n, 5),
         "single_gpu_min_frac": round(min_bytes / (ms_step * 1e-3) / (peak * 1e9), 4),
         "busbw": round(value * 2 * (P - 1) / P, 3),
@@ -445,7 +456,7 @@ def run_echo(args, rank: int, world: int, local: int) -> dict | None:
         "roofline": {"kernel": names[dom], "bound": "hbm", "achieved": round(achieved, 1),
                      "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
                      "traffic": traffic, "peak_kind": peak_kind},
-        "gpu_launches": 3 * args.steps,
+        "gpu_launches": (1 if fused else 3) * args.steps,
         "clocks": clk,
     }
     if e2e is not None:
@@ -1004,8 +1015,8 @@ def main(argv=None):
     ap.add_argument("--config", type=int, choices=[1, 2, 4, 5], default=None,
                     help="print one line for this workload instead of the benchmark line")
     ap.add_argument("--fused-limit", type=int, default=None, metavar="N",
-                    help="with --config or --sweep: calls with n <= N elements per rank run as one kernel "
-                         "(0: never; default: the library's 2^20)")
+                    help="calls with n <= N elements per rank run as one kernel (0: never). Default: the "
+                         "library's 2^20 with --config and --sweep; the three kernels on the benchmark line")
     ap.add_argument("--one-gpu", action="store_true",
                     help="sharded mode: every process uses GPU 0 (with --gpus 1)")
     ap.add_argument("--host-ordered", action="store_true",

@@ -77,9 +77,11 @@ constexpr int kVariantBits = ECHO_VARIANT_OWNER_SUM | ECHO_VARIANT_SENDER_EF | E
 constexpr int kTimingRing = 32;                 // event sets of timed calls in flight
 // Largest n per rank whose calls run as one kernel (kf_fused_allreduce) by
 // default; larger calls run the three pipelined kernels. At P = 8, bf16, the
-// one kernel took 4.1 to 6.7 us per call up to 2^19 elements per rank against
-// 6.7 to 12.9, and 15.2 against 18.2 us at 2^20; at 2^21 both took 29.5 us,
-// and beyond it the pipelined kernels are faster.
+// one kernel took 4.1 to 9.4 us per call up to 2^20 elements per rank, against
+// 6.6 to 18.2 us, where the three launches set the pipelined kernels' time.
+// Past that the one kernel's lead comes mostly from skipping the wire
+// read-back that one GPU allows and P GPUs do not, so the pipelined kernels
+// keep the larger calls.
 #ifndef ECHO_FUSED_LIMIT
 #define ECHO_FUSED_LIMIT (size_t(1) << 20)
 #endif

@@ -16,7 +16,10 @@
 // order, and writes the same buffers: both wires (every rank's stage-1 codes
 // and scales, the requantised total), the sender errors, the state and the P
 // outputs. The owner's restore uses the codes the lane has just produced, not
-// the wire bytes it wrote; on one GPU both hold the same codes.
+// the wire bytes it wrote; on one GPU both hold the same codes. That shortcut
+// needs every rank's partial on this GPU: ranks on separate GPUs (the
+// per-rank entry points) must read the wire at the receiver, and keep the
+// three stages.
 //
 // A warp takes 32 consecutive chunks (256 elements). Each lane first copies
 // its P partial chunks (and its P sender errors) into its own slots in shared
@@ -263,22 +266,30 @@ __global__ void __launch_bounds__(kThreads) kf_fused_allreduce(const KFArgs a)
 template <int P, bool BF16, bool F16>
 cudaError_t launch_p(const KFArgs &a, cudaStream_t st)
 {
-    // Set the shared-memory limit of this instantiation once, for its largest
-    // use (sender feedback); threads that race here set the same value.
-    static std::atomic<int> cached{0};
-    int resident = cached.load(std::memory_order_relaxed);
+    // The shared-memory limit of this instantiation is set once, for its
+    // largest use (sender feedback); its CTAs per SM are found once for each
+    // of its two shared-memory sizes. Threads that race here compute the
+    // same values.
+    static std::atomic<int> cached[2] = {{0}, {0}};
     auto kern = kf_fused_allreduce<P, BF16, F16>;
+    const int ef = a.sender_ef ? 1 : 0;
+    const int smem = static_cast<int>(kWarps * kf_warp_bytes(P, BF16, ef != 0));
+    int resident = cached[ef].load(std::memory_order_relaxed);
     if (resident == 0) {
+        int unused = 0;
         cudaError_t e = prepare_kernel(reinterpret_cast<const void *>(kern), kThreads,
-                                       kWarps * kf_warp_bytes(P, BF16, true), &resident);
+                                       kWarps * kf_warp_bytes(P, BF16, true), &unused);
+        if (e == cudaSuccess)
+            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&resident, reinterpret_cast<const void *>(kern),
+                                                              kThreads, smem);
         if (e != cudaSuccess)
             return e;
-        cached.store(resident, std::memory_order_relaxed);
+        resident = resident > 0 ? resident : 1;
+        cached[ef].store(resident, std::memory_order_relaxed);
     }
     const uint32_t items = (a.chunk_end - a.chunk_begin + 31u) >> 5;
     const int grid = persistent_grid((items + kWarps - 1) / kWarps, resident);
-    return launch_chained(kern, grid, kThreads, static_cast<int>(kWarps * kf_warp_bytes(P, BF16, a.sender_ef)), st,
-                          a);
+    return launch_chained(kern, grid, kThreads, smem, st, a);
 }
 
 template <int P>
