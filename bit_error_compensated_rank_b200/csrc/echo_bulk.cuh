@@ -110,6 +110,22 @@ __device__ __forceinline__ void bulk_store(void *gmem_dst, const void *smem_src,
                  : "memory");
 }
 
+// An L2 policy that makes the lines it touches the first to be evicted.
+__device__ __forceinline__ uint64_t l2_evict_first_policy()
+{
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+// bulk_store with an L2 cache policy (l2_evict_first_policy).
+__device__ __forceinline__ void bulk_store_hint(void *gmem_dst, const void *smem_src, uint32_t bytes, uint64_t policy)
+{
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group.L2::cache_hint [%0], [%1], %2, %3;" ::"l"(gmem_dst),
+                 "r"(smem_u32(smem_src)), "r"(bytes), "l"(policy)
+                 : "memory");
+}
+
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 
 // Wait until at most N committed store groups still read shared memory.
