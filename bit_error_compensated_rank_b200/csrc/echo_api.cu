@@ -75,16 +75,6 @@ constexpr long long kStallWaitCycles = 1LL << 20;
 constexpr size_t kHostPiece = size_t(1) << ECHO_HOST_PIECE_LOG2; // elements per pipelined host transfer
 constexpr int kVariantBits = ECHO_VARIANT_OWNER_SUM | ECHO_VARIANT_SENDER_EF | ECHO_VARIANT_FP16_SCALE;
 constexpr int kTimingRing = 32;                 // event sets of timed calls in flight
-// Largest n per rank whose calls run as one kernel (kf_fused_allreduce) by
-// default; larger calls run the three pipelined kernels. At P = 8, bf16, the
-// one kernel took 4.1 to 9.4 us per call up to 2^20 elements per rank, against
-// 6.6 to 18.2 us, where the three launches set the pipelined kernels' time.
-// Past that the one kernel's lead comes mostly from skipping the wire
-// read-back that one GPU allows and P GPUs do not, so the pipelined kernels
-// keep the larger calls.
-#ifndef ECHO_FUSED_LIMIT
-#define ECHO_FUSED_LIMIT (size_t(1) << 20)
-#endif
 
 size_t elem_bytes(int dtype) { return dtype == ECHO_BF16 ? 2 : 4; }
 

@@ -69,6 +69,16 @@
 #ifndef ECHO_K3_OUT_BUFS
 #define ECHO_K3_OUT_BUFS 2
 #endif
+// Largest n per rank whose calls run as one kernel (kf_fused_allreduce) by
+// default; larger calls run the three pipelined kernels. At P = 8, bf16, the
+// one kernel took 4.1 to 9.4 us per call up to 2^20 elements per rank, against
+// 6.6 to 18.2 us, where the three launches set the pipelined kernels' time.
+// Past that the one kernel's lead comes mostly from skipping the wire
+// read-back that one GPU allows and P GPUs do not, so the pipelined kernels
+// keep the larger calls.
+#ifndef ECHO_FUSED_LIMIT
+#define ECHO_FUSED_LIMIT (static_cast<size_t>(1) << 20)
+#endif
 // Shared memory one CTA may use (the B200 limit is 227 KB), and kernel 1's
 // budget per CTA so that two CTAs share an SM.
 #define ECHO_SMEM_BUDGET (225 * 1024)

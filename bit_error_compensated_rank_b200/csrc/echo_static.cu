@@ -200,7 +200,9 @@ extern "C" int echo_allreduce_static(int P, size_t n, int dtype, void *const ran
     if ((rc = static_base(&base)) != ECHO_OK)
         return rc;
 
-    // ---- the three kernels, as echo_allreduce enqueues them ----
+    // ---- the kernels, as echo_allreduce enqueues them with its default
+    // path choice: one kernel up to ECHO_FUSED_LIMIT elements per rank (the
+    // injected stall, which exercises the bounded waits, always runs three) ----
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     int *status = reinterpret_cast<int *>(base);
     uint8_t *codes1 = base + off_codes1, *scales1 = base + off_scales1;
@@ -208,6 +210,39 @@ extern "C" int echo_allreduce_static(int P, size_t n, int dtype, void *const ran
     const uint32_t chunks = static_cast<uint32_t>(n / echo::kChunk);
     const bool stall = stall_injected();
     const echo::PipeCtl ctl{status, stall ? kStallWaitCycles : kWaitCycles, stall};
+
+    if (!stall && n <= ECHO_FUSED_LIMIT) {
+        echo::KFArgs af{};
+        for (int r = 0; r < P; r++) {
+            af.x.p[r] = rank_ptrs[r];
+            af.out.p[r] = rank_ptrs[r];
+        }
+        af.f = f;
+        af.s = s;
+        af.codes = codes1;
+        af.scales = scales1;
+        af.qcodes = qcodes;
+        af.qscales = qscales;
+        af.n = n;
+        af.scale_stride = scale_stride;
+        af.chunk_begin = 0;
+        af.chunk_end = chunks;
+        af.lanes_log2 = 2; // groups of 32: 4 lanes
+        af.groups_per_seg = static_cast<uint32_t>(n / P / ECHO_GROUP);
+        af.lambda = lambda;
+        af.one_minus_lambda = 1.0f - lambda;
+        af.beta_f = beta_fast;
+        af.one_minus_beta_f = 1.0f - beta_fast;
+        af.beta_s = beta_slow;
+        af.one_minus_beta_s = 1.0f - beta_slow;
+        af.P = P;
+        af.bf16 = dtype == ECHO_BF16;
+        af.enable = enable != 0;
+        af.ctl = ctl;
+        if ((e = echo::launch_kf_fused_allreduce(af, st)) != cudaSuccess)
+            return fail(ECHO_ERR_CUDA, "launch kf_fused_allreduce: %s", cudaGetErrorString(e));
+        return ECHO_OK;
+    }
 
     echo::K1Args a1{};
     echo::K2Args a2{};

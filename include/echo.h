@@ -167,7 +167,8 @@ ECHO_API int echo_allreduce_host(echo_handle *h, const void *const host_send[], 
  * any stream capture.
  * All calls share the array and it keeps the last call's contents; calls
  * whose work overlaps on the GPU (other streams or threads at once) race on
- * it.
+ * it. Calls with n <= 2^20 run as one kernel, as echo_allreduce does by
+ * default (echo_set_fused_limit); larger ones run the three kernels.
  */
 #define ECHO_STATIC_SCRATCH_BYTES (32u * 1024u * 1024u)
 ECHO_API int echo_allreduce_static(int P, size_t n, int dtype, void *const rank_ptrs[], float *f, float *s,

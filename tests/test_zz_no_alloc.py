@@ -49,7 +49,9 @@ def _bits(t):
     return t.cpu().numpy().view(np.uint32)
 
 
-@pytest.mark.parametrize("P,n,dtype", [(8, 8 * 32 * 4096, "bf16"), (4, 4 * 32 * 2003, "fp32")])
+# n <= 2^20 runs as one kernel, larger n as the three kernels, on both sides
+@pytest.mark.parametrize("P,n,dtype", [(8, 8 * 32 * 4096, "bf16"), (4, 4 * 32 * 2003, "fp32"),
+                                       (4, 4 * 32 * 8200, "bf16")])
 def test_static_entry_point_matches_handle(P, n, dtype):
     import torch
     from bit_error_compensated_rank_b200 import echo
@@ -96,7 +98,8 @@ def test_static_entry_point_rejects_sizes_beyond_its_scratch():
     assert not any(bool(t.any()) for t in bufs)  # nothing was enqueued
 
 
-@pytest.mark.parametrize("P,n,dtype", [(4, 4 * 32 * 96, "bf16"), (3, 3 * 32 * 40, "fp32")])
+@pytest.mark.parametrize("P,n,dtype", [(4, 4 * 32 * 96, "bf16"), (3, 3 * 32 * 40, "fp32"),
+                                       (2, 2 * 32 * 16400, "bf16")])
 def test_static_entry_point_matches_oracle(oracle, P, n, dtype):
     import torch
     from bit_error_compensated_rank_b200 import echo
@@ -126,13 +129,14 @@ def test_static_entry_point_matches_oracle(oracle, P, n, dtype):
     assert echo.echo_static_status() == 0
 
 
-def test_static_calls_allocate_nothing():
+@pytest.mark.parametrize("n", [8 * 32 * 4096, 8 * 32 * 4200], ids=["one_kernel", "three_kernels"])
+def test_static_calls_allocate_nothing(n):
     """After the set-up call, further calls leave the device's free memory
     and torch's allocation counters exactly as they were."""
     import torch
     from bit_error_compensated_rank_b200 import echo
 
-    P, n = 8, 8 * 32 * 4096
+    P = 8
     bufs = [torch.randn(n, device="cuda").to(torch.bfloat16) for _ in range(P)]
     f = torch.zeros(n, dtype=torch.float32, device="cuda")
     s = torch.zeros(n, dtype=torch.float32, device="cuda")
