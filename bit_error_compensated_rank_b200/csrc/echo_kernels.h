@@ -85,6 +85,13 @@
 #ifndef ECHO_K1_CTA_BUDGET
 #define ECHO_K1_CTA_BUDGET (100 * 1024)
 #endif
+// With sender feedback a stage is written back before it is refilled, and
+// stages of at most 32 KB measured best: both feedbacks at P = 8 took 7.12
+// against 7.42 ms with 512- instead of 1024-element tiles (48 KB stages),
+// sender feedback alone at P = 2 to 8 kept its time.
+#ifndef ECHO_K1_EF_BUDGET
+#define ECHO_K1_EF_BUDGET (64 * 1024)
+#endif
 
 namespace echo {
 

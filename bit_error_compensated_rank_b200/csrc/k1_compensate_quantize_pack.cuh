@@ -82,18 +82,20 @@ constexpr int k1_bytes_per_elem(int P, bool bf16, bool comp, bool ef)
     return P * (bf16 ? 2 : 4) + (comp ? 8 : 0) + (ef ? 4 * P : 0);
 }
 
-// The largest tile whose stages fit ECHO_K1_CTA_BUDGET, from ECHO_K1_TILE
-// (times 16 / (P * element bytes) when the P partials of an element take
-// fewer than 16 bytes, so that a tile holds about as many partial bytes at
-// small P) down to 256 elements.
+// The largest tile whose stages fit the CTA's budget (ECHO_K1_CTA_BUDGET;
+// ECHO_K1_EF_BUDGET with sender feedback, whose stages are written back
+// before they are refilled), from ECHO_K1_TILE (times 16 / (P * element
+// bytes) when the P partials of an element take fewer than 16 bytes, so that
+// a tile holds about as many partial bytes at small P) down to 256 elements.
 constexpr int k1_tile(int P, bool bf16, bool comp, bool ef)
 {
     const int xb = P * (bf16 ? 2 : 4);
+    const int budget = ef ? ECHO_K1_EF_BUDGET : ECHO_K1_CTA_BUDGET;
     int t = xb < 16 ? ECHO_K1_TILE * (16 / xb) : ECHO_K1_TILE;
     // a one-rank tile with sender feedback also holds its code words (half a
     // byte per element)
     while (t > 256 && ECHO_K1_STAGES * (t * k1_bytes_per_elem(P, bf16, comp, ef) + (P == 1 && ef ? t / 2 : 0)) >
-                          ECHO_K1_CTA_BUDGET)
+                          budget)
         t /= 2;
     return t;
 }
