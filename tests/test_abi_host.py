@@ -206,3 +206,61 @@ def test_static_rejects_bad_arguments_before_cuda(echo, P, n, dtype, params, sta
 def test_static_status_needs_an_output(echo):
     assert echo._lib.echo_static_status(None, 0) == echo.ECHO_ERR_INVALID
     assert "NULL" in echo.echo_last_error()
+
+
+C_CLIENT = r"""
+#include <stdint.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "echo.h"
+
+/* A plain C99 client of the boundary: only calls that need no GPU. */
+int main(void)
+{
+    uint64_t out[4];
+    const size_t n = (size_t)8 * 32 * 1024;
+    echo_handle *h;
+    uint8_t blob[ECHO_DIST_HANDLE_BYTES];
+
+    if (echo_model_bytes(8, n, ECHO_BF16, 1, out) != ECHO_OK)
+        return 1;
+    /* P*b + 8 + P*w, P*w + 16 + w, P*w + P*b bytes per element (w = 17/32) */
+    if (out[0] != n * 16 + n * 8 + 8 * (n / 2 + n / 32))
+        return 2;
+    if (out[1] != 8 * (n / 2 + n / 32) + n * 16 + (n / 2 + n / 32))
+        return 3;
+    if (out[2] != 8 * (n / 2 + n / 32) + n * 16)
+        return 4;
+    if (out[3] != (uint64_t)2 * 7 * (n / 2 + n / 32))
+        return 5;
+    h = echo_create(1, n, 32, ECHO_BF16); /* P = 1 is refused before CUDA is touched */
+    if (h != NULL || echo_last_status() != ECHO_ERR_INVALID || strlen(echo_last_error()) == 0)
+        return 6;
+    if (echo_allreduce(NULL, NULL, ECHO_FWD, NULL) != ECHO_ERR_INVALID)
+        return 7;
+    if (echo_set_fused_limit(NULL, 0) != ECHO_ERR_INVALID)
+        return 8;
+    if (echo_destroy(NULL) != ECHO_OK)
+        return 9;
+    if (echo_dist_export(NULL, blob) != ECHO_ERR_INVALID)
+        return 10;
+    printf("ok\n");
+    return 0;
+}
+"""
+
+
+def test_header_compiles_as_c99_and_links(echo, tmp_path):
+    """The boundary as a C user sees it: the header compiles as strict C99
+    (no C++), the program links against libecho.so, and the calls that need no
+    GPU give the documented results."""
+    src = tmp_path / "client.c"
+    exe = tmp_path / "client"
+    src.write_text(C_CLIENT)
+    lib_dir = os.path.dirname(echo.LIB_PATH)
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I",
+                    os.path.join(ROOT, "include"), str(src), "-o", str(exe), "-L", lib_dir, "-lecho",
+                    "-Wl,-rpath," + lib_dir], check=True, capture_output=True, text=True)
+    res = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert res.returncode == 0 and res.stdout.strip() == "ok", (res.returncode, res.stdout, res.stderr)
