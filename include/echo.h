@@ -256,9 +256,10 @@ ECHO_API int echo_set_variant(echo_handle *h, int variant);
  * for bit and writes the same buffers (both wires, state, sender errors,
  * outputs); it does not read the stage-1 wire back. Every variant and group
  * size runs fused. 0 turns it off; the default is 2^20. It applies to
- * echo_allreduce, echo_allreduce_out and echo_allreduce_host, not to the
- * static or per-rank entry points. echo_stats still counts the three kernels'
- * model bytes. echo_get_fused_limit reads the setting (max_n non-NULL, else
+ * echo_allreduce, echo_allreduce_out and echo_allreduce_host. The static
+ * entry point makes the same choice with the default limit; the per-rank
+ * entry points (echo_dist_*) always run their three stages. echo_stats still
+ * counts the three kernels' model bytes. echo_get_fused_limit reads the setting (max_n non-NULL, else
  * ECHO_ERR_INVALID).
  */
 ECHO_API int echo_set_fused_limit(echo_handle *h, size_t max_n);
